@@ -1,0 +1,184 @@
+"""fp64 CPU oracle for the selective scan (S6) and its decode state update.
+
+TEST INFRASTRUCTURE ONLY: imported by the tests, by the smoke check and by the
+benchmark's CPU-baseline leg. The product (the CUDA library and its binding)
+never imports it. The arithmetic lives in ``s6_oracle.c`` (plain C, double
+precision, OpenMP across independent rows); this module compiles it with gcc
+on first use and marshals numpy arrays into it.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "s6_oracle.c")
+_LIB = os.path.join(_HERE, "_build", "libs6oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+F32, BF16 = 0, 1
+_DTYPES = {"f32": F32, "bf16": BF16}
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle (gcc -O2, no fast-math, OpenMP) and return the .so path."""
+    with _lock:
+        if (not force and os.path.exists(_LIB)
+                and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC)):
+            return _LIB
+        os.makedirs(os.path.dirname(_LIB), exist_ok=True)
+        tmp = _LIB + f".{os.getpid()}.tmp"
+        subprocess.check_call(["gcc", "-O2", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared",
+                               "-std=c11", "-Wall", "-Werror", _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+        return _LIB
+
+
+def _bind(path: str):
+    lib = ctypes.CDLL(path)
+    i64, ip, vp = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p
+    lib.s6_oracle_scan.restype = ip
+    lib.s6_oracle_scan.argtypes = [i64, i64, i64, i64, ip, vp, vp, vp, vp, vp, vp, vp, vp,
+                                   ip, vp, i64, vp, vp, vp, ip]
+    lib.s6_oracle_state_update.restype = ip
+    lib.s6_oracle_state_update.argtypes = [i64, i64, i64, ip, vp, vp, vp, vp, vp, vp, vp, vp,
+                                           vp, ip, vp, i64, vp, ip]
+    lib.s6_oracle_max_threads.restype = ip
+    lib.s6_oracle_max_threads.argtypes = []
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = _bind(build())
+    return _lib
+
+
+def max_threads() -> int:
+    return int(_load().s6_oracle_max_threads())
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _in(a, dtype: int):
+    if a is None:
+        return None
+    want = np.float32 if dtype == F32 else np.uint16
+    a = np.ascontiguousarray(a)
+    if a.dtype != want:
+        raise TypeError(f"oracle input has dtype {a.dtype}, expected {np.dtype(want)}")
+    return a
+
+
+def _f32(a):
+    return None if a is None else np.ascontiguousarray(a, dtype=np.float32)
+
+
+def scan(*, u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
+         dtype="f32", rows=None, h0=None, threads: int = 0, _lib_override=None):
+    """Selective scan forward in fp64.
+
+    ``u, delta, z``: (batch, dim, L); ``B, C``: (batch, dstate, L), float32
+    arrays or uint16 bf16 bits according to ``dtype``. ``A`` (dim, dstate),
+    ``D`` and ``delta_bias`` (dim,) float32. ``rows``: optional list of row
+    indices ``b*dim + d`` to compute (default: all rows in order). ``h0``:
+    optional initial state (n_rows, dstate).
+
+    Returns ``(y, h)``: y (batch, dim, L) float64 (or (n_rows, L) with
+    ``rows``) and the final state (batch, dim, dstate) (or (n_rows, dstate)).
+    """
+    dt = _DTYPES[dtype]
+    u, delta, B, C, z = (_in(a, dt) for a in (u, delta, B, C, z))
+    A, D, delta_bias = _f32(A), _f32(D), _f32(delta_bias)
+    batch, dim, L = u.shape
+    dstate = B.shape[1]
+    if delta.shape != u.shape or (z is not None and z.shape != u.shape):
+        raise ValueError("u, delta and z must share one (batch, dim, L) shape")
+    if B.shape != (batch, dstate, L) or C.shape != B.shape or A.shape != (dim, dstate):
+        raise ValueError("B, C must be (batch, dstate, L) and A (dim, dstate)")
+    if rows is None:
+        n_rows, rows_arr = batch * dim, None
+    else:
+        rows_arr = np.ascontiguousarray(rows, dtype=np.int64)
+        n_rows = rows_arr.size
+    h0_arr = None if h0 is None else np.ascontiguousarray(h0, dtype=np.float64).reshape(n_rows, dstate)
+    y = np.empty((n_rows, L), np.float64)
+    h = np.empty((n_rows, dstate), np.float64)
+    lib = _lib_override or _load()
+    rc = lib.s6_oracle_scan(batch, dim, dstate, L, dt, _ptr(u), _ptr(delta), _ptr(A), _ptr(B),
+                                _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias), int(bool(delta_softplus)),
+                                _ptr(rows_arr), n_rows, _ptr(h0_arr), _ptr(y), _ptr(h), int(threads))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    if rows is None:
+        return y.reshape(batch, dim, L), h.reshape(batch, dim, dstate)
+    return y, h
+
+
+def state_update(*, state, x, delta, A, B, C, D=None, z=None, delta_bias=None,
+                 delta_softplus=True, dtype="f32", rows=None, threads: int = 0,
+                 _lib_override=None):
+    """One decode step in fp64.
+
+    ``state``: float64 (batch, dim, dstate) (or (n_rows, dstate) with
+    ``rows``), updated in place. ``x, delta, z``: (batch, dim); ``B, C``:
+    (batch, dstate). Returns y (batch, dim) float64 (or (n_rows,)).
+    """
+    dt = _DTYPES[dtype]
+    x, delta, B, C, z = (_in(a, dt) for a in (x, delta, B, C, z))
+    A, D, delta_bias = _f32(A), _f32(D), _f32(delta_bias)
+    batch, dim = x.shape
+    dstate = B.shape[1]
+    if not (isinstance(state, np.ndarray) and state.dtype == np.float64 and state.flags.c_contiguous):
+        raise TypeError("state must be a C-contiguous float64 array (updated in place)")
+    if rows is None:
+        n_rows, rows_arr = batch * dim, None
+    else:
+        rows_arr = np.ascontiguousarray(rows, dtype=np.int64)
+        n_rows = rows_arr.size
+    if state.size != n_rows * dstate:
+        raise ValueError("state has the wrong size")
+    y = np.empty(n_rows, np.float64)
+    lib = _lib_override or _load()
+    rc = lib.s6_oracle_state_update(batch, dim, dstate, dt, _ptr(state), _ptr(x), _ptr(delta),
+                                        _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                                        _ptr(delta_bias), int(bool(delta_softplus)),
+                                        _ptr(rows_arr), n_rows, _ptr(y), int(threads))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return y.reshape(batch, dim) if rows is None else y
+
+
+class Variant:
+    """The oracle's entry points bound to another build of the oracle source.
+
+    Used only by the tests that plant a mistake in a copy of the oracle source
+    and check that the pins catch it.
+    """
+
+    def __init__(self, so_path: str):
+        self._lib = _bind(so_path)
+
+    def scan(self, **kw):
+        return scan(_lib_override=self._lib, **kw)
+
+    def state_update(self, **kw):
+        return state_update(_lib_override=self._lib, **kw)
+
+
+def compile_source(src_path: str, so_path: str) -> str:
+    """Compile an oracle source file (same flags as :func:`build`)."""
+    subprocess.check_call(["gcc", "-O2", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared",
+                           "-std=c11", src_path, "-o", so_path, "-lm"])
+    return so_path
+
+
+SOURCE = _SRC

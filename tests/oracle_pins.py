@@ -1,0 +1,387 @@
+"""Pins of the fp64 oracle to facts other than itself.
+
+Each ``pin_*`` function takes an oracle object (the ``oracle`` module, or an
+``oracle.Variant`` built from a copy of its source with a planted mistake) and
+raises ``AssertionError`` when the oracle disagrees with the fact it checks:
+values printed by the pages for a worked example, closed forms, brute force on
+tiny inputs, special cases that reduce to a library routine, and invariants.
+None of them re-types the oracle's loop: each computes the expected value by a
+different route (a convolution, a cumulative sum, an explicit matrix, a masked
+matrix product, a single-step formula).
+"""
+from __future__ import annotations
+
+import os
+
+import numpy as np
+from scipy.special import expit
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+GOLDEN = os.path.join(HERE, "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _f32(a):
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _rel(a, b):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    scale = max(np.abs(b).max(), 1e-300)
+    return float(np.abs(a - b).max() / scale)
+
+
+def read_selection_step():
+    rows = []
+    with open(os.path.join(GOLDEN, "selection_step.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append([float(v) for v in line.split()])
+    return rows
+
+
+def pin_selection_step(orc):
+    """The worked single step ("Notas sobre Mamba", "O mecanismo de seleção (S6)").
+
+    h = 1, x = 1, A = -1, B = 1, softplus off, no bias: with B = 0 the new
+    state is Abar itself; with B = 1 it is Abar + delta. Both must round to the
+    page's printed 4-decimal values, for four identical state channels.
+    """
+    N = 4
+    for delta, abar_p, bbar_p, h_p in read_selection_step():
+        for Bval, expect in ((0.0, abar_p), (1.0, h_p)):
+            state = np.ones((1, 1, N), np.float64)
+            orc.state_update(state=state, x=_f32([[1.0]]), delta=_f32([[delta]]),
+                             A=_f32(-np.ones((1, N))), B=_f32(np.full((1, N), Bval)),
+                             C=_f32(np.ones((1, N))), delta_softplus=False)
+            got = np.round(state.reshape(-1), 4)
+            assert np.all(np.abs(got - expect) < 1e-9), (delta, Bval, state.reshape(-1), expect)
+        # Bbar = delta * B with B = 1 is printed too: the state gained exactly delta.
+        s0 = np.ones((1, 1, N))
+        s1 = np.ones((1, 1, N))
+        kw = dict(x=_f32([[1.0]]), delta=_f32([[delta]]), A=_f32(-np.ones((1, N))),
+                  C=_f32(np.ones((1, N))), delta_softplus=False)
+        orc.state_update(state=s0, B=_f32(np.zeros((1, N))), **kw)
+        orc.state_update(state=s1, B=_f32(np.ones((1, N))), **kw)
+        assert abs(round(float((s1 - s0).max()), 4) - bbar_p) < 1e-12
+
+
+def pin_lti_convolution(orc, L=96, N=8, seed=11):
+    """Constant delta, B and C make the system time invariant ("Notas sobre
+    Mamba", "Preliminares"): y = K * x + D x with K_k = sum_n C_n Abar_n^k
+    delta B_n and Abar = exp(delta A) -- first-order Bbar = delta B. Computed by
+    np.convolve; agreement to 1e-12 relative.
+    """
+    g = _rng(seed)
+    dim = 3
+    A = -np.exp(g.normal(size=(dim, N))).astype(np.float32)
+    Bv = g.normal(size=N).astype(np.float32)
+    Cv = g.normal(size=N).astype(np.float32)
+    D = g.uniform(0.5, 1.5, size=dim).astype(np.float32)
+    x = g.normal(size=(1, dim, L)).astype(np.float32)
+    delta = 0.0625
+    Bt = np.repeat(Bv[None, :, None], L, axis=2)
+    Ct = np.repeat(Cv[None, :, None], L, axis=2)
+    y, h = orc.scan(u=x, delta=_f32(np.full((1, dim, L), delta)), A=A, B=_f32(Bt), C=_f32(Ct),
+                    D=D, delta_softplus=False)
+    k = np.arange(L)
+    for d in range(dim):
+        abar = np.exp(delta * A[d].astype(np.float64))
+        K = ((Cv.astype(np.float64) * delta * Bv.astype(np.float64))[None, :]
+             * np.power(abar[None, :], k[:, None])).sum(axis=1)
+        ref = np.convolve(x[0, d].astype(np.float64), K)[:L] + float(D[d]) * x[0, d].astype(np.float64)
+        assert _rel(y[0, d], ref) < 1e-12, (d, _rel(y[0, d], ref))
+        # final state: sum_k abar^k delta B x_{L-1-k}
+        href = (np.power(abar[None, :], k[::-1, None]) * (delta * Bv.astype(np.float64))[None, :]
+                * x[0, d].astype(np.float64)[:, None]).sum(axis=0)
+        assert _rel(h[0, d], href) < 1e-12
+
+
+def pin_zero_delta(orc, L=40, N=5, seed=12):
+    """delta = 0 keeps the state and ignores the token ("Notas sobre Mamba",
+    "O mecanismo de seleção (S6)"): Abar = 1, Bbar = 0, so h stays 0 and
+    y = D x silu(z), exactly.
+    """
+    g = _rng(seed)
+    batch, dim = 2, 3
+    x = g.normal(size=(batch, dim, L)).astype(np.float32)
+    z = g.normal(size=(batch, dim, L)).astype(np.float32)
+    D = g.uniform(0.5, 1.5, size=dim).astype(np.float32)
+    A = -np.exp(g.normal(size=(dim, N))).astype(np.float32)
+    B = g.normal(size=(batch, N, L)).astype(np.float32)
+    C = g.normal(size=(batch, N, L)).astype(np.float32)
+    y, h = orc.scan(u=x, delta=_f32(np.zeros((batch, dim, L))), A=A, B=B, C=C, D=D, z=z,
+                    delta_softplus=False)
+    assert np.all(h == 0.0)
+    ref = D[None, :, None].astype(np.float64) * x * (z * expit(z.astype(np.float64)))
+    assert _rel(y, ref) < 1e-15
+
+
+def pin_linearity(orc, L=50, N=6, seed=13):
+    """For fixed delta, B, C, z the map x -> (y, h_final) is linear ("Notas sobre
+    Mamba", the recurrence of "O mecanismo de seleção (S6)"). Inputs are
+    multiples of 1/8 so that 3 x1 - 2 x2 is exact in float32.
+    """
+    g = _rng(seed)
+    batch, dim = 2, 4
+    x1 = (g.integers(-16, 17, size=(batch, dim, L)) / 8.0).astype(np.float32)
+    x2 = (g.integers(-16, 17, size=(batch, dim, L)) / 8.0).astype(np.float32)
+    x3 = _f32(3.0 * x1 - 2.0 * x2)
+    kw = dict(delta=_f32(g.normal(scale=0.5, size=(batch, dim, L))),
+              A=_f32(-np.exp(g.normal(size=(dim, N)))),
+              B=_f32(g.normal(size=(batch, N, L))), C=_f32(g.normal(size=(batch, N, L))),
+              D=_f32(g.uniform(0.5, 1.5, size=dim)), z=_f32(g.normal(size=(batch, dim, L))),
+              delta_bias=_f32(g.normal(size=dim) - 2.0), delta_softplus=True)
+    y1, h1 = orc.scan(u=x1, **kw)
+    y2, h2 = orc.scan(u=x2, **kw)
+    y3, h3 = orc.scan(u=x3, **kw)
+    assert _rel(y3, 3 * y1 - 2 * y2) < 1e-12
+    assert _rel(h3, 3 * h1 - 2 * h2) < 1e-12
+    # and not trivially linear: the map is not the zero map
+    assert np.abs(y1).max() > 1e-3
+
+
+def pin_scalar_state_closed_form(orc, L=60, seed=14):
+    """N = 1: h_t = sum_{i<=t} exp(a (S_t - S_i)) delta_i B_i x_i with S the
+    cumulative sum of delta -- the log-space cumulative product the pages use
+    to build the decay mask ("Notas sobre Mamba", "A forma dual: atenção
+    mascarada"). y_t = C_t h_t + D x_t.
+    """
+    g = _rng(seed)
+    a = -0.75
+    x = g.normal(size=(1, 1, L)).astype(np.float32)
+    dl = g.uniform(0.01, 0.4, size=(1, 1, L)).astype(np.float32)
+    B = g.normal(size=(1, 1, L)).astype(np.float32)
+    C = g.normal(size=(1, 1, L)).astype(np.float32)
+    D = np.array([0.9], np.float32)
+    y, h = orc.scan(u=x, delta=dl, A=_f32([[a]]), B=B, C=C, D=D, delta_softplus=False)
+    d64 = dl[0, 0].astype(np.float64)
+    S = np.cumsum(d64)
+    w = d64 * B[0, 0].astype(np.float64) * x[0, 0].astype(np.float64)
+    href = np.array([np.sum(np.exp(a * (S[t] - S[:t + 1])) * w[:t + 1]) for t in range(L)])
+    yref = C[0, 0].astype(np.float64) * href + float(D[0]) * x[0, 0].astype(np.float64)
+    assert _rel(y[0, 0], yref) < 1e-12
+    assert abs(h[0, 0, 0] - href[-1]) <= 1e-12 * max(1.0, abs(href[-1]))
+
+
+def pin_unrolled_products(orc, seed=15):
+    """Brute force on tiny inputs: y = M x + D x with the lower-triangular
+    M_ji = sum_n C_j[n] (prod_{k=i+1..j} Abar_k[n]) Bbar_i[n] ("Notas sobre
+    Mamba", "SSMs como matrizes semisseparáveis"), for every L <= 16 and
+    random N <= 4, several batches and channels, softplus and bias on, gate on.
+    """
+    g = _rng(seed)
+    for L in range(1, 17):
+        N = int(g.integers(1, 5))
+        batch, dim = 2, 3
+        x = g.normal(size=(batch, dim, L)).astype(np.float32)
+        raw = g.normal(scale=0.5, size=(batch, dim, L)).astype(np.float32)
+        bias = (g.normal(size=dim) - 1.5).astype(np.float32)
+        A = (-np.exp(g.normal(size=(dim, N)))).astype(np.float32)
+        B = g.normal(size=(batch, N, L)).astype(np.float32)
+        C = g.normal(size=(batch, N, L)).astype(np.float32)
+        D = g.uniform(0.5, 1.5, size=dim).astype(np.float32)
+        z = g.normal(size=(batch, dim, L)).astype(np.float32)
+        y, h = orc.scan(u=x, delta=raw, A=A, B=B, C=C, D=D, z=z, delta_bias=bias,
+                        delta_softplus=True)
+        for b in range(batch):
+            for d in range(dim):
+                dl = np.logaddexp(0.0, raw[b, d].astype(np.float64) + float(bias[d]))
+                abar = np.exp(dl[:, None] * A[d].astype(np.float64)[None, :])      # (L, N)
+                bbar = dl[:, None] * B[b].T.astype(np.float64)                        # (L, N)
+                M = np.zeros((L, L))
+                for j in range(L):
+                    for i in range(j + 1):
+                        prod = np.prod(abar[i + 1:j + 1], axis=0) if j > i else np.ones(N)
+                        M[j, i] = np.sum(C[b, :, j].astype(np.float64) * prod * bbar[i])
+                xx = x[b, d].astype(np.float64)
+                yref = (M @ xx + float(D[d]) * xx) * (z[b, d] * expit(z[b, d].astype(np.float64)))
+                assert _rel(y[b, d], yref) < 1e-12, (L, N, b, d)
+                hT = np.zeros(N)
+                for i in range(L):
+                    hT += np.prod(abar[i + 1:], axis=0) * bbar[i] * xx[i]
+                assert _rel(h[b, d], hT) < 1e-12
+
+
+def pin_scalar_transition_masked_form(orc, L=32, N=16, seed=16):
+    """If A[d,n] = a for all n, Abar_t = a_t I and the scan equals the masked
+    form y = (Lmask o (C B^T)) (delta x) + D x with Lmask_ji = prod_{k=i+1..j}
+    a_k ("Notas sobre Mamba", "A forma dual: atenção mascarada"). Computed
+    with matrix products.
+    """
+    g = _rng(seed)
+    a = -0.375
+    x = g.normal(size=(1, 1, L)).astype(np.float32)
+    dl = g.uniform(0.05, 0.5, size=(1, 1, L)).astype(np.float32)
+    B = g.normal(size=(1, N, L)).astype(np.float32)
+    C = g.normal(size=(1, N, L)).astype(np.float32)
+    D = np.array([1.25], np.float32)
+    y, _ = orc.scan(u=x, delta=dl, A=_f32(np.full((1, N), a)), B=B, C=C, D=D,
+                    delta_softplus=False)
+    d64 = dl[0, 0].astype(np.float64)
+    S = np.cumsum(a * d64)
+    mask = np.tril(np.exp(S[:, None] - S[None, :]))
+    Cm = C[0].T.astype(np.float64)
+    Bm = B[0].T.astype(np.float64)
+    xx = x[0, 0].astype(np.float64)
+    yref = (mask * (Cm @ Bm.T)) @ (d64 * xx) + 1.25 * xx
+    assert _rel(y[0, 0], yref) < 1e-12
+
+
+def pin_segmentation(orc, L=77, m=30, N=4, seed=17):
+    """Associativity of the recurrence ("Notas sobre Mamba", "A varredura
+    paralela ciente do hardware"): the scan over [0, L) equals the scan over
+    [0, m) continued from its final state over [m, L).
+    """
+    g = _rng(seed)
+    batch, dim = 2, 3
+    t = dict(u=g.normal(size=(batch, dim, L)), delta=g.normal(scale=0.5, size=(batch, dim, L)),
+             z=g.normal(size=(batch, dim, L)), B=g.normal(size=(batch, N, L)),
+             C=g.normal(size=(batch, N, L)))
+    t = {k: _f32(v) for k, v in t.items()}
+    p = dict(A=_f32(-np.exp(g.normal(size=(dim, N)))), D=_f32(g.uniform(0.5, 1.5, size=dim)),
+             delta_bias=_f32(g.normal(size=dim) - 2.0), delta_softplus=True)
+    y, h = orc.scan(**t, **p)
+    y1, h1 = orc.scan(**{k: _f32(v[..., :m]) for k, v in t.items()}, **p)
+    y2, h2 = orc.scan(**{k: _f32(v[..., m:]) for k, v in t.items()}, **p,
+                      h0=h1.reshape(batch * dim, N))
+    assert _rel(np.concatenate([y1, y2], axis=-1), y) < 1e-13
+    assert _rel(h2, h) < 1e-13
+
+
+def pin_decode_equals_scan(orc, L=25, N=16, seed=18):
+    """L single-token steps from h = 0 reproduce the scan's y and final state
+    (recurrent mode for generation, "Notas sobre Mamba", "Preliminares"; the
+    step of "Mamba-2 e State Space Duality (SSD)").
+    """
+    g = _rng(seed)
+    batch, dim = 3, 2
+    t = dict(u=g.normal(size=(batch, dim, L)), delta=g.normal(scale=0.5, size=(batch, dim, L)),
+             z=g.normal(size=(batch, dim, L)), B=g.normal(size=(batch, N, L)),
+             C=g.normal(size=(batch, N, L)))
+    t = {k: _f32(v) for k, v in t.items()}
+    p = dict(A=_f32(-np.exp(g.normal(size=(dim, N)))), D=_f32(g.uniform(0.5, 1.5, size=dim)),
+             delta_bias=_f32(g.normal(size=dim) - 2.0), delta_softplus=True)
+    y, h = orc.scan(**t, **p)
+    state = np.zeros((batch, dim, N))
+    for s in range(L):
+        ys = orc.state_update(state=state, x=_f32(t["u"][..., s]), delta=_f32(t["delta"][..., s]),
+                              z=_f32(t["z"][..., s]), B=_f32(t["B"][..., s]),
+                              C=_f32(t["C"][..., s]), **p)
+        assert _rel(ys, y[..., s]) < 1e-14
+    assert _rel(state, h) < 1e-14
+
+
+def pin_large_delta_resets(orc, L=20, N=4, seed=19):
+    """A large step forgets the past and absorbs the token ("Notas sobre
+    Mamba", "O mecanismo de seleção (S6)"): with delta = 50, Abar underflows to
+    below 1e-21 and h_t = delta B_t x_t, y_t = C_t . h_t + D x_t.
+    """
+    g = _rng(seed)
+    x = g.normal(size=(1, 2, L)).astype(np.float32)
+    B = g.normal(size=(1, N, L)).astype(np.float32)
+    C = g.normal(size=(1, N, L)).astype(np.float32)
+    A = _f32(-np.arange(1, N + 1)[None, :].repeat(2, 0))
+    D = _f32([0.5, 1.5])
+    y, h = orc.scan(u=x, delta=_f32(np.full((1, 2, L), 50.0)), A=A, B=B, C=C, D=D,
+                    delta_softplus=False)
+    for d in range(2):
+        hb = 50.0 * B[0].astype(np.float64) * x[0, d].astype(np.float64)[None, :]
+        yref = (C[0].astype(np.float64) * hb).sum(axis=0) + float(D[d]) * x[0, d].astype(np.float64)
+        assert _rel(y[0, d], yref) < 1e-12
+        assert _rel(h[0, d], hb[:, -1]) < 1e-12
+
+
+def pin_softplus_of_biased_step(orc, seed=20):
+    """delta = softplus(raw + bias) ("Notas sobre Mamba", "O mecanismo de
+    seleção (S6)"): one step from h = 0 with B = x = 1 leaves h = delta, which
+    must equal log(1 + exp(raw + bias)) from numpy's logaddexp; the bias is
+    added before the softplus, so (raw, bias) and (raw + bias, 0) agree.
+    """
+    g = _rng(seed)
+    raw = np.array([-9.0, -4.25, -1.0, 0.0, 0.75, 3.5, 12.0, 19.5, 25.0], np.float32)
+    bias = np.float32(-0.5)
+    for r in raw:
+        hs = []
+        for rr, bb in ((r, bias), (np.float32(r + bias), np.float32(0.0))):
+            st = np.zeros((1, 1, 1))
+            orc.state_update(state=st, x=_f32([[1.0]]), delta=_f32([[rr]]), A=_f32([[-1.0]]),
+                             B=_f32([[1.0]]), C=_f32([[1.0]]), delta_bias=_f32([bb]),
+                             delta_softplus=True)
+            hs.append(float(st[0, 0, 0]))
+        v = float(np.float32(r + bias))
+        ref = float(np.logaddexp(0.0, v))
+        assert abs(hs[1] - ref) <= 1e-12 * ref, (r, hs[1], ref)
+        assert abs(hs[0] - hs[1]) <= 1e-12 * ref
+    del g
+
+
+def pin_gate(orc, L=33, N=3, seed=21):
+    """The output is multiplied by SiLU(z) = z * sigmoid(z) ("Notas sobre Mamba",
+    "O bloco Mamba"): y(z) = y(no z) * z * expit(z).
+    """
+    g = _rng(seed)
+    t = dict(u=g.normal(size=(1, 2, L)), delta=g.normal(scale=0.5, size=(1, 2, L)),
+             B=g.normal(size=(1, N, L)), C=g.normal(size=(1, N, L)))
+    t = {k: _f32(v) for k, v in t.items()}
+    p = dict(A=_f32(-np.exp(g.normal(size=(2, N)))), D=_f32([0.7, 1.1]),
+             delta_bias=_f32([-2.0, -3.0]))
+    z = g.normal(size=(1, 2, L)).astype(np.float32)
+    y0, h0 = orc.scan(**t, **p)
+    y1, h1 = orc.scan(**t, **p, z=z)
+    assert _rel(y1, y0 * z * expit(z.astype(np.float64))) < 1e-14
+    assert np.array_equal(h0, h1)
+
+
+def pin_bf16_decoding(orc, seed=22):
+    """bfloat16 inputs are read as the float32 value with the same top 16 bits:
+    the bf16 scan equals the f32 scan of the widened values, and a few bit
+    patterns have known values (0x3F80 = 1, 0xC040 = -3, 0x3E80 = 0.25).
+    """
+    g = _rng(seed)
+    L, N = 9, 2
+    known = np.array([0x3F80, 0xC040, 0x3E80], np.uint16)
+    vals = np.array([1.0, -3.0, 0.25])
+    st = np.zeros((1, 3, 1))
+    orc.state_update(state=st, x=known.reshape(1, 3), delta=np.full((1, 3), 0x3F80, np.uint16),
+                     A=_f32(-np.ones((3, 1))), B=np.full((1, 1), 0x3F80, np.uint16),
+                     C=np.full((1, 1), 0x3F80, np.uint16), delta_softplus=False, dtype="bf16")
+    assert np.allclose(st.reshape(-1), vals, rtol=0, atol=1e-15)
+
+    def bits(a):
+        return (np.asarray(a, np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+    def widen(b):
+        return (b.astype(np.uint32) << 16).view(np.float32)
+
+    t = dict(u=g.normal(size=(1, 2, L)), delta=g.normal(scale=0.5, size=(1, 2, L)),
+             B=g.normal(size=(1, N, L)), C=g.normal(size=(1, N, L)), z=g.normal(size=(1, 2, L)))
+    tb = {k: bits(v) for k, v in t.items()}
+    tf = {k: widen(v) for k, v in tb.items()}
+    p = dict(A=_f32(-np.exp(g.normal(size=(2, N)))), D=_f32([0.7, 1.1]),
+             delta_bias=_f32([-2.0, -3.0]))
+    yb, hb = orc.scan(**tb, **p, dtype="bf16")
+    yf, hf = orc.scan(**tf, **p, dtype="f32")
+    assert np.array_equal(yb, yf) and np.array_equal(hb, hf)
+
+
+ALL_PINS = [
+    pin_selection_step,
+    pin_lti_convolution,
+    pin_zero_delta,
+    pin_linearity,
+    pin_scalar_state_closed_form,
+    pin_unrolled_products,
+    pin_scalar_transition_masked_form,
+    pin_segmentation,
+    pin_decode_equals_scan,
+    pin_large_delta_resets,
+    pin_softplus_of_biased_step,
+    pin_gate,
+    pin_bf16_decoding,
+]

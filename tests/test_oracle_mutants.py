@@ -1,0 +1,50 @@
+"""Plant plausible mistakes in a copy of the oracle source and check that the
+pins catch every one of them (CPU only; the planted copies live in a
+temporary directory and are never used by anything else)."""
+import os
+
+import pytest
+
+import oracle
+from tests import oracle_pins
+
+# (name, text in s6_oracle.c, replacement)
+MUTANTS = [
+    ("drop_skip_term", "acc += (double)D[d] * x;", "acc += 0.0 * x;"),
+    ("sign_of_exponent", "exp(dt * a) * h[n]", "exp(-dt * a) * h[n]"),
+    ("zoh_input_matrix", "const double Bbar = dt * load_value(B, dtype, j);",
+     "const double Bbar = (exp(dt * a) - 1.0) / a * load_value(B, dtype, j);"),
+    ("readout_before_update",
+     "h[n] = exp(dt * a) * h[n] + Bbar * x;\n            acc += load_value(C, dtype, j) * h[n];",
+     "acc += load_value(C, dtype, j) * h[n];\n            h[n] = exp(dt * a) * h[n] + Bbar * x;"),
+    ("bias_after_softplus",
+     "if (delta_bias)\n            dt += (double)delta_bias[d];\n        if (delta_softplus)\n            dt = softplus(dt);",
+     "if (delta_softplus)\n            dt = softplus(dt);\n        if (delta_bias)\n            dt += (double)delta_bias[d];"),
+    ("no_gate", "acc *= silu(load_value(z, dtype, i));", "(void)0;"),
+    ("sigmoid_not_silu", "return v / (1.0 + exp(-v));", "return 1.0 / (1.0 + exp(-v));"),
+    ("transition_index_transposed", "(double)A[d * dstate + n]", "(double)A[n * dim + d]"),
+    ("input_index_uses_state_row", "const double Bbar = dt * load_value(B, dtype, j);",
+     "const double Bbar = dt * load_value(B, dtype, (b * dstate + n) * seqlen + (seqlen - 1 - t));"),
+    ("softplus_is_exp", "return v > 20.0 ? v : log1p(exp(v));", "return v > 20.0 ? v : exp(v);"),
+    ("bf16_shift", "<< 16;", "<< 15;"),
+    ("token_not_scaled", "h[n] = exp(dt * a) * h[n] + Bbar * x;", "h[n] = exp(dt * a) * h[n] + Bbar;"),
+    ("state_not_reset_per_row", "h[n] = h0 ? h0[r * dstate + n] : 0.0;",
+     "h[n] = h0 ? h0[r * dstate + n] : (r > 0 ? 0.5 : 0.0);"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_mutant(tmp_path, name, old, new):
+    src = open(oracle.SOURCE).read()
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    path = os.path.join(tmp_path, f"mutant_{name}.c")
+    with open(path, "w") as f:
+        f.write(src.replace(old, new))
+    orc = oracle.Variant(oracle.compile_source(path, os.path.join(tmp_path, f"{name}.so")))
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(orc)
+        except (AssertionError, ValueError, FloatingPointError):
+            caught.append(pin.__name__)
+    assert caught, f"no pin caught the planted mistake {name}"
