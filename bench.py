@@ -1,0 +1,442 @@
+#!/usr/bin/env python
+"""Benchmark of the selective scan (S6) forward on B200.
+
+One step = one selective-scan forward pass (softplus, discretisation, scan,
+readout, D skip, SiLU gate, final state) over one batch of the workload,
+launched through the C ABI. Default workload: the Mamba-130M-shaped layer
+(batch 8, d_inner 1536, N 16, L 2048, bf16 inputs, fp32 state).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   (the fp64 CPU oracle, timed on host cores)
+
+Prints one JSON line on rank 0. Metric: scan elements (batch*dim*L*N) per
+second, whole job (all ranks). Under torchrun every rank runs an independent
+replica on its own batch (weak scaling, no data-path collective); the barrier
+and the max-over-ranks reduction of the elapsed device time use NCCL.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from selective_state_space_27_b200.inputs import SCAN_WORKLOADS, make_scan_inputs  # noqa: E402
+
+METRIC = "selective-scan B·D·L·N elems/s at 1 B200; % of HBM/MUFU roofline"
+UNIT = "elem/s"
+L2_BYTES = 126 * 1024 * 1024
+ROTATE = 3  # input sets cycled through so that each step reads inputs not resident in L2
+
+# B200 unit counts for the arithmetic rooflines (per SM per clock): MUFU
+# transcendental results 16, FP32 lanes 128.
+SMS_B200 = 148
+MUFU_PER_CLK = 16
+FP32_PER_CLK = 128
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--workload", default="mamba130m_layer", choices=sorted(SCAN_WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="CPU-baseline budget (seconds of oracle work on rank 0)")
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing
+
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = False
+
+    def init(self, backend):
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = True
+
+    def barrier(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max(self, value: float, device=None) -> float:
+        if not self.pg:
+            return value
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([value], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------
+# algorithmic counts (per scan pass)
+
+def algorithmic_counts(w, in_bytes: int):
+    """Bytes, MUFU and FP32 operations the scan needs, independent of the kernel.
+
+    Bytes: u, delta, z read once; B, C read once; A, D, delta_bias read once;
+    y written once; final state written once.
+    MUFU: exp(delta A) per (b, d, t, n); softplus (exp + log) and the gate
+    (exp + reciprocal) per (b, d, t).
+    FP32: delta*A, delta*B*u, the state FMA and the readout FMA per element;
+    about 8 per (b, d, t) for softplus, skip and gate.
+    """
+    rows_t = w.batch * w.dim * w.seqlen
+    elems = rows_t * w.dstate
+    n_in = 3 if w.has_z else 2
+    bytes_ = (n_in * rows_t * in_bytes + 2 * w.batch * w.dstate * w.seqlen * in_bytes
+              + w.dim * w.dstate * 4 + 2 * w.dim * 4
+              + rows_t * in_bytes + w.batch * w.dim * w.dstate * 4)
+    mufu = elems + rows_t * (2 + (2 if w.has_z else 0))
+    fp32 = 4 * elems + 8 * rows_t
+    return {"elements": elems, "bytes": bytes_, "mufu": mufu, "fp32": fp32}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "sm_max_mhz": float(d.get("sm_max_mhz", 1965.0)),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def mark_begin(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append({"sm": float(parts[1]), "max": float(parts[2]), "power": float(parts[3]),
+                             "hw_slowdown": parts[5], "hw_thermal": parts[6],
+                             "sw_thermal": parts[7], "sw_power_cap": parts[8]})
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        # keep samples at load (the timed region keeps the SMs busy)
+        top = max(r["sm"] for r in rows)
+        busy = [r for r in rows if r["power"] > 0.5 * max(r2["power"] for r2 in rows)] or rows
+        reasons = set()
+        for r in busy:
+            for k in ("hw_slowdown", "hw_thermal", "sw_thermal", "sw_power_cap"):
+                if r[k].lower() == "active":
+                    reasons.add({"hw_thermal": "hw_thermal_slowdown",
+                                 "sw_thermal": "sw_thermal_slowdown"}.get(k, k))
+        return {"sm_mhz": statistics.median(r["sm"] for r in busy), "sm_max_mhz": busy[0]["max"],
+                "sm_mhz_peak_seen": top, "samples": len(busy),
+                "power_w_median": statistics.median(r["power"] for r in busy),
+                "reasons": sorted(reasons)}
+
+
+def physical_gpu(local_rank: int) -> str:
+    """nvidia-smi index (or UUID) of this rank's GPU."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return str(local_rank)
+
+
+# ----------------------------------------------------------------------------
+# CPU baseline: the oracle as it stands, on a bounded sample of the workload
+
+def cpu_rate(w, inp, seconds: float, rows_cap=None):
+    """Time the fp64 oracle on a seeded sample of rows; returns (elem/s, threads, sample)."""
+    import oracle
+    threads = oracle.max_threads()
+    total_rows = w.batch * w.dim
+    g = np.random.default_rng(12345)
+    n = min(total_rows, max(threads, 32))
+    t = time.perf_counter()
+    oracle.scan(**_oracle_kw(inp), rows=np.sort(g.choice(total_rows, n, replace=False)))
+    dt = time.perf_counter() - t
+    per_row = dt / n
+    n = int(min(total_rows, max(n, seconds / max(per_row, 1e-9))))
+    if rows_cap:
+        n = min(n, rows_cap)
+    rows = np.sort(g.choice(total_rows, n, replace=False))
+    t = time.perf_counter()
+    oracle.scan(**_oracle_kw(inp), rows=rows)
+    dt = time.perf_counter() - t
+    elems = n * w.seqlen * w.dstate
+    return elems / dt, threads, f"{n} of {total_rows} rows (seeded), full L={w.seqlen}, N={w.dstate}", dt
+
+
+def _oracle_kw(inp):
+    return dict(u=inp["u"], delta=inp["delta"], A=inp["A"], B=inp["B"], C=inp["C"], D=inp["D"],
+                z=inp["z"], delta_bias=inp["delta_bias"], delta_softplus=True, dtype=inp["dtype"])
+
+
+# ----------------------------------------------------------------------------
+
+def workload_config(w, extra=None):
+    cfg = {"workload": w.name, "batch": w.batch, "d_inner": w.dim, "d_state": w.dstate,
+           "seq_len": w.seqlen, "in_dtype": w.dtype, "state_dtype": "f32", "gate": w.has_z,
+           "l2": f"inputs rotated over {ROTATE} resident copies (> L2 of 126 MB)",
+           "parallelism": "replicas (independent batch per GPU)"}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+def run_reference(args, dist: Dist):
+    """The fp64 CPU oracle as the reference arm: rank 0 only."""
+    if dist.rank != 0:
+        return 0
+    import oracle
+    w = SCAN_WORKLOADS[args.workload]
+    inp = make_scan_inputs(w)
+    threads = oracle.max_threads()
+    total_rows = w.batch * w.dim
+    # size each step so the whole warm-up + timed run takes about a minute
+    rate, _, _, _ = cpu_rate(w, inp, 1.0, rows_cap=4096)
+    per_step_budget = 60.0 / max(1, args.steps + args.warmup)
+    n = int(max(1, min(total_rows, per_step_budget * rate / (w.seqlen * w.dstate))))
+    g = np.random.default_rng(777)
+    samples = [np.sort(g.choice(total_rows, n, replace=False)) for _ in range(4)]
+    kw = _oracle_kw(inp)
+    for s in range(args.warmup):
+        oracle.scan(**kw, rows=samples[s % 4])
+    t = time.perf_counter()
+    for s in range(args.steps):
+        oracle.scan(**kw, rows=samples[s % 4])
+    dt = time.perf_counter() - t
+    elems = args.steps * n * w.seqlen * w.dstate
+    value = elems / dt
+    sample = f"{n} of {total_rows} rows per step (seeded), full L={w.seqlen}, N={w.dstate}"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)", "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, dist: Dist):
+    import torch
+    import selective_state_space_27_b200 as ms
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device (the product path has no CPU fallback)")
+    dev = torch.device("cuda", dist.local_rank)
+    torch.cuda.set_device(dev)
+    dist.init("nccl")
+    w = SCAN_WORKLOADS[args.workload]
+    in_bytes = 4 if w.dtype == "f32" else 2
+    tdt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+
+    inp = make_scan_inputs(w, seed=w.seed + 1000 * dist.rank)
+
+    def host(a):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        return t.view(torch.bfloat16) if (a.dtype == np.uint16) else t
+
+    names = ["u", "delta", "B", "C"] + (["z"] if w.has_z else [])
+    pinned = {k: host(inp[k]).pin_memory() for k in names}
+    params = {k: torch.from_numpy(inp[k]).to(dev) for k in ("A", "D", "delta_bias")}
+    sets = [{k: v.to(dev, non_blocking=True) for k, v in pinned.items()} for _ in range(ROTATE)]
+    y = torch.empty((w.batch, w.dim, w.seqlen), dtype=tdt, device=dev)
+    hT = torch.empty((w.batch, w.dim, w.dstate), dtype=torch.float32, device=dev)
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream()
+    args_list = [ms.build_scan_args(s["u"], s["delta"], params["A"], s["B"], s["C"], y,
+                                    D=params["D"], z=s.get("z"), delta_bias=params["delta_bias"],
+                                    final_state=hT) for s in sets]
+    ws_bytes = ms.scan_workspace_size(args_list[0])
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    lib = ms.load_library()
+    import ctypes
+    launches_per_step = 2 if ws_bytes else 1
+
+    def step(i):
+        rc = lib.mamba_scan_fwd(ctypes.byref(args_list[i % ROTATE]), ws.data_ptr(), ws.numel(),
+                                stream.cuda_stream)
+        if rc != 0:
+            raise ms.MambaScanError(rc, lib.mamba_last_error().decode())
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(physical_gpu(dist.local_rank))
+    if dist.rank == 0:
+        sampler.start()
+    dist.barrier()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    sampler.mark_begin()
+    ev[0].record(stream)
+    for i in range(args.steps):
+        step(i)
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    sampler.mark_end()
+    dist.barrier()
+    elapsed_ms = ev[0].elapsed_time(ev[1])
+    clocks = sampler.stop() if dist.rank == 0 else None
+    elapsed_ms = dist.max(elapsed_ms, dev)
+
+    counts = algorithmic_counts(w, in_bytes)
+    total_elems = counts["elements"] * args.steps * dist.world
+    value = total_elems / (elapsed_ms / 1e3)
+    ms_per_step = elapsed_ms / args.steps
+
+    # ---- end to end through the C ABI with pinned host buffers ----------------
+    e2e = None
+    if args.e2e_steps > 0:
+        y_host = torch.empty(y.shape, dtype=tdt).pin_memory()
+        h_host = torch.empty(hT.shape, dtype=torch.float32).pin_memory()
+        dset = sets[0]
+        h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+        d2h = y_host.numel() * y_host.element_size() + h_host.numel() * 4
+
+        def e2e_step():
+            for k, v in pinned.items():
+                dset[k].copy_(v, non_blocking=True)
+            step(0)
+            y_host.copy_(y, non_blocking=True)
+            h_host.copy_(hT, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = dist.max(e0.elapsed_time(e1), dev)
+        e2e = {"value": counts["elements"] * args.e2e_steps * dist.world / (e2e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e2e_ms / args.e2e_steps}
+
+    # ---- roofline of the scan kernel (the only kernel of a step) --------------
+    peaks = load_peaks()
+    sm_mhz = peaks["sm_max_mhz"]
+    mufu_peak = SMS_B200 * MUFU_PER_CLK * sm_mhz * 1e6          # ex2-class results / s
+    fp32_peak = SMS_B200 * FP32_PER_CLK * sm_mhz * 1e6
+    t_kernel = ms_per_step / 1e3   # every launch of a step belongs to the scan
+    achieved_mufu = counts["mufu"] / t_kernel
+    t_bounds = {"hbm": counts["bytes"] / (peaks["hbm_gbs"] * 1e9), "mufu": counts["mufu"] / mufu_peak,
+                "fp32": counts["fp32"] / fp32_peak}
+    roofline = {
+        "bound": "alu", "unit": "Tmufu/s", "achieved": achieved_mufu / 1e12, "peak": mufu_peak / 1e12,
+        "frac": achieved_mufu / mufu_peak, "traffic": None,
+        "kernel": "scan_kernel (selective scan forward, fused)",
+        "peak_note": f"MUFU: {SMS_B200} SMs x {MUFU_PER_CLK}/clk x {sm_mhz:.0f} MHz (nominal max clock)",
+        "algorithmic_per_launch": counts,
+        "hbm": {"achieved_gbs": counts["bytes"] / t_kernel / 1e9, "peak_gbs": peaks["hbm_gbs"],
+                "frac": counts["bytes"] / t_kernel / 1e9 / peaks["hbm_gbs"], "peak_source": peaks["source"]},
+        "bound_times_us": {k: v * 1e6 for k, v in t_bounds.items()},
+        "kernel_us": t_kernel * 1e6,
+        "roofline_elem_per_s": counts["elements"] / max(t_bounds.values()),
+    }
+
+    cpu = None
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        rate, threads, sample, secs = cpu_rate(w, inp, args.cpu_seconds)
+        cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample,
+               "seconds": secs}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": dist.world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded)", "config": workload_config(w, {"global_batch": w.batch * dist.world}),
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": args.steps * launches_per_step, "clocks": clocks,
+    }
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.barrier()
+    dist.close()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    dist = Dist()
+    if args.impl == "reference":
+        return run_reference(args, dist)
+    return run_ours(args, dist)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

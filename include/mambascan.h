@@ -1,0 +1,187 @@
+/*
+ * mambascan.h -- C ABI of the B200 (sm_100a) selective-scan (S6) library.
+ *
+ * Two operations of the Mamba selective state-space layer:
+ *
+ *  mamba_scan_fwd      the fused selective scan over a whole sequence
+ *  mamba_state_update  the single-token state update used for decoding
+ *
+ * Both compute, per channel row (b, d) and state index n < dstate,
+ *
+ *   delta   = delta_raw + delta_bias[d]            (bias, if given, added first)
+ *   delta   = log(1 + exp(delta))                  if delta_softplus (identity above 20)
+ *   h[n]    = exp(delta * A[d,n]) * h[n] + delta * B[n] * x      (first-order Bbar)
+ *   y       = sum_n C[n] * h[n] + D[d] * x                        (after the update)
+ *   y       = y * z * sigmoid(z)                                  if z is given
+ *
+ * as defined on the pages this library follows:
+ *  - "Notas sobre Mamba", section "O mecanismo de seleção (S6)": input
+ *    dependent B_t, C_t and delta_t = softplus(Linear(x_t) + bias); diagonal
+ *    A = -exp(A_log); h_t = Abar_t h_{t-1} + Bbar_t x_t, y_t = C_t^T h_t;
+ *    Abar = exp(delta A), Bbar = delta B.
+ *  - "Notas sobre Mamba", section "Preliminares": the implementation uses the
+ *    first-order Bbar_t = delta_t B_t rather than the full ZOH expression.
+ *  - "Notas sobre Mamba", section "A varredura paralela ciente do hardware":
+ *    the recurrence is an associative scan over the pairs (Abar_t, Bbar_t x_t);
+ *    discretised parameters and the N-dimensional state stay on chip and only
+ *    the output is written back.
+ *  - "Mamba-2 e State Space Duality (SSD)", section "Como o Mamba-1 alcançou
+ *    complexidade linear": y_t = C_t h_t + D x_t and the decode step.
+ *  - "Notas sobre Mamba", section "O bloco Mamba": the S6 output is gated by
+ *    SiLU of the second branch z.
+ *
+ * Conventions shared by every entry point:
+ *  - All tensor pointers are DEVICE pointers, allocated and owned by the
+ *    caller. The library allocates nothing and keeps no state between calls
+ *    beyond a per-device cache of device properties.
+ *  - Strides are in ELEMENTS of the tensor's own type. The innermost axis
+ *    (L for the scan, dstate for states, dim for decode vectors) must be
+ *    contiguous (stride 1).
+ *  - `in_dtype` (ms_dtype) is the type of u/x, delta, B, C, z and y. A, D,
+ *    delta_bias and all states are float32. Arithmetic is float32.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and nothing synchronises. A status other than MS_OK means that
+ *    nothing was launched, except MS_ERR_CUDA, which reports a launch error
+ *    (kernels already queued by the same call may have run). Faults that
+ *    happen while a kernel runs surface at the caller's next synchronisation.
+ *  - Outputs must not alias inputs (the decode state is updated in place and
+ *    is the one in/out argument).
+ *  - Calls are thread safe; concurrent calls on different streams must not
+ *    share output or workspace buffers.
+ */
+#ifndef MAMBASCAN_H
+#define MAMBASCAN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MAMBASCAN_ABI_VERSION 1
+/* Largest state size N supported by the kernels. */
+#define MS_MAX_DSTATE 16
+
+typedef enum ms_status {
+    MS_OK = 0,
+    MS_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, bad stride, bad enum   */
+    MS_ERR_UNSUPPORTED = 2,  /* valid but outside what the kernels support (dstate>16)   */
+    MS_ERR_ALIGNMENT = 3,    /* a pointer is not aligned to its element size             */
+    MS_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed              */
+    MS_ERR_TIMEOUT = 5,      /* reserved: a bounded device wait gave up (none is used)    */
+    MS_ERR_WORKSPACE = 6     /* workspace missing or smaller than the size asked for      */
+} ms_status;
+
+typedef enum ms_dtype {
+    MS_F32 = 0,
+    MS_BF16 = 1
+} ms_dtype;
+
+/*
+ * Arguments of the selective scan forward.
+ *
+ *   u, delta, z, y : (batch, dim, seqlen), L contiguous, strides
+ *                    (*_batch_stride, *_dim_stride). z may be NULL (no gate).
+ *   B, C           : (batch, dstate, seqlen), L contiguous, strides
+ *                    (*_batch_stride, *_state_stride); shared by every channel d.
+ *   A              : (dim, dstate) float32, contiguous. Usually -exp(A_log).
+ *   D, delta_bias  : (dim) float32, or NULL for zero.
+ *   initial_state  : (batch, dim, dstate) float32 contiguous, or NULL for zero.
+ *   final_state    : (batch, dim, dstate) float32 contiguous, or NULL (not written).
+ *   force_segments : 0 = automatic. >0 splits the sequence of every row into
+ *                    that many segments joined by the multi-block carry pass
+ *                    (the count is capped at the number of 16-step blocks).
+ */
+typedef struct ms_scan_args {
+    int64_t batch, dim, dstate, seqlen;
+    int32_t in_dtype;
+    int32_t delta_softplus;
+
+    const void *u;      int64_t u_batch_stride, u_dim_stride;
+    const void *delta;  int64_t delta_batch_stride, delta_dim_stride;
+    const void *B;      int64_t B_batch_stride, B_state_stride;
+    const void *C;      int64_t C_batch_stride, C_state_stride;
+    const void *z;      int64_t z_batch_stride, z_dim_stride;
+    void *y;            int64_t y_batch_stride, y_dim_stride;
+
+    const float *A;
+    const float *D;
+    const float *delta_bias;
+    const float *initial_state;
+    float *final_state;
+
+    int32_t force_segments;
+    int32_t reserved;   /* must be 0 */
+} ms_scan_args;
+
+/*
+ * Arguments of the single-token state update (decode).
+ *
+ *   state          : (batch, dim, dstate) float32, dstate contiguous, strides
+ *                    (state_batch_stride, state_dim_stride). Updated IN PLACE.
+ *   x, delta, z, y : (batch, dim), dim contiguous, batch stride *_batch_stride.
+ *                    z may be NULL.
+ *   B, C           : (batch, dstate), dstate contiguous, batch stride *_batch_stride.
+ *   A              : (dim, dstate) float32 contiguous; D, delta_bias: (dim) or NULL.
+ */
+typedef struct ms_update_args {
+    int64_t batch, dim, dstate;
+    int32_t in_dtype;
+    int32_t delta_softplus;
+
+    float *state;       int64_t state_batch_stride, state_dim_stride;
+    const void *x;      int64_t x_batch_stride;
+    const void *delta;  int64_t delta_batch_stride;
+    const void *B;      int64_t B_batch_stride;
+    const void *C;      int64_t C_batch_stride;
+    const void *z;      int64_t z_batch_stride;
+    void *y;            int64_t y_batch_stride;
+
+    const float *A;
+    const float *D;
+    const float *delta_bias;
+} ms_update_args;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *mamba_status_string(int status);
+
+/* Message of the last MS_ERR_CUDA / MS_ERR_INVALID_ARG on this thread (static
+ * thread-local buffer, never NULL, "" if none). */
+const char *mamba_last_error(void);
+
+/* MAMBASCAN_ABI_VERSION of the loaded library. */
+int mamba_abi_version(void);
+
+/*
+ * Bytes of device workspace that mamba_scan_fwd needs for these arguments
+ * (written to *bytes; 0 when the sequence is not split into segments).
+ * Validates the arguments like mamba_scan_fwd, without touching the device
+ * memory they point to. The caller allocates the workspace (256-byte aligned)
+ * and may reuse it across calls on one stream.
+ */
+ms_status mamba_scan_workspace_size(const ms_scan_args *args, size_t *bytes);
+
+/*
+ * Selective scan forward: y for every (b, d, t) and, if requested, the state
+ * after the last step. The expanded (batch, dim, seqlen, dstate) state is
+ * never written to memory. `workspace` may be NULL when the size query gave 0.
+ * Errors: MS_ERR_INVALID_ARG, MS_ERR_UNSUPPORTED (dstate > 16),
+ * MS_ERR_ALIGNMENT (a pointer not aligned to its element type),
+ * MS_ERR_WORKSPACE, MS_ERR_CUDA.
+ */
+ms_status mamba_scan_fwd(const ms_scan_args *args, void *workspace, size_t workspace_bytes,
+                         void *stream);
+
+/*
+ * Single-token selective state update: state <- exp(delta A) state + delta B x
+ * in place, then y = C . state + D x (times silu(z)). One launch; no workspace.
+ * Errors: as mamba_scan_fwd, without MS_ERR_WORKSPACE.
+ */
+ms_status mamba_state_update(const ms_update_args *args, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MAMBASCAN_H */

@@ -1,0 +1,291 @@
+"""B200 (sm_100a) selective scan (S6): Python binding of the C ABI in include/mambascan.h.
+
+Two operations of the Mamba selective state-space layer ("Notas sobre Mamba",
+section "O mecanismo de seleção (S6)"; "Mamba-2 e State Space Duality (SSD)",
+section "Como o Mamba-1 alcançou complexidade linear"):
+
+* :func:`scan_fwd` -- the fused selective scan over a sequence: y and the final
+  state, with delta = softplus(delta_raw + delta_bias), Abar = exp(delta A),
+  Bbar = delta B, h_t = Abar_t h_{t-1} + Bbar_t u_t, y_t = C_t h_t + D u_t,
+  optionally times silu(z_t).
+* :func:`state_update` -- the same recurrence for one token, on a state
+  updated in place (decode).
+
+This module only marshals arguments: PyTorch supplies device memory and the
+current CUDA stream, and every step of the computation runs in the CUDA
+kernels of ``libmambascan.so``. There is no CPU fallback: if the library is
+missing or cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "scan_fwd", "state_update", "scan_workspace_size", "library_path", "load_library",
+    "MambaScanError", "ScanArgs", "UpdateArgs", "MS_F32", "MS_BF16", "MAX_DSTATE",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libmambascan.so")
+_lib = None
+
+MS_F32, MS_BF16 = 0, 1
+MAX_DSTATE = 16
+STATUS = {0: "MS_OK", 1: "MS_ERR_INVALID_ARG", 2: "MS_ERR_UNSUPPORTED", 3: "MS_ERR_ALIGNMENT",
+          4: "MS_ERR_CUDA", 5: "MS_ERR_TIMEOUT", 6: "MS_ERR_WORKSPACE"}
+
+_i64 = ctypes.c_int64
+_i32 = ctypes.c_int32
+_vp = ctypes.c_void_p
+
+
+class ScanArgs(ctypes.Structure):
+    """Mirror of ``ms_scan_args``."""
+    _fields_ = [
+        ("batch", _i64), ("dim", _i64), ("dstate", _i64), ("seqlen", _i64),
+        ("in_dtype", _i32), ("delta_softplus", _i32),
+        ("u", _vp), ("u_batch_stride", _i64), ("u_dim_stride", _i64),
+        ("delta", _vp), ("delta_batch_stride", _i64), ("delta_dim_stride", _i64),
+        ("B", _vp), ("B_batch_stride", _i64), ("B_state_stride", _i64),
+        ("C", _vp), ("C_batch_stride", _i64), ("C_state_stride", _i64),
+        ("z", _vp), ("z_batch_stride", _i64), ("z_dim_stride", _i64),
+        ("y", _vp), ("y_batch_stride", _i64), ("y_dim_stride", _i64),
+        ("A", _vp), ("D", _vp), ("delta_bias", _vp), ("initial_state", _vp), ("final_state", _vp),
+        ("force_segments", _i32), ("reserved", _i32),
+    ]
+
+
+class UpdateArgs(ctypes.Structure):
+    """Mirror of ``ms_update_args``."""
+    _fields_ = [
+        ("batch", _i64), ("dim", _i64), ("dstate", _i64),
+        ("in_dtype", _i32), ("delta_softplus", _i32),
+        ("state", _vp), ("state_batch_stride", _i64), ("state_dim_stride", _i64),
+        ("x", _vp), ("x_batch_stride", _i64),
+        ("delta", _vp), ("delta_batch_stride", _i64),
+        ("B", _vp), ("B_batch_stride", _i64),
+        ("C", _vp), ("C_batch_stride", _i64),
+        ("z", _vp), ("z_batch_stride", _i64),
+        ("y", _vp), ("y_batch_stride", _i64),
+        ("A", _vp), ("D", _vp), ("delta_bias", _vp),
+    ]
+
+
+class MambaScanError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load libmambascan.so (built by ``python -m selective_state_space_27_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"CUDA library not built: {_LIB_PATH} is missing "
+                               "(run python -m selective_state_space_27_b200.build)")
+        lib = ctypes.CDLL(_LIB_PATH)
+        lib.mamba_status_string.restype = ctypes.c_char_p
+        lib.mamba_status_string.argtypes = [ctypes.c_int]
+        lib.mamba_last_error.restype = ctypes.c_char_p
+        lib.mamba_last_error.argtypes = []
+        lib.mamba_abi_version.restype = ctypes.c_int
+        lib.mamba_abi_version.argtypes = []
+        lib.mamba_scan_workspace_size.restype = ctypes.c_int
+        lib.mamba_scan_workspace_size.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(ctypes.c_size_t)]
+        lib.mamba_scan_fwd.restype = ctypes.c_int
+        lib.mamba_scan_fwd.argtypes = [ctypes.POINTER(ScanArgs), _vp, ctypes.c_size_t, _vp]
+        lib.mamba_state_update.restype = ctypes.c_int
+        lib.mamba_state_update.argtypes = [ctypes.POINTER(UpdateArgs), _vp]
+        if lib.mamba_abi_version() != 1:
+            raise RuntimeError("libmambascan.so ABI version mismatch")
+        _lib = lib
+    return _lib
+
+
+def _check(status: int):
+    if status != 0:
+        msg = load_library().mamba_last_error().decode(errors="replace")
+        raise MambaScanError(status, msg)
+
+
+# ----------------------------------------------------------------------------
+# torch marshalling
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return MS_F32
+    if t.dtype == torch.bfloat16:
+        return MS_BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream_ptr(stream):
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _need_cuda(name, t, dtype=None, ndim=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions")
+    if t.dim() > 0 and t.stride(-1) != 1 and t.shape[-1] > 1:
+        raise ValueError(f"{name} must be contiguous in its last dimension")
+
+
+def build_scan_args(u, delta, A, B, C, y, *, D=None, z=None, delta_bias=None,
+                    delta_softplus=True, initial_state=None, final_state=None,
+                    force_segments=0) -> ScanArgs:
+    """Fill an ``ms_scan_args`` from torch tensors (no checks beyond dtype/layout)."""
+    torch = _torch()
+    batch, dim, L = u.shape
+    dstate = B.shape[1]
+    f32 = torch.float32
+    dt = u.dtype
+    for name, t in (("u", u), ("delta", delta), ("z", z), ("y", y)):
+        _need_cuda(name, t, dt, 3)
+        if t is not None and tuple(t.shape) != (batch, dim, L):
+            raise ValueError(f"{name} must have shape {(batch, dim, L)}, got {tuple(t.shape)}")
+    for name, t in (("B", B), ("C", C)):
+        _need_cuda(name, t, dt, 3)
+        if tuple(t.shape) != (batch, dstate, L):
+            raise ValueError(f"{name} must have shape {(batch, dstate, L)}, got {tuple(t.shape)}")
+    _need_cuda("A", A, f32, 2)
+    if tuple(A.shape) != (dim, dstate) or not A.is_contiguous():
+        raise ValueError("A must be a contiguous (dim, dstate) float32 tensor")
+    for name, t in (("D", D), ("delta_bias", delta_bias)):
+        _need_cuda(name, t, f32, 1)
+        if t is not None and (tuple(t.shape) != (dim,) or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous ({dim},) float32 tensor")
+    for name, t in (("initial_state", initial_state), ("final_state", final_state)):
+        _need_cuda(name, t, f32, 3)
+        if t is not None and (tuple(t.shape) != (batch, dim, dstate) or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous {(batch, dim, dstate)} float32 tensor")
+    a = ScanArgs()
+    a.batch, a.dim, a.dstate, a.seqlen = batch, dim, dstate, L
+    a.in_dtype = _dtype_code(u)
+    a.delta_softplus = 1 if delta_softplus else 0
+    a.u, a.u_batch_stride, a.u_dim_stride = _ptr(u), u.stride(0), u.stride(1)
+    a.delta, a.delta_batch_stride, a.delta_dim_stride = _ptr(delta), delta.stride(0), delta.stride(1)
+    a.B, a.B_batch_stride, a.B_state_stride = _ptr(B), B.stride(0), B.stride(1)
+    a.C, a.C_batch_stride, a.C_state_stride = _ptr(C), C.stride(0), C.stride(1)
+    if z is not None:
+        a.z, a.z_batch_stride, a.z_dim_stride = _ptr(z), z.stride(0), z.stride(1)
+    a.y, a.y_batch_stride, a.y_dim_stride = _ptr(y), y.stride(0), y.stride(1)
+    a.A, a.D, a.delta_bias = _ptr(A), _ptr(D), _ptr(delta_bias)
+    a.initial_state, a.final_state = _ptr(initial_state), _ptr(final_state)
+    a.force_segments = int(force_segments)
+    a.reserved = 0
+    return a
+
+
+def scan_workspace_size(args: ScanArgs) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load_library().mamba_scan_workspace_size(ctypes.byref(args), ctypes.byref(n)))
+    return int(n.value)
+
+
+def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
+             initial_state=None, return_last_state=True, out=None, force_segments=0,
+             workspace=None, stream=None):
+    """Selective scan forward on the current (or given) CUDA stream.
+
+    u, delta, z: (batch, dim, L); B, C: (batch, dstate, L) -- all float32 or
+    all bfloat16, contiguous along L. A: (dim, dstate) float32 (normally
+    -exp(A_log)); D, delta_bias: (dim,) float32. Returns y (u's dtype), and
+    the final float32 state (batch, dim, dstate) when ``return_last_state``.
+    ``workspace``: optional uint8 CUDA tensor reused for the multi-block carry
+    (allocated here when needed and not given).
+    """
+    torch = _torch()
+    y = torch.empty_like(u) if out is None else out
+    hT = None
+    if return_last_state:
+        hT = torch.empty((u.shape[0], u.shape[1], B.shape[1]), device=u.device, dtype=torch.float32)
+    args = build_scan_args(u, delta, A, B, C, y, D=D, z=z, delta_bias=delta_bias,
+                           delta_softplus=delta_softplus, initial_state=initial_state,
+                           final_state=hT, force_segments=force_segments)
+    lib = load_library()
+    with torch.cuda.device(u.device):
+        need = scan_workspace_size(args)
+        ws_ptr, ws_bytes = None, 0
+        if need:
+            if workspace is None or workspace.numel() < need:
+                workspace = torch.empty(need, dtype=torch.uint8, device=u.device)
+            ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
+        _check(lib.mamba_scan_fwd(ctypes.byref(args), ws_ptr, ws_bytes, _stream_ptr(stream)))
+    return (y, hT) if return_last_state else y
+
+
+def build_update_args(state, x, delta, A, B, C, y, *, D=None, z=None, delta_bias=None,
+                      delta_softplus=True) -> UpdateArgs:
+    torch = _torch()
+    batch, dim = x.shape
+    dstate = B.shape[1]
+    dt = x.dtype
+    _need_cuda("state", state, torch.float32, 3)
+    if tuple(state.shape) != (batch, dim, dstate):
+        raise ValueError(f"state must have shape {(batch, dim, dstate)}")
+    for name, t in (("x", x), ("delta", delta), ("z", z), ("y", y)):
+        _need_cuda(name, t, dt, 2)
+        if t is not None and tuple(t.shape) != (batch, dim):
+            raise ValueError(f"{name} must have shape {(batch, dim)}")
+    for name, t in (("B", B), ("C", C)):
+        _need_cuda(name, t, dt, 2)
+        if tuple(t.shape) != (batch, dstate):
+            raise ValueError(f"{name} must have shape {(batch, dstate)}")
+    _need_cuda("A", A, torch.float32, 2)
+    if tuple(A.shape) != (dim, dstate) or not A.is_contiguous():
+        raise ValueError("A must be a contiguous (dim, dstate) float32 tensor")
+    for name, t in (("D", D), ("delta_bias", delta_bias)):
+        _need_cuda(name, t, torch.float32, 1)
+        if t is not None and (tuple(t.shape) != (dim,) or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous ({dim},) float32 tensor")
+    a = UpdateArgs()
+    a.batch, a.dim, a.dstate = batch, dim, dstate
+    a.in_dtype = _dtype_code(x)
+    a.delta_softplus = 1 if delta_softplus else 0
+    a.state, a.state_batch_stride, a.state_dim_stride = _ptr(state), state.stride(0), state.stride(1)
+    a.x, a.x_batch_stride = _ptr(x), x.stride(0)
+    a.delta, a.delta_batch_stride = _ptr(delta), delta.stride(0)
+    a.B, a.B_batch_stride = _ptr(B), B.stride(0)
+    a.C, a.C_batch_stride = _ptr(C), C.stride(0)
+    if z is not None:
+        a.z, a.z_batch_stride = _ptr(z), z.stride(0)
+    a.y, a.y_batch_stride = _ptr(y), y.stride(0)
+    a.A, a.D, a.delta_bias = _ptr(A), _ptr(D), _ptr(delta_bias)
+    return a
+
+
+def state_update(state, x, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
+                 out=None, stream=None):
+    """One decode step: updates ``state`` (batch, dim, dstate) float32 in place; returns y (batch, dim)."""
+    torch = _torch()
+    y = torch.empty_like(x) if out is None else out
+    args = build_update_args(state, x, delta, A, B, C, y, D=D, z=z, delta_bias=delta_bias,
+                             delta_softplus=delta_softplus)
+    with torch.cuda.device(x.device):
+        _check(load_library().mamba_state_update(ctypes.byref(args), _stream_ptr(stream)))
+    return y

@@ -1,0 +1,225 @@
+// C ABI of the selective-scan library: argument validation, launch planning
+// and dispatch. Declarations and the contract are in include/mambascan.h.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "launch.h"
+#include "mambascan.h"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+void set_error(const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+}
+
+ms_status invalid(const char *what) {
+    set_error("invalid argument: %s", what);
+    return MS_ERR_INVALID_ARG;
+}
+
+ms_status cuda_fail(cudaError_t e, const char *where) {
+    set_error("%s: %s", where, cudaGetErrorString(e));
+    return MS_ERR_CUDA;
+}
+
+// Number of SMs of the current device, cached per device.
+constexpr int kMaxDevices = 64;
+int g_sms[kMaxDevices] = {0};
+std::mutex g_sms_mu;
+
+ms_status device_sms(int *out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev >= 0 && dev < kMaxDevices) {
+        std::lock_guard<std::mutex> lk(g_sms_mu);
+        if (g_sms[dev] == 0) {
+            int sms = 0;
+            e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+            g_sms[dev] = sms;
+        }
+        *out = g_sms[dev];
+        return MS_OK;
+    }
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    *out = sms;
+    return MS_OK;
+}
+
+bool elem_aligned(const void *ptr, int eb) {
+    return (reinterpret_cast<uintptr_t>(ptr) % static_cast<uintptr_t>(eb)) == 0;
+}
+
+ms_status check_scan(const ms_scan_args *a) {
+    if (!a) return invalid("args is NULL");
+    if (a->batch <= 0 || a->dim <= 0 || a->dstate <= 0 || a->seqlen <= 0)
+        return invalid("batch, dim, dstate and seqlen must be positive");
+    if (a->in_dtype != MS_F32 && a->in_dtype != MS_BF16) return invalid("in_dtype");
+    if (a->reserved != 0) return invalid("reserved must be 0");
+    if (a->force_segments < 0) return invalid("force_segments must be >= 0");
+    if (!a->u || !a->delta || !a->B || !a->C || !a->A || !a->y)
+        return invalid("u, delta, B, C, A and y are required");
+    if (a->u_batch_stride < 0 || a->u_dim_stride < 0 || a->delta_batch_stride < 0 ||
+        a->delta_dim_stride < 0 || a->B_batch_stride < 0 || a->B_state_stride < 0 ||
+        a->C_batch_stride < 0 || a->C_state_stride < 0 || a->y_batch_stride < 0 ||
+        a->y_dim_stride < 0 || (a->z && (a->z_batch_stride < 0 || a->z_dim_stride < 0)))
+        return invalid("strides must be non-negative");
+    if (a->dstate > MS_MAX_DSTATE) {
+        set_error("dstate %lld exceeds the supported maximum %d", static_cast<long long>(a->dstate),
+                  MS_MAX_DSTATE);
+        return MS_ERR_UNSUPPORTED;
+    }
+    if (a->batch > 65535) {
+        set_error("batch %lld exceeds 65535", static_cast<long long>(a->batch));
+        return MS_ERR_UNSUPPORTED;
+    }
+    const int eb = a->in_dtype == MS_F32 ? 4 : 2;
+    if (!elem_aligned(a->u, eb) || !elem_aligned(a->delta, eb) || !elem_aligned(a->B, eb) ||
+        !elem_aligned(a->C, eb) || !elem_aligned(a->y, eb) || (a->z && !elem_aligned(a->z, eb)) ||
+        !elem_aligned(a->A, 4) || (a->D && !elem_aligned(a->D, 4)) ||
+        (a->delta_bias && !elem_aligned(a->delta_bias, 4)) ||
+        (a->initial_state && !elem_aligned(a->initial_state, 4)) ||
+        (a->final_state && !elem_aligned(a->final_state, 4))) {
+        set_error("a pointer is not aligned to its element size");
+        return MS_ERR_ALIGNMENT;
+    }
+    return MS_OK;
+}
+
+ms::ScanParams to_params(const ms_scan_args *a) {
+    ms::ScanParams p{};
+    p.batch = a->batch; p.dim = a->dim; p.dstate = a->dstate; p.seqlen = a->seqlen;
+    p.u = a->u; p.u_sb = a->u_batch_stride; p.u_sd = a->u_dim_stride;
+    p.delta = a->delta; p.dl_sb = a->delta_batch_stride; p.dl_sd = a->delta_dim_stride;
+    p.B = a->B; p.B_sb = a->B_batch_stride; p.B_sn = a->B_state_stride;
+    p.C = a->C; p.C_sb = a->C_batch_stride; p.C_sn = a->C_state_stride;
+    p.z = a->z; p.z_sb = a->z_batch_stride; p.z_sd = a->z_dim_stride;
+    p.y = a->y; p.y_sb = a->y_batch_stride; p.y_sd = a->y_dim_stride;
+    p.A = a->A; p.D = a->D; p.delta_bias = a->delta_bias;
+    p.h0 = a->initial_state; p.hT = a->final_state;
+    p.softplus = a->delta_softplus ? 1 : 0;
+    return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *mamba_status_string(int status) {
+    switch (status) {
+        case MS_OK: return "MS_OK";
+        case MS_ERR_INVALID_ARG: return "MS_ERR_INVALID_ARG";
+        case MS_ERR_UNSUPPORTED: return "MS_ERR_UNSUPPORTED";
+        case MS_ERR_ALIGNMENT: return "MS_ERR_ALIGNMENT";
+        case MS_ERR_CUDA: return "MS_ERR_CUDA";
+        case MS_ERR_TIMEOUT: return "MS_ERR_TIMEOUT";
+        case MS_ERR_WORKSPACE: return "MS_ERR_WORKSPACE";
+        default: return "MS_UNKNOWN_STATUS";
+    }
+}
+
+const char *mamba_last_error(void) { return g_last_error; }
+
+int mamba_abi_version(void) { return MAMBASCAN_ABI_VERSION; }
+
+ms_status mamba_scan_workspace_size(const ms_scan_args *args, size_t *bytes) {
+    if (!bytes) return invalid("bytes is NULL");
+    *bytes = 0;
+    ms_status st = check_scan(args);
+    if (st != MS_OK) return st;
+    int sms = 0;
+    st = device_sms(&sms);
+    if (st != MS_OK) return st;
+    const ms::ScanParams p = to_params(args);
+    *bytes = ms::plan_scan(p, args->in_dtype, args->force_segments, sms).ws_bytes;
+    return MS_OK;
+}
+
+ms_status mamba_scan_fwd(const ms_scan_args *args, void *workspace, size_t workspace_bytes,
+                         void *stream) {
+    ms_status st = check_scan(args);
+    if (st != MS_OK) return st;
+    int sms = 0;
+    st = device_sms(&sms);
+    if (st != MS_OK) return st;
+    ms::ScanParams p = to_params(args);
+    const ms::ScanPlan plan = ms::plan_scan(p, args->in_dtype, args->force_segments, sms);
+    if (plan.ws_bytes > 0) {
+        if (!workspace || workspace_bytes < plan.ws_bytes) {
+            set_error("workspace of %zu bytes needed, %zu given", plan.ws_bytes,
+                      workspace ? workspace_bytes : static_cast<size_t>(0));
+            return MS_ERR_WORKSPACE;
+        }
+        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) {
+            set_error("workspace must be 256-byte aligned");
+            return MS_ERR_ALIGNMENT;
+        }
+        float *ws = static_cast<float *>(workspace);
+        const size_t half = plan.ws_bytes / 2 / sizeof(float);
+        p.ws_P = ws;
+        p.ws_H = ws + half;
+    }
+    p.nseg = plan.nseg;
+    p.seg_len = plan.seg_len;
+    const cudaError_t e = ms::launch_scan(p, plan, args->in_dtype, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "scan kernel launch");
+    return MS_OK;
+}
+
+ms_status mamba_state_update(const ms_update_args *a, void *stream) {
+    if (!a) return invalid("args is NULL");
+    if (a->batch <= 0 || a->dim <= 0 || a->dstate <= 0)
+        return invalid("batch, dim and dstate must be positive");
+    if (a->in_dtype != MS_F32 && a->in_dtype != MS_BF16) return invalid("in_dtype");
+    if (!a->state || !a->x || !a->delta || !a->B || !a->C || !a->A || !a->y)
+        return invalid("state, x, delta, B, C, A and y are required");
+    if (a->state_batch_stride < 0 || a->state_dim_stride < 0 || a->x_batch_stride < 0 ||
+        a->delta_batch_stride < 0 || a->B_batch_stride < 0 || a->C_batch_stride < 0 ||
+        a->y_batch_stride < 0 || (a->z && a->z_batch_stride < 0))
+        return invalid("strides must be non-negative");
+    if (a->dstate > MS_MAX_DSTATE) {
+        set_error("dstate %lld exceeds the supported maximum %d", static_cast<long long>(a->dstate),
+                  MS_MAX_DSTATE);
+        return MS_ERR_UNSUPPORTED;
+    }
+    if (a->batch * a->dim * 4 > (static_cast<int64_t>(1) << 40)) {
+        set_error("batch * dim too large");
+        return MS_ERR_UNSUPPORTED;
+    }
+    const int eb = a->in_dtype == MS_F32 ? 4 : 2;
+    if (!elem_aligned(a->state, 4) || !elem_aligned(a->x, eb) || !elem_aligned(a->delta, eb) ||
+        !elem_aligned(a->B, eb) || !elem_aligned(a->C, eb) || !elem_aligned(a->y, eb) ||
+        (a->z && !elem_aligned(a->z, eb)) || !elem_aligned(a->A, 4) ||
+        (a->D && !elem_aligned(a->D, 4)) || (a->delta_bias && !elem_aligned(a->delta_bias, 4))) {
+        set_error("a pointer is not aligned to its element size");
+        return MS_ERR_ALIGNMENT;
+    }
+    ms::UpdateParams p{};
+    p.batch = a->batch; p.dim = a->dim; p.dstate = a->dstate;
+    p.state = a->state; p.s_sb = a->state_batch_stride; p.s_sd = a->state_dim_stride;
+    p.x = a->x; p.x_sb = a->x_batch_stride;
+    p.delta = a->delta; p.dl_sb = a->delta_batch_stride;
+    p.B = a->B; p.B_sb = a->B_batch_stride;
+    p.C = a->C; p.C_sb = a->C_batch_stride;
+    p.z = a->z; p.z_sb = a->z_batch_stride;
+    p.y = a->y; p.y_sb = a->y_batch_stride;
+    p.A = a->A; p.D = a->D; p.delta_bias = a->delta_bias;
+    p.softplus = a->delta_softplus ? 1 : 0;
+    const cudaError_t e = ms::launch_state_update(p, a->in_dtype, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "state update kernel launch");
+    return MS_OK;
+}
+
+}  // extern "C"

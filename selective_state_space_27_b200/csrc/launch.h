@@ -1,0 +1,58 @@
+// Internal host-side interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ms {
+
+// Everything a scan kernel reads, in one by-value kernel parameter.
+struct ScanParams {
+    int64_t batch, dim, dstate, seqlen;
+    const void *u;     int64_t u_sb, u_sd;
+    const void *delta; int64_t dl_sb, dl_sd;
+    const void *B;     int64_t B_sb, B_sn;
+    const void *C;     int64_t C_sb, C_sn;
+    const void *z;     int64_t z_sb, z_sd;
+    void *y;           int64_t y_sb, y_sd;
+    const float *A, *D, *delta_bias, *h0;
+    float *hT;
+    int softplus;
+    int nseg;           // segments per row (1 = no multi-block carry)
+    int64_t seg_len;    // time steps per segment, a multiple of the chunk length
+    float *ws_P;        // (batch*dim, nseg, 16): decay product of each segment
+    float *ws_H;        // (batch*dim, nseg, 16): end state of each segment from zero
+};
+
+// Launch configuration chosen on the host for one scan call.
+struct ScanPlan {
+    int lg;             // lanes that share one row's chunk (4 or 8)
+    int warps;          // warps per CTA
+    int rows_per_cta;   // warps * (32 / lg)
+    int chunk;          // time steps per chunk = lg * 16
+    int vec;            // 1 if every row start is 16-byte aligned (vector path)
+    int nseg;
+    int64_t seg_len;
+    size_t ws_bytes;
+};
+
+ScanPlan plan_scan(const ScanParams &p, int in_dtype, int force_segments, int num_sms);
+cudaError_t launch_scan(const ScanParams &p, const ScanPlan &plan, int in_dtype,
+                        cudaStream_t stream);
+
+struct UpdateParams {
+    int64_t batch, dim, dstate;
+    float *state;      int64_t s_sb, s_sd;
+    const void *x;     int64_t x_sb;
+    const void *delta; int64_t dl_sb;
+    const void *B;     int64_t B_sb;
+    const void *C;     int64_t C_sb;
+    const void *z;     int64_t z_sb;
+    void *y;           int64_t y_sb;
+    const float *A, *D, *delta_bias;
+    int softplus;
+};
+
+cudaError_t launch_state_update(const UpdateParams &p, int in_dtype, cudaStream_t stream);
+
+}  // namespace ms

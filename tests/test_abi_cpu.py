@@ -1,0 +1,144 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol the header
+declares, its structs match the binding's mirrors, and host-side validation
+rejects bad arguments before touching CUDA."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import selective_state_space_27_b200 as ms
+from selective_state_space_27_b200 import build as msbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mambascan.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    msbuild.build()
+    return ms.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(mamba_[a-z_0-9]+)\s*\(",
+                       text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for want in ("mamba_scan_fwd", "mamba_state_update", "mamba_scan_workspace_size",
+                 "mamba_status_string", "mamba_last_error", "mamba_abi_version"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", ms.library_path()], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    for n in declared_functions():
+        assert hasattr(lib, n)
+
+
+def test_struct_layout_matches_binding(tmp_path):
+    src = tmp_path / "layout.c"
+    src.write_text(
+        '#include <stdio.h>\n#include <stddef.h>\n#include "mambascan.h"\n'
+        "int main(void){printf(\"%zu %zu %zu %zu %zu %zu\\n\", sizeof(ms_scan_args),"
+        " offsetof(ms_scan_args, y), offsetof(ms_scan_args, force_segments), sizeof(ms_update_args),"
+        " offsetof(ms_update_args, y), offsetof(ms_update_args, delta_bias)); return 0;}\n")
+    exe = tmp_path / "layout"
+    subprocess.check_call(["gcc", "-std=c11", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe)])
+    got = [int(v) for v in subprocess.check_output([str(exe)], text=True).split()]
+    want = [ctypes.sizeof(ms.ScanArgs), ms.ScanArgs.y.offset, ms.ScanArgs.force_segments.offset,
+            ctypes.sizeof(ms.UpdateArgs), ms.UpdateArgs.y.offset, ms.UpdateArgs.delta_bias.offset]
+    assert got == want
+
+
+def test_abi_version_and_status_strings(lib):
+    assert lib.mamba_abi_version() == 1
+    for code, name in ms.STATUS.items():
+        assert lib.mamba_status_string(code).decode() == name
+    assert lib.mamba_status_string(99).decode() == "MS_UNKNOWN_STATUS"
+
+
+def _valid_scan_args():
+    """Arguments that pass validation; pointers are fake (never dereferenced
+    here: every case below fails before any CUDA call)."""
+    a = ms.ScanArgs()
+    a.batch, a.dim, a.dstate, a.seqlen = 2, 8, 16, 64
+    a.in_dtype, a.delta_softplus = ms.MS_BF16, 1
+    base = 1 << 20
+    a.u, a.u_batch_stride, a.u_dim_stride = base, 8 * 64, 64
+    a.delta, a.delta_batch_stride, a.delta_dim_stride = base * 2, 8 * 64, 64
+    a.B, a.B_batch_stride, a.B_state_stride = base * 3, 16 * 64, 64
+    a.C, a.C_batch_stride, a.C_state_stride = base * 4, 16 * 64, 64
+    a.y, a.y_batch_stride, a.y_dim_stride = base * 5, 8 * 64, 64
+    a.A = base * 6
+    return a
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("batch", 0, 1), ("dim", -1, 1), ("dstate", 0, 1), ("seqlen", 0, 1),
+    ("in_dtype", 7, 1), ("reserved", 1, 1), ("force_segments", -2, 1),
+    ("u", None, 1), ("A", None, 1), ("y", None, 1),
+    ("u_dim_stride", -64, 1), ("dstate", 17, 2), ("batch", 70000, 2),
+    ("u", (1 << 20) + 1, 3), ("A", (1 << 20) * 6 + 2, 3),
+])
+def test_scan_validation_rejects(lib, field, value, status):
+    a = _valid_scan_args()
+    setattr(a, field, value)
+    n = ctypes.c_size_t(123)
+    rc = lib.mamba_scan_workspace_size(ctypes.byref(a), ctypes.byref(n))
+    assert rc == status, (rc, lib.mamba_last_error())
+    assert n.value == 0
+    rc = lib.mamba_scan_fwd(ctypes.byref(a), None, 0, None)
+    assert rc == status
+    assert lib.mamba_last_error().decode() != ""
+
+
+def test_scan_null_args(lib):
+    assert lib.mamba_scan_fwd(None, None, 0, None) == 1
+    n = ctypes.c_size_t(0)
+    assert lib.mamba_scan_workspace_size(None, ctypes.byref(n)) == 1
+    assert lib.mamba_scan_workspace_size(ctypes.byref(_valid_scan_args()), None) == 1
+
+
+def _valid_update_args():
+    a = ms.UpdateArgs()
+    a.batch, a.dim, a.dstate = 4, 8, 16
+    a.in_dtype, a.delta_softplus = ms.MS_BF16, 1
+    base = 1 << 20
+    a.state, a.state_batch_stride, a.state_dim_stride = base, 8 * 16, 16
+    a.x, a.x_batch_stride = base * 2, 8
+    a.delta, a.delta_batch_stride = base * 3, 8
+    a.B, a.B_batch_stride = base * 4, 16
+    a.C, a.C_batch_stride = base * 5, 16
+    a.y, a.y_batch_stride = base * 6, 8
+    a.A = base * 7
+    return a
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("batch", 0, 1), ("dstate", -3, 1), ("in_dtype", 2, 1), ("state", None, 1), ("x", None, 1),
+    ("C", None, 1), ("x_batch_stride", -1, 1), ("dstate", 32, 2), ("state", (1 << 20) + 2, 3),
+    ("x", (1 << 20) * 2 + 1, 3),
+])
+def test_update_validation_rejects(lib, field, value, status):
+    a = _valid_update_args()
+    setattr(a, field, value)
+    assert lib.mamba_state_update(ctypes.byref(a), None) == status
+    assert lib.mamba_state_update(None, None) == 1
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(ms, "_lib", None)
+    monkeypatch.setattr(ms, "_LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        ms.load_library()
