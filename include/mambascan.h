@@ -33,7 +33,8 @@
  * Conventions shared by every entry point:
  *  - All tensor pointers are DEVICE pointers, allocated and owned by the
  *    caller. The library allocates nothing and keeps no state between calls
- *    beyond a per-device cache of device properties.
+ *    beyond a per-device cache of device properties (and the fixed scratch
+ *    array of mamba_scan_fwd_noalloc, below).
  *  - Strides are in ELEMENTS of the tensor's own type. The innermost axis
  *    (L for the scan, dstate for states, dim for decode vectors) must be
  *    contiguous (stride 1).
@@ -179,6 +180,35 @@ ms_status mamba_scan_fwd(const ms_scan_args *args, void *workspace, size_t works
  * Errors: as mamba_scan_fwd, without MS_ERR_WORKSPACE.
  */
 ms_status mamba_state_update(const ms_update_args *args, void *stream);
+
+/* Size of the device array behind mamba_scan_fwd_noalloc (8 MiB per GPU). */
+#define MS_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/*
+ * mamba_scan_fwd_noalloc -- the same selective scan forward as mamba_scan_fwd
+ * for callers that cannot allocate device memory: a plugin inside a host
+ * application that owns every device allocation and passes in only its
+ * tensors, or a path on which cudaMalloc is off limits because it can stall
+ * the whole device. (The pages this library follows have no counterpart; this
+ * entry point exists for those callers.)
+ *
+ * The multi-block carry workspace that mamba_scan_fwd takes from its caller
+ * lives here in a fixed device array of MS_NOALLOC_SCRATCH_BYTES, which every
+ * GPU that loads the library holds until the process exits. The call
+ * allocates nothing. Inputs and outputs are the caller's, exactly as for
+ * mamba_scan_fwd.
+ *  - The first call on a device looks up the array's device address on that
+ *    (current) device; make that first call before any stream capture.
+ *  - All calls on a device share the array and it keeps the last call's
+ *    contents; every entry a call reads is written by that same call first,
+ *    so no clearing is needed, but calls whose kernels overlap on the GPU
+ *    (unordered streams) race on it and give wrong results.
+ *  - Calls that would need more carry scratch than the array holds (batch *
+ *    dim * segments * 128 bytes > MS_NOALLOC_SCRATCH_BYTES) are rejected with
+ *    MS_ERR_WORKSPACE and launch nothing.
+ * Errors: as mamba_scan_fwd.
+ */
+ms_status mamba_scan_fwd_noalloc(const ms_scan_args *args, void *stream);
 
 #ifdef __cplusplus
 }

@@ -115,6 +115,15 @@ ms::ScanParams to_params(const ms_scan_args *a) {
 
 }  // namespace
 
+namespace ms {
+void record_error(const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+}
+}  // namespace ms
+
 extern "C" {
 
 const char *mamba_status_string(int status) {

@@ -55,4 +55,7 @@ struct UpdateParams {
 
 cudaError_t launch_state_update(const UpdateParams &p, int in_dtype, cudaStream_t stream);
 
+// Record the message that mamba_last_error() returns on this thread.
+void record_error(const char *fmt, ...);
+
 }  // namespace ms
