@@ -181,6 +181,46 @@ ms_status mamba_scan_fwd(const ms_scan_args *args, void *workspace, size_t works
  */
 ms_status mamba_state_update(const ms_update_args *args, void *stream);
 
+/*
+ * Launch plan of a scan: which compiled kernel configuration runs it and how
+ * the work is cut. mamba_scan_plan_query returns the plan mamba_scan_fwd
+ * would use; mamba_scan_fwd_with_plan runs a caller-chosen plan (for tuning
+ * and for testing every configuration). Fields marked "out" are filled by the
+ * library and ignored on input.
+ */
+typedef struct ms_scan_plan {
+    int32_t config;          /* index of the kernel configuration, 0 .. mamba_scan_num_configs()-1 */
+    int32_t warps_per_cta;   /* 2 .. mamba_scan_config_info max_warps                             */
+    int32_t segments;        /* pieces the sequence of every row is cut into (>= 1)               */
+    int32_t lanes;           /* out: lanes per row pair (a group scans one chunk of lanes * 8 steps) */
+    int64_t segment_len;     /* out: time steps per segment                                      */
+    uint64_t workspace_bytes;/* out: workspace the plan needs (0 when segments == 1)              */
+} ms_scan_plan;
+
+/* Number of compiled scan kernel configurations. */
+int mamba_scan_num_configs(void);
+
+/*
+ * Properties of configuration `config`: lanes per row pair, state indices per
+ * pass (0 = the fully unrolled pipelined kernel, dstate 16 only; 1; 2) and the
+ * largest CTA in warps. Returns MS_ERR_INVALID_ARG for an unknown index.
+ */
+ms_status mamba_scan_config_info(int config, int *lanes, int *states_per_pass, int *max_warps);
+
+/* The plan mamba_scan_fwd would run for these arguments (validates like it). */
+ms_status mamba_scan_plan_query(const ms_scan_args *args, ms_scan_plan *plan);
+
+/*
+ * mamba_scan_fwd with the launch plan fixed by the caller. The plan is
+ * checked (index, CTA size, shared memory, segments <= number of chunks, and
+ * that the configuration can run these arguments: the pipelined kernels need
+ * dstate 16, and kernels with more than one state per pass need 16-byte
+ * aligned rows); an unusable plan returns MS_ERR_UNSUPPORTED and launches
+ * nothing. Same results as mamba_scan_fwd up to float32 rounding order.
+ */
+ms_status mamba_scan_fwd_with_plan(const ms_scan_args *args, const ms_scan_plan *plan, void *workspace,
+                                   size_t workspace_bytes, void *stream);
+
 /* Size of the device array behind mamba_scan_fwd_noalloc (8 MiB per GPU). */
 #define MS_NOALLOC_SCRATCH_BYTES (8u << 20)
 

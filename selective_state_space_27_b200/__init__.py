@@ -22,8 +22,9 @@ import ctypes
 import os
 
 __all__ = [
-    "scan_fwd", "state_update", "scan_workspace_size", "library_path", "load_library",
-    "MambaScanError", "ScanArgs", "UpdateArgs", "MS_F32", "MS_BF16", "MAX_DSTATE",
+    "scan_fwd", "state_update", "scan_workspace_size", "scan_plan", "scan_configs", "library_path",
+    "load_library", "MambaScanError", "ScanArgs", "UpdateArgs", "ScanPlan", "MS_F32", "MS_BF16",
+    "MAX_DSTATE",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -72,6 +73,14 @@ class UpdateArgs(ctypes.Structure):
     ]
 
 
+class ScanPlan(ctypes.Structure):
+    """Mirror of ``ms_scan_plan``."""
+    _fields_ = [
+        ("config", _i32), ("warps_per_cta", _i32), ("segments", _i32), ("lanes", _i32),
+        ("segment_len", _i64), ("workspace_bytes", ctypes.c_uint64),
+    ]
+
+
 class MambaScanError(RuntimeError):
     def __init__(self, status: int, message: str):
         super().__init__(f"{STATUS.get(status, status)}: {message}")
@@ -102,6 +111,16 @@ def load_library():
         lib.mamba_scan_fwd.argtypes = [ctypes.POINTER(ScanArgs), _vp, ctypes.c_size_t, _vp]
         lib.mamba_state_update.restype = ctypes.c_int
         lib.mamba_state_update.argtypes = [ctypes.POINTER(UpdateArgs), _vp]
+        lib.mamba_scan_num_configs.restype = ctypes.c_int
+        lib.mamba_scan_num_configs.argtypes = []
+        lib.mamba_scan_config_info.restype = ctypes.c_int
+        lib.mamba_scan_config_info.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int),
+                                               ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
+        lib.mamba_scan_plan_query.restype = ctypes.c_int
+        lib.mamba_scan_plan_query.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(ScanPlan)]
+        lib.mamba_scan_fwd_with_plan.restype = ctypes.c_int
+        lib.mamba_scan_fwd_with_plan.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(ScanPlan), _vp,
+                                                 ctypes.c_size_t, _vp]
         if lib.mamba_abi_version() != 1:
             raise RuntimeError("libmambascan.so ABI version mismatch")
         _lib = lib
@@ -207,9 +226,27 @@ def scan_workspace_size(args: ScanArgs) -> int:
     return int(n.value)
 
 
+def scan_configs():
+    """[(index, lanes, states_per_pass, max_warps)] of the compiled scan kernels."""
+    lib = load_library()
+    out = []
+    for i in range(lib.mamba_scan_num_configs()):
+        a, b, c = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+        _check(lib.mamba_scan_config_info(i, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)))
+        out.append((i, a.value, b.value, c.value))
+    return out
+
+
+def scan_plan(args: ScanArgs) -> ScanPlan:
+    """The launch plan mamba_scan_fwd would use for these arguments."""
+    plan = ScanPlan()
+    _check(load_library().mamba_scan_plan_query(ctypes.byref(args), ctypes.byref(plan)))
+    return plan
+
+
 def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
              initial_state=None, return_last_state=True, out=None, force_segments=0,
-             workspace=None, stream=None):
+             workspace=None, stream=None, plan=None):
     """Selective scan forward on the current (or given) CUDA stream.
 
     u, delta, z: (batch, dim, L); B, C: (batch, dstate, L) -- all float32 or
@@ -229,13 +266,21 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=
                            final_state=hT, force_segments=force_segments)
     lib = load_library()
     with torch.cuda.device(u.device):
-        need = scan_workspace_size(args)
+        if plan is None:
+            need = scan_workspace_size(args)
+        else:
+            # the workspace a fixed plan needs: rows * segments * 16 states * 2 floats
+            need = 0 if plan.segments <= 1 else 2 * u.shape[0] * u.shape[1] * plan.segments * 16 * 4
         ws_ptr, ws_bytes = None, 0
         if need:
             if workspace is None or workspace.numel() < need:
                 workspace = torch.empty(need, dtype=torch.uint8, device=u.device)
             ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
-        _check(lib.mamba_scan_fwd(ctypes.byref(args), ws_ptr, ws_bytes, _stream_ptr(stream)))
+        if plan is None:
+            _check(lib.mamba_scan_fwd(ctypes.byref(args), ws_ptr, ws_bytes, _stream_ptr(stream)))
+        else:
+            _check(lib.mamba_scan_fwd_with_plan(ctypes.byref(args), ctypes.byref(plan), ws_ptr, ws_bytes,
+                                                _stream_ptr(stream)))
     return (y, hT) if return_last_state else y
 
 

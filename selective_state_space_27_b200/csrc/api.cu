@@ -113,6 +113,29 @@ ms::ScanParams to_params(const ms_scan_args *a) {
     return p;
 }
 
+ms_status run_plan(ms::ScanParams p, const ms::ScanPlan &plan, int in_dtype, void *workspace,
+                   size_t workspace_bytes, void *stream) {
+    if (plan.ws_bytes > 0) {
+        if (!workspace || workspace_bytes < plan.ws_bytes) {
+            set_error("workspace of %zu bytes needed, %zu given", plan.ws_bytes,
+                      workspace ? workspace_bytes : static_cast<size_t>(0));
+            return MS_ERR_WORKSPACE;
+        }
+        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) {
+            set_error("workspace must be 256-byte aligned");
+            return MS_ERR_ALIGNMENT;
+        }
+        float *ws = static_cast<float *>(workspace);
+        p.ws_P = ws;
+        p.ws_H = ws + plan.ws_bytes / 2 / sizeof(float);
+    }
+    p.nseg = plan.nseg;
+    p.seg_len = plan.seg_len;
+    const cudaError_t e = ms::launch_scan(p, plan, in_dtype, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "scan kernel launch");
+    return MS_OK;
+}
+
 }  // namespace
 
 namespace ms {
@@ -163,28 +186,48 @@ ms_status mamba_scan_fwd(const ms_scan_args *args, void *workspace, size_t works
     int sms = 0;
     st = device_sms(&sms);
     if (st != MS_OK) return st;
-    ms::ScanParams p = to_params(args);
+    const ms::ScanParams p = to_params(args);
     const ms::ScanPlan plan = ms::plan_scan(p, args->in_dtype, args->force_segments, sms);
-    if (plan.ws_bytes > 0) {
-        if (!workspace || workspace_bytes < plan.ws_bytes) {
-            set_error("workspace of %zu bytes needed, %zu given", plan.ws_bytes,
-                      workspace ? workspace_bytes : static_cast<size_t>(0));
-            return MS_ERR_WORKSPACE;
-        }
-        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) {
-            set_error("workspace must be 256-byte aligned");
-            return MS_ERR_ALIGNMENT;
-        }
-        float *ws = static_cast<float *>(workspace);
-        const size_t half = plan.ws_bytes / 2 / sizeof(float);
-        p.ws_P = ws;
-        p.ws_H = ws + half;
-    }
-    p.nseg = plan.nseg;
-    p.seg_len = plan.seg_len;
-    const cudaError_t e = ms::launch_scan(p, plan, args->in_dtype, static_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess) return cuda_fail(e, "scan kernel launch");
+    return run_plan(p, plan, args->in_dtype, workspace, workspace_bytes, stream);
+}
+
+int mamba_scan_num_configs(void) { return ms::scan_num_configs(); }
+
+ms_status mamba_scan_config_info(int config, int *lanes, int *states_per_pass, int *max_warps) {
+    if (!ms::scan_config_info(config, lanes, states_per_pass, max_warps)) return invalid("unknown config");
     return MS_OK;
+}
+
+ms_status mamba_scan_plan_query(const ms_scan_args *args, ms_scan_plan *plan) {
+    if (!plan) return invalid("plan is NULL");
+    ms_status st = check_scan(args);
+    if (st != MS_OK) return st;
+    int sms = 0;
+    st = device_sms(&sms);
+    if (st != MS_OK) return st;
+    const ms::ScanPlan pl = ms::plan_scan(to_params(args), args->in_dtype, args->force_segments, sms);
+    plan->config = pl.config;
+    plan->warps_per_cta = pl.warps;
+    plan->segments = pl.nseg;
+    plan->lanes = pl.lg;
+    plan->segment_len = pl.seg_len;
+    plan->workspace_bytes = pl.ws_bytes;
+    return MS_OK;
+}
+
+ms_status mamba_scan_fwd_with_plan(const ms_scan_args *args, const ms_scan_plan *plan, void *workspace,
+                                   size_t workspace_bytes, void *stream) {
+    if (!plan) return invalid("plan is NULL");
+    ms_status st = check_scan(args);
+    if (st != MS_OK) return st;
+    const ms::ScanParams p = to_params(args);
+    ms::ScanPlan pl{};
+    if (!ms::make_plan(p, args->in_dtype, plan->config, plan->warps_per_cta, plan->segments, &pl)) {
+        set_error("plan (config %d, %d warps, %d segments) cannot run these arguments", plan->config,
+                  plan->warps_per_cta, plan->segments);
+        return MS_ERR_UNSUPPORTED;
+    }
+    return run_plan(p, pl, args->in_dtype, workspace, workspace_bytes, stream);
 }
 
 ms_status mamba_state_update(const ms_update_args *a, void *stream) {

@@ -26,10 +26,11 @@ struct ScanParams {
 
 // Launch configuration chosen on the host for one scan call.
 struct ScanPlan {
-    int lg;             // lanes that share one row's chunk (4 or 8)
+    int lg;             // lanes that share one row pair's chunk (4, 8 or 16)
+    int config;         // index of the compiled kernel configuration
     int warps;          // warps per CTA
     int rows_per_cta;   // warps * (32 / lg)
-    int chunk;          // time steps per chunk = lg * 16
+    int chunk;          // time steps per chunk = lg * 8
     int vec;            // 1 if every row start is 16-byte aligned (vector path)
     int nseg;
     int64_t seg_len;
@@ -37,6 +38,11 @@ struct ScanPlan {
 };
 
 ScanPlan plan_scan(const ScanParams &p, int in_dtype, int force_segments, int num_sms);
+// A plan with a fixed configuration, CTA size and segment count; returns false
+// (and leaves `out` unspecified) when the configuration cannot run `p`.
+bool make_plan(const ScanParams &p, int in_dtype, int config, int warps, int segments, ScanPlan *out);
+int scan_num_configs();
+bool scan_config_info(int config, int *lanes, int *states_per_pass, int *max_warps);
 cudaError_t launch_scan(const ScanParams &p, const ScanPlan &plan, int in_dtype,
                         cudaStream_t stream);
 

@@ -173,3 +173,57 @@ def test_long_context_forced_segments_sampled_rows():
     w = SCAN_WORKLOADS["long_context_131k"]
     inp = make_scan_inputs(w)
     check(inp, rows=sample_rows(w.batch, w.dim, 12, seed=3), force_segments=8)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_every_kernel_configuration(dtype):
+    """Each compiled configuration, forced through mamba_scan_fwd_with_plan, at
+    its smallest and largest CTA and with and without segments."""
+    import torch
+    ms = _ms()
+    # rows 16-byte aligned (every configuration can run) and a ragged last chunk
+    inp = make_scan_inputs(LAYER, batch=2, dim=88, seqlen=1000, dtype=dtype, seed=1100)
+    dev = device_inputs(inp)
+    yr, hr = oracle_scan(inp)
+    for cfg, lanes, states, max_warps in ms.scan_configs():
+        # the largest CTA whose shared memory fits (float32 tiles are twice as large)
+        largest = None
+        for warps in range(max_warps, 1, -1):
+            try:
+                ms.scan_fwd(**dev, plan=ms.ScanPlan(config=cfg, warps_per_cta=warps, segments=1))
+                largest = warps
+                break
+            except ms.MambaScanError as e:
+                assert e.status == 2
+        assert largest is not None, f"config {cfg} runs at no CTA size"
+        for warps in sorted({2, largest}):
+            for segments in (1, 3):
+                plan = ms.ScanPlan(config=cfg, warps_per_cta=warps, segments=segments)
+                y, hT = ms.scan_fwd(**dev, plan=plan)
+                torch.cuda.synchronize()
+                tag = f"config {cfg} (lanes {lanes}, states/pass {states}), {warps} warps, {segments} segments"
+                assert rel_err(to_host64(y), yr) <= TOL[dtype], tag
+                assert rel_err(to_host64(hT), hr) <= TOL[dtype], tag
+
+
+def test_plan_validation():
+    """Unusable plans are refused before any launch."""
+    import torch
+    ms = _ms()
+    inp = make_scan_inputs(LAYER, batch=1, dim=8, dstate=4, seqlen=128, seed=1200)
+    dev = device_inputs(inp)
+    configs = ms.scan_configs()
+    pipelined = [c for c, _, states, _ in configs if states == 0]
+    for plan in [ms.ScanPlan(config=len(configs), warps_per_cta=4, segments=1),
+                 ms.ScanPlan(config=0, warps_per_cta=1, segments=1),
+                 ms.ScanPlan(config=0, warps_per_cta=4, segments=0),
+                 ms.ScanPlan(config=pipelined[0], warps_per_cta=4, segments=1)]:   # needs dstate 16
+        with pytest.raises(ms.MambaScanError) as ei:
+            ms.scan_fwd(**dev, plan=plan)
+        assert ei.value.status == 2
+    torch.cuda.synchronize()
+    # the automatic plan is one of the compiled configurations
+    y = torch.empty_like(dev["u"])
+    args = ms.build_scan_args(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], y)
+    plan = ms.scan_plan(args)
+    assert 0 <= plan.config < len(configs) and plan.segments >= 1 and plan.warps_per_cta >= 2
