@@ -30,7 +30,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from selective_state_space_27_b200.inputs import SCAN_WORKLOADS, make_scan_inputs  # noqa: E402
+from selective_state_space_27_b200.inputs import (DECODE_WORKLOADS, SCAN_WORKLOADS,  # noqa: E402
+                                                  make_decode_state, make_decode_step, make_scan_inputs)
 
 METRIC = "selective-scan B·D·L·N elems/s at 1 B200; % of HBM/MUFU roofline"
 UNIT = "elem/s"
@@ -55,6 +56,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU-baseline budget (seconds of oracle work on rank 0)")
+    ap.add_argument("--decode-steps", type=int, default=1000,
+                    help="decode state-update steps timed on the (256, 5120, 16) decode workload (0: skip)")
     return ap.parse_args(argv)
 
 
@@ -409,6 +412,8 @@ def run_ours(args, dist: Dist):
         "roofline_elem_per_s": counts["elements"] / max(t_bounds.values()),
     }
 
+    decode = run_decode(args, dist, dev) if args.decode_steps > 0 else None
+
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         rate, threads, sample, secs = cpu_rate(w, inp, args.cpu_seconds)
@@ -420,7 +425,7 @@ def run_ours(args, dist: Dist):
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded)", "config": workload_config(w, {"global_batch": w.batch * dist.world}),
-        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode,
         "gpu_launches": args.steps * launches_per_step, "clocks": clocks,
     }
     if dist.rank == 0:
@@ -428,6 +433,82 @@ def run_ours(args, dist: Dist):
     dist.barrier()
     dist.close()
     return 0
+
+
+def run_decode(args, dist: Dist, dev):
+    """Time the single-token state update on the decode workload (batch 256,
+    d_inner 5120, N 16, fp32 state, bf16 tokens): ``--decode-steps`` sequential
+    steps cycling over 8 pre-uploaded seeded token sets, launched through the C
+    ABI. Two timings: steps back to back (the 84 MB state stays in the 126 MB
+    L2, as for one layer decoding alone), and steps with a 256 MB L2 flush
+    between them (the flush is outside the per-step events), which is what a
+    multi-layer model sees."""
+    import ctypes
+
+    import torch
+    import selective_state_space_27_b200 as ms
+
+    w = DECODE_WORKLOADS["decode_b256_d5120"]
+    st0 = make_decode_state(w, seed=w.seed + 1000 * dist.rank)
+    state = torch.from_numpy(st0["h0"]).to(dev)
+    prm = {k: torch.from_numpy(st0[k]).to(dev) for k in ("A", "D", "delta_bias")}
+    toks = []
+    for s in range(8):
+        t = make_decode_step(w, s, seed=w.seed + 1000 * dist.rank)
+        toks.append({k: torch.from_numpy(v).view(torch.bfloat16).to(dev) for k, v in t.items()})
+    y = torch.empty((w.batch, w.dim), dtype=torch.bfloat16, device=dev)
+    argl = [ms.build_update_args(state, t["x"], t["delta"], prm["A"], t["B"], t["C"], y, D=prm["D"], z=t["z"],
+                                 delta_bias=prm["delta_bias"]) for t in toks]
+    lib = ms.load_library()
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        rc = lib.mamba_state_update(ctypes.byref(argl[i % 8]), stream.cuda_stream)
+        if rc != 0:
+            raise ms.MambaScanError(rc, lib.mamba_last_error().decode())
+
+    for i in range(20):
+        step(i)
+    torch.cuda.synchronize()
+    n = args.decode_steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(n):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    hot_us = e0.elapsed_time(e1) * 1e3 / n
+    # flushed: a 256 MB write between steps evicts the state from L2
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    nf = min(n, 200)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nf)]
+    for i in range(nf):
+        flush.zero_()
+        evs[i][0].record(stream)
+        step(i)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    cold_us = sum(a.elapsed_time(b) for a, b in evs) * 1e3 / nf
+    hot_us = dist.max(hot_us, dev)
+    cold_us = dist.max(cold_us, dev)
+    rows = w.batch * w.dim
+    bytes_step = 2 * rows * w.dstate * 4 + 4 * rows * 2 + 2 * w.batch * w.dstate * 2 + w.dim * (w.dstate + 2) * 4
+    peaks = load_peaks()
+    elems = rows * w.dstate
+    return {
+        "workload": w.name, "batch": w.batch, "d_inner": w.dim, "d_state": w.dstate, "steps": n,
+        "metric": "decode state-update B*D*N elems/s", "unit": UNIT,
+        "value": dist.world * elems / (hot_us * 1e-6), "us_per_step": hot_us,
+        "value_l2_flushed": dist.world * elems / (cold_us * 1e-6), "us_per_step_l2_flushed": cold_us,
+        "tokens": "8 seeded token sets cycled",
+        "roofline": {"bound": "hbm", "unit": "GB/s", "algorithmic_bytes_per_step": bytes_step,
+                     "achieved_l2_flushed": bytes_step / (cold_us * 1e-6) / 1e9,
+                     "achieved_back_to_back": bytes_step / (hot_us * 1e-6) / 1e9,
+                     "peak": peaks["hbm_gbs"], "frac": bytes_step / (cold_us * 1e-6) / 1e9 / peaks["hbm_gbs"],
+                     "peak_source": peaks["source"],
+                     "note": "frac uses the L2-flushed timing; back-to-back steps keep the 84 MB state in L2"},
+        "gpu_launches": n + nf,
+    }
 
 
 def main(argv=None):

@@ -246,8 +246,8 @@ ms_status mamba_state_update(const ms_update_args *a, void *stream) {
                   MS_MAX_DSTATE);
         return MS_ERR_UNSUPPORTED;
     }
-    if (a->batch * a->dim * 4 > (static_cast<int64_t>(1) << 40)) {
-        set_error("batch * dim too large");
+    if (a->batch > 65535) {
+        set_error("batch %lld exceeds 65535", static_cast<long long>(a->batch));
         return MS_ERR_UNSUPPORTED;
     }
     const int eb = a->in_dtype == MS_F32 ? 4 : 2;

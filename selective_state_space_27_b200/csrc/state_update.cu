@@ -7,11 +7,16 @@
 //     h[n]  = exp(delta A[d,n]) h[n] + delta B[n] x        (in place)
 //     y     = (sum_n C[n] h[n] + D[d] x) * silu(z)
 //
-// Decode reads and writes the whole float32 state once per token, so the step
-// is bound by memory bandwidth. Four consecutive threads own one row (b, d);
-// thread q owns state entries [4q, 4q+4), which makes every state access a
-// fully coalesced 16-byte load and store. The partial readouts are summed with
-// two butterfly shuffles.
+// Decode reads and writes the whole float32 state once per token: the step is
+// bound by HBM bandwidth (~168 MB of state traffic per step for 256 x 5120 x
+// 16), so the kernel is built to keep many bytes in flight with few
+// instructions per byte. The grid is (dim blocks, batch): no index division.
+// Four consecutive threads share a row (b, d); thread q owns state entries
+// [4q, 4q+4), so every state access is a fully coalesced 16-byte load and
+// store and its A, B and C entries arrive as one vector load each. (A thread
+// may own several rows, kRowGroups apart, loading all of them before
+// computing; one row per thread at full occupancy measured faster.) The
+// partial readouts are summed with two butterfly shuffles.
 #include <type_traits>
 
 #include "device_math.cuh"
@@ -20,78 +25,120 @@
 namespace ms {
 namespace {
 
-constexpr int kThreadsPerRow = 4;
-constexpr int kBlock = 256;
+constexpr int kRowGroups = 64;                // row groups per block (4 threads each)
+constexpr int kBlock = kRowGroups * 4;
 
 template <typename T>
-__device__ __forceinline__ float ld(const void *base, int64_t i) {
-    return to_f32<T>(static_cast<const T *>(base)[i]);
+__device__ __forceinline__ float ldg1(const void *base, int64_t i) {
+    return to_f32<T>(__ldg(static_cast<const T *>(base) + i));
 }
 
-template <typename T, bool VEC16>
+// Four consecutive elements starting at `p` (aligned to 4 elements).
+template <typename T>
+__device__ __forceinline__ float4 ldg4(const T *p) {
+    if constexpr (std::is_same<T, float>::value) {
+        return __ldg(reinterpret_cast<const float4 *>(p));
+    } else {
+        const uint2 w = __ldg(reinterpret_cast<const uint2 *>(p));
+        return make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
+    }
+}
+
+// VEC: dstate == 16 with state rows, A rows and B/C rows aligned for vector
+// access. A thread owns state entries [4q, 4q+4) of kRowsPerThread rows and
+// issues all of their loads before any arithmetic, so that enough bytes are in
+// flight to cover HBM latency.
+template <typename T, bool VEC, int kRowsPerThread>
 __global__ void __launch_bounds__(kBlock) state_update_kernel(const UpdateParams p) {
-    const int64_t gt = static_cast<int64_t>(blockIdx.x) * kBlock + threadIdx.x;
-    const int64_t row = gt / kThreadsPerRow;
-    const int q = static_cast<int>(gt % kThreadsPerRow);
-    const int64_t rows = p.batch * p.dim;
-    const bool ok = row < rows;
-    const int64_t r = ok ? row : rows - 1;
-    const int64_t b = r / p.dim, d = r % p.dim;
+    constexpr int kRowsPerBlock = kRowGroups * kRowsPerThread;
+    const int tid = threadIdx.x;
+    const int q = tid & 3;
+    const int64_t b = blockIdx.y;
+    const int64_t d0 = static_cast<int64_t>(blockIdx.x) * kRowsPerBlock + (tid >> 2);
     const int dstate = static_cast<int>(p.dstate);
 
-    const float x = ld<T>(p.x, b * p.x_sb + d);
-    float dt = ld<T>(p.delta, b * p.dl_sb + d);
-    if (p.delta_bias) dt += p.delta_bias[d];
-    if (p.softplus) dt = softplus(dt);
-    const float dtx = dt * x;
-
-    float *st = p.state + b * p.s_sb + d * p.s_sd;
-    const float *Arow = p.A + d * dstate;
-    float acc = 0.f;
-    if constexpr (VEC16) {
-        // dstate == 16, state rows 16-byte aligned
-        const int n0 = 4 * q;
-        float4 h = ok ? reinterpret_cast<const float4 *>(st)[q] : make_float4(0.f, 0.f, 0.f, 0.f);
-        const float4 a4 = reinterpret_cast<const float4 *>(Arow)[q];
-        float hv[4] = {h.x, h.y, h.z, h.w};
-        const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+    int64_t dd[kRowsPerThread];
+    bool ok[kRowsPerThread];
+    float x[kRowsPerThread], dt[kRowsPerThread];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float a = ex2_approx(dt * (av[e] * kLog2e));
-            const float Bn = ld<T>(p.B, b * p.B_sb + n0 + e);
-            hv[e] = fmaf(a, hv[e], dtx * Bn);
-            acc = fmaf(ld<T>(p.C, b * p.C_sb + n0 + e), hv[e], acc);
-        }
-        if (ok) reinterpret_cast<float4 *>(st)[q] = make_float4(hv[0], hv[1], hv[2], hv[3]);
-    } else {
-        for (int n = q; n < dstate; n += kThreadsPerRow) {
-            const float a = ex2_approx(dt * (Arow[n] * kLog2e));
-            float h = ok ? st[n] : 0.f;
-            h = fmaf(a, h, dtx * ld<T>(p.B, b * p.B_sb + n));
-            acc = fmaf(ld<T>(p.C, b * p.C_sb + n), h, acc);
-            if (ok) st[n] = h;
-        }
+    for (int k = 0; k < kRowsPerThread; ++k) {
+        const int64_t d = d0 + k * kRowGroups;
+        ok[k] = d < p.dim;
+        dd[k] = ok[k] ? d : p.dim - 1;
+        x[k] = ldg1<T>(p.x, b * p.x_sb + dd[k]);
+        dt[k] = ldg1<T>(p.delta, b * p.dl_sb + dd[k]);
     }
-    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-    if (ok && q == 0) {
-        float yv = acc + (p.D ? p.D[d] * x : 0.f);
-        if (p.z) yv *= silu(ld<T>(p.z, b * p.z_sb + d));
-        static_cast<T *>(p.y)[b * p.y_sb + d] = from_f32<T>(yv);
+    if constexpr (VEC) {
+        float4 h[kRowsPerThread], a[kRowsPerThread];
+#pragma unroll
+        for (int k = 0; k < kRowsPerThread; ++k) {
+            h[k] = reinterpret_cast<const float4 *>(p.state + b * p.s_sb + dd[k] * p.s_sd)[q];
+            a[k] = __ldg(reinterpret_cast<const float4 *>(p.A + dd[k] * 16) + q);
+        }
+        const float4 Bv = ldg4<T>(static_cast<const T *>(p.B) + b * p.B_sb + 4 * q);
+        const float4 Cv = ldg4<T>(static_cast<const T *>(p.C) + b * p.C_sb + 4 * q);
+#pragma unroll
+        for (int k = 0; k < kRowsPerThread; ++k) {
+            float v = dt[k];
+            if (p.delta_bias) v += __ldg(p.delta_bias + dd[k]);
+            if (p.softplus) v = softplus(v);
+            const float dtx = v * x[k];
+            float4 o;
+            o.x = fmaf(ex2_approx(v * (a[k].x * kLog2e)), h[k].x, dtx * Bv.x);
+            o.y = fmaf(ex2_approx(v * (a[k].y * kLog2e)), h[k].y, dtx * Bv.y);
+            o.z = fmaf(ex2_approx(v * (a[k].z * kLog2e)), h[k].z, dtx * Bv.z);
+            o.w = fmaf(ex2_approx(v * (a[k].w * kLog2e)), h[k].w, dtx * Bv.w);
+            float acc = fmaf(Cv.x, o.x, fmaf(Cv.y, o.y, fmaf(Cv.z, o.z, Cv.w * o.w)));
+            if (ok[k]) reinterpret_cast<float4 *>(p.state + b * p.s_sb + dd[k] * p.s_sd)[q] = o;
+            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+            if (ok[k] && q == 0) {
+                float yv = acc + (p.D ? __ldg(p.D + dd[k]) * x[k] : 0.f);
+                if (p.z) yv *= silu(ldg1<T>(p.z, b * p.z_sb + dd[k]));
+                static_cast<T *>(p.y)[b * p.y_sb + dd[k]] = from_f32<T>(yv);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < kRowsPerThread; ++k) {
+            float v = dt[k];
+            if (p.delta_bias) v += __ldg(p.delta_bias + dd[k]);
+            if (p.softplus) v = softplus(v);
+            const float dtx = v * x[k];
+            float *st = p.state + b * p.s_sb + dd[k] * p.s_sd;
+            float acc = 0.f;
+            for (int n = q; n < dstate; n += 4) {
+                const float an = ex2_approx(v * (__ldg(p.A + dd[k] * dstate + n) * kLog2e));
+                float hn = st[n];
+                hn = fmaf(an, hn, dtx * ldg1<T>(p.B, b * p.B_sb + n));
+                acc = fmaf(ldg1<T>(p.C, b * p.C_sb + n), hn, acc);
+                if (ok[k]) st[n] = hn;
+            }
+            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+            if (ok[k] && q == 0) {
+                float yv = acc + (p.D ? __ldg(p.D + dd[k]) * x[k] : 0.f);
+                if (p.z) yv *= silu(ldg1<T>(p.z, b * p.z_sb + dd[k]));
+                static_cast<T *>(p.y)[b * p.y_sb + dd[k]] = from_f32<T>(yv);
+            }
+        }
     }
 }
 
 template <typename T>
 cudaError_t launch_t(const UpdateParams &p, cudaStream_t stream) {
-    const int64_t threads = p.batch * p.dim * kThreadsPerRow;
-    const int64_t blocks = (threads + kBlock - 1) / kBlock;
-    const bool vec16 = p.dstate == 16 && (reinterpret_cast<uintptr_t>(p.state) & 15u) == 0 &&
-                       (p.s_sb % 4) == 0 && (p.s_sd % 4) == 0 &&
-                       (reinterpret_cast<uintptr_t>(p.A) & 15u) == 0;
-    if (vec16)
-        state_update_kernel<T, true><<<static_cast<unsigned>(blocks), kBlock, 0, stream>>>(p);
+    const int eb = sizeof(T);
+    auto al = [](const void *ptr, int bytes) { return (reinterpret_cast<uintptr_t>(ptr) % bytes) == 0; };
+    const bool vec = p.dstate == 16 && al(p.state, 16) && (p.s_sb % 4) == 0 && (p.s_sd % 4) == 0 &&
+                     al(p.A, 16) && al(p.B, 4 * eb) && al(p.C, 4 * eb) && (p.B_sb % 4) == 0 &&
+                     (p.C_sb % 4) == 0;
+    constexpr int kRows = 1;   // rows per thread (occupancy beats per-thread batching here)
+    const dim3 grid(static_cast<unsigned>((p.dim + kRowGroups * kRows - 1) / (kRowGroups * kRows)),
+                    static_cast<unsigned>(p.batch));
+    if (vec)
+        state_update_kernel<T, true, kRows><<<grid, kBlock, 0, stream>>>(p);
     else
-        state_update_kernel<T, false><<<static_cast<unsigned>(blocks), kBlock, 0, stream>>>(p);
+        state_update_kernel<T, false, kRows><<<grid, kBlock, 0, stream>>>(p);
     return cudaGetLastError();
 }
 

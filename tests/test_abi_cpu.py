@@ -127,7 +127,8 @@ def _valid_update_args():
 
 @pytest.mark.parametrize("field,value,status", [
     ("batch", 0, 1), ("dstate", -3, 1), ("in_dtype", 2, 1), ("state", None, 1), ("x", None, 1),
-    ("C", None, 1), ("x_batch_stride", -1, 1), ("dstate", 32, 2), ("state", (1 << 20) + 2, 3),
+    ("C", None, 1), ("x_batch_stride", -1, 1), ("dstate", 32, 2), ("batch", 70000, 2),
+    ("state", (1 << 20) + 2, 3),
     ("x", (1 << 20) * 2 + 1, 3),
 ])
 def test_update_validation_rejects(lib, field, value, status):
