@@ -190,9 +190,9 @@ ms_status mamba_state_update(const ms_update_args *args, void *stream);
  */
 typedef struct ms_scan_plan {
     int32_t config;          /* index of the kernel configuration, 0 .. mamba_scan_num_configs()-1 */
-    int32_t warps_per_cta;   /* 2 .. mamba_scan_config_info max_warps                             */
+    int32_t warps_per_cta;   /* chunked: 2 .. max_warps; sequential: exactly max_warps (4)         */
     int32_t segments;        /* pieces the sequence of every row is cut into (>= 1)               */
-    int32_t lanes;           /* out: lanes per row pair (a group scans one chunk of lanes * 8 steps) */
+    int32_t lanes;           /* out: chunked: lanes per row pair; sequential: lanes per row        */
     int64_t segment_len;     /* out: time steps per segment                                      */
     uint64_t workspace_bytes;/* out: workspace the plan needs (0 when segments == 1)              */
 } ms_scan_plan;
@@ -201,11 +201,25 @@ typedef struct ms_scan_plan {
 int mamba_scan_num_configs(void);
 
 /*
- * Properties of configuration `config`: lanes per row pair, state indices per
- * pass (0 = the fully unrolled pipelined kernel, dstate 16 only; 1; 2) and the
- * largest CTA in warps. Returns MS_ERR_INVALID_ARG for an unknown index.
+ * Properties of configuration `config`.
+ *  - Chunked kernels (kind 0): lanes per row pair, state indices per pass
+ *    (0 = the fully unrolled pipelined kernel, dstate 16 only; 1; 2) and the
+ *    largest CTA in warps (plans take 2 .. max_warps warps and any number of
+ *    segments).
+ *  - Sequential kernels (kind 1): lanes per row, states per lane (16 / lanes)
+ *    and the fixed CTA size in warps (4); plans take exactly that many warps
+ *    and one segment, and need no workspace.
+ * Returns MS_ERR_INVALID_ARG for an unknown index.
  */
 ms_status mamba_scan_config_info(int config, int *lanes, int *states_per_pass, int *max_warps);
+
+/*
+ * Kind of configuration `config` (written to *kind): 0 = chunked kernel (each
+ * row's time axis is split across lanes and joined by a scan), 1 = sequential
+ * kernel (each lane runs the recurrence step by step for some of a row's
+ * states). Returns MS_ERR_INVALID_ARG for an unknown index or NULL kind.
+ */
+ms_status mamba_scan_config_kind(int config, int *kind);
 
 /* The plan mamba_scan_fwd would run for these arguments (validates like it). */
 ms_status mamba_scan_plan_query(const ms_scan_args *args, ms_scan_plan *plan);

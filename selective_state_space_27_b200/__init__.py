@@ -116,6 +116,8 @@ def load_library():
         lib.mamba_scan_config_info.restype = ctypes.c_int
         lib.mamba_scan_config_info.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int),
                                                ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
+        lib.mamba_scan_config_kind.restype = ctypes.c_int
+        lib.mamba_scan_config_kind.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
         lib.mamba_scan_plan_query.restype = ctypes.c_int
         lib.mamba_scan_plan_query.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(ScanPlan)]
         lib.mamba_scan_fwd_with_plan.restype = ctypes.c_int
@@ -227,13 +229,16 @@ def scan_workspace_size(args: ScanArgs) -> int:
 
 
 def scan_configs():
-    """[(index, lanes, states_per_pass, max_warps)] of the compiled scan kernels."""
+    """[(index, lanes, states_per_pass, max_warps, kind)] of the compiled scan
+    kernels; kind 0 = chunked (lanes per row pair), 1 = sequential (lanes per
+    row, fixed CTA of max_warps warps, one segment)."""
     lib = load_library()
     out = []
     for i in range(lib.mamba_scan_num_configs()):
-        a, b, c = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+        a, b, c, k = ctypes.c_int(), ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
         _check(lib.mamba_scan_config_info(i, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)))
-        out.append((i, a.value, b.value, c.value))
+        _check(lib.mamba_scan_config_kind(i, ctypes.byref(k)))
+        out.append((i, a.value, b.value, c.value, k.value))
     return out
 
 

@@ -198,6 +198,13 @@ ms_status mamba_scan_config_info(int config, int *lanes, int *states_per_pass, i
     return MS_OK;
 }
 
+ms_status mamba_scan_config_kind(int config, int *kind) {
+    if (!kind) return invalid("kind is NULL");
+    *kind = ms::scan_config_kind(config);
+    if (*kind < 0) return invalid("unknown config");
+    return MS_OK;
+}
+
 ms_status mamba_scan_plan_query(const ms_scan_args *args, ms_scan_plan *plan) {
     if (!plan) return invalid("plan is NULL");
     ms_status st = check_scan(args);

@@ -45,6 +45,37 @@ __device__ __forceinline__ float silu(float z) {
     return __fdividef(z, 1.f + __expf(-z));
 }
 
+// Packed float32 pairs: one f32x2 instruction serves two independent lanes of
+// work (two rows, two states or two time steps).
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 ex2x2(float2 v) { return f2(ex2_approx(v.x), ex2_approx(v.y)); }
+
+__device__ __forceinline__ float2 log1p_unit2(float2 e) {
+    float2 p = f2(0.014539077877998352f, 0.014539077877998352f);
+    p = fma2(p, e, f2(-0.06759698688983917f, -0.06759698688983917f));
+    p = fma2(p, e, f2(0.15056990087032318f, 0.15056990087032318f));
+    p = fma2(p, e, f2(-0.23573748767375946f, -0.23573748767375946f));
+    p = fma2(p, e, f2(0.3312585949897766f, 0.3312585949897766f));
+    p = fma2(p, e, f2(-0.499883770942688f, -0.499883770942688f));
+    p = fma2(p, e, f2(0.999998927116394f, 0.999998927116394f));
+    return mul2(p, e);
+}
+
+// softplus and SiLU of a pair (same formulas as the scalar versions above).
+__device__ __forceinline__ float2 softplus2(float2 v) {
+    const float2 m = mul2(f2(fabsf(v.x), fabsf(v.y)), f2(-kLog2e, -kLog2e));
+    const float2 l = log1p_unit2(ex2x2(m));
+    return add2(f2(fmaxf(v.x, 0.f), fmaxf(v.y, 0.f)), l);
+}
+__device__ __forceinline__ float2 silu2(float2 z) {
+    const float2 e = ex2x2(mul2(z, f2(-kLog2e, -kLog2e)));
+    const float2 s = add2(e, f2(1.f, 1.f));
+    return f2(__fdividef(z.x, s.x), __fdividef(z.y, s.y));
+}
+
 // bfloat16 <-> float32. Widening is exact (the bf16 bits are the top half of
 // the float); narrowing rounds to nearest even.
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -70,7 +101,19 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem, int src
                  "r"(src_bytes)
                  : "memory");
 }
+// 4- or 8-byte asynchronous copy (same zero-fill rule).
+template <int BYTES>
+__device__ __forceinline__ void cp_async_small(void *smem, const void *gmem, int src_bytes) {
+    static_assert(BYTES == 4 || BYTES == 8, "cp.async.ca copies 4, 8 or 16 bytes");
+    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.ca.shared.global [%0], [%1], %2, %3;\n" ::"r"(s), "l"(gmem), "n"(BYTES),
+                 "r"(src_bytes)
+                 : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+// Wait until at most N of this thread's committed groups are still in flight.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
 
 }  // namespace ms

@@ -26,7 +26,9 @@ struct ScanParams {
 
 // Launch configuration chosen on the host for one scan call.
 struct ScanPlan {
-    int lg;             // lanes that share one row pair's chunk (4, 8 or 16)
+    int kind;           // 0: chunked kernels (scan_fwd.cu); 1: sequential kernels (scan_rec.cu)
+    int lg;             // kind 0: lanes that share one row pair's chunk (4, 8 or 16);
+                        // kind 1: lanes per row (2, 4, 8 or 16)
     int config;         // index of the compiled kernel configuration
     int warps;          // warps per CTA
     int rows_per_cta;   // warps * (32 / lg)
@@ -43,8 +45,18 @@ ScanPlan plan_scan(const ScanParams &p, int in_dtype, int force_segments, int nu
 bool make_plan(const ScanParams &p, int in_dtype, int config, int warps, int segments, ScanPlan *out);
 int scan_num_configs();
 bool scan_config_info(int config, int *lanes, int *states_per_pass, int *max_warps);
+int scan_config_kind(int config);   // 0 chunked, 1 sequential, -1 unknown index
 cudaError_t launch_scan(const ScanParams &p, const ScanPlan &plan, int in_dtype,
                         cudaStream_t stream);
+
+// Sequential kernels (scan_rec.cu): CTAs of rec_threads() threads (recurrence
+// and I/O warps) owning rec_rows(lanes_per_row) rows, no workspace, one segment.
+int rec_smem_bytes(int in_dtype, int lanes_per_row);
+int rec_chunk();
+int rec_threads();
+int rec_rows(int lanes_per_row);
+int rec_ctas_per_sm(int in_dtype, int lanes_per_row, bool vec);
+cudaError_t launch_rec(const ScanParams &p, int lanes_per_row, bool vec, int in_dtype, cudaStream_t stream);
 
 struct UpdateParams {
     int64_t batch, dim, dstate;

@@ -79,26 +79,8 @@ __host__ __device__ __forceinline__ Layout layout(int W) {
     return s;
 }
 
-__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
-__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
-__device__ __forceinline__ float2 ex2x2(float2 v) { return f2(ex2_approx(v.x), ex2_approx(v.y)); }
 __device__ __forceinline__ float2 shfl_up2(float2 v, int off, int width) {
     return f2(__shfl_up_sync(0xffffffffu, v.x, off, width), __shfl_up_sync(0xffffffffu, v.y, off, width));
-}
-
-// log1p(e) = e p(e) on [0, 1] with p of degree 6 (max relative error of
-// log1p 1.7e-6 in float32 evaluation); coefficients from fit_log1p.py.
-__device__ __forceinline__ float2 log1p_unit2(float2 e) {
-    float2 p = f2(0.014539077877998352f, 0.014539077877998352f);
-    p = fma2(p, e, f2(-0.06759698688983917f, -0.06759698688983917f));
-    p = fma2(p, e, f2(0.15056990087032318f, 0.15056990087032318f));
-    p = fma2(p, e, f2(-0.23573748767375946f, -0.23573748767375946f));
-    p = fma2(p, e, f2(0.3312585949897766f, 0.3312585949897766f));
-    p = fma2(p, e, f2(-0.499883770942688f, -0.499883770942688f));
-    p = fma2(p, e, f2(0.999998927116394f, 0.999998927116394f));
-    return mul2(p, e);
 }
 
 // 64-bit register views of a float pair, for the predicated packed ops below.
@@ -134,22 +116,6 @@ __device__ __forceinline__ float2 enter_state(int take, float2 Pe, float2 He, fl
         : "+l"(r)
         : "l"(b64(Pe)), "l"(b64(He)), "r"(take));
     return unb64(r);
-}
-
-// softplus(v) = max(v, 0) + log1p(exp(-|v|)). Above v = 20 the second term is
-// below 2.1e-9, under half an ulp of v, so the float32 result is v itself:
-// the "identity above 20" rule holds without a separate branch.
-__device__ __forceinline__ float2 softplus2(float2 v) {
-    const float2 m = mul2(f2(fabsf(v.x), fabsf(v.y)), f2(-kLog2e, -kLog2e));
-    const float2 l = log1p_unit2(ex2x2(m));
-    return add2(f2(fmaxf(v.x, 0.f), fmaxf(v.y, 0.f)), l);
-}
-
-// SiLU(z) = z / (1 + e^-z)
-__device__ __forceinline__ float2 silu2(float2 z) {
-    const float2 e = ex2x2(mul2(z, f2(-kLog2e, -kLog2e)));
-    const float2 s = add2(e, f2(1.f, 1.f));
-    return f2(__fdividef(z.x, s.x), __fdividef(z.y, s.y));
 }
 
 // The lane's 8 steps of two consecutive rows of an input tile, as (row, row+1) pairs.
@@ -622,6 +588,18 @@ double config_cost(const Config &c) {
     return (c.lg == 4 ? 7.3 : c.lg == 8 ? 7.7 : 8.1) * (c.ni == 0 ? 0.94 : c.ni == 2 ? 0.97 : 1.0);
 }
 
+// The sequential kernels (scan_rec.cu) follow the chunked configurations in
+// the configuration index: lanes per row and their measured cost over the
+// MUFU bound on a busy SM (shared-memory wavefronts of the step-tile and B/C
+// loads grow with the lanes per row; fitted to B200 timings of Mamba-130M,
+// Mamba-1.4B and 131k-token layers).
+constexpr int kRecLanes[] = {2, 4, 8, 16};
+constexpr int kNumRec = sizeof(kRecLanes) / sizeof(kRecLanes[0]);
+constexpr double kRecCost[] = {1.6, 1.9, 2.5, 4.2};
+// SM clocks per unit of the chunked kernels' cost model (measured: a
+// Mamba-130M layer on cfg 7, 11 warps, took 485k clocks for 1.30M units).
+constexpr double kChunkedClocksPerUnit = 0.372;
+
 // Registers per thread of a kernel, cached (cudaFuncGetAttributes is slow).
 int kernel_regs(const void *k) {
     constexpr int kSlots = 64;
@@ -697,12 +675,62 @@ ScanPlan plan_scan(const ScanParams &p, int in_dtype, int force_segments, int nu
             }
         }
     }
+    // Sequential kernels: no segments; an SM runs its CTAs in waves of as many
+    // as are resident, every resident CTA adds one recurrence warp per
+    // sub-partition, and a lone CTA runs 1.4x slower per row than a shared SM.
+    int rec = -1;
+    if (force_segments <= 1 && p.dstate <= kMaxN) {
+        const double mufu = (kMaxN + 3) / 16.0;   // MUFU clocks per (row, step): 16 states + softplus + gate
+        best *= kChunkedClocksPerUnit;
+        for (int ri = 0; ri < kNumRec; ++ri) {
+            const int lpr = kRecLanes[ri];
+            const int per_sm = rec_ctas_per_sm(in_dtype, lpr, plan.vec);
+            if (per_sm < 1) continue;
+            const int64_t R = rec_rows(lpr);
+            const int64_t ctas = p.batch * ((p.dim + R - 1) / R);
+            const int64_t heavy = (ctas + sms - 1) / sms;
+            auto wave = [&](int64_t m) {
+                return (m == 1 ? 1.4 : static_cast<double>(m)) * R * static_cast<double>(p.seqlen) * mufu * kRecCost[ri];
+            };
+            const double t = (heavy / per_sm) * wave(per_sm) + (heavy % per_sm ? wave(heavy % per_sm) : 0.0);
+            if (t < best * 0.999) {
+                best = t;
+                rec = ri;
+            }
+        }
+    }
     ScanPlan out = plan;
-    make_plan(p, in_dtype, plan.config, plan.warps, plan.nseg, &out);
+    if (rec >= 0) {
+        make_plan(p, in_dtype, kNumConfigs + rec, rec_threads() / 32, 1, &out);
+    } else {
+        make_plan(p, in_dtype, plan.config, plan.warps, plan.nseg, &out);
+    }
     return out;
 }
 
 bool make_plan(const ScanParams &p, int in_dtype, int config, int warps, int segments, ScanPlan *out) {
+    if (config >= kNumConfigs && config < kNumConfigs + kNumRec) {
+        // sequential kernel: fixed CTA of rec_threads(), the whole sequence in one pass
+        if (warps != rec_threads() / 32 || segments != 1 || p.dstate > kMaxN) return false;
+        const int eb = in_dtype == 0 ? 4 : 2;
+        auto strides_ok = [&](int64_t s1, int64_t s2) { return (s1 * eb) % 16 == 0 && (s2 * eb) % 16 == 0; };
+        ScanPlan plan{};
+        plan.kind = 1;
+        plan.config = config;
+        plan.lg = kRecLanes[config - kNumConfigs];
+        plan.warps = warps;
+        plan.rows_per_cta = rec_rows(plan.lg);
+        plan.chunk = rec_chunk();
+        plan.vec = aligned16(p.u) && aligned16(p.delta) && aligned16(p.B) && aligned16(p.C) &&
+                   aligned16(p.y) && (p.z == nullptr || aligned16(p.z)) && strides_ok(p.u_sb, p.u_sd) &&
+                   strides_ok(p.dl_sb, p.dl_sd) && strides_ok(p.B_sb, p.B_sn) && strides_ok(p.C_sb, p.C_sn) &&
+                   strides_ok(p.y_sb, p.y_sd) && (p.z == nullptr || strides_ok(p.z_sb, p.z_sd));
+        plan.nseg = 1;
+        plan.seg_len = p.seqlen;
+        plan.ws_bytes = 0;
+        *out = plan;
+        return true;
+    }
     if (config < 0 || config >= kNumConfigs || segments < 1) return false;
     const Config cf = kConfigs[config];
     ScanPlan plan{};
@@ -733,9 +761,21 @@ bool make_plan(const ScanParams &p, int in_dtype, int config, int warps, int seg
     return true;
 }
 
-int scan_num_configs() { return kNumConfigs; }
+int scan_num_configs() { return kNumConfigs + kNumRec; }
+
+int scan_config_kind(int config) {
+    if (config < 0 || config >= kNumConfigs + kNumRec) return -1;
+    return config < kNumConfigs ? 0 : 1;
+}
 
 bool scan_config_info(int config, int *lanes, int *states_per_pass, int *max_warps) {
+    if (config >= kNumConfigs && config < kNumConfigs + kNumRec) {
+        const int lpr = kRecLanes[config - kNumConfigs];
+        if (lanes) *lanes = lpr;
+        if (states_per_pass) *states_per_pass = kMaxN / lpr;
+        if (max_warps) *max_warps = rec_threads() / 32;
+        return true;
+    }
     if (config < 0 || config >= kNumConfigs) return false;
     if (lanes) *lanes = kConfigs[config].lg;
     if (states_per_pass) *states_per_pass = kConfigs[config].ni;
@@ -744,6 +784,7 @@ bool scan_config_info(int config, int *lanes, int *states_per_pass, int *max_war
 }
 
 cudaError_t launch_scan(const ScanParams &p, const ScanPlan &plan, int in_dtype, cudaStream_t stream) {
+    if (plan.kind == 1) return launch_rec(p, plan.lg, plan.vec != 0, in_dtype, stream);
     const int W = plan.warps;
     const int smem = smem_bytes(in_dtype, plan.lg, W);
     const unsigned gx = static_cast<unsigned>((p.dim + plan.rows_per_cta - 1) / plan.rows_per_cta);

@@ -1,0 +1,638 @@
+// Selective scan (S6) forward, sequential form, for sm_100a.
+//
+// Same operation as scan_fwd.cu ("Notas sobre Mamba", sections "O mecanismo de
+// seleção (S6)" and "A varredura paralela ciente do hardware"; "Mamba-2 e
+// State Space Duality (SSD)", section "Como o Mamba-1 alcançou complexidade
+// linear"): for every row (b, d) and state index n
+//     h_t[n] = exp(delta_t A[d,n]) h_{t-1}[n] + delta_t B_t[n] u_t
+//     y_t    = sum_n C_t[n] h_t[n] + D[d] u_t      (then * silu(z_t))
+// with delta_t = softplus(delta_raw_t + delta_bias[d]).
+//
+// Design. The recurrence runs exactly as written, one time step after the
+// other, and the parallelism comes from the (row, state) pairs instead of the
+// time axis: LPR lanes share a row and each owns NPL = 16 / LPR of its states
+// in registers for the whole sequence. There is no scan, no carry and no
+// second pass, so the per-element work is the minimum the recurrence needs --
+// one ex2 on the MUFU plus, per pair of states, one packed multiply for
+// delta A, one for delta u B, one packed FMA for h and one for the readout.
+// The MUFU (16 results/clk/SM) is the bound. A (batch 8, d_inner 1536, N 16)
+// layer already has 196,608 independent (row, state) chains.
+//
+// The CTA is warp-specialised so that the MUFU never waits for the per-row
+// work around the recurrence:
+//  * 4 recurrence warps (one per SM sub-partition) own R = 128 / LPR rows of
+//    one batch entry and step their states through chunks of 16 steps,
+//    leaving each lane's partial readout sum_{own n} C_t[n] h_t[n] in shared
+//    memory;
+//  * 2 I/O warps prepare chunk c + 1 while the recurrence runs chunk c --
+//    delta = softplus(delta_raw + bias) and delta u stored as (delta, delta,
+//    delta u, delta u), the operand pairs of the packed multiplies, and the
+//    chunk's B and C tiles (shared by all rows) widened to float32 -- and
+//    finish chunk c - 1: sum the LPR partials, add D u, apply the SiLU gate
+//    and store y. Their global loads run one chunk ahead.
+// The two groups hand the double-buffered tiles over through named hardware
+// barriers (bar.arrive by the producer, bar.sync by the consumer; no spin
+// loops). Steps past the end of the sequence get delta = 0 (Abar = 1, Bbar u
+// = 0): the state reaches the final-state output unchanged.
+#include <mutex>
+#include <type_traits>
+
+#include "device_math.cuh"
+#include "launch.h"
+
+namespace ms {
+namespace {
+
+constexpr int kScanThreads = 128;   // 4 recurrence warps
+constexpr int kIoThreads = 64;      // 2 I/O warps
+constexpr int kThreads = kScanThreads + kIoThreads;
+constexpr int kSteps = 16;          // time steps per chunk
+constexpr int kStates = 16;         // states per row (smaller dstate is zero-padded)
+
+// Shared-memory layout of one of the two stages, in bytes. The step tile holds
+// one float4 per (row, step), with one float4 of padding after each I/O
+// thread's piece of IP steps; the readout tile holds, per row and lane, the
+// lane's partial readout of every step ([row][lane][step], YQ floats per lane
+// and YR per row). The paddings keep the recurrence warps' loads and stores
+// and the I/O warps' tile stores free of bank conflicts.
+template <int LPR> struct Shape {
+    static constexpr int NPL = kStates / LPR;           // states per lane
+    static constexpr int R = kScanThreads / LPR;        // rows per CTA
+    static constexpr int IPR = LPR / 2;                 // I/O threads per row
+    static constexpr int IP = kSteps / IPR;             // steps per I/O thread
+    static constexpr int XR = LPR == 2 ? 17 : LPR == 4 ? 18 : LPR == 8 ? 20 : 24;   // float4 per row
+    static constexpr int YQ = 20;
+    static constexpr int YR = LPR == 2 ? 40 : LPR == 4 ? 80 : LPR == 8 ? 176 : 336;
+    static constexpr int X_OFF = 0;
+    static constexpr int Y_OFF = X_OFF + R * XR * 16;
+    static constexpr int B_OFF = Y_OFF + R * YR * 4;
+    static constexpr int C_OFF = B_OFF + kSteps * kStates * 4;
+    static constexpr int STAGE = C_OFF + kSteps * kStates * 4;
+    static constexpr int BYTES = 2 * STAGE;
+    // CTAs per SM the launch bounds provide registers for
+    static constexpr int MINB = LPR == 2 ? 2 : LPR == 4 ? 3 : LPR == 8 ? 4 : 5;
+    static_assert(R * IPR == kIoThreads, "the I/O threads cover the rows");
+    static_assert(XR >= kSteps + IPR, "step tile row holds the padded pieces");
+    static_assert(YQ >= kSteps && YQ % 4 == 0 && YR >= LPR * YQ && YR % 4 == 0, "readout tile");
+};
+
+// The I/O warps' ring of raw inputs in shared memory, after the two stages:
+// kRawStages chunks in flight, each I/O thread filling and reading only its
+// own 16-byte slots (its u, delta and z pieces of PB bytes each, then its B/C
+// pieces), stored slot-major so that a warp's slot accesses are contiguous.
+constexpr int kRawStages = 4;   // a power of two
+template <typename T, int LPR> struct Raw {
+    static constexpr int EB = static_cast<int>(sizeof(T));
+    static constexpr int PB = Shape<LPR>::IP * EB;                   // bytes of one u/delta/z piece
+    static constexpr int PS = (PB + 15) / 16;                        // slots per piece
+    static constexpr int VE = 16 / EB;                               // elements per B/C piece
+    static constexpr int BC_PER = 2 * kStates * (kSteps / VE) / kIoThreads;   // B/C pieces per thread
+    static constexpr int SLOTS = 3 * PS + BC_PER;
+    static constexpr int STAGE = SLOTS * kIoThreads * 16;
+    static constexpr int OFF = Shape<LPR>::BYTES;
+    static constexpr int BYTES = OFF + kRawStages * STAGE;           // total dynamic shared memory
+    static_assert(BC_PER * kIoThreads * VE == 2 * kStates * kSteps, "B/C pieces split evenly");
+    static_assert(PB == 4 || PB == 8 || PB % 16 == 0, "piece sizes cp.async can copy");
+};
+
+// Named barriers (0 is __syncthreads): the producer arrives, the consumer
+// waits; kThreads threads complete each phase.
+//   XF(s): stage s's step and B/C tiles are ready       (I/O -> recurrence)
+//   XE(s): stage s's step and B/C tiles may be rewritten (recurrence -> I/O)
+//   YF(s): stage s's readout partials are ready          (recurrence -> I/O)
+//   YE(s): stage s's readout tile may be rewritten       (I/O -> recurrence)
+__device__ __forceinline__ int bar_xf(int s) { return 1 + s; }
+__device__ __forceinline__ int bar_xe(int s) { return 3 + s; }
+__device__ __forceinline__ int bar_yf(int s) { return 5 + s; }
+__device__ __forceinline__ int bar_ye(int s) { return 7 + s; }
+__device__ __forceinline__ void bar_wait(int id) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(kThreads) : "memory");
+}
+__device__ __forceinline__ void bar_signal(int id) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "n"(kThreads) : "memory");
+}
+
+// One step's operands of a lane: (delta, delta, delta u, delta u) and the
+// lane's B_t and C_t entries as pairs.
+template <int NPL> struct StepIn {
+    float2 b[NPL > 1 ? NPL / 2 : 1], c[NPL > 1 ? NPL / 2 : 1];
+};
+
+template <int NPL>
+__device__ __forceinline__ StepIn<NPL> load_bc_step(const float *Bl, const float *Cl) {
+    StepIn<NPL> s;
+    if constexpr (NPL == 1) {
+        s.b[0] = f2(*Bl, 0.f);
+        s.c[0] = f2(*Cl, 0.f);
+    } else if constexpr (NPL == 2) {
+        s.b[0] = *reinterpret_cast<const float2 *>(Bl);
+        s.c[0] = *reinterpret_cast<const float2 *>(Cl);
+    } else {
+#pragma unroll
+        for (int v = 0; v < NPL / 4; ++v) {
+            const float4 b4 = reinterpret_cast<const float4 *>(Bl)[v];
+            const float4 c4 = reinterpret_cast<const float4 *>(Cl)[v];
+            s.b[2 * v] = f2(b4.x, b4.y); s.b[2 * v + 1] = f2(b4.z, b4.w);
+            s.c[2 * v] = f2(c4.x, c4.y); s.c[2 * v + 1] = f2(c4.z, c4.w);
+        }
+    }
+    return s;
+}
+
+// P consecutive elements of one row in 32-bit words (bf16 pairs or floats).
+template <typename T, int P> struct Piece {
+    static constexpr int W = P * static_cast<int>(sizeof(T)) / 4;
+    uint32_t w[W];
+};
+
+template <typename T, int P>
+__device__ __forceinline__ float elem(const Piece<T, P> &pc, int e) {
+    if constexpr (std::is_same<T, float>::value) return __uint_as_float(pc.w[e]);
+    else return (e & 1) ? bf16_hi(pc.w[e >> 1]) : bf16_lo(pc.w[e >> 1]);
+}
+
+// Load `valid` (<= P) elements from src; the rest read as zero and are not
+// touched in memory. VEC: src is aligned to the piece size.
+template <typename T, int P, bool VEC>
+__device__ __forceinline__ void load_piece(Piece<T, P> &pc, const T *src, int64_t valid) {
+    constexpr int W = Piece<T, P>::W;
+    if (VEC && valid >= P) {
+        if constexpr (W == 1) {
+            pc.w[0] = __ldg(reinterpret_cast<const unsigned *>(src));
+        } else if constexpr (W == 2) {
+            const uint2 v = __ldg(reinterpret_cast<const uint2 *>(src));
+            pc.w[0] = v.x; pc.w[1] = v.y;
+        } else {
+#pragma unroll
+            for (int i = 0; i < W / 4; ++i) {
+                const uint4 v = __ldg(reinterpret_cast<const uint4 *>(src) + i);
+                pc.w[4 * i] = v.x; pc.w[4 * i + 1] = v.y; pc.w[4 * i + 2] = v.z; pc.w[4 * i + 3] = v.w;
+            }
+        }
+    } else if constexpr (std::is_same<T, float>::value) {
+#pragma unroll
+        for (int e = 0; e < P; ++e) pc.w[e] = e < valid ? __float_as_uint(__ldg(src + e)) : 0u;
+    } else {
+        const unsigned short *s = reinterpret_cast<const unsigned short *>(src);
+#pragma unroll
+        for (int i = 0; i < W; ++i) {
+            const uint32_t lo = 2 * i < valid ? __ldg(s + 2 * i) : 0u;
+            const uint32_t hi = 2 * i + 1 < valid ? __ldg(s + 2 * i + 1) : 0u;
+            pc.w[i] = lo | (hi << 16);
+        }
+    }
+}
+
+// Store the first `count` (<= P) of P float values as T.
+template <typename T, int P, bool VEC>
+__device__ __forceinline__ void store_piece(T *dst, const float (&v)[P], int64_t count) {
+    if constexpr (std::is_same<T, float>::value) {
+        if (VEC && count >= P) {
+            if constexpr (P == 2) {
+                *reinterpret_cast<float2 *>(dst) = make_float2(v[0], v[1]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < P / 4; ++i)
+                    reinterpret_cast<float4 *>(dst)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < P; ++e)
+                if (e < count) dst[e] = v[e];
+        }
+    } else {
+        uint32_t w[P / 2];
+#pragma unroll
+        for (int i = 0; i < P / 2; ++i) {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+            w[i] = *reinterpret_cast<const uint32_t *>(&h);
+        }
+        if (VEC && count >= P) {
+            if constexpr (P == 2) {
+                *reinterpret_cast<uint32_t *>(dst) = w[0];
+            } else if constexpr (P == 4) {
+                *reinterpret_cast<uint2 *>(dst) = make_uint2(w[0], w[1]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < P / 8; ++i)
+                    reinterpret_cast<uint4 *>(dst)[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+            }
+        } else {
+            unsigned short *o = reinterpret_cast<unsigned short *>(dst);
+#pragma unroll
+            for (int e = 0; e < P; ++e)
+                if (e < count) o[e] = static_cast<unsigned short>((e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xffffu));
+        }
+    }
+}
+
+// The recurrence warps: lane (r, q) owns states q NPL .. q NPL + NPL - 1 of row r.
+template <typename T, int LPR>
+__device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned char *smem, int tid) {
+    using S = Shape<LPR>;
+    constexpr int NPL = S::NPL, R = S::R, IP = S::IP;
+    constexpr int NP = NPL > 1 ? NPL / 2 : 1;
+    const int r = tid / LPR, q = tid % LPR;
+    const int64_t b = blockIdx.y;
+    const int64_t d = static_cast<int64_t>(blockIdx.x) * R + r;
+    const bool ok = d < p.dim;
+    const int64_t dc = ok ? d : p.dim - 1;    // clamped row: loads stay in bounds
+    const int dstate = static_cast<int>(p.dstate);
+    const int64_t nchunks = (p.seqlen + kSteps - 1) / kSteps;
+    const int64_t row = b * p.dim + dc;
+
+    // A log2(e) and the entering state of the lane's states, kept as the
+    // register pairs the packed instructions take (no moves in the loop).
+    float2 ap[NP], hp[NP];
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+        float a2[2] = {0.f, 0.f}, h2[2] = {0.f, 0.f};
+#pragma unroll
+        for (int e = 0; e < 2 && 2 * j + e < NPL; ++e) {
+            const int n = q * NPL + 2 * j + e;
+            if (n < dstate) {
+                a2[e] = __ldg(p.A + dc * dstate + n) * kLog2e;
+                if (p.h0) h2[e] = __ldg(p.h0 + row * dstate + n);
+            }
+        }
+        ap[j] = f2(a2[0], a2[1]);
+        hp[j] = f2(h2[0], h2[1]);
+    }
+
+    for (int64_t c = 0; c < nchunks; ++c) {
+        const int s = static_cast<int>(c & 1);
+        unsigned char *st = smem + s * S::STAGE;
+        const float4 *xrow = reinterpret_cast<const float4 *>(st + S::X_OFF) + r * S::XR;
+        float *yl = reinterpret_cast<float *>(st + S::Y_OFF) + r * S::YR + q * S::YQ;
+        const float *Bl = reinterpret_cast<const float *>(st + S::B_OFF) + q * NPL;
+        const float *Cl = reinterpret_cast<const float *>(st + S::C_OFF) + q * NPL;
+        bar_wait(bar_xf(s));
+        if (c >= 2) bar_wait(bar_ye(s));
+
+        // Software pipelined over the chunk: the step tile is read two steps
+        // ahead, B and C one step ahead, and the ex2 of step t + 1 is issued
+        // before the FMAs of step t, so neither shared-memory nor MUFU latency
+        // sits on the state's dependency chain. Partial readouts leave in
+        // float4 stores every 4 steps.
+        auto xat = [&](int t) { return xrow[t + t / IP]; };
+        auto decay = [&](const float4 &x, float2 (&a)[NP]) {
+            if constexpr (NPL == 1) {
+                a[0] = f2(ex2_approx(x.x * ap[0].x), 0.f);
+            } else {
+#pragma unroll
+                for (int j = 0; j < NP; ++j) a[j] = ex2x2(mul2(f2(x.x, x.y), ap[j]));
+            }
+        };
+        float4 x0 = xat(0), x1 = xat(1);
+        float2 acur[NP];
+        decay(x0, acur);
+        StepIn<NPL> cur = load_bc_step<NPL>(Bl, Cl);
+        float outs[4];
+#pragma unroll
+        for (int t = 0; t < kSteps; ++t) {
+            float4 x2 = x1;
+            if (t + 2 < kSteps) x2 = xat(t + 2);
+            StepIn<NPL> nxt = cur;
+            float2 anxt[NP];
+            if (t + 1 < kSteps) {
+                nxt = load_bc_step<NPL>(Bl + (t + 1) * kStates, Cl + (t + 1) * kStates);
+                decay(x1, anxt);
+            }
+            if constexpr (NPL == 1) {
+                hp[0].x = fmaf(acur[0].x, hp[0].x, x0.z * cur.b[0].x);
+                outs[t & 3] = cur.c[0].x * hp[0].x;
+            } else {
+                const float2 du = f2(x0.z, x0.w);
+                float2 acc;
+#pragma unroll
+                for (int j = 0; j < NP; ++j) {
+                    hp[j] = fma2(acur[j], hp[j], mul2(du, cur.b[j]));
+                    acc = j == 0 ? mul2(cur.c[j], hp[j]) : fma2(cur.c[j], hp[j], acc);
+                }
+                outs[t & 3] = acc.x + acc.y;
+            }
+            if ((t & 3) == 3)
+                *reinterpret_cast<float4 *>(yl + t - 3) = make_float4(outs[0], outs[1], outs[2], outs[3]);
+            if (t + 1 < kSteps) {
+                x0 = x1;
+                x1 = x2;
+                cur = nxt;
+#pragma unroll
+                for (int j = 0; j < NP; ++j) acur[j] = anxt[j];
+            }
+        }
+        if (c + 2 < nchunks) bar_signal(bar_xe(s));
+        bar_signal(bar_yf(s));
+    }
+
+    if (ok && p.hT) {
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+            const int n = q * NPL + i;
+            if (n < dstate) p.hT[row * dstate + n] = (i & 1) ? hp[i / 2].y : hp[i / 2].x;
+        }
+    }
+}
+
+// The I/O warps: thread (r, k) handles steps k IP .. k IP + IP - 1 of row r in
+// every chunk, plus BC_PER 16-byte pieces of the chunk's B/C tiles. Its raw
+// inputs travel through the ring kRawStages - 1 chunks ahead of use
+// (cp.async on the aligned path, plain loads otherwise); a thread waits only
+// for its own copies, so the ring needs no barrier.
+template <typename T, int LPR, bool VEC>
+__device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem, int i) {
+    using S = Shape<LPR>;
+    using RW = Raw<T, LPR>;
+    constexpr int R = S::R, IP = S::IP, IPR = S::IPR, EB = RW::EB, PB = RW::PB, PS = RW::PS;
+    constexpr int VE = RW::VE, BC_PER = RW::BC_PER;
+    static_assert(IP % 2 == 0, "pieces hold step pairs");
+    const int r = i / IPR, k = i % IPR;
+    const int64_t b = blockIdx.y;
+    const int64_t d = static_cast<int64_t>(blockIdx.x) * R + r;
+    const bool ok = d < p.dim;
+    const int64_t dc = ok ? d : p.dim - 1;
+    const int dstate = static_cast<int>(p.dstate);
+    const int64_t L = p.seqlen;
+    const int64_t nchunks = (L + kSteps - 1) / kSteps;
+
+    const float bias = p.delta_bias ? __ldg(p.delta_bias + dc) : 0.f;
+    const float Dd = p.D ? __ldg(p.D + dc) : 0.f;
+    const bool has_z = p.z != nullptr;
+    const int tk = k * IP;   // the thread's first step within a chunk
+    const T *src_row[3] = {static_cast<const T *>(p.u) + b * p.u_sb + dc * p.u_sd + tk,
+                           static_cast<const T *>(p.delta) + b * p.dl_sb + dc * p.dl_sd + tk,
+                           has_z ? static_cast<const T *>(p.z) + b * p.z_sb + dc * p.z_sd + tk : nullptr};
+    T *yrow = static_cast<T *>(p.y) + b * p.y_sb + dc * p.y_sd + tk;
+
+    // The thread's B/C pieces: tensor (0 = B, 1 = C), state n, steps bt .. bt + VE - 1.
+    int bc_off[BC_PER], bc_t[BC_PER];
+    bool bc_live[BC_PER];
+    const T *bc_src[BC_PER];
+#pragma unroll
+    for (int j = 0; j < BC_PER; ++j) {
+        const int pc = i + j * kIoThreads;
+        const int tensor = pc / (kStates * (kSteps / VE));
+        const int rem = pc % (kStates * (kSteps / VE));
+        const int n = rem % kStates;
+        bc_t[j] = (rem / kStates) * VE;
+        bc_off[j] = (tensor == 0 ? S::B_OFF : S::C_OFF) + (bc_t[j] * kStates + n) * 4;
+        bc_live[j] = n < dstate;
+        const T *base = tensor == 0 ? static_cast<const T *>(p.B) + b * p.B_sb : static_cast<const T *>(p.C) + b * p.C_sb;
+        bc_src[j] = (bc_live[j] ? base + n * (tensor == 0 ? p.B_sn : p.C_sn) : base) + bc_t[j];
+    }
+
+    unsigned char *ring = smem + RW::OFF;
+    auto slot = [&](int64_t c, int sl) {
+        return ring + static_cast<int>(c & (kRawStages - 1)) * RW::STAGE + (sl * kIoThreads + i) * 16;
+    };
+
+    // Issue the copies of chunk c's raw inputs into its ring stage.
+    auto stage_chunk = [&](int64_t c) {
+        const int64_t t0 = c * kSteps;
+        const bool full = t0 + kSteps <= L;
+        const int valid = full ? IP : static_cast<int>(min64(IP, max64(0, L - (t0 + tk))));
+#pragma unroll
+        for (int tsr = 0; tsr < 3; ++tsr) {
+            if (tsr == 2 && !has_z) break;
+            const T *src = src_row[tsr] + t0;
+            if constexpr (VEC) {
+#pragma unroll
+                for (int sl = 0; sl < PS; ++sl) {
+                    const int have = valid * EB - sl * 16;
+                    const int bytes = have < 0 ? 0 : (have > (PB < 16 ? PB : 16) ? (PB < 16 ? PB : 16) : have);
+                    const void *g = bytes > 0 ? static_cast<const void *>(reinterpret_cast<const unsigned char *>(src) + sl * 16)
+                                              : static_cast<const void *>(src_row[tsr]);
+                    if constexpr (PB >= 16) cp_async16(slot(c, tsr * PS + sl), g, bytes);
+                    else cp_async_small<PB>(slot(c, tsr * PS + sl), g, bytes);
+                }
+            } else {
+                Piece<T, IP> pc;
+                load_piece<T, IP, false>(pc, src, valid);
+#pragma unroll
+                for (int w = 0; w < Piece<T, IP>::W; ++w)
+                    reinterpret_cast<uint32_t *>(slot(c, tsr * PS + w / 4))[w % 4] = pc.w[w];
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < BC_PER; ++j) {
+            const int vb = bc_live[j] ? (full ? VE : static_cast<int>(min64(VE, max64(0, L - (t0 + bc_t[j]))))) : 0;
+            if constexpr (VEC) {
+                cp_async16(slot(c, 3 * PS + j), vb > 0 ? static_cast<const void *>(bc_src[j] + t0)
+                                                       : static_cast<const void *>(bc_src[j]), vb * EB);
+            } else {
+                Piece<T, VE> pc;
+                load_piece<T, VE, false>(pc, bc_src[j] + t0, vb);
+                *reinterpret_cast<uint4 *>(slot(c, 3 * PS + j)) = make_uint4(pc.w[0], pc.w[1], pc.w[2], pc.w[3]);
+            }
+        }
+    };
+    // The thread's piece of tensor tsr of chunk c, from the ring.
+    auto ring_piece = [&](int64_t c, int tsr) {
+        Piece<T, IP> pc;
+        if constexpr (PB == 4) {
+            pc.w[0] = *reinterpret_cast<const uint32_t *>(slot(c, tsr * PS));
+        } else if constexpr (PB == 8) {
+            const uint2 v = *reinterpret_cast<const uint2 *>(slot(c, tsr * PS));
+            pc.w[0] = v.x; pc.w[1] = v.y;
+        } else {
+#pragma unroll
+            for (int sl = 0; sl < PS; ++sl) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(slot(c, tsr * PS + sl));
+                pc.w[4 * sl] = v.x; pc.w[4 * sl + 1] = v.y; pc.w[4 * sl + 2] = v.z; pc.w[4 * sl + 3] = v.w;
+            }
+        }
+        return pc;
+    };
+    // Readout of chunk c from stage s: partial sums + D u, gate, store.
+    auto finish = [&](int64_t c, int s) {
+        const int64_t cnt = L - (c * kSteps + tk);
+        if (!ok || cnt <= 0) return;
+        const float *yp = reinterpret_cast<const float *>(smem + s * S::STAGE + S::Y_OFF) + r * S::YR + tk;
+        float2 sum[IP / 2];
+#pragma unroll
+        for (int e = 0; e < IP / 2; ++e) sum[e] = f2(0.f, 0.f);
+#pragma unroll
+        for (int j = 0; j < LPR; ++j) {
+            if constexpr (IP == 2) {
+                sum[0] = add2(sum[0], *reinterpret_cast<const float2 *>(yp + j * S::YQ));
+            } else {
+#pragma unroll
+                for (int v = 0; v < IP / 4; ++v) {
+                    const float4 a = reinterpret_cast<const float4 *>(yp + j * S::YQ)[v];
+                    sum[2 * v] = add2(sum[2 * v], f2(a.x, a.y));
+                    sum[2 * v + 1] = add2(sum[2 * v + 1], f2(a.z, a.w));
+                }
+            }
+        }
+        const Piece<T, IP> u = ring_piece(c, 0);
+        float outv[IP];
+        if (has_z) {
+            const Piece<T, IP> z = ring_piece(c, 2);
+#pragma unroll
+            for (int e = 0; e < IP; e += 2) {
+                const float2 yv = fma2(f2(Dd, Dd), f2(elem(u, e), elem(u, e + 1)), sum[e / 2]);
+                const float2 g = mul2(yv, silu2(f2(elem(z, e), elem(z, e + 1))));
+                outv[e] = g.x;
+                outv[e + 1] = g.y;
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < IP; e += 2) {
+                const float2 yv = fma2(f2(Dd, Dd), f2(elem(u, e), elem(u, e + 1)), sum[e / 2]);
+                outv[e] = yv.x;
+                outv[e + 1] = yv.y;
+            }
+        }
+        store_piece<T, IP, VEC>(yrow + c * kSteps, outv, cnt);
+    };
+    // Chunk c's step tile (delta, delta, delta u, delta u) and B/C tiles into stage s.
+    auto widen = [&](int64_t c, int s) {
+        unsigned char *st = smem + s * S::STAGE;
+        float4 *xrow = reinterpret_cast<float4 *>(st + S::X_OFF) + r * S::XR + tk + k;
+        const Piece<T, IP> u = ring_piece(c, 0), dl = ring_piece(c, 1);
+        const bool full = (c + 1) * kSteps <= L;
+        const int64_t cnt = L - (c * kSteps + tk);
+#pragma unroll
+        for (int e = 0; e < IP; e += 2) {
+            float2 v = add2(f2(elem(dl, e), elem(dl, e + 1)), f2(bias, bias));
+            if (p.softplus) v = softplus2(v);
+            if (!full) {   // steps past the end: delta = 0
+                if (e >= cnt) v.x = 0.f;
+                if (e + 1 >= cnt) v.y = 0.f;
+            }
+            const float2 du = mul2(v, f2(elem(u, e), elem(u, e + 1)));
+            xrow[e] = make_float4(v.x, v.x, du.x, du.x);
+            xrow[e + 1] = make_float4(v.y, v.y, du.y, du.y);
+        }
+#pragma unroll
+        for (int j = 0; j < BC_PER; ++j) {
+            const uint4 w = *reinterpret_cast<const uint4 *>(slot(c, 3 * PS + j));
+            Piece<T, VE> pc;
+            pc.w[0] = w.x; pc.w[1] = w.y; pc.w[2] = w.z; pc.w[3] = w.w;
+            float *dst = reinterpret_cast<float *>(st + bc_off[j]);
+#pragma unroll
+            for (int e = 0; e < VE; ++e) dst[e * kStates] = elem(pc, e);
+        }
+    };
+
+    // Prologue: chunks 0 .. kRawStages - 2 in flight (one commit group per
+    // chunk, empty past the end, so that the group count stays uniform).
+#pragma unroll
+    for (int c0 = 0; c0 < kRawStages - 1; ++c0) {
+        if (c0 < nchunks) stage_chunk(c0);
+        cp_async_commit();
+    }
+    for (int64_t c = 0; c < nchunks; ++c) {
+        const int s = static_cast<int>(c & 1);
+        cp_async_wait<kRawStages - 2>();   // chunk c's copies have landed
+        if (c >= 2) bar_wait(bar_xe(s));
+        widen(c, s);
+        bar_signal(bar_xf(s));
+        if (c >= 1) {
+            bar_wait(bar_yf(s ^ 1));
+            finish(c - 1, s ^ 1);
+            if (c + 1 < nchunks) bar_signal(bar_ye(s ^ 1));
+        }
+        // chunk c + kRawStages - 1 reuses the ring stage that chunk c - 1 just released
+        if (c + kRawStages - 1 < nchunks) stage_chunk(c + kRawStages - 1);
+        cp_async_commit();
+    }
+    if (nchunks > 0) {
+        const int s = static_cast<int>((nchunks - 1) & 1);
+        bar_wait(bar_yf(s));
+        finish(nchunks - 1, s);
+    }
+    cp_async_wait<0>();
+}
+
+template <typename T, int LPR, bool VEC>
+__global__ void __launch_bounds__(kThreads, Shape<LPR>::MINB) rec_kernel(const ScanParams p) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    if (threadIdx.x < kScanThreads) {
+        recurrence_role<T, LPR>(p, smem, threadIdx.x);
+    } else {
+        io_role<T, LPR, VEC>(p, smem, threadIdx.x - kScanThreads);
+    }
+}
+
+template <typename T, int LPR>
+const void *rec_ptr(bool vec) {
+    return vec ? reinterpret_cast<const void *>(rec_kernel<T, LPR, true>)
+               : reinterpret_cast<const void *>(rec_kernel<T, LPR, false>);
+}
+
+template <typename T>
+const void *rec_select(int lpr, bool vec) {
+    switch (lpr) {
+        case 2: return rec_ptr<T, 2>(vec);
+        case 4: return rec_ptr<T, 4>(vec);
+        case 8: return rec_ptr<T, 8>(vec);
+        default: return rec_ptr<T, 16>(vec);
+    }
+}
+
+const void *rec_kernel_for(int in_dtype, int lpr, bool vec) {
+    return in_dtype == 0 ? rec_select<float>(lpr, vec) : rec_select<__nv_bfloat16>(lpr, vec);
+}
+
+}  // namespace
+
+template <typename T>
+int smem_bytes_t(int lpr) {
+    switch (lpr) {
+        case 2: return Raw<T, 2>::BYTES;
+        case 4: return Raw<T, 4>::BYTES;
+        case 8: return Raw<T, 8>::BYTES;
+        default: return Raw<T, 16>::BYTES;
+    }
+}
+
+int rec_smem_bytes(int in_dtype, int lpr) {
+    return in_dtype == 0 ? smem_bytes_t<float>(lpr) : smem_bytes_t<__nv_bfloat16>(lpr);
+}
+
+int rec_chunk() { return kSteps; }
+int rec_threads() { return kThreads; }
+int rec_rows(int lpr) { return kScanThreads / lpr; }
+
+// Resident CTAs per SM of a sequential kernel (cached per kernel; the
+// shared-memory bound when no device answers).
+int rec_ctas_per_sm(int in_dtype, int lpr, bool vec) {
+    constexpr int kSlots = 32;
+    static const void *keys[kSlots];
+    static int vals[kSlots];
+    static int used = 0;
+    static std::mutex mu;
+    const void *k = rec_kernel_for(in_dtype, lpr, vec);
+    std::lock_guard<std::mutex> lk(mu);
+    for (int i = 0; i < used; ++i)
+        if (keys[i] == k) return vals[i];
+    const int smem = rec_smem_bytes(in_dtype, lpr);
+    int n = 0;
+    bool asked = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess &&
+                 cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, kThreads, smem) == cudaSuccess;
+    if (!asked) {
+        cudaGetLastError();
+        n = (228 * 1024) / (smem + 1024);
+    } else if (used < kSlots) {
+        keys[used] = k;
+        vals[used] = n;
+        ++used;
+    }
+    return n;
+}
+
+cudaError_t launch_rec(const ScanParams &p, int lpr, bool vec, int in_dtype, cudaStream_t stream) {
+    const void *k = rec_kernel_for(in_dtype, lpr, vec);
+    const int smem = rec_smem_bytes(in_dtype, lpr);
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const int R = kScanThreads / lpr;
+    const dim3 grid(static_cast<unsigned>((p.dim + R - 1) / R), static_cast<unsigned>(p.batch));
+    void *args[] = {const_cast<ScanParams *>(&p)};
+    e = cudaLaunchKernel(k, grid, dim3(kThreads), args, static_cast<size_t>(smem), stream);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+}  // namespace ms

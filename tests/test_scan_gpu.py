@@ -177,33 +177,76 @@ def test_long_context_forced_segments_sampled_rows():
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_every_kernel_configuration(dtype):
-    """Each compiled configuration, forced through mamba_scan_fwd_with_plan, at
-    its smallest and largest CTA and with and without segments."""
+    """Each compiled configuration, forced through mamba_scan_fwd_with_plan:
+    chunked kernels at their smallest and largest CTA, with and without
+    segments; sequential kernels at their fixed CTA (other shapes refused)."""
     import torch
     ms = _ms()
     # rows 16-byte aligned (every configuration can run) and a ragged last chunk
     inp = make_scan_inputs(LAYER, batch=2, dim=88, seqlen=1000, dtype=dtype, seed=1100)
     dev = device_inputs(inp)
     yr, hr = oracle_scan(inp)
-    for cfg, lanes, states, max_warps in ms.scan_configs():
-        # the largest CTA whose shared memory fits (float32 tiles are twice as large)
-        largest = None
-        for warps in range(max_warps, 1, -1):
-            try:
-                ms.scan_fwd(**dev, plan=ms.ScanPlan(config=cfg, warps_per_cta=warps, segments=1))
-                largest = warps
-                break
-            except ms.MambaScanError as e:
-                assert e.status == 2
-        assert largest is not None, f"config {cfg} runs at no CTA size"
-        for warps in sorted({2, largest}):
-            for segments in (1, 3):
-                plan = ms.ScanPlan(config=cfg, warps_per_cta=warps, segments=segments)
-                y, hT = ms.scan_fwd(**dev, plan=plan)
-                torch.cuda.synchronize()
-                tag = f"config {cfg} (lanes {lanes}, states/pass {states}), {warps} warps, {segments} segments"
-                assert rel_err(to_host64(y), yr) <= TOL[dtype], tag
-                assert rel_err(to_host64(hT), hr) <= TOL[dtype], tag
+    for cfg, lanes, states, max_warps, kind in ms.scan_configs():
+        if kind == 1:
+            for warps, segments in ((2, 1), (max_warps, 2)):
+                with pytest.raises(ms.MambaScanError) as ei:
+                    ms.scan_fwd(**dev, plan=ms.ScanPlan(config=cfg, warps_per_cta=warps, segments=segments))
+                assert ei.value.status == 2
+            shapes = [(max_warps, 1)]
+        else:
+            # the largest CTA whose shared memory fits (float32 tiles are twice as large)
+            largest = None
+            for warps in range(max_warps, 1, -1):
+                try:
+                    ms.scan_fwd(**dev, plan=ms.ScanPlan(config=cfg, warps_per_cta=warps, segments=1))
+                    largest = warps
+                    break
+                except ms.MambaScanError as e:
+                    assert e.status == 2
+            assert largest is not None, f"config {cfg} runs at no CTA size"
+            shapes = [(w, s) for w in sorted({2, largest}) for s in (1, 3)]
+        for warps, segments in shapes:
+            plan = ms.ScanPlan(config=cfg, warps_per_cta=warps, segments=segments)
+            y, hT = ms.scan_fwd(**dev, plan=plan)
+            torch.cuda.synchronize()
+            tag = f"config {cfg} (kind {kind}, lanes {lanes}, states {states}), {warps} warps, {segments} segments"
+            assert rel_err(to_host64(y), yr) <= TOL[dtype], tag
+            assert rel_err(to_host64(hT), hr) <= TOL[dtype], tag
+
+
+def _sequential_configs():
+    return [(cfg, lanes, warps) for cfg, lanes, _, warps, kind in _ms().scan_configs() if kind == 1]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("batch,dim,N,L,offset", [
+    (1, 3, 16, 1, 0), (2, 37, 16, 33, 0), (2, 130, 16, 1000, 0), (3, 20, 5, 97, 0),
+    (1, 64, 1, 64, 0), (2, 70, 16, 255, 1), (1, 9, 8, 31, 3),
+])
+def test_sequential_kernels(dtype, batch, dim, N, L, offset):
+    """Every sequential configuration on ragged rows, lengths and state sizes,
+    with an initial state, and (offset > 0) rows that are not 16-byte aligned
+    (the scalar load path), against the oracle."""
+    import torch
+    ms = _ms()
+    inp = make_scan_inputs(LAYER, batch=batch, dim=dim, dstate=N, seqlen=L + offset, dtype=dtype,
+                           seed=1500 + dim + L + N)
+    dev = device_inputs(inp)
+    if offset:   # drop the first `offset` steps of every row: views with misaligned row starts
+        for k in ("u", "delta", "z", "B", "C"):
+            dev[k] = dev[k][..., offset:]
+        for k in ("u", "delta", "z", "B", "C"):
+            inp[k] = np.ascontiguousarray(inp[k][..., offset:])
+        inp["seqlen"] = L
+    h0 = np.random.default_rng(dim).normal(size=(batch, dim, N)).astype(np.float32)
+    yr, hr = oracle_scan(inp, h0=h0.reshape(-1, N))
+    for cfg, lanes, warps in _sequential_configs():
+        plan = ms.ScanPlan(config=cfg, warps_per_cta=warps, segments=1)
+        y, hT = ms.scan_fwd(**dev, plan=plan, initial_state=torch.from_numpy(h0).cuda())
+        torch.cuda.synchronize()
+        tag = f"config {cfg} (lanes per row {lanes})"
+        assert rel_err(to_host64(y), yr) <= TOL[dtype], tag
+        assert rel_err(to_host64(hT), hr) <= TOL[dtype], tag
 
 
 def test_plan_validation():
@@ -213,7 +256,7 @@ def test_plan_validation():
     inp = make_scan_inputs(LAYER, batch=1, dim=8, dstate=4, seqlen=128, seed=1200)
     dev = device_inputs(inp)
     configs = ms.scan_configs()
-    pipelined = [c for c, _, states, _ in configs if states == 0]
+    pipelined = [c for c, _, states, _, kind in configs if states == 0 and kind == 0]
     for plan in [ms.ScanPlan(config=len(configs), warps_per_cta=4, segments=1),
                  ms.ScanPlan(config=0, warps_per_cta=1, segments=1),
                  ms.ScanPlan(config=0, warps_per_cta=4, segments=0),
