@@ -42,6 +42,10 @@ ROTATE = 3  # input sets cycled through so that each step reads inputs not resid
 # transcendental results 16, FP32 lanes 128.
 SMS_B200 = 148
 MUFU_PER_CLK = 16
+# DRAM bytes (read + write) per launch from an ncu capture of the named kernel
+# on the named workload (profiles/ holds the summary); any other kernel or
+# workload reports traffic null.
+NCU_TRAFFIC = {("mamba130m_layer", "rec_kernel<bf16, 4>"): 152191744 + 31394560}
 FP32_PER_CLK = 128
 
 
@@ -321,6 +325,12 @@ def run_ours(args, dist: Dist):
                                     D=params["D"], z=s.get("z"), delta_bias=params["delta_bias"],
                                     final_state=hT) for s in sets]
     ws_bytes = ms.scan_workspace_size(args_list[0])
+    plan = ms.scan_plan(args_list[0])
+    kind = {c: k for c, _, _, _, k in ms.scan_configs()}[plan.config]
+    kernel_name = (f"rec_kernel<{'bf16' if w.dtype == 'bf16' else 'f32'}, {plan.lanes}> (sequential, "
+                   f"warp-specialised, {plan.lanes} lanes per row)" if kind == 1 else
+                   f"scan_kernel (chunked, config {plan.config}, {plan.warps_per_cta} warps, "
+                   f"{plan.segments} segments)")
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     lib = ms.load_library()
     import ctypes
@@ -401,8 +411,8 @@ def run_ours(args, dist: Dist):
                 "fp32": counts["fp32"] / fp32_peak}
     roofline = {
         "bound": "alu", "unit": "Tmufu/s", "achieved": achieved_mufu / 1e12, "peak": mufu_peak / 1e12,
-        "frac": achieved_mufu / mufu_peak, "traffic": None,
-        "kernel": "scan_kernel (selective scan forward, fused)",
+        "frac": achieved_mufu / mufu_peak, "traffic": NCU_TRAFFIC.get((w.name, kernel_name.split(" (")[0])),
+        "kernel": kernel_name,
         "peak_note": f"MUFU: {SMS_B200} SMs x {MUFU_PER_CLK}/clk x {sm_mhz:.0f} MHz (nominal max clock)",
         "algorithmic_per_launch": counts,
         "hbm": {"achieved_gbs": counts["bytes"] / t_kernel / 1e9, "peak_gbs": peaks["hbm_gbs"],

@@ -24,16 +24,16 @@
 //    one batch entry and step their states through chunks of 16 steps,
 //    leaving each lane's partial readout sum_{own n} C_t[n] h_t[n] in shared
 //    memory;
-//  * 2 I/O warps prepare chunk c + 1 while the recurrence runs chunk c --
-//    delta = softplus(delta_raw + bias) and delta u stored as (delta, delta,
-//    delta u, delta u), the operand pairs of the packed multiplies, and the
-//    chunk's B and C tiles (shared by all rows) widened to float32 -- and
-//    finish chunk c - 1: sum the LPR partials, add D u, apply the SiLU gate
-//    and store y. Their global loads run one chunk ahead.
-// The two groups hand the double-buffered tiles over through named hardware
-// barriers (bar.arrive by the producer, bar.sync by the consumer; no spin
-// loops). Steps past the end of the sequence get delta = 0 (Abar = 1, Bbar u
-// = 0): the state reaches the final-state output unchanged.
+//  * 2 I/O warps run up to two chunks ahead of the recurrence, preparing
+//    chunk c -- delta = softplus(delta_raw + bias) and delta u, stored per
+//    step pair, and the chunk's B and C tiles (shared by all rows) widened to
+//    float32 -- and finishing chunk c - 2: sum the LPR partials, add D u,
+//    apply the SiLU gate and store y. Their raw inputs arrive through a
+//    cp.async ring three chunks ahead.
+// The two groups hand the tiles over through three stage buffers and named
+// hardware barriers (bar.arrive by the producer, bar.sync by the consumer; no
+// spin loops). Steps past the end of the sequence get delta = 0 (Abar = 1,
+// Bbar u = 0): the state reaches the final-state output unchanged.
 #include <mutex>
 #include <type_traits>
 
@@ -48,39 +48,53 @@ constexpr int kIoThreads = 64;      // 2 I/O warps
 constexpr int kThreads = kScanThreads + kIoThreads;
 constexpr int kSteps = 16;          // time steps per chunk
 constexpr int kStates = 16;         // states per row (smaller dstate is zero-padded)
+constexpr int kTileStages = 3;      // step/readout tile buffers between the two warp groups
 
-// Shared-memory layout of one of the two stages, in bytes. The step tile holds
-// one float4 per (row, step), with one float4 of padding after each I/O
-// thread's piece of IP steps; the readout tile holds, per row and lane, the
-// lane's partial readout of every step ([row][lane][step], YQ floats per lane
-// and YR per row). The paddings keep the recurrence warps' loads and stores
-// and the I/O warps' tile stores free of bank conflicts.
+// Shared-memory layout of one of the kTileStages stages, in bytes. The step tile holds
+// one float4 per (row, step pair): (delta_t, delta_t u_t, delta_t+1,
+// delta_t+1 u_t+1), XR float4 per row (odd, so that the 8 rows a quarter-warp
+// reads or writes fall on distinct banks). The readout tile holds, per row
+// and state group, the group's partial readout of every step ([row][group]
+// [step], YQ floats per group and YR per row). The B and C tiles are
+// [step][state] float32.
+//
+// Lane mapping of the recurrence warps. A 128-bit shared load costs two
+// wavefronts when every quarter-warp touches at most two distinct 16-byte
+// addresses and four otherwise (measured on B200), so for LPR = 2 and 4 the
+// lanes are group-major -- lane l of warp w takes row w (32 / LPR) + l %
+// (32 / LPR) and state group l / (32 / LPR): a quarter-warp then reads one
+// B/C address per step. For LPR = 8 and 16 (row-major, lane l takes row
+// (32 w + l) / LPR and group l % LPR) a quarter-warp covers at most two rows.
 template <int LPR> struct Shape {
     static constexpr int NPL = kStates / LPR;           // states per lane
     static constexpr int R = kScanThreads / LPR;        // rows per CTA
     static constexpr int IPR = LPR / 2;                 // I/O threads per row
     static constexpr int IP = kSteps / IPR;             // steps per I/O thread
-    static constexpr int XR = LPR == 2 ? 17 : LPR == 4 ? 18 : LPR == 8 ? 20 : 24;   // float4 per row
-    static constexpr int YQ = 20;
-    static constexpr int YR = LPR == 2 ? 40 : LPR == 4 ? 80 : LPR == 8 ? 176 : 336;
+    static constexpr bool GROUP_MAJOR = LPR <= 4;
+    static constexpr int XR = kSteps / 2 + 1;           // float4 per row of the step tile
+    static constexpr int YQ = LPR <= 4 ? 16 : 20;
+    static constexpr int YR = LPR == 2 ? 36 : LPR == 4 ? 68 : LPR == 8 ? 168 : 328;
     static constexpr int X_OFF = 0;
     static constexpr int Y_OFF = X_OFF + R * XR * 16;
     static constexpr int B_OFF = Y_OFF + R * YR * 4;
     static constexpr int C_OFF = B_OFF + kSteps * kStates * 4;
     static constexpr int STAGE = C_OFF + kSteps * kStates * 4;
-    static constexpr int BYTES = 2 * STAGE;
+    static constexpr int BYTES = kTileStages * STAGE;
     // CTAs per SM the launch bounds provide registers for
     static constexpr int MINB = LPR == 2 ? 2 : LPR == 4 ? 3 : LPR == 8 ? 4 : 5;
     static_assert(R * IPR == kIoThreads, "the I/O threads cover the rows");
-    static_assert(XR >= kSteps + IPR, "step tile row holds the padded pieces");
+    static_assert(XR % 2 == 1, "odd row stride");
     static_assert(YQ >= kSteps && YQ % 4 == 0 && YR >= LPR * YQ && YR % 4 == 0, "readout tile");
 };
 
-// The I/O warps' ring of raw inputs in shared memory, after the two stages:
-// kRawStages chunks in flight, each I/O thread filling and reading only its
-// own 16-byte slots (its u, delta and z pieces of PB bytes each, then its B/C
-// pieces), stored slot-major so that a warp's slot accesses are contiguous.
-constexpr int kRawStages = 4;   // a power of two
+// The I/O warps' ring of raw inputs in shared memory, after the tile stages.
+// It holds every chunk from the oldest one still to be finished (its u and z
+// feed the readout) to the newest one in flight, kRawAhead chunks ahead of the
+// one being widened. Each I/O thread fills and reads only its own 16-byte
+// slots (its u, delta and z pieces of PB bytes each, then its B/C pieces),
+// stored slot-major so that a warp's slot accesses are contiguous.
+constexpr int kRawStages = 5;
+constexpr int kRawAhead = kRawStages - kTileStages + 1;
 template <typename T, int LPR> struct Raw {
     static constexpr int EB = static_cast<int>(sizeof(T));
     static constexpr int PB = Shape<LPR>::IP * EB;                   // bytes of one u/delta/z piece
@@ -96,15 +110,17 @@ template <typename T, int LPR> struct Raw {
 };
 
 // Named barriers (0 is __syncthreads): the producer arrives, the consumer
-// waits; kThreads threads complete each phase.
+// waits; kThreads threads complete each phase. 4 kTileStages + 1 <= 16.
 //   XF(s): stage s's step and B/C tiles are ready       (I/O -> recurrence)
 //   XE(s): stage s's step and B/C tiles may be rewritten (recurrence -> I/O)
 //   YF(s): stage s's readout partials are ready          (recurrence -> I/O)
 //   YE(s): stage s's readout tile may be rewritten       (I/O -> recurrence)
 __device__ __forceinline__ int bar_xf(int s) { return 1 + s; }
-__device__ __forceinline__ int bar_xe(int s) { return 3 + s; }
-__device__ __forceinline__ int bar_yf(int s) { return 5 + s; }
-__device__ __forceinline__ int bar_ye(int s) { return 7 + s; }
+__device__ __forceinline__ int bar_xe(int s) { return 1 + kTileStages + s; }
+__device__ __forceinline__ int bar_yf(int s) { return 1 + 2 * kTileStages + s; }
+__device__ __forceinline__ int bar_ye(int s) { return 1 + 3 * kTileStages + s; }
+static_assert(4 * kTileStages + 1 <= 16, "named barriers per CTA");
+__device__ __forceinline__ int next_stage(int s, int n) { return s + 1 == n ? 0 : s + 1; }
 __device__ __forceinline__ void bar_wait(int id) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(kThreads) : "memory");
 }
@@ -112,8 +128,8 @@ __device__ __forceinline__ void bar_signal(int id) {
     asm volatile("bar.arrive %0, %1;" ::"r"(id), "n"(kThreads) : "memory");
 }
 
-// One step's operands of a lane: (delta, delta, delta u, delta u) and the
-// lane's B_t and C_t entries as pairs.
+// One step's B_t and C_t entries of a lane, as the pairs the packed
+// instructions take.
 template <int NPL> struct StepIn {
     float2 b[NPL > 1 ? NPL / 2 : 1], c[NPL > 1 ? NPL / 2 : 1];
 };
@@ -232,7 +248,10 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
     using S = Shape<LPR>;
     constexpr int NPL = S::NPL, R = S::R, IP = S::IP;
     constexpr int NP = NPL > 1 ? NPL / 2 : 1;
-    const int r = tid / LPR, q = tid % LPR;
+    constexpr int RW = 32 / LPR;   // rows per warp
+    const int lane = tid & 31, warp = tid >> 5;
+    const int r = S::GROUP_MAJOR ? warp * RW + lane % RW : tid / LPR;
+    const int q = S::GROUP_MAJOR ? lane / RW : tid % LPR;
     const int64_t b = blockIdx.y;
     const int64_t d = static_cast<int64_t>(blockIdx.x) * R + r;
     const bool ok = d < p.dim;
@@ -259,54 +278,52 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
         hp[j] = f2(h2[0], h2[1]);
     }
 
-    for (int64_t c = 0; c < nchunks; ++c) {
-        const int s = static_cast<int>(c & 1);
+    int s = 0;   // tile stage of chunk c
+    for (int64_t c = 0; c < nchunks; ++c, s = next_stage(s, kTileStages)) {
         unsigned char *st = smem + s * S::STAGE;
         const float4 *xrow = reinterpret_cast<const float4 *>(st + S::X_OFF) + r * S::XR;
         float *yl = reinterpret_cast<float *>(st + S::Y_OFF) + r * S::YR + q * S::YQ;
         const float *Bl = reinterpret_cast<const float *>(st + S::B_OFF) + q * NPL;
         const float *Cl = reinterpret_cast<const float *>(st + S::C_OFF) + q * NPL;
         bar_wait(bar_xf(s));
-        if (c >= 2) bar_wait(bar_ye(s));
+        if (c >= kTileStages) bar_wait(bar_ye(s));
 
-        // Software pipelined over the chunk: the step tile is read two steps
+        // Software pipelined over the chunk: step pairs are read one pair
         // ahead, B and C one step ahead, and the ex2 of step t + 1 is issued
         // before the FMAs of step t, so neither shared-memory nor MUFU latency
         // sits on the state's dependency chain. Partial readouts leave in
         // float4 stores every 4 steps.
-        auto xat = [&](int t) { return xrow[t + t / IP]; };
-        auto decay = [&](const float4 &x, float2 (&a)[NP]) {
+        auto decay = [&](float dt, float2 (&a)[NP]) {
             if constexpr (NPL == 1) {
-                a[0] = f2(ex2_approx(x.x * ap[0].x), 0.f);
+                a[0] = f2(ex2_approx(dt * ap[0].x), 0.f);
             } else {
 #pragma unroll
-                for (int j = 0; j < NP; ++j) a[j] = ex2x2(mul2(f2(x.x, x.y), ap[j]));
+                for (int j = 0; j < NP; ++j) a[j] = ex2x2(mul2(f2(dt, dt), ap[j]));
             }
         };
-        float4 x0 = xat(0), x1 = xat(1);
+        float4 xa = xrow[0], xb = xrow[1];   // steps (0, 1) and (2, 3)
         float2 acur[NP];
-        decay(x0, acur);
+        decay(xa.x, acur);
         StepIn<NPL> cur = load_bc_step<NPL>(Bl, Cl);
         float outs[4];
 #pragma unroll
         for (int t = 0; t < kSteps; ++t) {
-            float4 x2 = x1;
-            if (t + 2 < kSteps) x2 = xat(t + 2);
+            const bool odd = t & 1;
             StepIn<NPL> nxt = cur;
             float2 anxt[NP];
             if (t + 1 < kSteps) {
                 nxt = load_bc_step<NPL>(Bl + (t + 1) * kStates, Cl + (t + 1) * kStates);
-                decay(x1, anxt);
+                decay(odd ? xb.x : xa.z, anxt);
             }
+            const float du = odd ? xa.w : xa.y;
             if constexpr (NPL == 1) {
-                hp[0].x = fmaf(acur[0].x, hp[0].x, x0.z * cur.b[0].x);
+                hp[0].x = fmaf(acur[0].x, hp[0].x, du * cur.b[0].x);
                 outs[t & 3] = cur.c[0].x * hp[0].x;
             } else {
-                const float2 du = f2(x0.z, x0.w);
                 float2 acc;
 #pragma unroll
                 for (int j = 0; j < NP; ++j) {
-                    hp[j] = fma2(acur[j], hp[j], mul2(du, cur.b[j]));
+                    hp[j] = fma2(acur[j], hp[j], mul2(f2(du, du), cur.b[j]));
                     acc = j == 0 ? mul2(cur.c[j], hp[j]) : fma2(cur.c[j], hp[j], acc);
                 }
                 outs[t & 3] = acc.x + acc.y;
@@ -314,14 +331,16 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
             if ((t & 3) == 3)
                 *reinterpret_cast<float4 *>(yl + t - 3) = make_float4(outs[0], outs[1], outs[2], outs[3]);
             if (t + 1 < kSteps) {
-                x0 = x1;
-                x1 = x2;
                 cur = nxt;
 #pragma unroll
                 for (int j = 0; j < NP; ++j) acur[j] = anxt[j];
+                if (odd) {   // the pair (t + 1, t + 2) becomes current; fetch (t + 3, t + 4)
+                    xa = xb;
+                    if (t + 3 < kSteps) xb = xrow[(t + 3) / 2];
+                }
             }
         }
-        if (c + 2 < nchunks) bar_signal(bar_xe(s));
+        if (c + kTileStages < nchunks) bar_signal(bar_xe(s));
         bar_signal(bar_yf(s));
     }
 
@@ -336,9 +355,9 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
 
 // The I/O warps: thread (r, k) handles steps k IP .. k IP + IP - 1 of row r in
 // every chunk, plus BC_PER 16-byte pieces of the chunk's B/C tiles. Its raw
-// inputs travel through the ring kRawStages - 1 chunks ahead of use
-// (cp.async on the aligned path, plain loads otherwise); a thread waits only
-// for its own copies, so the ring needs no barrier.
+// inputs travel through the ring kRawAhead chunks ahead of use (cp.async on
+// the aligned path, plain loads otherwise); a thread waits only for its own
+// copies, so the ring needs no barrier.
 template <typename T, int LPR, bool VEC>
 __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem, int i) {
     using S = Shape<LPR>;
@@ -382,12 +401,10 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     }
 
     unsigned char *ring = smem + RW::OFF;
-    auto slot = [&](int64_t c, int sl) {
-        return ring + static_cast<int>(c & (kRawStages - 1)) * RW::STAGE + (sl * kIoThreads + i) * 16;
-    };
+    auto slot = [&](int rs, int sl) { return ring + rs * RW::STAGE + (sl * kIoThreads + i) * 16; };
 
-    // Issue the copies of chunk c's raw inputs into its ring stage.
-    auto stage_chunk = [&](int64_t c) {
+    // Issue the copies of chunk c's raw inputs into ring stage rs.
+    auto stage_chunk = [&](int64_t c, int rs) {
         const int64_t t0 = c * kSteps;
         const bool full = t0 + kSteps <= L;
         const int valid = full ? IP : static_cast<int>(min64(IP, max64(0, L - (t0 + tk))));
@@ -402,49 +419,50 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
                     const int bytes = have < 0 ? 0 : (have > (PB < 16 ? PB : 16) ? (PB < 16 ? PB : 16) : have);
                     const void *g = bytes > 0 ? static_cast<const void *>(reinterpret_cast<const unsigned char *>(src) + sl * 16)
                                               : static_cast<const void *>(src_row[tsr]);
-                    if constexpr (PB >= 16) cp_async16(slot(c, tsr * PS + sl), g, bytes);
-                    else cp_async_small<PB>(slot(c, tsr * PS + sl), g, bytes);
+                    if constexpr (PB >= 16) cp_async16(slot(rs, tsr * PS + sl), g, bytes);
+                    else cp_async_small<PB>(slot(rs, tsr * PS + sl), g, bytes);
                 }
             } else {
                 Piece<T, IP> pc;
                 load_piece<T, IP, false>(pc, src, valid);
 #pragma unroll
                 for (int w = 0; w < Piece<T, IP>::W; ++w)
-                    reinterpret_cast<uint32_t *>(slot(c, tsr * PS + w / 4))[w % 4] = pc.w[w];
+                    reinterpret_cast<uint32_t *>(slot(rs, tsr * PS + w / 4))[w % 4] = pc.w[w];
             }
         }
 #pragma unroll
         for (int j = 0; j < BC_PER; ++j) {
             const int vb = bc_live[j] ? (full ? VE : static_cast<int>(min64(VE, max64(0, L - (t0 + bc_t[j]))))) : 0;
             if constexpr (VEC) {
-                cp_async16(slot(c, 3 * PS + j), vb > 0 ? static_cast<const void *>(bc_src[j] + t0)
+                cp_async16(slot(rs, 3 * PS + j), vb > 0 ? static_cast<const void *>(bc_src[j] + t0)
                                                        : static_cast<const void *>(bc_src[j]), vb * EB);
             } else {
                 Piece<T, VE> pc;
                 load_piece<T, VE, false>(pc, bc_src[j] + t0, vb);
-                *reinterpret_cast<uint4 *>(slot(c, 3 * PS + j)) = make_uint4(pc.w[0], pc.w[1], pc.w[2], pc.w[3]);
+                *reinterpret_cast<uint4 *>(slot(rs, 3 * PS + j)) = make_uint4(pc.w[0], pc.w[1], pc.w[2], pc.w[3]);
             }
         }
     };
-    // The thread's piece of tensor tsr of chunk c, from the ring.
-    auto ring_piece = [&](int64_t c, int tsr) {
+    // The thread's piece of tensor tsr from ring stage rs.
+    auto ring_piece = [&](int rs, int tsr) {
         Piece<T, IP> pc;
         if constexpr (PB == 4) {
-            pc.w[0] = *reinterpret_cast<const uint32_t *>(slot(c, tsr * PS));
+            pc.w[0] = *reinterpret_cast<const uint32_t *>(slot(rs, tsr * PS));
         } else if constexpr (PB == 8) {
-            const uint2 v = *reinterpret_cast<const uint2 *>(slot(c, tsr * PS));
+            const uint2 v = *reinterpret_cast<const uint2 *>(slot(rs, tsr * PS));
             pc.w[0] = v.x; pc.w[1] = v.y;
         } else {
 #pragma unroll
             for (int sl = 0; sl < PS; ++sl) {
-                const uint4 v = *reinterpret_cast<const uint4 *>(slot(c, tsr * PS + sl));
+                const uint4 v = *reinterpret_cast<const uint4 *>(slot(rs, tsr * PS + sl));
                 pc.w[4 * sl] = v.x; pc.w[4 * sl + 1] = v.y; pc.w[4 * sl + 2] = v.z; pc.w[4 * sl + 3] = v.w;
             }
         }
         return pc;
     };
-    // Readout of chunk c from stage s: partial sums + D u, gate, store.
-    auto finish = [&](int64_t c, int s) {
+    // Readout of chunk c from tile stage s (u, z from ring stage rs): partial
+    // sums + D u, gate, store.
+    auto finish = [&](int64_t c, int s, int rs) {
         const int64_t cnt = L - (c * kSteps + tk);
         if (!ok || cnt <= 0) return;
         const float *yp = reinterpret_cast<const float *>(smem + s * S::STAGE + S::Y_OFF) + r * S::YR + tk;
@@ -464,10 +482,10 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
                 }
             }
         }
-        const Piece<T, IP> u = ring_piece(c, 0);
+        const Piece<T, IP> u = ring_piece(rs, 0);
         float outv[IP];
         if (has_z) {
-            const Piece<T, IP> z = ring_piece(c, 2);
+            const Piece<T, IP> z = ring_piece(rs, 2);
 #pragma unroll
             for (int e = 0; e < IP; e += 2) {
                 const float2 yv = fma2(f2(Dd, Dd), f2(elem(u, e), elem(u, e + 1)), sum[e / 2]);
@@ -485,11 +503,12 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
         }
         store_piece<T, IP, VEC>(yrow + c * kSteps, outv, cnt);
     };
-    // Chunk c's step tile (delta, delta, delta u, delta u) and B/C tiles into stage s.
-    auto widen = [&](int64_t c, int s) {
+    // Chunk c's step tile (step pairs of delta, delta u) and B/C tiles from
+    // ring stage rs into tile stage s.
+    auto widen = [&](int64_t c, int s, int rs) {
         unsigned char *st = smem + s * S::STAGE;
-        float4 *xrow = reinterpret_cast<float4 *>(st + S::X_OFF) + r * S::XR + tk + k;
-        const Piece<T, IP> u = ring_piece(c, 0), dl = ring_piece(c, 1);
+        float4 *xrow = reinterpret_cast<float4 *>(st + S::X_OFF) + r * S::XR + tk / 2;
+        const Piece<T, IP> u = ring_piece(rs, 0), dl = ring_piece(rs, 1);
         const bool full = (c + 1) * kSteps <= L;
         const int64_t cnt = L - (c * kSteps + tk);
 #pragma unroll
@@ -501,12 +520,11 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
                 if (e + 1 >= cnt) v.y = 0.f;
             }
             const float2 du = mul2(v, f2(elem(u, e), elem(u, e + 1)));
-            xrow[e] = make_float4(v.x, v.x, du.x, du.x);
-            xrow[e + 1] = make_float4(v.y, v.y, du.y, du.y);
+            xrow[e / 2] = make_float4(v.x, du.x, v.y, du.y);
         }
 #pragma unroll
         for (int j = 0; j < BC_PER; ++j) {
-            const uint4 w = *reinterpret_cast<const uint4 *>(slot(c, 3 * PS + j));
+            const uint4 w = *reinterpret_cast<const uint4 *>(slot(rs, 3 * PS + j));
             Piece<T, VE> pc;
             pc.w[0] = w.x; pc.w[1] = w.y; pc.w[2] = w.z; pc.w[3] = w.w;
             float *dst = reinterpret_cast<float *>(st + bc_off[j]);
@@ -515,32 +533,43 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
         }
     };
 
-    // Prologue: chunks 0 .. kRawStages - 2 in flight (one commit group per
-    // chunk, empty past the end, so that the group count stays uniform).
+    // Chunk c is widened in iteration c, finished in iteration c + kTileStages - 1
+    // (or after the loop), and its raw inputs are staged kRawAhead iterations
+    // before its widening into the ring stage that the chunk finished in the
+    // same iteration releases. Prologue: chunks 0 .. kRawAhead - 1 in flight,
+    // one commit group per chunk (empty past the end: the count stays uniform).
 #pragma unroll
-    for (int c0 = 0; c0 < kRawStages - 1; ++c0) {
-        if (c0 < nchunks) stage_chunk(c0);
+    for (int c0 = 0; c0 < kRawAhead; ++c0) {
+        if (c0 < nchunks) stage_chunk(c0, c0);
         cp_async_commit();
     }
+    int s = 0, rs = 0;                    // tile and ring stage of chunk c
+    int sf = 0, rf = 0;                   // tile and ring stage of the next chunk to finish
+    int ra = kRawAhead % kRawStages;      // ring stage of chunk c + kRawAhead
     for (int64_t c = 0; c < nchunks; ++c) {
-        const int s = static_cast<int>(c & 1);
-        cp_async_wait<kRawStages - 2>();   // chunk c's copies have landed
-        if (c >= 2) bar_wait(bar_xe(s));
-        widen(c, s);
+        cp_async_wait<kRawAhead - 1>();   // chunk c's copies have landed
+        if (c >= kTileStages) bar_wait(bar_xe(s));
+        widen(c, s, rs);
         bar_signal(bar_xf(s));
-        if (c >= 1) {
-            bar_wait(bar_yf(s ^ 1));
-            finish(c - 1, s ^ 1);
-            if (c + 1 < nchunks) bar_signal(bar_ye(s ^ 1));
+        const int64_t j = c - (kTileStages - 1);
+        if (j >= 0) {
+            bar_wait(bar_yf(sf));
+            finish(j, sf, rf);
+            if (j + kTileStages < nchunks) bar_signal(bar_ye(sf));
+            sf = next_stage(sf, kTileStages);
+            rf = next_stage(rf, kRawStages);
         }
-        // chunk c + kRawStages - 1 reuses the ring stage that chunk c - 1 just released
-        if (c + kRawStages - 1 < nchunks) stage_chunk(c + kRawStages - 1);
+        if (c + kRawAhead < nchunks) stage_chunk(c + kRawAhead, ra);
         cp_async_commit();
+        s = next_stage(s, kTileStages);
+        rs = next_stage(rs, kRawStages);
+        ra = next_stage(ra, kRawStages);
     }
-    if (nchunks > 0) {
-        const int s = static_cast<int>((nchunks - 1) & 1);
-        bar_wait(bar_yf(s));
-        finish(nchunks - 1, s);
+    for (int64_t j = max64(nchunks - (kTileStages - 1), 0); j < nchunks; ++j) {
+        bar_wait(bar_yf(sf));
+        finish(j, sf, rf);
+        sf = next_stage(sf, kTileStages);
+        rf = next_stage(rf, kRawStages);
     }
     cp_async_wait<0>();
 }
