@@ -48,6 +48,12 @@ def _bind(path: str):
     lib.s6_oracle_state_update.restype = ip
     lib.s6_oracle_state_update.argtypes = [i64, i64, i64, ip, vp, vp, vp, vp, vp, vp, vp, vp,
                                            vp, ip, vp, i64, vp, ip]
+    lib.s6_oracle_conv_scan.restype = ip
+    lib.s6_oracle_conv_scan.argtypes = [i64, i64, i64, i64, ip, vp, vp, vp, ip, ip, vp, vp, vp, vp,
+                                        vp, vp, vp, ip, vp, i64, vp, vp, vp, vp, ip]
+    lib.s6_oracle_conv_state_update.restype = ip
+    lib.s6_oracle_conv_state_update.argtypes = [i64, i64, i64, ip, vp, vp, vp, vp, vp, ip, ip, vp, vp,
+                                                vp, vp, vp, vp, vp, ip, vp, i64, vp, ip]
     lib.s6_oracle_max_threads.restype = ip
     lib.s6_oracle_max_threads.argtypes = []
     return lib
@@ -157,6 +163,87 @@ def state_update(*, state, x, delta, A, B, C, D=None, z=None, delta_bias=None,
     return y.reshape(batch, dim) if rows is None else y
 
 
+def conv_scan(*, x, conv_w, conv_b=None, conv_silu=True, delta, A, B, C, D=None, z=None,
+              delta_bias=None, delta_softplus=True, dtype="f32", rows=None, h0=None,
+              return_u=False, threads: int = 0, _lib_override=None):
+    """Causal depthwise convolution prologue + selective scan, in fp64.
+
+    ``x`` (batch, dim, L) is the convolution input (float32 or bf16 bits);
+    ``conv_w`` (dim, width) and ``conv_b`` (dim,) float32. The scan input is
+    u = silu(conv(x)) (or conv(x) with ``conv_silu=False``). Other arguments as
+    :func:`scan`. Returns ``(y, h)``, or ``(y, h, u)`` with ``return_u``.
+    """
+    dt = _DTYPES[dtype]
+    x, delta, B, C, z = (_in(a, dt) for a in (x, delta, B, C, z))
+    A, D, delta_bias, conv_w, conv_b = _f32(A), _f32(D), _f32(delta_bias), _f32(conv_w), _f32(conv_b)
+    batch, dim, L = x.shape
+    dstate = B.shape[1]
+    width = conv_w.shape[1]
+    if conv_w.shape != (dim, width) or (conv_b is not None and conv_b.shape != (dim,)):
+        raise ValueError("conv_w must be (dim, width) and conv_b (dim,)")
+    if delta.shape != x.shape or (z is not None and z.shape != x.shape):
+        raise ValueError("x, delta and z must share one (batch, dim, L) shape")
+    if B.shape != (batch, dstate, L) or C.shape != B.shape or A.shape != (dim, dstate):
+        raise ValueError("B, C must be (batch, dstate, L) and A (dim, dstate)")
+    if rows is None:
+        n_rows, rows_arr = batch * dim, None
+    else:
+        rows_arr = np.ascontiguousarray(rows, dtype=np.int64)
+        n_rows = rows_arr.size
+    h0_arr = None if h0 is None else np.ascontiguousarray(h0, dtype=np.float64).reshape(n_rows, dstate)
+    y = np.empty((n_rows, L), np.float64)
+    h = np.empty((n_rows, dstate), np.float64)
+    u = np.empty((n_rows, L), np.float64) if return_u else None
+    lib = _lib_override or _load()
+    rc = lib.s6_oracle_conv_scan(batch, dim, dstate, L, dt, _ptr(x), _ptr(conv_w), _ptr(conv_b), width,
+                                 int(bool(conv_silu)), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                 _ptr(z), _ptr(delta_bias), int(bool(delta_softplus)), _ptr(rows_arr),
+                                 n_rows, _ptr(h0_arr), _ptr(y), _ptr(h), _ptr(u), int(threads))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    if rows is None:
+        out = (y.reshape(batch, dim, L), h.reshape(batch, dim, dstate))
+        return out + (u.reshape(batch, dim, L),) if return_u else out
+    return (y, h, u) if return_u else (y, h)
+
+
+def conv_state_update(*, state, conv_state, x, conv_w, conv_b=None, conv_silu=True, delta, A, B, C,
+                      D=None, z=None, delta_bias=None, delta_softplus=True, dtype="f32", rows=None,
+                      threads: int = 0, _lib_override=None):
+    """One decode step with the convolution prologue, in fp64.
+
+    ``conv_state``: float64 (batch, dim, width) (or (n_rows, width)), the last
+    ``width`` convolution inputs oldest first, updated in place; ``state`` as
+    :func:`state_update`. Returns y (batch, dim) float64 (or (n_rows,)).
+    """
+    dt = _DTYPES[dtype]
+    x, delta, B, C, z = (_in(a, dt) for a in (x, delta, B, C, z))
+    A, D, delta_bias, conv_w, conv_b = _f32(A), _f32(D), _f32(delta_bias), _f32(conv_w), _f32(conv_b)
+    batch, dim = x.shape
+    dstate = B.shape[1]
+    width = conv_w.shape[1]
+    for a in (state, conv_state):
+        if not (isinstance(a, np.ndarray) and a.dtype == np.float64 and a.flags.c_contiguous):
+            raise TypeError("state and conv_state must be C-contiguous float64 arrays (updated in place)")
+    if rows is None:
+        n_rows, rows_arr = batch * dim, None
+    else:
+        rows_arr = np.ascontiguousarray(rows, dtype=np.int64)
+        n_rows = rows_arr.size
+    if state.size != n_rows * dstate or conv_state.size != n_rows * width:
+        raise ValueError("state or conv_state has the wrong size")
+    y = np.empty(n_rows, np.float64)
+    lib = _lib_override or _load()
+    rc = lib.s6_oracle_conv_state_update(batch, dim, dstate, dt, _ptr(state), _ptr(conv_state), _ptr(x),
+                                         _ptr(conv_w), _ptr(conv_b), width, int(bool(conv_silu)),
+                                         _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                                         _ptr(delta_bias), int(bool(delta_softplus)), _ptr(rows_arr),
+                                         n_rows, _ptr(y), int(threads))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return y.reshape(batch, dim) if rows is None else y
+
+
 class Variant:
     """The oracle's entry points bound to another build of the oracle source.
 
@@ -172,6 +259,12 @@ class Variant:
 
     def state_update(self, **kw):
         return state_update(_lib_override=self._lib, **kw)
+
+    def conv_scan(self, **kw):
+        return conv_scan(_lib_override=self._lib, **kw)
+
+    def conv_state_update(self, **kw):
+        return conv_state_update(_lib_override=self._lib, **kw)
 
 
 def compile_source(src_path: str, so_path: str) -> str:

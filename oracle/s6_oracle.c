@@ -45,9 +45,23 @@
  *
  * Inputs are decoded from exactly the values the GPU receives: float32, or
  * bfloat16 bit patterns widened to float32 (bits << 16), then to double.
+ *
+ * The convolution prologue (s6_oracle_conv_scan, s6_oracle_conv_state_update)
+ * follows "Notas sobre Mamba", section "O bloco Mamba": on the x branch, a
+ * short depthwise convolution and a SiLU come before the selective SSM, and
+ * "Mamba-2 e State Space Duality (SSD)" configures its width as d_conv = 4.
+ * The pages print no formula; the reading taken is the causal depthwise
+ * convolution of width K along t, one filter per channel d, with zero input
+ * before t = 0:
+ *
+ *   u[b,d,t] = silu( bias[d] + sum_{k=0}^{K-1} w[d,k] * x[b,d,t-(K-1)+k] )
+ *
+ * (w[d,K-1] weighs the current input). The decode form keeps the last K
+ * inputs of every row (oldest first) as its convolution state.
  */
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 #ifdef _OPENMP
 #include <omp.h>
@@ -81,14 +95,15 @@ static double silu(double v)
  * exit; y receives seqlen doubles.
  */
 static void scan_row(int64_t b, int64_t d, int64_t dim, int64_t dstate, int64_t seqlen,
-                     int dtype, const void *u, const void *delta, const float *A,
-                     const void *B, const void *C, const float *D, const void *z,
+                     int dtype, const void *u, const double *u_row, const void *delta,
+                     const float *A, const void *B, const void *C, const float *D, const void *z,
                      const float *delta_bias, int delta_softplus, double *h, double *y)
 {
     const int64_t row = b * dim + d;                 /* row of (batch, dim, L) */
     for (int64_t t = 0; t < seqlen; ++t) {
         const int64_t i = row * seqlen + t;
-        const double x = load_value(u, dtype, i);
+        /* the SSM input: the given u, or the row's convolution output */
+        const double x = u_row ? u_row[t] : load_value(u, dtype, i);
         double dt = load_value(delta, dtype, i);
         if (delta_bias)
             dt += (double)delta_bias[d];
@@ -152,7 +167,7 @@ int s6_oracle_scan(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, i
         double *h = h_out + r * dstate;
         for (int64_t n = 0; n < dstate; ++n)
             h[n] = h0 ? h0[r * dstate + n] : 0.0;
-        scan_row(b, d, dim, dstate, seqlen, dtype, u, delta, A, B, C, D, z, delta_bias,
+        scan_row(b, d, dim, dstate, seqlen, dtype, u, NULL, delta, A, B, C, D, z, delta_bias,
                  delta_softplus, h, y_out + r * seqlen);
     }
     return 0;
@@ -198,7 +213,130 @@ int s6_oracle_state_update(int64_t batch, int64_t dim, int64_t dstate, int dtype
         const int64_t b = row / dim, d = row % dim;
         /* With seqlen = 1 the (batch, dim, L) and (batch, N, L) layouts of the
          * scan are the (batch, dim) and (batch, N) layouts of one token. */
-        scan_row(b, d, dim, dstate, 1, dtype, x, delta, A, B, C, D, z, delta_bias,
+        scan_row(b, d, dim, dstate, 1, dtype, x, NULL, delta, A, B, C, D, z, delta_bias,
+                 delta_softplus, state + r * dstate, y_out + r);
+    }
+    return 0;
+}
+
+/*
+ * The convolution output of one row: u_row[t] = act(bias + sum_k w[k] *
+ * x[t-(K-1)+k]) with x = 0 before t = 0; act = SiLU when `conv_silu`.
+ */
+static void conv_row(int64_t row, int64_t seqlen, int dtype, const void *x, const float *w,
+                     double bias, int width, int conv_silu, double *u_row)
+{
+    for (int64_t t = 0; t < seqlen; ++t) {
+        double acc = bias;
+        for (int k = 0; k < width; ++k) {
+            const int64_t s = t - (width - 1) + k;
+            if (s >= 0)
+                acc += (double)w[k] * load_value(x, dtype, row * seqlen + s);
+        }
+        u_row[t] = conv_silu ? silu(acc) : acc;
+    }
+}
+
+/*
+ * Convolution prologue + selective scan: x (batch, dim, seqlen) of dtype
+ * `dtype` is convolved per channel with conv_w (dim, width) float32 and
+ * conv_b (dim) float32 or NULL, optionally passed through SiLU, and the result
+ * is the scan's input u. Everything else as s6_oracle_scan. u_out, when not
+ * NULL, receives the convolution output (n_rows, seqlen) doubles.
+ */
+int s6_oracle_conv_scan(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int dtype,
+                        const void *x, const float *conv_w, const float *conv_b, int width,
+                        int conv_silu, const void *delta, const float *A, const void *B,
+                        const void *C, const float *D, const void *z, const float *delta_bias,
+                        int delta_softplus, const int64_t *rows, int64_t n_rows,
+                        const double *h0, double *y_out, double *h_out, double *u_out,
+                        int nthreads)
+{
+    if (batch < 0 || dim < 0 || dstate < 0 || seqlen < 0 || width < 1)
+        return -1;
+    if (dtype != ORACLE_F32 && dtype != ORACLE_BF16)
+        return -1;
+    if (!rows)
+        n_rows = batch * dim;
+    if (n_rows > 0 && (!x || !conv_w || !delta || !A || !B || !C || !y_out || !h_out))
+        return -1;
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const int64_t row = rows ? rows[r] : r;
+        if (row < 0 || row >= batch * dim)
+            return -1;
+    }
+    int failed = 0;
+#ifdef _OPENMP
+    if (nthreads > 0)
+        omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const int64_t row = rows ? rows[r] : r;
+        const int64_t b = row / dim, d = row % dim;
+        double *u_row = u_out ? u_out + r * seqlen : (double *)malloc((size_t)(seqlen > 0 ? seqlen : 1) * sizeof(double));
+        if (!u_row) {
+            failed = 1;
+            continue;
+        }
+        conv_row(row, seqlen, dtype, x, conv_w + d * width, conv_b ? (double)conv_b[d] : 0.0, width,
+                 conv_silu, u_row);
+        double *h = h_out + r * dstate;
+        for (int64_t n = 0; n < dstate; ++n)
+            h[n] = h0 ? h0[r * dstate + n] : 0.0;
+        scan_row(b, d, dim, dstate, seqlen, dtype, NULL, u_row, delta, A, B, C, D, z, delta_bias,
+                 delta_softplus, h, y_out + r * seqlen);
+        if (!u_out)
+            free(u_row);
+    }
+    return failed ? -1 : 0;
+}
+
+/*
+ * Single-token decode step with the convolution prologue. conv_state holds,
+ * per row, the last `width` convolution inputs (oldest first) as doubles; the
+ * step drops the oldest, appends x, computes u = act(bias + sum_k w[k] *
+ * conv_state[k]) and then runs s6_oracle_state_update's body with u as input.
+ * conv_state is (n_rows, width), state (n_rows, dstate), y_out (n_rows).
+ */
+int s6_oracle_conv_state_update(int64_t batch, int64_t dim, int64_t dstate, int dtype,
+                                double *state, double *conv_state, const void *x,
+                                const float *conv_w, const float *conv_b, int width,
+                                int conv_silu, const void *delta, const float *A,
+                                const void *B, const void *C, const float *D, const void *z,
+                                const float *delta_bias, int delta_softplus,
+                                const int64_t *rows, int64_t n_rows, double *y_out, int nthreads)
+{
+    if (batch < 0 || dim < 0 || dstate < 0 || width < 1)
+        return -1;
+    if (dtype != ORACLE_F32 && dtype != ORACLE_BF16)
+        return -1;
+    if (!rows)
+        n_rows = batch * dim;
+    if (n_rows > 0 && (!state || !conv_state || !x || !conv_w || !delta || !A || !B || !C || !y_out))
+        return -1;
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const int64_t row = rows ? rows[r] : r;
+        if (row < 0 || row >= batch * dim)
+            return -1;
+    }
+#ifdef _OPENMP
+    if (nthreads > 0)
+        omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(static)
+#endif
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const int64_t row = rows ? rows[r] : r;
+        const int64_t b = row / dim, d = row % dim;
+        double *cs = conv_state + r * width;
+        for (int k = 0; k + 1 < width; ++k)
+            cs[k] = cs[k + 1];
+        cs[width - 1] = load_value(x, dtype, row);
+        double acc = conv_b ? (double)conv_b[d] : 0.0;
+        for (int k = 0; k < width; ++k)
+            acc += (double)conv_w[d * width + k] * cs[k];
+        const double u = conv_silu ? silu(acc) : acc;
+        scan_row(b, d, dim, dstate, 1, dtype, NULL, &u, delta, A, B, C, D, z, delta_bias,
                  delta_softplus, state + r * dstate, y_out + r);
     }
     return 0;

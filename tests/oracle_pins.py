@@ -370,6 +370,109 @@ def pin_bf16_decoding(orc, seed=22):
     assert np.array_equal(yb, yf) and np.array_equal(hb, hf)
 
 
+# ---- convolution prologue ("Notas sobre Mamba", "O bloco Mamba": short
+# depthwise convolution + SiLU before the SSM; width d_conv = 4 in "Mamba-2 e
+# State Space Duality (SSD)"). Reading: causal, zero input before t = 0,
+# w[d, K-1] weighs the current input.
+
+def _conv_case(g, batch=2, dim=3, L=37, N=4, width=4):
+    return dict(x=_f32(g.normal(size=(batch, dim, L))), conv_w=_f32(g.normal(size=(dim, width))),
+                conv_b=_f32(g.normal(size=dim)), delta=_f32(g.normal(scale=0.5, size=(batch, dim, L))),
+                A=_f32(-np.exp(g.normal(size=(dim, N)))), B=_f32(g.normal(size=(batch, N, L))),
+                C=_f32(g.normal(size=(batch, N, L))), D=_f32(g.uniform(0.5, 1.5, size=dim)),
+                delta_bias=_f32(g.normal(size=dim) - 2.0))
+
+
+def pin_conv_matches_numpy_convolve(orc, seed=30):
+    """The convolution output against numpy's full convolution truncated to
+    the first L outputs (the causal form), for every width 1..4, with and
+    without the SiLU (scipy's expit)."""
+    g = _rng(seed)
+    for width in (1, 2, 3, 4):
+        case = _conv_case(g, width=width)
+        for act in (False, True):
+            _, _, u = orc.conv_scan(**case, conv_silu=act, return_u=True)
+            x, w, b = case["x"].astype(np.float64), case["conv_w"].astype(np.float64), case["conv_b"]
+            batch, dim, L = x.shape
+            want = np.empty_like(x)
+            for bi in range(batch):
+                for d in range(dim):
+                    pre = np.convolve(x[bi, d], w[d][::-1])[:L] + float(b[d])
+                    want[bi, d] = pre * expit(pre) if act else pre
+            assert _rel(u, want) <= 1e-12, (width, act)
+
+
+def pin_conv_impulse_response(orc, seed=31):
+    """A unit impulse at t0 returns the filter taps from t0 on, newest tap
+    first, and nothing before t0 (causality)."""
+    g = _rng(seed)
+    case = _conv_case(g, batch=1, dim=2, L=16, width=4)
+    case["x"] = np.zeros_like(case["x"])
+    case["x"][0, 1, 5] = 1.0
+    case["conv_b"] = np.zeros_like(case["conv_b"])
+    _, _, u = orc.conv_scan(**case, conv_silu=False, return_u=True)
+    w = case["conv_w"][1].astype(np.float64)
+    want = np.zeros(16)
+    want[5:9] = w[::-1]
+    assert np.array_equal(u[0, 1], want)
+    assert np.array_equal(u[0, 0], np.zeros(16))
+
+
+def pin_conv_identity_filter_is_plain_scan(orc, seed=32):
+    """Taps (0, ..., 0, 1), no bias, no SiLU: u = x, so the result is the plain
+    scan of x, bit for bit."""
+    g = _rng(seed)
+    case = _conv_case(g, width=4)
+    case["conv_w"] = _f32(np.tile([0.0, 0.0, 0.0, 1.0], (3, 1)))
+    case["conv_b"] = None
+    y, h = orc.conv_scan(**case, conv_silu=False)
+    x = case.pop("x")
+    for k in ("conv_w", "conv_b"):
+        case.pop(k)
+    y2, h2 = orc.scan(u=x, **case)
+    assert np.array_equal(y, y2) and np.array_equal(h, h2)
+
+
+def pin_conv_output_feeds_scan(orc, seed=33):
+    """The scan of the fused path equals the plain scan of numpy's
+    convolution + SiLU (rounded to float32, hence the tolerance)."""
+    g = _rng(seed)
+    case = _conv_case(g, width=3)
+    y, h = orc.conv_scan(**case)
+    x, w, b = case["x"].astype(np.float64), case["conv_w"].astype(np.float64), case["conv_b"]
+    batch, dim, L = x.shape
+    u = np.empty_like(x)
+    for bi in range(batch):
+        for d in range(dim):
+            pre = np.convolve(x[bi, d], w[d][::-1])[:L] + float(b[d])
+            u[bi, d] = pre * expit(pre)
+    rest = {k: v for k, v in case.items() if k not in ("x", "conv_w", "conv_b")}
+    y2, h2 = orc.scan(u=_f32(u), **rest)
+    assert _rel(y, y2) <= 1e-5 and _rel(h, h2) <= 1e-5
+
+
+def pin_conv_decode_equals_scan(orc, seed=34):
+    """L decode steps with the convolution state reproduce the fused scan's
+    outputs and final state, and leave the last `width` inputs in the
+    convolution state, oldest first."""
+    g = _rng(seed)
+    case = _conv_case(g, batch=2, dim=3, L=19, N=5, width=4)
+    y, h = orc.conv_scan(**case)
+    batch, dim, L = case["x"].shape
+    N = case["B"].shape[1]
+    state = np.zeros((batch, dim, N))
+    cstate = np.zeros((batch, dim, 4))
+    ys = np.empty((batch, dim, L))
+    for t in range(L):
+        ys[:, :, t] = orc.conv_state_update(
+            state=state, conv_state=cstate, x=_f32(case["x"][:, :, t]), conv_w=case["conv_w"],
+            conv_b=case["conv_b"], delta=_f32(case["delta"][:, :, t]), A=case["A"],
+            B=_f32(case["B"][:, :, t]), C=_f32(case["C"][:, :, t]), D=case["D"],
+            delta_bias=case["delta_bias"])
+    assert _rel(ys, y) <= 1e-12 and _rel(state, h) <= 1e-12
+    assert np.array_equal(cstate, case["x"][:, :, L - 4:].astype(np.float64))
+
+
 ALL_PINS = [
     pin_selection_step,
     pin_lti_convolution,
@@ -384,4 +487,9 @@ ALL_PINS = [
     pin_softplus_of_biased_step,
     pin_gate,
     pin_bf16_decoding,
+    pin_conv_matches_numpy_convolve,
+    pin_conv_impulse_response,
+    pin_conv_identity_filter_is_plain_scan,
+    pin_conv_output_feeds_scan,
+    pin_conv_decode_equals_scan,
 ]

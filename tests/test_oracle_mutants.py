@@ -28,8 +28,17 @@ MUTANTS = [
     ("softplus_is_exp", "return v > 20.0 ? v : log1p(exp(v));", "return v > 20.0 ? v : exp(v);"),
     ("bf16_shift", "<< 16;", "<< 15;"),
     ("token_not_scaled", "h[n] = exp(dt * a) * h[n] + Bbar * x;", "h[n] = exp(dt * a) * h[n] + Bbar;"),
-    ("state_not_reset_per_row", "h[n] = h0 ? h0[r * dstate + n] : 0.0;",
-     "h[n] = h0 ? h0[r * dstate + n] : (r > 0 ? 0.5 : 0.0);"),
+    ("state_not_reset_per_row",
+     "h[n] = h0 ? h0[r * dstate + n] : 0.0;\n        scan_row(b, d, dim, dstate, seqlen, dtype, u, NULL,",
+     "h[n] = h0 ? h0[r * dstate + n] : (r > 0 ? 0.5 : 0.0);\n        scan_row(b, d, dim, dstate, seqlen, dtype, u, NULL,"),
+    ("conv_taps_not_reversed", "acc += (double)w[k] * load_value(x, dtype, row * seqlen + s);",
+     "acc += (double)w[width - 1 - k] * load_value(x, dtype, row * seqlen + s);"),
+    ("conv_window_off_by_one", "const int64_t s = t - (width - 1) + k;", "const int64_t s = t - width + k;"),
+    ("conv_no_silu", "u_row[t] = conv_silu ? silu(acc) : acc;", "u_row[t] = acc;"),
+    ("conv_bias_dropped", "double acc = bias;", "double acc = 0.0 * bias;"),
+    ("conv_state_not_shifted", "cs[k] = cs[k + 1];", "cs[k] = cs[k];"),
+    ("conv_decode_taps_reversed", "acc += (double)conv_w[d * width + k] * cs[k];",
+     "acc += (double)conv_w[d * width + width - 1 - k] * cs[k];"),
 ]
 
 
