@@ -235,6 +235,59 @@ ms_status mamba_scan_plan_query(const ms_scan_args *args, ms_scan_plan *plan);
 ms_status mamba_scan_fwd_with_plan(const ms_scan_args *args, const ms_scan_plan *plan, void *workspace,
                                    size_t workspace_bytes, void *stream);
 
+/* ---- Convolution prologue ------------------------------------------------
+ * The Mamba block ("Notas sobre Mamba", section "O bloco Mamba", block
+ * diagram) puts a short depthwise convolution and a SiLU on the x branch
+ * before the selective SSM; "Mamba-2 e State Space Duality (SSD)" configures
+ * its width as d_conv = 4. The pages print no formula; the library computes
+ * the causal depthwise convolution, one filter per channel d, with zero input
+ * before t = 0:
+ *     u[b,d,t] = act( bias[d] + sum_{k<width} weight[d,k] * x[b,d,t-width+1+k] )
+ * with act = SiLU (or the identity), weight[d,width-1] on the current input,
+ * and u is the SSM input of the scan (its D u skip term included). */
+#define MS_MAX_CONV_WIDTH 4
+
+typedef struct ms_conv1d_args {
+    const float *weight;   /* (dim, width) float32, contiguous, required                  */
+    const float *bias;     /* (dim) float32, or NULL (no bias)                            */
+    int32_t width;         /* taps, 1 .. MS_MAX_CONV_WIDTH                                */
+    int32_t silu;          /* 1: act = SiLU; 0: act = identity                            */
+} ms_conv1d_args;
+
+/*
+ * Convolution prologue fused into the selective scan: args->u holds x, the
+ * convolution input ((batch, dim, seqlen), the layout and dtype of u); every
+ * other argument means what it means for mamba_scan_fwd. u itself is never
+ * written to memory. Runs on the sequential kernels with 2 or 4 lanes per row,
+ * in one segment, with no workspace. `plan` is NULL (automatic) or one of those
+ * configurations (warps_per_cta = max_warps, segments = 1). The caller owns
+ * every buffer; the call enqueues one kernel on `stream`.
+ * Errors: as mamba_scan_fwd; MS_ERR_INVALID_ARG for a NULL conv or weight or a
+ * silu flag other than 0/1, or width < 1; MS_ERR_UNSUPPORTED for width >
+ * MS_MAX_CONV_WIDTH, force_segments > 1, or a plan that cannot fuse the
+ * prologue; MS_ERR_ALIGNMENT for a misaligned weight or bias.
+ */
+ms_status mamba_conv_scan_fwd(const ms_scan_args *args, const ms_conv1d_args *conv,
+                              const ms_scan_plan *plan, void *stream);
+
+/*
+ * Decode step with the convolution prologue: args->x is the new convolution
+ * input. conv_state (batch, dim, width) in the input dtype (element strides
+ * conv_state_batch_stride and conv_state_dim_stride; the width axis is
+ * contiguous) holds each row's last `width` inputs, oldest first; it is
+ * updated in place (the oldest input dropped, x appended), then u =
+ * act(bias + weight . conv_state) is the input of the state update
+ * (mamba_state_update with u for x). A zero conv_state is the state of a
+ * sequence that has not started, matching the scan's zero input before t = 0.
+ * Errors: as mamba_state_update; MS_ERR_INVALID_ARG for a NULL conv, weight or
+ * conv_state, negative strides, silu other than 0/1 or width < 1;
+ * MS_ERR_UNSUPPORTED for width > MS_MAX_CONV_WIDTH; MS_ERR_ALIGNMENT for a
+ * pointer not aligned to its element size.
+ */
+ms_status mamba_conv_state_update(const ms_update_args *args, const ms_conv1d_args *conv, void *conv_state,
+                                  int64_t conv_state_batch_stride, int64_t conv_state_dim_stride,
+                                  void *stream);
+
 /* Size of the device array behind mamba_scan_fwd_noalloc (8 MiB per GPU). */
 #define MS_NOALLOC_SCRATCH_BYTES (8u << 20)
 

@@ -24,6 +24,7 @@ import os
 __all__ = [
     "scan_fwd", "state_update", "scan_workspace_size", "scan_plan", "scan_configs", "library_path",
     "load_library", "MambaScanError", "ScanArgs", "UpdateArgs", "ScanPlan", "MS_F32", "MS_BF16",
+    "Conv1dArgs", "conv_scan_fwd", "conv_state_update", "build_conv_args",
     "MAX_DSTATE",
 ]
 
@@ -73,6 +74,11 @@ class UpdateArgs(ctypes.Structure):
     ]
 
 
+class Conv1dArgs(ctypes.Structure):
+    """Mirror of ``ms_conv1d_args``."""
+    _fields_ = [("weight", _vp), ("bias", _vp), ("width", _i32), ("silu", _i32)]
+
+
 class ScanPlan(ctypes.Structure):
     """Mirror of ``ms_scan_plan``."""
     _fields_ = [
@@ -116,6 +122,12 @@ def load_library():
         lib.mamba_scan_config_info.restype = ctypes.c_int
         lib.mamba_scan_config_info.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int),
                                                ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
+        lib.mamba_conv_scan_fwd.restype = ctypes.c_int
+        lib.mamba_conv_scan_fwd.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(Conv1dArgs),
+                                            ctypes.POINTER(ScanPlan), _vp]
+        lib.mamba_conv_state_update.restype = ctypes.c_int
+        lib.mamba_conv_state_update.argtypes = [ctypes.POINTER(UpdateArgs), ctypes.POINTER(Conv1dArgs), _vp,
+                                                ctypes.c_int64, ctypes.c_int64, _vp]
         lib.mamba_scan_config_kind.restype = ctypes.c_int
         lib.mamba_scan_config_kind.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
         lib.mamba_scan_plan_query.restype = ctypes.c_int
@@ -338,4 +350,63 @@ def state_update(state, x, delta, A, B, C, D=None, z=None, delta_bias=None, delt
                              delta_softplus=delta_softplus)
     with torch.cuda.device(x.device):
         _check(load_library().mamba_state_update(ctypes.byref(args), _stream_ptr(stream)))
+    return y
+
+
+def build_conv_args(weight, bias=None, silu=True) -> Conv1dArgs:
+    """Fill an ``ms_conv1d_args`` from a (dim, width) float32 weight and an
+    optional (dim,) float32 bias."""
+    torch = _torch()
+    _need_cuda("conv weight", weight, torch.float32, 2)
+    if not weight.is_contiguous():
+        raise ValueError("conv weight must be contiguous (dim, width)")
+    _need_cuda("conv bias", bias, torch.float32, 1)
+    if bias is not None and (tuple(bias.shape) != (weight.shape[0],) or not bias.is_contiguous()):
+        raise ValueError("conv bias must be a contiguous (dim,) float32 tensor")
+    c = Conv1dArgs()
+    c.weight, c.bias, c.width, c.silu = _ptr(weight), _ptr(bias), weight.shape[1], 1 if silu else 0
+    return c
+
+
+def conv_scan_fwd(x, conv_weight, delta, A, B, C, D=None, z=None, delta_bias=None, conv_bias=None,
+                  conv_silu=True, delta_softplus=True, initial_state=None, return_last_state=True, out=None,
+                  stream=None, plan=None):
+    """Causal depthwise convolution + SiLU prologue fused into the selective
+    scan: ``x`` (batch, dim, L) is the convolution input, ``conv_weight``
+    (dim, width) and ``conv_bias`` (dim,) float32; the scan input is
+    u = silu(conv(x)). Other arguments as :func:`scan_fwd` (no segments)."""
+    torch = _torch()
+    y = torch.empty_like(x) if out is None else out
+    hT = None
+    if return_last_state:
+        hT = torch.empty((x.shape[0], x.shape[1], B.shape[1]), device=x.device, dtype=torch.float32)
+    args = build_scan_args(x, delta, A, B, C, y, D=D, z=z, delta_bias=delta_bias, delta_softplus=delta_softplus,
+                           initial_state=initial_state, final_state=hT)
+    conv = build_conv_args(conv_weight, conv_bias, conv_silu)
+    if conv_weight.shape[0] != x.shape[1]:
+        raise ValueError("conv weight must have one row per channel")
+    with torch.cuda.device(x.device):
+        _check(load_library().mamba_conv_scan_fwd(ctypes.byref(args), ctypes.byref(conv),
+                                                  None if plan is None else ctypes.byref(plan),
+                                                  _stream_ptr(stream)))
+    return (y, hT) if return_last_state else y
+
+
+def conv_state_update(state, conv_state, x, conv_weight, delta, A, B, C, D=None, z=None, delta_bias=None,
+                      conv_bias=None, conv_silu=True, delta_softplus=True, out=None, stream=None):
+    """One decode step with the convolution prologue: ``conv_state`` (batch,
+    dim, width) in x's dtype holds the last ``width`` inputs (oldest first) and
+    is updated in place with ``x``; ``state`` as :func:`state_update`."""
+    torch = _torch()
+    y = torch.empty_like(x) if out is None else out
+    args = build_update_args(state, x, delta, A, B, C, y, D=D, z=z, delta_bias=delta_bias,
+                             delta_softplus=delta_softplus)
+    conv = build_conv_args(conv_weight, conv_bias, conv_silu)
+    _need_cuda("conv_state", conv_state, x.dtype, 3)
+    if tuple(conv_state.shape) != (x.shape[0], x.shape[1], conv_weight.shape[1]) or conv_state.stride(2) != 1:
+        raise ValueError("conv_state must be (batch, dim, width) with a contiguous width axis")
+    with torch.cuda.device(x.device):
+        _check(load_library().mamba_conv_state_update(ctypes.byref(args), ctypes.byref(conv), _ptr(conv_state),
+                                                      conv_state.stride(0), conv_state.stride(1),
+                                                      _stream_ptr(stream)))
     return y

@@ -113,6 +113,65 @@ ms::ScanParams to_params(const ms_scan_args *a) {
     return p;
 }
 
+ms_status check_conv(const ms_conv1d_args *c) {
+    if (!c) return invalid("conv is NULL");
+    if (!c->weight) return invalid("conv weight is required");
+    if (c->silu != 0 && c->silu != 1) return invalid("conv silu must be 0 or 1");
+    if (c->width < 1) return invalid("conv width must be >= 1");
+    if (c->width > MS_MAX_CONV_WIDTH) {
+        set_error("conv width %d exceeds the supported maximum %d", c->width, MS_MAX_CONV_WIDTH);
+        return MS_ERR_UNSUPPORTED;
+    }
+    if (!elem_aligned(c->weight, 4) || (c->bias && !elem_aligned(c->bias, 4))) {
+        set_error("conv weight or bias is not aligned to 4 bytes");
+        return MS_ERR_ALIGNMENT;
+    }
+    return MS_OK;
+}
+
+// Validate a decode call and fill its kernel parameters.
+ms_status update_params(const ms_update_args *a, ms::UpdateParams *p) {
+    if (!a) return invalid("args is NULL");
+    if (a->batch <= 0 || a->dim <= 0 || a->dstate <= 0)
+        return invalid("batch, dim and dstate must be positive");
+    if (a->in_dtype != MS_F32 && a->in_dtype != MS_BF16) return invalid("in_dtype");
+    if (!a->state || !a->x || !a->delta || !a->B || !a->C || !a->A || !a->y)
+        return invalid("state, x, delta, B, C, A and y are required");
+    if (a->state_batch_stride < 0 || a->state_dim_stride < 0 || a->x_batch_stride < 0 ||
+        a->delta_batch_stride < 0 || a->B_batch_stride < 0 || a->C_batch_stride < 0 ||
+        a->y_batch_stride < 0 || (a->z && a->z_batch_stride < 0))
+        return invalid("strides must be non-negative");
+    if (a->dstate > MS_MAX_DSTATE) {
+        set_error("dstate %lld exceeds the supported maximum %d", static_cast<long long>(a->dstate),
+                  MS_MAX_DSTATE);
+        return MS_ERR_UNSUPPORTED;
+    }
+    if (a->batch > 65535) {
+        set_error("batch %lld exceeds 65535", static_cast<long long>(a->batch));
+        return MS_ERR_UNSUPPORTED;
+    }
+    const int eb = a->in_dtype == MS_F32 ? 4 : 2;
+    if (!elem_aligned(a->state, 4) || !elem_aligned(a->x, eb) || !elem_aligned(a->delta, eb) ||
+        !elem_aligned(a->B, eb) || !elem_aligned(a->C, eb) || !elem_aligned(a->y, eb) ||
+        (a->z && !elem_aligned(a->z, eb)) || !elem_aligned(a->A, 4) ||
+        (a->D && !elem_aligned(a->D, 4)) || (a->delta_bias && !elem_aligned(a->delta_bias, 4))) {
+        set_error("a pointer is not aligned to its element size");
+        return MS_ERR_ALIGNMENT;
+    }
+    *p = ms::UpdateParams{};
+    p->batch = a->batch; p->dim = a->dim; p->dstate = a->dstate;
+    p->state = a->state; p->s_sb = a->state_batch_stride; p->s_sd = a->state_dim_stride;
+    p->x = a->x; p->x_sb = a->x_batch_stride;
+    p->delta = a->delta; p->dl_sb = a->delta_batch_stride;
+    p->B = a->B; p->B_sb = a->B_batch_stride;
+    p->C = a->C; p->C_sb = a->C_batch_stride;
+    p->z = a->z; p->z_sb = a->z_batch_stride;
+    p->y = a->y; p->y_sb = a->y_batch_stride;
+    p->A = a->A; p->D = a->D; p->delta_bias = a->delta_bias;
+    p->softplus = a->delta_softplus ? 1 : 0;
+    return MS_OK;
+}
+
 ms_status run_plan(ms::ScanParams p, const ms::ScanPlan &plan, int in_dtype, void *workspace,
                    size_t workspace_bytes, void *stream) {
     if (plan.ws_bytes > 0) {
@@ -238,47 +297,74 @@ ms_status mamba_scan_fwd_with_plan(const ms_scan_args *args, const ms_scan_plan 
 }
 
 ms_status mamba_state_update(const ms_update_args *a, void *stream) {
-    if (!a) return invalid("args is NULL");
-    if (a->batch <= 0 || a->dim <= 0 || a->dstate <= 0)
-        return invalid("batch, dim and dstate must be positive");
-    if (a->in_dtype != MS_F32 && a->in_dtype != MS_BF16) return invalid("in_dtype");
-    if (!a->state || !a->x || !a->delta || !a->B || !a->C || !a->A || !a->y)
-        return invalid("state, x, delta, B, C, A and y are required");
-    if (a->state_batch_stride < 0 || a->state_dim_stride < 0 || a->x_batch_stride < 0 ||
-        a->delta_batch_stride < 0 || a->B_batch_stride < 0 || a->C_batch_stride < 0 ||
-        a->y_batch_stride < 0 || (a->z && a->z_batch_stride < 0))
-        return invalid("strides must be non-negative");
-    if (a->dstate > MS_MAX_DSTATE) {
-        set_error("dstate %lld exceeds the supported maximum %d", static_cast<long long>(a->dstate),
-                  MS_MAX_DSTATE);
-        return MS_ERR_UNSUPPORTED;
-    }
-    if (a->batch > 65535) {
-        set_error("batch %lld exceeds 65535", static_cast<long long>(a->batch));
-        return MS_ERR_UNSUPPORTED;
-    }
-    const int eb = a->in_dtype == MS_F32 ? 4 : 2;
-    if (!elem_aligned(a->state, 4) || !elem_aligned(a->x, eb) || !elem_aligned(a->delta, eb) ||
-        !elem_aligned(a->B, eb) || !elem_aligned(a->C, eb) || !elem_aligned(a->y, eb) ||
-        (a->z && !elem_aligned(a->z, eb)) || !elem_aligned(a->A, 4) ||
-        (a->D && !elem_aligned(a->D, 4)) || (a->delta_bias && !elem_aligned(a->delta_bias, 4))) {
-        set_error("a pointer is not aligned to its element size");
-        return MS_ERR_ALIGNMENT;
-    }
-    ms::UpdateParams p{};
-    p.batch = a->batch; p.dim = a->dim; p.dstate = a->dstate;
-    p.state = a->state; p.s_sb = a->state_batch_stride; p.s_sd = a->state_dim_stride;
-    p.x = a->x; p.x_sb = a->x_batch_stride;
-    p.delta = a->delta; p.dl_sb = a->delta_batch_stride;
-    p.B = a->B; p.B_sb = a->B_batch_stride;
-    p.C = a->C; p.C_sb = a->C_batch_stride;
-    p.z = a->z; p.z_sb = a->z_batch_stride;
-    p.y = a->y; p.y_sb = a->y_batch_stride;
-    p.A = a->A; p.D = a->D; p.delta_bias = a->delta_bias;
-    p.softplus = a->delta_softplus ? 1 : 0;
+    ms::UpdateParams p;
+    const ms_status st = update_params(a, &p);
+    if (st != MS_OK) return st;
     const cudaError_t e = ms::launch_state_update(p, a->in_dtype, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "state update kernel launch");
     return MS_OK;
+}
+
+ms_status mamba_conv_state_update(const ms_update_args *a, const ms_conv1d_args *conv, void *conv_state,
+                                  int64_t conv_state_batch_stride, int64_t conv_state_dim_stride,
+                                  void *stream) {
+    ms::UpdateParams p;
+    ms_status st = update_params(a, &p);
+    if (st != MS_OK) return st;
+    st = check_conv(conv);
+    if (st != MS_OK) return st;
+    if (!conv_state) return invalid("conv_state is required");
+    if (conv_state_batch_stride < 0 || conv_state_dim_stride < 0)
+        return invalid("conv_state strides must be non-negative");
+    if (!elem_aligned(conv_state, a->in_dtype == MS_F32 ? 4 : 2)) {
+        set_error("conv_state is not aligned to its element size");
+        return MS_ERR_ALIGNMENT;
+    }
+    p.conv_state = conv_state;
+    p.cs_sb = conv_state_batch_stride;
+    p.cs_sd = conv_state_dim_stride;
+    p.conv_w = conv->weight;
+    p.conv_b = conv->bias;
+    p.conv_width = conv->width;
+    p.conv_silu = conv->silu;
+    const cudaError_t e = ms::launch_state_update(p, a->in_dtype, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "state update kernel launch");
+    return MS_OK;
+}
+
+ms_status mamba_conv_scan_fwd(const ms_scan_args *args, const ms_conv1d_args *conv, const ms_scan_plan *plan,
+                              void *stream) {
+    ms_status st = check_scan(args);
+    if (st != MS_OK) return st;
+    st = check_conv(conv);
+    if (st != MS_OK) return st;
+    if (args->force_segments > 1) {
+        set_error("the convolution prologue runs in one segment (force_segments %d)", args->force_segments);
+        return MS_ERR_UNSUPPORTED;
+    }
+    ms::ScanParams p = to_params(args);
+    p.conv_w = conv->weight;
+    p.conv_b = conv->bias;
+    p.conv_width = conv->width;
+    p.conv_silu = conv->silu;
+    ms::ScanPlan pl{};
+    if (plan) {
+        if (!ms::make_plan(p, args->in_dtype, plan->config, plan->warps_per_cta, plan->segments, &pl)) {
+            set_error("plan (config %d, %d warps, %d segments) cannot run the convolution prologue", plan->config,
+                      plan->warps_per_cta, plan->segments);
+            return MS_ERR_UNSUPPORTED;
+        }
+    } else {
+        int sms = 0;
+        st = device_sms(&sms);
+        if (st != MS_OK) return st;
+        pl = ms::plan_scan(p, args->in_dtype, 0, sms);
+        if (pl.kind != 1) {
+            set_error("no kernel configuration fuses the convolution prologue for these arguments");
+            return MS_ERR_UNSUPPORTED;
+        }
+    }
+    return run_plan(p, pl, args->in_dtype, nullptr, 0, stream);
 }
 
 }  // extern "C"

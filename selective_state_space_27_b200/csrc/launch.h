@@ -22,6 +22,11 @@ struct ScanParams {
     int64_t seg_len;    // time steps per segment, a multiple of the chunk length
     float *ws_P;        // (batch*dim, nseg, 16): decay product of each segment
     float *ws_H;        // (batch*dim, nseg, 16): end state of each segment from zero
+    // Convolution prologue (sequential kernels only): when conv_w is set, u
+    // holds the convolution input x and the SSM input is
+    // act(conv_b[d] + sum_k conv_w[d*conv_width + k] x[t - conv_width + 1 + k]).
+    const float *conv_w, *conv_b;
+    int conv_width, conv_silu;
 };
 
 // Launch configuration chosen on the host for one scan call.
@@ -39,6 +44,8 @@ struct ScanPlan {
     size_t ws_bytes;
 };
 
+// With p.conv_w set only the sequential configurations that fuse the
+// convolution prologue (lanes 2 and 4) are considered.
 ScanPlan plan_scan(const ScanParams &p, int in_dtype, int force_segments, int num_sms);
 // A plan with a fixed configuration, CTA size and segment count; returns false
 // (and leaves `out` unspecified) when the configuration cannot run `p`.
@@ -51,11 +58,12 @@ cudaError_t launch_scan(const ScanParams &p, const ScanPlan &plan, int in_dtype,
 
 // Sequential kernels (scan_rec.cu): CTAs of rec_threads() threads (recurrence
 // and I/O warps) owning rec_rows(lanes_per_row) rows, no workspace, one segment.
-int rec_smem_bytes(int in_dtype, int lanes_per_row);
+int rec_smem_bytes(int in_dtype, int lanes_per_row, bool conv);
 int rec_chunk();
 int rec_threads();
 int rec_rows(int lanes_per_row);
-int rec_ctas_per_sm(int in_dtype, int lanes_per_row, bool vec);
+int rec_ctas_per_sm(int in_dtype, int lanes_per_row, bool vec, bool conv);
+bool rec_supports_conv(int lanes_per_row);
 cudaError_t launch_rec(const ScanParams &p, int lanes_per_row, bool vec, int in_dtype, cudaStream_t stream);
 
 struct UpdateParams {
@@ -69,6 +77,12 @@ struct UpdateParams {
     void *y;           int64_t y_sb;
     const float *A, *D, *delta_bias;
     int softplus;
+    // Convolution prologue: when conv_w is set, x is the convolution input and
+    // conv_state (batch, dim, conv_width; element strides cs_sb, cs_sd, the
+    // width axis contiguous) holds the last conv_width inputs, oldest first.
+    void *conv_state;  int64_t cs_sb, cs_sd;
+    const float *conv_w, *conv_b;
+    int conv_width, conv_silu;
 };
 
 cudaError_t launch_state_update(const UpdateParams &p, int in_dtype, cudaStream_t stream);

@@ -638,8 +638,9 @@ ScanPlan plan_scan(const ScanParams &p, int in_dtype, int force_segments, int nu
                strides_ok(p.y_sb, p.y_sd) && (p.z == nullptr || strides_ok(p.z_sb, p.z_sd));
 
     const int sms = num_sms > 0 ? num_sms : 148;
+    const bool conv = p.conv_w != nullptr;   // only sequential kernels fuse the convolution prologue
     double best = 1e300;
-    for (int ci = 0; ci < kNumConfigs; ++ci) {
+    for (int ci = 0; ci < (conv ? 0 : kNumConfigs); ++ci) {
         const Config cf = kConfigs[ci];
         if (cf.ni != 1 && !plan.vec) continue;
         if (cf.ni == 0 && p.dstate != kMaxN) continue;
@@ -684,7 +685,8 @@ ScanPlan plan_scan(const ScanParams &p, int in_dtype, int force_segments, int nu
         best *= kChunkedClocksPerUnit;
         for (int ri = 0; ri < kNumRec; ++ri) {
             const int lpr = kRecLanes[ri];
-            const int per_sm = rec_ctas_per_sm(in_dtype, lpr, plan.vec);
+            if (conv && !rec_supports_conv(lpr)) continue;
+            const int per_sm = rec_ctas_per_sm(in_dtype, lpr, plan.vec, conv);
             if (per_sm < 1) continue;
             const int64_t R = rec_rows(lpr);
             const int64_t ctas = p.batch * ((p.dim + R - 1) / R);
@@ -712,6 +714,7 @@ bool make_plan(const ScanParams &p, int in_dtype, int config, int warps, int seg
     if (config >= kNumConfigs && config < kNumConfigs + kNumRec) {
         // sequential kernel: fixed CTA of rec_threads(), the whole sequence in one pass
         if (warps != rec_threads() / 32 || segments != 1 || p.dstate > kMaxN) return false;
+        if (p.conv_w && !rec_supports_conv(kRecLanes[config - kNumConfigs])) return false;
         const int eb = in_dtype == 0 ? 4 : 2;
         auto strides_ok = [&](int64_t s1, int64_t s2) { return (s1 * eb) % 16 == 0 && (s2 * eb) % 16 == 0; };
         ScanPlan plan{};
@@ -731,7 +734,7 @@ bool make_plan(const ScanParams &p, int in_dtype, int config, int warps, int seg
         *out = plan;
         return true;
     }
-    if (config < 0 || config >= kNumConfigs || segments < 1) return false;
+    if (config < 0 || config >= kNumConfigs || segments < 1 || p.conv_w) return false;
     const Config cf = kConfigs[config];
     ScanPlan plan{};
     const int eb = in_dtype == 0 ? 4 : 2;

@@ -89,24 +89,36 @@ template <int LPR> struct Shape {
 
 // The I/O warps' ring of raw inputs in shared memory, after the tile stages.
 // It holds every chunk from the oldest one still to be finished (its u and z
-// feed the readout) to the newest one in flight, kRawAhead chunks ahead of the
+// feed the readout) to the newest one in flight, RA chunks ahead of the
 // one being widened. Each I/O thread fills and reads only its own 16-byte
 // slots (its u, delta and z pieces of PB bytes each, then its B/C pieces),
 // stored slot-major so that a warp's slot accesses are contiguous.
 constexpr int kRawStages = 5;
-constexpr int kRawAhead = kRawStages - kTileStages + 1;
-template <typename T, int LPR> struct Raw {
+// With the convolution prologue (CONV) every thread also copies the 16 bytes
+// before its u piece (the convolution's look-back, VE >= 4 elements) into one
+// more slot, and a skip tile per tile stage ([row][step] floats after the
+// ring) carries D u from the widening to the readout.
+template <typename T, int LPR, bool CONV = false> struct Raw {
     static constexpr int EB = static_cast<int>(sizeof(T));
     static constexpr int PB = Shape<LPR>::IP * EB;                   // bytes of one u/delta/z piece
     static constexpr int PS = (PB + 15) / 16;                        // slots per piece
     static constexpr int VE = 16 / EB;                               // elements per B/C piece
     static constexpr int BC_PER = 2 * kStates * (kSteps / VE) / kIoThreads;   // B/C pieces per thread
-    static constexpr int SLOTS = 3 * PS + BC_PER;
+    static constexpr int HALO = 3 * PS + BC_PER;                     // slot of the look-back (CONV)
+    static constexpr int SLOTS = 3 * PS + BC_PER + (CONV ? 1 : 0);
     static constexpr int STAGE = SLOTS * kIoThreads * 16;
+    // ring depth: one stage less with the prologue, so that its larger slots
+    // and the skip tiles still leave room for 3 (LPR 4) or 2 (LPR 2) CTAs per SM
+    static constexpr int RS = CONV ? kRawStages - 1 : kRawStages;
+    static constexpr int RA = RS - kTileStages + 1;                   // chunks staged ahead
     static constexpr int OFF = Shape<LPR>::BYTES;
-    static constexpr int BYTES = OFF + kRawStages * STAGE;           // total dynamic shared memory
+    static constexpr int SKR = kSteps + 4;                            // floats per row of the skip tile
+    static constexpr int SK_OFF = OFF + RS * STAGE;
+    static constexpr int SK_STAGE = Shape<LPR>::R * SKR * 4;
+    static constexpr int BYTES = SK_OFF + (CONV ? kTileStages * SK_STAGE : 0);   // total dynamic shared memory
     static_assert(BC_PER * kIoThreads * VE == 2 * kStates * kSteps, "B/C pieces split evenly");
     static_assert(PB == 4 || PB == 8 || PB % 16 == 0, "piece sizes cp.async can copy");
+    static_assert(!CONV || (PB % 16 == 0 && VE >= 4), "look-back: 16-byte aligned pieces, >= 3 earlier inputs");
 };
 
 // Named barriers (0 is __syncthreads): the producer arrives, the consumer
@@ -246,7 +258,7 @@ __device__ __forceinline__ void store_piece(T *dst, const float (&v)[P], int64_t
 template <typename T, int LPR>
 __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned char *smem, int tid) {
     using S = Shape<LPR>;
-    constexpr int NPL = S::NPL, R = S::R, IP = S::IP;
+    constexpr int NPL = S::NPL, R = S::R;
     constexpr int NP = NPL > 1 ? NPL / 2 : 1;
     constexpr int RW = 32 / LPR;   // rows per warp
     const int lane = tid & 31, warp = tid >> 5;
@@ -355,13 +367,13 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
 
 // The I/O warps: thread (r, k) handles steps k IP .. k IP + IP - 1 of row r in
 // every chunk, plus BC_PER 16-byte pieces of the chunk's B/C tiles. Its raw
-// inputs travel through the ring kRawAhead chunks ahead of use (cp.async on
+// inputs travel through the ring RA chunks ahead of use (cp.async on
 // the aligned path, plain loads otherwise); a thread waits only for its own
 // copies, so the ring needs no barrier.
-template <typename T, int LPR, bool VEC>
+template <typename T, int LPR, bool VEC, bool CONV>
 __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem, int i) {
     using S = Shape<LPR>;
-    using RW = Raw<T, LPR>;
+    using RW = Raw<T, LPR, CONV>;
     constexpr int R = S::R, IP = S::IP, IPR = S::IPR, EB = RW::EB, PB = RW::PB, PS = RW::PS;
     constexpr int VE = RW::VE, BC_PER = RW::BC_PER;
     static_assert(IP % 2 == 0, "pieces hold step pairs");
@@ -378,6 +390,16 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     const float Dd = p.D ? __ldg(p.D + dc) : 0.f;
     const bool has_z = p.z != nullptr;
     const int tk = k * IP;   // the thread's first step within a chunk
+    // Convolution taps right-aligned in a window of 4 (leading taps beyond the
+    // width stay 0): cw[3] weighs the current input.
+    float cw[4] = {0.f, 0.f, 0.f, 0.f}, cb = 0.f;
+    if constexpr (CONV) {
+        const int K = p.conv_width;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (j >= 4 - K) cw[j] = __ldg(p.conv_w + dc * K + (j - (4 - K)));
+        cb = p.conv_b ? __ldg(p.conv_b + dc) : 0.f;
+    }
     const T *src_row[3] = {static_cast<const T *>(p.u) + b * p.u_sb + dc * p.u_sd + tk,
                            static_cast<const T *>(p.delta) + b * p.dl_sb + dc * p.dl_sd + tk,
                            has_z ? static_cast<const T *>(p.z) + b * p.z_sb + dc * p.z_sd + tk : nullptr};
@@ -428,6 +450,20 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
 #pragma unroll
                 for (int w = 0; w < Piece<T, IP>::W; ++w)
                     reinterpret_cast<uint32_t *>(slot(rs, tsr * PS + w / 4))[w % 4] = pc.w[w];
+            }
+        }
+        if constexpr (CONV) {
+            // the VE inputs before the piece (the convolution's look-back); for
+            // the first piece of the sequence they lie before t = 0 and read as 0
+            const int64_t th = t0 + tk - VE;
+            const int hv = th < 0 ? 0 : static_cast<int>(min64(VE, max64(0, L - th)));
+            const T *hsrc = hv > 0 ? src_row[0] + t0 - VE : src_row[0];
+            if constexpr (VEC) {
+                cp_async16(slot(rs, RW::HALO), hsrc, hv * EB);
+            } else {
+                Piece<T, VE> pc;
+                load_piece<T, VE, false>(pc, hsrc, hv);
+                *reinterpret_cast<uint4 *>(slot(rs, RW::HALO)) = make_uint4(pc.w[0], pc.w[1], pc.w[2], pc.w[3]);
             }
         }
 #pragma unroll
@@ -482,13 +518,22 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
                 }
             }
         }
-        const Piece<T, IP> u = ring_piece(rs, 0);
+        float2 skip[IP / 2];   // D u
+        if constexpr (CONV) {
+            const float *sk = reinterpret_cast<const float *>(smem + RW::SK_OFF + s * RW::SK_STAGE) + r * RW::SKR + tk;
+#pragma unroll
+            for (int e = 0; e < IP; e += 2) skip[e / 2] = *reinterpret_cast<const float2 *>(sk + e);
+        } else {
+            const Piece<T, IP> u = ring_piece(rs, 0);
+#pragma unroll
+            for (int e = 0; e < IP; e += 2) skip[e / 2] = mul2(f2(Dd, Dd), f2(elem(u, e), elem(u, e + 1)));
+        }
         float outv[IP];
         if (has_z) {
             const Piece<T, IP> z = ring_piece(rs, 2);
 #pragma unroll
             for (int e = 0; e < IP; e += 2) {
-                const float2 yv = fma2(f2(Dd, Dd), f2(elem(u, e), elem(u, e + 1)), sum[e / 2]);
+                const float2 yv = add2(skip[e / 2], sum[e / 2]);
                 const float2 g = mul2(yv, silu2(f2(elem(z, e), elem(z, e + 1))));
                 outv[e] = g.x;
                 outv[e + 1] = g.y;
@@ -496,7 +541,7 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
         } else {
 #pragma unroll
             for (int e = 0; e < IP; e += 2) {
-                const float2 yv = fma2(f2(Dd, Dd), f2(elem(u, e), elem(u, e + 1)), sum[e / 2]);
+                const float2 yv = add2(skip[e / 2], sum[e / 2]);
                 outv[e] = yv.x;
                 outv[e + 1] = yv.y;
             }
@@ -508,7 +553,33 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     auto widen = [&](int64_t c, int s, int rs) {
         unsigned char *st = smem + s * S::STAGE;
         float4 *xrow = reinterpret_cast<float4 *>(st + S::X_OFF) + r * S::XR + tk / 2;
-        const Piece<T, IP> u = ring_piece(rs, 0), dl = ring_piece(rs, 1);
+        const Piece<T, IP> xin = ring_piece(rs, 0), dl = ring_piece(rs, 1);
+        // the SSM input u: the raw u, or the convolution prologue applied to x
+        float2 u2[IP / 2];
+        if constexpr (CONV) {
+            const uint4 hw = *reinterpret_cast<const uint4 *>(slot(rs, RW::HALO));
+            Piece<T, VE> hl;
+            hl.w[0] = hw.x; hl.w[1] = hw.y; hl.w[2] = hw.z; hl.w[3] = hw.w;
+            // input j of the window [look-back | piece]
+            auto win = [&](int j) { return j < VE ? elem(hl, j) : elem(xin, j - VE); };
+            float* sk = reinterpret_cast<float *>(smem + RW::SK_OFF + s * RW::SK_STAGE) + r * RW::SKR + tk;
+#pragma unroll
+            for (int e = 0; e < IP; e += 2) {
+                float a0 = cb, a1 = cb;
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    a0 = fmaf(cw[m], win(e + VE - 3 + m), a0);
+                    a1 = fmaf(cw[m], win(e + 1 + VE - 3 + m), a1);
+                }
+                float2 uv = f2(a0, a1);
+                if (p.conv_silu) uv = silu2(uv);
+                u2[e / 2] = uv;
+                *reinterpret_cast<float2 *>(sk + e) = mul2(f2(Dd, Dd), uv);
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < IP; e += 2) u2[e / 2] = f2(elem(xin, e), elem(xin, e + 1));
+        }
         const bool full = (c + 1) * kSteps <= L;
         const int64_t cnt = L - (c * kSteps + tk);
 #pragma unroll
@@ -519,7 +590,7 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
                 if (e >= cnt) v.x = 0.f;
                 if (e + 1 >= cnt) v.y = 0.f;
             }
-            const float2 du = mul2(v, f2(elem(u, e), elem(u, e + 1)));
+            const float2 du = mul2(v, u2[e / 2]);
             xrow[e / 2] = make_float4(v.x, du.x, v.y, du.y);
         }
 #pragma unroll
@@ -534,20 +605,20 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     };
 
     // Chunk c is widened in iteration c, finished in iteration c + kTileStages - 1
-    // (or after the loop), and its raw inputs are staged kRawAhead iterations
-    // before its widening into the ring stage that the chunk finished in the
-    // same iteration releases. Prologue: chunks 0 .. kRawAhead - 1 in flight,
+    // (or after the loop), and its raw inputs are staged RA = RS - kTileStages
+    // + 1 iterations before its widening into the ring stage that the chunk
+    // finished in the same iteration releases. Prologue: chunks 0 .. RA - 1 in flight,
     // one commit group per chunk (empty past the end: the count stays uniform).
 #pragma unroll
-    for (int c0 = 0; c0 < kRawAhead; ++c0) {
+    for (int c0 = 0; c0 < RW::RA; ++c0) {
         if (c0 < nchunks) stage_chunk(c0, c0);
         cp_async_commit();
     }
     int s = 0, rs = 0;                    // tile and ring stage of chunk c
     int sf = 0, rf = 0;                   // tile and ring stage of the next chunk to finish
-    int ra = kRawAhead % kRawStages;      // ring stage of chunk c + kRawAhead
+    int ra = RW::RA % RW::RS;             // ring stage of chunk c + RA
     for (int64_t c = 0; c < nchunks; ++c) {
-        cp_async_wait<kRawAhead - 1>();   // chunk c's copies have landed
+        cp_async_wait<RW::RA - 1>();      // chunk c's copies have landed
         if (c >= kTileStages) bar_wait(bar_xe(s));
         widen(c, s, rs);
         bar_signal(bar_xf(s));
@@ -557,86 +628,100 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
             finish(j, sf, rf);
             if (j + kTileStages < nchunks) bar_signal(bar_ye(sf));
             sf = next_stage(sf, kTileStages);
-            rf = next_stage(rf, kRawStages);
+            rf = next_stage(rf, RW::RS);
         }
-        if (c + kRawAhead < nchunks) stage_chunk(c + kRawAhead, ra);
+        if (c + RW::RA < nchunks) stage_chunk(c + RW::RA, ra);
         cp_async_commit();
         s = next_stage(s, kTileStages);
-        rs = next_stage(rs, kRawStages);
-        ra = next_stage(ra, kRawStages);
+        rs = next_stage(rs, RW::RS);
+        ra = next_stage(ra, RW::RS);
     }
     for (int64_t j = max64(nchunks - (kTileStages - 1), 0); j < nchunks; ++j) {
         bar_wait(bar_yf(sf));
         finish(j, sf, rf);
         sf = next_stage(sf, kTileStages);
-        rf = next_stage(rf, kRawStages);
+        rf = next_stage(rf, RW::RS);
     }
     cp_async_wait<0>();
 }
 
-template <typename T, int LPR, bool VEC>
+template <typename T, int LPR, bool VEC, bool CONV>
 __global__ void __launch_bounds__(kThreads, Shape<LPR>::MINB) rec_kernel(const ScanParams p) {
     extern __shared__ __align__(16) unsigned char smem[];
     if (threadIdx.x < kScanThreads) {
         recurrence_role<T, LPR>(p, smem, threadIdx.x);
     } else {
-        io_role<T, LPR, VEC>(p, smem, threadIdx.x - kScanThreads);
+        io_role<T, LPR, VEC, CONV>(p, smem, threadIdx.x - kScanThreads);
     }
 }
 
 template <typename T, int LPR>
-const void *rec_ptr(bool vec) {
-    return vec ? reinterpret_cast<const void *>(rec_kernel<T, LPR, true>)
-               : reinterpret_cast<const void *>(rec_kernel<T, LPR, false>);
+const void *rec_ptr(bool vec, bool conv) {
+    if constexpr (LPR == 2 || LPR == 4) {   // the convolution prologue needs 16-byte pieces
+        if (conv)
+            return vec ? reinterpret_cast<const void *>(rec_kernel<T, LPR, true, true>)
+                       : reinterpret_cast<const void *>(rec_kernel<T, LPR, false, true>);
+    }
+    return vec ? reinterpret_cast<const void *>(rec_kernel<T, LPR, true, false>)
+               : reinterpret_cast<const void *>(rec_kernel<T, LPR, false, false>);
 }
 
 template <typename T>
-const void *rec_select(int lpr, bool vec) {
+const void *rec_select(int lpr, bool vec, bool conv) {
     switch (lpr) {
-        case 2: return rec_ptr<T, 2>(vec);
-        case 4: return rec_ptr<T, 4>(vec);
-        case 8: return rec_ptr<T, 8>(vec);
-        default: return rec_ptr<T, 16>(vec);
+        case 2: return rec_ptr<T, 2>(vec, conv);
+        case 4: return rec_ptr<T, 4>(vec, conv);
+        case 8: return rec_ptr<T, 8>(vec, conv);
+        default: return rec_ptr<T, 16>(vec, conv);
     }
 }
 
-const void *rec_kernel_for(int in_dtype, int lpr, bool vec) {
-    return in_dtype == 0 ? rec_select<float>(lpr, vec) : rec_select<__nv_bfloat16>(lpr, vec);
+const void *rec_kernel_for(int in_dtype, int lpr, bool vec, bool conv) {
+    return in_dtype == 0 ? rec_select<float>(lpr, vec, conv) : rec_select<__nv_bfloat16>(lpr, vec, conv);
+}
+
+template <typename T, int LPR>
+int smem_bytes_lpr(bool conv) {
+    if constexpr (LPR == 2 || LPR == 4) {
+        if (conv) return Raw<T, LPR, true>::BYTES;
+    }
+    return Raw<T, LPR, false>::BYTES;
+}
+
+template <typename T>
+int smem_bytes_t(int lpr, bool conv) {
+    switch (lpr) {
+        case 2: return smem_bytes_lpr<T, 2>(conv);
+        case 4: return smem_bytes_lpr<T, 4>(conv);
+        case 8: return smem_bytes_lpr<T, 8>(conv);
+        default: return smem_bytes_lpr<T, 16>(conv);
+    }
 }
 
 }  // namespace
 
-template <typename T>
-int smem_bytes_t(int lpr) {
-    switch (lpr) {
-        case 2: return Raw<T, 2>::BYTES;
-        case 4: return Raw<T, 4>::BYTES;
-        case 8: return Raw<T, 8>::BYTES;
-        default: return Raw<T, 16>::BYTES;
-    }
+int rec_smem_bytes(int in_dtype, int lpr, bool conv) {
+    return in_dtype == 0 ? smem_bytes_t<float>(lpr, conv) : smem_bytes_t<__nv_bfloat16>(lpr, conv);
 }
 
-int rec_smem_bytes(int in_dtype, int lpr) {
-    return in_dtype == 0 ? smem_bytes_t<float>(lpr) : smem_bytes_t<__nv_bfloat16>(lpr);
-}
-
+bool rec_supports_conv(int lpr) { return lpr == 2 || lpr == 4; }
 int rec_chunk() { return kSteps; }
 int rec_threads() { return kThreads; }
 int rec_rows(int lpr) { return kScanThreads / lpr; }
 
 // Resident CTAs per SM of a sequential kernel (cached per kernel; the
 // shared-memory bound when no device answers).
-int rec_ctas_per_sm(int in_dtype, int lpr, bool vec) {
-    constexpr int kSlots = 32;
+int rec_ctas_per_sm(int in_dtype, int lpr, bool vec, bool conv) {
+    constexpr int kSlots = 64;
     static const void *keys[kSlots];
     static int vals[kSlots];
     static int used = 0;
     static std::mutex mu;
-    const void *k = rec_kernel_for(in_dtype, lpr, vec);
+    const void *k = rec_kernel_for(in_dtype, lpr, vec, conv);
     std::lock_guard<std::mutex> lk(mu);
     for (int i = 0; i < used; ++i)
         if (keys[i] == k) return vals[i];
-    const int smem = rec_smem_bytes(in_dtype, lpr);
+    const int smem = rec_smem_bytes(in_dtype, lpr, conv);
     int n = 0;
     bool asked = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess &&
                  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, kThreads, smem) == cudaSuccess;
@@ -652,8 +737,10 @@ int rec_ctas_per_sm(int in_dtype, int lpr, bool vec) {
 }
 
 cudaError_t launch_rec(const ScanParams &p, int lpr, bool vec, int in_dtype, cudaStream_t stream) {
-    const void *k = rec_kernel_for(in_dtype, lpr, vec);
-    const int smem = rec_smem_bytes(in_dtype, lpr);
+    const bool conv = p.conv_w != nullptr;
+    if (conv && !rec_supports_conv(lpr)) return cudaErrorInvalidValue;
+    const void *k = rec_kernel_for(in_dtype, lpr, vec, conv);
+    const int smem = rec_smem_bytes(in_dtype, lpr, conv);
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const int R = kScanThreads / lpr;

@@ -1,4 +1,6 @@
-// Single-token selective state update (decode) for sm_100a.
+// Single-token selective state update (decode) for sm_100a, optionally with
+// the causal depthwise convolution prologue in front ("Notas sobre Mamba",
+// section "O bloco Mamba": short convolution + SiLU before the SSM).
 //
 // The recurrence for one step ("Mamba-2 e State Space Duality (SSD)", section
 // "Como o Mamba-1 alcançou complexidade linear", the decode step; "Notas sobre
@@ -44,11 +46,34 @@ __device__ __forceinline__ float4 ldg4(const T *p) {
     }
 }
 
+// Convolution prologue of one decode step for row (b, d): the state
+// (conv_width inputs, oldest first) drops its oldest entry and takes x; the
+// return value is act(bias + sum_k w[k] window[k]). Called by one lane per row.
+template <typename T>
+__device__ __forceinline__ float conv_step(const UpdateParams &p, int64_t b, int64_t d, float x, bool store) {
+    T *cs = static_cast<T *>(p.conv_state) + b * p.cs_sb + d * p.cs_sd;
+    const int K = p.conv_width;
+    const float *w = p.conv_w + d * K;
+    float acc = p.conv_b ? __ldg(p.conv_b + d) : 0.f;
+    float prev[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) prev[j] = (j + 1 < K) ? to_f32<T>(cs[j + 1]) : 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        if (j < K) {
+            const float v = (j + 1 < K) ? prev[j] : x;
+            acc = fmaf(__ldg(w + j), v, acc);
+            if (store) cs[j] = from_f32<T>(v);
+        }
+    }
+    return p.conv_silu ? silu(acc) : acc;
+}
+
 // VEC: dstate == 16 with state rows, A rows and B/C rows aligned for vector
 // access. A thread owns state entries [4q, 4q+4) of kRowsPerThread rows and
 // issues all of their loads before any arithmetic, so that enough bytes are in
 // flight to cover HBM latency.
-template <typename T, bool VEC, int kRowsPerThread>
+template <typename T, bool VEC, int kRowsPerThread, bool CONV>
 __global__ void __launch_bounds__(kBlock) state_update_kernel(const UpdateParams p) {
     constexpr int kRowsPerBlock = kRowGroups * kRowsPerThread;
     const int tid = threadIdx.x;
@@ -67,6 +92,13 @@ __global__ void __launch_bounds__(kBlock) state_update_kernel(const UpdateParams
         dd[k] = ok[k] ? d : p.dim - 1;
         x[k] = ldg1<T>(p.x, b * p.x_sb + dd[k]);
         dt[k] = ldg1<T>(p.delta, b * p.dl_sb + dd[k]);
+        if constexpr (CONV) {
+            // the row's first lane steps the convolution state; u reaches the
+            // other three lanes of the row by shuffle
+            float u = 0.f;
+            if (q == 0) u = conv_step<T>(p, b, dd[k], x[k], ok[k]);
+            x[k] = __shfl_sync(0xffffffffu, u, (tid & 31) & ~3);
+        }
     }
     if constexpr (VEC) {
         float4 h[kRowsPerThread], a[kRowsPerThread];
@@ -135,10 +167,13 @@ cudaError_t launch_t(const UpdateParams &p, cudaStream_t stream) {
     constexpr int kRows = 1;   // rows per thread (occupancy beats per-thread batching here)
     const dim3 grid(static_cast<unsigned>((p.dim + kRowGroups * kRows - 1) / (kRowGroups * kRows)),
                     static_cast<unsigned>(p.batch));
+    const bool conv = p.conv_w != nullptr;
     if (vec)
-        state_update_kernel<T, true, kRows><<<grid, kBlock, 0, stream>>>(p);
+        conv ? state_update_kernel<T, true, kRows, true><<<grid, kBlock, 0, stream>>>(p)
+             : state_update_kernel<T, true, kRows, false><<<grid, kBlock, 0, stream>>>(p);
     else
-        state_update_kernel<T, false, kRows><<<grid, kBlock, 0, stream>>>(p);
+        conv ? state_update_kernel<T, false, kRows, true><<<grid, kBlock, 0, stream>>>(p)
+             : state_update_kernel<T, false, kRows, false><<<grid, kBlock, 0, stream>>>(p);
     return cudaGetLastError();
 }
 

@@ -41,7 +41,8 @@ BASE_SEED = 20261202
 
 # One draw stream per tensor, so that the value of a tensor does not depend on
 # which other tensors were drawn.
-_STREAM = {"u": 1, "delta": 2, "B": 3, "C": 4, "z": 5, "D": 6, "dt": 7, "h0": 8}
+_STREAM = {"u": 1, "delta": 2, "B": 3, "C": 4, "z": 5, "D": 6, "dt": 7, "h0": 8, "conv_w": 9, "conv_b": 10,
+           "conv_state": 11}
 _CHUNK = 1 << 22
 
 
@@ -240,3 +241,20 @@ def make_decode_step(w: DecodeWorkload, step: int, *, batch=None, dim=None, dsta
         "C": _store(_normal((bt, ns), sd, _STREAM["C"]), dt_),
         "z": _store(_normal((bt, dm), sd, _STREAM["z"]), dt_) if hz else None,
     }
+
+
+def make_conv_params(dim: int, width: int = 4, seed: int = BASE_SEED) -> dict:
+    """Depthwise convolution taps (dim, width) and bias (dim,), float32, drawn
+    U(-1/sqrt(width), 1/sqrt(width)) like a default-initialised depthwise
+    Conv1d (fan-in = width)."""
+    bound = 1.0 / np.sqrt(width)
+    gw = default_rng(SeedSequence(seed, spawn_key=(_STREAM["conv_w"],)))
+    gb = default_rng(SeedSequence(seed, spawn_key=(_STREAM["conv_b"],)))
+    return {"conv_w": gw.uniform(-bound, bound, size=(dim, width)).astype(np.float32),
+            "conv_b": gb.uniform(-bound, bound, size=dim).astype(np.float32)}
+
+
+def make_conv_state(batch: int, dim: int, width: int, dtype: str, seed: int = BASE_SEED) -> np.ndarray:
+    """A convolution state (batch, dim, width) of N(0,1) inputs in the storage
+    dtype (float32, or bf16 bits)."""
+    return _store(_normal((batch, dim, width), seed, _STREAM["conv_state"]), dtype)

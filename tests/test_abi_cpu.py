@@ -31,7 +31,8 @@ def declared_functions():
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
-    for want in ("mamba_scan_fwd", "mamba_state_update", "mamba_scan_workspace_size",
+    for want in ("mamba_scan_fwd", "mamba_state_update", "mamba_scan_workspace_size", "mamba_conv_scan_fwd",
+                 "mamba_conv_state_update",
                  "mamba_status_string", "mamba_last_error", "mamba_abi_version"):
         assert want in names
 
@@ -143,3 +144,40 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(ms, "_LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="not built"):
         ms.load_library()
+
+
+def _valid_conv():
+    c = ms.Conv1dArgs()
+    c.weight, c.bias, c.width, c.silu = (1 << 20) * 9, (1 << 20) * 10, 4, 1
+    return c
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("weight", None, 1), ("width", 0, 1), ("width", 5, 2), ("silu", 2, 1), ("weight", (1 << 20) * 9 + 2, 3),
+    ("bias", (1 << 20) * 10 + 1, 3),
+])
+def test_conv_scan_validation_rejects(lib, field, value, status):
+    c = _valid_conv()
+    setattr(c, field, value)
+    assert lib.mamba_conv_scan_fwd(ctypes.byref(_valid_scan_args()), ctypes.byref(c), None, None) == status
+    assert lib.mamba_last_error().decode() != ""
+
+
+def test_conv_scan_null_and_segments(lib):
+    assert lib.mamba_conv_scan_fwd(ctypes.byref(_valid_scan_args()), None, None, None) == 1
+    a = _valid_scan_args()
+    a.force_segments = 2
+    assert lib.mamba_conv_scan_fwd(ctypes.byref(a), ctypes.byref(_valid_conv()), None, None) == 2
+    a = _valid_scan_args()
+    a.dstate = 0
+    assert lib.mamba_conv_scan_fwd(ctypes.byref(a), ctypes.byref(_valid_conv()), None, None) == 1
+
+
+@pytest.mark.parametrize("state,sb,sd,status", [
+    (None, 32, 4, 1), ((1 << 20) * 11, -1, 4, 1), ((1 << 20) * 11, 32, -4, 1), ((1 << 20) * 11 + 1, 32, 4, 3),
+])
+def test_conv_state_update_validation_rejects(lib, state, sb, sd, status):
+    rc = lib.mamba_conv_state_update(ctypes.byref(_valid_update_args()), ctypes.byref(_valid_conv()), state,
+                                     sb, sd, None)
+    assert rc == status
+    assert lib.mamba_conv_state_update(ctypes.byref(_valid_update_args()), None, (1 << 20) * 11, 32, 4, None) == 1
