@@ -60,6 +60,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU-baseline budget (seconds of oracle work on rank 0)")
+    ap.add_argument("--prologue-steps", type=int, default=200,
+                    help="steps of the scan with the fused convolution prologue (0 skips the leg)")
     ap.add_argument("--decode-steps", type=int, default=1000,
                     help="decode state-update steps timed on the (256, 5120, 16) decode workload (0: skip)")
     return ap.parse_args(argv)
@@ -423,6 +425,8 @@ def run_ours(args, dist: Dist):
     }
 
     decode = run_decode(args, dist, dev) if args.decode_steps > 0 else None
+    prologue = (run_prologue(args, dist, dev, w, sets, params, y, hT, counts, mufu_peak)
+                if args.prologue_steps > 0 else None)
 
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
@@ -435,7 +439,7 @@ def run_ours(args, dist: Dist):
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded)", "config": workload_config(w, {"global_batch": w.batch * dist.world}),
-        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode,
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode, "conv_prologue": prologue,
         "gpu_launches": args.steps * launches_per_step, "clocks": clocks,
     }
     if dist.rank == 0:
@@ -443,6 +447,55 @@ def run_ours(args, dist: Dist):
     dist.barrier()
     dist.close()
     return 0
+
+
+def run_prologue(args, dist: Dist, dev, w, sets, params, y, hT, counts, mufu_peak):
+    """Time the scan with the causal depthwise convolution + SiLU prologue
+    fused in front (width 4, seeded taps): the same workload and rotating input
+    sets as the headline step, with u read as the convolution input x."""
+    import ctypes
+
+    import torch
+    import selective_state_space_27_b200 as ms
+    from selective_state_space_27_b200.inputs import make_conv_params
+
+    conv_np = make_conv_params(w.dim, 4, seed=w.seed + 77)
+    conv_t = {k: torch.from_numpy(v).to(dev) for k, v in conv_np.items()}
+    conv = ms.build_conv_args(conv_t["conv_w"], conv_t["conv_b"], True)
+    argl = [ms.build_scan_args(s["u"], s["delta"], params["A"], s["B"], s["C"], y, D=params["D"], z=s.get("z"),
+                               delta_bias=params["delta_bias"], final_state=hT) for s in sets]
+    lib = ms.load_library()
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        rc = lib.mamba_conv_scan_fwd(ctypes.byref(argl[i % len(argl)]), ctypes.byref(conv), None,
+                                     stream.cuda_stream)
+        if rc != 0:
+            raise ms.MambaScanError(rc, lib.mamba_last_error().decode())
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    torch.cuda.synchronize()
+    n = args.prologue_steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(n):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    us = dist.max(e0.elapsed_time(e1) * 1e3 / n, dev)
+    rows_t = w.batch * w.dim * w.seqlen
+    mufu = counts["mufu"] + 2 * rows_t          # + exp and reciprocal of the prologue's SiLU
+    return {
+        "workload": w.name, "width": 4, "silu": True, "steps": n,
+        "metric": "conv prologue + selective scan B*D*L*N elems/s", "unit": UNIT,
+        "value": dist.world * counts["elements"] / (us * 1e-6), "us_per_step": us,
+        "roofline": {"bound": "alu", "unit": "Tmufu/s", "achieved": mufu / (us * 1e-6) / 1e12,
+                     "peak": mufu_peak / 1e12, "frac": mufu / (us * 1e-6) / mufu_peak,
+                     "algorithmic_mufu": mufu,
+                     "note": "bytes as the plain scan (x replaces u); the convolution adds 4 FMA per (b, d, t)"},
+        "gpu_launches": n,
+    }
 
 
 def run_decode(args, dist: Dist, dev):
