@@ -54,6 +54,9 @@ def _bind(path: str):
     lib.s6_oracle_conv_state_update.restype = ip
     lib.s6_oracle_conv_state_update.argtypes = [i64, i64, i64, ip, vp, vp, vp, vp, vp, ip, ip, vp, vp,
                                                 vp, vp, vp, vp, vp, ip, vp, i64, vp, ip]
+    lib.s6_oracle_trap_scan.restype = ip
+    lib.s6_oracle_trap_scan.argtypes = [i64, i64, i64, i64, ip, vp, vp, vp, vp, vp, vp, vp, vp, vp, ip, vp,
+                                        i64, vp, vp, vp, ip]
     lib.s6_oracle_max_threads.restype = ip
     lib.s6_oracle_max_threads.argtypes = []
     return lib
@@ -244,6 +247,39 @@ def conv_state_update(*, state, conv_state, x, conv_w, conv_b=None, conv_silu=Tr
     return y.reshape(batch, dim) if rows is None else y
 
 
+def trap_scan(*, u, delta, lambda_raw, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
+              dtype="f32", rows=None, h0=None, threads: int = 0, _lib_override=None):
+    """Exponential-trapezoidal selective scan (Mamba-3) in fp64: as :func:`scan`
+    plus ``lambda_raw`` (batch, dim, L), the pre-activation of the gate
+    lambda = sigmoid(lambda_raw). Returns ``(y, h)``."""
+    dt = _DTYPES[dtype]
+    u, delta, lambda_raw, B, C, z = (_in(a, dt) for a in (u, delta, lambda_raw, B, C, z))
+    A, D, delta_bias = _f32(A), _f32(D), _f32(delta_bias)
+    batch, dim, L = u.shape
+    dstate = B.shape[1]
+    if delta.shape != u.shape or lambda_raw.shape != u.shape or (z is not None and z.shape != u.shape):
+        raise ValueError("u, delta, lambda_raw and z must share one (batch, dim, L) shape")
+    if B.shape != (batch, dstate, L) or C.shape != B.shape or A.shape != (dim, dstate):
+        raise ValueError("B, C must be (batch, dstate, L) and A (dim, dstate)")
+    if rows is None:
+        n_rows, rows_arr = batch * dim, None
+    else:
+        rows_arr = np.ascontiguousarray(rows, dtype=np.int64)
+        n_rows = rows_arr.size
+    h0_arr = None if h0 is None else np.ascontiguousarray(h0, dtype=np.float64).reshape(n_rows, dstate)
+    y = np.empty((n_rows, L), np.float64)
+    h = np.empty((n_rows, dstate), np.float64)
+    lib = _lib_override or _load()
+    rc = lib.s6_oracle_trap_scan(batch, dim, dstate, L, dt, _ptr(u), _ptr(delta), _ptr(lambda_raw), _ptr(A),
+                                 _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias), int(bool(delta_softplus)),
+                                 _ptr(rows_arr), n_rows, _ptr(h0_arr), _ptr(y), _ptr(h), int(threads))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    if rows is None:
+        return y.reshape(batch, dim, L), h.reshape(batch, dim, dstate)
+    return y, h
+
+
 class Variant:
     """The oracle's entry points bound to another build of the oracle source.
 
@@ -265,6 +301,9 @@ class Variant:
 
     def conv_state_update(self, **kw):
         return conv_state_update(_lib_override=self._lib, **kw)
+
+    def trap_scan(self, **kw):
+        return trap_scan(_lib_override=self._lib, **kw)
 
 
 def compile_source(src_path: str, so_path: str) -> str:

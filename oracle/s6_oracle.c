@@ -58,6 +58,14 @@
  *
  * (w[d,K-1] weighs the current input). The decode form keeps the last K
  * inputs of every row (oldest first) as its convolution state.
+ *
+ * The exponential-trapezoidal scan (s6_oracle_trap_scan) follows "Notas sobre
+ * Mamba", section "Recorrência trapezoidal" (Mamba-3):
+ *   h_t = alpha_t h_{t-1} + beta_t B_{t-1} x_{t-1} + gamma_t B_t x_t,
+ *   alpha_t = exp(delta_t A), beta_t = (1 - lambda_t) delta_t alpha_t,
+ *   gamma_t = lambda_t delta_t,  lambda_t = sigmoid(lambda_raw_t),
+ * with B_{-1} x_{-1} = 0 (the section's code starts its previous-input term
+ * at zero) and the same readout, skip and gate as the scan.
  */
 #include <math.h>
 #include <stdint.h>
@@ -340,6 +348,83 @@ int s6_oracle_conv_state_update(int64_t batch, int64_t dim, int64_t dstate, int 
                  delta_softplus, state + r * dstate, y_out + r);
     }
     return 0;
+}
+
+static double sigmoid(double v)
+{
+    return 1.0 / (1.0 + exp(-v));
+}
+
+/*
+ * Exponential-trapezoidal selective scan: as s6_oracle_scan, plus lambda_raw
+ * (batch, dim, seqlen) of dtype `dtype`, the pre-activation of the per-token
+ * mixing gate lambda = sigmoid(lambda_raw).
+ */
+int s6_oracle_trap_scan(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, int dtype,
+                        const void *u, const void *delta, const void *lambda_raw, const float *A,
+                        const void *B, const void *C, const float *D, const void *z,
+                        const float *delta_bias, int delta_softplus, const int64_t *rows, int64_t n_rows,
+                        const double *h0, double *y_out, double *h_out, int nthreads)
+{
+    if (batch < 0 || dim < 0 || dstate < 0 || seqlen < 0)
+        return -1;
+    if (dtype != ORACLE_F32 && dtype != ORACLE_BF16)
+        return -1;
+    if (!rows)
+        n_rows = batch * dim;
+    if (n_rows > 0 && (!u || !delta || !lambda_raw || !A || !B || !C || !y_out || !h_out))
+        return -1;
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const int64_t row = rows ? rows[r] : r;
+        if (row < 0 || row >= batch * dim)
+            return -1;
+    }
+    int failed = 0;
+#ifdef _OPENMP
+    if (nthreads > 0)
+        omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const int64_t row = rows ? rows[r] : r;
+        const int64_t b = row / dim, d = row % dim;
+        double *h = h_out + r * dstate;
+        double *v_prev = (double *)calloc((size_t)(dstate > 0 ? dstate : 1), sizeof(double));
+        if (!v_prev) {
+            failed = 1;
+            continue;
+        }
+        for (int64_t n = 0; n < dstate; ++n)
+            h[n] = h0 ? h0[r * dstate + n] : 0.0;
+        for (int64_t t = 0; t < seqlen; ++t) {
+            const int64_t i = row * seqlen + t;
+            const double x = load_value(u, dtype, i);
+            double dt = load_value(delta, dtype, i);
+            if (delta_bias)
+                dt += (double)delta_bias[d];
+            if (delta_softplus)
+                dt = softplus(dt);
+            const double lam = sigmoid(load_value(lambda_raw, dtype, i));
+            double acc = 0.0;
+            for (int64_t n = 0; n < dstate; ++n) {
+                const int64_t j = (b * dstate + n) * seqlen + t;
+                const double alpha = exp(dt * (double)A[d * dstate + n]);
+                const double beta = (1.0 - lam) * dt * alpha;
+                const double gamma = lam * dt;
+                const double v = load_value(B, dtype, j) * x;     /* B_t x_t */
+                h[n] = alpha * h[n] + beta * v_prev[n] + gamma * v;
+                v_prev[n] = v;
+                acc += load_value(C, dtype, j) * h[n];
+            }
+            if (D)
+                acc += (double)D[d] * x;
+            if (z)
+                acc *= silu(load_value(z, dtype, i));
+            y_out[r * seqlen + t] = acc;
+        }
+        free(v_prev);
+    }
+    return failed ? -1 : 0;
 }
 
 int s6_oracle_max_threads(void)

@@ -473,6 +473,107 @@ def pin_conv_decode_equals_scan(orc, seed=34):
     assert np.array_equal(cstate, case["x"][:, :, L - 4:].astype(np.float64))
 
 
+# ---- exponential-trapezoidal recurrence ("Notas sobre Mamba", section
+# "Recorrência trapezoidal": h_t = alpha_t h_{t-1} + beta_t B_{t-1} x_{t-1}
+# + gamma_t B_t x_t, lambda_t = sigmoid(.), B_{-1} x_{-1} = 0).
+
+def _trap_case(g, batch=2, dim=3, L=29, N=5):
+    return dict(u=_f32(g.normal(size=(batch, dim, L))), delta=_f32(g.normal(scale=0.5, size=(batch, dim, L))),
+                lambda_raw=_f32(g.normal(size=(batch, dim, L))), A=_f32(-np.exp(g.normal(size=(dim, N)))),
+                B=_f32(g.normal(size=(batch, N, L))), C=_f32(g.normal(size=(batch, N, L))),
+                D=_f32(g.uniform(0.5, 1.5, size=dim)), z=_f32(g.normal(size=(batch, dim, L))),
+                delta_bias=_f32(g.normal(size=dim) - 2.0))
+
+
+def _read_trapezoid_check():
+    rows = []
+    with open(os.path.join(GOLDEN, "trapezoid_check.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                lam, val = line.split()
+                rows.append((float(lam), float(val)))
+    return rows
+
+
+def _page_trajectories(orc, lam):
+    """The section's experiment through the oracle: one channel, N = 6 states,
+    the state trajectory read out one state at a time (C_t = e_n, no skip, no
+    gate). Returns (trapezoidal, exponential-Euler) trajectories (L, N)."""
+    g = np.random.default_rng(2)
+    L, N = 24, 6
+    A = -np.exp(g.normal(size=N))
+    B = g.normal(size=(L, N))
+    x = g.normal(size=L)
+    delta = np.exp(g.normal(size=L) * 0.3)
+    lam_raw = np.full(L, 40.0 if lam == 1.0 else 0.0)    # sigmoid(40) = 1 and sigmoid(0) = 1/2 in fp64
+    common = dict(u=_f32(x.reshape(1, 1, L)), delta=_f32(delta.reshape(1, 1, L)), A=_f32(A.reshape(1, N)),
+                  B=_f32(B.T.reshape(1, N, L)), delta_softplus=False)
+    trap = np.empty((L, N))
+    euler = np.empty((L, N))
+    for n in range(N):
+        C = np.zeros((1, N, L), np.float32)
+        C[0, n, :] = 1.0
+        trap[:, n] = orc.trap_scan(lambda_raw=_f32(lam_raw.reshape(1, 1, L)), C=C, **common)[0][0, 0]
+        euler[:, n] = orc.scan(C=C, **common)[0][0, 0]
+    return trap, euler
+
+
+def pin_trap_page_check(orc):
+    """The section's printed check: lambda = 1 reproduces exponential-Euler (to
+    rounding), lambda = 1/2 differs by 1.50 (the printed value, 2 decimals)."""
+    for lam, printed in _read_trapezoid_check():
+        trap, euler = _page_trajectories(orc, lam)
+        diff = float(np.abs(trap - euler).max())
+        if lam == 1.0:
+            assert diff <= 1e-13, diff
+        else:
+            assert f"{diff:.2e}" == f"{printed:.2e}", (diff, printed)
+
+
+def pin_trap_unrolled_sum(orc, seed=40):
+    """Brute force: h_t = sum_{s<=t} (prod_{k=s+1..t} alpha_k) (gamma_s B_s x_s
+    + beta_s B_{s-1} x_{s-1}), built from cumulative products, then y = C h +
+    D x times silu(z)."""
+    g = _rng(seed)
+    case = _trap_case(g, batch=1, dim=2, L=14, N=3)
+    y, h = orc.trap_scan(**case)
+    x = case["u"][0].astype(np.float64)
+    dr = case["delta"][0].astype(np.float64) + case["delta_bias"][:, None]
+    dt = np.logaddexp(0.0, dr)
+    lam = expit(case["lambda_raw"][0].astype(np.float64))
+    Bm = case["B"][0].astype(np.float64)          # (N, L)
+    Cm = case["C"][0].astype(np.float64)
+    L = x.shape[1]
+    for d in range(2):
+        ys = np.zeros(L)
+        for n in range(3):
+            alpha = np.exp(dt[d] * float(case["A"][d, n]))
+            beta = (1.0 - lam[d]) * dt[d] * alpha
+            gamma = lam[d] * dt[d]
+            v = Bm[n] * x[d]
+            src = gamma * v + beta * np.concatenate([[0.0], v[:-1]])
+            ht = np.array([sum(np.prod(alpha[s + 1:t + 1]) * src[s] for s in range(t + 1)) for t in range(L)])
+            ys += Cm[n] * ht
+            assert abs(ht[-1] - h[0, d, n]) <= 1e-12 * max(1.0, abs(ht[-1]))
+        zz = case["z"][0, d].astype(np.float64)
+        ys = (ys + float(case["D"][d]) * x[d]) * zz * expit(zz)
+        assert _rel(y[0, d], ys) <= 1e-12
+
+
+def pin_trap_linearity(orc, seed=41):
+    """Linear in x for fixed delta, lambda, B, C (no gate)."""
+    g = _rng(seed)
+    case = _trap_case(g)
+    case["z"] = None
+    x1, x2 = case.pop("u"), _f32(g.normal(size=case["delta"].shape))
+    a, b = 0.75, -1.25
+    y1, h1 = orc.trap_scan(u=x1, **case)
+    y2, h2 = orc.trap_scan(u=x2, **case)
+    y3, h3 = orc.trap_scan(u=_f32(a * x1.astype(np.float64) + b * x2.astype(np.float64)), **case)
+    assert _rel(y3, a * y1 + b * y2) <= 1e-6 and _rel(h3, a * h1 + b * h2) <= 1e-6
+
+
 ALL_PINS = [
     pin_selection_step,
     pin_lti_convolution,
@@ -492,4 +593,7 @@ ALL_PINS = [
     pin_conv_identity_filter_is_plain_scan,
     pin_conv_output_feeds_scan,
     pin_conv_decode_equals_scan,
+    pin_trap_page_check,
+    pin_trap_unrolled_sum,
+    pin_trap_linearity,
 ]

@@ -10,7 +10,8 @@ from tests import oracle_pins
 
 # (name, text in s6_oracle.c, replacement)
 MUTANTS = [
-    ("drop_skip_term", "acc += (double)D[d] * x;", "acc += 0.0 * x;"),
+    ("drop_skip_term", "acc += (double)D[d] * x;\n        if (z)\n            acc *= silu(load_value(z, dtype, i));\n        y[t] = acc;",
+     "acc += 0.0 * x;\n        if (z)\n            acc *= silu(load_value(z, dtype, i));\n        y[t] = acc;"),
     ("sign_of_exponent", "exp(dt * a) * h[n]", "exp(-dt * a) * h[n]"),
     ("zoh_input_matrix", "const double Bbar = dt * load_value(B, dtype, j);",
      "const double Bbar = (exp(dt * a) - 1.0) / a * load_value(B, dtype, j);"),
@@ -20,9 +21,10 @@ MUTANTS = [
     ("bias_after_softplus",
      "if (delta_bias)\n            dt += (double)delta_bias[d];\n        if (delta_softplus)\n            dt = softplus(dt);",
      "if (delta_softplus)\n            dt = softplus(dt);\n        if (delta_bias)\n            dt += (double)delta_bias[d];"),
-    ("no_gate", "acc *= silu(load_value(z, dtype, i));", "(void)0;"),
+    ("no_gate", "acc *= silu(load_value(z, dtype, i));\n        y[t] = acc;", "(void)0;\n        y[t] = acc;"),
     ("sigmoid_not_silu", "return v / (1.0 + exp(-v));", "return 1.0 / (1.0 + exp(-v));"),
-    ("transition_index_transposed", "(double)A[d * dstate + n]", "(double)A[n * dim + d]"),
+    ("transition_index_transposed", "const double a = (double)A[d * dstate + n];",
+     "const double a = (double)A[n * dim + d];"),
     ("input_index_uses_state_row", "const double Bbar = dt * load_value(B, dtype, j);",
      "const double Bbar = dt * load_value(B, dtype, (b * dstate + n) * seqlen + (seqlen - 1 - t));"),
     ("softplus_is_exp", "return v > 20.0 ? v : log1p(exp(v));", "return v > 20.0 ? v : exp(v);"),
@@ -37,6 +39,12 @@ MUTANTS = [
     ("conv_no_silu", "u_row[t] = conv_silu ? silu(acc) : acc;", "u_row[t] = acc;"),
     ("conv_bias_dropped", "double acc = bias;", "double acc = 0.0 * bias;"),
     ("conv_state_not_shifted", "cs[k] = cs[k + 1];", "cs[k] = cs[k];"),
+    ("trap_beta_without_decay", "const double beta = (1.0 - lam) * dt * alpha;",
+     "const double beta = (1.0 - lam) * dt;"),
+    ("trap_gate_weights_swapped", "const double gamma = lam * dt;", "const double gamma = (1.0 - lam) * dt;"),
+    ("trap_previous_input_frozen", "v_prev[n] = v;", "v_prev[n] = 0.0 * v;"),
+    ("trap_no_sigmoid", "const double lam = sigmoid(load_value(lambda_raw, dtype, i));",
+     "const double lam = load_value(lambda_raw, dtype, i);"),
     ("conv_decode_taps_reversed", "acc += (double)conv_w[d * width + k] * cs[k];",
      "acc += (double)conv_w[d * width + width - 1 - k] * cs[k];"),
 ]
