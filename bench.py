@@ -62,6 +62,8 @@ def parse_args(argv=None):
                     help="CPU-baseline budget (seconds of oracle work on rank 0)")
     ap.add_argument("--prologue-steps", type=int, default=200,
                     help="steps of the scan with the fused convolution prologue (0 skips the leg)")
+    ap.add_argument("--trap-steps", type=int, default=200,
+                    help="steps of the exponential-trapezoidal scan (0 skips the leg)")
     ap.add_argument("--decode-steps", type=int, default=1000,
                     help="decode state-update steps timed on the (256, 5120, 16) decode workload (0: skip)")
     return ap.parse_args(argv)
@@ -427,6 +429,7 @@ def run_ours(args, dist: Dist):
     decode = run_decode(args, dist, dev) if args.decode_steps > 0 else None
     prologue = (run_prologue(args, dist, dev, w, sets, params, y, hT, counts, mufu_peak)
                 if args.prologue_steps > 0 else None)
+    trap = run_trap(args, dist, dev, w, sets, params, y, hT, counts, mufu_peak) if args.trap_steps > 0 else None
 
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
@@ -440,6 +443,7 @@ def run_ours(args, dist: Dist):
         "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded)", "config": workload_config(w, {"global_batch": w.batch * dist.world}),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode, "conv_prologue": prologue,
+        "trapezoidal": trap,
         "gpu_launches": args.steps * launches_per_step, "clocks": clocks,
     }
     if dist.rank == 0:
@@ -494,6 +498,51 @@ def run_prologue(args, dist: Dist, dev, w, sets, params, y, hT, counts, mufu_pea
                      "peak": mufu_peak / 1e12, "frac": mufu / (us * 1e-6) / mufu_peak,
                      "algorithmic_mufu": mufu,
                      "note": "bytes as the plain scan (x replaces u); the convolution adds 4 FMA per (b, d, t)"},
+        "gpu_launches": n,
+    }
+
+
+def run_trap(args, dist: Dist, dev, w, sets, params, y, hT, counts, mufu_peak):
+    """Time the exponential-trapezoidal scan (Mamba-3) on the headline workload
+    and input sets, with a seeded lambda_raw ~ N(0, 1) per (b, d, t)."""
+    import ctypes
+
+    import torch
+    import selective_state_space_27_b200 as ms
+    from selective_state_space_27_b200.inputs import make_lambda_raw
+
+    lam_np = make_lambda_raw(w.batch, w.dim, w.seqlen, w.dtype, seed=w.seed + 1000 * dist.rank + 91)
+    lam = torch.from_numpy(lam_np)
+    lam = (lam.view(torch.bfloat16) if w.dtype == "bf16" else lam).to(dev)
+    argl = [ms.build_scan_args(s["u"], s["delta"], params["A"], s["B"], s["C"], y, D=params["D"], z=s.get("z"),
+                               delta_bias=params["delta_bias"], final_state=hT) for s in sets]
+    lib = ms.load_library()
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        rc = lib.mamba_trap_scan_fwd(ctypes.byref(argl[i % len(argl)]), lam.data_ptr(), lam.stride(0),
+                                     lam.stride(1), None, stream.cuda_stream)
+        if rc != 0:
+            raise ms.MambaScanError(rc, lib.mamba_last_error().decode())
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    torch.cuda.synchronize()
+    n = args.trap_steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(n):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    us = dist.max(e0.elapsed_time(e1) * 1e3 / n, dev)
+    mufu = counts["mufu"] + 2 * w.batch * w.dim * w.seqlen      # + exp and reciprocal of lambda's sigmoid
+    return {
+        "workload": w.name, "steps": n, "metric": "trapezoidal selective scan B*D*L*N elems/s", "unit": UNIT,
+        "value": dist.world * counts["elements"] / (us * 1e-6), "us_per_step": us,
+        "roofline": {"bound": "alu", "unit": "Tmufu/s", "achieved": mufu / (us * 1e-6) / 1e12,
+                     "peak": mufu_peak / 1e12, "frac": mufu / (us * 1e-6) / mufu_peak, "algorithmic_mufu": mufu,
+                     "note": "bytes as the plain scan + lambda_raw read once"},
         "gpu_launches": n,
     }
 

@@ -288,6 +288,27 @@ ms_status mamba_conv_state_update(const ms_update_args *args, const ms_conv1d_ar
                                   int64_t conv_state_batch_stride, int64_t conv_state_dim_stride,
                                   void *stream);
 
+/*
+ * Exponential-trapezoidal selective scan (Mamba-3; "Notas sobre Mamba",
+ * section "Recorrência trapezoidal"):
+ *     h_t = alpha_t h_{t-1} + beta_t B_{t-1} u_{t-1} + gamma_t B_t u_t,
+ *     alpha_t = exp(delta_t A), beta_t = (1 - lambda_t) delta_t alpha_t,
+ *     gamma_t = lambda_t delta_t,  lambda_t = sigmoid(lambda_raw_t),
+ * with B_{-1} u_{-1} = 0, and the readout, skip term and gate of
+ * mamba_scan_fwd. lambda_raw is (batch, dim, seqlen) in the input dtype, one
+ * value per (b, d, t), contiguous along t, with element strides
+ * lambda_batch_stride and lambda_dim_stride. lambda = 1 everywhere is the
+ * exponential-Euler scan of mamba_scan_fwd. A nonzero initial state is the
+ * state before t = 0; the previous-input term still starts at zero. Runs on the
+ * sequential kernels with 2 or 4 lanes per row, in one segment, with no
+ * workspace; `plan` is NULL (automatic) or one of those configurations.
+ * Errors: as mamba_scan_fwd; MS_ERR_INVALID_ARG for a NULL lambda_raw or
+ * negative strides; MS_ERR_UNSUPPORTED for force_segments > 1 or a plan that
+ * cannot run the rule; MS_ERR_ALIGNMENT for a misaligned lambda_raw.
+ */
+ms_status mamba_trap_scan_fwd(const ms_scan_args *args, const void *lambda_raw, int64_t lambda_batch_stride,
+                              int64_t lambda_dim_stride, const ms_scan_plan *plan, void *stream);
+
 /* Size of the device array behind mamba_scan_fwd_noalloc (8 MiB per GPU). */
 #define MS_NOALLOC_SCRATCH_BYTES (8u << 20)
 

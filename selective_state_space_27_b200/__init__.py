@@ -24,7 +24,7 @@ import os
 __all__ = [
     "scan_fwd", "state_update", "scan_workspace_size", "scan_plan", "scan_configs", "library_path",
     "load_library", "MambaScanError", "ScanArgs", "UpdateArgs", "ScanPlan", "MS_F32", "MS_BF16",
-    "Conv1dArgs", "conv_scan_fwd", "conv_state_update", "build_conv_args",
+    "Conv1dArgs", "conv_scan_fwd", "conv_state_update", "build_conv_args", "trap_scan_fwd",
     "MAX_DSTATE",
 ]
 
@@ -128,6 +128,9 @@ def load_library():
         lib.mamba_conv_state_update.restype = ctypes.c_int
         lib.mamba_conv_state_update.argtypes = [ctypes.POINTER(UpdateArgs), ctypes.POINTER(Conv1dArgs), _vp,
                                                 ctypes.c_int64, ctypes.c_int64, _vp]
+        lib.mamba_trap_scan_fwd.restype = ctypes.c_int
+        lib.mamba_trap_scan_fwd.argtypes = [ctypes.POINTER(ScanArgs), _vp, ctypes.c_int64, ctypes.c_int64,
+                                            ctypes.POINTER(ScanPlan), _vp]
         lib.mamba_scan_config_kind.restype = ctypes.c_int
         lib.mamba_scan_config_kind.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
         lib.mamba_scan_plan_query.restype = ctypes.c_int
@@ -410,3 +413,25 @@ def conv_state_update(state, conv_state, x, conv_weight, delta, A, B, C, D=None,
                                                       conv_state.stride(0), conv_state.stride(1),
                                                       _stream_ptr(stream)))
     return y
+
+
+def trap_scan_fwd(u, delta, lambda_raw, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
+                  initial_state=None, return_last_state=True, out=None, stream=None, plan=None):
+    """Exponential-trapezoidal selective scan (Mamba-3): as :func:`scan_fwd`
+    plus ``lambda_raw`` (batch, dim, L) in u's dtype, lambda = sigmoid(lambda_raw)
+    mixing the previous and the current input (no segments)."""
+    torch = _torch()
+    _need_cuda("lambda_raw", lambda_raw, u.dtype, 3)
+    if tuple(lambda_raw.shape) != tuple(u.shape):
+        raise ValueError("lambda_raw must have u's shape")
+    y = torch.empty_like(u) if out is None else out
+    hT = None
+    if return_last_state:
+        hT = torch.empty((u.shape[0], u.shape[1], B.shape[1]), device=u.device, dtype=torch.float32)
+    args = build_scan_args(u, delta, A, B, C, y, D=D, z=z, delta_bias=delta_bias, delta_softplus=delta_softplus,
+                           initial_state=initial_state, final_state=hT)
+    with torch.cuda.device(u.device):
+        _check(load_library().mamba_trap_scan_fwd(ctypes.byref(args), _ptr(lambda_raw), lambda_raw.stride(0),
+                                                  lambda_raw.stride(1), None if plan is None else ctypes.byref(plan),
+                                                  _stream_ptr(stream)))
+    return (y, hT) if return_last_state else y

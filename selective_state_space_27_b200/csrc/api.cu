@@ -367,4 +367,42 @@ ms_status mamba_conv_scan_fwd(const ms_scan_args *args, const ms_conv1d_args *co
     return run_plan(p, pl, args->in_dtype, nullptr, 0, stream);
 }
 
+ms_status mamba_trap_scan_fwd(const ms_scan_args *args, const void *lambda_raw, int64_t lambda_batch_stride,
+                              int64_t lambda_dim_stride, const ms_scan_plan *plan, void *stream) {
+    ms_status st = check_scan(args);
+    if (st != MS_OK) return st;
+    if (!lambda_raw) return invalid("lambda_raw is required");
+    if (lambda_batch_stride < 0 || lambda_dim_stride < 0) return invalid("lambda strides must be non-negative");
+    if (!elem_aligned(lambda_raw, args->in_dtype == MS_F32 ? 4 : 2)) {
+        set_error("lambda_raw is not aligned to its element size");
+        return MS_ERR_ALIGNMENT;
+    }
+    if (args->force_segments > 1) {
+        set_error("the trapezoidal rule runs in one segment (force_segments %d)", args->force_segments);
+        return MS_ERR_UNSUPPORTED;
+    }
+    ms::ScanParams p = to_params(args);
+    p.lambda_raw = lambda_raw;
+    p.lm_sb = lambda_batch_stride;
+    p.lm_sd = lambda_dim_stride;
+    ms::ScanPlan pl{};
+    if (plan) {
+        if (!ms::make_plan(p, args->in_dtype, plan->config, plan->warps_per_cta, plan->segments, &pl)) {
+            set_error("plan (config %d, %d warps, %d segments) cannot run the trapezoidal rule", plan->config,
+                      plan->warps_per_cta, plan->segments);
+            return MS_ERR_UNSUPPORTED;
+        }
+    } else {
+        int sms = 0;
+        st = device_sms(&sms);
+        if (st != MS_OK) return st;
+        pl = ms::plan_scan(p, args->in_dtype, 0, sms);
+        if (pl.kind != 1) {
+            set_error("no kernel configuration runs the trapezoidal rule for these arguments");
+            return MS_ERR_UNSUPPORTED;
+        }
+    }
+    return run_plan(p, pl, args->in_dtype, nullptr, 0, stream);
+}
+
 }  // extern "C"

@@ -27,6 +27,11 @@ struct ScanParams {
     // act(conv_b[d] + sum_k conv_w[d*conv_width + k] x[t - conv_width + 1 + k]).
     const float *conv_w, *conv_b;
     int conv_width, conv_silu;
+    // Exponential-trapezoidal recurrence (sequential kernels only): when set,
+    // lambda = sigmoid(lambda_raw) per (b, d, t) mixes the previous and the
+    // current input, h_t = a_t h_{t-1} + (1-lambda_t) delta_t a_t B_{t-1} u_{t-1}
+    // + lambda_t delta_t B_t u_t.
+    const void *lambda_raw; int64_t lm_sb, lm_sd;
 };
 
 // Launch configuration chosen on the host for one scan call.
@@ -44,8 +49,9 @@ struct ScanPlan {
     size_t ws_bytes;
 };
 
-// With p.conv_w set only the sequential configurations that fuse the
-// convolution prologue (lanes 2 and 4) are considered.
+// With p.conv_w or p.lambda_raw set only the sequential configurations that
+// fuse the convolution prologue or run the trapezoidal rule (lanes 2 and 4)
+// are considered.
 ScanPlan plan_scan(const ScanParams &p, int in_dtype, int force_segments, int num_sms);
 // A plan with a fixed configuration, CTA size and segment count; returns false
 // (and leaves `out` unspecified) when the configuration cannot run `p`.
@@ -58,12 +64,14 @@ cudaError_t launch_scan(const ScanParams &p, const ScanPlan &plan, int in_dtype,
 
 // Sequential kernels (scan_rec.cu): CTAs of rec_threads() threads (recurrence
 // and I/O warps) owning rec_rows(lanes_per_row) rows, no workspace, one segment.
-int rec_smem_bytes(int in_dtype, int lanes_per_row, bool conv);
+// Variants of the sequential kernel: 0 plain, 1 convolution prologue, 2 trapezoidal rule.
+int rec_variant(const ScanParams &p);
+int rec_smem_bytes(int in_dtype, int lanes_per_row, int variant);
 int rec_chunk();
 int rec_threads();
 int rec_rows(int lanes_per_row);
-int rec_ctas_per_sm(int in_dtype, int lanes_per_row, bool vec, bool conv);
-bool rec_supports_conv(int lanes_per_row);
+int rec_ctas_per_sm(int in_dtype, int lanes_per_row, bool vec, int variant);
+bool rec_supports_variant(int lanes_per_row, int variant);
 cudaError_t launch_rec(const ScanParams &p, int lanes_per_row, bool vec, int in_dtype, cudaStream_t stream);
 
 struct UpdateParams {

@@ -635,12 +635,14 @@ ScanPlan plan_scan(const ScanParams &p, int in_dtype, int force_segments, int nu
     plan.vec = aligned16(p.u) && aligned16(p.delta) && aligned16(p.B) && aligned16(p.C) &&
                aligned16(p.y) && (p.z == nullptr || aligned16(p.z)) && strides_ok(p.u_sb, p.u_sd) &&
                strides_ok(p.dl_sb, p.dl_sd) && strides_ok(p.B_sb, p.B_sn) && strides_ok(p.C_sb, p.C_sn) &&
-               strides_ok(p.y_sb, p.y_sd) && (p.z == nullptr || strides_ok(p.z_sb, p.z_sd));
+               strides_ok(p.y_sb, p.y_sd) && (p.z == nullptr || strides_ok(p.z_sb, p.z_sd)) &&
+               (p.lambda_raw == nullptr || (aligned16(p.lambda_raw) && strides_ok(p.lm_sb, p.lm_sd)));
 
     const int sms = num_sms > 0 ? num_sms : 148;
-    const bool conv = p.conv_w != nullptr;   // only sequential kernels fuse the convolution prologue
+    // only sequential kernels fuse the convolution prologue or run the trapezoidal rule
+    const int variant = rec_variant(p);
     double best = 1e300;
-    for (int ci = 0; ci < (conv ? 0 : kNumConfigs); ++ci) {
+    for (int ci = 0; ci < (variant ? 0 : kNumConfigs); ++ci) {
         const Config cf = kConfigs[ci];
         if (cf.ni != 1 && !plan.vec) continue;
         if (cf.ni == 0 && p.dstate != kMaxN) continue;
@@ -685,8 +687,8 @@ ScanPlan plan_scan(const ScanParams &p, int in_dtype, int force_segments, int nu
         best *= kChunkedClocksPerUnit;
         for (int ri = 0; ri < kNumRec; ++ri) {
             const int lpr = kRecLanes[ri];
-            if (conv && !rec_supports_conv(lpr)) continue;
-            const int per_sm = rec_ctas_per_sm(in_dtype, lpr, plan.vec, conv);
+            if (!rec_supports_variant(lpr, variant)) continue;
+            const int per_sm = rec_ctas_per_sm(in_dtype, lpr, plan.vec, variant);
             if (per_sm < 1) continue;
             const int64_t R = rec_rows(lpr);
             const int64_t ctas = p.batch * ((p.dim + R - 1) / R);
@@ -714,7 +716,7 @@ bool make_plan(const ScanParams &p, int in_dtype, int config, int warps, int seg
     if (config >= kNumConfigs && config < kNumConfigs + kNumRec) {
         // sequential kernel: fixed CTA of rec_threads(), the whole sequence in one pass
         if (warps != rec_threads() / 32 || segments != 1 || p.dstate > kMaxN) return false;
-        if (p.conv_w && !rec_supports_conv(kRecLanes[config - kNumConfigs])) return false;
+        if (!rec_supports_variant(kRecLanes[config - kNumConfigs], rec_variant(p))) return false;
         const int eb = in_dtype == 0 ? 4 : 2;
         auto strides_ok = [&](int64_t s1, int64_t s2) { return (s1 * eb) % 16 == 0 && (s2 * eb) % 16 == 0; };
         ScanPlan plan{};
@@ -727,14 +729,15 @@ bool make_plan(const ScanParams &p, int in_dtype, int config, int warps, int seg
         plan.vec = aligned16(p.u) && aligned16(p.delta) && aligned16(p.B) && aligned16(p.C) &&
                    aligned16(p.y) && (p.z == nullptr || aligned16(p.z)) && strides_ok(p.u_sb, p.u_sd) &&
                    strides_ok(p.dl_sb, p.dl_sd) && strides_ok(p.B_sb, p.B_sn) && strides_ok(p.C_sb, p.C_sn) &&
-                   strides_ok(p.y_sb, p.y_sd) && (p.z == nullptr || strides_ok(p.z_sb, p.z_sd));
+                   strides_ok(p.y_sb, p.y_sd) && (p.z == nullptr || strides_ok(p.z_sb, p.z_sd)) &&
+                   (p.lambda_raw == nullptr || (aligned16(p.lambda_raw) && strides_ok(p.lm_sb, p.lm_sd)));
         plan.nseg = 1;
         plan.seg_len = p.seqlen;
         plan.ws_bytes = 0;
         *out = plan;
         return true;
     }
-    if (config < 0 || config >= kNumConfigs || segments < 1 || p.conv_w) return false;
+    if (config < 0 || config >= kNumConfigs || segments < 1 || rec_variant(p) != 0) return false;
     const Config cf = kConfigs[config];
     ScanPlan plan{};
     const int eb = in_dtype == 0 ? 4 : 2;

@@ -65,13 +65,15 @@ constexpr int kTileStages = 3;      // step/readout tile buffers between the two
 // (32 / LPR) and state group l / (32 / LPR): a quarter-warp then reads one
 // B/C address per step. For LPR = 8 and 16 (row-major, lane l takes row
 // (32 w + l) / LPR and group l % LPR) a quarter-warp covers at most two rows.
-template <int LPR> struct Shape {
+// With the trapezoidal rule (TRAP) the step tile holds one float4 per step:
+// (delta, lambda delta u, (1 - lambda) delta u_prev, 0).
+template <int LPR, bool TRAP = false> struct Shape {
     static constexpr int NPL = kStates / LPR;           // states per lane
     static constexpr int R = kScanThreads / LPR;        // rows per CTA
     static constexpr int IPR = LPR / 2;                 // I/O threads per row
     static constexpr int IP = kSteps / IPR;             // steps per I/O thread
     static constexpr bool GROUP_MAJOR = LPR <= 4;
-    static constexpr int XR = kSteps / 2 + 1;           // float4 per row of the step tile
+    static constexpr int XR = TRAP ? kSteps + 1 : kSteps / 2 + 1;   // float4 per row of the step tile
     static constexpr int YQ = LPR <= 4 ? 16 : 20;
     static constexpr int YR = LPR == 2 ? 36 : LPR == 4 ? 68 : LPR == 8 ? 168 : 328;
     static constexpr int X_OFF = 0;
@@ -94,31 +96,38 @@ template <int LPR> struct Shape {
 // slots (its u, delta and z pieces of PB bytes each, then its B/C pieces),
 // stored slot-major so that a warp's slot accesses are contiguous.
 constexpr int kRawStages = 5;
-// With the convolution prologue (CONV) every thread also copies the 16 bytes
-// before its u piece (the convolution's look-back, VE >= 4 elements) into one
-// more slot, and a skip tile per tile stage ([row][step] floats after the
-// ring) carries D u from the widening to the readout.
-template <typename T, int LPR, bool CONV = false> struct Raw {
+// Kernel variants: 0 plain; 1 convolution prologue; 2 trapezoidal rule.
+// With the convolution prologue every thread also copies the 16 bytes before
+// its u piece (the convolution's look-back, VE >= 4 elements) into one more
+// slot, and a skip tile per tile stage ([row][step] floats after the ring)
+// carries D u from the widening to the readout. The trapezoidal rule uses the
+// same look-back slot (for u_{t-1}) and stages lambda_raw pieces as well.
+template <typename T, int LPR, int VAR = 0> struct Raw {
+    static constexpr bool CONV = VAR == 1, TRAP = VAR == 2;
+    using SH = Shape<LPR, TRAP>;
     static constexpr int EB = static_cast<int>(sizeof(T));
-    static constexpr int PB = Shape<LPR>::IP * EB;                   // bytes of one u/delta/z piece
+    static constexpr int PB = SH::IP * EB;                           // bytes of one u/delta/z piece
     static constexpr int PS = (PB + 15) / 16;                        // slots per piece
     static constexpr int VE = 16 / EB;                               // elements per B/C piece
     static constexpr int BC_PER = 2 * kStates * (kSteps / VE) / kIoThreads;   // B/C pieces per thread
-    static constexpr int HALO = 3 * PS + BC_PER;                     // slot of the look-back (CONV)
-    static constexpr int SLOTS = 3 * PS + BC_PER + (CONV ? 1 : 0);
+    static constexpr int HALO = 3 * PS + BC_PER;                     // slot of the look-back (variants 1, 2)
+    static constexpr int LAM = HALO + 1;                             // first slot of lambda_raw (variant 2)
+    static constexpr int SLOTS = 3 * PS + BC_PER + (VAR ? 1 : 0) + (TRAP ? PS : 0);
     static constexpr int STAGE = SLOTS * kIoThreads * 16;
-    // ring depth: one stage less with the prologue, so that its larger slots
-    // and the skip tiles still leave room for 3 (LPR 4) or 2 (LPR 2) CTAs per SM
-    static constexpr int RS = CONV ? kRawStages - 1 : kRawStages;
+    // ring depth: shorter for the variants, whose larger slots, skip tiles
+    // (prologue) or wider step tiles (trapezoidal) must still leave room for
+    // 3 (LPR 4) CTAs per SM
+    static constexpr int RS = TRAP ? kRawStages - 2 : CONV ? kRawStages - 1 : kRawStages;
     static constexpr int RA = RS - kTileStages + 1;                   // chunks staged ahead
-    static constexpr int OFF = Shape<LPR>::BYTES;
+    static constexpr int OFF = SH::BYTES;
     static constexpr int SKR = kSteps + 4;                            // floats per row of the skip tile
     static constexpr int SK_OFF = OFF + RS * STAGE;
-    static constexpr int SK_STAGE = Shape<LPR>::R * SKR * 4;
+    static constexpr int SK_STAGE = SH::R * SKR * 4;
     static constexpr int BYTES = SK_OFF + (CONV ? kTileStages * SK_STAGE : 0);   // total dynamic shared memory
     static_assert(BC_PER * kIoThreads * VE == 2 * kStates * kSteps, "B/C pieces split evenly");
     static_assert(PB == 4 || PB == 8 || PB % 16 == 0, "piece sizes cp.async can copy");
-    static_assert(!CONV || (PB % 16 == 0 && VE >= 4), "look-back: 16-byte aligned pieces, >= 3 earlier inputs");
+    static_assert(VAR == 0 || (PB % 16 == 0 && VE >= 4), "look-back: 16-byte aligned pieces, >= 3 earlier inputs");
+    static_assert(RA >= 1, "at least one chunk staged ahead");
 };
 
 // Named barriers (0 is __syncthreads): the producer arrives, the consumer
@@ -255,9 +264,9 @@ __device__ __forceinline__ void store_piece(T *dst, const float (&v)[P], int64_t
 }
 
 // The recurrence warps: lane (r, q) owns states q NPL .. q NPL + NPL - 1 of row r.
-template <typename T, int LPR>
+template <typename T, int LPR, bool TRAP>
 __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned char *smem, int tid) {
-    using S = Shape<LPR>;
+    using S = Shape<LPR, TRAP>;
     constexpr int NPL = S::NPL, R = S::R;
     constexpr int NP = NPL > 1 ? NPL / 2 : 1;
     constexpr int RW = 32 / LPR;   // rows per warp
@@ -290,6 +299,9 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
         hp[j] = f2(h2[0], h2[1]);
     }
 
+    float2 bprev[NP];   // trapezoidal rule: the lane's B_{t-1} entries (B_{-1} u_{-1} = 0 via its coefficient)
+#pragma unroll
+    for (int j = 0; j < NP; ++j) bprev[j] = f2(0.f, 0.f);
     int s = 0;   // tile stage of chunk c
     for (int64_t c = 0; c < nchunks; ++c, s = next_stage(s, kTileStages)) {
         unsigned char *st = smem + s * S::STAGE;
@@ -313,6 +325,50 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
                 for (int j = 0; j < NP; ++j) a[j] = ex2x2(mul2(f2(dt, dt), ap[j]));
             }
         };
+        if constexpr (TRAP) {
+            // h_t = a_t (h_{t-1} + p_t B_{t-1}) + q_t B_t with p_t = (1 - lambda_t)
+            // delta_t u_{t-1} and q_t = lambda_t delta_t u_t (one float4 per step)
+            float4 xc = xrow[0], xn = xrow[1];
+            float2 acur[NP];
+            decay(xc.x, acur);
+            StepIn<NPL> cur = load_bc_step<NPL>(Bl, Cl);
+            float outs[4];
+#pragma unroll
+            for (int t = 0; t < kSteps; ++t) {
+                StepIn<NPL> nxt = cur;
+                float2 anxt[NP];
+                float4 xnn = xn;
+                if (t + 1 < kSteps) {
+                    nxt = load_bc_step<NPL>(Bl + (t + 1) * kStates, Cl + (t + 1) * kStates);
+                    decay(xn.x, anxt);
+                    if (t + 2 < kSteps) xnn = xrow[t + 2];
+                }
+                const float qv = xc.y, pv = xc.z;
+                if constexpr (NPL == 1) {
+                    hp[0].x = fmaf(acur[0].x, fmaf(pv, bprev[0].x, hp[0].x), qv * cur.b[0].x);
+                    outs[t & 3] = cur.c[0].x * hp[0].x;
+                } else {
+                    float2 acc;
+#pragma unroll
+                    for (int j = 0; j < NP; ++j) {
+                        hp[j] = fma2(acur[j], fma2(f2(pv, pv), bprev[j], hp[j]), mul2(f2(qv, qv), cur.b[j]));
+                        acc = j == 0 ? mul2(cur.c[j], hp[j]) : fma2(cur.c[j], hp[j], acc);
+                    }
+                    outs[t & 3] = acc.x + acc.y;
+                }
+                if ((t & 3) == 3)
+                    *reinterpret_cast<float4 *>(yl + t - 3) = make_float4(outs[0], outs[1], outs[2], outs[3]);
+#pragma unroll
+                for (int j = 0; j < NP; ++j) bprev[j] = cur.b[j];
+                if (t + 1 < kSteps) {
+                    cur = nxt;
+#pragma unroll
+                    for (int j = 0; j < NP; ++j) acur[j] = anxt[j];
+                    xc = xn;
+                    xn = xnn;
+                }
+            }
+        } else {
         float4 xa = xrow[0], xb = xrow[1];   // steps (0, 1) and (2, 3)
         float2 acur[NP];
         decay(xa.x, acur);
@@ -352,6 +408,7 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
                 }
             }
         }
+        }
         if (c + kTileStages < nchunks) bar_signal(bar_xe(s));
         bar_signal(bar_yf(s));
     }
@@ -370,10 +427,11 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
 // inputs travel through the ring RA chunks ahead of use (cp.async on
 // the aligned path, plain loads otherwise); a thread waits only for its own
 // copies, so the ring needs no barrier.
-template <typename T, int LPR, bool VEC, bool CONV>
+template <typename T, int LPR, bool VEC, int VAR>
 __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem, int i) {
-    using S = Shape<LPR>;
-    using RW = Raw<T, LPR, CONV>;
+    constexpr bool CONV = VAR == 1, TRAP = VAR == 2;
+    using S = Shape<LPR, TRAP>;
+    using RW = Raw<T, LPR, VAR>;
     constexpr int R = S::R, IP = S::IP, IPR = S::IPR, EB = RW::EB, PB = RW::PB, PS = RW::PS;
     constexpr int VE = RW::VE, BC_PER = RW::BC_PER;
     static_assert(IP % 2 == 0, "pieces hold step pairs");
@@ -404,6 +462,7 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
                            static_cast<const T *>(p.delta) + b * p.dl_sb + dc * p.dl_sd + tk,
                            has_z ? static_cast<const T *>(p.z) + b * p.z_sb + dc * p.z_sd + tk : nullptr};
     T *yrow = static_cast<T *>(p.y) + b * p.y_sb + dc * p.y_sd + tk;
+    const T *lrow = TRAP ? static_cast<const T *>(p.lambda_raw) + b * p.lm_sb + dc * p.lm_sd + tk : nullptr;
 
     // The thread's B/C pieces: tensor (0 = B, 1 = C), state n, steps bt .. bt + VE - 1.
     int bc_off[BC_PER], bc_t[BC_PER];
@@ -452,9 +511,29 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
                     reinterpret_cast<uint32_t *>(slot(rs, tsr * PS + w / 4))[w % 4] = pc.w[w];
             }
         }
-        if constexpr (CONV) {
-            // the VE inputs before the piece (the convolution's look-back); for
-            // the first piece of the sequence they lie before t = 0 and read as 0
+        if constexpr (TRAP) {
+            const T *src = lrow + t0;
+            if constexpr (VEC) {
+#pragma unroll
+                for (int sl = 0; sl < PS; ++sl) {
+                    const int have = valid * EB - sl * 16;
+                    const int bytes = have < 0 ? 0 : (have > 16 ? 16 : have);
+                    cp_async16(slot(rs, RW::LAM + sl), bytes > 0 ? static_cast<const void *>(
+                                   reinterpret_cast<const unsigned char *>(src) + sl * 16) : static_cast<const void *>(lrow),
+                               bytes);
+                }
+            } else {
+                Piece<T, IP> pc;
+                load_piece<T, IP, false>(pc, src, valid);
+#pragma unroll
+                for (int w = 0; w < Piece<T, IP>::W; ++w)
+                    reinterpret_cast<uint32_t *>(slot(rs, RW::LAM + w / 4))[w % 4] = pc.w[w];
+            }
+        }
+        if constexpr (CONV || TRAP) {
+            // the VE inputs before the piece (the convolution's look-back; the
+            // trapezoidal rule's u_{t-1}); for the first piece of the sequence
+            // they lie before t = 0 and read as 0
             const int64_t th = t0 + tk - VE;
             const int hv = th < 0 ? 0 : static_cast<int>(min64(VE, max64(0, L - th)));
             const T *hsrc = hv > 0 ? src_row[0] + t0 - VE : src_row[0];
@@ -479,23 +558,25 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
             }
         }
     };
-    // The thread's piece of tensor tsr from ring stage rs.
-    auto ring_piece = [&](int rs, int tsr) {
+    // The thread's piece starting at slot `first` of ring stage rs.
+    auto ring_slots = [&](int rs, int first) {
         Piece<T, IP> pc;
         if constexpr (PB == 4) {
-            pc.w[0] = *reinterpret_cast<const uint32_t *>(slot(rs, tsr * PS));
+            pc.w[0] = *reinterpret_cast<const uint32_t *>(slot(rs, first));
         } else if constexpr (PB == 8) {
-            const uint2 v = *reinterpret_cast<const uint2 *>(slot(rs, tsr * PS));
+            const uint2 v = *reinterpret_cast<const uint2 *>(slot(rs, first));
             pc.w[0] = v.x; pc.w[1] = v.y;
         } else {
 #pragma unroll
             for (int sl = 0; sl < PS; ++sl) {
-                const uint4 v = *reinterpret_cast<const uint4 *>(slot(rs, tsr * PS + sl));
+                const uint4 v = *reinterpret_cast<const uint4 *>(slot(rs, first + sl));
                 pc.w[4 * sl] = v.x; pc.w[4 * sl + 1] = v.y; pc.w[4 * sl + 2] = v.z; pc.w[4 * sl + 3] = v.w;
             }
         }
         return pc;
     };
+    // The thread's piece of tensor tsr (0 u, 1 delta, 2 z) from ring stage rs.
+    auto ring_piece = [&](int rs, int tsr) { return ring_slots(rs, tsr * PS); };
     // Readout of chunk c from tile stage s (u, z from ring stage rs): partial
     // sums + D u, gate, store.
     auto finish = [&](int64_t c, int s, int rs) {
@@ -552,7 +633,7 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     // ring stage rs into tile stage s.
     auto widen = [&](int64_t c, int s, int rs) {
         unsigned char *st = smem + s * S::STAGE;
-        float4 *xrow = reinterpret_cast<float4 *>(st + S::X_OFF) + r * S::XR + tk / 2;
+        float4 *xrow = reinterpret_cast<float4 *>(st + S::X_OFF) + r * S::XR + (TRAP ? tk : tk / 2);
         const Piece<T, IP> xin = ring_piece(rs, 0), dl = ring_piece(rs, 1);
         // the SSM input u: the raw u, or the convolution prologue applied to x
         float2 u2[IP / 2];
@@ -582,6 +663,15 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
         }
         const bool full = (c + 1) * kSteps <= L;
         const int64_t cnt = L - (c * kSteps + tk);
+        float uprev = 0.f;   // trapezoidal rule: u_{t-1} of the piece's first step
+        Piece<T, IP> lam;
+        if constexpr (TRAP) {
+            const uint4 hw = *reinterpret_cast<const uint4 *>(slot(rs, RW::HALO));
+            Piece<T, VE> hl;
+            hl.w[0] = hw.x; hl.w[1] = hw.y; hl.w[2] = hw.z; hl.w[3] = hw.w;
+            uprev = elem(hl, VE - 1);
+            lam = ring_slots(rs, RW::LAM);
+        }
 #pragma unroll
         for (int e = 0; e < IP; e += 2) {
             float2 v = add2(f2(elem(dl, e), elem(dl, e + 1)), f2(bias, bias));
@@ -590,8 +680,21 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
                 if (e >= cnt) v.x = 0.f;
                 if (e + 1 >= cnt) v.y = 0.f;
             }
-            const float2 du = mul2(v, u2[e / 2]);
-            xrow[e / 2] = make_float4(v.x, du.x, v.y, du.y);
+            if constexpr (TRAP) {
+                // lambda = sigmoid(lambda_raw); q = lambda delta u_t, p = (1 - lambda) delta u_{t-1}
+                const float2 lr = f2(elem(lam, e), elem(lam, e + 1));
+                const float2 ex = ex2x2(mul2(lr, f2(-kLog2e, -kLog2e)));
+                const float2 lm = f2(__fdividef(1.f, 1.f + ex.x), __fdividef(1.f, 1.f + ex.y));
+                const float2 ld = mul2(lm, v);                          // lambda delta
+                const float2 q = mul2(ld, u2[e / 2]);
+                const float2 prev = f2(e == 0 ? uprev : u2[e / 2 - 1].y, u2[e / 2].x);
+                const float2 pq = mul2(add2(v, f2(-ld.x, -ld.y)), prev);   // (1 - lambda) delta u_{t-1}
+                xrow[e] = make_float4(v.x, q.x, pq.x, 0.f);
+                xrow[e + 1] = make_float4(v.y, q.y, pq.y, 0.f);
+            } else {
+                const float2 du = mul2(v, u2[e / 2]);
+                xrow[e / 2] = make_float4(v.x, du.x, v.y, du.y);
+            }
         }
 #pragma unroll
         for (int j = 0; j < BC_PER; ++j) {
@@ -645,83 +748,90 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     cp_async_wait<0>();
 }
 
-template <typename T, int LPR, bool VEC, bool CONV>
+template <typename T, int LPR, bool VEC, int VAR>
 __global__ void __launch_bounds__(kThreads, Shape<LPR>::MINB) rec_kernel(const ScanParams p) {
     extern __shared__ __align__(16) unsigned char smem[];
     if (threadIdx.x < kScanThreads) {
-        recurrence_role<T, LPR>(p, smem, threadIdx.x);
+        recurrence_role<T, LPR, VAR == 2>(p, smem, threadIdx.x);
     } else {
-        io_role<T, LPR, VEC, CONV>(p, smem, threadIdx.x - kScanThreads);
+        io_role<T, LPR, VEC, VAR>(p, smem, threadIdx.x - kScanThreads);
     }
 }
 
+template <typename T, int LPR, int VAR>
+const void *rec_ptr_v(bool vec) {
+    return vec ? reinterpret_cast<const void *>(rec_kernel<T, LPR, true, VAR>)
+               : reinterpret_cast<const void *>(rec_kernel<T, LPR, false, VAR>);
+}
+
 template <typename T, int LPR>
-const void *rec_ptr(bool vec, bool conv) {
-    if constexpr (LPR == 2 || LPR == 4) {   // the convolution prologue needs 16-byte pieces
-        if (conv)
-            return vec ? reinterpret_cast<const void *>(rec_kernel<T, LPR, true, true>)
-                       : reinterpret_cast<const void *>(rec_kernel<T, LPR, false, true>);
+const void *rec_ptr(bool vec, int variant) {
+    if constexpr (LPR == 2 || LPR == 4) {   // the variants need 16-byte pieces
+        if (variant == 1) return rec_ptr_v<T, LPR, 1>(vec);
+        if (variant == 2) return rec_ptr_v<T, LPR, 2>(vec);
     }
-    return vec ? reinterpret_cast<const void *>(rec_kernel<T, LPR, true, false>)
-               : reinterpret_cast<const void *>(rec_kernel<T, LPR, false, false>);
+    return rec_ptr_v<T, LPR, 0>(vec);
 }
 
 template <typename T>
-const void *rec_select(int lpr, bool vec, bool conv) {
+const void *rec_select(int lpr, bool vec, int variant) {
     switch (lpr) {
-        case 2: return rec_ptr<T, 2>(vec, conv);
-        case 4: return rec_ptr<T, 4>(vec, conv);
-        case 8: return rec_ptr<T, 8>(vec, conv);
-        default: return rec_ptr<T, 16>(vec, conv);
+        case 2: return rec_ptr<T, 2>(vec, variant);
+        case 4: return rec_ptr<T, 4>(vec, variant);
+        case 8: return rec_ptr<T, 8>(vec, variant);
+        default: return rec_ptr<T, 16>(vec, variant);
     }
 }
 
-const void *rec_kernel_for(int in_dtype, int lpr, bool vec, bool conv) {
-    return in_dtype == 0 ? rec_select<float>(lpr, vec, conv) : rec_select<__nv_bfloat16>(lpr, vec, conv);
+const void *rec_kernel_for(int in_dtype, int lpr, bool vec, int variant) {
+    return in_dtype == 0 ? rec_select<float>(lpr, vec, variant) : rec_select<__nv_bfloat16>(lpr, vec, variant);
 }
 
 template <typename T, int LPR>
-int smem_bytes_lpr(bool conv) {
+int smem_bytes_lpr(int variant) {
     if constexpr (LPR == 2 || LPR == 4) {
-        if (conv) return Raw<T, LPR, true>::BYTES;
+        if (variant == 1) return Raw<T, LPR, 1>::BYTES;
+        if (variant == 2) return Raw<T, LPR, 2>::BYTES;
     }
-    return Raw<T, LPR, false>::BYTES;
+    return Raw<T, LPR, 0>::BYTES;
 }
 
 template <typename T>
-int smem_bytes_t(int lpr, bool conv) {
+int smem_bytes_t(int lpr, int variant) {
     switch (lpr) {
-        case 2: return smem_bytes_lpr<T, 2>(conv);
-        case 4: return smem_bytes_lpr<T, 4>(conv);
-        case 8: return smem_bytes_lpr<T, 8>(conv);
-        default: return smem_bytes_lpr<T, 16>(conv);
+        case 2: return smem_bytes_lpr<T, 2>(variant);
+        case 4: return smem_bytes_lpr<T, 4>(variant);
+        case 8: return smem_bytes_lpr<T, 8>(variant);
+        default: return smem_bytes_lpr<T, 16>(variant);
     }
 }
 
 }  // namespace
 
-int rec_smem_bytes(int in_dtype, int lpr, bool conv) {
-    return in_dtype == 0 ? smem_bytes_t<float>(lpr, conv) : smem_bytes_t<__nv_bfloat16>(lpr, conv);
+int rec_variant(const ScanParams &p) { return p.lambda_raw ? 2 : p.conv_w ? 1 : 0; }
+
+int rec_smem_bytes(int in_dtype, int lpr, int variant) {
+    return in_dtype == 0 ? smem_bytes_t<float>(lpr, variant) : smem_bytes_t<__nv_bfloat16>(lpr, variant);
 }
 
-bool rec_supports_conv(int lpr) { return lpr == 2 || lpr == 4; }
+bool rec_supports_variant(int lpr, int variant) { return variant == 0 || lpr == 2 || lpr == 4; }
 int rec_chunk() { return kSteps; }
 int rec_threads() { return kThreads; }
 int rec_rows(int lpr) { return kScanThreads / lpr; }
 
 // Resident CTAs per SM of a sequential kernel (cached per kernel; the
 // shared-memory bound when no device answers).
-int rec_ctas_per_sm(int in_dtype, int lpr, bool vec, bool conv) {
+int rec_ctas_per_sm(int in_dtype, int lpr, bool vec, int variant) {
     constexpr int kSlots = 64;
     static const void *keys[kSlots];
     static int vals[kSlots];
     static int used = 0;
     static std::mutex mu;
-    const void *k = rec_kernel_for(in_dtype, lpr, vec, conv);
+    const void *k = rec_kernel_for(in_dtype, lpr, vec, variant);
     std::lock_guard<std::mutex> lk(mu);
     for (int i = 0; i < used; ++i)
         if (keys[i] == k) return vals[i];
-    const int smem = rec_smem_bytes(in_dtype, lpr, conv);
+    const int smem = rec_smem_bytes(in_dtype, lpr, variant);
     int n = 0;
     bool asked = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess &&
                  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, kThreads, smem) == cudaSuccess;
@@ -737,10 +847,10 @@ int rec_ctas_per_sm(int in_dtype, int lpr, bool vec, bool conv) {
 }
 
 cudaError_t launch_rec(const ScanParams &p, int lpr, bool vec, int in_dtype, cudaStream_t stream) {
-    const bool conv = p.conv_w != nullptr;
-    if (conv && !rec_supports_conv(lpr)) return cudaErrorInvalidValue;
-    const void *k = rec_kernel_for(in_dtype, lpr, vec, conv);
-    const int smem = rec_smem_bytes(in_dtype, lpr, conv);
+    const int variant = rec_variant(p);
+    if (!rec_supports_variant(lpr, variant) || (p.conv_w && p.lambda_raw)) return cudaErrorInvalidValue;
+    const void *k = rec_kernel_for(in_dtype, lpr, vec, variant);
+    const int smem = rec_smem_bytes(in_dtype, lpr, variant);
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const int R = kScanThreads / lpr;

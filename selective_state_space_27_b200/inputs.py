@@ -42,7 +42,7 @@ BASE_SEED = 20261202
 # One draw stream per tensor, so that the value of a tensor does not depend on
 # which other tensors were drawn.
 _STREAM = {"u": 1, "delta": 2, "B": 3, "C": 4, "z": 5, "D": 6, "dt": 7, "h0": 8, "conv_w": 9, "conv_b": 10,
-           "conv_state": 11}
+           "conv_state": 11, "lambda_raw": 12}
 _CHUNK = 1 << 22
 
 
@@ -258,3 +258,9 @@ def make_conv_state(batch: int, dim: int, width: int, dtype: str, seed: int = BA
     """A convolution state (batch, dim, width) of N(0,1) inputs in the storage
     dtype (float32, or bf16 bits)."""
     return _store(_normal((batch, dim, width), seed, _STREAM["conv_state"]), dtype)
+
+
+def make_lambda_raw(batch: int, dim: int, seqlen: int, dtype: str, seed: int = BASE_SEED) -> np.ndarray:
+    """Pre-activation of the trapezoidal rule's per-token gate, N(0, 1) in the
+    storage dtype (float32, or bf16 bits), shape (batch, dim, seqlen)."""
+    return _store(_normal((batch, dim, seqlen), seed, _STREAM["lambda_raw"]), dtype)

@@ -181,3 +181,14 @@ def test_conv_state_update_validation_rejects(lib, state, sb, sd, status):
                                      sb, sd, None)
     assert rc == status
     assert lib.mamba_conv_state_update(ctypes.byref(_valid_update_args()), None, (1 << 20) * 11, 32, 4, None) == 1
+
+
+@pytest.mark.parametrize("lam,sb,sd,segments,status", [
+    (None, 512, 64, 0, 1), ((1 << 20) * 12, -1, 64, 0, 1), ((1 << 20) * 12 + 1, 512, 64, 0, 3),
+    ((1 << 20) * 12, 512, 64, 2, 2),
+])
+def test_trap_scan_validation_rejects(lib, lam, sb, sd, segments, status):
+    a = _valid_scan_args()
+    a.force_segments = segments
+    assert lib.mamba_trap_scan_fwd(ctypes.byref(a), lam, sb, sd, None, None) == status
+    assert lib.mamba_last_error().decode() != ""
