@@ -57,6 +57,10 @@ def _bind(path: str):
     lib.s6_oracle_trap_scan.restype = ip
     lib.s6_oracle_trap_scan.argtypes = [i64, i64, i64, i64, ip, vp, vp, vp, vp, vp, vp, vp, vp, vp, ip, vp,
                                         i64, vp, vp, vp, ip]
+    lib.s6_oracle_scan_d.restype = ip
+    lib.s6_oracle_scan_d.argtypes = [i64, i64, i64, i64] + [vp] * 8 + [ip, vp, vp, vp]
+    lib.s6_oracle_scan_bwd.restype = ip
+    lib.s6_oracle_scan_bwd.argtypes = [i64, i64, i64, i64] + [vp] * 8 + [ip] + [vp] * 12
     lib.s6_oracle_max_threads.restype = ip
     lib.s6_oracle_max_threads.argtypes = []
     return lib
@@ -280,6 +284,61 @@ def trap_scan(*, u, delta, lambda_raw, A, B, C, D=None, z=None, delta_bias=None,
     return y, h
 
 
+def as_f64(a, dtype=None):
+    """Values of an oracle input as float64: float32 arrays, bf16 bit patterns
+    (uint16, widened exactly) or float64 arrays."""
+    if a is None:
+        return None
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        return np.ascontiguousarray((a.astype(np.uint32) << 16).view(np.float32).astype(np.float64))
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def scan_d(*, u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True, h0=None,
+           _lib_override=None):
+    """The forward scan with every input in float64 (the backward's reference
+    forward; used by the finite-difference pins). Returns ``(y, h)``."""
+    u, delta, A, B, C, D, z, delta_bias, h0 = (as_f64(a) for a in (u, delta, A, B, C, D, z, delta_bias, h0))
+    batch, dim, L = u.shape
+    N = B.shape[1]
+    y = np.empty((batch, dim, L))
+    h = np.empty((batch, dim, N))
+    lib = _lib_override or _load()
+    rc = lib.s6_oracle_scan_d(batch, dim, N, L, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                              _ptr(delta_bias), int(bool(delta_softplus)), _ptr(h0), _ptr(y), _ptr(h))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return y, h
+
+
+def scan_bwd(*, u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, delta_softplus=True, h0=None, dhT=None,
+             _lib_override=None):
+    """Gradients of the scan in float64 for the loss sum(y * dy) + sum(hT * dhT).
+
+    Inputs as :func:`scan` (float32, bf16 bits or float64 arrays), ``dy``
+    (batch, dim, L), ``dhT`` (batch, dim, N). Returns a dict with du, ddelta
+    (w.r.t. delta_raw), dz, dA, dB, dC, dD, ddelta_bias, dh0 (float64; dz is
+    None without z)."""
+    u, delta, A, B, C, D, z, delta_bias, h0, dy, dhT = (
+        as_f64(a) for a in (u, delta, A, B, C, D, z, delta_bias, h0, dy, dhT))
+    batch, dim, L = u.shape
+    N = B.shape[1]
+    out = {"du": np.empty((batch, dim, L)), "ddelta": np.empty((batch, dim, L)),
+           "dz": np.empty((batch, dim, L)) if z is not None else None, "dA": np.empty((dim, N)),
+           "dB": np.empty((batch, N, L)), "dC": np.empty((batch, N, L)), "dD": np.empty(dim),
+           "ddelta_bias": np.empty(dim), "dh0": np.empty((batch, dim, N))}
+    lib = _lib_override or _load()
+    rc = lib.s6_oracle_scan_bwd(batch, dim, N, L, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                _ptr(z), _ptr(delta_bias), int(bool(delta_softplus)), _ptr(h0), _ptr(dy), _ptr(dhT),
+                                _ptr(out["du"]), _ptr(out["ddelta"]), _ptr(out["dz"]), _ptr(out["dA"]),
+                                _ptr(out["dB"]), _ptr(out["dC"]), _ptr(out["dD"]), _ptr(out["ddelta_bias"]),
+                                _ptr(out["dh0"]))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return out
+
+
 class Variant:
     """The oracle's entry points bound to another build of the oracle source.
 
@@ -304,6 +363,12 @@ class Variant:
 
     def trap_scan(self, **kw):
         return trap_scan(_lib_override=self._lib, **kw)
+
+    def scan_d(self, **kw):
+        return scan_d(_lib_override=self._lib, **kw)
+
+    def scan_bwd(self, **kw):
+        return scan_bwd(_lib_override=self._lib, **kw)
 
 
 def compile_source(src_path: str, so_path: str) -> str:

@@ -75,12 +75,16 @@
 #include <omp.h>
 #endif
 
-enum { ORACLE_F32 = 0, ORACLE_BF16 = 1 };
+/* ORACLE_F64 (double inputs) exists for the finite-difference pins of the
+ * backward pass; the GPU never sees it. */
+enum { ORACLE_F32 = 0, ORACLE_BF16 = 1, ORACLE_F64 = 2 };
 
 static double load_value(const void *p, int dtype, int64_t i)
 {
     if (dtype == ORACLE_F32)
         return (double)((const float *)p)[i];
+    if (dtype == ORACLE_F64)
+        return ((const double *)p)[i];
     uint32_t bits = (uint32_t)((const uint16_t *)p)[i] << 16;
     float f;
     memcpy(&f, &bits, sizeof f);
@@ -153,7 +157,7 @@ int s6_oracle_scan(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, i
 {
     if (batch < 0 || dim < 0 || dstate < 0 || seqlen < 0)
         return -1;
-    if (dtype != ORACLE_F32 && dtype != ORACLE_BF16)
+    if (dtype != ORACLE_F32 && dtype != ORACLE_BF16 && dtype != ORACLE_F64)
         return -1;
     if (!rows)
         n_rows = batch * dim;
@@ -425,6 +429,143 @@ int s6_oracle_trap_scan(int64_t batch, int64_t dim, int64_t dstate, int64_t seql
         free(v_prev);
     }
     return failed ? -1 : 0;
+}
+
+/* ---- Backward pass --------------------------------------------------------
+ * Gradients of the scan by reverse-mode differentiation of the forward
+ * definition (the backward half of "A varredura paralela ciente do hardware",
+ * which recomputes the states instead of storing them; here the fp64
+ * reference simply keeps them). With s_t = sum_n C h + D u (before the gate),
+ * y_t = s_t silu(z_t) and a_tn = exp(delta_t A_n):
+ *   ds_t  = dy_t silu(z_t);  dz_t = dy_t s_t silu'(z_t)
+ *   g_tn  = ds_t C_tn + a_{t+1,n} g_{t+1,n}   (g_{L-1} also receives dhT)
+ *   dC_tn += ds_t h_tn;  dB_tn += g_tn delta_t u_t;  dD += ds_t u_t
+ *   du_t  = sum_n g_tn delta_t B_tn + ds_t D
+ *   ddelta_t = sum_n g_tn (B_tn u_t + h_{t-1,n} a_tn A_n)  (times sigmoid(raw) under softplus)
+ *   dA_n  += g_tn h_{t-1,n} a_tn delta_t;  dh0_n = a_0n g_0n
+ * All arrays are doubles, contiguous: u, delta, z, dy (batch, dim, L); B, C
+ * (batch, N, L); A (dim, N); D, delta_bias (dim); h0, dhT, dh0 (batch, dim, N).
+ */
+static void scan_row_d(int64_t L, int64_t N, const double *u, const double *dr, const double *A_row,
+                       const double *Bb, const double *Cb, double D, const double *z, double bias,
+                       int softplus_on, double *h, double *y, double *s_pre, double *H, double *Ad,
+                       double *dts)
+{
+    for (int64_t t = 0; t < L; ++t) {
+        double dt = dr[t] + bias;
+        if (softplus_on)
+            dt = softplus(dt);
+        if (dts)
+            dts[t] = dt;
+        double acc = 0.0;
+        for (int64_t n = 0; n < N; ++n) {
+            const double a = exp(dt * A_row[n]);
+            h[n] = a * h[n] + dt * Bb[n * L + t] * u[t];
+            acc += Cb[n * L + t] * h[n];
+            if (H)
+                H[t * N + n] = h[n];
+            if (Ad)
+                Ad[t * N + n] = a;
+        }
+        acc += D * u[t];
+        if (s_pre)
+            s_pre[t] = acc;
+        y[t] = z ? acc * silu(z[t]) : acc;
+    }
+}
+
+/* All-double forward: y (batch, dim, L) and the final state (batch, dim, N). */
+int s6_oracle_scan_d(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, const double *u,
+                     const double *delta, const double *A, const double *B, const double *C,
+                     const double *D, const double *z, const double *delta_bias, int delta_softplus,
+                     const double *h0, double *y_out, double *h_out)
+{
+    if (batch < 0 || dim < 0 || dstate < 0 || seqlen < 0 || !u || !delta || !A || !B || !C || !y_out || !h_out)
+        return -1;
+    for (int64_t b = 0; b < batch; ++b)
+        for (int64_t d = 0; d < dim; ++d) {
+            const int64_t row = b * dim + d;
+            double *h = h_out + row * dstate;
+            for (int64_t n = 0; n < dstate; ++n)
+                h[n] = h0 ? h0[row * dstate + n] : 0.0;
+            scan_row_d(seqlen, dstate, u + row * seqlen, delta + row * seqlen, A + d * dstate,
+                       B + b * dstate * seqlen, C + b * dstate * seqlen, D ? D[d] : 0.0,
+                       z ? z + row * seqlen : NULL, delta_bias ? delta_bias[d] : 0.0, delta_softplus, h,
+                       y_out + row * seqlen, NULL, NULL, NULL, NULL);
+        }
+    return 0;
+}
+
+int s6_oracle_scan_bwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, const double *u,
+                       const double *delta, const double *A, const double *B, const double *C,
+                       const double *D, const double *z, const double *delta_bias, int delta_softplus,
+                       const double *h0, const double *dy, const double *dhT, double *du, double *ddelta,
+                       double *dz, double *dA, double *dB, double *dC, double *dD, double *ddelta_bias,
+                       double *dh0)
+{
+    if (batch < 0 || dim < 0 || dstate < 0 || seqlen < 0 || !u || !delta || !A || !B || !C || !dy || !du ||
+        !ddelta || !dA || !dB || !dC || !dD || !ddelta_bias || !dh0 || (z && !dz))
+        return -1;
+    const int64_t L = seqlen, N = dstate;
+    memset(dA, 0, (size_t)(dim * N) * sizeof(double));
+    memset(dB, 0, (size_t)(batch * N * L) * sizeof(double));
+    memset(dC, 0, (size_t)(batch * N * L) * sizeof(double));
+    memset(dD, 0, (size_t)dim * sizeof(double));
+    memset(ddelta_bias, 0, (size_t)dim * sizeof(double));
+    double *H = (double *)malloc((size_t)(L * N + 1) * sizeof(double));
+    double *Ad = (double *)malloc((size_t)(L * N + 1) * sizeof(double));
+    double *sp = (double *)malloc((size_t)(L + 1) * sizeof(double));
+    double *dts = (double *)malloc((size_t)(L + 1) * sizeof(double));
+    double *yy = (double *)malloc((size_t)(L + 1) * sizeof(double));
+    double *h = (double *)malloc((size_t)(N + 1) * sizeof(double));
+    double *g = (double *)malloc((size_t)(N + 1) * sizeof(double));
+    if (!H || !Ad || !sp || !dts || !yy || !h || !g) {
+        free(H); free(Ad); free(sp); free(dts); free(yy); free(h); free(g);
+        return -1;
+    }
+    for (int64_t b = 0; b < batch; ++b)
+        for (int64_t d = 0; d < dim; ++d) {
+            const int64_t row = b * dim + d;
+            const double *ur = u + row * L, *dr = delta + row * L, *zr = z ? z + row * L : NULL;
+            const double *Bb = B + b * N * L, *Cb = C + b * N * L, *Ar = A + d * N;
+            const double Dd = D ? D[d] : 0.0, bias = delta_bias ? delta_bias[d] : 0.0;
+            for (int64_t n = 0; n < N; ++n)
+                h[n] = h0 ? h0[row * N + n] : 0.0;
+            scan_row_d(L, N, ur, dr, Ar, Bb, Cb, Dd, zr, bias, delta_softplus, h, yy, sp, H, Ad, dts);
+            for (int64_t n = 0; n < N; ++n)
+                g[n] = dhT ? dhT[row * N + n] : 0.0;     /* a_{t+1} g_{t+1} carried down */
+            for (int64_t t = L - 1; t >= 0; --t) {
+                double ds = dy[row * L + t];
+                if (zr) {
+                    const double zz = zr[t], sg = 1.0 / (1.0 + exp(-zz));
+                    dz[row * L + t] = ds * sp[t] * sg * (1.0 + zz * (1.0 - sg));
+                    ds *= zz * sg;
+                }
+                const double dt = dts[t];
+                double du_t = ds * Dd, ddt = 0.0;
+                dD[d] += ds * ur[t];
+                for (int64_t n = 0; n < N; ++n) {
+                    const double hprev = t > 0 ? H[(t - 1) * N + n] : (h0 ? h0[row * N + n] : 0.0);
+                    const double a = Ad[t * N + n];
+                    const double gn = g[n] + ds * Cb[n * L + t];
+                    dC[(b * N + n) * L + t] += ds * H[t * N + n];
+                    dB[(b * N + n) * L + t] += gn * dt * ur[t];
+                    du_t += gn * dt * Bb[n * L + t];
+                    ddt += gn * (Bb[n * L + t] * ur[t] + hprev * a * Ar[n]);
+                    dA[d * N + n] += gn * hprev * a * dt;
+                    g[n] = a * gn;
+                }
+                du[row * L + t] = du_t;
+                if (delta_softplus)
+                    ddt *= 1.0 / (1.0 + exp(-(dr[t] + bias)));
+                ddelta[row * L + t] = ddt;
+                ddelta_bias[d] += ddt;
+            }
+            for (int64_t n = 0; n < N; ++n)
+                dh0[row * N + n] = g[n];
+        }
+    free(H); free(Ad); free(sp); free(dts); free(yy); free(h); free(g);
+    return 0;
 }
 
 int s6_oracle_max_threads(void)

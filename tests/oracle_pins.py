@@ -574,6 +574,76 @@ def pin_trap_linearity(orc, seed=41):
     assert _rel(y3, a * y1 + b * y2) <= 1e-6 and _rel(h3, a * h1 + b * h2) <= 1e-6
 
 
+# ---- backward pass (gradients of the scan, the training half the pages
+# recompute instead of storing: "A varredura paralela ciente do hardware") ----
+
+def _bwd_case(g, batch=2, dim=2, N=3, L=9, softplus=True):
+    """Without the softplus the step is used as given, so it is drawn positive
+    (a step of the discretised system; negative steps make the state grow and
+    the finite differences lose digits)."""
+    delta = g.normal(scale=0.5, size=(batch, dim, L))
+    bias = g.normal(size=dim) - 1.0
+    if not softplus:
+        delta, bias = np.abs(delta), g.uniform(0.05, 0.2, size=dim)
+    return dict(u=g.normal(size=(batch, dim, L)), delta=delta,
+                A=-np.exp(g.normal(size=(dim, N))), B=g.normal(size=(batch, N, L)), C=g.normal(size=(batch, N, L)),
+                D=g.uniform(0.5, 1.5, size=dim), z=g.normal(size=(batch, dim, L)),
+                delta_bias=bias, h0=g.normal(size=(batch, dim, N)), delta_softplus=softplus)
+
+
+def pin_double_forward_matches_scan(orc, seed=50):
+    """The all-double forward (the backward's reference) computes the same
+    values as the float32 scan on float32 inputs."""
+    g = _rng(seed)
+    case = _bwd_case(g)
+    f32 = {k: (_f32(v) if isinstance(v, np.ndarray) else v) for k, v in case.items()}
+    y1, h1 = orc.scan_d(**{k: (v.astype(np.float64) if isinstance(v, np.ndarray) else v) for k, v in f32.items()})
+    h0 = f32.pop("h0")
+    y2, h2 = orc.scan(**f32, h0=h0.reshape(-1, h0.shape[-1]))
+    assert _rel(y1, y2) <= 1e-14 and _rel(h1, h2) <= 1e-14
+
+
+def pin_backward_finite_differences(orc, seed=51, eps=1e-6):
+    """Every gradient of sum(y dy) + sum(hT dhT) against central finite
+    differences of the all-double forward, input by input, with and without
+    the softplus."""
+    for softplus in (True, False):
+        g = _rng(seed + softplus)
+        case = _bwd_case(g, softplus=softplus)
+        dy = g.normal(size=case["u"].shape)
+        dhT = g.normal(size=case["h0"].shape)
+        grads = orc.scan_bwd(**case, dy=dy, dhT=dhT)
+
+        def loss(c):
+            y, h = orc.scan_d(**c)
+            return float((y * dy).sum() + (h * dhT).sum())
+
+        for name, gname in (("u", "du"), ("delta", "ddelta"), ("z", "dz"), ("A", "dA"), ("B", "dB"), ("C", "dC"),
+                            ("D", "dD"), ("delta_bias", "ddelta_bias"), ("h0", "dh0")):
+            base = case[name]
+            fd = np.empty_like(base)
+            for idx in np.ndindex(base.shape):
+                plus = dict(case); minus = dict(case)
+                bp = base.copy(); bm = base.copy()
+                bp[idx] += eps; bm[idx] -= eps
+                plus[name] = bp; minus[name] = bm
+                fd[idx] = (loss(plus) - loss(minus)) / (2 * eps)
+            assert _rel(grads[gname], fd) <= 1e-6, (softplus, name, _rel(grads[gname], fd))
+
+
+def pin_backward_linear_in_output_gradients(orc, seed=52):
+    """The gradients are linear in (dy, dhT)."""
+    g = _rng(seed)
+    case = _bwd_case(g)
+    dy1, dy2 = g.normal(size=case["u"].shape), g.normal(size=case["u"].shape)
+    dh1, dh2 = g.normal(size=case["h0"].shape), g.normal(size=case["h0"].shape)
+    g1 = orc.scan_bwd(**case, dy=dy1, dhT=dh1)
+    g2 = orc.scan_bwd(**case, dy=dy2, dhT=dh2)
+    g3 = orc.scan_bwd(**case, dy=2.0 * dy1 - 3.0 * dy2, dhT=2.0 * dh1 - 3.0 * dh2)
+    for k in g1:
+        assert _rel(g3[k], 2.0 * g1[k] - 3.0 * g2[k]) <= 1e-12, k
+
+
 ALL_PINS = [
     pin_selection_step,
     pin_lti_convolution,
@@ -596,4 +666,7 @@ ALL_PINS = [
     pin_trap_page_check,
     pin_trap_unrolled_sum,
     pin_trap_linearity,
+    pin_double_forward_matches_scan,
+    pin_backward_finite_differences,
+    pin_backward_linear_in_output_gradients,
 ]

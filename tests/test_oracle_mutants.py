@@ -45,6 +45,17 @@ MUTANTS = [
     ("trap_previous_input_frozen", "v_prev[n] = v;", "v_prev[n] = 0.0 * v;"),
     ("trap_no_sigmoid", "const double lam = sigmoid(load_value(lambda_raw, dtype, i));",
      "const double lam = load_value(lambda_raw, dtype, i);"),
+    ("bwd_decay_term_dropped", "ddt += gn * (Bb[n * L + t] * ur[t] + hprev * a * Ar[n]);",
+     "ddt += gn * (Bb[n * L + t] * ur[t]);"),
+    ("bwd_transition_uses_new_state", "dA[d * N + n] += gn * hprev * a * dt;",
+     "dA[d * N + n] += gn * H[t * N + n] * a * dt;"),
+    ("bwd_final_state_gradient_ignored", "g[n] = dhT ? dhT[row * N + n] : 0.0;", "g[n] = 0.0;"),
+    ("bwd_softplus_derivative_missing", "ddt *= 1.0 / (1.0 + exp(-(dr[t] + bias)));", "ddt *= 1.0;"),
+    ("bwd_gate_derivative_is_silu", "dz[row * L + t] = ds * sp[t] * sg * (1.0 + zz * (1.0 - sg));",
+     "dz[row * L + t] = ds * sp[t] * zz * sg;"),
+    ("bwd_input_matrix_gradient_misses_token", "dB[(b * N + n) * L + t] += gn * dt * ur[t];",
+     "dB[(b * N + n) * L + t] += gn * dt;"),
+    ("bwd_carry_not_decayed", "g[n] = a * gn;", "g[n] = gn;"),
     ("conv_decode_taps_reversed", "acc += (double)conv_w[d * width + k] * cs[k];",
      "acc += (double)conv_w[d * width + width - 1 - k] * cs[k];"),
 ]
