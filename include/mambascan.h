@@ -309,6 +309,47 @@ ms_status mamba_conv_state_update(const ms_update_args *args, const ms_conv1d_ar
 ms_status mamba_trap_scan_fwd(const ms_scan_args *args, const void *lambda_raw, int64_t lambda_batch_stride,
                               int64_t lambda_dim_stride, const ms_scan_plan *plan, void *stream);
 
+/* ---- Backward pass ---------------------------------------------------------
+ * Gradients of the selective scan for the loss sum(y dy) + sum(h_T dh_T)
+ * ("Notas sobre Mamba", section "A varredura paralela ciente do hardware":
+ * the backward pass recomputes the states instead of storing them). The
+ * forward's arguments come in an ms_scan_args (its y and final_state are not
+ * used); the gradients come out here. Layouts: dy, du, ddelta, dz as u
+ * (batch, dim, seqlen) in the input dtype, contiguous along t; ddelta is the
+ * gradient w.r.t. the raw delta (through the softplus and the bias). dB and
+ * dC are (batch, dstate, seqlen) float32, contiguous (summed over dim, since B
+ * and C are shared across channels); dA is (dim, dstate), dD and
+ * ddelta_bias (dim), summed over the batch; dinitial_state and dfinal_state
+ * are (batch, dim, dstate) float32, contiguous. dA, dB, dC, dD and
+ * ddelta_bias are written (zeroed by the call, then accumulated). */
+typedef struct ms_scan_bwd_args {
+    const void *dy;          int64_t dy_batch_stride, dy_dim_stride;            /* required */
+    const float *dfinal_state;                                                /* or NULL (zero) */
+    void *du;                int64_t du_batch_stride, du_dim_stride;            /* required */
+    void *ddelta;            int64_t ddelta_batch_stride, ddelta_dim_stride;    /* required */
+    void *dz;                int64_t dz_batch_stride, dz_dim_stride;            /* required iff z */
+    float *dA;                                                                /* required */
+    float *dB, *dC;                                                           /* required */
+    float *dD;                                                                /* required iff D */
+    float *ddelta_bias;                                                       /* required iff delta_bias */
+    float *dinitial_state;                                                    /* or NULL */
+} ms_scan_bwd_args;
+
+/* Device workspace for mamba_scan_bwd (the chunk checkpoints of the states:
+ * batch * dim * ceil(seqlen / 16) * 16 floats). */
+ms_status mamba_scan_bwd_workspace_size(const ms_scan_args *args, size_t *bytes);
+
+/*
+ * Backward pass: one kernel launch (after clearing the accumulated outputs)
+ * on `stream`. The caller owns every buffer, the workspace included (256-byte
+ * aligned). Errors: as mamba_scan_fwd for the forward arguments;
+ * MS_ERR_INVALID_ARG for a NULL bwd, a missing required gradient or negative
+ * strides; MS_ERR_ALIGNMENT for misaligned pointers; MS_ERR_WORKSPACE for a
+ * missing or short workspace.
+ */
+ms_status mamba_scan_bwd(const ms_scan_args *args, const ms_scan_bwd_args *bwd, void *workspace,
+                         size_t workspace_bytes, void *stream);
+
 /* Size of the device array behind mamba_scan_fwd_noalloc (8 MiB per GPU). */
 #define MS_NOALLOC_SCRATCH_BYTES (8u << 20)
 

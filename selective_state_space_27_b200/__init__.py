@@ -25,6 +25,7 @@ __all__ = [
     "scan_fwd", "state_update", "scan_workspace_size", "scan_plan", "scan_configs", "library_path",
     "load_library", "MambaScanError", "ScanArgs", "UpdateArgs", "ScanPlan", "MS_F32", "MS_BF16",
     "Conv1dArgs", "conv_scan_fwd", "conv_state_update", "build_conv_args", "trap_scan_fwd",
+    "ScanBwdArgs", "scan_bwd",
     "MAX_DSTATE",
 ]
 
@@ -79,6 +80,18 @@ class Conv1dArgs(ctypes.Structure):
     _fields_ = [("weight", _vp), ("bias", _vp), ("width", _i32), ("silu", _i32)]
 
 
+class ScanBwdArgs(ctypes.Structure):
+    """Mirror of ``ms_scan_bwd_args``."""
+    _fields_ = [
+        ("dy", _vp), ("dy_batch_stride", _i64), ("dy_dim_stride", _i64),
+        ("dfinal_state", _vp),
+        ("du", _vp), ("du_batch_stride", _i64), ("du_dim_stride", _i64),
+        ("ddelta", _vp), ("ddelta_batch_stride", _i64), ("ddelta_dim_stride", _i64),
+        ("dz", _vp), ("dz_batch_stride", _i64), ("dz_dim_stride", _i64),
+        ("dA", _vp), ("dB", _vp), ("dC", _vp), ("dD", _vp), ("ddelta_bias", _vp), ("dinitial_state", _vp),
+    ]
+
+
 class ScanPlan(ctypes.Structure):
     """Mirror of ``ms_scan_plan``."""
     _fields_ = [
@@ -131,6 +144,11 @@ def load_library():
         lib.mamba_trap_scan_fwd.restype = ctypes.c_int
         lib.mamba_trap_scan_fwd.argtypes = [ctypes.POINTER(ScanArgs), _vp, ctypes.c_int64, ctypes.c_int64,
                                             ctypes.POINTER(ScanPlan), _vp]
+        lib.mamba_scan_bwd_workspace_size.restype = ctypes.c_int
+        lib.mamba_scan_bwd_workspace_size.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(ctypes.c_size_t)]
+        lib.mamba_scan_bwd.restype = ctypes.c_int
+        lib.mamba_scan_bwd.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(ScanBwdArgs), _vp, ctypes.c_size_t,
+                                       _vp]
         lib.mamba_scan_config_kind.restype = ctypes.c_int
         lib.mamba_scan_config_kind.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
         lib.mamba_scan_plan_query.restype = ctypes.c_int
@@ -435,3 +453,54 @@ def trap_scan_fwd(u, delta, lambda_raw, A, B, C, D=None, z=None, delta_bias=None
                                                   lambda_raw.stride(1), None if plan is None else ctypes.byref(plan),
                                                   _stream_ptr(stream)))
     return (y, hT) if return_last_state else y
+
+
+def scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, delta_softplus=True, initial_state=None,
+             dfinal_state=None, workspace=None, stream=None):
+    """Gradients of :func:`scan_fwd` for the loss sum(y * dy) + sum(h_T * dfinal_state).
+
+    Forward inputs as :func:`scan_fwd`; ``dy`` (batch, dim, L) in u's dtype;
+    ``dfinal_state`` (batch, dim, dstate) float32 or None. Returns a dict:
+    du, ddelta (w.r.t. the raw delta), dz (None without z) in u's dtype; dA
+    (dim, dstate), dB, dC (batch, dstate, L), dD, ddelta_bias (dim,) (None
+    when the input is None) and dinitial_state (batch, dim, dstate), float32.
+    """
+    torch = _torch()
+    batch, dim, L = u.shape
+    N = B.shape[1]
+    # the forward's arguments; its output pointer is not used by the backward (u stands in for it)
+    args = build_scan_args(u, delta, A, B, C, u, D=D, z=z, delta_bias=delta_bias, delta_softplus=delta_softplus,
+                           initial_state=initial_state)
+    _need_cuda("dy", dy, u.dtype, 3)
+    if tuple(dy.shape) != tuple(u.shape):
+        raise ValueError("dy must have u's shape")
+    if dfinal_state is not None:
+        _need_cuda("dfinal_state", dfinal_state, torch.float32, 3)
+        if tuple(dfinal_state.shape) != (batch, dim, N) or not dfinal_state.is_contiguous():
+            raise ValueError("dfinal_state must be a contiguous (batch, dim, dstate) float32 tensor")
+    f32 = dict(device=u.device, dtype=torch.float32)
+    out = {"du": torch.empty_like(u), "ddelta": torch.empty_like(u), "dz": torch.empty_like(u) if z is not None else None,
+           "dA": torch.empty((dim, N), **f32), "dB": torch.empty((batch, N, L), **f32),
+           "dC": torch.empty((batch, N, L), **f32), "dD": torch.empty(dim, **f32) if D is not None else None,
+           "ddelta_bias": torch.empty(dim, **f32) if delta_bias is not None else None,
+           "dinitial_state": torch.empty((batch, dim, N), **f32)}
+    g = ScanBwdArgs()
+    g.dy, g.dy_batch_stride, g.dy_dim_stride = _ptr(dy), dy.stride(0), dy.stride(1)
+    g.dfinal_state = _ptr(dfinal_state)
+    for k in ("du", "ddelta", "dz"):
+        t = out[k]
+        if t is not None:
+            setattr(g, k, _ptr(t))
+            setattr(g, f"{k}_batch_stride", t.stride(0))
+            setattr(g, f"{k}_dim_stride", t.stride(1))
+    for k in ("dA", "dB", "dC", "dD", "ddelta_bias", "dinitial_state"):
+        setattr(g, k, _ptr(out[k]))
+    lib = load_library()
+    with torch.cuda.device(u.device):
+        n = ctypes.c_size_t(0)
+        _check(lib.mamba_scan_bwd_workspace_size(ctypes.byref(args), ctypes.byref(n)))
+        if workspace is None or workspace.numel() < n.value:
+            workspace = torch.empty(max(n.value, 1), dtype=torch.uint8, device=u.device)
+        _check(lib.mamba_scan_bwd(ctypes.byref(args), ctypes.byref(g), workspace.data_ptr(), workspace.numel(),
+                                  _stream_ptr(stream)))
+    return out

@@ -405,4 +405,69 @@ ms_status mamba_trap_scan_fwd(const ms_scan_args *args, const void *lambda_raw, 
     return run_plan(p, pl, args->in_dtype, nullptr, 0, stream);
 }
 
+ms_status mamba_scan_bwd_workspace_size(const ms_scan_args *args, size_t *bytes) {
+    if (!bytes) return invalid("bytes is NULL");
+    *bytes = 0;
+    const ms_status st = check_scan(args);
+    if (st != MS_OK) return st;
+    *bytes = ms::bwd_workspace_bytes(to_params(args));
+    return MS_OK;
+}
+
+ms_status mamba_scan_bwd(const ms_scan_args *args, const ms_scan_bwd_args *g, void *workspace,
+                         size_t workspace_bytes, void *stream) {
+    ms_status st = check_scan(args);
+    if (st != MS_OK) return st;
+    if (!g) return invalid("bwd is NULL");
+    if (!g->dy || !g->du || !g->ddelta || !g->dA || !g->dB || !g->dC)
+        return invalid("dy, du, ddelta, dA, dB and dC are required");
+    if ((args->z && !g->dz) || (args->D && !g->dD) || (args->delta_bias && !g->ddelta_bias))
+        return invalid("dz, dD and ddelta_bias are required when z, D and delta_bias are given");
+    if (g->dy_batch_stride < 0 || g->dy_dim_stride < 0 || g->du_batch_stride < 0 || g->du_dim_stride < 0 ||
+        g->ddelta_batch_stride < 0 || g->ddelta_dim_stride < 0 ||
+        (g->dz && (g->dz_batch_stride < 0 || g->dz_dim_stride < 0)))
+        return invalid("gradient strides must be non-negative");
+    const int eb = args->in_dtype == MS_F32 ? 4 : 2;
+    if (!elem_aligned(g->dy, eb) || !elem_aligned(g->du, eb) || !elem_aligned(g->ddelta, eb) ||
+        (g->dz && !elem_aligned(g->dz, eb)) || !elem_aligned(g->dA, 4) || !elem_aligned(g->dB, 4) ||
+        !elem_aligned(g->dC, 4) || (g->dD && !elem_aligned(g->dD, 4)) ||
+        (g->ddelta_bias && !elem_aligned(g->ddelta_bias, 4)) ||
+        (g->dfinal_state && !elem_aligned(g->dfinal_state, 4)) ||
+        (g->dinitial_state && !elem_aligned(g->dinitial_state, 4))) {
+        set_error("a gradient pointer is not aligned to its element size");
+        return MS_ERR_ALIGNMENT;
+    }
+    const ms::ScanParams p = to_params(args);
+    const size_t need = ms::bwd_workspace_bytes(p);
+    if (!workspace || workspace_bytes < need) {
+        set_error("workspace of %zu bytes needed, %zu given", need, workspace ? workspace_bytes : static_cast<size_t>(0));
+        return MS_ERR_WORKSPACE;
+    }
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) {
+        set_error("workspace must be 256-byte aligned");
+        return MS_ERR_ALIGNMENT;
+    }
+    ms::BwdParams q{};
+    q.dy = g->dy; q.dy_sb = g->dy_batch_stride; q.dy_sd = g->dy_dim_stride;
+    q.dhT = g->dfinal_state;
+    q.du = g->du; q.du_sb = g->du_batch_stride; q.du_sd = g->du_dim_stride;
+    q.ddelta = g->ddelta; q.dd_sb = g->ddelta_batch_stride; q.dd_sd = g->ddelta_dim_stride;
+    q.dz = g->dz; q.dz_sb = g->dz_batch_stride; q.dz_sd = g->dz_dim_stride;
+    q.dA = g->dA; q.dB = g->dB; q.dC = g->dC; q.dD = g->dD; q.dbias = g->ddelta_bias;
+    q.dh0 = g->dinitial_state;
+    q.ckpt = static_cast<float *>(workspace);
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t bc = static_cast<size_t>(args->batch * args->dstate * args->seqlen) * sizeof(float);
+    cudaError_t e = cudaMemsetAsync(g->dA, 0, static_cast<size_t>(args->dim * args->dstate) * sizeof(float), s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(g->dB, 0, bc, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(g->dC, 0, bc, s);
+    if (e == cudaSuccess && g->dD) e = cudaMemsetAsync(g->dD, 0, static_cast<size_t>(args->dim) * sizeof(float), s);
+    if (e == cudaSuccess && g->ddelta_bias)
+        e = cudaMemsetAsync(g->ddelta_bias, 0, static_cast<size_t>(args->dim) * sizeof(float), s);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the gradient accumulators");
+    e = ms::launch_bwd(p, q, args->in_dtype, s);
+    if (e != cudaSuccess) return cuda_fail(e, "backward kernel launch");
+    return MS_OK;
+}
+
 }  // extern "C"

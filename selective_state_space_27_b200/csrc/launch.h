@@ -74,6 +74,23 @@ int rec_ctas_per_sm(int in_dtype, int lanes_per_row, bool vec, int variant);
 bool rec_supports_variant(int lanes_per_row, int variant);
 cudaError_t launch_rec(const ScanParams &p, int lanes_per_row, bool vec, int in_dtype, cudaStream_t stream);
 
+// Backward pass (scan_bwd.cu): output gradients in, input gradients out.
+// du, ddelta, dz: (batch, dim, L) in the input dtype; dB, dC: (batch, dstate,
+// L) float32 contiguous; dA (dim, dstate), dD and dbias (dim), dh0 (batch,
+// dim, dstate) float32. dA, dB, dC, dD and dbias are accumulated with atomics
+// and must be zero before the launch. ckpt: bwd_workspace_bytes(p) bytes.
+struct BwdParams {
+    const void *dy;    int64_t dy_sb, dy_sd;
+    const float *dhT;
+    void *du;          int64_t du_sb, du_sd;
+    void *ddelta;      int64_t dd_sb, dd_sd;
+    void *dz;          int64_t dz_sb, dz_sd;
+    float *dA, *dB, *dC, *dD, *dbias, *dh0;
+    float *ckpt;
+};
+size_t bwd_workspace_bytes(const ScanParams &p);
+cudaError_t launch_bwd(const ScanParams &p, const BwdParams &q, int in_dtype, cudaStream_t stream);
+
 struct UpdateParams {
     int64_t batch, dim, dstate;
     float *state;      int64_t s_sb, s_sd;

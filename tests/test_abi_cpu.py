@@ -192,3 +192,49 @@ def test_trap_scan_validation_rejects(lib, lam, sb, sd, segments, status):
     a.force_segments = segments
     assert lib.mamba_trap_scan_fwd(ctypes.byref(a), lam, sb, sd, None, None) == status
     assert lib.mamba_last_error().decode() != ""
+
+
+def test_bwd_struct_layout_matches_binding(tmp_path):
+    src = tmp_path / "bwd_layout.c"
+    src.write_text(
+        '#include <stdio.h>\n#include <stddef.h>\n#include "mambascan.h"\n'
+        "int main(void){printf(\"%zu %zu %zu %zu\\n\", sizeof(ms_scan_bwd_args), offsetof(ms_scan_bwd_args, dz),"
+        " offsetof(ms_scan_bwd_args, dA), offsetof(ms_scan_bwd_args, dinitial_state)); return 0;}\n")
+    exe = tmp_path / "bwd_layout"
+    subprocess.check_call(["gcc", "-std=c11", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe)])
+    got = [int(v) for v in subprocess.check_output([str(exe)], text=True).split()]
+    want = [ctypes.sizeof(ms.ScanBwdArgs), ms.ScanBwdArgs.dz.offset, ms.ScanBwdArgs.dA.offset,
+            ms.ScanBwdArgs.dinitial_state.offset]
+    assert got == want
+
+
+def _valid_bwd():
+    g = ms.ScanBwdArgs()
+    base = 1 << 20
+    g.dy, g.dy_batch_stride, g.dy_dim_stride = base * 20, 512, 64
+    g.du, g.du_batch_stride, g.du_dim_stride = base * 21, 512, 64
+    g.ddelta, g.ddelta_batch_stride, g.ddelta_dim_stride = base * 22, 512, 64
+    g.dA, g.dB, g.dC = base * 23, base * 24, base * 25
+    return g
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("dy", None, 1), ("du", None, 1), ("dA", None, 1), ("dy_batch_stride", -1, 1),
+    ("dy", (1 << 20) * 20 + 1, 3), ("dB", (1 << 20) * 24 + 2, 3),
+])
+def test_bwd_validation_rejects(lib, field, value, status):
+    g = _valid_bwd()
+    setattr(g, field, value)
+    assert lib.mamba_scan_bwd(ctypes.byref(_valid_scan_args()), ctypes.byref(g), (1 << 20) * 30, 1 << 30,
+                              None) == status
+
+
+def test_bwd_needs_workspace_and_matching_gradients(lib):
+    a = _valid_scan_args()
+    assert lib.mamba_scan_bwd(ctypes.byref(a), None, None, 0, None) == 1
+    assert lib.mamba_scan_bwd(ctypes.byref(a), ctypes.byref(_valid_bwd()), None, 0, None) == 6
+    n = ctypes.c_size_t(0)
+    assert lib.mamba_scan_bwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
+    assert n.value == 2 * 8 * 4 * 16 * 4
+    a.D = (1 << 20) * 7                      # D given: dD required
+    assert lib.mamba_scan_bwd(ctypes.byref(a), ctypes.byref(_valid_bwd()), (1 << 20) * 30, 1 << 30, None) == 1
