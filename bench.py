@@ -64,6 +64,8 @@ def parse_args(argv=None):
                     help="steps of the scan with the fused convolution prologue (0 skips the leg)")
     ap.add_argument("--trap-steps", type=int, default=200,
                     help="steps of the exponential-trapezoidal scan (0 skips the leg)")
+    ap.add_argument("--bwd-steps", type=int, default=20,
+                    help="steps of the scan backward (0 skips the leg)")
     ap.add_argument("--decode-steps", type=int, default=1000,
                     help="decode state-update steps timed on the (256, 5120, 16) decode workload (0: skip)")
     return ap.parse_args(argv)
@@ -430,6 +432,7 @@ def run_ours(args, dist: Dist):
     prologue = (run_prologue(args, dist, dev, w, sets, params, y, hT, counts, mufu_peak)
                 if args.prologue_steps > 0 else None)
     trap = run_trap(args, dist, dev, w, sets, params, y, hT, counts, mufu_peak) if args.trap_steps > 0 else None
+    bwd = run_bwd(args, dist, dev, w, sets, params, counts, mufu_peak) if args.bwd_steps > 0 else None
 
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
@@ -443,7 +446,7 @@ def run_ours(args, dist: Dist):
         "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded)", "config": workload_config(w, {"global_batch": w.batch * dist.world}),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode, "conv_prologue": prologue,
-        "trapezoidal": trap,
+        "trapezoidal": trap, "backward": bwd,
         "gpu_launches": args.steps * launches_per_step, "clocks": clocks,
     }
     if dist.rank == 0:
@@ -544,6 +547,72 @@ def run_trap(args, dist: Dist, dev, w, sets, params, y, hT, counts, mufu_peak):
                      "peak": mufu_peak / 1e12, "frac": mufu / (us * 1e-6) / mufu_peak, "algorithmic_mufu": mufu,
                      "note": "bytes as the plain scan + lambda_raw read once"},
         "gpu_launches": n,
+    }
+
+
+def run_bwd(args, dist: Dist, dev, w, sets, params, counts, mufu_peak):
+    """Time the scan backward (gradients for a seeded dy, recomputing the
+    states from 16-step checkpoints) on the headline workload, through the C
+    ABI with preallocated outputs and workspace."""
+    import ctypes
+
+    import torch
+    import selective_state_space_27_b200 as ms
+    from selective_state_space_27_b200.inputs import bf16_bits_from_f32
+
+    g = np.random.default_rng(w.seed + 1000 * dist.rank + 5)
+    dy_np = g.normal(size=(w.batch, w.dim, w.seqlen)).astype(np.float32)
+    dy = torch.from_numpy(dy_np if w.dtype == "f32" else bf16_bits_from_f32(dy_np))
+    dy = (dy.view(torch.bfloat16) if w.dtype == "bf16" else dy).to(dev)
+    s0 = sets[0]
+    args0 = ms.build_scan_args(s0["u"], s0["delta"], params["A"], s0["B"], s0["C"], s0["u"], D=params["D"],
+                               z=s0.get("z"), delta_bias=params["delta_bias"])
+    f32 = dict(device=dev, dtype=torch.float32)
+    outs = {"du": torch.empty_like(s0["u"]), "ddelta": torch.empty_like(s0["u"]),
+            "dz": torch.empty_like(s0["u"]) if w.has_z else None, "dA": torch.empty((w.dim, w.dstate), **f32),
+            "dB": torch.empty((w.batch, w.dstate, w.seqlen), **f32),
+            "dC": torch.empty((w.batch, w.dstate, w.seqlen), **f32), "dD": torch.empty(w.dim, **f32),
+            "ddelta_bias": torch.empty(w.dim, **f32)}
+    gb = ms.ScanBwdArgs()
+    gb.dy, gb.dy_batch_stride, gb.dy_dim_stride = dy.data_ptr(), dy.stride(0), dy.stride(1)
+    for k in ("du", "ddelta", "dz"):
+        if outs[k] is not None:
+            setattr(gb, k, outs[k].data_ptr())
+            setattr(gb, f"{k}_batch_stride", outs[k].stride(0))
+            setattr(gb, f"{k}_dim_stride", outs[k].stride(1))
+    for k in ("dA", "dB", "dC", "dD", "ddelta_bias"):
+        setattr(gb, k, outs[k].data_ptr())
+    lib = ms.load_library()
+    n_ws = ctypes.c_size_t(0)
+    lib.mamba_scan_bwd_workspace_size(ctypes.byref(args0), ctypes.byref(n_ws))
+    ws = torch.empty(max(n_ws.value, 256), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        rc = lib.mamba_scan_bwd(ctypes.byref(args0), ctypes.byref(gb), ws.data_ptr(), ws.numel(), stream.cuda_stream)
+        if rc != 0:
+            raise ms.MambaScanError(rc, lib.mamba_last_error().decode())
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    n = args.bwd_steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    us = dist.max(e0.elapsed_time(e1) * 1e3 / n, dev)
+    rows_t = w.batch * w.dim * w.seqlen
+    mufu = 2 * counts["elements"] + 6 * rows_t   # forward sweep + recompute ex2 per element; softplus, gates per (b,d,t)
+    return {
+        "workload": w.name, "steps": n, "metric": "scan backward B*D*L*N elems/s", "unit": UNIT,
+        "value": dist.world * counts["elements"] / (us * 1e-6), "us_per_step": us,
+        "roofline": {"bound": "alu", "unit": "Tmufu/s", "achieved": mufu / (us * 1e-6) / 1e12,
+                     "peak": mufu_peak / 1e12, "frac": mufu / (us * 1e-6) / mufu_peak, "algorithmic_mufu": mufu,
+                     "note": "two ex2 per element: the checkpoint sweep and the per-chunk recomputation"},
+        "gpu_launches": 6 * n,
     }
 
 

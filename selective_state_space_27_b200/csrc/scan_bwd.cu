@@ -19,10 +19,12 @@
 // float per chain and chunk: 1/16 of the expanded state). Phase B walks the
 // chunks backward: it recomputes the chunk's 16 states from the previous
 // checkpoint into registers and runs the adjoint recurrence through them.
-// Per-(row, t) sums over the 16 states use half-warp shuffles; the B and C
-// gradients are summed over the CTA's rows in shared memory and added to
-// global memory with atomics, as are the A, D and delta_bias gradients (sums
-// over the batch). The caller's reduction outputs are zeroed first.
+// Per-(row, t) sums over the 16 states go through [row][state][step] tiles
+// in shared memory (written by the chain threads, summed by one thread per
+// (row, step); both access patterns are free of bank conflicts); the B and C
+// gradients are summed over the CTA's rows the same way and added to global
+// memory with atomics, as are the A, D and delta_bias gradients (sums over
+// the batch). The caller's reduction outputs are zeroed first.
 #include <type_traits>
 
 #include "device_math.cuh"
@@ -48,12 +50,27 @@ __device__ __forceinline__ float half_warp_sum(float v) {
     return v;
 }
 
+// Dynamic shared memory of a CTA, in floats.
+constexpr int kRT = kRows * (kT + 1);            // a [row][step] tile
+constexpr int kTN = kT * (kN + 1);               // a [step][state] tile
+constexpr int kRNT = kRows * kN * (kT + 1);      // a [row][state][step] (or [step][row][state]) tile
+constexpr int kBwdSmemFloats = 4 * kRT + 2 * kTN + 4 * kRNT;
+
 template <typename T>
 __global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(const ScanParams p, const BwdParams q) {
-    __shared__ float dts[kRows][kT + 1], dus[kRows][kT + 1], uus[kRows][kT + 1], dss[kRows][kT + 1];
-    __shared__ float Bs[kT][kN + 1], Cs[kT][kN + 1];
-    __shared__ float pB[kT][kRows][kN + 1], pC[kT][kRows][kN + 1];
-    __shared__ float rdu[kRows][kT + 1], rdd[kRows][kT + 1];
+    extern __shared__ __align__(16) float smf[];
+    auto dts = reinterpret_cast<float (*)[kT + 1]>(smf);
+    auto dus = reinterpret_cast<float (*)[kT + 1]>(smf + kRT);
+    auto uus = reinterpret_cast<float (*)[kT + 1]>(smf + 2 * kRT);
+    auto dss = reinterpret_cast<float (*)[kT + 1]>(smf + 3 * kRT);
+    auto Bs = reinterpret_cast<float (*)[kN + 1]>(smf + 4 * kRT);
+    auto Cs = reinterpret_cast<float (*)[kN + 1]>(smf + 4 * kRT + kTN);
+    float *tiles = smf + 4 * kRT + 2 * kTN;
+    auto pB = reinterpret_cast<float (*)[kRows][kN + 1]>(tiles);              // [step][row][state]
+    auto pC = reinterpret_cast<float (*)[kRows][kN + 1]>(tiles + kRNT);
+    auto pS = reinterpret_cast<float (*)[kN][kT + 1]>(tiles);                 // [row][state][step], before pB
+    auto pDU = reinterpret_cast<float (*)[kN][kT + 1]>(tiles + 2 * kRNT);
+    auto pDD = reinterpret_cast<float (*)[kN][kT + 1]>(tiles + 3 * kRNT);
 
     const int tid = threadIdx.x;
     const int r = tid / kN, n = tid % kN;          // chain (row, state); also item (row, step n)
@@ -72,31 +89,50 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(const ScanParams p,
     const float Dd = p.D ? __ldg(p.D + dc) : 0.f;
     float *ckpt = q.ckpt + row * nchunks * kN + n;
 
-    // Stage chunk c: per (row, step) delta, delta u and u; per (step, state) B (and C).
-    auto stage = [&](int64_t c, bool with_c) {
-        const int64_t t = c * kT + n;                 // item (row r, step n)
-        const bool in = ok && t < L;
-        float u = 0.f, dt = 0.f;
-        if (in) {
-            u = ldv<T>(p.u, b * p.u_sb + dc * p.u_sd + t);
-            float v = ldv<T>(p.delta, b * p.dl_sb + dc * p.dl_sd + t) + bias;
-            dt = p.softplus ? softplus(v) : v;
+    // The raw values one thread contributes to chunk c's tiles: item (row r,
+    // step n) -- u, delta_raw, dy, z -- and (step, state) (tid / 16, tid % 16)
+    // of the B and C tiles. Loaded one chunk ahead of use, so the global
+    // latency hides behind the current chunk's work.
+    struct RawVals { float u, dl, dy, z, bv, cv; };
+    auto load_raw = [&](int64_t c, bool grads) {
+        RawVals v{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        const int64_t t = c * kT + n;
+        if (ok && t < L) {
+            v.u = ldv<T>(p.u, b * p.u_sb + dc * p.u_sd + t);
+            v.dl = ldv<T>(p.delta, b * p.dl_sb + dc * p.dl_sd + t);
+            if (grads) {
+                v.dy = ldv<T>(q.dy, b * q.dy_sb + dc * q.dy_sd + t);
+                if (p.z) v.z = ldv<T>(p.z, b * p.z_sb + dc * p.z_sd + t);
+            }
         }
-        dts[r][n] = dt;                                // steps past the end: delta = 0 (identity)
-        dus[r][n] = dt * u;
-        uus[r][n] = u;
-        const int tt = tid / kN, nn = tid % kN;        // (step, state) of the B/C tile
+        const int tt = tid / kN, nn = tid % kN;
         const int64_t ts = c * kT + tt;
-        const bool bin = nn < dstate && ts < L;
-        Bs[tt][nn] = bin ? ldv<T>(p.B, b * p.B_sb + nn * p.B_sn + ts) : 0.f;
-        if (with_c) Cs[tt][nn] = bin ? ldv<T>(p.C, b * p.C_sb + nn * p.C_sn + ts) : 0.f;
+        if (nn < dstate && ts < L) {
+            v.bv = ldv<T>(p.B, b * p.B_sb + nn * p.B_sn + ts);
+            if (grads) v.cv = ldv<T>(p.C, b * p.C_sb + nn * p.C_sn + ts);
+        }
+        return v;
+    };
+    // Stage chunk c's tiles from its raw values: per (row, step) delta, delta u
+    // and u (steps past the end: delta = 0, the identity); per (step, state) B, C.
+    auto stage = [&](int64_t c, const RawVals &v) {
+        const bool in = ok && c * kT + n < L;
+        const float dt = in ? (p.softplus ? softplus(v.dl + bias) : v.dl + bias) : 0.f;
+        dts[r][n] = dt;
+        dus[r][n] = dt * v.u;
+        uus[r][n] = v.u;
+        Bs[tid / kN][tid % kN] = v.bv;
+        Cs[tid / kN][tid % kN] = v.cv;
     };
 
     // ---- Phase F: checkpoints at the end of every chunk but the last ----
     const float h_init = (live && p.h0) ? p.h0[row * dstate + n] : 0.f;
     float h = h_init;
+    RawVals nxt = nchunks > 1 ? load_raw(0, false) : RawVals{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int64_t c = 0; c + 1 < nchunks; ++c) {
-        stage(c, false);
+        const RawVals cur = nxt;
+        stage(c, cur);
+        if (c + 2 < nchunks) nxt = load_raw(c + 1, false);
         __syncthreads();
 #pragma unroll
         for (int t = 0; t < kT; ++t) h = fmaf(ex2_approx(dts[r][t] * A2), h, dus[r][t] * Bs[t][n]);
@@ -107,13 +143,15 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(const ScanParams p,
     // ---- Phase B ----
     float G = (live && ok && q.dhT) ? q.dhT[row * dstate + n] : 0.f;   // a_{t+1} g_{t+1}, carried down
     float dA_acc = 0.f, dD_acc = 0.f, dbias_acc = 0.f;
+    nxt = load_raw(nchunks - 1, true);
     for (int64_t c = nchunks - 1; c >= 0; --c) {
-        stage(c, true);
+        const RawVals cur = nxt;
+        stage(c, cur);
+        if (c > 0) nxt = load_raw(c - 1, true);
         // dy and z of item (row r, step n)
         const int64_t ti = c * kT + n;
         const bool in = ok && ti < L;
-        const float dyv = in ? ldv<T>(q.dy, b * q.dy_sb + dc * q.dy_sd + ti) : 0.f;
-        const float zv = (in && p.z) ? ldv<T>(p.z, b * p.z_sb + dc * p.z_sd + ti) : 0.f;
+        const float dyv = cur.dy, zv = cur.z;
         __syncthreads();
 
         // recompute the chunk's states from the previous checkpoint
@@ -128,13 +166,13 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(const ScanParams p,
                 H[t] = hh;
             }
         }
-        // ds, dz of item (row r, step n); s_t needs the row's sum over states
-        float s_mine = 0.f;
+        // ds, dz of item (row r, step n); s_t sums C h over the row's states
 #pragma unroll
-        for (int t = 0; t < kT; ++t) {
-            const float st = half_warp_sum(Cs[t][n] * H[t]);
-            if (t == n) s_mine = st + Dd * uus[r][t];
-        }
+        for (int t = 0; t < kT; ++t) pS[r][n][t] = Cs[t][n] * H[t];
+        __syncthreads();
+        float s_mine = Dd * uus[r][n];
+#pragma unroll
+        for (int nn = 0; nn < kN; ++nn) s_mine += pS[r][nn][n];
         float dsv = dyv;
         if (p.z) {
             const float sg = __fdividef(1.f, 1.f + ex2_approx(-zv * kLog2e));
@@ -155,12 +193,8 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(const ScanParams p,
             const float gn = fmaf(ds, Cs[t][n], G);
             pC[t][r][n] = ds * H[t];
             pB[t][r][n] = gn * dus[r][t];
-            const float du_p = half_warp_sum(gn * dt * Bv);
-            const float dd_p = half_warp_sum(gn * fmaf(Bv, uus[r][t], hprev * Av[t] * Areal));
-            if (n == t) {
-                rdu[r][t] = du_p;
-                rdd[r][t] = dd_p;
-            }
+            pDU[r][n][t] = gn * dt * Bv;
+            pDD[r][n][t] = gn * fmaf(Bv, uus[r][t], hprev * Av[t] * Areal);
             dA_acc = fmaf(gn * hprev, Av[t] * dt, dA_acc);
             G = Av[t] * gn;
         }
@@ -168,12 +202,13 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(const ScanParams p,
 
         // item (row r, step n): du, ddelta; B/C gradients of (step, state) = (tid / 16, tid % 16)
         if (in) {
-            const float du = fmaf(dss[r][n], Dd, rdu[r][n]);
-            float dd = rdd[r][n];
-            if (p.softplus) {
-                const float v = ldv<T>(p.delta, b * p.dl_sb + dc * p.dl_sd + ti) + bias;
-                dd *= __fdividef(1.f, 1.f + ex2_approx(-v * kLog2e));
+            float du = dss[r][n] * Dd, dd = 0.f;
+#pragma unroll
+            for (int nn = 0; nn < kN; ++nn) {
+                du += pDU[r][nn][n];
+                dd += pDD[r][nn][n];
             }
+            if (p.softplus) dd *= __fdividef(1.f, 1.f + ex2_approx(-(cur.dl + bias) * kLog2e));
             static_cast<T *>(q.du)[b * q.du_sb + dc * q.du_sd + ti] = from_f32<T>(du);
             static_cast<T *>(q.ddelta)[b * q.dd_sb + dc * q.dd_sd + ti] = from_f32<T>(dd);
             dbias_acc += dd;
@@ -217,10 +252,14 @@ size_t bwd_workspace_bytes(const ScanParams &p) {
 
 cudaError_t launch_bwd(const ScanParams &p, const BwdParams &q, int in_dtype, cudaStream_t stream) {
     const dim3 grid(static_cast<unsigned>((p.dim + kRows - 1) / kRows), static_cast<unsigned>(p.batch));
-    if (in_dtype == 0)
-        bwd_kernel<float><<<grid, kBwdThreads, 0, stream>>>(p, q);
-    else
-        bwd_kernel<__nv_bfloat16><<<grid, kBwdThreads, 0, stream>>>(p, q);
+    const int smem = kBwdSmemFloats * static_cast<int>(sizeof(float));
+    const void *k = in_dtype == 0 ? reinterpret_cast<const void *>(bwd_kernel<float>)
+                                  : reinterpret_cast<const void *>(bwd_kernel<__nv_bfloat16>);
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    void *args[] = {const_cast<ScanParams *>(&p), const_cast<BwdParams *>(&q)};
+    e = cudaLaunchKernel(k, grid, dim3(kBwdThreads), args, static_cast<size_t>(smem), stream);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
