@@ -45,7 +45,7 @@ MUFU_PER_CLK = 16
 # DRAM bytes (read + write) per launch from an ncu capture of the named kernel
 # on the named workload (profiles/ holds the summary); any other kernel or
 # workload reports traffic null.
-NCU_TRAFFIC = {("mamba130m_layer", "rec_kernel<bf16, 4>"): 152191744 + 31394560}
+NCU_TRAFFIC = {("mamba130m_layer", "rec_kernel<bf16, 4>"): 152201728 + 32785152}
 FP32_PER_CLK = 128
 
 
