@@ -73,9 +73,14 @@ template <int LPR, bool TRAP = false> struct Shape {
     static constexpr int IPR = LPR / 2;                 // I/O threads per row
     static constexpr int IP = kSteps / IPR;             // steps per I/O thread
     static constexpr bool GROUP_MAJOR = LPR <= 4;
+    // LPR 4: the four groups of a row sit in lanes r, r + 8, r + 16, r + 24 of
+    // one warp and sum their partial readouts with shuffles; the readout tile
+    // then holds one float per (row, step), YR floats per row (36: the 32
+    // stores of a warp fall on distinct banks).
+    static constexpr bool WARP_SUM = LPR == 4;
     static constexpr int XR = TRAP ? kSteps + 1 : kSteps / 2 + 1;   // float4 per row of the step tile
     static constexpr int YQ = LPR <= 4 ? 16 : 20;
-    static constexpr int YR = LPR == 2 ? 36 : LPR == 4 ? 68 : LPR == 8 ? 168 : 328;
+    static constexpr int YR = LPR == 2 ? 36 : LPR == 4 ? 36 : LPR == 8 ? 168 : 328;
     static constexpr int X_OFF = 0;
     static constexpr int Y_OFF = X_OFF + R * XR * 16;
     static constexpr int B_OFF = Y_OFF + R * YR * 4;
@@ -86,7 +91,8 @@ template <int LPR, bool TRAP = false> struct Shape {
     static constexpr int MINB = LPR == 2 ? 2 : LPR == 4 ? 3 : LPR == 8 ? 4 : 5;
     static_assert(R * IPR == kIoThreads, "the I/O threads cover the rows");
     static_assert(XR % 2 == 1, "odd row stride");
-    static_assert(YQ >= kSteps && YQ % 4 == 0 && YR >= LPR * YQ && YR % 4 == 0, "readout tile");
+    static_assert(YQ >= kSteps && YQ % 4 == 0 && (WARP_SUM ? YR >= kSteps : YR >= LPR * YQ) && YR % 4 == 0,
+                  "readout tile");
 };
 
 // The I/O warps' ring of raw inputs in shared memory, after the tile stages.
@@ -306,7 +312,22 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
     for (int64_t c = 0; c < nchunks; ++c, s = next_stage(s, kTileStages)) {
         unsigned char *st = smem + s * S::STAGE;
         const float4 *xrow = reinterpret_cast<const float4 *>(st + S::X_OFF) + r * S::XR;
-        float *yl = reinterpret_cast<float *>(st + S::Y_OFF) + r * S::YR + q * S::YQ;
+        float *yl = reinterpret_cast<float *>(st + S::Y_OFF) + r * S::YR + (S::WARP_SUM ? 0 : q * S::YQ);
+        // The partial readouts of steps t0 .. t0 + 3: stored per lane, or (LPR
+        // 4) summed over the row's four groups in a transposed reduction whose
+        // lane q keeps step t0 + q.
+        auto emit4 = [&](int t0, const float (&o)[4]) {
+            if constexpr (S::WARP_SUM) {
+                const bool hi = q & 2, lo = q & 1;
+                float k0 = hi ? o[2] : o[0], k1 = hi ? o[3] : o[1];
+                k0 += __shfl_xor_sync(0xffffffffu, hi ? o[0] : o[2], 16);
+                k1 += __shfl_xor_sync(0xffffffffu, hi ? o[1] : o[3], 16);
+                const float tot = (lo ? k1 : k0) + __shfl_xor_sync(0xffffffffu, lo ? k0 : k1, 8);
+                yl[t0 + q] = tot;
+            } else {
+                *reinterpret_cast<float4 *>(yl + t0) = make_float4(o[0], o[1], o[2], o[3]);
+            }
+        };
         const float *Bl = reinterpret_cast<const float *>(st + S::B_OFF) + q * NPL;
         const float *Cl = reinterpret_cast<const float *>(st + S::C_OFF) + q * NPL;
         bar_wait(bar_xf(s));
@@ -356,8 +377,7 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
                     }
                     outs[t & 3] = acc.x + acc.y;
                 }
-                if ((t & 3) == 3)
-                    *reinterpret_cast<float4 *>(yl + t - 3) = make_float4(outs[0], outs[1], outs[2], outs[3]);
+                if ((t & 3) == 3) emit4(t - 3, outs);
 #pragma unroll
                 for (int j = 0; j < NP; ++j) bprev[j] = cur.b[j];
                 if (t + 1 < kSteps) {
@@ -396,8 +416,7 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
                 }
                 outs[t & 3] = acc.x + acc.y;
             }
-            if ((t & 3) == 3)
-                *reinterpret_cast<float4 *>(yl + t - 3) = make_float4(outs[0], outs[1], outs[2], outs[3]);
+            if ((t & 3) == 3) emit4(t - 3, outs);
             if (t + 1 < kSteps) {
                 cur = nxt;
 #pragma unroll
@@ -587,7 +606,7 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
 #pragma unroll
         for (int e = 0; e < IP / 2; ++e) sum[e] = f2(0.f, 0.f);
 #pragma unroll
-        for (int j = 0; j < LPR; ++j) {
+        for (int j = 0; j < (S::WARP_SUM ? 1 : LPR); ++j) {
             if constexpr (IP == 2) {
                 sum[0] = add2(sum[0], *reinterpret_cast<const float2 *>(yp + j * S::YQ));
             } else {
