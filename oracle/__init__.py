@@ -2,9 +2,11 @@
 
 TEST INFRASTRUCTURE ONLY: imported by the tests, by the smoke check and by the
 benchmark's CPU-baseline leg. The product (the CUDA library and its binding)
-never imports it. The arithmetic lives in ``s6_oracle.c`` (plain C, double
-precision, OpenMP across independent rows); this module compiles it with gcc
-on first use and marshals numpy arrays into it.
+never imports it. The arithmetic lives in ``s6_oracle.c`` (the selective scan,
+its decode step, convolution prologue, trapezoidal variant and gradients) and
+``ssd_oracle.c`` (the Mamba-2 scalar-decay SSM in recurrent form): plain C,
+double precision, OpenMP across independent rows. This module compiles them
+with gcc on first use and marshals numpy arrays into them.
 """
 from __future__ import annotations
 
@@ -16,7 +18,7 @@ import threading
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_SRC = os.path.join(_HERE, "s6_oracle.c")
+_SRCS = [os.path.join(_HERE, "s6_oracle.c"), os.path.join(_HERE, "ssd_oracle.c")]
 _LIB = os.path.join(_HERE, "_build", "libs6oracle.so")
 _lock = threading.Lock()
 _lib = None
@@ -29,12 +31,12 @@ def build(force: bool = False) -> str:
     """Compile the oracle (gcc -O2, no fast-math, OpenMP) and return the .so path."""
     with _lock:
         if (not force and os.path.exists(_LIB)
-                and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC)):
+                and os.path.getmtime(_LIB) >= max(os.path.getmtime(s) for s in _SRCS)):
             return _LIB
         os.makedirs(os.path.dirname(_LIB), exist_ok=True)
         tmp = _LIB + f".{os.getpid()}.tmp"
         subprocess.check_call(["gcc", "-O2", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared",
-                               "-std=c11", "-Wall", "-Werror", _SRC, "-o", tmp, "-lm"])
+                               "-std=c11", "-Wall", "-Werror", *_SRCS, "-o", tmp, "-lm"])
         os.replace(tmp, _LIB)
         return _LIB
 
@@ -61,6 +63,10 @@ def _bind(path: str):
     lib.s6_oracle_scan_d.argtypes = [i64, i64, i64, i64] + [vp] * 8 + [ip, vp, vp, vp]
     lib.s6_oracle_scan_bwd.restype = ip
     lib.s6_oracle_scan_bwd.argtypes = [i64, i64, i64, i64] + [vp] * 8 + [ip] + [vp] * 12
+    lib.ssd_oracle_rec_d.restype = ip
+    lib.ssd_oracle_rec_d.argtypes = [i64, i64, i64] + [vp] * 6
+    lib.ssd_oracle_scan.restype = ip
+    lib.ssd_oracle_scan.argtypes = [i64] * 6 + [ip] + [vp] * 8 + [ip, vp, i64, vp, vp, vp, ip]
     lib.s6_oracle_max_threads.restype = ip
     lib.s6_oracle_max_threads.argtypes = []
     return lib
@@ -339,6 +345,66 @@ def scan_bwd(*, u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, delta_so
     return out
 
 
+def ssd_rec(*, a, B, C, X, H0=None, _lib_override=None):
+    """Recurrent form of one head in the page's parametrisation, in fp64:
+    H = a[t] H + X[t] B[t]^T, Y[t] = H C[t]. ``a`` (L,), ``B, C`` (L, N), ``X``
+    (L, P); ``H0`` optional (P, N). Returns ``(Y (L, P), H (P, N))``."""
+    a, B, C, X = (np.ascontiguousarray(v, dtype=np.float64) for v in (a, B, C, X))
+    L, P = X.shape
+    N = B.shape[1]
+    if a.shape != (L,) or B.shape != (L, N) or C.shape != (L, N):
+        raise ValueError("a must be (L,), B and C (L, N), X (L, P)")
+    H = np.zeros((P, N)) if H0 is None else np.array(H0, dtype=np.float64, order="C").reshape(P, N)
+    Y = np.empty((L, P))
+    lib = _lib_override or _load()
+    if lib.ssd_oracle_rec_d(L, P, N, _ptr(a), _ptr(B), _ptr(C), _ptr(X), _ptr(H), _ptr(Y)) != 0:
+        raise ValueError("oracle rejected its arguments")
+    return Y, H
+
+
+def ssd_scan(*, x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True, dtype="f32",
+             pairs=None, h0=None, threads: int = 0, _lib_override=None):
+    """Mamba-2 scalar-decay SSM forward in fp64 (recurrent form).
+
+    ``x, z``: (batch, L, nheads, headdim); ``dt``: (batch, L, nheads); ``B, C``:
+    (batch, L, ngroups, dstate) -- float32 arrays or uint16 bf16 bits according
+    to ``dtype``. ``A`` (nheads,), ``D`` and ``dt_bias`` (nheads,) float32.
+    ``pairs``: optional list of ``b*nheads + h`` to compute (default: all, in
+    order). ``h0``: optional initial state (n_pairs, headdim, dstate).
+
+    Returns ``(y, h)``: y (batch, L, nheads, headdim) float64 and the final
+    state (batch, nheads, headdim, dstate); with ``pairs``, y is
+    (n_pairs, L, headdim) and h (n_pairs, headdim, dstate).
+    """
+    dtc = _DTYPES[dtype]
+    x, dt, B, C, z = (_in(v, dtc) for v in (x, dt, B, C, z))
+    A, D, dt_bias = _f32(A), _f32(D), _f32(dt_bias)
+    batch, L, nheads, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    if dt.shape != (batch, L, nheads) or (z is not None and z.shape != x.shape):
+        raise ValueError("dt must be (batch, L, nheads) and z like x")
+    if B.shape != (batch, L, G, N) or C.shape != B.shape or A.shape != (nheads,):
+        raise ValueError("B, C must be (batch, L, ngroups, dstate) and A (nheads,)")
+    if pairs is None:
+        n_pairs, pairs_arr = batch * nheads, None
+    else:
+        pairs_arr = np.ascontiguousarray(pairs, dtype=np.int64)
+        n_pairs = pairs_arr.size
+    h0_arr = None if h0 is None else np.ascontiguousarray(h0, dtype=np.float64).reshape(n_pairs, P, N)
+    y = np.empty((n_pairs, L, P))
+    h = np.empty((n_pairs, P, N))
+    lib = _lib_override or _load()
+    rc = lib.ssd_oracle_scan(batch, L, nheads, P, G, N, dtc, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C),
+                             _ptr(D), _ptr(z), _ptr(dt_bias), int(bool(dt_softplus)), _ptr(pairs_arr), n_pairs,
+                             _ptr(h0_arr), _ptr(y), _ptr(h), int(threads))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    if pairs is None:
+        return (y.reshape(batch, nheads, L, P).transpose(0, 2, 1, 3).copy(),
+                h.reshape(batch, nheads, P, N))
+    return y, h
+
+
 class Variant:
     """The oracle's entry points bound to another build of the oracle source.
 
@@ -370,12 +436,20 @@ class Variant:
     def scan_bwd(self, **kw):
         return scan_bwd(_lib_override=self._lib, **kw)
 
+    def ssd_rec(self, **kw):
+        return ssd_rec(_lib_override=self._lib, **kw)
 
-def compile_source(src_path: str, so_path: str) -> str:
-    """Compile an oracle source file (same flags as :func:`build`)."""
+    def ssd_scan(self, **kw):
+        return ssd_scan(_lib_override=self._lib, **kw)
+
+
+def compile_source(src_paths, so_path: str) -> str:
+    """Compile oracle source files (same flags as :func:`build`) into one library."""
+    if isinstance(src_paths, str):
+        src_paths = [src_paths]
     subprocess.check_call(["gcc", "-O2", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared",
-                           "-std=c11", src_path, "-o", so_path, "-lm"])
+                           "-std=c11", *src_paths, "-o", so_path, "-lm"])
     return so_path
 
 
-SOURCE = _SRC
+SOURCES = tuple(_SRCS)

@@ -644,6 +644,152 @@ def pin_backward_linear_in_output_gradients(orc, seed=52):
         assert _rel(g3[k], 2.0 * g1[k] - 3.0 * g2[k]) <= 1e-12, k
 
 
+def _read_ssd_dual_check():
+    with open(os.path.join(GOLDEN, "ssd_dual_check.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                L, N, P, lo, hi, seed, printed = line.split()
+                return int(L), int(N), int(P), float(lo), float(hi), int(seed), float(printed)
+    raise AssertionError("ssd_dual_check.txt holds no case")
+
+
+def pin_ssd_page_check(orc):
+    """The page's printed duality check ("Notas sobre Mamba", "A forma dual:
+    atenção mascarada"): on its own seeded inputs, the recurrent form equals
+    Y = (Lmask o C B^T) X, Lmask_ji = prod_{k=i+1..j} a_k, to the rounding of
+    fp64 (the page prints a largest difference of 9.44e-15). The mask here is
+    built from explicit products, not from the page's cumulative log-sum.
+    """
+    L, N, P, lo, hi, seed, printed = _read_ssd_dual_check()
+    g = _rng(seed)
+    a = g.uniform(lo, hi, size=L)
+    B = g.normal(size=(L, N))
+    C = g.normal(size=(L, N))
+    X = g.normal(size=(L, P))
+    Y, _ = orc.ssd_rec(a=a, B=B, C=C, X=X)
+    mask = np.zeros((L, L))
+    for j in range(L):
+        for i in range(j + 1):
+            mask[j, i] = np.prod(a[i + 1:j + 1])
+    Yq = (mask * (C @ B.T)) @ X
+    diff = float(np.abs(Y - Yq).max())
+    assert diff <= 100.0 * printed, diff
+
+
+def _ssd_case(g, batch=2, L=23, nheads=4, ngroups=2, P=3, N=5, dtype="f32"):
+    t = dict(x=g.normal(size=(batch, L, nheads, P)), dt=g.normal(scale=0.5, size=(batch, L, nheads)),
+             B=g.normal(size=(batch, L, ngroups, N)), C=g.normal(size=(batch, L, ngroups, N)),
+             z=g.normal(size=(batch, L, nheads, P)))
+    t = {k: _f32(v) for k, v in t.items()}
+    p = dict(A=_f32(-g.uniform(1.0, 16.0, size=nheads)), D=_f32(g.uniform(0.5, 1.5, size=nheads)),
+             dt_bias=_f32(np.log(np.expm1(np.exp(g.uniform(np.log(1e-3), np.log(1e-1), size=nheads))))),
+             dt_softplus=True)
+    return t, p
+
+
+def pin_ssd_equals_selective_scan(orc, seed=60):
+    """A scalar transition per head is the selective scan with A[d, n] equal
+    to the head's A for every n ("Notas sobre Mamba", "A forma dual: atenção
+    mascarada"): each channel p of head h is an S6 row whose step, bias and
+    skip are the head's and whose B and C are the head's group's. Checked
+    against the (separately pinned) selective-scan oracle, including an
+    initial state and the final state."""
+    g = _rng(seed)
+    batch, L, H, G, P, N = 2, 23, 4, 2, 3, 5
+    t, p = _ssd_case(g, batch, L, H, G, P, N)
+    h0 = g.normal(size=(batch * H, P, N))
+    y, hT = orc.ssd_scan(**t, **p, h0=h0)
+    for b in range(batch):
+        for h in range(H):
+            grp = h // (H // G)
+            u = _f32(t["x"][b, :, h, :].T[None])
+            z = _f32(t["z"][b, :, h, :].T[None])
+            dl = _f32(np.broadcast_to(t["dt"][b, :, h], (1, P, L)))
+            Bs = _f32(t["B"][b, :, grp, :].T[None])
+            Cs = _f32(t["C"][b, :, grp, :].T[None])
+            ys, hs = orc.scan(u=u, delta=dl, A=_f32(np.full((P, N), p["A"][h])), B=Bs, C=Cs,
+                              D=_f32(np.full(P, p["D"][h])), z=z, delta_bias=_f32(np.full(P, p["dt_bias"][h])),
+                              delta_softplus=True, h0=h0[b * H + h])
+            assert _rel(y[b, :, h, :], ys[0].T) < 1e-12
+            assert _rel(hT[b, h], hs[0]) < 1e-12
+
+
+def pin_ssd_layer_quadratic(orc, seed=61):
+    """The whole layer (softplus step with bias, skip, gate, two groups) in
+    its dual form: per head, y = (Lmask o C_g B_g^T)(delta x) + D x, gated by
+    z sigmoid(z), with Lmask_ji = exp(S_j - S_i), S = cumsum(delta A) ("Notas
+    sobre Mamba", "A forma dual: atenção mascarada"; "Mamba-2 e State Space
+    Duality (SSD)", "A teoria do State Space Duality (SSD) no Mamba-2").
+    softplus and the sigmoid come from numpy and scipy."""
+    g = _rng(seed)
+    batch, L, H, G, P, N = 2, 31, 4, 2, 3, 6
+    t, p = _ssd_case(g, batch, L, H, G, P, N)
+    y, _ = orc.ssd_scan(**t, **p)
+    for b in range(batch):
+        for h in range(H):
+            grp = h // (H // G)
+            dl = np.logaddexp(0.0, t["dt"][b, :, h].astype(np.float64) + float(p["dt_bias"][h]))
+            S = np.cumsum(dl * float(p["A"][h]))
+            mask = np.tril(np.exp(S[:, None] - S[None, :]))
+            Bm = t["B"][b, :, grp, :].astype(np.float64)
+            Cm = t["C"][b, :, grp, :].astype(np.float64)
+            X = t["x"][b, :, h, :].astype(np.float64)
+            zz = t["z"][b, :, h, :].astype(np.float64)
+            yref = ((mask * (Cm @ Bm.T)) @ (dl[:, None] * X) + float(p["D"][h]) * X) * zz * expit(zz)
+            assert _rel(y[b, :, h, :], yref) < 1e-12
+
+
+def pin_ssd_segmentation_and_pairs(orc, seed=62, m=11):
+    """The layer over [0, L) equals the layer over [0, m) continued from its
+    final state over [m, L) (state passing between blocks, "Notas sobre
+    Mamba", "O algoritmo SSD"); a listed subset of (batch, head) pairs gives
+    the same rows as the full run."""
+    g = _rng(seed)
+    batch, L, H, G, P, N = 2, 29, 4, 1, 4, 3
+    t, p = _ssd_case(g, batch, L, H, G, P, N)
+    y, hT = orc.ssd_scan(**t, **p)
+    y1, h1 = orc.ssd_scan(**{k: _f32(v[:, :m]) for k, v in t.items()}, **p)
+    y2, h2 = orc.ssd_scan(**{k: _f32(v[:, m:]) for k, v in t.items()}, **p, h0=h1.reshape(batch * H, P, N))
+    assert _rel(np.concatenate([y1, y2], axis=1), y) < 1e-13
+    assert _rel(h2, hT) < 1e-13
+    ys, hs = orc.ssd_scan(**t, **p, pairs=[5, 0])
+    assert np.array_equal(ys[0], y[1, :, 1, :]) and np.array_equal(ys[1], y[0, :, 0, :])
+    assert np.array_equal(hs[0], hT[1, 1]) and np.array_equal(hs[1], hT[0, 0])
+
+
+def pin_ssd_zero_step_keeps_state(orc, seed=63):
+    """delta = 0 (no bias, no softplus): a_t = 1 and the input term vanishes,
+    so the state stays at h0 and y_t = h0 C_t + D x_t ("Notas sobre Mamba",
+    "O mecanismo de seleção (S6)": a small step keeps the state and ignores
+    the token)."""
+    g = _rng(seed)
+    batch, L, H, G, P, N = 1, 9, 2, 1, 3, 4
+    t, p = _ssd_case(g, batch, L, H, G, P, N)
+    t["dt"] = _f32(np.zeros_like(t["dt"]))
+    t.pop("z")
+    h0 = g.normal(size=(batch * H, P, N))
+    y, hT = orc.ssd_scan(**t, A=p["A"], D=p["D"], dt_softplus=False, h0=h0)
+    for h in range(H):
+        C = t["C"][0, :, 0, :].astype(np.float64)
+        yref = C @ h0[h].T + float(p["D"][h]) * t["x"][0, :, h, :].astype(np.float64)
+        assert _rel(y[0, :, h, :], yref) < 1e-14
+        assert np.array_equal(hT[0, h], h0[h])
+
+
+def pin_ssd_bf16_decoding(orc, seed=64):
+    """bf16 inputs are read as their exact float32 values: the layer on bf16
+    bit patterns equals the layer on the same values widened to float32."""
+    g = _rng(seed)
+    t, p = _ssd_case(g, 1, 13, 2, 1, 4, 3)
+    bits = {k: (np.ascontiguousarray(v).view(np.uint32) >> np.uint32(16)).astype(np.uint16) for k, v in t.items()}
+    wide = {k: (b.astype(np.uint32) << np.uint32(16)).view(np.float32) for k, b in bits.items()}
+    y16, h16 = orc.ssd_scan(**bits, **p, dtype="bf16")
+    y32, h32 = orc.ssd_scan(**wide, **p, dtype="f32")
+    assert np.array_equal(y16, y32) and np.array_equal(h16, h32)
+    assert _rel(y16, orc.ssd_scan(**t, **p, dtype="f32")[0]) > 1e-6
+
+
 ALL_PINS = [
     pin_selection_step,
     pin_lti_convolution,
@@ -669,4 +815,10 @@ ALL_PINS = [
     pin_double_forward_matches_scan,
     pin_backward_finite_differences,
     pin_backward_linear_in_output_gradients,
+    pin_ssd_page_check,
+    pin_ssd_equals_selective_scan,
+    pin_ssd_layer_quadratic,
+    pin_ssd_segmentation_and_pairs,
+    pin_ssd_zero_step_keeps_state,
+    pin_ssd_bf16_decoding,
 ]

@@ -8,7 +8,7 @@ import pytest
 import oracle
 from tests import oracle_pins
 
-# (name, text in s6_oracle.c, replacement)
+# (name, text in one of the oracle sources, replacement)
 MUTANTS = [
     ("drop_skip_term", "acc += (double)D[d] * x;\n        if (z)\n            acc *= silu(load_value(z, dtype, i));\n        y[t] = acc;",
      "acc += 0.0 * x;\n        if (z)\n            acc *= silu(load_value(z, dtype, i));\n        y[t] = acc;"),
@@ -58,17 +58,40 @@ MUTANTS = [
     ("bwd_carry_not_decayed", "g[n] = a * gn;", "g[n] = gn;"),
     ("conv_decode_taps_reversed", "acc += (double)conv_w[d * width + k] * cs[k];",
      "acc += (double)conv_w[d * width + width - 1 - k] * cs[k];"),
+    ("ssd_group_index_modulo", "g = h / heads_per_group;", "g = h % ngroups;"),
+    ("ssd_skip_dropped", "acc += (double)D[h] * xv;", "acc += 0.0 * xv;"),
+    ("ssd_decay_sign", "const double a = exp(delta * (double)A[h]);", "const double a = exp(-delta * (double)A[h]);"),
+    ("ssd_input_not_discretised", "const double xbar = delta * xv;", "const double xbar = xv;"),
+    ("ssd_readout_reads_C_as_B", "acc += *hpn * ssd_load(C, dtype, brow + n);",
+     "acc += *hpn * ssd_load(B, dtype, brow + n);"),
+    ("ssd_bias_after_softplus",
+     "if (dt_bias)\n                delta += (double)dt_bias[h];\n            if (dt_softplus)\n"
+     "                delta = delta > 20.0 ? delta : log1p(exp(delta));",
+     "if (dt_softplus)\n                delta = delta > 20.0 ? delta : log1p(exp(delta));\n"
+     "            if (dt_bias)\n                delta += (double)dt_bias[h];"),
+    ("ssd_gate_dropped", "acc *= zv / (1.0 + exp(-zv));", "acc *= 1.0 + 0.0 * zv;"),
+    ("ssd_state_not_reset_per_pair", "H[i] = h0 ? h0[r * P * N + i] : 0.0;",
+     "H[i] = h0 ? h0[r * P * N + i] : (r > 0 ? 0.25 : 0.0);"),
+    ("ssd_bf16_shift", "<< 16u;", "<< 15u;"),
+    ("ssd_rec_decay_applied_to_input", "*hpn = a[t] * *hpn + X[t * P + p] * B[t * N + n];",
+     "*hpn = a[t] * (*hpn + X[t * P + p] * B[t * N + n]);"),
+    ("ssd_rec_readout_before_update",
+     "*hpn = a[t] * *hpn + X[t * P + p] * B[t * N + n];\n                acc += *hpn * C[t * N + n];",
+     "acc += *hpn * C[t * N + n];\n                *hpn = a[t] * *hpn + X[t * P + p] * B[t * N + n];"),
 ]
 
 
 @pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
 def test_pins_catch_mutant(tmp_path, name, old, new):
-    src = open(oracle.SOURCE).read()
-    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
-    path = os.path.join(tmp_path, f"mutant_{name}.c")
-    with open(path, "w") as f:
-        f.write(src.replace(old, new))
-    orc = oracle.Variant(oracle.compile_source(path, os.path.join(tmp_path, f"{name}.so")))
+    texts = {src: open(src).read() for src in oracle.SOURCES}
+    assert sum(t.count(old) for t in texts.values()) == 1, f"mutation site for {name} not found exactly once"
+    paths = []
+    for src, text in texts.items():
+        path = os.path.join(tmp_path, os.path.basename(src))
+        with open(path, "w") as f:
+            f.write(text.replace(old, new))
+        paths.append(path)
+    orc = oracle.Variant(oracle.compile_source(paths, os.path.join(tmp_path, f"{name}.so")))
     caught = []
     for pin in oracle_pins.ALL_PINS:
         try:
