@@ -6,7 +6,10 @@
  *  mamba_scan_fwd      the fused selective scan over a whole sequence
  *  mamba_state_update  the single-token state update used for decoding
  *
- * Both compute, per channel row (b, d) and state index n < dstate,
+ * and, beside them, the convolution prologue, the trapezoidal (Mamba-3) rule,
+ * the backward pass and the Mamba-2 chunked SSD forward (mamba_ssd_fwd,
+ * documented with its own arguments further down). The first two compute,
+ * per channel row (b, d) and state index n < dstate,
  *
  *   delta   = delta_raw + delta_bias[d]            (bias, if given, added first)
  *   delta   = log(1 + exp(delta))                  if delta_softplus (identity above 20)
@@ -70,7 +73,7 @@ typedef enum ms_status {
     MS_ERR_UNSUPPORTED = 2,  /* valid but outside what the kernels support (dstate>16)   */
     MS_ERR_ALIGNMENT = 3,    /* a pointer is not aligned to its element size             */
     MS_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed              */
-    MS_ERR_TIMEOUT = 5,      /* reserved: a bounded device wait gave up (none is used)    */
+    MS_ERR_TIMEOUT = 5,      /* a bounded device wait gave up (SSD status word only)       */
     MS_ERR_WORKSPACE = 6     /* workspace missing or smaller than the size asked for      */
 } ms_status;
 
@@ -349,6 +352,77 @@ ms_status mamba_scan_bwd_workspace_size(const ms_scan_args *args, size_t *bytes)
  */
 ms_status mamba_scan_bwd(const ms_scan_args *args, const ms_scan_bwd_args *bwd, void *workspace,
                          size_t workspace_bytes, void *stream);
+
+/* ---- Mamba-2 scalar-decay SSM (structured state space duality, SSD) --------
+ * Per batch b and head h, sequentially in t, on a state H of 64 x 128 values
+ * (headdim x dstate):
+ *     delta = dt[b,t,h] + dt_bias[h];  delta = log(1 + exp(delta)) if dt_softplus
+ *     H     = exp(delta A[h]) H + (delta x[b,t,h,:]) B[b,t,g,:]^T
+ *     y[b,t,h,:] = H C[b,t,g,:] + D[h] x[b,t,h,:];  y *= z sigmoid(z) if z
+ * with g = h / (nheads / ngroups). Sources: "Notas sobre Mamba", section "A
+ * forma dual: atenção mascarada" (Abar_t = a_t I and the recurrent form of
+ * its check) and section "O algoritmo SSD" (diagonal blocks by the quadratic
+ * form, off-diagonal blocks by passing a state from block to block);
+ * "Mamba-2 e State Space Duality (SSD)", sections "A teoria do State Space
+ * Duality (SSD) no Mamba-2" (decay exp(sum delta_k a_k)) and "O algoritmo de
+ * decomposição em blocos do SSD" (fixed blocks, tensor cores inside a block,
+ * a recurrent scan of block states between blocks).
+ *
+ * Layouts (element strides; the listed inner axes are contiguous):
+ *   x, z, y : (batch, seqlen, nheads, 64) bf16, head and headdim axes contiguous
+ *   dt      : (batch, seqlen, nheads) bf16, head axis contiguous
+ *   B, C    : (batch, seqlen, ngroups, 128) bf16, group and state axes contiguous
+ *   A       : (nheads) float32, usually -exp(A_log); D, dt_bias: (nheads) or NULL
+ *   initial_state, final_state : (batch, nheads, 64, 128) float32 contiguous, or NULL
+ * Only bf16 inputs, headdim 64 and dstate 128 are supported. The batch and
+ * token strides of x, z, y, B and C must be multiples of 8 elements and their
+ * base pointers 16-byte aligned (the kernel moves them in 16-byte pieces and
+ * through tensor maps); x's token stride must be at least nheads * 64 and the
+ * token stride of B and C at least ngroups * 128.
+ */
+#define MS_SSD_HEADDIM 64
+#define MS_SSD_DSTATE 128
+typedef struct ms_ssd_args {
+    int64_t batch, seqlen, nheads, ngroups;
+    int32_t in_dtype;        /* MS_BF16 */
+    int32_t dt_softplus;
+
+    const void *x;      int64_t x_batch_stride, x_token_stride;
+    const void *dt;     int64_t dt_batch_stride, dt_token_stride;
+    const void *B;      int64_t B_batch_stride, B_token_stride;
+    const void *C;      int64_t C_batch_stride, C_token_stride;
+    const void *z;      int64_t z_batch_stride, z_token_stride;    /* z may be NULL */
+    void *y;            int64_t y_batch_stride, y_token_stride;
+
+    const float *A;
+    const float *D;
+    const float *dt_bias;
+    const float *initial_state;
+    float *final_state;
+} ms_ssd_args;
+
+/* Device workspace of mamba_ssd_fwd: a status word (int32 at offset 0). */
+#define MS_SSD_WORKSPACE_BYTES 256
+
+/*
+ * SSD forward: one kernel launch on `stream` (after clearing the status word),
+ * one CTA per (batch, head) walking the sequence in blocks of 128 tokens. The
+ * block products run on the tensor cores in bf16 with fp32 accumulation; the
+ * state passed between blocks stays in fp32 on chip. The caller owns the
+ * workspace (MS_SSD_WORKSPACE_BYTES, 16-byte aligned). After synchronizing,
+ * its first int32 is 0 when the kernel finished normally, MS_ERR_TIMEOUT when
+ * one of the kernel's internal pipeline waits gave up after about a second
+ * (the outputs are then incomplete), or MS_ERR_ALIGNMENT when the kernel's
+ * shared memory window was not 1024-byte aligned (nothing was computed).
+ * The tensor maps the kernel reads through are encoded on the host by the
+ * driver's encoder, looked up once per process. Errors: MS_ERR_INVALID_ARG
+ * for NULL or negative sizes, strides or pointers, or nheads not a multiple
+ * of ngroups; MS_ERR_UNSUPPORTED for a dtype other than bf16 or a driver
+ * without tensor-map support; MS_ERR_ALIGNMENT for misaligned pointers or
+ * strides; MS_ERR_WORKSPACE for a missing or short workspace; MS_ERR_CUDA for
+ * a failed launch.
+ */
+ms_status mamba_ssd_fwd(const ms_ssd_args *args, void *workspace, size_t workspace_bytes, void *stream);
 
 /* Size of the device array behind mamba_scan_fwd_noalloc (8 MiB per GPU). */
 #define MS_NOALLOC_SCRATCH_BYTES (8u << 20)

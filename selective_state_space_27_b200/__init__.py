@@ -25,7 +25,7 @@ __all__ = [
     "scan_fwd", "state_update", "scan_workspace_size", "scan_plan", "scan_configs", "library_path",
     "load_library", "MambaScanError", "ScanArgs", "UpdateArgs", "ScanPlan", "MS_F32", "MS_BF16",
     "Conv1dArgs", "conv_scan_fwd", "conv_state_update", "build_conv_args", "trap_scan_fwd",
-    "ScanBwdArgs", "scan_bwd",
+    "ScanBwdArgs", "scan_bwd", "SsdArgs", "build_ssd_args", "ssd_fwd", "ssd_check", "SSD_WORKSPACE_BYTES",
     "MAX_DSTATE",
 ]
 
@@ -35,6 +35,7 @@ _lib = None
 
 MS_F32, MS_BF16 = 0, 1
 MAX_DSTATE = 16
+SSD_HEADDIM, SSD_DSTATE, SSD_WORKSPACE_BYTES = 64, 128, 256
 STATUS = {0: "MS_OK", 1: "MS_ERR_INVALID_ARG", 2: "MS_ERR_UNSUPPORTED", 3: "MS_ERR_ALIGNMENT",
           4: "MS_ERR_CUDA", 5: "MS_ERR_TIMEOUT", 6: "MS_ERR_WORKSPACE"}
 
@@ -89,6 +90,21 @@ class ScanBwdArgs(ctypes.Structure):
         ("ddelta", _vp), ("ddelta_batch_stride", _i64), ("ddelta_dim_stride", _i64),
         ("dz", _vp), ("dz_batch_stride", _i64), ("dz_dim_stride", _i64),
         ("dA", _vp), ("dB", _vp), ("dC", _vp), ("dD", _vp), ("ddelta_bias", _vp), ("dinitial_state", _vp),
+    ]
+
+
+class SsdArgs(ctypes.Structure):
+    """Mirror of ``ms_ssd_args``."""
+    _fields_ = [
+        ("batch", _i64), ("seqlen", _i64), ("nheads", _i64), ("ngroups", _i64),
+        ("in_dtype", _i32), ("dt_softplus", _i32),
+        ("x", _vp), ("x_batch_stride", _i64), ("x_token_stride", _i64),
+        ("dt", _vp), ("dt_batch_stride", _i64), ("dt_token_stride", _i64),
+        ("B", _vp), ("B_batch_stride", _i64), ("B_token_stride", _i64),
+        ("C", _vp), ("C_batch_stride", _i64), ("C_token_stride", _i64),
+        ("z", _vp), ("z_batch_stride", _i64), ("z_token_stride", _i64),
+        ("y", _vp), ("y_batch_stride", _i64), ("y_token_stride", _i64),
+        ("A", _vp), ("D", _vp), ("dt_bias", _vp), ("initial_state", _vp), ("final_state", _vp),
     ]
 
 
@@ -156,6 +172,8 @@ def load_library():
         lib.mamba_scan_fwd_with_plan.restype = ctypes.c_int
         lib.mamba_scan_fwd_with_plan.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(ScanPlan), _vp,
                                                  ctypes.c_size_t, _vp]
+        lib.mamba_ssd_fwd.restype = ctypes.c_int
+        lib.mamba_ssd_fwd.argtypes = [ctypes.POINTER(SsdArgs), _vp, ctypes.c_size_t, _vp]
         if lib.mamba_abi_version() != 1:
             raise RuntimeError("libmambascan.so ABI version mismatch")
         _lib = lib
@@ -504,3 +522,88 @@ def scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, delta_softp
         _check(lib.mamba_scan_bwd(ctypes.byref(args), ctypes.byref(g), workspace.data_ptr(), workspace.numel(),
                                   _stream_ptr(stream)))
     return out
+
+
+def build_ssd_args(x, dt, A, B, C, y, *, D=None, z=None, dt_bias=None, dt_softplus=True, initial_state=None,
+                   final_state=None) -> SsdArgs:
+    """Fill an ``ms_ssd_args`` from torch tensors: x, z, y (batch, L, nheads,
+    64), dt (batch, L, nheads), B, C (batch, L, ngroups, 128), all bf16 with
+    the inner axes contiguous; A, D, dt_bias (nheads,) float32; states
+    (batch, nheads, 64, 128) float32 contiguous."""
+    torch = _torch()
+    for name, t in (("x", x), ("y", y), ("z", z)):
+        _need_cuda(name, t, None, 4)
+        if t is not None and (t.shape[3] != SSD_HEADDIM or (t.shape[2] > 1 and t.stride(2) != SSD_HEADDIM)):
+            raise ValueError(f"{name} must be (batch, L, nheads, 64) with the last two axes contiguous")
+    batch, L, nheads, _ = x.shape
+    for name, t in (("y", y), ("z", z)):
+        if t is not None and tuple(t.shape) != tuple(x.shape):
+            raise ValueError(f"{name} must have x's shape")
+    _need_cuda("dt", dt, None, 3)
+    if tuple(dt.shape) != (batch, L, nheads):
+        raise ValueError("dt must be (batch, L, nheads)")
+    for name, t in (("B", B), ("C", C)):
+        _need_cuda(name, t, None, 4)
+        if (t.shape[0] != batch or t.shape[1] != L or t.shape[3] != SSD_DSTATE
+                or (t.shape[2] > 1 and t.stride(2) != SSD_DSTATE)):
+            raise ValueError(f"{name} must be (batch, L, ngroups, 128) with the last two axes contiguous")
+    if tuple(C.shape) != tuple(B.shape):
+        raise ValueError("B and C must have one shape")
+    for name, t in (("A", A), ("D", D), ("dt_bias", dt_bias)):
+        _need_cuda(name, t, torch.float32, 1)
+        if t is not None and (tuple(t.shape) != (nheads,) or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous ({nheads},) float32 tensor")
+    for name, t in (("initial_state", initial_state), ("final_state", final_state)):
+        _need_cuda(name, t, torch.float32, 4)
+        if t is not None and (tuple(t.shape) != (batch, nheads, SSD_HEADDIM, SSD_DSTATE) or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous (batch, nheads, 64, 128) float32 tensor")
+    a = SsdArgs()
+    a.batch, a.seqlen, a.nheads, a.ngroups = batch, L, nheads, B.shape[2]
+    a.in_dtype = _dtype_code(x)
+    a.dt_softplus = 1 if dt_softplus else 0
+    for name, t in (("x", x), ("dt", dt), ("B", B), ("C", C), ("z", z), ("y", y)):
+        if t is not None:
+            setattr(a, name, _ptr(t))
+            setattr(a, f"{name}_batch_stride", t.stride(0))
+            setattr(a, f"{name}_token_stride", t.stride(1))
+    a.A, a.D, a.dt_bias = _ptr(A), _ptr(D), _ptr(dt_bias)
+    a.initial_state, a.final_state = _ptr(initial_state), _ptr(final_state)
+    return a
+
+
+def ssd_check(workspace, stream=None):
+    """Synchronize ``stream`` and raise :class:`MambaScanError` if the SSD
+    kernel that used ``workspace`` reported a failed internal wait."""
+    torch = _torch()
+    (stream or torch.cuda.current_stream(workspace.device)).synchronize()
+    code = int(workspace[:4].view(torch.int32)[0].item())
+    if code != 0:
+        raise MambaScanError(code, "the SSD kernel reported a failure in its status word")
+
+
+def ssd_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True, initial_state=None,
+            return_final_state=True, out=None, workspace=None, check=True, stream=None):
+    """Mamba-2 scalar-decay SSM forward (chunked SSD on the tensor cores).
+
+    Shapes as :func:`build_ssd_args`. Returns ``(y, final_state)``
+    (final_state None when not asked for). ``workspace``: a uint8 CUDA tensor
+    of at least ``SSD_WORKSPACE_BYTES`` bytes holding the status word (one is
+    allocated when None). With ``check`` the call synchronizes the stream and
+    raises if the kernel reported a failed wait; without it, call
+    :func:`ssd_check` on the workspace later.
+    """
+    torch = _torch()
+    y = torch.empty_like(x) if out is None else out
+    hT = None
+    if return_final_state:
+        hT = torch.empty((x.shape[0], x.shape[2], SSD_HEADDIM, SSD_DSTATE), device=x.device, dtype=torch.float32)
+    args = build_ssd_args(x, dt, A, B, C, y, D=D, z=z, dt_bias=dt_bias, dt_softplus=dt_softplus,
+                          initial_state=initial_state, final_state=hT)
+    if workspace is None:
+        workspace = torch.empty(SSD_WORKSPACE_BYTES, dtype=torch.uint8, device=x.device)
+    with torch.cuda.device(x.device):
+        _check(load_library().mamba_ssd_fwd(ctypes.byref(args), workspace.data_ptr(), workspace.numel(),
+                                             _stream_ptr(stream)))
+    if check:
+        ssd_check(workspace, stream)
+    return y, hT

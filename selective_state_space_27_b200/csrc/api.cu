@@ -470,4 +470,78 @@ ms_status mamba_scan_bwd(const ms_scan_args *args, const ms_scan_bwd_args *g, vo
     return MS_OK;
 }
 
+ms_status mamba_ssd_fwd(const ms_ssd_args *a, void *workspace, size_t workspace_bytes, void *stream) {
+    if (!a) return invalid("args is NULL");
+    if (a->batch <= 0 || a->seqlen <= 0 || a->nheads <= 0 || a->ngroups <= 0)
+        return invalid("batch, seqlen, nheads and ngroups must be positive");
+    if (a->nheads % a->ngroups != 0) return invalid("nheads must be a multiple of ngroups");
+    if (!a->x || !a->dt || !a->B || !a->C || !a->y || !a->A) return invalid("x, dt, B, C, y and A are required");
+    if (a->in_dtype != MS_BF16) {
+        if (a->in_dtype != MS_F32) return invalid("unknown in_dtype");
+        set_error("the SSD kernel takes bf16 inputs only");
+        return MS_ERR_UNSUPPORTED;
+    }
+    if (a->seqlen > (int64_t(1) << 30) || a->batch * a->nheads > (int64_t(1) << 30))
+        return invalid("seqlen or batch * nheads too large");
+    const int64_t strides[] = {a->x_batch_stride, a->x_token_stride, a->dt_batch_stride, a->dt_token_stride,
+                               a->B_batch_stride, a->B_token_stride, a->C_batch_stride, a->C_token_stride,
+                               a->y_batch_stride, a->y_token_stride, a->z_batch_stride, a->z_token_stride};
+    for (int i = 0; i < (a->z ? 12 : 10); ++i)
+        if (strides[i] < 0) return invalid("strides must be non-negative");
+    if (a->x_token_stride < a->nheads * MS_SSD_HEADDIM || a->y_token_stride < a->nheads * MS_SSD_HEADDIM ||
+        (a->z && a->z_token_stride < a->nheads * MS_SSD_HEADDIM))
+        return invalid("the token stride of x, y and z must cover nheads * 64 elements");
+    if (a->B_token_stride < a->ngroups * MS_SSD_DSTATE || a->C_token_stride < a->ngroups * MS_SSD_DSTATE)
+        return invalid("the token stride of B and C must cover ngroups * 128 elements");
+    if (a->dt_token_stride < a->nheads) return invalid("the token stride of dt must cover nheads elements");
+    for (int i : {0, 1, 4, 5, 6, 7, 8, 9}) {
+        if (strides[i] % 8 != 0) {
+            set_error("batch and token strides of x, y, B, C (and z) must be multiples of 8 elements");
+            return MS_ERR_ALIGNMENT;
+        }
+    }
+    if (a->z && (a->z_batch_stride % 8 != 0 || a->z_token_stride % 8 != 0)) {
+        set_error("batch and token strides of x, y, B, C (and z) must be multiples of 8 elements");
+        return MS_ERR_ALIGNMENT;
+    }
+    if (!elem_aligned(a->x, 16) || !elem_aligned(a->B, 16) || !elem_aligned(a->C, 16) || !elem_aligned(a->y, 16) ||
+        (a->z && !elem_aligned(a->z, 16)) || !elem_aligned(a->dt, 2) || !elem_aligned(a->A, 4) ||
+        (a->D && !elem_aligned(a->D, 4)) || (a->dt_bias && !elem_aligned(a->dt_bias, 4)) ||
+        (a->initial_state && !elem_aligned(a->initial_state, 4)) ||
+        (a->final_state && !elem_aligned(a->final_state, 4))) {
+        set_error("x, y, B, C and z must be 16-byte aligned, the other pointers aligned to their elements");
+        return MS_ERR_ALIGNMENT;
+    }
+    if (!workspace || workspace_bytes < MS_SSD_WORKSPACE_BYTES) {
+        set_error("workspace of %d bytes needed, %zu given", MS_SSD_WORKSPACE_BYTES,
+                  workspace ? workspace_bytes : static_cast<size_t>(0));
+        return MS_ERR_WORKSPACE;
+    }
+    if (!elem_aligned(workspace, 16)) {
+        set_error("workspace must be 16-byte aligned");
+        return MS_ERR_ALIGNMENT;
+    }
+    ms::SsdParams p{};
+    p.x = a->x; p.x_sb = a->x_batch_stride; p.x_st = a->x_token_stride;
+    p.dt = a->dt; p.dt_sb = a->dt_batch_stride; p.dt_st = a->dt_token_stride;
+    p.B = a->B; p.B_sb = a->B_batch_stride; p.B_st = a->B_token_stride;
+    p.C = a->C; p.C_sb = a->C_batch_stride; p.C_st = a->C_token_stride;
+    p.z = a->z; p.z_sb = a->z_batch_stride; p.z_st = a->z_token_stride;
+    p.y = a->y; p.y_sb = a->y_batch_stride; p.y_st = a->y_token_stride;
+    p.A = a->A; p.D = a->D; p.dt_bias = a->dt_bias; p.h0 = a->initial_state; p.hT = a->final_state;
+    p.batch = a->batch; p.seqlen = a->seqlen; p.nheads = a->nheads; p.ngroups = a->ngroups;
+    p.softplus = a->dt_softplus ? 1 : 0;
+    p.status = static_cast<int *>(workspace);
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int), s);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the SSD status word");
+    e = ms::launch_ssd(p, s);
+    if (e == cudaErrorNotSupported) {
+        set_error("the driver offers no tensor-map encoder");
+        return MS_ERR_UNSUPPORTED;
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "SSD kernel launch");
+    return MS_OK;
+}
+
 }  // extern "C"

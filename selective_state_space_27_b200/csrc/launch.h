@@ -112,6 +112,33 @@ struct UpdateParams {
 
 cudaError_t launch_state_update(const UpdateParams &p, int in_dtype, cudaStream_t stream);
 
+// Mamba-2 scalar-decay SSM (SSD) forward, bf16 inputs, headdim 64, dstate 128.
+// x and z, y: (batch, seqlen, nheads, 64), the last two axes contiguous, batch
+// and token element strides *_sb, *_st. dt: (batch, seqlen, nheads), head
+// axis contiguous. B, C: (batch, seqlen, ngroups, 128), the last two axes
+// contiguous. h0 / hT: (batch, nheads, 64, 128) float32 contiguous or null.
+// status: a device int that receives MS_ERR_TIMEOUT if a pipeline wait of
+// the kernel gave up (it is not cleared by the launch).
+struct SsdParams {
+    const void *x;     int64_t x_sb, x_st;
+    const void *dt;    int64_t dt_sb, dt_st;
+    const void *B;     int64_t B_sb, B_st;
+    const void *C;     int64_t C_sb, C_st;
+    const void *z;     int64_t z_sb, z_st;
+    void *y;           int64_t y_sb, y_st;
+    const float *A, *D, *dt_bias, *h0;
+    float *hT;
+    int64_t batch, seqlen, nheads, ngroups;
+    int softplus;
+    int *status;
+};
+constexpr int kSsdHeadDim = 64;
+constexpr int kSsdState = 128;
+constexpr int kSsdChunk = 128;
+// Encodes the kernel's tensor maps and launches it. Returns cudaErrorNotSupported
+// when the driver offers no tensor-map encoder.
+cudaError_t launch_ssd(const SsdParams &p, cudaStream_t stream);
+
 // Record the message that mamba_last_error() returns on this thread.
 void record_error(const char *fmt, ...);
 

@@ -1,0 +1,685 @@
+// ssd_fwd.cu -- Mamba-2 scalar-decay SSM forward (the structured state space
+// duality, SSD) in chunks of 128 tokens on the sm_100a tensor cores.
+//
+// What it computes, per batch b and head h (the recurrent definition):
+//   delta_t = softplus(dt[b,t,h] + dt_bias[h]),  a_t = exp(delta_t A[h])
+//   H_t = a_t H_{t-1} + (delta_t x_t) B_t^T   (H: headdim x dstate = 64 x 128)
+//   y_t = H_t C_t + D[h] x_t,  y_t *= silu(z_t)
+// ("Notas sobre Mamba", sections "A forma dual: atenção mascarada" and "O
+// algoritmo SSD"; "Mamba-2 e State Space Duality (SSD)", section "O algoritmo
+// de decomposição em blocos do SSD").
+//
+// How: the pages' chunked algorithm. Within a chunk of Q = 128 tokens, with
+// s_t the running sum of delta A inside the chunk (s_end its last value):
+//   G     = C B^T                                   (Q x Q, contraction over N)
+//   M'_ji = [i <= j] exp(s_j - s_i) delta_i G_ji     (decay mask and step)
+//   Yd    = M' X                                    (diagonal block)
+//   Yo    = C H_prev^T,  y_j = Yd_j + exp(s_j) Yo_j + D x_j   (off-diagonal)
+//   Xt_i  = exp(s_end - s_i) delta_i X_i,  S = B^T Xt  (chunk state)
+//   H     = exp(s_end) H_prev + S^T                 (state passing)
+// The four products are tcgen05 MMAs (bf16 operands from shared memory,
+// fp32 accumulators in tensor memory); the decay, the state passing, the
+// skip and the gate run in the epilogue warps. One CTA owns one (b, h) and
+// walks its chunks in order, so the state never leaves the SM.
+//
+// Roles (320 threads): warps 0-7 epilogue (warp w reads TMEM lanes
+// 32 (w % 4) .. +31, i.e. rows of the chunk, and handles column half w / 4);
+// warp 8 issues the TMA loads; warp 9 owns the tensor memory and issues the
+// MMAs. Every wait on an mbarrier gives up after about a second, records
+// MS_ERR_TIMEOUT in the status word and lets the CTA drain and exit.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "launch.h"
+#include "mambascan.h"
+
+namespace {
+
+constexpr int kQ = 128;          // tokens per chunk
+constexpr int kP = 64;           // headdim
+constexpr int kN = 128;          // dstate
+constexpr int kStages = 2;       // input stages (X, B, C of one chunk each)
+constexpr int kEpiWarps = 8;
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kThreads = kEpiThreads + 64;
+constexpr int kTmaWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1;
+
+// Shared memory, from a 1024-byte aligned base. Every operand tile is made of
+// 128-byte-swizzled atoms (rows of 128 bytes, 8-row groups of 1024 bytes).
+constexpr uint32_t kXTile = kQ * 128;                    // 128 tokens x 64 bf16
+constexpr uint32_t kBCTile = 2 * kQ * 128;               // 128 tokens x 128 bf16, two 64-wide atoms
+constexpr uint32_t kStageBytes = kXTile + 2 * kBCTile;   // X, B, C
+constexpr uint32_t kOffM = kStages * kStageBytes;        // M' (128 x 128 bf16, two atoms along i)
+constexpr uint32_t kOffXt = kOffM + 2 * kQ * 128;        // Xt (128 tokens x 64 bf16)
+constexpr uint32_t kOffH = kOffXt + kXTile;              // H (64 rows p x 128 bf16, two atoms along n)
+constexpr uint32_t kHAtom = kP * 128;
+constexpr uint32_t kOffStep = kOffH + 2 * kHAtom;        // float delta[2][Q], s2[2][Q]; float wsum[4]; int abort
+constexpr uint32_t kOffAbort = kOffStep + 4 * kQ * 4 + 16;
+constexpr uint32_t kOffBar = kOffStep + 4 * kQ * 4 + 32;
+enum Bar { kFull0, kFull1, kEmpty0, kEmpty1, kGFull0, kGFull1, kPReady, kSFull, kYFull, kHReady, kYFree, kDrain,
+           kNumBars };
+constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
+constexpr uint32_t kSmemBytes = kOffTmemSlot + 8;
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+static_assert(kOffM % 1024 == 0 && kOffXt % 1024 == 0 && kOffH % 1024 == 0 && kStageBytes % 1024 == 0,
+              "swizzle atoms need 1024-byte alignment");
+
+// Tensor memory: 512 columns x 128 lanes of fp32.
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColG = 0;      // two buffers of 128 columns
+constexpr uint32_t kColYd = 256;   // 64 columns
+constexpr uint32_t kColYo = 320;   // 64 columns
+constexpr uint32_t kColS = 384;    // 64 columns
+
+constexpr uint32_t kStageTx = kStageBytes;   // bytes the TMA delivers per stage
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ---- small PTX wrappers ----------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Wait for the phase of the given parity to complete; false after about a
+// second (the caller then records a timeout and stops).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity)
+{
+    if (mbar_test(bar, parity))
+        return true;
+    const uint64_t t0 = global_ns();
+    while (!mbar_test(bar, parity))
+        if (global_ns() - t0 > kWaitLimitNs)
+            return false;
+    return true;
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int c0, int c1,
+                                            int c2)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
+        "[%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void async_proxy_fence() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory"); }
+__device__ __forceinline__ void wg0_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+
+// Shared-memory matrix descriptor of a 128-byte-swizzled operand: start
+// address, leading and stride byte offsets (16-byte units), version 1,
+// layout type 2 (128-byte swizzle).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr, uint32_t lbo, uint32_t sbo)
+{
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor of a kind::f16 MMA with bf16 A and B, fp32 D.
+// a_mn / b_mn select the MN-major (instead of K-major) operand layout.
+__host__ __device__ constexpr uint32_t bf16_idesc(int M, int N, bool a_mn, bool b_mn)
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+// 32 consecutive fp32 columns of this warp's 32 lanes; thread i gets lane i.
+// The wait is part of the same statement so no use can move above it.
+__device__ __forceinline__ void tmem_load32(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+        v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ float ex2(float v)
+{
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Byte offset of 16-byte chunk q of row r inside a 128-byte-swizzled atom.
+__device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t q) { return r * 128u + ((q ^ (r & 7u)) << 4); }
+
+// A bounded wait that also gives up at once when another role of the CTA has
+// already given up (abort flag in shared memory).
+__device__ __forceinline__ bool role_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag)
+{
+    if (mbar_test(bar, parity))
+        return true;
+    const uint64_t t0 = global_ns();
+    while (!mbar_test(bar, parity)) {
+        if (*abort_flag || global_ns() - t0 > kWaitLimitNs)
+            return false;
+    }
+    return true;
+}
+
+__device__ __forceinline__ void give_up(int *status, volatile int *abort_flag)
+{
+    *abort_flag = 1;
+    atomicExch(status, (int)MS_ERR_TIMEOUT);
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t cols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot), "r"(cols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_free(uint32_t taddr, uint32_t cols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols) : "memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v)
+{
+    asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+}
+
+__device__ __forceinline__ float load_bf16(const void *p, int64_t i)
+{
+    return __uint_as_float((uint32_t)reinterpret_cast<const uint16_t *>(p)[i] << 16);
+}
+
+// The running state H[p][n] of this thread (n = its row r, p = 32 hf + j) as
+// bf16 into the K-major operand tile of the Yo product (rows p, K = n).
+__device__ __forceinline__ void store_state_tile(uint32_t tile, int r, int hf, const float (&H)[32])
+{
+    const uint32_t col = tile + (uint32_t)(r >> 6) * kHAtom + (uint32_t)(r & 7) * 2u;
+    const uint32_t q = (uint32_t)(r & 63) >> 3;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        const __nv_bfloat16 v = __float2bfloat16_rn(H[j]);
+        st_shared_u16(col + sw128((uint32_t)(32 * hf + j), q), *reinterpret_cast<const uint16_t *>(&v));
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap b_map,
+           const __grid_constant__ CUtensorMap c_map, const ms::SsdParams p)
+{
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t bh = blockIdx.x;
+    const int64_t b = bh / p.nheads, h = bh % p.nheads;
+    const int64_t g = h / (p.nheads / p.ngroups);
+    const int L = (int)p.seqlen;
+    const int nchunks = (L + kQ - 1) / kQ;
+    const uint32_t base = smem_addr(smem);
+    if (base & 1023u) {   // the swizzled tiles need a 1024-byte aligned window
+        if (threadIdx.x == 0)
+            atomicExch(p.status, (int)MS_ERR_ALIGNMENT);
+        return;
+    }
+    auto bar = [&](int i) { return base + kOffBar + 8u * (uint32_t)i; };
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffAbort);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(kFull0), 1);
+        mbar_init(bar(kFull1), 1);
+        mbar_init(bar(kEmpty0), kEpiWarps);
+        mbar_init(bar(kEmpty1), kEpiWarps);
+        mbar_init(bar(kGFull0), 1);
+        mbar_init(bar(kGFull1), 1);
+        mbar_init(bar(kPReady), kEpiWarps);
+        mbar_init(bar(kSFull), 1);
+        mbar_init(bar(kYFull), 1);
+        mbar_init(bar(kHReady), kEpiWarps);
+        mbar_init(bar(kYFree), kEpiWarps);
+        mbar_init(bar(kDrain), 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == kMmaWarp)
+        tmem_alloc(base + kOffTmemSlot, kTmemCols);
+    tc_before_sync();
+    __syncthreads();
+    tc_after_sync();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + kOffTmemSlot);
+
+    if (warp == kTmaWarp) {
+        // ---- producer: X, B and C of chunk c into stage c % 2 ----
+        if (lane == 0) {
+            int issued = 0;
+            for (int c = 0; c < nchunks; ++c) {
+                const int st = c & 1;
+                if (c >= 2 && !role_wait(bar(kEmpty0 + st), ((c >> 1) + 1) & 1, abort_flag)) {
+                    give_up(p.status, abort_flag);
+                    break;
+                }
+                const uint32_t sx = base + (uint32_t)st * kStageBytes, sb = sx + kXTile, sc = sb + kBCTile;
+                const uint32_t full = bar(kFull0 + st);
+                mbar_arrive_tx(full, kStageTx);
+                tma_load_3d(sx, &x_map, full, (int)(h * kP), c * kQ, (int)b);
+                tma_load_3d(sb, &b_map, full, (int)(g * kN), c * kQ, (int)b);
+                tma_load_3d(sb + kQ * 128, &b_map, full, (int)(g * kN + 64), c * kQ, (int)b);
+                tma_load_3d(sc, &c_map, full, (int)(g * kN), c * kQ, (int)b);
+                tma_load_3d(sc + kQ * 128, &c_map, full, (int)(g * kN + 64), c * kQ, (int)b);
+                issued = c + 1;
+            }
+            // the loads in flight must land before the CTA leaves
+            for (int c = issued > 2 ? issued - 2 : 0; c < issued; ++c)
+                mbar_wait(bar(kFull0 + (c & 1)), (c >> 1) & 1);
+        }
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        // ---- MMA issue (one thread) ----
+        if (lane == 0) {
+            constexpr uint32_t id_g = bf16_idesc(128, 128, false, false);   // G = C B^T
+            constexpr uint32_t id_yo = bf16_idesc(128, 64, false, false);   // Yo = C H^T
+            constexpr uint32_t id_s = bf16_idesc(128, 64, true, true);      // S = B^T Xt
+            constexpr uint32_t id_yd = bf16_idesc(128, 64, false, true);    // Yd = M' X
+            for (int c = 0; c < nchunks; ++c) {
+                const int st = c & 1;
+                const uint32_t sx = base + (uint32_t)st * kStageBytes, sb = sx + kXTile, sc = sb + kBCTile;
+                if (!role_wait(bar(kFull0 + st), (c >> 1) & 1, abort_flag)) {
+                    give_up(p.status, abort_flag);
+                    break;
+                }
+                tc_after_sync();
+                const uint32_t tg = tmem + kColG + 128u * (uint32_t)(c & 1);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t off = (uint32_t)(k >> 2) * (kQ * 128) + (uint32_t)(k & 3) * 32u;
+                    mma_bf16(tg, sw128_desc(sc + off, 16, 1024), sw128_desc(sb + off, 16, 1024), id_g, k > 0);
+                }
+                mma_commit(bar(kGFull0 + (c & 1)));
+                // Yo needs the state of the previous chunk and the Y columns free
+                if (!role_wait(bar(kHReady), c & 1, abort_flag) ||
+                    (c > 0 && !role_wait(bar(kYFree), (c - 1) & 1, abort_flag))) {
+                    give_up(p.status, abort_flag);
+                    break;
+                }
+                tc_after_sync();
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t offc = (uint32_t)(k >> 2) * (kQ * 128) + (uint32_t)(k & 3) * 32u;
+                    const uint32_t offh = (uint32_t)(k >> 2) * kHAtom + (uint32_t)(k & 3) * 32u;
+                    mma_bf16(tmem + kColYo, sw128_desc(sc + offc, 16, 1024),
+                             sw128_desc(base + kOffH + offh, 16, 1024), id_yo, k > 0);
+                }
+                // S and Yd need M' and Xt of this chunk
+                if (!role_wait(bar(kPReady), c & 1, abort_flag)) {
+                    give_up(p.status, abort_flag);
+                    break;
+                }
+                tc_after_sync();
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_bf16(tmem + kColS, sw128_desc(sb + (uint32_t)k * 2048u, kQ * 128, 1024),
+                             sw128_desc(base + kOffXt + (uint32_t)k * 2048u, kXTile, 1024), id_s, k > 0);
+                mma_commit(bar(kSFull));
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t offm = (uint32_t)(k >> 2) * (kQ * 128) + (uint32_t)(k & 3) * 32u;
+                    mma_bf16(tmem + kColYd, sw128_desc(base + kOffM + offm, 16, 1024),
+                             sw128_desc(sx + (uint32_t)k * 2048u, kXTile, 1024), id_yd, k > 0);
+                }
+                mma_commit(bar(kYFull));
+            }
+            // every MMA issued must finish before the tensor memory is freed
+            mma_commit(bar(kDrain));
+            mbar_wait(bar(kDrain), 0);
+        }
+        __syncwarp();
+    } else {
+        // ---- epilogue: warps 0-7; thread = row r of the chunk, column half hf ----
+        const int sub = warp & 3, hf = warp >> 2;
+        const int r = sub * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(sub * 32) << 16;
+        float *stepf = reinterpret_cast<float *>(smem + kOffStep);
+        float *wsum = stepf + 4 * kQ;
+        const float Ah2 = p.A[h] * kLog2e;
+        const float bias = p.dt_bias ? p.dt_bias[h] : 0.f;
+        const float Dh = p.D ? p.D[h] : 0.f;
+        // this thread keeps H[p][n] for n = r and p = 32 hf + j
+        const int64_t hoff = (bh * kP + 32 * hf) * kN + r;
+        float H[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            H[j] = p.h0 ? p.h0[hoff + (int64_t)j * kN] : 0.f;
+        // rows 0-63 of M' never reach columns 64-127 (causal mask): zero them once
+        if (hf == 1 && sub < 2)
+            for (int q = 0; q < 8; ++q)
+                st_shared_v4(base + kOffM + kQ * 128 + sw128((uint32_t)r, (uint32_t)q), 0u, 0u, 0u, 0u);
+        store_state_tile(base + kOffH, r, hf, H);
+        async_proxy_fence();
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(bar(kHReady));
+
+        bool ok = true;
+        auto epi_wait = [&](uint32_t barrier, uint32_t parity) {
+            if (ok)
+                ok = __all_sync(0xffffffffu, role_wait(barrier, parity, abort_flag));
+            if (!ok && lane == 0)
+                give_up(p.status, abort_flag);
+            return ok;
+        };
+        const uint16_t *dtp = reinterpret_cast<const uint16_t *>(p.dt) + b * p.dt_sb + h;
+        float dt_next = (hf == 0 && r < L) ? load_bf16(dtp, (int64_t)r * p.dt_st) : 0.f;
+        for (int c = 0; c < nchunks; ++c) {
+            const int st = c & 1, t0 = c * kQ;
+            const bool live = t0 + r < L;
+            const uint32_t sx = base + (uint32_t)st * kStageBytes;
+            float *dl = stepf + (c & 1) * kQ;
+            float *s2 = stepf + 2 * kQ + (c & 1) * kQ;
+            // the gate of this thread's 32 outputs, fetched early
+            uint4 zq[4] = {};
+            if (p.z && live) {
+                const uint4 *zp = reinterpret_cast<const uint4 *>(reinterpret_cast<const uint16_t *>(p.z) + b * p.z_sb +
+                                                                  (int64_t)(t0 + r) * p.z_st + h * kP + 32 * hf);
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    zq[q] = __ldg(zp + q);
+            }
+            // step sizes and the running sum of delta A (log2 units) in the chunk
+            if (hf == 0) {
+                float d = 0.f;
+                if (live) {
+                    d = dt_next + bias;
+                    if (p.softplus)
+                        d = d > 20.f ? d : log1pf(__expf(d));
+                }
+                dt_next = (t0 + kQ + r < L) ? load_bf16(dtp, (int64_t)(t0 + kQ + r) * p.dt_st) : 0.f;
+                float v = d * Ah2;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float u = __shfl_up_sync(0xffffffffu, v, o);
+                    if (lane >= o)
+                        v += u;
+                }
+                if (lane == 31)
+                    wsum[sub] = v;
+                wg0_sync();
+                for (int w = 0; w < sub; ++w)
+                    v += wsum[w];
+                dl[r] = d;
+                s2[r] = v;
+            }
+            epi_sync();
+
+            // (1) M' = mask o G and Xt, the operands of Yd and S
+            epi_wait(bar(kFull0 + st), (c >> 1) & 1);
+            epi_wait(bar(kGFull0 + (c & 1)), (c >> 1) & 1);
+            const float sr = s2[r];
+            if (ok) {
+                tc_after_sync();
+                if (!(hf == 1 && sub < 2)) {
+                    const uint32_t mt = base + kOffM + (uint32_t)hf * (kQ * 128);
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        float gv[32];
+                        tmem_load32(tmem + lane_base + kColG + 128u * (uint32_t)(c & 1) + 64u * hf + 32u * half, gv);
+                        const int i0 = 64 * hf + 32 * half;
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const float4 sa = *reinterpret_cast<const float4 *>(s2 + i0 + 8 * q4);
+                            const float4 sb4 = *reinterpret_cast<const float4 *>(s2 + i0 + 8 * q4 + 4);
+                            const float4 da = *reinterpret_cast<const float4 *>(dl + i0 + 8 * q4);
+                            const float4 db4 = *reinterpret_cast<const float4 *>(dl + i0 + 8 * q4 + 4);
+                            const float si[8] = {sa.x, sa.y, sa.z, sa.w, sb4.x, sb4.y, sb4.z, sb4.w};
+                            const float di[8] = {da.x, da.y, da.z, da.w, db4.x, db4.y, db4.z, db4.w};
+                            float m[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                const int i = i0 + 8 * q4 + e;
+                                m[e] = i <= r ? gv[8 * q4 + e] * ex2(sr - si[e]) * di[e] : 0.f;
+                            }
+                            st_shared_v4(mt + sw128((uint32_t)r, (uint32_t)(4 * half + q4)), pack_bf16(m[0], m[1]),
+                                         pack_bf16(m[2], m[3]), pack_bf16(m[4], m[5]), pack_bf16(m[6], m[7]));
+                        }
+                    }
+                }
+                const float wr = ex2(s2[kQ - 1] - sr) * dl[r];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t off = sw128((uint32_t)r, (uint32_t)(4 * hf + q));
+                    const uint4 v = ld_shared_v4(sx + off);
+                    st_shared_v4(base + kOffXt + off, pack_bf16(bf16_lo(v.x) * wr, bf16_hi(v.x) * wr),
+                                 pack_bf16(bf16_lo(v.y) * wr, bf16_hi(v.y) * wr),
+                                 pack_bf16(bf16_lo(v.z) * wr, bf16_hi(v.z) * wr),
+                                 pack_bf16(bf16_lo(v.w) * wr, bf16_hi(v.w) * wr));
+                }
+            }
+            async_proxy_fence();
+            tc_before_sync();
+            __syncwarp();
+            if (lane == 0 && ok)
+                mbar_arrive(bar(kPReady));
+
+            // (2) state passing: H = exp(s_end) H + S^T
+            epi_wait(bar(kSFull), c & 1);
+            if (ok) {
+                tc_after_sync();
+                float sv[32];
+                tmem_load32(tmem + lane_base + kColS + 32u * hf, sv);
+                const float ac = ex2(s2[kQ - 1]);
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    H[j] = fmaf(ac, H[j], sv[j]);
+                store_state_tile(base + kOffH, r, hf, H);
+            }
+            async_proxy_fence();
+            tc_before_sync();
+            __syncwarp();
+            if (lane == 0 && ok)
+                mbar_arrive(bar(kHReady));
+
+            // (3) y = Yd + exp(s_r) Yo + D x, gated
+            epi_wait(bar(kYFull), c & 1);
+            if (ok) {
+                tc_after_sync();
+                float yd[32], yo[32];
+                tmem_load32(tmem + lane_base + kColYd + 32u * hf, yd);
+                tmem_load32(tmem + lane_base + kColYo + 32u * hf, yo);
+                tc_before_sync();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(bar(kYFree));
+                if (live) {
+                    const float er = ex2(sr);
+                    uint4 out[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint4 xv = ld_shared_v4(sx + sw128((uint32_t)r, (uint32_t)(4 * hf + q)));
+                        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                        const uint32_t zw[4] = {zq[q].x, zq[q].y, zq[q].z, zq[q].w};
+                        uint32_t ow[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int j = 8 * q + 2 * e;
+                            float o0 = fmaf(er, yo[j], yd[j]) + Dh * bf16_lo(xw[e]);
+                            float o1 = fmaf(er, yo[j + 1], yd[j + 1]) + Dh * bf16_hi(xw[e]);
+                            if (p.z) {
+                                const float z0 = bf16_lo(zw[e]), z1 = bf16_hi(zw[e]);
+                                o0 *= z0 / (1.f + __expf(-z0));
+                                o1 *= z1 / (1.f + __expf(-z1));
+                            }
+                            ow[e] = pack_bf16(o0, o1);
+                        }
+                        out[q] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                    }
+                    uint4 *yp = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.y) + b * p.y_sb +
+                                                          (int64_t)(t0 + r) * p.y_st + h * kP + 32 * hf);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        yp[q] = out[q];
+                }
+            }
+            __syncwarp();
+            if (lane == 0 && ok)
+                mbar_arrive(bar(kEmpty0 + st));
+        }
+        if (ok && p.hT) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                p.hT[hoff + (int64_t)j * kN] = H[j];
+        }
+    }
+    tc_before_sync();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_after_sync();
+        tmem_free(tmem, kTmemCols);
+    }
+}
+
+}  // namespace
+
+namespace ms {
+namespace {
+
+using EncodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                 const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// The driver's tensor-map encoder, looked up once through the runtime.
+EncodeTiled encoder()
+{
+    static const EncodeTiled fn = [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return static_cast<EncodeTiled>(nullptr);
+        return reinterpret_cast<EncodeTiled>(ptr);
+    }();
+    return fn;
+}
+
+// A bf16 map over (inner, tokens, batch) delivering 64 x 128 x 1 boxes into
+// 128-byte-swizzled shared memory; rows past the last token read as zero.
+bool encode_map(CUtensorMap *m, const void *ptr, int64_t inner, int64_t tokens, int64_t batch, int64_t token_stride,
+                int64_t batch_stride)
+{
+    const EncodeTiled fn = encoder();
+    if (!fn)
+        return false;
+    if (batch == 1)
+        batch_stride = token_stride * tokens;
+    const cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)tokens, (cuuint64_t)batch};
+    const cuuint64_t strides[2] = {(cuuint64_t)token_stride * 2u, (cuuint64_t)batch_stride * 2u};
+    const cuuint32_t box[3] = {64u, (cuuint32_t)kQ, 1u};
+    const cuuint32_t elem[3] = {1u, 1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, elem,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_ssd(const SsdParams &p, cudaStream_t stream)
+{
+    CUtensorMap xm, bm, cm;
+    if (!encode_map(&xm, p.x, p.nheads * kP, p.seqlen, p.batch, p.x_st, p.x_sb) ||
+        !encode_map(&bm, p.B, p.ngroups * kN, p.seqlen, p.batch, p.B_st, p.B_sb) ||
+        !encode_map(&cm, p.C, p.ngroups * kN, p.seqlen, p.batch, p.C_st, p.C_sb))
+        return cudaErrorNotSupported;
+    cudaError_t e = cudaFuncSetAttribute(ssd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e != cudaSuccess)
+        return e;
+    ssd_kernel<<<(unsigned)(p.batch * p.nheads), kThreads, kSmemBytes, stream>>>(xm, bm, cm, p);
+    return cudaGetLastError();
+}
+
+}  // namespace ms

@@ -35,6 +35,10 @@ __all__ = [
     "make_decode_step",
     "bf16_bits_from_f32",
     "f32_from_bf16_bits",
+    "SsdWorkload",
+    "SSD_WORKLOADS",
+    "make_ssd_inputs",
+    "make_ssd_state",
 ]
 
 BASE_SEED = 20261202
@@ -42,7 +46,8 @@ BASE_SEED = 20261202
 # One draw stream per tensor, so that the value of a tensor does not depend on
 # which other tensors were drawn.
 _STREAM = {"u": 1, "delta": 2, "B": 3, "C": 4, "z": 5, "D": 6, "dt": 7, "h0": 8, "conv_w": 9, "conv_b": 10,
-           "conv_state": 11, "lambda_raw": 12}
+           "conv_state": 11, "lambda_raw": 12, "ssd_x": 13, "ssd_dt": 14, "ssd_B": 15, "ssd_C": 16, "ssd_z": 17,
+           "ssd_head": 18, "ssd_h0": 19}
 _CHUNK = 1 << 22
 
 
@@ -84,6 +89,36 @@ SCAN_WORKLOADS = {
 
 DECODE_WORKLOADS = {
     "decode_b256_d5120": DecodeWorkload("decode_b256_d5120", 256, 5120, 16, 1000, "bf16", True, BASE_SEED + 4),
+}
+
+
+@dataclasses.dataclass(frozen=True)
+class SsdWorkload:
+    """A Mamba-2 SSD layer: x (batch, L, nheads, headdim), B and C (batch, L,
+    ngroups, dstate)."""
+    name: str
+    batch: int
+    seqlen: int
+    nheads: int
+    ngroups: int
+    headdim: int
+    dstate: int
+    has_z: bool
+    seed: int
+
+    @property
+    def elements(self) -> int:
+        """State elements (b, t, h, p, n) updated by one pass."""
+        return self.batch * self.seqlen * self.nheads * self.headdim * self.dstate
+
+
+# The Mamba-2 layer of "Mamba-2 e State Space Duality (SSD)", section
+# "Implementando Mamba-2 em pipelines de inferência": batch 4, 8192 tokens,
+# d_model 2048 with expand 2 (d_inner 4096 = 64 heads of headdim 64), d_state
+# 128, bf16; one group of B and C. The small case has a ragged last block.
+SSD_WORKLOADS = {
+    "ssd_small": SsdWorkload("ssd_small", 2, 300, 4, 1, 64, 128, True, BASE_SEED + 10),
+    "mamba2_layer_d2048": SsdWorkload("mamba2_layer_d2048", 4, 8192, 64, 1, 64, 128, True, BASE_SEED + 11),
 }
 
 
@@ -264,3 +299,42 @@ def make_lambda_raw(batch: int, dim: int, seqlen: int, dtype: str, seed: int = B
     """Pre-activation of the trapezoidal rule's per-token gate, N(0, 1) in the
     storage dtype (float32, or bf16 bits), shape (batch, dim, seqlen)."""
     return _store(_normal((batch, dim, seqlen), seed, _STREAM["lambda_raw"]), dtype)
+
+
+def make_ssd_inputs(w: SsdWorkload, *, batch=None, seqlen=None, nheads=None, ngroups=None, has_z=None,
+                    seed=None) -> dict:
+    """Draw one Mamba-2 SSD workload on the host (bf16 bits for x, dt, B, C, z).
+
+    Recipe (Mamba-2 initialisation): per head A = -U[1, 16] (A_log = log of a
+    uniform draw in [1, 16]), D ~ U[0.5, 1.5], dt_bias = log(expm1(dt)) with dt
+    log-uniform in [1e-3, 1e-1]; per token dt_raw ~ N(0, 0.5^2); x, B, C, z ~
+    N(0, 1). Returns x, z (batch, L, nheads, headdim), dt (batch, L, nheads),
+    B, C (batch, L, ngroups, dstate) as uint16 bf16 bits, and float32 A, D,
+    dt_bias (nheads,), plus the shape fields.
+    """
+    bt = w.batch if batch is None else batch
+    L = w.seqlen if seqlen is None else seqlen
+    H = w.nheads if nheads is None else nheads
+    G = w.ngroups if ngroups is None else ngroups
+    hz = w.has_z if has_z is None else has_z
+    sd = w.seed if seed is None else seed
+    gh = default_rng(SeedSequence(sd, spawn_key=(_STREAM["ssd_head"],)))
+    A = (-gh.uniform(1.0, 16.0, size=H)).astype(np.float32)
+    D = gh.uniform(0.5, 1.5, size=H).astype(np.float32)
+    dt0 = np.exp(gh.uniform(np.log(1e-3), np.log(1e-1), size=H))
+    dt_bias = np.log(np.expm1(dt0)).astype(np.float32)
+    P, N = w.headdim, w.dstate
+    return {
+        "batch": bt, "seqlen": L, "nheads": H, "ngroups": G, "headdim": P, "dstate": N,
+        "x": bf16_bits_from_f32(_normal((bt, L, H, P), sd, _STREAM["ssd_x"])),
+        "dt": bf16_bits_from_f32(_normal((bt, L, H), sd, _STREAM["ssd_dt"], 0.5)),
+        "B": bf16_bits_from_f32(_normal((bt, L, G, N), sd, _STREAM["ssd_B"])),
+        "C": bf16_bits_from_f32(_normal((bt, L, G, N), sd, _STREAM["ssd_C"])),
+        "z": bf16_bits_from_f32(_normal((bt, L, H, P), sd, _STREAM["ssd_z"])) if hz else None,
+        "A": A, "D": D, "dt_bias": dt_bias,
+    }
+
+
+def make_ssd_state(batch: int, nheads: int, headdim: int = 64, dstate: int = 128, seed: int = BASE_SEED) -> np.ndarray:
+    """An initial SSD state (batch, nheads, headdim, dstate) float32 ~ N(0, 1)."""
+    return _normal((batch, nheads, headdim, dstate), seed, _STREAM["ssd_h0"])

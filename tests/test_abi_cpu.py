@@ -32,7 +32,7 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for want in ("mamba_scan_fwd", "mamba_state_update", "mamba_scan_workspace_size", "mamba_conv_scan_fwd",
-                 "mamba_conv_state_update",
+                 "mamba_conv_state_update", "mamba_ssd_fwd",
                  "mamba_status_string", "mamba_last_error", "mamba_abi_version"):
         assert want in names
 
@@ -238,3 +238,53 @@ def test_bwd_needs_workspace_and_matching_gradients(lib):
     assert n.value == 2 * 8 * 4 * 16 * 4
     a.D = (1 << 20) * 7                      # D given: dD required
     assert lib.mamba_scan_bwd(ctypes.byref(a), ctypes.byref(_valid_bwd()), (1 << 20) * 30, 1 << 30, None) == 1
+
+
+def test_ssd_struct_layout_matches_binding(tmp_path):
+    src = tmp_path / "ssd_layout.c"
+    src.write_text(
+        '#include <stdio.h>\n#include <stddef.h>\n#include "mambascan.h"\n'
+        "int main(void){printf(\"%zu %zu %zu %zu %zu\\n\", sizeof(ms_ssd_args), offsetof(ms_ssd_args, x),"
+        " offsetof(ms_ssd_args, z_token_stride), offsetof(ms_ssd_args, A), offsetof(ms_ssd_args, final_state));"
+        " return 0;}\n")
+    exe = tmp_path / "ssd_layout"
+    subprocess.check_call(["gcc", "-std=c11", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe)])
+    got = [int(v) for v in subprocess.check_output([str(exe)], text=True).split()]
+    want = [ctypes.sizeof(ms.SsdArgs), ms.SsdArgs.x.offset, ms.SsdArgs.z_token_stride.offset, ms.SsdArgs.A.offset,
+            ms.SsdArgs.final_state.offset]
+    assert got == want
+
+
+def _valid_ssd_args():
+    a = ms.SsdArgs()
+    base = 1 << 20
+    a.batch, a.seqlen, a.nheads, a.ngroups = 2, 300, 4, 1
+    a.in_dtype, a.dt_softplus = ms.MS_BF16, 1
+    a.x, a.x_batch_stride, a.x_token_stride = base * 1, 300 * 256, 256
+    a.dt, a.dt_batch_stride, a.dt_token_stride = base * 2, 1200, 4
+    a.B, a.B_batch_stride, a.B_token_stride = base * 3, 300 * 128, 128
+    a.C, a.C_batch_stride, a.C_token_stride = base * 4, 300 * 128, 128
+    a.y, a.y_batch_stride, a.y_token_stride = base * 5, 300 * 256, 256
+    a.A = base * 6
+    return a
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("x", None, 1), ("A", None, 1), ("seqlen", 0, 1), ("ngroups", 3, 1), ("x_token_stride", 200, 1),
+    ("B_token_stride", 64, 1), ("dt_token_stride", 2, 1), ("y_batch_stride", -8, 1),
+    ("in_dtype", 0, 2), ("in_dtype", 7, 1),
+    ("x_token_stride", 260, 3), ("B_batch_stride", 300 * 128 + 4, 3), ("x", (1 << 20) + 8, 3),
+    ("dt", (1 << 20) * 2 + 1, 3), ("A", (1 << 20) * 6 + 2, 3),
+])
+def test_ssd_validation_rejects(lib, field, value, status):
+    a = _valid_ssd_args()
+    setattr(a, field, value)
+    assert lib.mamba_ssd_fwd(ctypes.byref(a), (1 << 20) * 9, 256, None) == status
+
+
+def test_ssd_needs_args_and_workspace(lib):
+    assert lib.mamba_ssd_fwd(None, (1 << 20) * 9, 256, None) == 1
+    a = _valid_ssd_args()
+    assert lib.mamba_ssd_fwd(ctypes.byref(a), None, 0, None) == 6
+    assert lib.mamba_ssd_fwd(ctypes.byref(a), (1 << 20) * 9, 128, None) == 6
+    assert lib.mamba_ssd_fwd(ctypes.byref(a), (1 << 20) * 9 + 4, 256, None) == 3
