@@ -22,9 +22,10 @@
 // skip and the gate run in the epilogue warps. One CTA owns one (b, h) and
 // walks its chunks in order, so the state never leaves the SM.
 //
-// Roles (320 threads): warps 0-7 epilogue (warp w reads TMEM lanes
-// 32 (w % 4) .. +31, i.e. rows of the chunk, and handles column half w / 4);
-// warp 8 issues the TMA loads; warp 9 owns the tensor memory and issues the
+// Roles (576 threads): warps 0-15 epilogue (warp w reads TMEM lanes
+// 32 (w % 4) .. +31, i.e. rows of the chunk, and handles column quarter
+// w / 4); warp 16 issues the TMA loads and computes each chunk's step sizes
+// and decay sums ahead of time; warp 17 owns the tensor memory and issues the
 // MMAs. Every wait on an mbarrier gives up after about a second, records
 // MS_ERR_TIMEOUT in the status word and lets the CTA drain and exit.
 #include <cuda.h>
@@ -32,6 +33,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "device_math.cuh"
 #include "launch.h"
 #include "mambascan.h"
 
@@ -41,7 +43,7 @@ constexpr int kQ = 128;          // tokens per chunk
 constexpr int kP = 64;           // headdim
 constexpr int kN = 128;          // dstate
 constexpr int kStages = 2;       // input stages (X, B, C of one chunk each)
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 16;
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kThreads = kEpiThreads + 64;
 constexpr int kTmaWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1;
@@ -55,11 +57,12 @@ constexpr uint32_t kOffM = kStages * kStageBytes;        // M' (128 x 128 bf16, 
 constexpr uint32_t kOffXt = kOffM + 2 * kQ * 128;        // Xt (128 tokens x 64 bf16)
 constexpr uint32_t kOffH = kOffXt + kXTile;              // H (64 rows p x 128 bf16, two atoms along n)
 constexpr uint32_t kHAtom = kP * 128;
-constexpr uint32_t kOffStep = kOffH + 2 * kHAtom;        // float delta[2][Q], s2[2][Q]; float wsum[4]; int abort
-constexpr uint32_t kOffAbort = kOffStep + 4 * kQ * 4 + 16;
-constexpr uint32_t kOffBar = kOffStep + 4 * kQ * 4 + 32;
+// step data of two chunks: float delta[2][Q], float s2[2][Q], bf16 cf[2][Q]; then int abort
+constexpr uint32_t kOffStep = kOffH + 2 * kHAtom;
+constexpr uint32_t kOffAbort = kOffStep + 2 * kQ * 10;
+constexpr uint32_t kOffBar = kOffAbort + 16;
 enum Bar { kFull0, kFull1, kEmpty0, kEmpty1, kGFull0, kGFull1, kPReady, kSFull, kYFull, kHReady, kYFree, kDrain,
-           kNumBars };
+           kStep0, kStep1, kNumBars };
 constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kOffTmemSlot + 8;
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
@@ -146,8 +149,6 @@ __device__ __forceinline__ void tc_before_sync() { asm volatile("tcgen05.fence::
 __device__ __forceinline__ void tc_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void async_proxy_fence() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory"); }
-__device__ __forceinline__ void wg0_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
 
 // Shared-memory matrix descriptor of a 128-byte-swizzled operand: start
 // address, leading and stride byte offsets (16-byte units), version 1,
@@ -182,23 +183,21 @@ __device__ __forceinline__ void mma_commit(uint32_t bar)
                  : "memory");
 }
 
-// 32 consecutive fp32 columns of this warp's 32 lanes; thread i gets lane i.
+// 16 consecutive fp32 columns of this warp's 32 lanes; thread i gets lane i.
 // The wait is part of the same statement so no use can move above it.
-__device__ __forceinline__ void tmem_load32(uint32_t taddr, float (&v)[32])
+__device__ __forceinline__ void tmem_load16(uint32_t taddr, float (&v)[16])
 {
-    uint32_t r[32];
+    uint32_t r[16];
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];\n\t"
         "tcgen05.wait::ld.sync.aligned;"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr)
         : "memory");
 #pragma unroll
-    for (int i = 0; i < 32; ++i)
+    for (int i = 0; i < 16; ++i)
         v[i] = __uint_as_float(r[i]);
 }
 
@@ -207,6 +206,15 @@ __device__ __forceinline__ float ex2(float v)
     float r;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
     return r;
+}
+
+// silu(z) = z sigmoid(z) = z (1 + tanh(z / 2)) / 2, one MUFU operation.
+__device__ __forceinline__ float silu_fast(float z)
+{
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * z));
+    const float hz = 0.5f * z;
+    return fmaf(hz, t, hz);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
@@ -279,16 +287,16 @@ __device__ __forceinline__ float load_bf16(const void *p, int64_t i)
     return __uint_as_float((uint32_t)reinterpret_cast<const uint16_t *>(p)[i] << 16);
 }
 
-// The running state H[p][n] of this thread (n = its row r, p = 32 hf + j) as
+// The running state H[p][n] of this thread (n = its row r, p = 16 hq + j) as
 // bf16 into the K-major operand tile of the Yo product (rows p, K = n).
-__device__ __forceinline__ void store_state_tile(uint32_t tile, int r, int hf, const float (&H)[32])
+__device__ __forceinline__ void store_state_tile(uint32_t tile, int r, int hq, const float (&H)[16])
 {
     const uint32_t col = tile + (uint32_t)(r >> 6) * kHAtom + (uint32_t)(r & 7) * 2u;
     const uint32_t q = (uint32_t)(r & 63) >> 3;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
+    for (int j = 0; j < 16; ++j) {
         const __nv_bfloat16 v = __float2bfloat16_rn(H[j]);
-        st_shared_u16(col + sw128((uint32_t)(32 * hf + j), q), *reinterpret_cast<const uint16_t *>(&v));
+        st_shared_u16(col + sw128((uint32_t)(16 * hq + j), q), *reinterpret_cast<const uint16_t *>(&v));
     }
 }
 
@@ -325,6 +333,8 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
         mbar_init(bar(kHReady), kEpiWarps);
         mbar_init(bar(kYFree), kEpiWarps);
         mbar_init(bar(kDrain), 1);
+        mbar_init(bar(kStep0), 32);
+        mbar_init(bar(kStep1), 32);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -336,15 +346,32 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + kOffTmemSlot);
 
     if (warp == kTmaWarp) {
-        // ---- producer: X, B and C of chunk c into stage c % 2 ----
-        if (lane == 0) {
-            int issued = 0;
-            for (int c = 0; c < nchunks; ++c) {
-                const int st = c & 1;
-                if (c >= 2 && !role_wait(bar(kEmpty0 + st), ((c >> 1) + 1) & 1, abort_flag)) {
+        // ---- producer: X, B and C of chunk c into stage c % 2 (lane 0), and the chunk's step
+        // data (all lanes, four tokens each) into step buffer c % 2 ----
+        float *dl_all = reinterpret_cast<float *>(smem + kOffStep);
+        float *s2_all = dl_all + 2 * kQ;
+        uint16_t *cf_all = reinterpret_cast<uint16_t *>(s2_all + 2 * kQ);
+        const float Ah2 = p.A[h] * kLog2e;
+        const float bias = p.dt_bias ? p.dt_bias[h] : 0.f;
+        const uint16_t *dtp = reinterpret_cast<const uint16_t *>(p.dt) + b * p.dt_sb + h;
+        auto load_dt = [&](int c, float (&v)[4]) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int t = c * kQ + 4 * lane + k;
+                v[k] = t < L ? load_bf16(dtp, (int64_t)t * p.dt_st) : 0.f;
+            }
+        };
+        float dtv[4];
+        load_dt(0, dtv);
+        int issued = 0;
+        for (int c = 0; c < nchunks; ++c) {
+            const int st = c & 1;
+            if (c >= 2 && !__all_sync(0xffffffffu, role_wait(bar(kEmpty0 + st), ((c >> 1) + 1) & 1, abort_flag))) {
+                if (lane == 0)
                     give_up(p.status, abort_flag);
-                    break;
-                }
+                break;
+            }
+            if (lane == 0) {
                 const uint32_t sx = base + (uint32_t)st * kStageBytes, sb = sx + kXTile, sc = sb + kBCTile;
                 const uint32_t full = bar(kFull0 + st);
                 mbar_arrive_tx(full, kStageTx);
@@ -353,12 +380,53 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
                 tma_load_3d(sb + kQ * 128, &b_map, full, (int)(g * kN + 64), c * kQ, (int)b);
                 tma_load_3d(sc, &c_map, full, (int)(g * kN), c * kQ, (int)b);
                 tma_load_3d(sc + kQ * 128, &c_map, full, (int)(g * kN + 64), c * kQ, (int)b);
-                issued = c + 1;
             }
-            // the loads in flight must land before the CTA leaves
+            issued = c + 1;
+            // step sizes of tokens 4 lane .. 4 lane + 3 and the running sum of delta A (log2 units)
+            float d[4], v[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int t = c * kQ + 4 * lane + k;
+                d[k] = 0.f;
+                if (t < L) {
+                    d[k] = dtv[k] + bias;
+                    if (p.softplus)
+                        d[k] = ms::softplus(d[k]);
+                }
+            }
+            if (c + 1 < nchunks)
+                load_dt(c + 1, dtv);
+            v[0] = d[0] * Ah2;
+#pragma unroll
+            for (int k = 1; k < 4; ++k)
+                v[k] = fmaf(d[k], Ah2, v[k - 1]);
+            float incl = v[3];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float u = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o)
+                    incl += u;
+            }
+            const float excl = incl - v[3];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                v[k] += excl;
+            // s at the last token of this 32-token block (lanes 8 j .. 8 j + 7 hold block j)
+            const float vend = __shfl_sync(0xffffffffu, v[3], (lane & ~7) | 7);
+            float cfv[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                cfv[k] = ex2(vend - v[k]) * d[k];
+            *reinterpret_cast<float4 *>(dl_all + st * kQ + 4 * lane) = make_float4(d[0], d[1], d[2], d[3]);
+            *reinterpret_cast<float4 *>(s2_all + st * kQ + 4 * lane) = make_float4(v[0], v[1], v[2], v[3]);
+            *reinterpret_cast<uint2 *>(cf_all + st * kQ + 4 * lane) =
+                make_uint2(pack_bf16(cfv[0], cfv[1]), pack_bf16(cfv[2], cfv[3]));
+            mbar_arrive(bar(kStep0 + st));
+        }
+        // the loads in flight must land before the CTA leaves
+        if (lane == 0)
             for (int c = issued > 2 ? issued - 2 : 0; c < issued; ++c)
                 mbar_wait(bar(kFull0 + (c & 1)), (c >> 1) & 1);
-        }
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // ---- MMA issue (one thread) ----
@@ -421,26 +489,29 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
         }
         __syncwarp();
     } else {
-        // ---- epilogue: warps 0-7; thread = row r of the chunk, column half hf ----
-        const int sub = warp & 3, hf = warp >> 2;
+        // ---- epilogue: warps 0-15; thread = row r of the chunk, column quarter hq ----
+        // Software-pipelined over chunks: while the tensor core computes S and Yd of
+        // chunk c + 1, the warps gate and store y of chunk c.
+        const int sub = warp & 3, hq = warp >> 2;
         const int r = sub * 32 + lane;
         const uint32_t lane_base = (uint32_t)(sub * 32) << 16;
-        float *stepf = reinterpret_cast<float *>(smem + kOffStep);
-        float *wsum = stepf + 4 * kQ;
-        const float Ah2 = p.A[h] * kLog2e;
-        const float bias = p.dt_bias ? p.dt_bias[h] : 0.f;
+        const float *dl_all = reinterpret_cast<const float *>(smem + kOffStep);
+        const float *s2_all = dl_all + 2 * kQ;
+        const uint16_t *cf_all = reinterpret_cast<const uint16_t *>(s2_all + 2 * kQ);
         const float Dh = p.D ? p.D[h] : 0.f;
-        // this thread keeps H[p][n] for n = r and p = 32 hf + j
-        const int64_t hoff = (bh * kP + 32 * hf) * kN + r;
-        float H[32];
+        // this thread keeps H[p][n] for n = r and p = 16 hq + j
+        const int64_t hoff = (bh * kP + 16 * hq) * kN + r;
+        float H[16];
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
+        for (int j = 0; j < 16; ++j)
             H[j] = p.h0 ? p.h0[hoff + (int64_t)j * kN] : 0.f;
-        // rows 0-63 of M' never reach columns 64-127 (causal mask): zero them once
-        if (hf == 1 && sub < 2)
-            for (int q = 0; q < 8; ++q)
-                st_shared_v4(base + kOffM + kQ * 128 + sw128((uint32_t)r, (uint32_t)q), 0u, 0u, 0u, 0u);
-        store_state_tile(base + kOffH, r, hf, H);
+        // warp (sub, hq) owns the 32 x 32 block (rows sub, columns hq) of M'; blocks strictly
+        // above the diagonal are zero (causal mask) and are written once
+        const uint32_t mblk = base + kOffM + (uint32_t)(hq >> 1) * (kQ * 128);
+        if (hq > sub)
+            for (int q = 0; q < 4; ++q)
+                st_shared_v4(mblk + sw128((uint32_t)r, (uint32_t)(4 * (hq & 1) + q)), 0u, 0u, 0u, 0u);
+        store_state_tile(base + kOffH, r, hq, H);
         async_proxy_fence();
         __syncwarp();
         if (lane == 0)
@@ -454,85 +525,62 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
                 give_up(p.status, abort_flag);
             return ok;
         };
-        const uint16_t *dtp = reinterpret_cast<const uint16_t *>(p.dt) + b * p.dt_sb + h;
-        float dt_next = (hf == 0 && r < L) ? load_bf16(dtp, (int64_t)r * p.dt_st) : 0.f;
-        for (int c = 0; c < nchunks; ++c) {
-            const int st = c & 1, t0 = c * kQ;
-            const bool live = t0 + r < L;
-            const uint32_t sx = base + (uint32_t)st * kStageBytes;
-            float *dl = stepf + (c & 1) * kQ;
-            float *s2 = stepf + 2 * kQ + (c & 1) * kQ;
-            // the gate of this thread's 32 outputs, fetched early
-            uint4 zq[4] = {};
-            if (p.z && live) {
-                const uint4 *zp = reinterpret_cast<const uint4 *>(reinterpret_cast<const uint16_t *>(p.z) + b * p.z_sb +
-                                                                  (int64_t)(t0 + r) * p.z_st + h * kP + 32 * hf);
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    zq[q] = __ldg(zp + q);
-            }
-            // step sizes and the running sum of delta A (log2 units) in the chunk
-            if (hf == 0) {
-                float d = 0.f;
-                if (live) {
-                    d = dt_next + bias;
-                    if (p.softplus)
-                        d = d > 20.f ? d : log1pf(__expf(d));
-                }
-                dt_next = (t0 + kQ + r < L) ? load_bf16(dtp, (int64_t)(t0 + kQ + r) * p.dt_st) : 0.f;
-                float v = d * Ah2;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float u = __shfl_up_sync(0xffffffffu, v, o);
-                    if (lane >= o)
-                        v += u;
-                }
-                if (lane == 31)
-                    wsum[sub] = v;
-                wg0_sync();
-                for (int w = 0; w < sub; ++w)
-                    v += wsum[w];
-                dl[r] = d;
-                s2[r] = v;
-            }
-            epi_sync();
 
-            // (1) M' = mask o G and Xt, the operands of Yd and S
-            epi_wait(bar(kFull0 + st), (c >> 1) & 1);
-            epi_wait(bar(kGFull0 + (c & 1)), (c >> 1) & 1);
-            const float sr = s2[r];
+        // Build the operands M' and Xt of chunk k from its step data; returns s_r and s_end.
+        auto prepare = [&](int k, float &sr, float &se) {
+            const int stk = k & 1;
+            const float *dl = dl_all + stk * kQ, *s2 = s2_all + stk * kQ;
+            const uint16_t *cf = cf_all + stk * kQ;
+            epi_wait(bar(kStep0 + stk), (k >> 1) & 1);
+            epi_wait(bar(kFull0 + stk), (k >> 1) & 1);
+            epi_wait(bar(kGFull0 + (k & 1)), (k >> 1) & 1);
+            sr = s2[r];
+            se = s2[kQ - 1];
             if (ok) {
                 tc_after_sync();
-                if (!(hf == 1 && sub < 2)) {
-                    const uint32_t mt = base + kOffM + (uint32_t)hf * (kQ * 128);
+                if (hq <= sub) {
+                    // below the diagonal exp(s_r - s_i) = exp(s_r - s_e) exp(s_e - s_i), s_e the block's
+                    // last token, both factors <= 1; on the diagonal block the exponent is taken directly
+                    const float rf = hq < sub ? ex2(sr - s2[32 * hq + 31]) : 0.f;
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
-                        float gv[32];
-                        tmem_load32(tmem + lane_base + kColG + 128u * (uint32_t)(c & 1) + 64u * hf + 32u * half, gv);
-                        const int i0 = 64 * hf + 32 * half;
+                        float gv[16];
+                        tmem_load16(tmem + lane_base + kColG + 128u * (uint32_t)(k & 1) + 32u * (uint32_t)hq +
+                                        16u * (uint32_t)half,
+                                    gv);
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            const float4 sa = *reinterpret_cast<const float4 *>(s2 + i0 + 8 * q4);
-                            const float4 sb4 = *reinterpret_cast<const float4 *>(s2 + i0 + 8 * q4 + 4);
-                            const float4 da = *reinterpret_cast<const float4 *>(dl + i0 + 8 * q4);
-                            const float4 db4 = *reinterpret_cast<const float4 *>(dl + i0 + 8 * q4 + 4);
-                            const float si[8] = {sa.x, sa.y, sa.z, sa.w, sb4.x, sb4.y, sb4.z, sb4.w};
-                            const float di[8] = {da.x, da.y, da.z, da.w, db4.x, db4.y, db4.z, db4.w};
+                        for (int q8 = 0; q8 < 2; ++q8) {
+                            const int i0 = 32 * hq + 16 * half + 8 * q8;
                             float m[8];
+                            if (hq < sub) {
+                                const uint4 cw = *reinterpret_cast<const uint4 *>(cf + i0);
+                                const float ci[8] = {bf16_lo(cw.x), bf16_hi(cw.x), bf16_lo(cw.y), bf16_hi(cw.y),
+                                                     bf16_lo(cw.z), bf16_hi(cw.z), bf16_lo(cw.w), bf16_hi(cw.w)};
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                const int i = i0 + 8 * q4 + e;
-                                m[e] = i <= r ? gv[8 * q4 + e] * ex2(sr - si[e]) * di[e] : 0.f;
+                                for (int e = 0; e < 8; ++e)
+                                    m[e] = gv[8 * q8 + e] * ci[e] * rf;
+                            } else {
+                                const float4 sa = *reinterpret_cast<const float4 *>(s2 + i0);
+                                const float4 sb4 = *reinterpret_cast<const float4 *>(s2 + i0 + 4);
+                                const float4 da = *reinterpret_cast<const float4 *>(dl + i0);
+                                const float4 db4 = *reinterpret_cast<const float4 *>(dl + i0 + 4);
+                                const float si[8] = {sa.x, sa.y, sa.z, sa.w, sb4.x, sb4.y, sb4.z, sb4.w};
+                                const float di[8] = {da.x, da.y, da.z, da.w, db4.x, db4.y, db4.z, db4.w};
+#pragma unroll
+                                for (int e = 0; e < 8; ++e)
+                                    m[e] = i0 + e <= r ? gv[8 * q8 + e] * ex2(sr - si[e]) * di[e] : 0.f;
                             }
-                            st_shared_v4(mt + sw128((uint32_t)r, (uint32_t)(4 * half + q4)), pack_bf16(m[0], m[1]),
-                                         pack_bf16(m[2], m[3]), pack_bf16(m[4], m[5]), pack_bf16(m[6], m[7]));
+                            st_shared_v4(mblk + sw128((uint32_t)r, (uint32_t)(4 * (hq & 1) + 2 * half + q8)),
+                                         pack_bf16(m[0], m[1]), pack_bf16(m[2], m[3]), pack_bf16(m[4], m[5]),
+                                         pack_bf16(m[6], m[7]));
                         }
                     }
                 }
-                const float wr = ex2(s2[kQ - 1] - sr) * dl[r];
+                const float wr = ex2(se - sr) * dl[r];
+                const uint32_t sx = base + (uint32_t)stk * kStageBytes;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint32_t off = sw128((uint32_t)r, (uint32_t)(4 * hf + q));
+                for (int q = 0; q < 2; ++q) {
+                    const uint32_t off = sw128((uint32_t)r, (uint32_t)(2 * hq + q));
                     const uint4 v = ld_shared_v4(sx + off);
                     st_shared_v4(base + kOffXt + off, pack_bf16(bf16_lo(v.x) * wr, bf16_hi(v.x) * wr),
                                  pack_bf16(bf16_lo(v.y) * wr, bf16_hi(v.y) * wr),
@@ -545,18 +593,35 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
             __syncwarp();
             if (lane == 0 && ok)
                 mbar_arrive(bar(kPReady));
+        };
+
+        float sr_c = 0.f, se_c = 0.f;   // s_r and s_end of the chunk being finished
+        if (nchunks > 0)
+            prepare(0, sr_c, se_c);
+        for (int c = 0; c < nchunks; ++c) {
+            const int st = c & 1, t0 = c * kQ;
+            const bool live = t0 + r < L;
+            const uint32_t sx = base + (uint32_t)st * kStageBytes;
+            // the gate of this thread's 16 outputs
+            uint4 zq[2] = {};
+            if (p.z && live) {
+                const uint4 *zp = reinterpret_cast<const uint4 *>(reinterpret_cast<const uint16_t *>(p.z) + b * p.z_sb +
+                                                                  (int64_t)(t0 + r) * p.z_st + h * kP + 16 * hq);
+                zq[0] = __ldg(zp);
+                zq[1] = __ldg(zp + 1);
+            }
 
             // (2) state passing: H = exp(s_end) H + S^T
             epi_wait(bar(kSFull), c & 1);
             if (ok) {
                 tc_after_sync();
-                float sv[32];
-                tmem_load32(tmem + lane_base + kColS + 32u * hf, sv);
-                const float ac = ex2(s2[kQ - 1]);
+                float sv[16];
+                tmem_load16(tmem + lane_base + kColS + 16u * hq, sv);
+                const float ac = ex2(se_c);
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
+                for (int j = 0; j < 16; ++j)
                     H[j] = fmaf(ac, H[j], sv[j]);
-                store_state_tile(base + kOffH, r, hf, H);
+                store_state_tile(base + kOffH, r, hq, H);
             }
             async_proxy_fence();
             tc_before_sync();
@@ -564,54 +629,70 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
             if (lane == 0 && ok)
                 mbar_arrive(bar(kHReady));
 
-            // (3) y = Yd + exp(s_r) Yo + D x, gated
+            // (3a) y = Yd + exp(s_r) Yo + D x into registers; the Y columns and the stage are then free
+            float yv[16];
             epi_wait(bar(kYFull), c & 1);
             if (ok) {
                 tc_after_sync();
-                float yd[32], yo[32];
-                tmem_load32(tmem + lane_base + kColYd + 32u * hf, yd);
-                tmem_load32(tmem + lane_base + kColYo + 32u * hf, yo);
+                float yd[16];
+                tmem_load16(tmem + lane_base + kColYd + 16u * hq, yd);
+                tmem_load16(tmem + lane_base + kColYo + 16u * hq, yv);
                 tc_before_sync();
                 __syncwarp();
                 if (lane == 0)
                     mbar_arrive(bar(kYFree));
-                if (live) {
-                    const float er = ex2(sr);
-                    uint4 out[4];
+                const float er = ex2(sr_c);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint4 xv = ld_shared_v4(sx + sw128((uint32_t)r, (uint32_t)(4 * hf + q)));
-                        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-                        const uint32_t zw[4] = {zq[q].x, zq[q].y, zq[q].z, zq[q].w};
-                        uint32_t ow[4];
+                for (int q = 0; q < 2; ++q) {
+                    const uint4 xv = ld_shared_v4(sx + sw128((uint32_t)r, (uint32_t)(2 * hq + q)));
+                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int j = 8 * q + 2 * e;
-                            float o0 = fmaf(er, yo[j], yd[j]) + Dh * bf16_lo(xw[e]);
-                            float o1 = fmaf(er, yo[j + 1], yd[j + 1]) + Dh * bf16_hi(xw[e]);
-                            if (p.z) {
-                                const float z0 = bf16_lo(zw[e]), z1 = bf16_hi(zw[e]);
-                                o0 *= z0 / (1.f + __expf(-z0));
-                                o1 *= z1 / (1.f + __expf(-z1));
-                            }
-                            ow[e] = pack_bf16(o0, o1);
-                        }
-                        out[q] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                    for (int e = 0; e < 4; ++e) {
+                        const int j = 8 * q + 2 * e;
+                        yv[j] = fmaf(er, yv[j], fmaf(Dh, bf16_lo(xw[e]), yd[j]));
+                        yv[j + 1] = fmaf(er, yv[j + 1], fmaf(Dh, bf16_hi(xw[e]), yd[j + 1]));
                     }
-                    uint4 *yp = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.y) + b * p.y_sb +
-                                                          (int64_t)(t0 + r) * p.y_st + h * kP + 32 * hf);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        yp[q] = out[q];
                 }
             }
             __syncwarp();
             if (lane == 0 && ok)
                 mbar_arrive(bar(kEmpty0 + st));
+
+            // (1) operands of the next chunk, so that its products overlap the rest of this one
+            float sr_n = 0.f, se_n = 0.f;
+            if (c + 1 < nchunks)
+                prepare(c + 1, sr_n, se_n);
+
+            // (3b) gate and store y of chunk c
+            if (ok && live) {
+                uint4 out[2];
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const uint32_t zw[4] = {zq[q].x, zq[q].y, zq[q].z, zq[q].w};
+                    uint32_t ow[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int j = 8 * q + 2 * e;
+                        float o0 = yv[j], o1 = yv[j + 1];
+                        if (p.z) {
+                            o0 *= silu_fast(bf16_lo(zw[e]));
+                            o1 *= silu_fast(bf16_hi(zw[e]));
+                        }
+                        ow[e] = pack_bf16(o0, o1);
+                    }
+                    out[q] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                }
+                uint4 *yp = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.y) + b * p.y_sb +
+                                                      (int64_t)(t0 + r) * p.y_st + h * kP + 16 * hq);
+                yp[0] = out[0];
+                yp[1] = out[1];
+            }
+            sr_c = sr_n;
+            se_c = se_n;
         }
         if (ok && p.hT) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
+            for (int j = 0; j < 16; ++j)
                 p.hT[hoff + (int64_t)j * kN] = H[j];
         }
     }
