@@ -109,15 +109,18 @@ __device__ __forceinline__ void mbar_arrive_tx(uint32_t bar, uint32_t bytes)
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
 
+// One test of the phase; while it is incomplete the warp is suspended (it
+// issues nothing) until the phase completes or about 20 us pass, so waiting
+// warps leave the issue slots to the warps that work.
 __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity)
 {
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(done)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "r"(20000u)
         : "memory");
     return done != 0;
 }
@@ -200,6 +203,39 @@ __device__ __forceinline__ void tmem_load16(uint32_t taddr, float (&v)[16])
     for (int i = 0; i < 16; ++i)
         v[i] = __uint_as_float(r[i]);
 }
+
+// 8 consecutive fp32 columns of this warp's lanes, without waiting; pair with
+// tmem_wait_regs on the same registers before using them.
+__device__ __forceinline__ void tmem_load8_async(uint32_t taddr, uint32_t (&r)[8])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr)
+                 : "memory");
+}
+
+#define MS_R8(a, j) "+r"(a[j][0]), "+r"(a[j][1]), "+r"(a[j][2]), "+r"(a[j][3]), "+r"(a[j][4]), "+r"(a[j][5]), \
+                    "+r"(a[j][6]), "+r"(a[j][7])
+// Wait for this thread's outstanding tensor-memory loads; the registers are
+// operands so that no use of them is scheduled above the wait.
+template <int G> __device__ __forceinline__ void tmem_wait_regs(uint32_t (&a)[G][8]);
+template <> __device__ __forceinline__ void tmem_wait_regs<1>(uint32_t (&a)[1][8])
+{
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : MS_R8(a, 0) : : "memory");
+}
+template <> __device__ __forceinline__ void tmem_wait_regs<2>(uint32_t (&a)[2][8])
+{
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : MS_R8(a, 0), MS_R8(a, 1) : : "memory");
+}
+template <> __device__ __forceinline__ void tmem_wait_regs<3>(uint32_t (&a)[3][8])
+{
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : MS_R8(a, 0), MS_R8(a, 1), MS_R8(a, 2) : : "memory");
+}
+template <> __device__ __forceinline__ void tmem_wait_regs<4>(uint32_t (&a)[4][8])
+{
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : MS_R8(a, 0), MS_R8(a, 1), MS_R8(a, 2), MS_R8(a, 3) : : "memory");
+}
+#undef MS_R8
 
 __device__ __forceinline__ float ex2(float v)
 {
@@ -297,6 +333,66 @@ __device__ __forceinline__ void store_state_tile(uint32_t tile, int r, int hq, c
     for (int j = 0; j < 16; ++j) {
         const __nv_bfloat16 v = __float2bfloat16_rn(H[j]);
         st_shared_u16(col + sw128((uint32_t)(16 * hq + j), q), *reinterpret_cast<const uint16_t *>(&v));
+    }
+}
+
+// M' for row r (row block K, this warp's quarter hq): column groups of 8 at
+// 32 j + 8 hq for j = 0..K. Groups below the diagonal block use the factored
+// decay exp(s_r - s_e(j)) exp(s_e(j) - s_i) delta_i (cf); the group in the
+// diagonal block takes exp(s_r - s_i) directly and masks i > r.
+// Groups j = J0 .. J0 + G - 1 of build_mask_rows, loaded together.
+template <int K, int J0, int G>
+__device__ __forceinline__ void build_mask_groups(uint32_t tg, uint32_t m_tile, int r, int hq, float sr,
+                                                  const float *dl, const float *s2, const uint16_t *cf)
+{
+    uint32_t g[G][8];
+#pragma unroll
+    for (int u = 0; u < G; ++u)
+        tmem_load8_async(tg + 32u * (uint32_t)(J0 + u) + 8u * (uint32_t)hq, g[u]);
+    tmem_wait_regs<G>(g);
+#pragma unroll
+    for (int u = 0; u < G; ++u) {
+        const int j = J0 + u;
+        const int i0 = 32 * j + 8 * hq;
+        float m[8];
+        if (j < K) {
+            const float rf = ex2(sr - s2[32 * j + 31]);
+            const uint4 cw = *reinterpret_cast<const uint4 *>(cf + i0);
+            const float ci[8] = {bf16_lo(cw.x), bf16_hi(cw.x), bf16_lo(cw.y), bf16_hi(cw.y),
+                                 bf16_lo(cw.z), bf16_hi(cw.z), bf16_lo(cw.w), bf16_hi(cw.w)};
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                m[e] = __uint_as_float(g[u][e]) * ci[e] * rf;
+        } else {
+            const float4 sa = *reinterpret_cast<const float4 *>(s2 + i0);
+            const float4 sb4 = *reinterpret_cast<const float4 *>(s2 + i0 + 4);
+            const float4 da = *reinterpret_cast<const float4 *>(dl + i0);
+            const float4 db4 = *reinterpret_cast<const float4 *>(dl + i0 + 4);
+            const float si[8] = {sa.x, sa.y, sa.z, sa.w, sb4.x, sb4.y, sb4.z, sb4.w};
+            const float di[8] = {da.x, da.y, da.z, da.w, db4.x, db4.y, db4.z, db4.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                m[e] = i0 + e <= r ? __uint_as_float(g[u][e]) * ex2(sr - si[e]) * di[e] : 0.f;
+        }
+        st_shared_v4(m_tile + (uint32_t)(i0 >> 6) * (kQ * 128) + sw128((uint32_t)r, (uint32_t)((i0 & 63) >> 3)),
+                     pack_bf16(m[0], m[1]), pack_bf16(m[2], m[3]), pack_bf16(m[4], m[5]), pack_bf16(m[6], m[7]));
+    }
+}
+
+// M' for row r (row block K, this warp's quarter hq): column groups of 8 at
+// 32 j + 8 hq for j = 0..K. Groups below the diagonal block use the factored
+// decay exp(s_r - s_e(j)) exp(s_e(j) - s_i) delta_i (cf); the group in the
+// diagonal block takes exp(s_r - s_i) directly and masks i > r. Every warp of
+// an SMSP thus gets one diagonal group and K lower groups.
+template <int K>
+__device__ __forceinline__ void build_mask_rows(uint32_t tg, uint32_t m_tile, int r, int hq, float sr,
+                                                const float *dl, const float *s2, const uint16_t *cf)
+{
+    if constexpr (K < 2) {
+        build_mask_groups<K, 0, K + 1>(tg, m_tile, r, hq, sr, dl, s2, cf);
+    } else {
+        build_mask_groups<K, 0, 2>(tg, m_tile, r, hq, sr, dl, s2, cf);
+        build_mask_groups<K, 2, K - 1>(tg, m_tile, r, hq, sr, dl, s2, cf);
     }
 }
 
@@ -505,12 +601,14 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
 #pragma unroll
         for (int j = 0; j < 16; ++j)
             H[j] = p.h0 ? p.h0[hoff + (int64_t)j * kN] : 0.f;
-        // warp (sub, hq) owns the 32 x 32 block (rows sub, columns hq) of M'; blocks strictly
-        // above the diagonal are zero (causal mask) and are written once
-        const uint32_t mblk = base + kOffM + (uint32_t)(hq >> 1) * (kQ * 128);
-        if (hq > sub)
-            for (int q = 0; q < 4; ++q)
-                st_shared_v4(mblk + sw128((uint32_t)r, (uint32_t)(4 * (hq & 1) + q)), 0u, 0u, 0u, 0u);
+        // rows of block sub: M' columns in blocks above the diagonal are zero (causal mask)
+        // and are written once, this warp taking the groups 32 j + 8 hq
+        for (int j = sub + 1; j < 4; ++j) {
+            const int i0 = 32 * j + 8 * hq;
+            st_shared_v4(base + kOffM + (uint32_t)(i0 >> 6) * (kQ * 128) +
+                             sw128((uint32_t)r, (uint32_t)((i0 & 63) >> 3)),
+                         0u, 0u, 0u, 0u);
+        }
         store_state_tile(base + kOffH, r, hq, H);
         async_proxy_fence();
         __syncwarp();
@@ -538,43 +636,12 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
             se = s2[kQ - 1];
             if (ok) {
                 tc_after_sync();
-                if (hq <= sub) {
-                    // below the diagonal exp(s_r - s_i) = exp(s_r - s_e) exp(s_e - s_i), s_e the block's
-                    // last token, both factors <= 1; on the diagonal block the exponent is taken directly
-                    const float rf = hq < sub ? ex2(sr - s2[32 * hq + 31]) : 0.f;
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        float gv[16];
-                        tmem_load16(tmem + lane_base + kColG + 128u * (uint32_t)(k & 1) + 32u * (uint32_t)hq +
-                                        16u * (uint32_t)half,
-                                    gv);
-#pragma unroll
-                        for (int q8 = 0; q8 < 2; ++q8) {
-                            const int i0 = 32 * hq + 16 * half + 8 * q8;
-                            float m[8];
-                            if (hq < sub) {
-                                const uint4 cw = *reinterpret_cast<const uint4 *>(cf + i0);
-                                const float ci[8] = {bf16_lo(cw.x), bf16_hi(cw.x), bf16_lo(cw.y), bf16_hi(cw.y),
-                                                     bf16_lo(cw.z), bf16_hi(cw.z), bf16_lo(cw.w), bf16_hi(cw.w)};
-#pragma unroll
-                                for (int e = 0; e < 8; ++e)
-                                    m[e] = gv[8 * q8 + e] * ci[e] * rf;
-                            } else {
-                                const float4 sa = *reinterpret_cast<const float4 *>(s2 + i0);
-                                const float4 sb4 = *reinterpret_cast<const float4 *>(s2 + i0 + 4);
-                                const float4 da = *reinterpret_cast<const float4 *>(dl + i0);
-                                const float4 db4 = *reinterpret_cast<const float4 *>(dl + i0 + 4);
-                                const float si[8] = {sa.x, sa.y, sa.z, sa.w, sb4.x, sb4.y, sb4.z, sb4.w};
-                                const float di[8] = {da.x, da.y, da.z, da.w, db4.x, db4.y, db4.z, db4.w};
-#pragma unroll
-                                for (int e = 0; e < 8; ++e)
-                                    m[e] = i0 + e <= r ? gv[8 * q8 + e] * ex2(sr - si[e]) * di[e] : 0.f;
-                            }
-                            st_shared_v4(mblk + sw128((uint32_t)r, (uint32_t)(4 * (hq & 1) + 2 * half + q8)),
-                                         pack_bf16(m[0], m[1]), pack_bf16(m[2], m[3]), pack_bf16(m[4], m[5]),
-                                         pack_bf16(m[6], m[7]));
-                        }
-                    }
+                const uint32_t tg = tmem + lane_base + kColG + 128u * (uint32_t)(k & 1);
+                switch (sub) {
+                case 0: build_mask_rows<0>(tg, base + kOffM, r, hq, sr, dl, s2, cf); break;
+                case 1: build_mask_rows<1>(tg, base + kOffM, r, hq, sr, dl, s2, cf); break;
+                case 2: build_mask_rows<2>(tg, base + kOffM, r, hq, sr, dl, s2, cf); break;
+                default: build_mask_rows<3>(tg, base + kOffM, r, hq, sr, dl, s2, cf); break;
                 }
                 const float wr = ex2(se - sr) * dl[r];
                 const uint32_t sx = base + (uint32_t)stk * kStageBytes;
