@@ -45,7 +45,8 @@ MUFU_PER_CLK = 16
 # DRAM bytes (read + write) per launch from an ncu capture of the named kernel
 # on the named workload (profiles/ holds the summary); any other kernel or
 # workload reports traffic null.
-NCU_TRAFFIC = {("mamba130m_layer", "rec_kernel<bf16, 4>"): 152201728 + 32785152}
+NCU_TRAFFIC = {("mamba130m_layer", "rec_kernel<bf16, 4>"): 152333568 + 33228544,
+               ("mamba2_layer_d2048", "ssd_kernel"): 563181568 + 244632320}
 FP32_PER_CLK = 128
 
 
@@ -66,6 +67,8 @@ def parse_args(argv=None):
                     help="steps of the exponential-trapezoidal scan (0 skips the leg)")
     ap.add_argument("--bwd-steps", type=int, default=20,
                     help="steps of the scan backward (0 skips the leg)")
+    ap.add_argument("--ssd-steps", type=int, default=50,
+                    help="steps of the Mamba-2 chunked SSD forward on its (4, 8192, 64 heads) layer (0 skips)")
     ap.add_argument("--decode-steps", type=int, default=1000,
                     help="decode state-update steps timed on the (256, 5120, 16) decode workload (0: skip)")
     return ap.parse_args(argv)
@@ -138,8 +141,8 @@ def load_peaks():
         with open(path) as f:
             d = json.load(f)
         return {"hbm_gbs": float(d["hbm_gbs"]), "sm_max_mhz": float(d.get("sm_max_mhz", 1965.0)),
-                "source": "measured"}
-    return {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "source": "fallback"}
+                "bf16_tflops": float(d.get("bf16_tflops", 1590.0)), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "bf16_tflops": 1590.0, "source": "fallback"}
 
 
 # ----------------------------------------------------------------------------
@@ -433,6 +436,7 @@ def run_ours(args, dist: Dist):
                 if args.prologue_steps > 0 else None)
     trap = run_trap(args, dist, dev, w, sets, params, y, hT, counts, mufu_peak) if args.trap_steps > 0 else None
     bwd = run_bwd(args, dist, dev, w, sets, params, counts, mufu_peak) if args.bwd_steps > 0 else None
+    ssd = run_ssd(args, dist, dev, peaks) if args.ssd_steps > 0 else None
 
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
@@ -446,7 +450,7 @@ def run_ours(args, dist: Dist):
         "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded)", "config": workload_config(w, {"global_batch": w.batch * dist.world}),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode, "conv_prologue": prologue,
-        "trapezoidal": trap, "backward": bwd,
+        "trapezoidal": trap, "backward": bwd, "ssd": ssd,
         "gpu_launches": args.steps * launches_per_step, "clocks": clocks,
     }
     if dist.rank == 0:
@@ -613,6 +617,86 @@ def run_bwd(args, dist: Dist, dev, w, sets, params, counts, mufu_peak):
                      "peak": mufu_peak / 1e12, "frac": mufu / (us * 1e-6) / mufu_peak, "algorithmic_mufu": mufu,
                      "note": "two ex2 per element: the checkpoint sweep and the per-chunk recomputation"},
         "gpu_launches": 6 * n,
+    }
+
+
+def ssd_counts(w, chunk=128):
+    """Algorithmic work of one SSD forward pass.
+
+    Bytes: x, z and dt read once, B and C read once, y written once, the
+    final state written once, A, D and dt_bias read once. Tensor FLOPs of the
+    chunked form per (token, head): 2 Q N for C B^T, 2 Q P for the masked
+    product with X, and 2 N P each for the chunk state and the state readout.
+    """
+    tok = w.batch * w.seqlen
+    th = tok * w.nheads
+    bytes_ = (th * w.headdim * 2 * (3 if w.has_z else 2) + th * 2 + 2 * tok * w.ngroups * w.dstate * 2
+              + 3 * w.nheads * 4 + w.batch * w.nheads * w.headdim * w.dstate * 4)
+    flops = th * (2 * chunk * w.dstate + 2 * chunk * w.headdim + 4 * w.dstate * w.headdim)
+    return {"elements": w.elements, "bytes": bytes_, "tensor_flops": flops}
+
+
+def run_ssd(args, dist: Dist, dev, peaks):
+    """Time the Mamba-2 chunked SSD forward (tcgen05 kernel) on the page's
+    layer: batch 4, 8192 tokens, 64 heads of 64 channels, d_state 128, one
+    group, bf16, with gate. Its inputs (about 560 MB) exceed the L2."""
+    import ctypes
+
+    import torch
+    import selective_state_space_27_b200 as ms
+    from selective_state_space_27_b200.inputs import SSD_WORKLOADS, make_ssd_inputs
+
+    w = SSD_WORKLOADS["mamba2_layer_d2048"]
+    inp = make_ssd_inputs(w, seed=w.seed + 1000 * dist.rank)
+
+    def dev_t(a, bf16):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        return (t.view(torch.bfloat16) if bf16 else t).to(dev)
+
+    t = {k: dev_t(inp[k], True) for k in ("x", "dt", "B", "C", "z")}
+    prm = {k: dev_t(inp[k], False) for k in ("A", "D", "dt_bias")}
+    y = torch.empty_like(t["x"])
+    hT = torch.empty((w.batch, w.nheads, w.headdim, w.dstate), dtype=torch.float32, device=dev)
+    status = torch.zeros(ms.SSD_WORKSPACE_BYTES, dtype=torch.uint8, device=dev)
+    a = ms.build_ssd_args(t["x"], t["dt"], prm["A"], t["B"], t["C"], y, D=prm["D"], z=t["z"],
+                          dt_bias=prm["dt_bias"], final_state=hT)
+    lib = ms.load_library()
+    stream = torch.cuda.current_stream()
+
+    def step():
+        rc = lib.mamba_ssd_fwd(ctypes.byref(a), status.data_ptr(), status.numel(), stream.cuda_stream)
+        if rc != 0:
+            raise ms.MambaScanError(rc, lib.mamba_last_error().decode())
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    n = args.ssd_steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms.ssd_check(status)
+    us = dist.max(e0.elapsed_time(e1) * 1e3 / n, dev)
+    c = ssd_counts(w)
+    gbs = c["bytes"] / (us * 1e-6) / 1e9
+    tflops = c["tensor_flops"] / (us * 1e-6) / 1e12
+    return {
+        "workload": w.name, "steps": n, "metric": "Mamba-2 SSD forward B*L*H*P*N state elems/s", "unit": UNIT,
+        "value": dist.world * c["elements"] / (us * 1e-6), "us_per_step": us,
+        "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "nheads": w.nheads,
+                   "headdim": w.headdim, "dstate": w.dstate, "ngroups": w.ngroups, "chunk": 128, "dtype": "bf16",
+                   "l2": "inputs larger than L2"},
+        "roofline": {"bound": "hbm", "unit": "GB/s", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                     "frac": gbs / peaks["hbm_gbs"], "traffic": NCU_TRAFFIC.get((w.name, "ssd_kernel")),
+                     "peak_source": peaks["source"], "algorithmic_per_launch": c,
+                     "tensor": {"achieved_tflops": tflops, "peak_tflops": peaks["bf16_tflops"],
+                                "frac": tflops / peaks["bf16_tflops"]},
+                     "bound_times_us": {"hbm": c["bytes"] / (peaks["hbm_gbs"] * 1e9) * 1e6,
+                                        "tensor": c["tensor_flops"] / (peaks["bf16_tflops"] * 1e12) * 1e6}},
+        "gpu_launches": n,
     }
 
 
