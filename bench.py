@@ -46,7 +46,7 @@ MUFU_PER_CLK = 16
 # on the named workload (profiles/ holds the summary); any other kernel or
 # workload reports traffic null.
 NCU_TRAFFIC = {("mamba130m_layer", "rec_kernel<bf16, 4>"): 152333568 + 33228544,
-               ("mamba2_layer_d2048", "ssd_kernel"): 563181568 + 244632320}
+               ("mamba2_layer_d2048", "ssd_kernel"): 563163904 + 244780288}
 FP32_PER_CLK = 128
 
 
