@@ -50,8 +50,11 @@ __device__ __forceinline__ float half_warp_sum(float v) {
     return v;
 }
 
-// Dynamic shared memory of a CTA, in floats.
-constexpr int kRT = kRows * (kT + 1);            // a [row][step] tile
+// Dynamic shared memory of a CTA, in floats. The per-row step tiles have rows
+// of 20 floats (16-byte aligned) so that a chain thread reads four steps of its
+// row with one vector load.
+constexpr int kTS = kT + 4;
+constexpr int kRT = kRows * kTS;                 // a [row][step] tile
 constexpr int kTN = kT * (kN + 1);               // a [step][state] tile
 constexpr int kRNT = kRows * kN * (kT + 1);      // a [row][state][step] (or [step][row][state]) tile
 constexpr int kBwdSmemFloats = 4 * kRT + 2 * kTN + 4 * kRNT;
@@ -59,10 +62,10 @@ constexpr int kBwdSmemFloats = 4 * kRT + 2 * kTN + 4 * kRNT;
 template <typename T>
 __global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(const ScanParams p, const BwdParams q) {
     extern __shared__ __align__(16) float smf[];
-    auto dts = reinterpret_cast<float (*)[kT + 1]>(smf);
-    auto dus = reinterpret_cast<float (*)[kT + 1]>(smf + kRT);
-    auto uus = reinterpret_cast<float (*)[kT + 1]>(smf + 2 * kRT);
-    auto dss = reinterpret_cast<float (*)[kT + 1]>(smf + 3 * kRT);
+    auto dts = reinterpret_cast<float (*)[kTS]>(smf);
+    auto dus = reinterpret_cast<float (*)[kTS]>(smf + kRT);
+    auto uus = reinterpret_cast<float (*)[kTS]>(smf + 2 * kRT);
+    auto dss = reinterpret_cast<float (*)[kTS]>(smf + 3 * kRT);
     auto Bs = reinterpret_cast<float (*)[kN + 1]>(smf + 4 * kRT);
     auto Cs = reinterpret_cast<float (*)[kN + 1]>(smf + 4 * kRT + kTN);
     float *tiles = smf + 4 * kRT + 2 * kTN;
@@ -135,7 +138,13 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(const ScanParams p,
         if (c + 2 < nchunks) nxt = load_raw(c + 1, false);
         __syncthreads();
 #pragma unroll
-        for (int t = 0; t < kT; ++t) h = fmaf(ex2_approx(dts[r][t] * A2), h, dus[r][t] * Bs[t][n]);
+        for (int t4 = 0; t4 < kT; t4 += 4) {
+            const float4 dt4 = *reinterpret_cast<const float4 *>(&dts[r][t4]);
+            const float4 du4 = *reinterpret_cast<const float4 *>(&dus[r][t4]);
+            const float dtv[4] = {dt4.x, dt4.y, dt4.z, dt4.w}, duv[4] = {du4.x, du4.y, du4.z, du4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) h = fmaf(ex2_approx(dtv[e] * A2), h, duv[e] * Bs[t4 + e][n]);
+        }
         if (ok) ckpt[c * kN] = h;   // rows past the end share a clamped index: no checkpoints
         __syncthreads();
     }
@@ -160,10 +169,16 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(const ScanParams p,
         {
             float hh = hs;
 #pragma unroll
-            for (int t = 0; t < kT; ++t) {
-                Av[t] = ex2_approx(dts[r][t] * A2);
-                hh = fmaf(Av[t], hh, dus[r][t] * Bs[t][n]);
-                H[t] = hh;
+            for (int t4 = 0; t4 < kT; t4 += 4) {
+                const float4 dt4 = *reinterpret_cast<const float4 *>(&dts[r][t4]);
+                const float4 du4 = *reinterpret_cast<const float4 *>(&dus[r][t4]);
+                const float dtv[4] = {dt4.x, dt4.y, dt4.z, dt4.w}, duv[4] = {du4.x, du4.y, du4.z, du4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    Av[t4 + e] = ex2_approx(dtv[e] * A2);
+                    hh = fmaf(Av[t4 + e], hh, duv[e] * Bs[t4 + e][n]);
+                    H[t4 + e] = hh;
+                }
             }
         }
         // ds, dz of item (row r, step n); s_t sums C h over the row's states
@@ -187,16 +202,26 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(const ScanParams p,
 
         // adjoint recurrence through the chunk
 #pragma unroll
-        for (int t = kT - 1; t >= 0; --t) {
-            const float ds = dss[r][t], dt = dts[r][t], Bv = Bs[t][n];
-            const float hprev = t > 0 ? H[t - 1] : hs;
-            const float gn = fmaf(ds, Cs[t][n], G);
-            pC[t][r][n] = ds * H[t];
-            pB[t][r][n] = gn * dus[r][t];
-            pDU[r][n][t] = gn * dt * Bv;
-            pDD[r][n][t] = gn * fmaf(Bv, uus[r][t], hprev * Av[t] * Areal);
-            dA_acc = fmaf(gn * hprev, Av[t] * dt, dA_acc);
-            G = Av[t] * gn;
+        for (int t4 = kT - 4; t4 >= 0; t4 -= 4) {
+            const float4 ds4 = *reinterpret_cast<const float4 *>(&dss[r][t4]);
+            const float4 dt4 = *reinterpret_cast<const float4 *>(&dts[r][t4]);
+            const float4 du4 = *reinterpret_cast<const float4 *>(&dus[r][t4]);
+            const float4 uu4 = *reinterpret_cast<const float4 *>(&uus[r][t4]);
+            const float dsv4[4] = {ds4.x, ds4.y, ds4.z, ds4.w}, dtv4[4] = {dt4.x, dt4.y, dt4.z, dt4.w};
+            const float duv4[4] = {du4.x, du4.y, du4.z, du4.w}, uuv4[4] = {uu4.x, uu4.y, uu4.z, uu4.w};
+#pragma unroll
+            for (int e = 3; e >= 0; --e) {
+                const int t = t4 + e;
+                const float ds = dsv4[e], dt = dtv4[e], Bv = Bs[t][n];
+                const float hprev = t > 0 ? H[t - 1] : hs;
+                const float gn = fmaf(ds, Cs[t][n], G);
+                pC[t][r][n] = ds * H[t];
+                pB[t][r][n] = gn * duv4[e];
+                pDU[r][n][t] = gn * dt * Bv;
+                pDD[r][n][t] = gn * fmaf(Bv, uuv4[e], hprev * Av[t] * Areal);
+                dA_acc = fmaf(gn * hprev, Av[t] * dt, dA_acc);
+                G = Av[t] * gn;
+            }
         }
         __syncthreads();
 
