@@ -19,9 +19,10 @@
 // float per chain and chunk: 1/16 of the expanded state). Phase B walks the
 // chunks backward: it recomputes the chunk's 16 states from the previous
 // checkpoint into registers and runs the adjoint recurrence through them.
-// Per-(row, t) sums over the 16 states go through [row][state][step] tiles
+// Per-(row, t) sums over the 16 states go through [row][step][state] tiles
 // in shared memory (written by the chain threads, summed by one thread per
-// (row, step); both access patterns are free of bank conflicts); the B and C
+// (row, step) with four vector loads; both access patterns are free of bank
+// conflicts); the B and C
 // gradients are summed over the CTA's rows the same way and added to global
 // memory with atomics, as are the A, D and delta_bias gradients (sums over
 // the batch). The caller's reduction outputs are zeroed first.
@@ -56,8 +57,13 @@ __device__ __forceinline__ float half_warp_sum(float v) {
 constexpr int kTS = kT + 4;
 constexpr int kRT = kRows * kTS;                 // a [row][step] tile
 constexpr int kTN = kT * (kN + 1);               // a [step][state] tile
-constexpr int kRNT = kRows * kN * (kT + 1);      // a [row][state][step] (or [step][row][state]) tile
-constexpr int kBwdSmemFloats = 4 * kRT + 2 * kTN + 4 * kRNT;
+constexpr int kRNT = kRows * kN * (kT + 1);      // a [step][row][state] tile
+// [row][step][state] tiles summed over the states by one thread per (row, step):
+// steps 20 floats apart, rows 336 (both write and read patterns conflict free)
+constexpr int kQS = kN + 4, kQR = kT * kQS + 16;
+constexpr int kRTN = kRows * kQR;
+constexpr int kBwdSmemFloats = 4 * kRT + 2 * kTN + 2 * kRNT + 2 * kRTN;
+static_assert(kRTN <= 2 * kRNT, "the readout tile aliases the B and C gradient tiles");
 
 template <typename T>
 __global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(const ScanParams p, const BwdParams q) {
@@ -71,9 +77,17 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(const ScanParams p,
     float *tiles = smf + 4 * kRT + 2 * kTN;
     auto pB = reinterpret_cast<float (*)[kRows][kN + 1]>(tiles);              // [step][row][state]
     auto pC = reinterpret_cast<float (*)[kRows][kN + 1]>(tiles + kRNT);
-    auto pS = reinterpret_cast<float (*)[kN][kT + 1]>(tiles);                 // [row][state][step], before pB
-    auto pDU = reinterpret_cast<float (*)[kN][kT + 1]>(tiles + 2 * kRNT);
-    auto pDD = reinterpret_cast<float (*)[kN][kT + 1]>(tiles + 3 * kRNT);
+    float *pS = tiles;                                                          // [row][step][state], before pB
+    float *pDU = tiles + 2 * kRNT;
+    float *pDD = tiles + 2 * kRNT + kRTN;
+    auto rts = [](int row, int step, int state) { return row * kQR + step * kQS + state; };
+    // sum over the 16 states of (row, step) in a [row][step][state] tile
+    auto state_sum = [&](const float *tile, int row, int step) {
+        const float4 *v = reinterpret_cast<const float4 *>(tile + rts(row, step, 0));
+        const float4 a = v[0], b4 = v[1], c4 = v[2], d4 = v[3];
+        return ((a.x + a.y) + (a.z + a.w)) + ((b4.x + b4.y) + (b4.z + b4.w)) + ((c4.x + c4.y) + (c4.z + c4.w)) +
+               ((d4.x + d4.y) + (d4.z + d4.w));
+    };
 
     const int tid = threadIdx.x;
     const int r = tid / kN, n = tid % kN;          // chain (row, state); also item (row, step n)
@@ -183,11 +197,9 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(const ScanParams p,
         }
         // ds, dz of item (row r, step n); s_t sums C h over the row's states
 #pragma unroll
-        for (int t = 0; t < kT; ++t) pS[r][n][t] = Cs[t][n] * H[t];
+        for (int t = 0; t < kT; ++t) pS[rts(r, t, n)] = Cs[t][n] * H[t];
         __syncthreads();
-        float s_mine = Dd * uus[r][n];
-#pragma unroll
-        for (int nn = 0; nn < kN; ++nn) s_mine += pS[r][nn][n];
+        const float s_mine = Dd * uus[r][n] + state_sum(pS, r, n);
         float dsv = dyv;
         if (p.z) {
             const float sg = __fdividef(1.f, 1.f + ex2_approx(-zv * kLog2e));
@@ -217,8 +229,8 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(const ScanParams p,
                 const float gn = fmaf(ds, Cs[t][n], G);
                 pC[t][r][n] = ds * H[t];
                 pB[t][r][n] = gn * duv4[e];
-                pDU[r][n][t] = gn * dt * Bv;
-                pDD[r][n][t] = gn * fmaf(Bv, uuv4[e], hprev * Av[t] * Areal);
+                pDU[rts(r, t, n)] = gn * dt * Bv;
+                pDD[rts(r, t, n)] = gn * fmaf(Bv, uuv4[e], hprev * Av[t] * Areal);
                 dA_acc = fmaf(gn * hprev, Av[t] * dt, dA_acc);
                 G = Av[t] * gn;
             }
@@ -227,12 +239,8 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(const ScanParams p,
 
         // item (row r, step n): du, ddelta; B/C gradients of (step, state) = (tid / 16, tid % 16)
         if (in) {
-            float du = dss[r][n] * Dd, dd = 0.f;
-#pragma unroll
-            for (int nn = 0; nn < kN; ++nn) {
-                du += pDU[r][nn][n];
-                dd += pDD[r][nn][n];
-            }
+            const float du = dss[r][n] * Dd + state_sum(pDU, r, n);
+            float dd = state_sum(pDD, r, n);
             if (p.softplus) dd *= __fdividef(1.f, 1.f + ex2_approx(-(cur.dl + bias) * kLog2e));
             static_cast<T *>(q.du)[b * q.du_sb + dc * q.du_sd + ti] = from_f32<T>(du);
             static_cast<T *>(q.ddelta)[b * q.dd_sb + dc * q.dd_sd + ti] = from_f32<T>(dd);
