@@ -634,7 +634,7 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
 #pragma unroll
             for (int e = 0; e < IP; e += 2) {
                 const float2 yv = add2(skip[e / 2], sum[e / 2]);
-                const float2 g = mul2(yv, silu2(f2(elem(z, e), elem(z, e + 1))));
+                const float2 g = mul2(yv, silu2_out<T>(f2(elem(z, e), elem(z, e + 1))));
                 outv[e] = g.x;
                 outv[e + 1] = g.y;
             }
@@ -672,7 +672,7 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
                     a1 = fmaf(cw[m], win(e + 1 + VE - 3 + m), a1);
                 }
                 float2 uv = f2(a0, a1);
-                if (p.conv_silu) uv = silu2(uv);
+                if (p.conv_silu) uv = silu2_out<T>(uv);
                 u2[e / 2] = uv;
                 *reinterpret_cast<float2 *>(sk + e) = mul2(f2(Dd, Dd), uv);
             }
