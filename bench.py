@@ -45,7 +45,7 @@ MUFU_PER_CLK = 16
 # DRAM bytes (read + write) per launch from an ncu capture of the named kernel
 # on the named workload (profiles/ holds the summary); any other kernel or
 # workload reports traffic null.
-NCU_TRAFFIC = {("mamba130m_layer", "rec_kernel<bf16, 4>"): 152333568 + 33228544,
+NCU_TRAFFIC = {("mamba130m_layer", "rec_kernel<bf16, 4>"): 152333056 + 31869696,
                ("mamba2_layer_d2048", "ssd_kernel"): 563163904 + 244780288}
 FP32_PER_CLK = 128
 

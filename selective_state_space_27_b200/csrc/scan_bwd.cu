@@ -57,7 +57,11 @@ __device__ __forceinline__ float half_warp_sum(float v) {
 constexpr int kTS = kT + 4;
 constexpr int kRT = kRows * kTS;                 // a [row][step] tile
 constexpr int kTN = kT * (kN + 1);               // a [step][state] tile
-constexpr int kRNT = kRows * kN * (kT + 1);      // a [step][row][state] tile
+// [step][row][state] tiles summed over the rows by one thread per (step, state):
+// rows 16 floats apart, steps 272, so that the two rows a warp writes and the
+// two steps a warp sums fall on disjoint banks
+constexpr int kBR = kN, kBT = kRows * kN + 16;
+constexpr int kRNT = kT * kBT;
 // [row][step][state] tiles summed over the states by one thread per (row, step):
 // steps 20 floats apart, rows 336 (both write and read patterns conflict free)
 constexpr int kQS = kN + 4, kQR = kT * kQS + 16;
@@ -75,8 +79,9 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(const ScanParams p,
     auto Bs = reinterpret_cast<float (*)[kN + 1]>(smf + 4 * kRT);
     auto Cs = reinterpret_cast<float (*)[kN + 1]>(smf + 4 * kRT + kTN);
     float *tiles = smf + 4 * kRT + 2 * kTN;
-    auto pB = reinterpret_cast<float (*)[kRows][kN + 1]>(tiles);              // [step][row][state]
-    auto pC = reinterpret_cast<float (*)[kRows][kN + 1]>(tiles + kRNT);
+    float *pB = tiles;                                                          // [step][row][state]
+    float *pC = tiles + kRNT;
+    auto trs = [](int step, int row, int state) { return step * kBT + row * kBR + state; };
     float *pS = tiles;                                                          // [row][step][state], before pB
     float *pDU = tiles + 2 * kRNT;
     float *pDD = tiles + 2 * kRNT + kRTN;
@@ -227,8 +232,8 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(const ScanParams p,
                 const float ds = dsv4[e], dt = dtv4[e], Bv = Bs[t][n];
                 const float hprev = t > 0 ? H[t - 1] : hs;
                 const float gn = fmaf(ds, Cs[t][n], G);
-                pC[t][r][n] = ds * H[t];
-                pB[t][r][n] = gn * duv4[e];
+                pC[trs(t, r, n)] = ds * H[t];
+                pB[trs(t, r, n)] = gn * duv4[e];
                 pDU[rts(r, t, n)] = gn * dt * Bv;
                 pDD[rts(r, t, n)] = gn * fmaf(Bv, uuv4[e], hprev * Av[t] * Areal);
                 dA_acc = fmaf(gn * hprev, Av[t] * dt, dA_acc);
@@ -253,8 +258,8 @@ __global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(const ScanParams p,
                 float sb = 0.f, sc = 0.f;
 #pragma unroll
                 for (int rr = 0; rr < kRows; ++rr) {
-                    sb += pB[tt][rr][nn];
-                    sc += pC[tt][rr][nn];
+                    sb += pB[trs(tt, rr, nn)];
+                    sc += pC[trs(tt, rr, nn)];
                 }
                 atomicAdd(q.dB + (b * dstate + nn) * L + ts, sb);
                 atomicAdd(q.dC + (b * dstate + nn) * L + ts, sc);
