@@ -7,10 +7,22 @@
 #include <cstring>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "launch.h"
 #include "mambascan.h"
 
 namespace {
+
+// An NVTX range named after the entry point for the duration of the call, so
+// that profilers (ncu --nvtx, nsys) can attribute the launches; without a
+// profiler attached the push and pop return at once.
+struct CallRange {
+    explicit CallRange(const char *name) { nvtxRangePushA(name); }
+    ~CallRange() { nvtxRangePop(); }
+    CallRange(const CallRange &) = delete;
+    CallRange &operator=(const CallRange &) = delete;
+};
 
 thread_local char g_last_error[512] = "";
 
@@ -240,6 +252,7 @@ ms_status mamba_scan_workspace_size(const ms_scan_args *args, size_t *bytes) {
 
 ms_status mamba_scan_fwd(const ms_scan_args *args, void *workspace, size_t workspace_bytes,
                          void *stream) {
+    const CallRange range("mamba_scan_fwd");
     ms_status st = check_scan(args);
     if (st != MS_OK) return st;
     int sms = 0;
@@ -283,6 +296,7 @@ ms_status mamba_scan_plan_query(const ms_scan_args *args, ms_scan_plan *plan) {
 
 ms_status mamba_scan_fwd_with_plan(const ms_scan_args *args, const ms_scan_plan *plan, void *workspace,
                                    size_t workspace_bytes, void *stream) {
+    const CallRange range("mamba_scan_fwd_with_plan");
     if (!plan) return invalid("plan is NULL");
     ms_status st = check_scan(args);
     if (st != MS_OK) return st;
@@ -297,6 +311,7 @@ ms_status mamba_scan_fwd_with_plan(const ms_scan_args *args, const ms_scan_plan 
 }
 
 ms_status mamba_state_update(const ms_update_args *a, void *stream) {
+    const CallRange range("mamba_state_update");
     ms::UpdateParams p;
     const ms_status st = update_params(a, &p);
     if (st != MS_OK) return st;
@@ -308,6 +323,7 @@ ms_status mamba_state_update(const ms_update_args *a, void *stream) {
 ms_status mamba_conv_state_update(const ms_update_args *a, const ms_conv1d_args *conv, void *conv_state,
                                   int64_t conv_state_batch_stride, int64_t conv_state_dim_stride,
                                   void *stream) {
+    const CallRange range("mamba_conv_state_update");
     ms::UpdateParams p;
     ms_status st = update_params(a, &p);
     if (st != MS_OK) return st;
@@ -334,6 +350,7 @@ ms_status mamba_conv_state_update(const ms_update_args *a, const ms_conv1d_args 
 
 ms_status mamba_conv_scan_fwd(const ms_scan_args *args, const ms_conv1d_args *conv, const ms_scan_plan *plan,
                               void *stream) {
+    const CallRange range("mamba_conv_scan_fwd");
     ms_status st = check_scan(args);
     if (st != MS_OK) return st;
     st = check_conv(conv);
@@ -369,6 +386,7 @@ ms_status mamba_conv_scan_fwd(const ms_scan_args *args, const ms_conv1d_args *co
 
 ms_status mamba_trap_scan_fwd(const ms_scan_args *args, const void *lambda_raw, int64_t lambda_batch_stride,
                               int64_t lambda_dim_stride, const ms_scan_plan *plan, void *stream) {
+    const CallRange range("mamba_trap_scan_fwd");
     ms_status st = check_scan(args);
     if (st != MS_OK) return st;
     if (!lambda_raw) return invalid("lambda_raw is required");
@@ -416,6 +434,7 @@ ms_status mamba_scan_bwd_workspace_size(const ms_scan_args *args, size_t *bytes)
 
 ms_status mamba_scan_bwd(const ms_scan_args *args, const ms_scan_bwd_args *g, void *workspace,
                          size_t workspace_bytes, void *stream) {
+    const CallRange range("mamba_scan_bwd");
     ms_status st = check_scan(args);
     if (st != MS_OK) return st;
     if (!g) return invalid("bwd is NULL");
@@ -471,6 +490,7 @@ ms_status mamba_scan_bwd(const ms_scan_args *args, const ms_scan_bwd_args *g, vo
 }
 
 ms_status mamba_ssd_fwd(const ms_ssd_args *a, void *workspace, size_t workspace_bytes, void *stream) {
+    const CallRange range("mamba_ssd_fwd");
     if (!a) return invalid("args is NULL");
     if (a->batch <= 0 || a->seqlen <= 0 || a->nheads <= 0 || a->ngroups <= 0)
         return invalid("batch, seqlen, nheads and ngroups must be positive");

@@ -22,6 +22,8 @@
 
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "launch.h"
 #include "mambascan.h"
 
@@ -69,7 +71,7 @@ ms_status device_setup(void **scratch, int *sms) {
 
 }  // namespace
 
-extern "C" ms_status mamba_scan_fwd_noalloc(const ms_scan_args *args, void *stream) {
+static ms_status noalloc_call(const ms_scan_args *args, void *stream) {
     // Validate exactly as mamba_scan_fwd does (the message, if any, is already recorded).
     size_t need = 0;
     ms_status st = mamba_scan_workspace_size(args, &need);
@@ -106,4 +108,11 @@ extern "C" ms_status mamba_scan_fwd_noalloc(const ms_scan_args *args, void *stre
     const cudaError_t e = ms::launch_scan(p, plan, args->in_dtype, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(MS_ERR_CUDA, "scan kernel launch: %s", cudaGetErrorString(e));
     return MS_OK;
+}
+
+extern "C" ms_status mamba_scan_fwd_noalloc(const ms_scan_args *args, void *stream) {
+    nvtxRangePushA("mamba_scan_fwd_noalloc");
+    const ms_status st = noalloc_call(args, stream);
+    nvtxRangePop();
+    return st;
 }

@@ -486,7 +486,7 @@ scan_kernel(const ScanParams p) {
                 float2 z2[kK];
                 lds_pair<T>(xrow + 2 * R * ROWB, ROWB, z2);
 #pragma unroll
-                for (int i = 0; i < kK; ++i) y2[i] = mul2(y2[i], silu2(z2[i]));
+                for (int i = 0; i < kK; ++i) y2[i] = mul2(y2[i], silu2_out<T>(z2[i]));
             }
             if (count > 0) {
                 if (okA) store_row<T>(static_cast<T *>(p.y) + b * p.y_sb + dA * p.y_sd + tl, y2, false, count, VEC);
