@@ -61,6 +61,22 @@ constexpr uint32_t kHAtom = kP * 128;
 constexpr uint32_t kOffStep = kOffH + 2 * kHAtom;
 constexpr uint32_t kOffAbort = kOffStep + 2 * kQ * 10;
 constexpr uint32_t kOffBar = kOffAbort + 16;
+// mbarriers and their phases (chunk c completes phase c of a single barrier, or
+// phase c / 2 of barrier c % 2 of a pair; waits use that parity):
+//   full[c%2]   TMA bytes of stage c landed          <- producer expect_tx + TMA
+//   empty[c%2]  stage c no longer read                <- 16 epilogue warps after y(c)
+//   gfull[c%2]  G(c) in TMEM buffer c%2               <- tcgen05.commit
+//   pready      M'(c), Xt(c) written (phase c)        <- 16 epilogue warps
+//   sfull/yfull S(c) / Yd(c) done (phase c)           <- tcgen05.commit
+//   hready      H_{c-1} in its tile (phase c; phase 0 is the initial state)
+//   yfree       Yd/Yo of chunk c read (phase c)       <- 16 epilogue warps
+//   step[c%2]   step data of chunk c written           <- 32 producer lanes
+// No waiter can fall two phases behind: every barrier's next phase needs an
+// event that itself follows the wait (e.g. gfull[c%2] for chunk c + 2 needs
+// pready(c + 1), which follows the epilogue's wait on gfull for chunk c + 1;
+// full[c%2] for chunk c + 2 needs empty(c), which follows the waits on
+// full[c%2] for chunk c; hready phase c + 1 needs S(c), issued after the
+// issuer's wait on hready phase c).
 enum Bar { kFull0, kFull1, kEmpty0, kEmpty1, kGFull0, kGFull1, kPReady, kSFull, kYFull, kHReady, kYFree, kDrain,
            kStep0, kStep1, kNumBars };
 constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
