@@ -59,6 +59,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-seconds", type=float, default=60.0,
+                    help="--impl reference: seconds of oracle work for the whole warm-up + timed run")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU-baseline budget (seconds of oracle work on rank 0)")
     ap.add_argument("--prologue-steps", type=int, default=200,
@@ -273,9 +275,9 @@ def run_reference(args, dist: Dist):
     inp = make_scan_inputs(w)
     threads = oracle.max_threads()
     total_rows = w.batch * w.dim
-    # size each step so the whole warm-up + timed run takes about a minute
-    rate, _, _, _ = cpu_rate(w, inp, 1.0, rows_cap=4096)
-    per_step_budget = 60.0 / max(1, args.steps + args.warmup)
+    # size each step so the whole warm-up + timed run takes about --ref-seconds
+    rate, _, _, _ = cpu_rate(w, inp, min(1.0, args.ref_seconds), rows_cap=4096)
+    per_step_budget = args.ref_seconds / max(1, args.steps + args.warmup)
     n = int(max(1, min(total_rows, per_step_budget * rate / (w.seqlen * w.dstate))))
     g = np.random.default_rng(777)
     samples = [np.sort(g.choice(total_rows, n, replace=False)) for _ in range(4)]
