@@ -161,3 +161,50 @@ def test_ssd_rejects_unsupported_arguments():
         ms.ssd_fwd(dev["x"], dev["dt"], dev["A"], torch.cat([dev["B"]] * 4, dim=2)[:, :, :3].contiguous(),
                    torch.cat([dev["C"]] * 4, dim=2)[:, :, :3].contiguous())
     assert ei.value.status == 1
+
+
+def test_ssd_one_group_per_head():
+    """ngroups = nheads: every head reads its own B and C."""
+    inp = make_ssd_inputs(SMALL, batch=2, seqlen=333, nheads=4, ngroups=4, seed=3500)
+    y, hT = _run(_dev(inp))
+    yr, hr = _oracle(inp)
+    assert rel_err(y, yr) <= TOL["bf16"]
+    assert rel_err(hT, hr) <= TOL["bf16"]
+
+
+def test_ssd_mamba2_layer_from_initial_state():
+    """The full Mamba-2 layer continued from a seeded nonzero state; sampled
+    (batch, head) pairs against the oracle started from the same state."""
+    import torch
+    inp = make_ssd_inputs(LAYER, seed=LAYER.seed + 7)
+    h0 = make_ssd_state(LAYER.batch, LAYER.nheads, seed=3600)
+    y, hT = _run(_dev(inp), h0=torch.from_numpy(h0).cuda())
+    pairs = [3, 77, 200, LAYER.batch * LAYER.nheads - 1]
+    yr, hr = _oracle(inp, pairs=pairs, h0=h0.reshape(-1, 64, 128)[pairs])
+    for k, pr in enumerate(pairs):
+        b, h = divmod(pr, LAYER.nheads)
+        assert rel_err(y[b, :, h, :], yr[k]) <= TOL["bf16"], pr
+        assert rel_err(hT[b, h], hr[k]) <= TOL["bf16"], pr
+
+
+def test_ssd_batch_slices():
+    """x, dt, B, C, z and y as every other batch entry of larger tensors
+    (batch strides twice the dense ones)."""
+    import torch
+    ms = _ms()
+    inp = make_ssd_inputs(SMALL, batch=2, seqlen=150, nheads=2, seed=3700)
+    dev = _dev(inp)
+    big = {}
+    for k in ("x", "dt", "B", "C", "z"):
+        t = dev[k]
+        b2 = torch.zeros((4,) + tuple(t.shape[1:]), dtype=t.dtype, device="cuda")
+        b2[0::2] = t
+        big[k] = b2[0::2]
+    ybig = torch.zeros((4,) + tuple(dev["x"].shape[1:]), dtype=torch.bfloat16, device="cuda")
+    y_out = ybig[0::2]
+    _, hT = ms.ssd_fwd(big["x"], big["dt"], dev["A"], big["B"], big["C"], D=dev["D"], z=big["z"],
+                       dt_bias=dev["dt_bias"], out=y_out)
+    yr, hr = _oracle(inp)
+    assert rel_err(to_host64(y_out), yr) <= TOL["bf16"]
+    assert rel_err(to_host64(hT), hr) <= TOL["bf16"]
+    assert float(ybig[1::2].abs().max()) == 0.0
