@@ -3,8 +3,12 @@
 
 One step = one selective-scan forward pass (softplus, discretisation, scan,
 readout, D skip, SiLU gate, final state) over one batch of the workload,
-launched through the C ABI. Default workload: the Mamba-130M-shaped layer
-(batch 8, d_inner 1536, N 16, L 2048, bf16 inputs, fp32 state).
+launched through the C ABI. Default workload: the long-context layer (batch 1,
+d_inner 5120, N 16, L 131072, bf16 inputs, fp32 state), the largest
+single-GPU configuration; the other layer shapes (Mamba-130M- and
+Mamba-1.4B-shaped) are timed as legs of the same run, each with its own
+roofline, beside the decode step, the convolution prologue, the trapezoidal
+rule, the backward pass and the Mamba-2 SSD forward.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --impl reference ...   (the fp64 CPU oracle, timed on host cores)
@@ -53,11 +57,16 @@ FP32_PER_CLK = 128
 def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10000)
-    ap.add_argument("--warmup", type=int, default=50)
-    ap.add_argument("--workload", default="mamba130m_layer", choices=sorted(SCAN_WORKLOADS))
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="long_context_131k", choices=sorted(SCAN_WORKLOADS))
+    ap.add_argument("--leg-workloads", default="mamba130m_layer,mamba1p4b_layer",
+                    help="other scan workloads timed as legs (comma separated; empty: none)")
+    ap.add_argument("--leg-steps", type=int, default=50, help="timed steps of each scan-workload leg")
+    ap.add_argument("--side-workload", default="mamba130m_layer", choices=sorted(SCAN_WORKLOADS),
+                    help="workload of the convolution-prologue, trapezoidal and backward legs")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=60.0,
                     help="--impl reference: seconds of oracle work for the whole warm-up + timed run")
@@ -259,8 +268,7 @@ def _oracle_kw(inp):
 def workload_config(w, extra=None):
     cfg = {"workload": w.name, "batch": w.batch, "d_inner": w.dim, "d_state": w.dstate,
            "seq_len": w.seqlen, "in_dtype": w.dtype, "state_dtype": "f32", "gate": w.has_z,
-           "l2": f"inputs rotated over {ROTATE} resident copies (> L2 of 126 MB)",
-           "parallelism": "replicas (independent batch per GPU)"}
+           "l2": l2_note(w), "parallelism": "replicas (independent batch per GPU)"}
     if extra:
         cfg.update(extra)
     return cfg
@@ -295,13 +303,220 @@ def run_reference(args, dist: Dist):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic (seeded)", "config": workload_config(w),
+        "data": "synthetic (seeded)", "config": workload_config(w, {"l2": l2_note(w)}),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def rotate_count(w) -> int:
+    """Input sets cycled through so that every step reads inputs that are not
+    resident in L2: one set when a set alone is several times the L2."""
+    in_bytes = 4 if w.dtype == "f32" else 2
+    set_bytes = (3 if w.has_z else 2) * w.batch * w.dim * w.seqlen * in_bytes
+    return 1 if set_bytes > 4 * L2_BYTES else ROTATE
+
+
+def l2_note(w) -> str:
+    n = rotate_count(w)
+    return ("inputs larger than L2 (one set)" if n == 1 else
+            f"inputs rotated over {n} resident copies (> L2 of 126 MB)")
+
+
+class ScanSetup:
+    """Seeded inputs of one scan workload on the device, the C-ABI argument
+    structs of its rotating input sets, the workspace and the launch plan."""
+
+    def __init__(self, w, dev, rank, pin=False):
+        import torch
+        import selective_state_space_27_b200 as ms
+        self.w = w
+        self.in_bytes = 4 if w.dtype == "f32" else 2
+        self.tdt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+        self.inp = make_scan_inputs(w, seed=w.seed + 1000 * rank)
+
+        def host(a):
+            t = torch.from_numpy(np.ascontiguousarray(a))
+            return t.view(torch.bfloat16) if (a.dtype == np.uint16) else t
+
+        self.names = ["u", "delta", "B", "C"] + (["z"] if w.has_z else [])
+        src = {k: host(self.inp[k]) for k in self.names}
+        self.pinned = {k: v.pin_memory() for k, v in src.items()} if pin else None
+        self.params = {k: torch.from_numpy(self.inp[k]).to(dev) for k in ("A", "D", "delta_bias")}
+        self.rotate = rotate_count(w)
+        self.sets = [{k: v.to(dev) for k, v in (self.pinned or src).items()} for _ in range(self.rotate)]
+        self.y = torch.empty((w.batch, w.dim, w.seqlen), dtype=self.tdt, device=dev)
+        self.hT = torch.empty((w.batch, w.dim, w.dstate), dtype=torch.float32, device=dev)
+        self.args = [self.scan_args(st, self.y, self.hT) for st in self.sets]
+        self.plan = ms.scan_plan(self.args[0])
+        self.ws = torch.empty(max(ms.scan_workspace_size(self.args[0]), 256), dtype=torch.uint8, device=dev)
+        kind = {c: k for c, _, _, _, k in ms.scan_configs()}[self.plan.config]
+        self.kernel = (f"rec_kernel<{'bf16' if w.dtype == 'bf16' else 'f32'}, {self.plan.lanes}>" if kind == 1
+                       else "scan_kernel")
+        self.kernel_desc = (
+            f"{self.kernel} (sequential, warp-specialised, {self.plan.lanes} lanes per row, "
+            + (f"persistent schedule over {self.plan.ctas} CTAs)" if self.plan.ctas else "one CTA per block of rows)")
+            if kind == 1 else
+            f"scan_kernel (chunked, config {self.plan.config}, {self.plan.warps_per_cta} warps, "
+            f"{self.plan.segments} segments)")
+        self.launches_per_step = 2 if (kind == 0 and self.plan.segments > 1) else 1
+        self.counts = algorithmic_counts(w, self.in_bytes)
+        torch.cuda.synchronize()
+
+    def scan_args(self, st, y, hT):
+        import selective_state_space_27_b200 as ms
+        return ms.build_scan_args(st["u"], st["delta"], self.params["A"], st["B"], st["C"], y, D=self.params["D"],
+                                  z=st.get("z"), delta_bias=self.params["delta_bias"], final_state=hT)
+
+    def step(self, lib, i, stream, args=None):
+        import ctypes
+        import selective_state_space_27_b200 as ms
+        a = args if args is not None else self.args[i % self.rotate]
+        rc = lib.mamba_scan_fwd(ctypes.byref(a), self.ws.data_ptr(), self.ws.numel(), stream.cuda_stream)
+        if rc != 0:
+            raise ms.MambaScanError(rc, lib.mamba_last_error().decode())
+
+
+def time_steps(fn, n, stream):
+    """CUDA-event time (ms) of n calls of fn() on `stream`, synchronized on both sides."""
+    import torch
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(n):
+        fn(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def scan_roofline(setup, us, mufu, peaks):
+    """Roofline of one scan launch: the binding bound is the MUFU (one ex2 per
+    element + the softplus and gate transcendentals per (b, d, t)), against the
+    MUFU throughput measured on this device; HBM and FP32 fractions beside."""
+    c = setup.counts
+    t = us * 1e-6
+    fp32_peak = SMS_B200 * FP32_PER_CLK * peaks["sm_max_mhz"] * 1e6
+    t_bounds = {"hbm": c["bytes"] / (peaks["hbm_gbs"] * 1e9), "mufu": c["mufu"] / mufu["measured_per_s"],
+                "fp32": c["fp32"] / fp32_peak}
+    return {
+        "bound": "alu", "unit": "Tmufu/s", "achieved": c["mufu"] / t / 1e12, "peak": mufu["measured_per_s"] / 1e12,
+        "frac": c["mufu"] / t / mufu["measured_per_s"],
+        "traffic": NCU_TRAFFIC.get((setup.w.name, setup.kernel)),
+        "kernel": setup.kernel_desc,
+        "peak_note": (f"measured: ex2.approx throughput of this device ({mufu['measured_per_clk_per_sm']:.2f} per clk "
+                      f"per SM, mamba_probe_unit_throughput); nominal {SMS_B200} SMs x {MUFU_PER_CLK}/clk x "
+                      f"{peaks['sm_max_mhz']:.0f} MHz = {mufu['nominal_per_s'] / 1e12:.3f} T/s"),
+        "frac_of_nominal": c["mufu"] / t / mufu["nominal_per_s"],
+        "algorithmic_per_launch": c,
+        "hbm": {"achieved_gbs": c["bytes"] / t / 1e9, "peak_gbs": peaks["hbm_gbs"],
+                "frac": c["bytes"] / t / 1e9 / peaks["hbm_gbs"], "peak_source": peaks["source"]},
+        "bound_times_us": {k: v * 1e6 for k, v in t_bounds.items()},
+        "kernel_us": us,
+        "roofline_elem_per_s": c["elements"] / max(t_bounds.values()),
+    }
+
+
+def measure_mufu(peaks):
+    import selective_state_space_27_b200 as ms
+    per_s, per_clk = ms.probe_unit_throughput("ex2")
+    tanh_s, _ = ms.probe_unit_throughput("tanh")
+    return {"measured_per_s": per_s, "measured_per_clk_per_sm": per_clk, "tanh_per_s": tanh_s,
+            "nominal_per_s": SMS_B200 * MUFU_PER_CLK * peaks["sm_max_mhz"] * 1e6}
+
+
+def run_scan_leg(args, dist, dev, w, mufu, peaks, lib, stream):
+    """Time another scan workload through mamba_scan_fwd: its own plan,
+    rotating input sets when they fit in L2, and roofline."""
+    setup = ScanSetup(w, dev, dist.rank)
+    for i in range(max(3, args.warmup)):
+        setup.step(lib, i, stream)
+    n = args.leg_steps
+    ms_ = dist.max(time_steps(lambda i: setup.step(lib, i, stream), n, stream), dev)
+    us = ms_ * 1e3 / n
+    out = {"workload": w.name, "config": workload_config(w, {"l2": l2_note(w)}), "steps": n, "us_per_step": us,
+           "value": dist.world * setup.counts["elements"] / (us * 1e-6), "unit": UNIT,
+           "roofline": scan_roofline(setup, us, mufu, peaks), "gpu_launches": n * setup.launches_per_step}
+    del setup
+    return out
+
+
+def run_e2e(args, dist, dev, setup, lib, stream):
+    """The same step end to end through the C ABI from pinned host buffers:
+    every step copies its inputs host -> device and y and the final state
+    device -> host. Steps are pipelined over two device buffer sets on three
+    streams (copy in, compute, copy out), so the copy-in of step i+1, the
+    scan of step i and the copy-out of step i-1 overlap; the timed region runs
+    from the first copy-in to the last copy-out."""
+    import torch
+    w = setup.w
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    bufs = [setup.sets[0], {k: torch.empty_like(v) for k, v in setup.sets[0].items()}]
+    ys = [setup.y, torch.empty_like(setup.y)]
+    hs = [setup.hT, torch.empty_like(setup.hT)]
+    argl = [setup.scan_args(bufs[j], ys[j], hs[j]) for j in range(2)]
+    y_host = torch.empty(setup.y.shape, dtype=setup.tdt).pin_memory()
+    h_host = torch.empty(setup.hT.shape, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in setup.pinned.values())
+    d2h = y_host.numel() * y_host.element_size() + h_host.numel() * 4
+
+    def run(n):
+        ev_in = [torch.cuda.Event() for _ in range(n)]
+        ev_cmp = [torch.cuda.Event() for _ in range(n)]
+        ev_out = [torch.cuda.Event() for _ in range(n)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(s_in)
+        for i in range(n):
+            j = i % 2
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_cmp[i - 2])      # the scan of step i-2 has read buffer j
+                for k, v in setup.pinned.items():
+                    bufs[j][k].copy_(v, non_blocking=True)
+                ev_in[i].record(s_in)
+            stream.wait_event(ev_in[i])
+            if i >= 2:
+                stream.wait_event(ev_out[i - 2])        # step i-2's outputs have left buffer j
+            setup.step(lib, 0, stream, args=argl[j])
+            ev_cmp[i].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_cmp[i])
+                y_host.copy_(ys[j], non_blocking=True)
+                h_host.copy_(hs[j], non_blocking=True)
+                ev_out[i].record(s_out)
+        t1.record(s_out)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1)
+
+    run(2)
+    dist.barrier()
+    n = args.e2e_steps
+    e2e_ms = dist.max(run(n), dev)
+    return {"value": setup.counts["elements"] * n * dist.world / (e2e_ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / n,
+            "pipeline": "copy-in, scan and copy-out of consecutive steps overlap (3 streams, 2 buffer sets)"}
+
+
+def cpu_single_core(w_name, seconds):
+    """The oracle on one host core over a seeded sample of rows of `w_name`."""
+    import oracle
+    w = SCAN_WORKLOADS[w_name]
+    inp = make_scan_inputs(w)
+    total_rows = w.batch * w.dim
+    g = np.random.default_rng(4321)
+    t = time.perf_counter()
+    oracle.scan(**_oracle_kw(inp), rows=np.sort(g.choice(total_rows, 4, replace=False)), threads=1)
+    per_row = (time.perf_counter() - t) / 4
+    n = int(min(total_rows, max(4, seconds / max(per_row, 1e-9))))
+    rows = np.sort(g.choice(total_rows, n, replace=False))
+    t = time.perf_counter()
+    oracle.scan(**_oracle_kw(inp), rows=rows, threads=1)
+    dt = time.perf_counter() - t
+    return {"workload": w_name, "value": n * w.seqlen * w.dstate / dt, "unit": UNIT, "cores": 1,
+            "sample": f"{n} of {total_rows} rows (seeded), full L={w.seqlen}, N={w.dstate}", "seconds": dt}
 
 
 def run_ours(args, dist: Dist):
@@ -314,47 +529,14 @@ def run_ours(args, dist: Dist):
     torch.cuda.set_device(dev)
     dist.init("nccl")
     w = SCAN_WORKLOADS[args.workload]
-    in_bytes = 4 if w.dtype == "f32" else 2
-    tdt = torch.float32 if w.dtype == "f32" else torch.bfloat16
-
-    inp = make_scan_inputs(w, seed=w.seed + 1000 * dist.rank)
-
-    def host(a):
-        t = torch.from_numpy(np.ascontiguousarray(a))
-        return t.view(torch.bfloat16) if (a.dtype == np.uint16) else t
-
-    names = ["u", "delta", "B", "C"] + (["z"] if w.has_z else [])
-    pinned = {k: host(inp[k]).pin_memory() for k in names}
-    params = {k: torch.from_numpy(inp[k]).to(dev) for k in ("A", "D", "delta_bias")}
-    sets = [{k: v.to(dev, non_blocking=True) for k, v in pinned.items()} for _ in range(ROTATE)]
-    y = torch.empty((w.batch, w.dim, w.seqlen), dtype=tdt, device=dev)
-    hT = torch.empty((w.batch, w.dim, w.dstate), dtype=torch.float32, device=dev)
-    torch.cuda.synchronize()
-
-    stream = torch.cuda.current_stream()
-    args_list = [ms.build_scan_args(s["u"], s["delta"], params["A"], s["B"], s["C"], y,
-                                    D=params["D"], z=s.get("z"), delta_bias=params["delta_bias"],
-                                    final_state=hT) for s in sets]
-    ws_bytes = ms.scan_workspace_size(args_list[0])
-    plan = ms.scan_plan(args_list[0])
-    kind = {c: k for c, _, _, _, k in ms.scan_configs()}[plan.config]
-    kernel_name = (f"rec_kernel<{'bf16' if w.dtype == 'bf16' else 'f32'}, {plan.lanes}> (sequential, "
-                   f"warp-specialised, {plan.lanes} lanes per row)" if kind == 1 else
-                   f"scan_kernel (chunked, config {plan.config}, {plan.warps_per_cta} warps, "
-                   f"{plan.segments} segments)")
-    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    peaks = load_peaks()
+    mufu = measure_mufu(peaks)
     lib = ms.load_library()
-    import ctypes
-    launches_per_step = 2 if ws_bytes else 1
-
-    def step(i):
-        rc = lib.mamba_scan_fwd(ctypes.byref(args_list[i % ROTATE]), ws.data_ptr(), ws.numel(),
-                                stream.cuda_stream)
-        if rc != 0:
-            raise ms.MambaScanError(rc, lib.mamba_last_error().decode())
+    stream = torch.cuda.current_stream()
+    setup = ScanSetup(w, dev, dist.rank, pin=args.e2e_steps > 0)
 
     for i in range(args.warmup):
-        step(i)
+        setup.step(lib, i, stream)
     torch.cuda.synchronize()
 
     sampler = ClockSampler(physical_gpu(dist.local_rank))
@@ -366,7 +548,7 @@ def run_ours(args, dist: Dist):
     sampler.mark_begin()
     ev[0].record(stream)
     for i in range(args.steps):
-        step(i)
+        setup.step(lib, i, stream)
     ev[1].record(stream)
     torch.cuda.synchronize()
     sampler.mark_end()
@@ -374,86 +556,54 @@ def run_ours(args, dist: Dist):
     elapsed_ms = ev[0].elapsed_time(ev[1])
     clocks = sampler.stop() if dist.rank == 0 else None
     elapsed_ms = dist.max(elapsed_ms, dev)
+    if setup.plan.ctas and ms.scan_status(setup.ws) != 0:
+        raise SystemExit("bench.py: a persistent scan reported a failed carry wait")
 
-    counts = algorithmic_counts(w, in_bytes)
+    counts = setup.counts
     total_elems = counts["elements"] * args.steps * dist.world
     value = total_elems / (elapsed_ms / 1e3)
     ms_per_step = elapsed_ms / args.steps
+    roofline = scan_roofline(setup, ms_per_step * 1e3, mufu, peaks)
 
-    # ---- end to end through the C ABI with pinned host buffers ----------------
-    e2e = None
-    if args.e2e_steps > 0:
-        y_host = torch.empty(y.shape, dtype=tdt).pin_memory()
-        h_host = torch.empty(hT.shape, dtype=torch.float32).pin_memory()
-        dset = sets[0]
-        h2d = sum(t.numel() * t.element_size() for t in pinned.values())
-        d2h = y_host.numel() * y_host.element_size() + h_host.numel() * 4
+    e2e = run_e2e(args, dist, dev, setup, lib, stream) if args.e2e_steps > 0 else None
+    launches = args.steps * setup.launches_per_step
+    del setup
+    torch.cuda.empty_cache()
 
-        def e2e_step():
-            for k, v in pinned.items():
-                dset[k].copy_(v, non_blocking=True)
-            step(0)
-            y_host.copy_(y, non_blocking=True)
-            h_host.copy_(hT, non_blocking=True)
-
-        for _ in range(3):
-            e2e_step()
-        torch.cuda.synchronize()
-        dist.barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms = dist.max(e0.elapsed_time(e1), dev)
-        e2e = {"value": counts["elements"] * args.e2e_steps * dist.world / (e2e_ms / 1e3), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": e2e_ms / args.e2e_steps}
-
-    # ---- roofline of the scan kernel (the only kernel of a step) --------------
-    peaks = load_peaks()
-    sm_mhz = peaks["sm_max_mhz"]
-    mufu_peak = SMS_B200 * MUFU_PER_CLK * sm_mhz * 1e6          # ex2-class results / s
-    fp32_peak = SMS_B200 * FP32_PER_CLK * sm_mhz * 1e6
-    t_kernel = ms_per_step / 1e3   # every launch of a step belongs to the scan
-    achieved_mufu = counts["mufu"] / t_kernel
-    t_bounds = {"hbm": counts["bytes"] / (peaks["hbm_gbs"] * 1e9), "mufu": counts["mufu"] / mufu_peak,
-                "fp32": counts["fp32"] / fp32_peak}
-    roofline = {
-        "bound": "alu", "unit": "Tmufu/s", "achieved": achieved_mufu / 1e12, "peak": mufu_peak / 1e12,
-        "frac": achieved_mufu / mufu_peak, "traffic": NCU_TRAFFIC.get((w.name, kernel_name.split(" (")[0])),
-        "kernel": kernel_name,
-        "peak_note": f"MUFU: {SMS_B200} SMs x {MUFU_PER_CLK}/clk x {sm_mhz:.0f} MHz (nominal max clock)",
-        "algorithmic_per_launch": counts,
-        "hbm": {"achieved_gbs": counts["bytes"] / t_kernel / 1e9, "peak_gbs": peaks["hbm_gbs"],
-                "frac": counts["bytes"] / t_kernel / 1e9 / peaks["hbm_gbs"], "peak_source": peaks["source"]},
-        "bound_times_us": {k: v * 1e6 for k, v in t_bounds.items()},
-        "kernel_us": t_kernel * 1e6,
-        "roofline_elem_per_s": counts["elements"] / max(t_bounds.values()),
-    }
+    legs = {}
+    for name in [s for s in args.leg_workloads.split(",") if s]:
+        if name != w.name:
+            legs[name] = run_scan_leg(args, dist, dev, SCAN_WORKLOADS[name], mufu, peaks, lib, stream)
+            torch.cuda.empty_cache()
 
     decode = run_decode(args, dist, dev) if args.decode_steps > 0 else None
-    prologue = (run_prologue(args, dist, dev, w, sets, params, y, hT, counts, mufu_peak)
+    side = None
+    if args.prologue_steps > 0 or args.trap_steps > 0 or args.bwd_steps > 0:
+        side = ScanSetup(SCAN_WORKLOADS[args.side_workload], dev, dist.rank)
+    mufu_peak = mufu["measured_per_s"]
+    prologue = (run_prologue(args, dist, dev, side.w, side.sets, side.params, side.y, side.hT, side.counts, mufu_peak)
                 if args.prologue_steps > 0 else None)
-    trap = run_trap(args, dist, dev, w, sets, params, y, hT, counts, mufu_peak) if args.trap_steps > 0 else None
-    bwd = run_bwd(args, dist, dev, w, sets, params, counts, mufu_peak) if args.bwd_steps > 0 else None
+    trap = (run_trap(args, dist, dev, side.w, side.sets, side.params, side.y, side.hT, side.counts, mufu_peak)
+            if args.trap_steps > 0 else None)
+    bwd = run_bwd(args, dist, dev, side.w, side.sets, side.params, side.counts, mufu_peak) if args.bwd_steps > 0 else None
+    del side
+    torch.cuda.empty_cache()
     ssd = run_ssd(args, dist, dev, peaks) if args.ssd_steps > 0 else None
 
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
-        rate, threads, sample, secs = cpu_rate(w, inp, args.cpu_seconds)
+        rate, threads, sample, secs = cpu_rate(w, make_scan_inputs(w), args.cpu_seconds)
         cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample,
-               "seconds": secs}
+               "seconds": secs, "single_core": cpu_single_core("mamba130m_layer", min(5.0, args.cpu_seconds))}
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": dist.world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-        "data": "synthetic (seeded)", "config": workload_config(w, {"global_batch": w.batch * dist.world}),
-        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "decode": decode, "conv_prologue": prologue,
-        "trapezoidal": trap, "backward": bwd, "ssd": ssd,
-        "gpu_launches": args.steps * launches_per_step, "clocks": clocks,
+        "data": "synthetic (seeded)", "config": workload_config(w, {"l2": l2_note(w)}),
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "mufu_probe": mufu, "scan_legs": legs,
+        "decode": decode, "conv_prologue": prologue, "trapezoidal": trap, "backward": bwd, "ssd": ssd,
+        "gpu_launches": launches, "clocks": clocks,
     }
     if dist.rank == 0:
         print(json.dumps(line), flush=True)

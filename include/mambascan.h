@@ -63,7 +63,7 @@
 extern "C" {
 #endif
 
-#define MAMBASCAN_ABI_VERSION 1
+#define MAMBASCAN_ABI_VERSION 2
 /* Largest state size N supported by the kernels. */
 #define MS_MAX_DSTATE 16
 
@@ -73,7 +73,7 @@ typedef enum ms_status {
     MS_ERR_UNSUPPORTED = 2,  /* valid but outside what the kernels support (dstate>16)   */
     MS_ERR_ALIGNMENT = 3,    /* a pointer is not aligned to its element size             */
     MS_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed              */
-    MS_ERR_TIMEOUT = 5,      /* a bounded device wait gave up (SSD status word only)       */
+    MS_ERR_TIMEOUT = 5,      /* a bounded device wait gave up (reported in a status word)  */
     MS_ERR_WORKSPACE = 6     /* workspace missing or smaller than the size asked for      */
 } ms_status;
 
@@ -159,7 +159,9 @@ int mamba_abi_version(void);
 
 /*
  * Bytes of device workspace that mamba_scan_fwd needs for these arguments
- * (written to *bytes; 0 when the sequence is not split into segments).
+ * (written to *bytes; 0 when the plan neither splits the sequence into
+ * segments nor uses the persistent schedule described at
+ * mamba_scan_fwd_with_plan).
  * Validates the arguments like mamba_scan_fwd, without touching the device
  * memory they point to. The caller allocates the workspace (256-byte aligned)
  * and may reuse it across calls on one stream.
@@ -197,7 +199,11 @@ typedef struct ms_scan_plan {
     int32_t segments;        /* pieces the sequence of every row is cut into (>= 1)               */
     int32_t lanes;           /* out: chunked: lanes per row pair; sequential: lanes per row        */
     int64_t segment_len;     /* out: time steps per segment                                      */
-    uint64_t workspace_bytes;/* out: workspace the plan needs (0 when segments == 1)              */
+    uint64_t workspace_bytes;/* out: workspace the plan needs                                    */
+    int32_t ctas;            /* sequential kernels: 0 = one CTA per unit of rows (batch entry x
+                                block of rows); > 0 = persistent schedule over this many CTAs
+                                (below); chunked kernels: 0                                      */
+    int32_t reserved;        /* must be 0                                                        */
 } ms_scan_plan;
 
 /* Number of compiled scan kernel configurations. */
@@ -227,6 +233,10 @@ ms_status mamba_scan_config_kind(int config, int *kind);
 /* The plan mamba_scan_fwd would run for these arguments (validates like it). */
 ms_status mamba_scan_plan_query(const ms_scan_args *args, ms_scan_plan *plan);
 
+/* Bytes of workspace (*bytes) that mamba_scan_fwd_with_plan needs to run
+ * `plan` on these arguments; MS_ERR_UNSUPPORTED if the plan cannot run them. */
+ms_status mamba_scan_plan_workspace_size(const ms_scan_args *args, const ms_scan_plan *plan, size_t *bytes);
+
 /*
  * mamba_scan_fwd with the launch plan fixed by the caller. The plan is
  * checked (index, CTA size, shared memory, segments <= number of chunks, and
@@ -234,6 +244,22 @@ ms_status mamba_scan_plan_query(const ms_scan_args *args, ms_scan_plan *plan);
  * dstate 16, and kernels with more than one state per pass need 16-byte
  * aligned rows); an unusable plan returns MS_ERR_UNSUPPORTED and launches
  * nothing. Same results as mamba_scan_fwd up to float32 rounding order.
+ *
+ * Persistent schedule (sequential kernels, plan->ctas > 0). The rows are cut
+ * into units (one batch entry x the CTA's block of rows) and every unit's
+ * sequence into chunks of 16 steps; the chunks of all units, unit after
+ * unit, are divided into plan->ctas equal ranges, one per CTA, so every SM
+ * does the same share of the recurrence whatever the number of rows. A unit
+ * whose chunks fall into two ranges is started by one CTA, which leaves its
+ * state in the workspace, and continued by the next CTA from that state (the
+ * recurrence itself is unchanged: no step is computed twice). plan->ctas may
+ * not exceed the number of units nor the CTAs the device can hold at once;
+ * the launch is cooperative, so all of them run concurrently. The workspace
+ * (mamba_scan_plan_workspace_size) starts with a status word, an int32 that
+ * the call clears and the kernel sets to MS_ERR_TIMEOUT if a CTA gave up
+ * waiting (about 4 s) for the state it continues from (the outputs are then
+ * wrong); flags and states follow. The automatic plan uses this schedule when
+ * it balances the SMs better than one CTA per unit.
  */
 ms_status mamba_scan_fwd_with_plan(const ms_scan_args *args, const ms_scan_plan *plan, void *workspace,
                                    size_t workspace_bytes, void *stream);
@@ -399,6 +425,16 @@ typedef struct ms_ssd_args {
     const float *dt_bias;
     const float *initial_state;
     float *final_state;
+
+    /* Limit of each of the kernel's internal pipeline waits, in microseconds;
+     * 0 = the default of about one second. */
+    uint32_t wait_limit_us;
+    /* Fault-injection hook for tests of the timeout path: k > 0 makes the
+     * kernel withhold the loads of block k - 1 (of every (batch, head)), so
+     * the wait for them runs out and the status word reports MS_ERR_TIMEOUT;
+     * no load or product of that block is ever issued, so nothing is left in
+     * flight. 0 = normal operation. */
+    int32_t withhold_block;
 } ms_ssd_args;
 
 /* Device workspace of mamba_ssd_fwd: a status word (int32 at offset 0). */
@@ -424,6 +460,24 @@ typedef struct ms_ssd_args {
  */
 ms_status mamba_ssd_fwd(const ms_ssd_args *args, void *workspace, size_t workspace_bytes, void *stream);
 
+/* ---- Measurement helper -----------------------------------------------------
+ * Measured throughput of one arithmetic unit on the current device, the
+ * denominators of the scan's roofline (the pages bound the selective scan by
+ * the non-tensor units: "Mamba-2 e State Space Duality (SSD)", section "O
+ * gargalo de hardware no scan associativo do Mamba-1"). unit: 0 = ex2.approx
+ * (the MUFU exponential every element of the scan takes), 1 = tanh.approx
+ * (MUFU), 2 = float32 FMA, 3 = packed f32x2 FMA (two results per
+ * instruction). Every SM runs 32 warps of 16 independent dependency chains.
+ * Writes results per second (*ops_per_s, from CUDA events around one launch
+ * after a warm-up launch) and per clock per SM (*ops_per_clk_per_sm, from the
+ * SM cycle counter). `scratch` is 256 bytes of caller-owned device memory,
+ * 256-byte aligned (overwritten). Unlike the compute entry points this call is
+ * synchronous: it returns after synchronizing `stream`. Errors:
+ * MS_ERR_INVALID_ARG (unit outside 0..3, NULL scratch or outputs),
+ * MS_ERR_ALIGNMENT (misaligned scratch), MS_ERR_CUDA. */
+ms_status mamba_probe_unit_throughput(int unit, void *scratch, double *ops_per_s, double *ops_per_clk_per_sm,
+                                      void *stream);
+
 /* Size of the device array behind mamba_scan_fwd_noalloc (8 MiB per GPU). */
 #define MS_NOALLOC_SCRATCH_BYTES (8u << 20)
 
@@ -435,20 +489,22 @@ ms_status mamba_ssd_fwd(const ms_ssd_args *args, void *workspace, size_t workspa
  * the whole device. (The pages this library follows have no counterpart; this
  * entry point exists for those callers.)
  *
- * The multi-block carry workspace that mamba_scan_fwd takes from its caller
- * lives here in a fixed device array of MS_NOALLOC_SCRATCH_BYTES, which every
- * GPU that loads the library holds until the process exits. The call
- * allocates nothing. Inputs and outputs are the caller's, exactly as for
+ * The workspace that mamba_scan_fwd takes from its caller (the multi-block
+ * carry, or the persistent schedule's status word, flags and handed-over
+ * states) lives here in a fixed device array of MS_NOALLOC_SCRATCH_BYTES,
+ * which every GPU that loads the library holds until the process exits. The
+ * call allocates nothing. Inputs and outputs are the caller's, exactly as for
  * mamba_scan_fwd.
  *  - The first call on a device looks up the array's device address on that
  *    (current) device; make that first call before any stream capture.
  *  - All calls on a device share the array and it keeps the last call's
- *    contents; every entry a call reads is written by that same call first,
- *    so no clearing is needed, but calls whose kernels overlap on the GPU
- *    (unordered streams) race on it and give wrong results.
- *  - Calls that would need more carry scratch than the array holds (batch *
- *    dim * segments * 128 bytes > MS_NOALLOC_SCRATCH_BYTES) are rejected with
- *    MS_ERR_WORKSPACE and launch nothing.
+ *    contents; the call itself clears (on the stream, before its kernel) the
+ *    part that must start at zero and writes every other entry before reading
+ *    it, so the caller clears nothing, but calls whose kernels overlap on the
+ *    GPU (unordered streams) race on it and give wrong results.
+ *  - Calls that would need more scratch than the array holds (the size
+ *    mamba_scan_workspace_size reports exceeds MS_NOALLOC_SCRATCH_BYTES) are
+ *    rejected with MS_ERR_WORKSPACE and launch nothing.
  * Errors: as mamba_scan_fwd.
  */
 ms_status mamba_scan_fwd_noalloc(const ms_scan_args *args, void *stream);

@@ -26,7 +26,7 @@ __all__ = [
     "load_library", "MambaScanError", "ScanArgs", "UpdateArgs", "ScanPlan", "MS_F32", "MS_BF16",
     "Conv1dArgs", "conv_scan_fwd", "conv_state_update", "build_conv_args", "trap_scan_fwd",
     "ScanBwdArgs", "scan_bwd", "SsdArgs", "build_ssd_args", "ssd_fwd", "ssd_check", "SSD_WORKSPACE_BYTES",
-    "MAX_DSTATE",
+    "MAX_DSTATE", "probe_unit_throughput", "PROBE_UNITS", "plan_workspace_size", "scan_status",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -105,6 +105,7 @@ class SsdArgs(ctypes.Structure):
         ("z", _vp), ("z_batch_stride", _i64), ("z_token_stride", _i64),
         ("y", _vp), ("y_batch_stride", _i64), ("y_token_stride", _i64),
         ("A", _vp), ("D", _vp), ("dt_bias", _vp), ("initial_state", _vp), ("final_state", _vp),
+        ("wait_limit_us", ctypes.c_uint32), ("withhold_block", _i32),
     ]
 
 
@@ -112,7 +113,7 @@ class ScanPlan(ctypes.Structure):
     """Mirror of ``ms_scan_plan``."""
     _fields_ = [
         ("config", _i32), ("warps_per_cta", _i32), ("segments", _i32), ("lanes", _i32),
-        ("segment_len", _i64), ("workspace_bytes", ctypes.c_uint64),
+        ("segment_len", _i64), ("workspace_bytes", ctypes.c_uint64), ("ctas", _i32), ("reserved", _i32),
     ]
 
 
@@ -169,12 +170,18 @@ def load_library():
         lib.mamba_scan_config_kind.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
         lib.mamba_scan_plan_query.restype = ctypes.c_int
         lib.mamba_scan_plan_query.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(ScanPlan)]
+        lib.mamba_scan_plan_workspace_size.restype = ctypes.c_int
+        lib.mamba_scan_plan_workspace_size.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(ScanPlan),
+                                                       ctypes.POINTER(ctypes.c_size_t)]
         lib.mamba_scan_fwd_with_plan.restype = ctypes.c_int
         lib.mamba_scan_fwd_with_plan.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(ScanPlan), _vp,
                                                  ctypes.c_size_t, _vp]
         lib.mamba_ssd_fwd.restype = ctypes.c_int
         lib.mamba_ssd_fwd.argtypes = [ctypes.POINTER(SsdArgs), _vp, ctypes.c_size_t, _vp]
-        if lib.mamba_abi_version() != 1:
+        lib.mamba_probe_unit_throughput.restype = ctypes.c_int
+        lib.mamba_probe_unit_throughput.argtypes = [ctypes.c_int, _vp, ctypes.POINTER(ctypes.c_double),
+                                                    ctypes.POINTER(ctypes.c_double), _vp]
+        if lib.mamba_abi_version() != 2:
             raise RuntimeError("libmambascan.so ABI version mismatch")
         _lib = lib
     return _lib
@@ -212,6 +219,14 @@ def _stream_ptr(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
     return stream.cuda_stream
+
+
+def _keep_until_done(t, stream):
+    """A scratch tensor allocated here on the current stream but used by a
+    launch on ``stream``: tell the caching allocator not to hand its memory to
+    other work before that stream has finished with it."""
+    if stream is not None:
+        t.record_stream(stream)
 
 
 def _need_cuda(name, t, dtype=None, ndim=None):
@@ -279,6 +294,21 @@ def scan_workspace_size(args: ScanArgs) -> int:
     return int(n.value)
 
 
+def plan_workspace_size(args: ScanArgs, plan: ScanPlan) -> int:
+    """Workspace bytes that ``plan`` needs for these arguments."""
+    n = ctypes.c_size_t(0)
+    _check(load_library().mamba_scan_plan_workspace_size(ctypes.byref(args), ctypes.byref(plan), ctypes.byref(n)))
+    return int(n.value)
+
+
+def scan_status(workspace) -> int:
+    """The status word a persistent-schedule scan leaves at the start of its
+    workspace (0, or MS_ERR_TIMEOUT = 5). Synchronizes the device."""
+    torch = _torch()
+    torch.cuda.synchronize(workspace.device)
+    return int(workspace[:4].view(torch.int32)[0].item())
+
+
 def scan_configs():
     """[(index, lanes, states_per_pass, max_warps, kind)] of the compiled scan
     kernels; kind 0 = chunked (lanes per row pair), 1 = sequential (lanes per
@@ -325,18 +355,20 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=
         if plan is None:
             need = scan_workspace_size(args)
         else:
-            # the workspace a fixed plan needs: rows * segments * 16 states * 2 floats
-            need = 0 if plan.segments <= 1 else 2 * u.shape[0] * u.shape[1] * plan.segments * 16 * 4
-        ws_ptr, ws_bytes = None, 0
+            need = plan_workspace_size(args, plan)
+        ws_ptr, ws_bytes, own_ws = None, 0, False
         if need:
             if workspace is None or workspace.numel() < need:
                 workspace = torch.empty(need, dtype=torch.uint8, device=u.device)
+                own_ws = True
             ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
         if plan is None:
             _check(lib.mamba_scan_fwd(ctypes.byref(args), ws_ptr, ws_bytes, _stream_ptr(stream)))
         else:
             _check(lib.mamba_scan_fwd_with_plan(ctypes.byref(args), ctypes.byref(plan), ws_ptr, ws_bytes,
                                                 _stream_ptr(stream)))
+        if own_ws:
+            _keep_until_done(workspace, stream)
     return (y, hT) if return_last_state else y
 
 
@@ -517,10 +549,13 @@ def scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, delta_softp
     with torch.cuda.device(u.device):
         n = ctypes.c_size_t(0)
         _check(lib.mamba_scan_bwd_workspace_size(ctypes.byref(args), ctypes.byref(n)))
-        if workspace is None or workspace.numel() < n.value:
+        own_ws = workspace is None or workspace.numel() < n.value
+        if own_ws:
             workspace = torch.empty(max(n.value, 1), dtype=torch.uint8, device=u.device)
         _check(lib.mamba_scan_bwd(ctypes.byref(args), ctypes.byref(g), workspace.data_ptr(), workspace.numel(),
                                   _stream_ptr(stream)))
+        if own_ws:
+            _keep_until_done(workspace, stream)
     return out
 
 
@@ -582,7 +617,8 @@ def ssd_check(workspace, stream=None):
 
 
 def ssd_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True, initial_state=None,
-            return_final_state=True, out=None, workspace=None, check=True, stream=None):
+            return_final_state=True, out=None, workspace=None, check=True, stream=None, wait_limit_us=0,
+            withhold_block=0):
     """Mamba-2 scalar-decay SSM forward (chunked SSD on the tensor cores).
 
     Shapes as :func:`build_ssd_args`. Returns ``(y, final_state)``
@@ -590,7 +626,9 @@ def ssd_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True, init
     of at least ``SSD_WORKSPACE_BYTES`` bytes holding the status word (one is
     allocated when None). With ``check`` the call synchronizes the stream and
     raises if the kernel reported a failed wait; without it, call
-    :func:`ssd_check` on the workspace later.
+    :func:`ssd_check` on the workspace later. ``wait_limit_us`` bounds each
+    of the kernel's pipeline waits (0: about one second); ``withhold_block``
+    is the fault-injection hook of ``ms_ssd_args`` (tests only).
     """
     torch = _torch()
     y = torch.empty_like(x) if out is None else out
@@ -599,11 +637,34 @@ def ssd_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True, init
         hT = torch.empty((x.shape[0], x.shape[2], SSD_HEADDIM, SSD_DSTATE), device=x.device, dtype=torch.float32)
     args = build_ssd_args(x, dt, A, B, C, y, D=D, z=z, dt_bias=dt_bias, dt_softplus=dt_softplus,
                           initial_state=initial_state, final_state=hT)
-    if workspace is None:
+    args.wait_limit_us = int(wait_limit_us)
+    args.withhold_block = int(withhold_block)
+    own_ws = workspace is None
+    if own_ws:
         workspace = torch.empty(SSD_WORKSPACE_BYTES, dtype=torch.uint8, device=x.device)
     with torch.cuda.device(x.device):
         _check(load_library().mamba_ssd_fwd(ctypes.byref(args), workspace.data_ptr(), workspace.numel(),
                                              _stream_ptr(stream)))
+        if own_ws:
+            _keep_until_done(workspace, stream)
     if check:
         ssd_check(workspace, stream)
     return y, hT
+
+
+PROBE_UNITS = {"ex2": 0, "tanh": 1, "ffma": 2, "ffma2": 3}
+
+
+def probe_unit_throughput(unit: str, device=None, stream=None):
+    """Measured throughput of one arithmetic unit on ``device`` (see
+    ``mamba_probe_unit_throughput``): returns (results per second, results per
+    clock per SM). ``unit``: "ex2", "tanh", "ffma" or "ffma2". Synchronous."""
+    torch = _torch()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        scratch = torch.empty(256, dtype=torch.uint8, device=dev)
+        per_s, per_clk = ctypes.c_double(0.0), ctypes.c_double(0.0)
+        _check(load_library().mamba_probe_unit_throughput(PROBE_UNITS[unit], scratch.data_ptr(),
+                                                          ctypes.byref(per_s), ctypes.byref(per_clk),
+                                                          _stream_ptr(stream)))
+    return per_s.value, per_clk.value

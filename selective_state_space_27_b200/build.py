@@ -15,7 +15,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmambascan.so")
-SOURCES = ["api.cu", "scan_fwd.cu", "scan_rec.cu", "scan_bwd.cu", "state_update.cu", "noalloc.cu", "ssd_fwd.cu"]
+SOURCES = ["api.cu", "scan_fwd.cu", "scan_rec.cu", "scan_bwd.cu", "state_update.cu", "noalloc.cu", "ssd_fwd.cu", "probe.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -196,12 +196,8 @@ ms_status run_plan(ms::ScanParams p, const ms::ScanPlan &plan, int in_dtype, voi
             set_error("workspace must be 256-byte aligned");
             return MS_ERR_ALIGNMENT;
         }
-        float *ws = static_cast<float *>(workspace);
-        p.ws_P = ws;
-        p.ws_H = ws + plan.ws_bytes / 2 / sizeof(float);
     }
-    p.nseg = plan.nseg;
-    p.seg_len = plan.seg_len;
+    ms::bind_workspace(p, plan, workspace);
     const cudaError_t e = ms::launch_scan(p, plan, in_dtype, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "scan kernel launch");
     return MS_OK;
@@ -291,6 +287,28 @@ ms_status mamba_scan_plan_query(const ms_scan_args *args, ms_scan_plan *plan) {
     plan->lanes = pl.lg;
     plan->segment_len = pl.seg_len;
     plan->workspace_bytes = pl.ws_bytes;
+    plan->ctas = pl.ctas;
+    plan->reserved = 0;
+    return MS_OK;
+}
+
+ms_status mamba_scan_plan_workspace_size(const ms_scan_args *args, const ms_scan_plan *plan, size_t *bytes) {
+    if (!bytes) return invalid("bytes is NULL");
+    *bytes = 0;
+    if (!plan) return invalid("plan is NULL");
+    ms_status st = check_scan(args);
+    if (st != MS_OK) return st;
+    int sms = 0;
+    st = device_sms(&sms);
+    if (st != MS_OK) return st;
+    ms::ScanPlan pl{};
+    if (!ms::make_plan(to_params(args), args->in_dtype, plan->config, plan->warps_per_cta, plan->segments,
+                       plan->ctas, sms, &pl)) {
+        set_error("plan (config %d, %d warps, %d segments, %d CTAs) cannot run these arguments", plan->config,
+                  plan->warps_per_cta, plan->segments, plan->ctas);
+        return MS_ERR_UNSUPPORTED;
+    }
+    *bytes = pl.ws_bytes;
     return MS_OK;
 }
 
@@ -301,10 +319,14 @@ ms_status mamba_scan_fwd_with_plan(const ms_scan_args *args, const ms_scan_plan 
     ms_status st = check_scan(args);
     if (st != MS_OK) return st;
     const ms::ScanParams p = to_params(args);
+    int sms = 0;
+    st = device_sms(&sms);
+    if (st != MS_OK) return st;
     ms::ScanPlan pl{};
-    if (!ms::make_plan(p, args->in_dtype, plan->config, plan->warps_per_cta, plan->segments, &pl)) {
-        set_error("plan (config %d, %d warps, %d segments) cannot run these arguments", plan->config,
-                  plan->warps_per_cta, plan->segments);
+    if (plan->reserved != 0 ||
+        !ms::make_plan(p, args->in_dtype, plan->config, plan->warps_per_cta, plan->segments, plan->ctas, sms, &pl)) {
+        set_error("plan (config %d, %d warps, %d segments, %d CTAs) cannot run these arguments", plan->config,
+                  plan->warps_per_cta, plan->segments, plan->ctas);
         return MS_ERR_UNSUPPORTED;
     }
     return run_plan(p, pl, args->in_dtype, workspace, workspace_bytes, stream);
@@ -366,7 +388,8 @@ ms_status mamba_conv_scan_fwd(const ms_scan_args *args, const ms_conv1d_args *co
     p.conv_silu = conv->silu;
     ms::ScanPlan pl{};
     if (plan) {
-        if (!ms::make_plan(p, args->in_dtype, plan->config, plan->warps_per_cta, plan->segments, &pl)) {
+        if (plan->ctas != 0 || plan->reserved != 0 ||
+            !ms::make_plan(p, args->in_dtype, plan->config, plan->warps_per_cta, plan->segments, 0, 0, &pl)) {
             set_error("plan (config %d, %d warps, %d segments) cannot run the convolution prologue", plan->config,
                       plan->warps_per_cta, plan->segments);
             return MS_ERR_UNSUPPORTED;
@@ -405,7 +428,8 @@ ms_status mamba_trap_scan_fwd(const ms_scan_args *args, const void *lambda_raw, 
     p.lm_sd = lambda_dim_stride;
     ms::ScanPlan pl{};
     if (plan) {
-        if (!ms::make_plan(p, args->in_dtype, plan->config, plan->warps_per_cta, plan->segments, &pl)) {
+        if (plan->ctas != 0 || plan->reserved != 0 ||
+            !ms::make_plan(p, args->in_dtype, plan->config, plan->warps_per_cta, plan->segments, 0, 0, &pl)) {
             set_error("plan (config %d, %d warps, %d segments) cannot run the trapezoidal rule", plan->config,
                       plan->warps_per_cta, plan->segments);
             return MS_ERR_UNSUPPORTED;
@@ -552,6 +576,9 @@ ms_status mamba_ssd_fwd(const ms_ssd_args *a, void *workspace, size_t workspace_
     p.batch = a->batch; p.seqlen = a->seqlen; p.nheads = a->nheads; p.ngroups = a->ngroups;
     p.softplus = a->dt_softplus ? 1 : 0;
     p.status = static_cast<int *>(workspace);
+    if (a->withhold_block < 0) return invalid("withhold_block must be >= 0");
+    p.wait_limit_ns = a->wait_limit_us ? 1000ull * a->wait_limit_us : 1000000000ull;
+    p.withhold_block = a->withhold_block;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int), s);
     if (e != cudaSuccess) return cuda_fail(e, "clearing the SSD status word");

@@ -32,6 +32,17 @@ struct ScanParams {
     // current input, h_t = a_t h_{t-1} + (1-lambda_t) delta_t a_t B_{t-1} u_{t-1}
     // + lambda_t delta_t B_t u_t.
     const void *lambda_raw; int64_t lm_sb, lm_sd;
+    // Persistent schedule of the sequential kernels (sk_ctas > 0): the chunks
+    // of all units (one batch entry x one block of rows) form one list, cut
+    // into sk_ctas equal ranges, one per CTA. A unit whose chunks fall into two
+    // ranges is started by the CTA that owns its first chunks and continued by
+    // the next CTA from the state left in sk_carry (ready when sk_flag[unit] is
+    // set). sk_ctas == 0: one CTA per unit.
+    int sk_ctas;
+    int sk_units;             // batch * row blocks
+    float *sk_carry;          // (units, rows per unit, 16) states handed over
+    int *sk_flag;             // (units) zero at launch, 1 once the unit's carry is written
+    int *sk_status;           // receives MS_ERR_TIMEOUT if a carry wait gave up
 };
 
 // Launch configuration chosen on the host for one scan call.
@@ -47,7 +58,16 @@ struct ScanPlan {
     int nseg;
     int64_t seg_len;
     size_t ws_bytes;
+    int ctas;           // kind 1: 0 = one CTA per unit; > 0 = persistent schedule over this many CTAs
 };
+
+// Workspace of a persistent sequential scan: a status word (first 256 bytes),
+// the units' carry flags, then their carry states; everything before the
+// carry states is cleared on the stream before each launch.
+size_t rec_persistent_ws_bytes(int64_t units, int rows_per_unit);
+size_t rec_persistent_clear_bytes(int64_t units);
+// Point p's persistent-schedule fields into the workspace `ws`.
+void rec_bind_workspace(ScanParams &p, void *ws, int64_t units, int ctas);
 
 // With p.conv_w or p.lambda_raw set only the sequential configurations that
 // fuse the convolution prologue or run the trapezoidal rule (lanes 2 and 4)
@@ -55,7 +75,13 @@ struct ScanPlan {
 ScanPlan plan_scan(const ScanParams &p, int in_dtype, int force_segments, int num_sms);
 // A plan with a fixed configuration, CTA size and segment count; returns false
 // (and leaves `out` unspecified) when the configuration cannot run `p`.
-bool make_plan(const ScanParams &p, int in_dtype, int config, int warps, int segments, ScanPlan *out);
+// ctas: sequential configurations only, 0 = one CTA per unit, > 0 = persistent
+// schedule over that many CTAs (at most rec_max_ctas).
+bool make_plan(const ScanParams &p, int in_dtype, int config, int warps, int segments, int ctas, int num_sms,
+               ScanPlan *out);
+// Point the kernel parameters at the plan's workspace (multi-block carry, or
+// the persistent schedule's flags and carry states).
+void bind_workspace(ScanParams &p, const ScanPlan &plan, void *workspace);
 int scan_num_configs();
 bool scan_config_info(int config, int *lanes, int *states_per_pass, int *max_warps);
 int scan_config_kind(int config);   // 0 chunked, 1 sequential, -1 unknown index
@@ -73,6 +99,9 @@ int rec_rows(int lanes_per_row);
 int rec_ctas_per_sm(int in_dtype, int lanes_per_row, bool vec, int variant);
 bool rec_supports_variant(int lanes_per_row, int variant);
 cudaError_t launch_rec(const ScanParams &p, int lanes_per_row, bool vec, int in_dtype, cudaStream_t stream);
+// Largest CTA count a persistent sequential launch can use (every CTA resident
+// at once, at most one per unit).
+int rec_max_ctas(const ScanParams &p, int in_dtype, int lanes_per_row, bool vec, int num_sms);
 
 // Backward pass (scan_bwd.cu): output gradients in, input gradients out.
 // du, ddelta, dz: (batch, dim, L) in the input dtype; dB, dC: (batch, dstate,
@@ -131,6 +160,8 @@ struct SsdParams {
     int64_t batch, seqlen, nheads, ngroups;
     int softplus;
     int *status;
+    uint64_t wait_limit_ns;   // limit of each pipeline wait
+    int withhold_block;       // tests: k > 0 withholds block k - 1's loads (the wait for them runs out)
 };
 constexpr int kSsdHeadDim = 64;
 constexpr int kSsdState = 128;

@@ -98,13 +98,7 @@ static ms_status noalloc_call(const ms_scan_args *args, void *stream) {
     p.h0 = args->initial_state; p.hT = args->final_state;
     p.softplus = args->delta_softplus ? 1 : 0;
     const ms::ScanPlan plan = ms::plan_scan(p, args->in_dtype, args->force_segments, sms);
-    if (plan.ws_bytes > 0) {
-        float *ws = static_cast<float *>(scratch);
-        p.ws_P = ws;
-        p.ws_H = ws + plan.ws_bytes / 2 / sizeof(float);
-    }
-    p.nseg = plan.nseg;
-    p.seg_len = plan.seg_len;
+    ms::bind_workspace(p, plan, scratch);
     const cudaError_t e = ms::launch_scan(p, plan, args->in_dtype, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(MS_ERR_CUDA, "scan kernel launch: %s", cudaGetErrorString(e));
     return MS_OK;

@@ -596,6 +596,9 @@ double config_cost(const Config &c) {
 constexpr int kRecLanes[] = {2, 4, 8, 16};
 constexpr int kNumRec = sizeof(kRecLanes) / sizeof(kRecLanes[0]);
 constexpr double kRecCost[] = {1.6, 1.9, 2.5, 4.2};
+// Relative cost of the persistent schedule's bookkeeping (cursors, carry
+// hand-over) per unit of work.
+constexpr double kRecPersistentCost = 1.02;
 // SM clocks per unit of the chunked kernels' cost model (measured: a
 // Mamba-130M layer on cfg 7, 11 warps, took 485k clocks for 1.30M units).
 constexpr double kChunkedClocksPerUnit = 0.372;
@@ -681,7 +684,7 @@ ScanPlan plan_scan(const ScanParams &p, int in_dtype, int force_segments, int nu
     // Sequential kernels: no segments; an SM runs its CTAs in waves of as many
     // as are resident, every resident CTA adds one recurrence warp per
     // sub-partition, and a lone CTA runs 1.4x slower per row than a shared SM.
-    int rec = -1;
+    int rec = -1, rec_ctas = 0;
     if (force_segments <= 1 && p.dstate <= kMaxN) {
         const double mufu = (kMaxN + 3) / 16.0;   // MUFU clocks per (row, step): 16 states + softplus + gate
         best *= kChunkedClocksPerUnit;
@@ -693,26 +696,41 @@ ScanPlan plan_scan(const ScanParams &p, int in_dtype, int force_segments, int nu
             const int64_t R = rec_rows(lpr);
             const int64_t ctas = p.batch * ((p.dim + R - 1) / R);
             const int64_t heavy = (ctas + sms - 1) / sms;
-            auto wave = [&](int64_t m) {
-                return (m == 1 ? 1.4 : static_cast<double>(m)) * R * static_cast<double>(p.seqlen) * mufu * kRecCost[ri];
+            auto wave = [&](double m) {
+                return (m <= 1.0 ? 1.4 : m) * R * static_cast<double>(p.seqlen) * mufu * kRecCost[ri];
             };
             const double t = (heavy / per_sm) * wave(per_sm) + (heavy % per_sm ? wave(heavy % per_sm) : 0.0);
             if (t < best * 0.999) {
                 best = t;
                 rec = ri;
+                rec_ctas = 0;
+            }
+            // persistent schedule: m CTAs on every SM share the units' work exactly
+            if (variant == 0 && p.batch * p.dim <= (int64_t(1) << 30) && (p.seqlen + 15) / 16 < (int64_t(1) << 30)) {
+                for (int m = 1; m <= per_sm && static_cast<int64_t>(m) * sms <= ctas; ++m) {
+                    const double tp = static_cast<double>(ctas) / (static_cast<double>(m) * sms) * wave(m) *
+                                      kRecPersistentCost;
+                    if (tp < best * 0.999) {
+                        best = tp;
+                        rec = ri;
+                        rec_ctas = m * sms;
+                    }
+                }
             }
         }
     }
     ScanPlan out = plan;
     if (rec >= 0) {
-        make_plan(p, in_dtype, kNumConfigs + rec, rec_threads() / 32, 1, &out);
+        make_plan(p, in_dtype, kNumConfigs + rec, rec_threads() / 32, 1, rec_ctas, sms, &out);
     } else {
-        make_plan(p, in_dtype, plan.config, plan.warps, plan.nseg, &out);
+        make_plan(p, in_dtype, plan.config, plan.warps, plan.nseg, 0, sms, &out);
     }
     return out;
 }
 
-bool make_plan(const ScanParams &p, int in_dtype, int config, int warps, int segments, ScanPlan *out) {
+bool make_plan(const ScanParams &p, int in_dtype, int config, int warps, int segments, int ctas, int num_sms,
+               ScanPlan *out) {
+    if (ctas < 0) return false;
     if (config >= kNumConfigs && config < kNumConfigs + kNumRec) {
         // sequential kernel: fixed CTA of rec_threads(), the whole sequence in one pass
         if (warps != rec_threads() / 32 || segments != 1 || p.dstate > kMaxN) return false;
@@ -734,9 +752,22 @@ bool make_plan(const ScanParams &p, int in_dtype, int config, int warps, int seg
         plan.nseg = 1;
         plan.seg_len = p.seqlen;
         plan.ws_bytes = 0;
+        plan.ctas = 0;
+        if (ctas > 0) {
+            // persistent schedule: every CTA resident, at most one per unit,
+            // no trapezoidal rule (its carry would need the previous step's input)
+            const int64_t units = p.batch * ((p.dim + plan.rows_per_cta - 1) / plan.rows_per_cta);
+            if (rec_variant(p) == 2 || units > (int64_t(1) << 30) || p.batch * p.dim > (int64_t(1) << 30) ||
+                (p.seqlen + rec_chunk() - 1) / rec_chunk() >= (int64_t(1) << 30))
+                return false;
+            if (ctas > rec_max_ctas(p, in_dtype, plan.lg, plan.vec != 0, num_sms > 0 ? num_sms : 148)) return false;
+            plan.ctas = ctas;
+            plan.ws_bytes = rec_persistent_ws_bytes(units, plan.rows_per_cta);
+        }
         *out = plan;
         return true;
     }
+    if (ctas != 0) return false;
     if (config < 0 || config >= kNumConfigs || segments < 1 || rec_variant(p) != 0) return false;
     const Config cf = kConfigs[config];
     ScanPlan plan{};
@@ -787,6 +818,20 @@ bool scan_config_info(int config, int *lanes, int *states_per_pass, int *max_war
     if (states_per_pass) *states_per_pass = kConfigs[config].ni;
     if (max_warps) *max_warps = kConfigs[config].maxt / 32;
     return true;
+}
+
+void bind_workspace(ScanParams &p, const ScanPlan &plan, void *workspace) {
+    p.nseg = plan.nseg;
+    p.seg_len = plan.seg_len;
+    if (plan.ws_bytes == 0) return;
+    if (plan.kind == 1) {
+        const int64_t units = p.batch * ((p.dim + plan.rows_per_cta - 1) / plan.rows_per_cta);
+        rec_bind_workspace(p, workspace, units, plan.ctas);
+    } else {
+        float *ws = static_cast<float *>(workspace);
+        p.ws_P = ws;
+        p.ws_H = ws + plan.ws_bytes / 2 / sizeof(float);
+    }
 }
 
 cudaError_t launch_scan(const ScanParams &p, const ScanPlan &plan, int in_dtype, cudaStream_t stream) {

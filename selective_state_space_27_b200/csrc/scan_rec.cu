@@ -155,6 +155,151 @@ __device__ __forceinline__ void bar_signal(int id) {
     asm volatile("bar.arrive %0, %1;" ::"r"(id), "n"(kThreads) : "memory");
 }
 
+// ---- Work schedule ----------------------------------------------------------
+// A unit is one batch entry x one block of R rows; its sequence is cut into
+// nc chunks of kSteps steps. Without the persistent schedule a CTA owns one
+// unit (blockIdx.x = row block, blockIdx.y = batch entry). With it
+// (p.sk_ctas > 0), the chunks of all units, unit after unit, form one list
+// that is cut into sk_ctas equal ranges, one per CTA, so that every SM gets
+// the same amount of recurrence whatever the number of units. A range is
+// [us:cs, ue:ce) in (unit, chunk) coordinates; since there are at most as
+// many CTAs as units it holds the end of unit us (from chunk cs), whole units
+// us+1 .. ue-1 and the start of unit ue (up to chunk ce). The CTA first runs
+// the start of ue, which begins at t = 0 and whose end state it hands over
+// (sk_carry, sk_flag) to the CTA that owns the rest of ue; then the whole
+// units; and last the end of us, from the state the previous CTA left. By
+// then that CTA has long finished the start of us: it ran those chunks first,
+// and there are fewer of them than the chunks this CTA ran before needing
+// them.
+struct Sched {
+    int us, cs, ue, ce;   // the range (ce in 1 .. nc)
+    int nc, blocks;       // chunks per unit, row blocks per batch entry
+    int64_t K;            // chunks of this CTA
+};
+
+__device__ __forceinline__ Sched make_sched(const ScanParams &p, int R) {
+    Sched s;
+    s.nc = static_cast<int>((p.seqlen + kSteps - 1) / kSteps);
+    s.blocks = static_cast<int>((p.dim + R - 1) / R);
+    if (p.sk_ctas == 0) {
+        s.us = s.ue = static_cast<int>(blockIdx.y) * s.blocks + static_cast<int>(blockIdx.x);
+        s.cs = 0;
+        s.ce = s.nc;
+        s.K = s.nc;
+    } else {
+        const int64_t T = static_cast<int64_t>(p.sk_units) * s.nc;
+        const int64_t G = p.sk_ctas, g = blockIdx.x, q = T / G, r = T % G;
+        const int64_t a = g * q + (g * r) / G;                 // floor(g T / G) without overflow
+        const int64_t e = (g + 1) * q + ((g + 1) * r) / G;
+        s.us = static_cast<int>(a / s.nc);
+        s.cs = static_cast<int>(a - static_cast<int64_t>(s.us) * s.nc);
+        s.ue = static_cast<int>((e - 1) / s.nc);
+        s.ce = static_cast<int>(e - static_cast<int64_t>(s.ue) * s.nc);
+        s.K = e - a;
+    }
+    return s;
+}
+
+// Position in a CTA's work: unit u (batch entry b, first row d0) and chunk c;
+// seg 0 = the start of unit ue, 1 = the whole units, 2 = the end of unit us.
+struct Cur {
+    int u, c, b, d0, seg;
+};
+
+__device__ __forceinline__ void cur_unit(Cur &k, const Sched &s, int u, int R) {
+    k.u = u;
+    k.b = u / s.blocks;
+    k.d0 = (u - k.b * s.blocks) * R;
+}
+__device__ __forceinline__ int head_end(const Sched &s) { return s.us == s.ue ? s.ce : s.nc; }
+__device__ __forceinline__ Cur cur_begin(const Sched &s, int R) {
+    Cur k;
+    if (s.us == s.ue) {
+        k.seg = 2;
+        cur_unit(k, s, s.us, R);
+        k.c = s.cs;
+    } else {
+        k.seg = 0;
+        cur_unit(k, s, s.ue, R);
+        k.c = 0;
+    }
+    return k;
+}
+__device__ __forceinline__ void cur_next(Cur &k, const Sched &s, int R) {
+    ++k.c;
+    if (k.seg == 0) {
+        if (k.c == s.ce) {
+            if (s.us + 1 < s.ue) {
+                k.seg = 1;
+                cur_unit(k, s, s.us + 1, R);
+                k.c = 0;
+            } else {
+                k.seg = 2;
+                cur_unit(k, s, s.us, R);
+                k.c = s.cs;
+            }
+        }
+    } else if (k.seg == 1) {
+        if (k.c == s.nc) {
+            if (k.u + 1 < s.ue) {
+                cur_unit(k, s, k.u + 1, R);
+                k.c = 0;
+            } else {
+                k.seg = 2;
+                cur_unit(k, s, s.us, R);
+                k.c = s.cs;
+            }
+        }
+    } else if (k.c == head_end(s)) {
+        k.seg = 3;
+    }
+}
+// first / last chunk of the piece the cursor is in
+__device__ __forceinline__ bool cur_first(const Cur &k, const Sched &s) { return k.c == (k.seg == 2 ? s.cs : 0); }
+__device__ __forceinline__ bool cur_last(const Cur &k, const Sched &s) {
+    return k.c + 1 == (k.seg == 0 ? s.ce : k.seg == 1 ? s.nc : head_end(s));
+}
+
+// Carry hand-over between CTAs. The writer's threads store the states, fence,
+// meet at a barrier of the recurrence warps, and one thread sets the flag with
+// release semantics; the reader's first thread polls the flag with acquire
+// semantics (sleeping between polls, giving up after kCarryWaitNs with
+// MS_ERR_TIMEOUT in the status word), then the recurrence warps meet and read
+// the states from L2.
+constexpr int kBarRecA = 13, kBarRecB = 14;   // named barriers of the 128 recurrence threads
+constexpr unsigned long long kCarryWaitNs = 4000000000ull;
+constexpr int kStatusTimeout = 5;               // MS_ERR_TIMEOUT
+
+__device__ __forceinline__ void rec_bar(int id) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(kScanThreads) : "memory");
+}
+__device__ __forceinline__ int ld_acquire(const int *f) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release(int *f, int v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(f), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void wait_carry(const ScanParams &p, int unit, int tid) {
+    if (tid == 0 && !ld_acquire(p.sk_flag + unit)) {
+        const unsigned long long t0 = global_ns();
+        while (!ld_acquire(p.sk_flag + unit)) {
+            __nanosleep(200);
+            if (global_ns() - t0 > kCarryWaitNs) {
+                atomicExch(p.sk_status, kStatusTimeout);
+                break;
+            }
+        }
+    }
+    rec_bar(kBarRecA);
+}
+
 // One step's B_t and C_t entries of a lane, as the pairs the packed
 // instructions take.
 template <int NPL> struct StepIn {
@@ -269,7 +414,8 @@ __device__ __forceinline__ void store_piece(T *dst, const float (&v)[P], int64_t
     }
 }
 
-// The recurrence warps: lane (r, q) owns states q NPL .. q NPL + NPL - 1 of row r.
+// The recurrence warps: lane (r, q) owns states q NPL .. q NPL + NPL - 1 of
+// row r of the unit being processed.
 template <typename T, int LPR, bool TRAP>
 __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned char *smem, int tid) {
     using S = Shape<LPR, TRAP>;
@@ -279,37 +425,48 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
     const int lane = tid & 31, warp = tid >> 5;
     const int r = S::GROUP_MAJOR ? warp * RW + lane % RW : tid / LPR;
     const int q = S::GROUP_MAJOR ? lane / RW : tid % LPR;
-    const int64_t b = blockIdx.y;
-    const int64_t d = static_cast<int64_t>(blockIdx.x) * R + r;
-    const bool ok = d < p.dim;
-    const int64_t dc = ok ? d : p.dim - 1;    // clamped row: loads stay in bounds
     const int dstate = static_cast<int>(p.dstate);
-    const int64_t nchunks = (p.seqlen + kSteps - 1) / kSteps;
-    const int64_t row = b * p.dim + dc;
+    const Sched sc = make_sched(p, R);
+    Cur kc = cur_begin(sc, R);
 
-    // A log2(e) and the entering state of the lane's states, kept as the
-    // register pairs the packed instructions take (no moves in the loop).
+    // A log2(e) and the state of the lane's states, kept as the register pairs
+    // the packed instructions take (no moves in the loop); set at the start of
+    // every piece of work.
     float2 ap[NP], hp[NP];
+    float2 bprev[NP];   // trapezoidal rule: the lane's B_{t-1} entries (B_{-1} u_{-1} = 0 via its coefficient)
+    bool ok = false;
+    int64_t row = 0;
 #pragma unroll
-    for (int j = 0; j < NP; ++j) {
-        float a2[2] = {0.f, 0.f}, h2[2] = {0.f, 0.f};
+    for (int j = 0; j < NP; ++j) ap[j] = hp[j] = bprev[j] = f2(0.f, 0.f);
+    int s = 0;   // tile stage of chunk it
+    for (int64_t it = 0; it < sc.K; ++it, s = next_stage(s, kTileStages), cur_next(kc, sc, R)) {
+        if (cur_first(kc, sc)) {
+            // a new piece: the rows of unit kc.u, entering state from the
+            // initial state (chunk 0) or from the CTA that ran the unit's start
+            const int64_t d = static_cast<int64_t>(kc.d0) + r;
+            ok = d < p.dim;
+            const int64_t dc = ok ? d : p.dim - 1;    // clamped row: loads stay in bounds
+            row = static_cast<int64_t>(kc.b) * p.dim + dc;
+            const bool carried = kc.c > 0;
+            if (carried) wait_carry(p, kc.u, tid);
+            const float *hsrc = carried ? p.sk_carry + (static_cast<int64_t>(kc.u) * R + r) * kStates
+                                        : (p.h0 ? p.h0 + row * dstate : nullptr);
 #pragma unroll
-        for (int e = 0; e < 2 && 2 * j + e < NPL; ++e) {
-            const int n = q * NPL + 2 * j + e;
-            if (n < dstate) {
-                a2[e] = __ldg(p.A + dc * dstate + n) * kLog2e;
-                if (p.h0) h2[e] = __ldg(p.h0 + row * dstate + n);
+            for (int j = 0; j < NP; ++j) {
+                float a2[2] = {0.f, 0.f}, h2[2] = {0.f, 0.f};
+#pragma unroll
+                for (int e = 0; e < 2 && 2 * j + e < NPL; ++e) {
+                    const int n = q * NPL + 2 * j + e;
+                    if (n < dstate) {
+                        a2[e] = __ldg(p.A + dc * dstate + n) * kLog2e;
+                        if (hsrc) h2[e] = carried ? __ldcg(hsrc + n) : __ldg(hsrc + n);
+                    }
+                }
+                ap[j] = f2(a2[0], a2[1]);
+                hp[j] = f2(h2[0], h2[1]);
+                bprev[j] = f2(0.f, 0.f);
             }
         }
-        ap[j] = f2(a2[0], a2[1]);
-        hp[j] = f2(h2[0], h2[1]);
-    }
-
-    float2 bprev[NP];   // trapezoidal rule: the lane's B_{t-1} entries (B_{-1} u_{-1} = 0 via its coefficient)
-#pragma unroll
-    for (int j = 0; j < NP; ++j) bprev[j] = f2(0.f, 0.f);
-    int s = 0;   // tile stage of chunk c
-    for (int64_t c = 0; c < nchunks; ++c, s = next_stage(s, kTileStages)) {
         unsigned char *st = smem + s * S::STAGE;
         const float4 *xrow = reinterpret_cast<const float4 *>(st + S::X_OFF) + r * S::XR;
         float *yl = reinterpret_cast<float *>(st + S::Y_OFF) + r * S::YR + (S::WARP_SUM ? 0 : q * S::YQ);
@@ -331,7 +488,7 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
         const float *Bl = reinterpret_cast<const float *>(st + S::B_OFF) + q * NPL;
         const float *Cl = reinterpret_cast<const float *>(st + S::C_OFF) + q * NPL;
         bar_wait(bar_xf(s));
-        if (c >= kTileStages) bar_wait(bar_ye(s));
+        if (it >= kTileStages) bar_wait(bar_ye(s));
 
         // Software pipelined over the chunk: step pairs are read one pair
         // ahead, B and C one step ahead, and the ex2 of step t + 1 is issued
@@ -428,15 +585,29 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
             }
         }
         }
-        if (c + kTileStages < nchunks) bar_signal(bar_xe(s));
+        if (it + kTileStages < sc.K) bar_signal(bar_xe(s));
         bar_signal(bar_yf(s));
-    }
 
-    if (ok && p.hT) {
+        if (cur_last(kc, sc)) {
+            if (kc.c + 1 == sc.nc) {   // the end of the sequence: the final state
+                if (ok && p.hT) {
 #pragma unroll
-        for (int i = 0; i < NPL; ++i) {
-            const int n = q * NPL + i;
-            if (n < dstate) p.hT[row * dstate + n] = (i & 1) ? hp[i / 2].y : hp[i / 2].x;
+                    for (int i = 0; i < NPL; ++i) {
+                        const int n = q * NPL + i;
+                        if (n < dstate) p.hT[row * dstate + n] = (i & 1) ? hp[i / 2].y : hp[i / 2].x;
+                    }
+                }
+            } else {   // hand the state over to the CTA that continues this unit
+                float *dst = p.sk_carry + (static_cast<int64_t>(kc.u) * R + r) * kStates;
+#pragma unroll
+                for (int i = 0; i < NPL; ++i) {
+                    const int n = q * NPL + i;
+                    if (n < dstate) dst[n] = (i & 1) ? hp[i / 2].y : hp[i / 2].x;
+                }
+                __threadfence();
+                rec_bar(kBarRecB);
+                if (tid == 0) st_release(p.sk_flag + kc.u, 1);
+            }
         }
     }
 }
@@ -455,57 +626,49 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     constexpr int VE = RW::VE, BC_PER = RW::BC_PER;
     static_assert(IP % 2 == 0, "pieces hold step pairs");
     const int r = i / IPR, k = i % IPR;
-    const int64_t b = blockIdx.y;
-    const int64_t d = static_cast<int64_t>(blockIdx.x) * R + r;
-    const bool ok = d < p.dim;
-    const int64_t dc = ok ? d : p.dim - 1;
     const int dstate = static_cast<int>(p.dstate);
     const int64_t L = p.seqlen;
-    const int64_t nchunks = (L + kSteps - 1) / kSteps;
-
-    const float bias = p.delta_bias ? __ldg(p.delta_bias + dc) : 0.f;
-    const float Dd = p.D ? __ldg(p.D + dc) : 0.f;
     const bool has_z = p.z != nullptr;
     const int tk = k * IP;   // the thread's first step within a chunk
-    // Convolution taps right-aligned in a window of 4 (leading taps beyond the
-    // width stay 0): cw[3] weighs the current input.
-    float cw[4] = {0.f, 0.f, 0.f, 0.f}, cb = 0.f;
-    if constexpr (CONV) {
-        const int K = p.conv_width;
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-            if (j >= 4 - K) cw[j] = __ldg(p.conv_w + dc * K + (j - (4 - K)));
-        cb = p.conv_b ? __ldg(p.conv_b + dc) : 0.f;
-    }
-    const T *src_row[3] = {static_cast<const T *>(p.u) + b * p.u_sb + dc * p.u_sd + tk,
-                           static_cast<const T *>(p.delta) + b * p.dl_sb + dc * p.dl_sd + tk,
-                           has_z ? static_cast<const T *>(p.z) + b * p.z_sb + dc * p.z_sd + tk : nullptr};
-    T *yrow = static_cast<T *>(p.y) + b * p.y_sb + dc * p.y_sd + tk;
-    const T *lrow = TRAP ? static_cast<const T *>(p.lambda_raw) + b * p.lm_sb + dc * p.lm_sd + tk : nullptr;
+    const Sched sc = make_sched(p, R);
+
+    // The thread's row of a unit (clamped into range: loads stay in bounds).
+    struct RowCtx {
+        int64_t b, dc;
+        bool ok;
+    };
+    auto rowctx = [&](const Cur &kk) {
+        RowCtx x;
+        const int64_t d = static_cast<int64_t>(kk.d0) + r;
+        x.ok = d < p.dim;
+        x.dc = x.ok ? d : p.dim - 1;
+        x.b = kk.b;
+        return x;
+    };
 
     // The thread's B/C pieces: tensor (0 = B, 1 = C), state n, steps bt .. bt + VE - 1.
-    int bc_off[BC_PER], bc_t[BC_PER];
-    bool bc_live[BC_PER];
-    const T *bc_src[BC_PER];
+    int bc_off[BC_PER], bc_t[BC_PER], bc_n[BC_PER], bc_tensor[BC_PER];
 #pragma unroll
     for (int j = 0; j < BC_PER; ++j) {
         const int pc = i + j * kIoThreads;
-        const int tensor = pc / (kStates * (kSteps / VE));
+        bc_tensor[j] = pc / (kStates * (kSteps / VE));
         const int rem = pc % (kStates * (kSteps / VE));
-        const int n = rem % kStates;
+        bc_n[j] = rem % kStates;
         bc_t[j] = (rem / kStates) * VE;
-        bc_off[j] = (tensor == 0 ? S::B_OFF : S::C_OFF) + (bc_t[j] * kStates + n) * 4;
-        bc_live[j] = n < dstate;
-        const T *base = tensor == 0 ? static_cast<const T *>(p.B) + b * p.B_sb : static_cast<const T *>(p.C) + b * p.C_sb;
-        bc_src[j] = (bc_live[j] ? base + n * (tensor == 0 ? p.B_sn : p.C_sn) : base) + bc_t[j];
+        bc_off[j] = (bc_tensor[j] == 0 ? S::B_OFF : S::C_OFF) + (bc_t[j] * kStates + bc_n[j]) * 4;
     }
 
     unsigned char *ring = smem + RW::OFF;
     auto slot = [&](int rs, int sl) { return ring + rs * RW::STAGE + (sl * kIoThreads + i) * 16; };
 
-    // Issue the copies of chunk c's raw inputs into ring stage rs.
-    auto stage_chunk = [&](int64_t c, int rs) {
-        const int64_t t0 = c * kSteps;
+    // Issue the copies of the raw inputs of chunk kk into ring stage rs.
+    auto stage_chunk = [&](const Cur &kk, int rs) {
+        const RowCtx x = rowctx(kk);
+        const T *src_row[3] = {static_cast<const T *>(p.u) + x.b * p.u_sb + x.dc * p.u_sd + tk,
+                               static_cast<const T *>(p.delta) + x.b * p.dl_sb + x.dc * p.dl_sd + tk,
+                               has_z ? static_cast<const T *>(p.z) + x.b * p.z_sb + x.dc * p.z_sd + tk : nullptr};
+        const T *lrow = TRAP ? static_cast<const T *>(p.lambda_raw) + x.b * p.lm_sb + x.dc * p.lm_sd + tk : nullptr;
+        const int64_t t0 = static_cast<int64_t>(kk.c) * kSteps;
         const bool full = t0 + kSteps <= L;
         const int valid = full ? IP : static_cast<int>(min64(IP, max64(0, L - (t0 + tk))));
 #pragma unroll
@@ -566,13 +729,17 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
         }
 #pragma unroll
         for (int j = 0; j < BC_PER; ++j) {
-            const int vb = bc_live[j] ? (full ? VE : static_cast<int>(min64(VE, max64(0, L - (t0 + bc_t[j]))))) : 0;
+            const bool live = bc_n[j] < dstate;
+            const T *base = bc_tensor[j] == 0 ? static_cast<const T *>(p.B) + x.b * p.B_sb
+                                              : static_cast<const T *>(p.C) + x.b * p.C_sb;
+            const T *bsrc = (live ? base + bc_n[j] * (bc_tensor[j] == 0 ? p.B_sn : p.C_sn) : base) + bc_t[j];
+            const int vb = live ? (full ? VE : static_cast<int>(min64(VE, max64(0, L - (t0 + bc_t[j]))))) : 0;
             if constexpr (VEC) {
-                cp_async16(slot(rs, 3 * PS + j), vb > 0 ? static_cast<const void *>(bc_src[j] + t0)
-                                                       : static_cast<const void *>(bc_src[j]), vb * EB);
+                cp_async16(slot(rs, 3 * PS + j), vb > 0 ? static_cast<const void *>(bsrc + t0)
+                                                       : static_cast<const void *>(bsrc), vb * EB);
             } else {
                 Piece<T, VE> pc;
-                load_piece<T, VE, false>(pc, bc_src[j] + t0, vb);
+                load_piece<T, VE, false>(pc, bsrc + t0, vb);
                 *reinterpret_cast<uint4 *>(slot(rs, 3 * PS + j)) = make_uint4(pc.w[0], pc.w[1], pc.w[2], pc.w[3]);
             }
         }
@@ -598,9 +765,13 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     auto ring_piece = [&](int rs, int tsr) { return ring_slots(rs, tsr * PS); };
     // Readout of chunk c from tile stage s (u, z from ring stage rs): partial
     // sums + D u, gate, store.
-    auto finish = [&](int64_t c, int s, int rs) {
+    auto finish = [&](const Cur &kk, int s, int rs) {
+        const RowCtx x = rowctx(kk);
+        const int64_t c = kk.c;
         const int64_t cnt = L - (c * kSteps + tk);
-        if (!ok || cnt <= 0) return;
+        if (!x.ok || cnt <= 0) return;
+        const float Dd = p.D ? __ldg(p.D + x.dc) : 0.f;
+        T *yrow = static_cast<T *>(p.y) + x.b * p.y_sb + x.dc * p.y_sd + tk;
         const float *yp = reinterpret_cast<const float *>(smem + s * S::STAGE + S::Y_OFF) + r * S::YR + tk;
         float2 sum[IP / 2];
 #pragma unroll
@@ -650,7 +821,21 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     };
     // Chunk c's step tile (step pairs of delta, delta u) and B/C tiles from
     // ring stage rs into tile stage s.
-    auto widen = [&](int64_t c, int s, int rs) {
+    auto widen = [&](const Cur &kk, int s, int rs) {
+        const RowCtx x = rowctx(kk);
+        const int64_t c = kk.c;
+        const float bias = p.delta_bias ? __ldg(p.delta_bias + x.dc) : 0.f;
+        // Convolution taps right-aligned in a window of 4 (leading taps beyond
+        // the width stay 0): cw[3] weighs the current input.
+        float cw[4] = {0.f, 0.f, 0.f, 0.f}, cb = 0.f, Dd = 0.f;
+        if constexpr (CONV) {
+            const int K = p.conv_width;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (j >= 4 - K) cw[j] = __ldg(p.conv_w + x.dc * K + (j - (4 - K)));
+            cb = p.conv_b ? __ldg(p.conv_b + x.dc) : 0.f;
+            Dd = p.D ? __ldg(p.D + x.dc) : 0.f;
+        }
         unsigned char *st = smem + s * S::STAGE;
         float4 *xrow = reinterpret_cast<float4 *>(st + S::X_OFF) + r * S::XR + (TRAP ? tk : tk / 2);
         const Piece<T, IP> xin = ring_piece(rs, 0), dl = ring_piece(rs, 1);
@@ -726,43 +911,56 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
         }
     };
 
-    // Chunk c is widened in iteration c, finished in iteration c + kTileStages - 1
-    // (or after the loop), and its raw inputs are staged RA = RS - kTileStages
-    // + 1 iterations before its widening into the ring stage that the chunk
-    // finished in the same iteration releases. Prologue: chunks 0 .. RA - 1 in flight,
-    // one commit group per chunk (empty past the end: the count stays uniform).
+    // Chunk it (of the CTA's list) is widened in iteration it, finished in
+    // iteration it + kTileStages - 1 (or after the loop), and its raw inputs
+    // are staged RA = RS - kTileStages + 1 iterations before its widening into
+    // the ring stage that the chunk finished in the same iteration releases.
+    // Prologue: chunks 0 .. RA - 1 in flight, one commit group per chunk
+    // (empty past the end: the count stays uniform). Each of the three steps
+    // follows the CTA's work with its own cursor.
+    const int64_t K = sc.K;
+    Cur ka = cur_begin(sc, R), kw = ka, kf = ka;
 #pragma unroll
     for (int c0 = 0; c0 < RW::RA; ++c0) {
-        if (c0 < nchunks) stage_chunk(c0, c0);
+        if (c0 < K) {
+            stage_chunk(ka, c0);
+            cur_next(ka, sc, R);
+        }
         cp_async_commit();
     }
-    int s = 0, rs = 0;                    // tile and ring stage of chunk c
+    int s = 0, rs = 0;                    // tile and ring stage of chunk it
     int sf = 0, rf = 0;                   // tile and ring stage of the next chunk to finish
-    int ra = RW::RA % RW::RS;             // ring stage of chunk c + RA
-    for (int64_t c = 0; c < nchunks; ++c) {
-        cp_async_wait<RW::RA - 1>();      // chunk c's copies have landed
-        if (c >= kTileStages) bar_wait(bar_xe(s));
-        widen(c, s, rs);
+    int ra = RW::RA % RW::RS;             // ring stage of chunk it + RA
+    for (int64_t it = 0; it < K; ++it) {
+        cp_async_wait<RW::RA - 1>();      // chunk it's copies have landed
+        if (it >= kTileStages) bar_wait(bar_xe(s));
+        widen(kw, s, rs);
         bar_signal(bar_xf(s));
-        const int64_t j = c - (kTileStages - 1);
+        const int64_t j = it - (kTileStages - 1);
         if (j >= 0) {
             bar_wait(bar_yf(sf));
-            finish(j, sf, rf);
-            if (j + kTileStages < nchunks) bar_signal(bar_ye(sf));
+            finish(kf, sf, rf);
+            if (j + kTileStages < K) bar_signal(bar_ye(sf));
             sf = next_stage(sf, kTileStages);
             rf = next_stage(rf, RW::RS);
+            cur_next(kf, sc, R);
         }
-        if (c + RW::RA < nchunks) stage_chunk(c + RW::RA, ra);
+        if (it + RW::RA < K) {
+            stage_chunk(ka, ra);
+            cur_next(ka, sc, R);
+        }
         cp_async_commit();
         s = next_stage(s, kTileStages);
         rs = next_stage(rs, RW::RS);
         ra = next_stage(ra, RW::RS);
+        cur_next(kw, sc, R);
     }
-    for (int64_t j = max64(nchunks - (kTileStages - 1), 0); j < nchunks; ++j) {
+    for (int64_t j = max64(K - (kTileStages - 1), 0); j < K; ++j) {
         bar_wait(bar_yf(sf));
-        finish(j, sf, rf);
+        finish(kf, sf, rf);
         sf = next_stage(sf, kTileStages);
         rf = next_stage(rf, RW::RS);
+        cur_next(kf, sc, R);
     }
     cp_async_wait<0>();
 }
@@ -865,17 +1063,69 @@ int rec_ctas_per_sm(int in_dtype, int lpr, bool vec, int variant) {
     return n;
 }
 
+namespace {
+constexpr size_t kStatusBytes = 256;
+size_t round256(size_t n) { return (n + 255) / 256 * 256; }
+}  // namespace
+
+size_t rec_persistent_clear_bytes(int64_t units) {
+    return kStatusBytes + round256(static_cast<size_t>(units) * sizeof(int));
+}
+
+size_t rec_persistent_ws_bytes(int64_t units, int rows_per_unit) {
+    return rec_persistent_clear_bytes(units) +
+           static_cast<size_t>(units) * static_cast<size_t>(rows_per_unit) * kStates * sizeof(float);
+}
+
+void rec_bind_workspace(ScanParams &p, void *ws, int64_t units, int ctas) {
+    unsigned char *w = static_cast<unsigned char *>(ws);
+    p.sk_ctas = ctas;
+    p.sk_units = static_cast<int>(units);
+    p.sk_status = reinterpret_cast<int *>(w);
+    p.sk_flag = reinterpret_cast<int *>(w + kStatusBytes);
+    p.sk_carry = reinterpret_cast<float *>(w + rec_persistent_clear_bytes(units));
+}
+
+int rec_max_ctas(const ScanParams &p, int in_dtype, int lpr, bool vec, int num_sms) {
+    const int per_sm = rec_ctas_per_sm(in_dtype, lpr, vec, rec_variant(p));
+    const int64_t R = kScanThreads / lpr;
+    const int64_t units = p.batch * ((p.dim + R - 1) / R);
+    return static_cast<int>(min64(units, static_cast<int64_t>(per_sm) * num_sms));
+}
+
+// Persistent launches (p.sk_ctas > 0) are cooperative: the runtime starts them
+// only if every CTA can be resident at once, so a CTA that waits for another
+// one's carry never waits for a CTA that has not started. The flags and the
+// status word are cleared on the stream first.
 cudaError_t launch_rec(const ScanParams &p, int lpr, bool vec, int in_dtype, cudaStream_t stream) {
     const int variant = rec_variant(p);
     if (!rec_supports_variant(lpr, variant) || (p.conv_w && p.lambda_raw)) return cudaErrorInvalidValue;
+    if (p.sk_ctas > 0 && (variant == 2 || !p.sk_carry || !p.sk_flag || !p.sk_status)) return cudaErrorInvalidValue;
     const void *k = rec_kernel_for(in_dtype, lpr, vec, variant);
     const int smem = rec_smem_bytes(in_dtype, lpr, variant);
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const int R = kScanThreads / lpr;
-    const dim3 grid(static_cast<unsigned>((p.dim + R - 1) / R), static_cast<unsigned>(p.batch));
     void *args[] = {const_cast<ScanParams *>(&p)};
-    e = cudaLaunchKernel(k, grid, dim3(kThreads), args, static_cast<size_t>(smem), stream);
+    if (p.sk_ctas == 0) {
+        const dim3 grid(static_cast<unsigned>((p.dim + R - 1) / R), static_cast<unsigned>(p.batch));
+        e = cudaLaunchKernel(k, grid, dim3(kThreads), args, static_cast<size_t>(smem), stream);
+        if (e != cudaSuccess) return e;
+        return cudaGetLastError();
+    }
+    e = cudaMemsetAsync(p.sk_status, 0, rec_persistent_clear_bytes(p.sk_units), stream);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(p.sk_ctas));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr{};
+    attr.id = cudaLaunchAttributeCooperative;
+    attr.val.cooperative = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelExC(&cfg, k, args);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

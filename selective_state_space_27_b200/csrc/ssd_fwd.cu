@@ -283,13 +283,13 @@ __device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t q) { return r * 1
 
 // A bounded wait that also gives up at once when another role of the CTA has
 // already given up (abort flag in shared memory).
-__device__ __forceinline__ bool role_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag)
+__device__ __forceinline__ bool role_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag, uint64_t limit_ns)
 {
     if (mbar_test(bar, parity))
         return true;
     const uint64_t t0 = global_ns();
     while (!mbar_test(bar, parity)) {
-        if (*abort_flag || global_ns() - t0 > kWaitLimitNs)
+        if (*abort_flag || global_ns() - t0 > limit_ns)
             return false;
     }
     return true;
@@ -431,6 +431,7 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
     }
     auto bar = [&](int i) { return base + kOffBar + 8u * (uint32_t)i; };
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffAbort);
+    const uint64_t wlim = p.wait_limit_ns;
 
     if (threadIdx.x == 0) {
         mbar_init(bar(kFull0), 1);
@@ -478,12 +479,13 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
         int issued = 0;
         for (int c = 0; c < nchunks; ++c) {
             const int st = c & 1;
-            if (c >= 2 && !__all_sync(0xffffffffu, role_wait(bar(kEmpty0 + st), ((c >> 1) + 1) & 1, abort_flag))) {
+            if (c >= 2 && !__all_sync(0xffffffffu, role_wait(bar(kEmpty0 + st), ((c >> 1) + 1) & 1, abort_flag, wlim))) {
                 if (lane == 0)
                     give_up(p.status, abort_flag);
                 break;
             }
-            if (lane == 0) {
+            // (a test can withhold one block's loads: its full barrier then never completes)
+            if (lane == 0 && c + 1 != p.withhold_block) {
                 const uint32_t sx = base + (uint32_t)st * kStageBytes, sb = sx + kXTile, sc = sb + kBCTile;
                 const uint32_t full = bar(kFull0 + st);
                 mbar_arrive_tx(full, kStageTx);
@@ -538,7 +540,8 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
         // the loads in flight must land before the CTA leaves
         if (lane == 0)
             for (int c = issued > 2 ? issued - 2 : 0; c < issued; ++c)
-                mbar_wait(bar(kFull0 + (c & 1)), (c >> 1) & 1);
+                if (c + 1 != p.withhold_block)
+                    mbar_wait(bar(kFull0 + (c & 1)), (c >> 1) & 1);
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // ---- MMA issue (one thread) ----
@@ -550,7 +553,7 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
             for (int c = 0; c < nchunks; ++c) {
                 const int st = c & 1;
                 const uint32_t sx = base + (uint32_t)st * kStageBytes, sb = sx + kXTile, sc = sb + kBCTile;
-                if (!role_wait(bar(kFull0 + st), (c >> 1) & 1, abort_flag)) {
+                if (!role_wait(bar(kFull0 + st), (c >> 1) & 1, abort_flag, wlim)) {
                     give_up(p.status, abort_flag);
                     break;
                 }
@@ -563,8 +566,8 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
                 }
                 mma_commit(bar(kGFull0 + (c & 1)));
                 // Yo needs the state of the previous chunk and the Y columns free
-                if (!role_wait(bar(kHReady), c & 1, abort_flag) ||
-                    (c > 0 && !role_wait(bar(kYFree), (c - 1) & 1, abort_flag))) {
+                if (!role_wait(bar(kHReady), c & 1, abort_flag, wlim) ||
+                    (c > 0 && !role_wait(bar(kYFree), (c - 1) & 1, abort_flag, wlim))) {
                     give_up(p.status, abort_flag);
                     break;
                 }
@@ -577,7 +580,7 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
                              sw128_desc(base + kOffH + offh, 16, 1024), id_yo, k > 0);
                 }
                 // S and Yd need M' and Xt of this chunk
-                if (!role_wait(bar(kPReady), c & 1, abort_flag)) {
+                if (!role_wait(bar(kPReady), c & 1, abort_flag, wlim)) {
                     give_up(p.status, abort_flag);
                     break;
                 }
@@ -634,7 +637,7 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
         bool ok = true;
         auto epi_wait = [&](uint32_t barrier, uint32_t parity) {
             if (ok)
-                ok = __all_sync(0xffffffffu, role_wait(barrier, parity, abort_flag));
+                ok = __all_sync(0xffffffffu, role_wait(barrier, parity, abort_flag, wlim));
             if (!ok && lane == 0)
                 give_up(p.status, abort_flag);
             return ok;

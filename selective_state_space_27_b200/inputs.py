@@ -39,6 +39,8 @@ __all__ = [
     "SSD_WORKLOADS",
     "make_ssd_inputs",
     "make_ssd_state",
+    "make_delta_regime",
+    "DELTA_REGIMES",
 ]
 
 BASE_SEED = 20261202
@@ -47,7 +49,7 @@ BASE_SEED = 20261202
 # which other tensors were drawn.
 _STREAM = {"u": 1, "delta": 2, "B": 3, "C": 4, "z": 5, "D": 6, "dt": 7, "h0": 8, "conv_w": 9, "conv_b": 10,
            "conv_state": 11, "lambda_raw": 12, "ssd_x": 13, "ssd_dt": 14, "ssd_B": 15, "ssd_C": 16, "ssd_z": 17,
-           "ssd_head": 18, "ssd_h0": 19}
+           "ssd_head": 18, "ssd_h0": 19, "regime": 20, "regime_pick": 21}
 _CHUNK = 1 << 22
 
 
@@ -338,3 +340,40 @@ def make_ssd_inputs(w: SsdWorkload, *, batch=None, seqlen=None, nheads=None, ngr
 def make_ssd_state(batch: int, nheads: int, headdim: int = 64, dstate: int = 128, seed: int = BASE_SEED) -> np.ndarray:
     """An initial SSD state (batch, nheads, headdim, dstate) float32 ~ N(0, 1)."""
     return _normal((batch, nheads, headdim, dstate), seed, _STREAM["ssd_h0"])
+
+
+# Step values outside the layer recipe, for the method's degenerate regimes
+# ("Notas sobre Mamba", section "O mecanismo de seleção (S6)": a large step
+# resets the state to the current input, a step near zero keeps the state and
+# ignores the input):
+#   "large"  U[10, 50]    -- exp(delta A) underflows for every state
+#   "edge"   U[15, 40]    -- a softplus argument on both sides of 20
+#   "zero"   exactly 0    -- Abar = 1 and Bbar = 0
+#   "mixed"  per element 0 (30%), |N(0, 0.5^2)| / 8 (50%) or U[10, 50] (20%):
+#            resets and holds inside one sequence
+DELTA_REGIMES = ("large", "edge", "zero", "mixed")
+
+
+def make_delta_regime(shape, regime: str, dtype: str, seed: int = BASE_SEED) -> np.ndarray:
+    """Raw step values of one of ``DELTA_REGIMES`` in the storage dtype
+    (float32, or bf16 bits), shape ``shape``."""
+    if regime not in DELTA_REGIMES:
+        raise ValueError(f"unknown regime {regime!r}")
+    out = np.zeros(shape, np.float32)
+    if regime in ("large", "edge"):
+        lo, hi = (10.0, 50.0) if regime == "large" else (15.0, 40.0)
+
+        def draw(g, sl):
+            sl[:] = g.uniform(lo, hi, size=sl.size).astype(np.float32)
+
+        _fill(out, seed, _STREAM["regime"], draw)
+    elif regime == "mixed":
+        small = np.abs(_normal(shape, seed, _STREAM["regime"], 0.5)) / np.float32(8.0)
+        big = np.empty(shape, np.float32)
+        _fill(big, seed, _STREAM["regime"] + 100, lambda g, sl: sl.__setitem__(
+            slice(None), g.uniform(10.0, 50.0, size=sl.size).astype(np.float32)))
+        pick = np.empty(shape, np.float32)
+        _fill(pick, seed, _STREAM["regime_pick"], lambda g, sl: sl.__setitem__(
+            slice(None), g.random(size=sl.size, dtype=np.float32)))
+        out = np.where(pick < 0.3, np.float32(0.0), np.where(pick < 0.8, small, big)).astype(np.float32)
+    return _store(out, dtype)

@@ -63,7 +63,7 @@ def test_struct_layout_matches_binding(tmp_path):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.mamba_abi_version() == 1
+    assert lib.mamba_abi_version() == 2
     for code, name in ms.STATUS.items():
         assert lib.mamba_status_string(code).decode() == name
     assert lib.mamba_status_string(99).decode() == "MS_UNKNOWN_STATUS"

@@ -270,3 +270,25 @@ def test_plan_validation():
     args = ms.build_scan_args(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], y)
     plan = ms.scan_plan(args)
     assert 0 <= plan.config < len(configs) and plan.segments >= 1 and plan.warps_per_cta >= 2
+
+
+def test_side_stream_with_segments():
+    """A launch on a stream other than the current one, with the multi-block
+    carry workspace allocated by the binding: work queued meanwhile on the
+    current stream must not receive the workspace's memory while the scan
+    still uses it."""
+    import torch
+    ms = _ms()
+    inp = make_scan_inputs(LAYER, batch=2, dim=48, seqlen=6000 + 7, seed=1300)
+    dev = device_inputs(inp)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    y, hT = ms.scan_fwd(**dev, force_segments=6, stream=side)
+    # churn the allocator on the current stream while the side stream runs
+    junk = [torch.full((1 << 16,), 7, dtype=torch.uint8, device="cuda") for _ in range(64)]
+    del junk
+    side.synchronize()
+    torch.cuda.synchronize()
+    yr, hr = oracle_scan(inp)
+    assert rel_err(to_host64(y), yr) <= TOL["bf16"]
+    assert rel_err(to_host64(hT), hr) <= TOL["bf16"]

@@ -208,3 +208,41 @@ def test_ssd_batch_slices():
     assert rel_err(to_host64(y_out), yr) <= TOL["bf16"]
     assert rel_err(to_host64(hT), hr) <= TOL["bf16"]
     assert float(ybig[1::2].abs().max()) == 0.0
+
+
+@pytest.mark.parametrize("block", [1, 3])
+def test_ssd_timeout_path(block):
+    """The kernel's bounded pipeline waits: with block `block - 1`'s loads
+    withheld (the fault-injection hook of ms_ssd_args) and a 2 ms wait limit,
+    the wait for those loads runs out, the status word reads MS_ERR_TIMEOUT,
+    the CTA drains the loads and products it did issue and exits, and the
+    context stays usable: a normal call straight after it matches the oracle."""
+    import torch
+    ms = _ms()
+    inp = make_ssd_inputs(SMALL, batch=2, seqlen=700, nheads=2, seed=3300 + block)
+    dev = _dev(inp)
+    ws = torch.zeros(ms.SSD_WORKSPACE_BYTES, dtype=torch.uint8, device="cuda")
+    ms.ssd_fwd(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], D=dev["D"], z=dev["z"], dt_bias=dev["dt_bias"],
+               workspace=ws, check=False, wait_limit_us=2000, withhold_block=block)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32)[0].item()) == 5   # MS_ERR_TIMEOUT
+    with pytest.raises(ms.MambaScanError) as ei:
+        ms.ssd_check(ws)
+    assert ei.value.status == 5
+    y, hT = ms.ssd_fwd(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], D=dev["D"], z=dev["z"],
+                       dt_bias=dev["dt_bias"], workspace=ws)
+    yr, hr = _oracle(inp)
+    assert rel_err(to_host64(y), yr) <= TOL["bf16"]
+    assert rel_err(to_host64(hT), hr) <= TOL["bf16"]
+
+
+def test_ssd_withheld_block_past_the_end_is_harmless():
+    """A withheld block index beyond the sequence changes nothing."""
+    inp = make_ssd_inputs(SMALL, batch=1, seqlen=200, nheads=2, seed=3400)
+    dev = _dev(inp)
+    ms = _ms()
+    y, hT = ms.ssd_fwd(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], D=dev["D"], z=dev["z"],
+                       dt_bias=dev["dt_bias"], withhold_block=50, wait_limit_us=100000)
+    yr, hr = _oracle(inp)
+    assert rel_err(to_host64(y), yr) <= TOL["bf16"]
+    assert rel_err(to_host64(hT), hr) <= TOL["bf16"]
