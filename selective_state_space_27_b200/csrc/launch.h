@@ -59,6 +59,7 @@ struct ScanPlan {
     int64_t seg_len;
     size_t ws_bytes;
     int ctas;           // kind 1: 0 = one CTA per unit; > 0 = persistent schedule over this many CTAs
+    int iow;            // kind 1: I/O warps per CTA (2 or 4)
 };
 
 // Workspace of a persistent sequential scan: a status word (first 256 bytes),
@@ -91,17 +92,19 @@ cudaError_t launch_scan(const ScanParams &p, const ScanPlan &plan, int in_dtype,
 // Sequential kernels (scan_rec.cu): CTAs of rec_threads() threads (recurrence
 // and I/O warps) owning rec_rows(lanes_per_row) rows, no workspace, one segment.
 // Variants of the sequential kernel: 0 plain, 1 convolution prologue, 2 trapezoidal rule.
+// iow: I/O warps per CTA (2, or 4 for the plain scan with 2, 4 or 8 lanes per row).
 int rec_variant(const ScanParams &p);
-int rec_smem_bytes(int in_dtype, int lanes_per_row, int variant);
+int rec_smem_bytes(int in_dtype, int lanes_per_row, int variant, int iow);
 int rec_chunk();
-int rec_threads();
+int rec_threads(int iow);
 int rec_rows(int lanes_per_row);
-int rec_ctas_per_sm(int in_dtype, int lanes_per_row, bool vec, int variant);
-bool rec_supports_variant(int lanes_per_row, int variant);
-cudaError_t launch_rec(const ScanParams &p, int lanes_per_row, bool vec, int in_dtype, cudaStream_t stream);
+int rec_ctas_per_sm(int in_dtype, int lanes_per_row, bool vec, int variant, int iow);
+bool rec_supports_variant(int lanes_per_row, int variant, int iow);
+cudaError_t launch_rec(const ScanParams &p, int lanes_per_row, bool vec, int in_dtype, int iow,
+                       cudaStream_t stream);
 // Largest CTA count a persistent sequential launch can use (every CTA resident
 // at once, at most one per unit).
-int rec_max_ctas(const ScanParams &p, int in_dtype, int lanes_per_row, bool vec, int num_sms);
+int rec_max_ctas(const ScanParams &p, int in_dtype, int lanes_per_row, bool vec, int num_sms, int iow);
 
 // Backward pass (scan_bwd.cu): output gradients in, input gradients out.
 // du, ddelta, dz: (batch, dim, L) in the input dtype; dB, dC: (batch, dstate,

@@ -593,9 +593,11 @@ double config_cost(const Config &c) {
 // MUFU bound on a busy SM (shared-memory wavefronts of the step-tile and B/C
 // loads grow with the lanes per row; fitted to B200 timings of Mamba-130M,
 // Mamba-1.4B and 131k-token layers).
-constexpr int kRecLanes[] = {2, 4, 8, 16};
+// Configurations kNumConfigs + 0 .. 3 have 2 I/O warps, + 4 .. 6 have 4.
+constexpr int kRecLanes[] = {2, 4, 8, 16, 2, 4, 8};
+constexpr int kRecIow[] = {2, 2, 2, 2, 4, 4, 4};
 constexpr int kNumRec = sizeof(kRecLanes) / sizeof(kRecLanes[0]);
-constexpr double kRecCost[] = {1.6, 1.9, 2.5, 4.2};
+constexpr double kRecCost[] = {1.6, 1.9, 2.5, 4.2, 1.6, 1.9, 2.5};
 // Relative cost of the persistent schedule's bookkeeping (cursors, carry
 // hand-over) per unit of work.
 constexpr double kRecPersistentCost = 1.02;
@@ -689,9 +691,9 @@ ScanPlan plan_scan(const ScanParams &p, int in_dtype, int force_segments, int nu
         const double mufu = (kMaxN + 3) / 16.0;   // MUFU clocks per (row, step): 16 states + softplus + gate
         best *= kChunkedClocksPerUnit;
         for (int ri = 0; ri < kNumRec; ++ri) {
-            const int lpr = kRecLanes[ri];
-            if (!rec_supports_variant(lpr, variant)) continue;
-            const int per_sm = rec_ctas_per_sm(in_dtype, lpr, plan.vec, variant);
+            const int lpr = kRecLanes[ri], iow = kRecIow[ri];
+            if (!rec_supports_variant(lpr, variant, iow)) continue;
+            const int per_sm = rec_ctas_per_sm(in_dtype, lpr, plan.vec, variant, iow);
             if (per_sm < 1) continue;
             const int64_t R = rec_rows(lpr);
             const int64_t ctas = p.batch * ((p.dim + R - 1) / R);
@@ -721,7 +723,7 @@ ScanPlan plan_scan(const ScanParams &p, int in_dtype, int force_segments, int nu
     }
     ScanPlan out = plan;
     if (rec >= 0) {
-        make_plan(p, in_dtype, kNumConfigs + rec, rec_threads() / 32, 1, rec_ctas, sms, &out);
+        make_plan(p, in_dtype, kNumConfigs + rec, rec_threads(kRecIow[rec]) / 32, 1, rec_ctas, sms, &out);
     } else {
         make_plan(p, in_dtype, plan.config, plan.warps, plan.nseg, 0, sms, &out);
     }
@@ -733,13 +735,15 @@ bool make_plan(const ScanParams &p, int in_dtype, int config, int warps, int seg
     if (ctas < 0) return false;
     if (config >= kNumConfigs && config < kNumConfigs + kNumRec) {
         // sequential kernel: fixed CTA of rec_threads(), the whole sequence in one pass
-        if (warps != rec_threads() / 32 || segments != 1 || p.dstate > kMaxN) return false;
-        if (!rec_supports_variant(kRecLanes[config - kNumConfigs], rec_variant(p))) return false;
+        const int iow = kRecIow[config - kNumConfigs];
+        if (warps != rec_threads(iow) / 32 || segments != 1 || p.dstate > kMaxN) return false;
+        if (!rec_supports_variant(kRecLanes[config - kNumConfigs], rec_variant(p), iow)) return false;
         const int eb = in_dtype == 0 ? 4 : 2;
         auto strides_ok = [&](int64_t s1, int64_t s2) { return (s1 * eb) % 16 == 0 && (s2 * eb) % 16 == 0; };
         ScanPlan plan{};
         plan.kind = 1;
         plan.config = config;
+        plan.iow = iow;
         plan.lg = kRecLanes[config - kNumConfigs];
         plan.warps = warps;
         plan.rows_per_cta = rec_rows(plan.lg);
@@ -760,7 +764,7 @@ bool make_plan(const ScanParams &p, int in_dtype, int config, int warps, int seg
             if (rec_variant(p) == 2 || units > (int64_t(1) << 30) || p.batch * p.dim > (int64_t(1) << 30) ||
                 (p.seqlen + rec_chunk() - 1) / rec_chunk() >= (int64_t(1) << 30))
                 return false;
-            if (ctas > rec_max_ctas(p, in_dtype, plan.lg, plan.vec != 0, num_sms > 0 ? num_sms : 148)) return false;
+            if (ctas > rec_max_ctas(p, in_dtype, plan.lg, plan.vec != 0, num_sms > 0 ? num_sms : 148, iow)) return false;
             plan.ctas = ctas;
             plan.ws_bytes = rec_persistent_ws_bytes(units, plan.rows_per_cta);
         }
@@ -810,7 +814,7 @@ bool scan_config_info(int config, int *lanes, int *states_per_pass, int *max_war
         const int lpr = kRecLanes[config - kNumConfigs];
         if (lanes) *lanes = lpr;
         if (states_per_pass) *states_per_pass = kMaxN / lpr;
-        if (max_warps) *max_warps = rec_threads() / 32;
+        if (max_warps) *max_warps = rec_threads(kRecIow[config - kNumConfigs]) / 32;
         return true;
     }
     if (config < 0 || config >= kNumConfigs) return false;
@@ -835,7 +839,7 @@ void bind_workspace(ScanParams &p, const ScanPlan &plan, void *workspace) {
 }
 
 cudaError_t launch_scan(const ScanParams &p, const ScanPlan &plan, int in_dtype, cudaStream_t stream) {
-    if (plan.kind == 1) return launch_rec(p, plan.lg, plan.vec != 0, in_dtype, stream);
+    if (plan.kind == 1) return launch_rec(p, plan.lg, plan.vec != 0, in_dtype, plan.iow, stream);
     const int W = plan.warps;
     const int smem = smem_bytes(in_dtype, plan.lg, W);
     const unsigned gx = static_cast<unsigned>((p.dim + plan.rows_per_cta - 1) / plan.rows_per_cta);

@@ -44,8 +44,8 @@ namespace ms {
 namespace {
 
 constexpr int kScanThreads = 128;   // 4 recurrence warps
-constexpr int kIoThreads = 64;      // 2 I/O warps
-constexpr int kThreads = kScanThreads + kIoThreads;
+// I/O warps per CTA: 2, or 4 (one per SM sub-partition, so that every
+// sub-partition carries the same share of the per-row work).
 constexpr int kSteps = 16;          // time steps per chunk
 constexpr int kStates = 16;         // states per row (smaller dstate is zero-padded)
 constexpr int kTileStages = 3;      // step/readout tile buffers between the two warp groups
@@ -67,10 +67,12 @@ constexpr int kTileStages = 3;      // step/readout tile buffers between the two
 // (32 w + l) / LPR and group l % LPR) a quarter-warp covers at most two rows.
 // With the trapezoidal rule (TRAP) the step tile holds one float4 per step:
 // (delta, lambda delta u, (1 - lambda) delta u_prev, 0).
-template <int LPR, bool TRAP = false> struct Shape {
+template <int LPR, bool TRAP = false, int IOW = 2> struct Shape {
+    static constexpr int IOT = 32 * IOW;                // I/O threads
+    static constexpr int THREADS = kScanThreads + IOT;  // threads per CTA
     static constexpr int NPL = kStates / LPR;           // states per lane
     static constexpr int R = kScanThreads / LPR;        // rows per CTA
-    static constexpr int IPR = LPR / 2;                 // I/O threads per row
+    static constexpr int IPR = IOT / R;                 // I/O threads per row
     static constexpr int IP = kSteps / IPR;             // steps per I/O thread
     static constexpr bool GROUP_MAJOR = LPR <= 4;
     // LPR 4: the four groups of a row sit in lanes r, r + 8, r + 16, r + 24 of
@@ -88,8 +90,8 @@ template <int LPR, bool TRAP = false> struct Shape {
     static constexpr int STAGE = C_OFF + kSteps * kStates * 4;
     static constexpr int BYTES = kTileStages * STAGE;
     // CTAs per SM the launch bounds provide registers for
-    static constexpr int MINB = LPR == 2 ? 2 : LPR == 4 ? 3 : LPR == 8 ? 4 : 5;
-    static_assert(R * IPR == kIoThreads, "the I/O threads cover the rows");
+    static constexpr int MINB = IOW == 4 ? (LPR == 8 ? 3 : 2) : LPR == 2 ? 2 : LPR == 4 ? 3 : LPR == 8 ? 4 : 5;
+    static_assert(R * IPR == IOT && IP >= 2, "the I/O threads cover the rows, two steps or more each");
     static_assert(XR % 2 == 1, "odd row stride");
     static_assert(YQ >= kSteps && YQ % 4 == 0 && (WARP_SUM ? YR >= kSteps : YR >= LPR * YQ) && YR % 4 == 0,
                   "readout tile");
@@ -108,18 +110,20 @@ constexpr int kRawStages = 5;
 // slot, and a skip tile per tile stage ([row][step] floats after the ring)
 // carries D u from the widening to the readout. The trapezoidal rule uses the
 // same look-back slot (for u_{t-1}) and stages lambda_raw pieces as well.
-template <typename T, int LPR, int VAR = 0> struct Raw {
+template <typename T, int LPR, int VAR = 0, int IOW = 2> struct Raw {
     static constexpr bool CONV = VAR == 1, TRAP = VAR == 2;
-    using SH = Shape<LPR, TRAP>;
+    using SH = Shape<LPR, TRAP, IOW>;
+    static constexpr int IOT = SH::IOT;
     static constexpr int EB = static_cast<int>(sizeof(T));
     static constexpr int PB = SH::IP * EB;                           // bytes of one u/delta/z piece
     static constexpr int PS = (PB + 15) / 16;                        // slots per piece
     static constexpr int VE = 16 / EB;                               // elements per B/C piece
-    static constexpr int BC_PER = 2 * kStates * (kSteps / VE) / kIoThreads;   // B/C pieces per thread
+    static constexpr int BC_TOTAL = 2 * kStates * (kSteps / VE);            // B/C pieces per chunk
+    static constexpr int BC_PER = (BC_TOTAL + IOT - 1) / IOT;                 // B/C pieces per thread (at most)
     static constexpr int HALO = 3 * PS + BC_PER;                     // slot of the look-back (variants 1, 2)
     static constexpr int LAM = HALO + 1;                             // first slot of lambda_raw (variant 2)
     static constexpr int SLOTS = 3 * PS + BC_PER + (VAR ? 1 : 0) + (TRAP ? PS : 0);
-    static constexpr int STAGE = SLOTS * kIoThreads * 16;
+    static constexpr int STAGE = SLOTS * IOT * 16;
     // ring depth: shorter for the variants, whose larger slots, skip tiles
     // (prologue) or wider step tiles (trapezoidal) must still leave room for
     // 3 (LPR 4) CTAs per SM
@@ -130,14 +134,14 @@ template <typename T, int LPR, int VAR = 0> struct Raw {
     static constexpr int SK_OFF = OFF + RS * STAGE;
     static constexpr int SK_STAGE = SH::R * SKR * 4;
     static constexpr int BYTES = SK_OFF + (CONV ? kTileStages * SK_STAGE : 0);   // total dynamic shared memory
-    static_assert(BC_PER * kIoThreads * VE == 2 * kStates * kSteps, "B/C pieces split evenly");
+    static_assert(BC_TOTAL * VE == 2 * kStates * kSteps, "B/C pieces cover the tiles");
     static_assert(PB == 4 || PB == 8 || PB % 16 == 0, "piece sizes cp.async can copy");
     static_assert(VAR == 0 || (PB % 16 == 0 && VE >= 4), "look-back: 16-byte aligned pieces, >= 3 earlier inputs");
     static_assert(RA >= 1, "at least one chunk staged ahead");
 };
 
 // Named barriers (0 is __syncthreads): the producer arrives, the consumer
-// waits; kThreads threads complete each phase. 4 kTileStages + 1 <= 16.
+// waits; all NT threads of the CTA complete each phase. 4 kTileStages + 1 <= 16.
 //   XF(s): stage s's step and B/C tiles are ready       (I/O -> recurrence)
 //   XE(s): stage s's step and B/C tiles may be rewritten (recurrence -> I/O)
 //   YF(s): stage s's readout partials are ready          (recurrence -> I/O)
@@ -148,11 +152,11 @@ __device__ __forceinline__ int bar_yf(int s) { return 1 + 2 * kTileStages + s; }
 __device__ __forceinline__ int bar_ye(int s) { return 1 + 3 * kTileStages + s; }
 static_assert(4 * kTileStages + 1 <= 16, "named barriers per CTA");
 __device__ __forceinline__ int next_stage(int s, int n) { return s + 1 == n ? 0 : s + 1; }
-__device__ __forceinline__ void bar_wait(int id) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(kThreads) : "memory");
+template <int NT> __device__ __forceinline__ void bar_wait(int id) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(NT) : "memory");
 }
-__device__ __forceinline__ void bar_signal(int id) {
-    asm volatile("bar.arrive %0, %1;" ::"r"(id), "n"(kThreads) : "memory");
+template <int NT> __device__ __forceinline__ void bar_signal(int id) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "n"(NT) : "memory");
 }
 
 // ---- Work schedule ----------------------------------------------------------
@@ -200,64 +204,51 @@ __device__ __forceinline__ Sched make_sched(const ScanParams &p, int R) {
     return s;
 }
 
-// Position in a CTA's work: unit u (batch entry b, first row d0) and chunk c;
-// seg 0 = the start of unit ue, 1 = the whole units, 2 = the end of unit us.
-struct Cur {
-    int u, c, b, d0, seg;
+// The CTA's work as pieces, in processing order: piece 0 is the start of unit
+// ue, pieces 1 .. n-2 the whole units us+1 .. ue-1, piece n-1 the end of unit
+// us (a single piece when the range lies inside one unit).
+struct PieceRange {
+    int u, c0, c1;   // chunks [c0, c1) of unit u
+};
+__device__ __forceinline__ int num_pieces(const Sched &s) { return s.us == s.ue ? 1 : s.ue - s.us + 1; }
+__device__ __forceinline__ PieceRange piece_at(const Sched &s, int i) {
+    if (s.us == s.ue) return {s.us, s.cs, s.ce};
+    if (i == 0) return {s.ue, 0, s.ce};
+    if (i == s.ue - s.us) return {s.us, s.cs, s.nc};
+    return {s.us + i, 0, s.nc};
+}
+
+// A position in the CTA's list of chunks (piece i, chunk c of unit u); next()
+// reports when it enters a new piece, so that per-row data is looked up once
+// per piece rather than once per chunk.
+struct PCur {
+    int i, c, c1, u;
+    __device__ __forceinline__ void begin(const Sched &s) {
+        const PieceRange pr = piece_at(s, 0);
+        i = 0; c = pr.c0; c1 = pr.c1; u = pr.u;
+    }
+    __device__ __forceinline__ bool next(const Sched &s) {
+        if (++c < c1) return false;
+        if (++i < num_pieces(s)) {
+            const PieceRange pr = piece_at(s, i);
+            c = pr.c0; c1 = pr.c1; u = pr.u;
+        }
+        return true;
+    }
 };
 
-__device__ __forceinline__ void cur_unit(Cur &k, const Sched &s, int u, int R) {
-    k.u = u;
-    k.b = u / s.blocks;
-    k.d0 = (u - k.b * s.blocks) * R;
-}
-__device__ __forceinline__ int head_end(const Sched &s) { return s.us == s.ue ? s.ce : s.nc; }
-__device__ __forceinline__ Cur cur_begin(const Sched &s, int R) {
-    Cur k;
-    if (s.us == s.ue) {
-        k.seg = 2;
-        cur_unit(k, s, s.us, R);
-        k.c = s.cs;
-    } else {
-        k.seg = 0;
-        cur_unit(k, s, s.ue, R);
-        k.c = 0;
-    }
-    return k;
-}
-__device__ __forceinline__ void cur_next(Cur &k, const Sched &s, int R) {
-    ++k.c;
-    if (k.seg == 0) {
-        if (k.c == s.ce) {
-            if (s.us + 1 < s.ue) {
-                k.seg = 1;
-                cur_unit(k, s, s.us + 1, R);
-                k.c = 0;
-            } else {
-                k.seg = 2;
-                cur_unit(k, s, s.us, R);
-                k.c = s.cs;
-            }
-        }
-    } else if (k.seg == 1) {
-        if (k.c == s.nc) {
-            if (k.u + 1 < s.ue) {
-                cur_unit(k, s, k.u + 1, R);
-                k.c = 0;
-            } else {
-                k.seg = 2;
-                cur_unit(k, s, s.us, R);
-                k.c = s.cs;
-            }
-        }
-    } else if (k.c == head_end(s)) {
-        k.seg = 3;
-    }
-}
-// first / last chunk of the piece the cursor is in
-__device__ __forceinline__ bool cur_first(const Cur &k, const Sched &s) { return k.c == (k.seg == 2 ? s.cs : 0); }
-__device__ __forceinline__ bool cur_last(const Cur &k, const Sched &s) {
-    return k.c + 1 == (k.seg == 0 ? s.ce : k.seg == 1 ? s.nc : head_end(s));
+// Batch entry and (clamped) channel row of the thread's row r in unit u.
+struct UnitRow {
+    int64_t b, dc;
+    bool ok;
+};
+__device__ __forceinline__ UnitRow unit_row(const ScanParams &p, const Sched &s, int u, int R, int r) {
+    UnitRow x;
+    x.b = u / s.blocks;
+    const int64_t d = static_cast<int64_t>(u - static_cast<int>(x.b) * s.blocks) * R + r;
+    x.ok = d < p.dim;
+    x.dc = x.ok ? d : p.dim - 1;
+    return x;
 }
 
 // Carry hand-over between CTAs. The writer's threads store the states, fence,
@@ -416,9 +407,10 @@ __device__ __forceinline__ void store_piece(T *dst, const float (&v)[P], int64_t
 
 // The recurrence warps: lane (r, q) owns states q NPL .. q NPL + NPL - 1 of
 // row r of the unit being processed.
-template <typename T, int LPR, bool TRAP>
+template <typename T, int LPR, bool TRAP, int IOW>
 __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned char *smem, int tid) {
-    using S = Shape<LPR, TRAP>;
+    using S = Shape<LPR, TRAP, IOW>;
+    constexpr int NT = S::THREADS;
     constexpr int NPL = S::NPL, R = S::R;
     constexpr int NP = NPL > 1 ? NPL / 2 : 1;
     constexpr int RW = 32 / LPR;   // rows per warp
@@ -427,29 +419,26 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
     const int q = S::GROUP_MAJOR ? lane / RW : tid % LPR;
     const int dstate = static_cast<int>(p.dstate);
     const Sched sc = make_sched(p, R);
-    Cur kc = cur_begin(sc, R);
 
     // A log2(e) and the state of the lane's states, kept as the register pairs
     // the packed instructions take (no moves in the loop); set at the start of
     // every piece of work.
     float2 ap[NP], hp[NP];
     float2 bprev[NP];   // trapezoidal rule: the lane's B_{t-1} entries (B_{-1} u_{-1} = 0 via its coefficient)
-    bool ok = false;
-    int64_t row = 0;
-#pragma unroll
-    for (int j = 0; j < NP; ++j) ap[j] = hp[j] = bprev[j] = f2(0.f, 0.f);
-    int s = 0;   // tile stage of chunk it
-    for (int64_t it = 0; it < sc.K; ++it, s = next_stage(s, kTileStages), cur_next(kc, sc, R)) {
-        if (cur_first(kc, sc)) {
-            // a new piece: the rows of unit kc.u, entering state from the
-            // initial state (chunk 0) or from the CTA that ran the unit's start
-            const int64_t d = static_cast<int64_t>(kc.d0) + r;
-            ok = d < p.dim;
-            const int64_t dc = ok ? d : p.dim - 1;    // clamped row: loads stay in bounds
-            row = static_cast<int64_t>(kc.b) * p.dim + dc;
-            const bool carried = kc.c > 0;
-            if (carried) wait_carry(p, kc.u, tid);
-            const float *hsrc = carried ? p.sk_carry + (static_cast<int64_t>(kc.u) * R + r) * kStates
+    int s = 0;          // tile stage of chunk it
+    int64_t it = 0;     // position in the CTA's list of chunks
+    const int npieces = num_pieces(sc);
+    for (int pi = 0; pi < npieces; ++pi) {
+        const PieceRange pr = piece_at(sc, pi);
+        // the rows of unit pr.u, entering state from the initial state (chunk
+        // 0) or from the CTA that ran the unit's start
+        const UnitRow ur = unit_row(p, sc, pr.u, R, r);
+        const int64_t row = ur.b * p.dim + ur.dc;
+        const bool carried = pr.c0 > 0;
+        if (carried) wait_carry(p, pr.u, tid);
+        {
+            const int64_t dc = ur.dc;
+            const float *hsrc = carried ? p.sk_carry + (static_cast<int64_t>(pr.u) * R + r) * kStates
                                         : (p.h0 ? p.h0 + row * dstate : nullptr);
 #pragma unroll
             for (int j = 0; j < NP; ++j) {
@@ -467,6 +456,7 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
                 bprev[j] = f2(0.f, 0.f);
             }
         }
+        for (int c = pr.c0; c < pr.c1; ++c, ++it, s = next_stage(s, kTileStages)) {
         unsigned char *st = smem + s * S::STAGE;
         const float4 *xrow = reinterpret_cast<const float4 *>(st + S::X_OFF) + r * S::XR;
         float *yl = reinterpret_cast<float *>(st + S::Y_OFF) + r * S::YR + (S::WARP_SUM ? 0 : q * S::YQ);
@@ -487,8 +477,8 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
         };
         const float *Bl = reinterpret_cast<const float *>(st + S::B_OFF) + q * NPL;
         const float *Cl = reinterpret_cast<const float *>(st + S::C_OFF) + q * NPL;
-        bar_wait(bar_xf(s));
-        if (it >= kTileStages) bar_wait(bar_ye(s));
+        bar_wait<NT>(bar_xf(s));
+        if (it >= kTileStages) bar_wait<NT>(bar_ye(s));
 
         // Software pipelined over the chunk: step pairs are read one pair
         // ahead, B and C one step ahead, and the ex2 of step t + 1 is issued
@@ -546,21 +536,34 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
                 }
             }
         } else {
-        float4 xa = xrow[0], xb = xrow[1];   // steps (0, 1) and (2, 3)
-        float2 acur[NP];
-        decay(xa.x, acur);
-        StepIn<NPL> cur = load_bc_step<NPL>(Bl, Cl);
+        // B and C of step t + D and its exponentials are issued while step t
+        // runs (D = 2 when the lane holds 4 states or fewer, else 1), so that
+        // with one recurrence warp on a sub-partition neither the shared-memory
+        // nor the MUFU latency reaches the state's dependency chain. xw holds
+        // the step pairs t/2, t/2 + 1 and t/2 + 2 of the step tile.
+        constexpr int D = NPL <= 4 ? 2 : 1;
+        float4 xw[3] = {xrow[0], xrow[1], xrow[2]};
+        auto dlt = [&](int step, int t) -> float {
+            const float4 &w = xw[(step >> 1) - (t >> 1)];
+            return (step & 1) ? w.z : w.x;
+        };
+        StepIn<NPL> bq[D + 1];
+        float2 aq[D + 1][NP];
+#pragma unroll
+        for (int k = 0; k < D; ++k) {
+            bq[k] = load_bc_step<NPL>(Bl + k * kStates, Cl + k * kStates);
+            decay(dlt(k, 0), aq[k]);
+        }
         float outs[4];
 #pragma unroll
         for (int t = 0; t < kSteps; ++t) {
-            const bool odd = t & 1;
-            StepIn<NPL> nxt = cur;
-            float2 anxt[NP];
-            if (t + 1 < kSteps) {
-                nxt = load_bc_step<NPL>(Bl + (t + 1) * kStates, Cl + (t + 1) * kStates);
-                decay(odd ? xb.x : xa.z, anxt);
+            if (t + D < kSteps) {
+                bq[(t + D) % (D + 1)] = load_bc_step<NPL>(Bl + (t + D) * kStates, Cl + (t + D) * kStates);
+                decay(dlt(t + D, t), aq[(t + D) % (D + 1)]);
             }
-            const float du = odd ? xa.w : xa.y;
+            const StepIn<NPL> &cur = bq[t % (D + 1)];
+            const float2 (&acur)[NP] = aq[t % (D + 1)];
+            const float du = (t & 1) ? xw[0].w : xw[0].y;
             if constexpr (NPL == 1) {
                 hp[0].x = fmaf(acur[0].x, hp[0].x, du * cur.b[0].x);
                 outs[t & 3] = cur.c[0].x * hp[0].x;
@@ -574,40 +577,35 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
                 outs[t & 3] = acc.x + acc.y;
             }
             if ((t & 3) == 3) emit4(t - 3, outs);
-            if (t + 1 < kSteps) {
-                cur = nxt;
-#pragma unroll
-                for (int j = 0; j < NP; ++j) acur[j] = anxt[j];
-                if (odd) {   // the pair (t + 1, t + 2) becomes current; fetch (t + 3, t + 4)
-                    xa = xb;
-                    if (t + 3 < kSteps) xb = xrow[(t + 3) / 2];
-                }
+            if (t & 1) {   // the pair (t + 1, t + 2) becomes current
+                xw[0] = xw[1];
+                xw[1] = xw[2];
+                if ((t >> 1) + 3 < kSteps / 2) xw[2] = xrow[(t >> 1) + 3];
             }
         }
         }
-        if (it + kTileStages < sc.K) bar_signal(bar_xe(s));
-        bar_signal(bar_yf(s));
+        if (it + kTileStages < sc.K) bar_signal<NT>(bar_xe(s));
+        bar_signal<NT>(bar_yf(s));
+        }
 
-        if (cur_last(kc, sc)) {
-            if (kc.c + 1 == sc.nc) {   // the end of the sequence: the final state
-                if (ok && p.hT) {
-#pragma unroll
-                    for (int i = 0; i < NPL; ++i) {
-                        const int n = q * NPL + i;
-                        if (n < dstate) p.hT[row * dstate + n] = (i & 1) ? hp[i / 2].y : hp[i / 2].x;
-                    }
-                }
-            } else {   // hand the state over to the CTA that continues this unit
-                float *dst = p.sk_carry + (static_cast<int64_t>(kc.u) * R + r) * kStates;
+        if (pr.c1 == sc.nc) {   // the end of the sequence: the final state
+            if (ur.ok && p.hT) {
 #pragma unroll
                 for (int i = 0; i < NPL; ++i) {
                     const int n = q * NPL + i;
-                    if (n < dstate) dst[n] = (i & 1) ? hp[i / 2].y : hp[i / 2].x;
+                    if (n < dstate) p.hT[row * dstate + n] = (i & 1) ? hp[i / 2].y : hp[i / 2].x;
                 }
-                __threadfence();
-                rec_bar(kBarRecB);
-                if (tid == 0) st_release(p.sk_flag + kc.u, 1);
             }
+        } else {   // hand the state over to the CTA that continues this unit
+            float *dst = p.sk_carry + (static_cast<int64_t>(pr.u) * R + r) * kStates;
+#pragma unroll
+            for (int i = 0; i < NPL; ++i) {
+                const int n = q * NPL + i;
+                if (n < dstate) dst[n] = (i & 1) ? hp[i / 2].y : hp[i / 2].x;
+            }
+            __threadfence();
+            rec_bar(kBarRecB);
+            if (tid == 0) st_release(p.sk_flag + pr.u, 1);
         }
     }
 }
@@ -617,11 +615,12 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
 // inputs travel through the ring RA chunks ahead of use (cp.async on
 // the aligned path, plain loads otherwise); a thread waits only for its own
 // copies, so the ring needs no barrier.
-template <typename T, int LPR, bool VEC, int VAR>
+template <typename T, int LPR, bool VEC, int VAR, int IOW>
 __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem, int i) {
     constexpr bool CONV = VAR == 1, TRAP = VAR == 2;
-    using S = Shape<LPR, TRAP>;
-    using RW = Raw<T, LPR, VAR>;
+    using S = Shape<LPR, TRAP, IOW>;
+    using RW = Raw<T, LPR, VAR, IOW>;
+    constexpr int NT = S::THREADS, IOT = S::IOT;
     constexpr int R = S::R, IP = S::IP, IPR = S::IPR, EB = RW::EB, PB = RW::PB, PS = RW::PS;
     constexpr int VE = RW::VE, BC_PER = RW::BC_PER;
     static_assert(IP % 2 == 0, "pieces hold step pairs");
@@ -632,25 +631,13 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     const int tk = k * IP;   // the thread's first step within a chunk
     const Sched sc = make_sched(p, R);
 
-    // The thread's row of a unit (clamped into range: loads stay in bounds).
-    struct RowCtx {
-        int64_t b, dc;
-        bool ok;
-    };
-    auto rowctx = [&](const Cur &kk) {
-        RowCtx x;
-        const int64_t d = static_cast<int64_t>(kk.d0) + r;
-        x.ok = d < p.dim;
-        x.dc = x.ok ? d : p.dim - 1;
-        x.b = kk.b;
-        return x;
-    };
-
     // The thread's B/C pieces: tensor (0 = B, 1 = C), state n, steps bt .. bt + VE - 1.
     int bc_off[BC_PER], bc_t[BC_PER], bc_n[BC_PER], bc_tensor[BC_PER];
+    bool bc_mine[BC_PER];
 #pragma unroll
     for (int j = 0; j < BC_PER; ++j) {
-        const int pc = i + j * kIoThreads;
+        const int pc = i + j * IOT;
+        bc_mine[j] = pc < RW::BC_TOTAL;
         bc_tensor[j] = pc / (kStates * (kSteps / VE));
         const int rem = pc % (kStates * (kSteps / VE));
         bc_n[j] = rem % kStates;
@@ -658,17 +645,58 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
         bc_off[j] = (bc_tensor[j] == 0 ? S::B_OFF : S::C_OFF) + (bc_t[j] * kStates + bc_n[j]) * 4;
     }
 
-    unsigned char *ring = smem + RW::OFF;
-    auto slot = [&](int rs, int sl) { return ring + rs * RW::STAGE + (sl * kIoThreads + i) * 16; };
+    // Per-piece data of the three steps, looked up when a step enters a new
+    // piece: the row's input pointers (at step tk of chunk 0) for staging; the
+    // bias (and convolution taps) for widening; the output pointer and D for
+    // finishing.
+    const T *srow[3], *lrow = nullptr, *bsrc[BC_PER];
+    auto stage_ctx = [&](int u) {
+        const UnitRow x = unit_row(p, sc, u, R, r);
+        srow[0] = static_cast<const T *>(p.u) + x.b * p.u_sb + x.dc * p.u_sd + tk;
+        srow[1] = static_cast<const T *>(p.delta) + x.b * p.dl_sb + x.dc * p.dl_sd + tk;
+        srow[2] = has_z ? static_cast<const T *>(p.z) + x.b * p.z_sb + x.dc * p.z_sd + tk : srow[0];
+        if constexpr (TRAP) lrow = static_cast<const T *>(p.lambda_raw) + x.b * p.lm_sb + x.dc * p.lm_sd + tk;
+#pragma unroll
+        for (int j = 0; j < BC_PER; ++j) {
+            const bool live = bc_mine[j] && bc_n[j] < dstate;
+            const T *base = bc_tensor[j] == 0 ? static_cast<const T *>(p.B) + x.b * p.B_sb
+                                              : static_cast<const T *>(p.C) + x.b * p.C_sb;
+            bsrc[j] = (live ? base + bc_n[j] * (bc_tensor[j] == 0 ? p.B_sn : p.C_sn) : base) + bc_t[j];
+        }
+    };
+    // Convolution taps right-aligned in a window of 4 (leading taps beyond
+    // the width stay 0): cw[3] weighs the current input.
+    float bias = 0.f, cw[4] = {0.f, 0.f, 0.f, 0.f}, cb = 0.f, Dw = 0.f;
+    auto widen_ctx = [&](int u) {
+        const UnitRow x = unit_row(p, sc, u, R, r);
+        bias = p.delta_bias ? __ldg(p.delta_bias + x.dc) : 0.f;
+        if constexpr (CONV) {
+            const int K = p.conv_width;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (j >= 4 - K) cw[j] = __ldg(p.conv_w + x.dc * K + (j - (4 - K)));
+            cb = p.conv_b ? __ldg(p.conv_b + x.dc) : 0.f;
+            Dw = p.D ? __ldg(p.D + x.dc) : 0.f;
+        }
+    };
+    T *yrow = nullptr;
+    float Df = 0.f;
+    bool fok = false;
+    auto finish_ctx = [&](int u) {
+        const UnitRow x = unit_row(p, sc, u, R, r);
+        fok = x.ok;
+        Df = p.D ? __ldg(p.D + x.dc) : 0.f;
+        yrow = static_cast<T *>(p.y) + x.b * p.y_sb + x.dc * p.y_sd + tk;
+    };
 
-    // Issue the copies of the raw inputs of chunk kk into ring stage rs.
-    auto stage_chunk = [&](const Cur &kk, int rs) {
-        const RowCtx x = rowctx(kk);
-        const T *src_row[3] = {static_cast<const T *>(p.u) + x.b * p.u_sb + x.dc * p.u_sd + tk,
-                               static_cast<const T *>(p.delta) + x.b * p.dl_sb + x.dc * p.dl_sd + tk,
-                               has_z ? static_cast<const T *>(p.z) + x.b * p.z_sb + x.dc * p.z_sd + tk : nullptr};
-        const T *lrow = TRAP ? static_cast<const T *>(p.lambda_raw) + x.b * p.lm_sb + x.dc * p.lm_sd + tk : nullptr;
-        const int64_t t0 = static_cast<int64_t>(kk.c) * kSteps;
+    unsigned char *ring = smem + RW::OFF;
+    auto slot = [&](int rs, int sl) { return ring + rs * RW::STAGE + (sl * IOT + i) * 16; };
+
+    // Issue the copies of the raw inputs of chunk c (of the staging step's
+    // piece) into ring stage rs.
+    auto stage_chunk = [&](int c, int rs) {
+        const T *const *src_row = srow;
+        const int64_t t0 = static_cast<int64_t>(c) * kSteps;
         const bool full = t0 + kSteps <= L;
         const int valid = full ? IP : static_cast<int>(min64(IP, max64(0, L - (t0 + tk))));
 #pragma unroll
@@ -729,17 +757,15 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
         }
 #pragma unroll
         for (int j = 0; j < BC_PER; ++j) {
+            if (!bc_mine[j]) continue;
             const bool live = bc_n[j] < dstate;
-            const T *base = bc_tensor[j] == 0 ? static_cast<const T *>(p.B) + x.b * p.B_sb
-                                              : static_cast<const T *>(p.C) + x.b * p.C_sb;
-            const T *bsrc = (live ? base + bc_n[j] * (bc_tensor[j] == 0 ? p.B_sn : p.C_sn) : base) + bc_t[j];
             const int vb = live ? (full ? VE : static_cast<int>(min64(VE, max64(0, L - (t0 + bc_t[j]))))) : 0;
             if constexpr (VEC) {
-                cp_async16(slot(rs, 3 * PS + j), vb > 0 ? static_cast<const void *>(bsrc + t0)
-                                                       : static_cast<const void *>(bsrc), vb * EB);
+                cp_async16(slot(rs, 3 * PS + j), vb > 0 ? static_cast<const void *>(bsrc[j] + t0)
+                                                       : static_cast<const void *>(bsrc[j]), vb * EB);
             } else {
                 Piece<T, VE> pc;
-                load_piece<T, VE, false>(pc, bsrc + t0, vb);
+                load_piece<T, VE, false>(pc, bsrc[j] + t0, vb);
                 *reinterpret_cast<uint4 *>(slot(rs, 3 * PS + j)) = make_uint4(pc.w[0], pc.w[1], pc.w[2], pc.w[3]);
             }
         }
@@ -765,13 +791,11 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     auto ring_piece = [&](int rs, int tsr) { return ring_slots(rs, tsr * PS); };
     // Readout of chunk c from tile stage s (u, z from ring stage rs): partial
     // sums + D u, gate, store.
-    auto finish = [&](const Cur &kk, int s, int rs) {
-        const RowCtx x = rowctx(kk);
-        const int64_t c = kk.c;
+    auto finish = [&](int c_, int s, int rs) {
+        const int64_t c = c_;
         const int64_t cnt = L - (c * kSteps + tk);
-        if (!x.ok || cnt <= 0) return;
-        const float Dd = p.D ? __ldg(p.D + x.dc) : 0.f;
-        T *yrow = static_cast<T *>(p.y) + x.b * p.y_sb + x.dc * p.y_sd + tk;
+        if (!fok || cnt <= 0) return;
+        const float Dd = Df;
         const float *yp = reinterpret_cast<const float *>(smem + s * S::STAGE + S::Y_OFF) + r * S::YR + tk;
         float2 sum[IP / 2];
 #pragma unroll
@@ -821,21 +845,9 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     };
     // Chunk c's step tile (step pairs of delta, delta u) and B/C tiles from
     // ring stage rs into tile stage s.
-    auto widen = [&](const Cur &kk, int s, int rs) {
-        const RowCtx x = rowctx(kk);
-        const int64_t c = kk.c;
-        const float bias = p.delta_bias ? __ldg(p.delta_bias + x.dc) : 0.f;
-        // Convolution taps right-aligned in a window of 4 (leading taps beyond
-        // the width stay 0): cw[3] weighs the current input.
-        float cw[4] = {0.f, 0.f, 0.f, 0.f}, cb = 0.f, Dd = 0.f;
-        if constexpr (CONV) {
-            const int K = p.conv_width;
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (j >= 4 - K) cw[j] = __ldg(p.conv_w + x.dc * K + (j - (4 - K)));
-            cb = p.conv_b ? __ldg(p.conv_b + x.dc) : 0.f;
-            Dd = p.D ? __ldg(p.D + x.dc) : 0.f;
-        }
+    auto widen = [&](int c_, int s, int rs) {
+        const int64_t c = c_;
+        const float Dd = Dw;
         unsigned char *st = smem + s * S::STAGE;
         float4 *xrow = reinterpret_cast<float4 *>(st + S::X_OFF) + r * S::XR + (TRAP ? tk : tk / 2);
         const Piece<T, IP> xin = ring_piece(rs, 0), dl = ring_piece(rs, 1);
@@ -902,6 +914,7 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
         }
 #pragma unroll
         for (int j = 0; j < BC_PER; ++j) {
+            if (!bc_mine[j]) continue;
             const uint4 w = *reinterpret_cast<const uint4 *>(slot(rs, 3 * PS + j));
             Piece<T, VE> pc;
             pc.w[0] = w.x; pc.w[1] = w.y; pc.w[2] = w.z; pc.w[3] = w.w;
@@ -919,12 +932,18 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     // (empty past the end: the count stays uniform). Each of the three steps
     // follows the CTA's work with its own cursor.
     const int64_t K = sc.K;
-    Cur ka = cur_begin(sc, R), kw = ka, kf = ka;
+    PCur ka, kw, kf;
+    ka.begin(sc);
+    kw = ka;
+    kf = ka;
+    stage_ctx(ka.u);
+    widen_ctx(kw.u);
+    finish_ctx(kf.u);
 #pragma unroll
     for (int c0 = 0; c0 < RW::RA; ++c0) {
         if (c0 < K) {
-            stage_chunk(ka, c0);
-            cur_next(ka, sc, R);
+            stage_chunk(ka.c, c0);
+            if (ka.next(sc)) stage_ctx(ka.u);
         }
         cp_async_commit();
     }
@@ -933,93 +952,109 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     int ra = RW::RA % RW::RS;             // ring stage of chunk it + RA
     for (int64_t it = 0; it < K; ++it) {
         cp_async_wait<RW::RA - 1>();      // chunk it's copies have landed
-        if (it >= kTileStages) bar_wait(bar_xe(s));
-        widen(kw, s, rs);
-        bar_signal(bar_xf(s));
+        if (it >= kTileStages) bar_wait<NT>(bar_xe(s));
+        widen(kw.c, s, rs);
+        bar_signal<NT>(bar_xf(s));
         const int64_t j = it - (kTileStages - 1);
         if (j >= 0) {
-            bar_wait(bar_yf(sf));
-            finish(kf, sf, rf);
-            if (j + kTileStages < K) bar_signal(bar_ye(sf));
+            bar_wait<NT>(bar_yf(sf));
+            finish(kf.c, sf, rf);
+            if (j + kTileStages < K) bar_signal<NT>(bar_ye(sf));
             sf = next_stage(sf, kTileStages);
             rf = next_stage(rf, RW::RS);
-            cur_next(kf, sc, R);
+            if (kf.next(sc)) finish_ctx(kf.u);
         }
         if (it + RW::RA < K) {
-            stage_chunk(ka, ra);
-            cur_next(ka, sc, R);
+            stage_chunk(ka.c, ra);
+            if (ka.next(sc)) stage_ctx(ka.u);
         }
         cp_async_commit();
         s = next_stage(s, kTileStages);
         rs = next_stage(rs, RW::RS);
         ra = next_stage(ra, RW::RS);
-        cur_next(kw, sc, R);
+        if (kw.next(sc)) widen_ctx(kw.u);
     }
     for (int64_t j = max64(K - (kTileStages - 1), 0); j < K; ++j) {
-        bar_wait(bar_yf(sf));
-        finish(kf, sf, rf);
+        bar_wait<NT>(bar_yf(sf));
+        finish(kf.c, sf, rf);
         sf = next_stage(sf, kTileStages);
         rf = next_stage(rf, RW::RS);
-        cur_next(kf, sc, R);
+        if (kf.next(sc)) finish_ctx(kf.u);
     }
     cp_async_wait<0>();
 }
 
-template <typename T, int LPR, bool VEC, int VAR>
-__global__ void __launch_bounds__(kThreads, Shape<LPR>::MINB) rec_kernel(const ScanParams p) {
+template <typename T, int LPR, bool VEC, int VAR, int IOW>
+__global__ void __launch_bounds__(Shape<LPR, VAR == 2, IOW>::THREADS, Shape<LPR, VAR == 2, IOW>::MINB)
+    rec_kernel(const ScanParams p) {
     extern __shared__ __align__(16) unsigned char smem[];
     if (threadIdx.x < kScanThreads) {
-        recurrence_role<T, LPR, VAR == 2>(p, smem, threadIdx.x);
+        recurrence_role<T, LPR, VAR == 2, IOW>(p, smem, threadIdx.x);
     } else {
-        io_role<T, LPR, VEC, VAR>(p, smem, threadIdx.x - kScanThreads);
+        io_role<T, LPR, VEC, VAR, IOW>(p, smem, threadIdx.x - kScanThreads);
     }
 }
 
-template <typename T, int LPR, int VAR>
+// Compiled variants: every lanes-per-row count with 2 I/O warps for the plain
+// scan, the convolution prologue (2 and 4 lanes) and the trapezoidal rule (2
+// and 4 lanes); 4 I/O warps for the plain scan with 2, 4 or 8 lanes.
+bool variant_compiled(int lpr, int variant, int iow) {
+    if (iow == 2) return variant == 0 || lpr == 2 || lpr == 4;
+    return iow == 4 && variant == 0 && (lpr == 2 || lpr == 4 || lpr == 8);
+}
+
+template <typename T, int LPR, int VAR, int IOW>
 const void *rec_ptr_v(bool vec) {
-    return vec ? reinterpret_cast<const void *>(rec_kernel<T, LPR, true, VAR>)
-               : reinterpret_cast<const void *>(rec_kernel<T, LPR, false, VAR>);
+    return vec ? reinterpret_cast<const void *>(rec_kernel<T, LPR, true, VAR, IOW>)
+               : reinterpret_cast<const void *>(rec_kernel<T, LPR, false, VAR, IOW>);
 }
 
 template <typename T, int LPR>
-const void *rec_ptr(bool vec, int variant) {
+const void *rec_ptr(bool vec, int variant, int iow) {
+    if constexpr (LPR != 16) {
+        if (iow == 4) return rec_ptr_v<T, LPR, 0, 4>(vec);
+    }
     if constexpr (LPR == 2 || LPR == 4) {   // the variants need 16-byte pieces
-        if (variant == 1) return rec_ptr_v<T, LPR, 1>(vec);
-        if (variant == 2) return rec_ptr_v<T, LPR, 2>(vec);
+        if (variant == 1) return rec_ptr_v<T, LPR, 1, 2>(vec);
+        if (variant == 2) return rec_ptr_v<T, LPR, 2, 2>(vec);
     }
-    return rec_ptr_v<T, LPR, 0>(vec);
+    return rec_ptr_v<T, LPR, 0, 2>(vec);
 }
 
 template <typename T>
-const void *rec_select(int lpr, bool vec, int variant) {
+const void *rec_select(int lpr, bool vec, int variant, int iow) {
     switch (lpr) {
-        case 2: return rec_ptr<T, 2>(vec, variant);
-        case 4: return rec_ptr<T, 4>(vec, variant);
-        case 8: return rec_ptr<T, 8>(vec, variant);
-        default: return rec_ptr<T, 16>(vec, variant);
+        case 2: return rec_ptr<T, 2>(vec, variant, iow);
+        case 4: return rec_ptr<T, 4>(vec, variant, iow);
+        case 8: return rec_ptr<T, 8>(vec, variant, iow);
+        default: return rec_ptr<T, 16>(vec, variant, iow);
     }
 }
 
-const void *rec_kernel_for(int in_dtype, int lpr, bool vec, int variant) {
-    return in_dtype == 0 ? rec_select<float>(lpr, vec, variant) : rec_select<__nv_bfloat16>(lpr, vec, variant);
+const void *rec_kernel_for(int in_dtype, int lpr, bool vec, int variant, int iow) {
+    return in_dtype == 0 ? rec_select<float>(lpr, vec, variant, iow)
+                         : rec_select<__nv_bfloat16>(lpr, vec, variant, iow);
 }
 
 template <typename T, int LPR>
-int smem_bytes_lpr(int variant) {
-    if constexpr (LPR == 2 || LPR == 4) {
-        if (variant == 1) return Raw<T, LPR, 1>::BYTES;
-        if (variant == 2) return Raw<T, LPR, 2>::BYTES;
+int smem_bytes_lpr(int variant, int iow) {
+    if constexpr (LPR != 16) {
+        if (iow == 4) return Raw<T, LPR, 0, 4>::BYTES;
     }
-    return Raw<T, LPR, 0>::BYTES;
+    if constexpr (LPR == 2 || LPR == 4) {
+        if (variant == 1) return Raw<T, LPR, 1, 2>::BYTES;
+        if (variant == 2) return Raw<T, LPR, 2, 2>::BYTES;
+    }
+    return Raw<T, LPR, 0, 2>::BYTES;
 }
 
 template <typename T>
-int smem_bytes_t(int lpr, int variant) {
+int smem_bytes_t(int lpr, int variant, int iow) {
     switch (lpr) {
-        case 2: return smem_bytes_lpr<T, 2>(variant);
-        case 4: return smem_bytes_lpr<T, 4>(variant);
-        case 8: return smem_bytes_lpr<T, 8>(variant);
-        default: return smem_bytes_lpr<T, 16>(variant);
+        case 2: return smem_bytes_lpr<T, 2>(variant, iow);
+        case 4: return smem_bytes_lpr<T, 4>(variant, iow);
+        case 8: return smem_bytes_lpr<T, 8>(variant, iow);
+        default: return smem_bytes_lpr<T, 16>(variant, iow);
     }
 }
 
@@ -1027,31 +1062,31 @@ int smem_bytes_t(int lpr, int variant) {
 
 int rec_variant(const ScanParams &p) { return p.lambda_raw ? 2 : p.conv_w ? 1 : 0; }
 
-int rec_smem_bytes(int in_dtype, int lpr, int variant) {
-    return in_dtype == 0 ? smem_bytes_t<float>(lpr, variant) : smem_bytes_t<__nv_bfloat16>(lpr, variant);
+int rec_smem_bytes(int in_dtype, int lpr, int variant, int iow) {
+    return in_dtype == 0 ? smem_bytes_t<float>(lpr, variant, iow) : smem_bytes_t<__nv_bfloat16>(lpr, variant, iow);
 }
 
-bool rec_supports_variant(int lpr, int variant) { return variant == 0 || lpr == 2 || lpr == 4; }
+bool rec_supports_variant(int lpr, int variant, int iow) { return variant_compiled(lpr, variant, iow); }
 int rec_chunk() { return kSteps; }
-int rec_threads() { return kThreads; }
+int rec_threads(int iow) { return kScanThreads + 32 * iow; }
 int rec_rows(int lpr) { return kScanThreads / lpr; }
 
 // Resident CTAs per SM of a sequential kernel (cached per kernel; the
 // shared-memory bound when no device answers).
-int rec_ctas_per_sm(int in_dtype, int lpr, bool vec, int variant) {
+int rec_ctas_per_sm(int in_dtype, int lpr, bool vec, int variant, int iow) {
     constexpr int kSlots = 64;
     static const void *keys[kSlots];
     static int vals[kSlots];
     static int used = 0;
     static std::mutex mu;
-    const void *k = rec_kernel_for(in_dtype, lpr, vec, variant);
+    const void *k = rec_kernel_for(in_dtype, lpr, vec, variant, iow);
     std::lock_guard<std::mutex> lk(mu);
     for (int i = 0; i < used; ++i)
         if (keys[i] == k) return vals[i];
-    const int smem = rec_smem_bytes(in_dtype, lpr, variant);
+    const int smem = rec_smem_bytes(in_dtype, lpr, variant, iow);
     int n = 0;
     bool asked = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess &&
-                 cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, kThreads, smem) == cudaSuccess;
+                 cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, rec_threads(iow), smem) == cudaSuccess;
     if (!asked) {
         cudaGetLastError();
         n = (228 * 1024) / (smem + 1024);
@@ -1086,8 +1121,8 @@ void rec_bind_workspace(ScanParams &p, void *ws, int64_t units, int ctas) {
     p.sk_carry = reinterpret_cast<float *>(w + rec_persistent_clear_bytes(units));
 }
 
-int rec_max_ctas(const ScanParams &p, int in_dtype, int lpr, bool vec, int num_sms) {
-    const int per_sm = rec_ctas_per_sm(in_dtype, lpr, vec, rec_variant(p));
+int rec_max_ctas(const ScanParams &p, int in_dtype, int lpr, bool vec, int num_sms, int iow) {
+    const int per_sm = rec_ctas_per_sm(in_dtype, lpr, vec, rec_variant(p), iow);
     const int64_t R = kScanThreads / lpr;
     const int64_t units = p.batch * ((p.dim + R - 1) / R);
     return static_cast<int>(min64(units, static_cast<int64_t>(per_sm) * num_sms));
@@ -1097,19 +1132,20 @@ int rec_max_ctas(const ScanParams &p, int in_dtype, int lpr, bool vec, int num_s
 // only if every CTA can be resident at once, so a CTA that waits for another
 // one's carry never waits for a CTA that has not started. The flags and the
 // status word are cleared on the stream first.
-cudaError_t launch_rec(const ScanParams &p, int lpr, bool vec, int in_dtype, cudaStream_t stream) {
+cudaError_t launch_rec(const ScanParams &p, int lpr, bool vec, int in_dtype, int iow, cudaStream_t stream) {
     const int variant = rec_variant(p);
-    if (!rec_supports_variant(lpr, variant) || (p.conv_w && p.lambda_raw)) return cudaErrorInvalidValue;
+    if (!rec_supports_variant(lpr, variant, iow) || (p.conv_w && p.lambda_raw)) return cudaErrorInvalidValue;
     if (p.sk_ctas > 0 && (variant == 2 || !p.sk_carry || !p.sk_flag || !p.sk_status)) return cudaErrorInvalidValue;
-    const void *k = rec_kernel_for(in_dtype, lpr, vec, variant);
-    const int smem = rec_smem_bytes(in_dtype, lpr, variant);
+    const void *k = rec_kernel_for(in_dtype, lpr, vec, variant, iow);
+    const int smem = rec_smem_bytes(in_dtype, lpr, variant, iow);
+    const int threads = rec_threads(iow);
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const int R = kScanThreads / lpr;
     void *args[] = {const_cast<ScanParams *>(&p)};
     if (p.sk_ctas == 0) {
         const dim3 grid(static_cast<unsigned>((p.dim + R - 1) / R), static_cast<unsigned>(p.batch));
-        e = cudaLaunchKernel(k, grid, dim3(kThreads), args, static_cast<size_t>(smem), stream);
+        e = cudaLaunchKernel(k, grid, dim3(threads), args, static_cast<size_t>(smem), stream);
         if (e != cudaSuccess) return e;
         return cudaGetLastError();
     }
@@ -1117,7 +1153,7 @@ cudaError_t launch_rec(const ScanParams &p, int lpr, bool vec, int in_dtype, cud
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(static_cast<unsigned>(p.sk_ctas));
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(threads);
     cfg.dynamicSmemBytes = static_cast<size_t>(smem);
     cfg.stream = stream;
     cudaLaunchAttribute attr{};

@@ -13,12 +13,15 @@
 // bound by HBM bandwidth (~168 MB of state traffic per step for 256 x 5120 x
 // 16), so the kernel is built to keep many bytes in flight with few
 // instructions per byte. The grid is (dim blocks, batch): no index division.
-// Four consecutive threads share a row (b, d); thread q owns state entries
-// [4q, 4q+4), so every state access is a fully coalesced 16-byte load and
-// store and its A, B and C entries arrive as one vector load each. (A thread
-// may own several rows, kRowGroups apart, loading all of them before
-// computing; one row per thread at full occupancy measured faster.) The
-// partial readouts are summed with two butterfly shuffles.
+// With 16 states, two consecutive threads share a row (b, d): thread q owns
+// the float4 pieces q and q + 2 of the row's state, so each of its two
+// state loads (and stores) covers whole 32-byte sectors across the warp, it
+// keeps 32 bytes of state in flight, and the per-row work (softplus of the
+// step, skip, gate) is done twice per row instead of four times. (Measured on
+// B200 with the L2 flushed between steps: 38.8 us per step for 256 x 5120 x
+// 16, against 46.5 us with four threads per row and 49.3 us with one.) The
+// two partial readouts are summed with one shuffle. Other state sizes take a
+// scalar path with four threads per row.
 #include <type_traits>
 
 #include "device_math.cuh"
@@ -27,8 +30,9 @@
 namespace ms {
 namespace {
 
-constexpr int kRowGroups = 64;                // row groups per block (4 threads each)
-constexpr int kBlock = kRowGroups * 4;
+constexpr int kBlock = 256;
+constexpr int kRowGroups = kBlock / 4;         // rows per block on the scalar path (4 threads each)
+constexpr int kVecRows = kBlock / 2;           // rows per block on the vector path (2 threads each)
 
 template <typename T>
 __device__ __forceinline__ float ldg1(const void *base, int64_t i) {
@@ -69,91 +73,98 @@ __device__ __forceinline__ float conv_step(const UpdateParams &p, int64_t b, int
     return p.conv_silu ? silu(acc) : acc;
 }
 
-// VEC: dstate == 16 with state rows, A rows and B/C rows aligned for vector
-// access. A thread owns state entries [4q, 4q+4) of kRowsPerThread rows and
-// issues all of their loads before any arithmetic, so that enough bytes are in
-// flight to cover HBM latency.
-template <typename T, bool VEC, int kRowsPerThread, bool CONV>
+// dstate == 16, state rows, A rows and B/C rows aligned for vector access:
+// two threads per row, thread q owning the float4 pieces q and q + 2.
+template <typename T, bool CONV>
+__global__ void __launch_bounds__(kBlock) state_update_vec_kernel(const UpdateParams p) {
+    const int tid = threadIdx.x;
+    const int q = tid & 1;
+    const int64_t b = blockIdx.y;
+    const int64_t d = static_cast<int64_t>(blockIdx.x) * kVecRows + (tid >> 1);
+    const bool ok = d < p.dim;
+    const int64_t dc = ok ? d : p.dim - 1;
+    float4 *st = reinterpret_cast<float4 *>(p.state + b * p.s_sb + dc * p.s_sd);
+    const float4 *ar = reinterpret_cast<const float4 *>(p.A + dc * 16);
+    // every load first, so that 32 bytes of state per thread are in flight
+    const float4 h0 = st[q], h1 = st[q + 2];
+    const float4 a0 = __ldg(ar + q), a1 = __ldg(ar + q + 2);
+    float x = ldg1<T>(p.x, b * p.x_sb + dc);
+    const float dt = ldg1<T>(p.delta, b * p.dl_sb + dc);
+    const float4 B0 = ldg4<T>(static_cast<const T *>(p.B) + b * p.B_sb + 4 * q);
+    const float4 B1 = ldg4<T>(static_cast<const T *>(p.B) + b * p.B_sb + 4 * q + 8);
+    const float4 C0 = ldg4<T>(static_cast<const T *>(p.C) + b * p.C_sb + 4 * q);
+    const float4 C1 = ldg4<T>(static_cast<const T *>(p.C) + b * p.C_sb + 4 * q + 8);
+    if constexpr (CONV) {
+        // the row's first lane steps the convolution state; u reaches the
+        // other lane of the row by shuffle
+        float u = 0.f;
+        if (q == 0) u = conv_step<T>(p, b, dc, x, ok);
+        x = __shfl_sync(0xffffffffu, u, (tid & 31) & ~1);
+    }
+    float v = dt;
+    if (p.delta_bias) v += __ldg(p.delta_bias + dc);
+    if (p.softplus) v = softplus(v);
+    const float v2 = v * kLog2e, dtx = v * x;
+    float4 o0, o1;
+    o0.x = fmaf(ex2_approx(v2 * a0.x), h0.x, dtx * B0.x);
+    o0.y = fmaf(ex2_approx(v2 * a0.y), h0.y, dtx * B0.y);
+    o0.z = fmaf(ex2_approx(v2 * a0.z), h0.z, dtx * B0.z);
+    o0.w = fmaf(ex2_approx(v2 * a0.w), h0.w, dtx * B0.w);
+    o1.x = fmaf(ex2_approx(v2 * a1.x), h1.x, dtx * B1.x);
+    o1.y = fmaf(ex2_approx(v2 * a1.y), h1.y, dtx * B1.y);
+    o1.z = fmaf(ex2_approx(v2 * a1.z), h1.z, dtx * B1.z);
+    o1.w = fmaf(ex2_approx(v2 * a1.w), h1.w, dtx * B1.w);
+    if (ok) {
+        st[q] = o0;
+        st[q + 2] = o1;
+    }
+    float acc = fmaf(C0.x, o0.x, fmaf(C0.y, o0.y, fmaf(C0.z, o0.z, C0.w * o0.w)));
+    acc = fmaf(C1.x, o1.x, fmaf(C1.y, o1.y, fmaf(C1.z, o1.z, fmaf(C1.w, o1.w, acc))));
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    if (ok && q == 0) {
+        float yv = acc + (p.D ? __ldg(p.D + dc) * x : 0.f);
+        if (p.z) yv *= silu(ldg1<T>(p.z, b * p.z_sb + dc));
+        static_cast<T *>(p.y)[b * p.y_sb + dc] = from_f32<T>(yv);
+    }
+}
+
+// Any dstate <= 16 or unaligned rows: four threads per row, thread q taking
+// the states n = q, q + 4, ... with scalar accesses.
+template <typename T, bool CONV>
 __global__ void __launch_bounds__(kBlock) state_update_kernel(const UpdateParams p) {
-    constexpr int kRowsPerBlock = kRowGroups * kRowsPerThread;
     const int tid = threadIdx.x;
     const int q = tid & 3;
     const int64_t b = blockIdx.y;
-    const int64_t d0 = static_cast<int64_t>(blockIdx.x) * kRowsPerBlock + (tid >> 2);
+    const int64_t d = static_cast<int64_t>(blockIdx.x) * kRowGroups + (tid >> 2);
     const int dstate = static_cast<int>(p.dstate);
-
-    int64_t dd[kRowsPerThread];
-    bool ok[kRowsPerThread];
-    float x[kRowsPerThread], dt[kRowsPerThread];
-#pragma unroll
-    for (int k = 0; k < kRowsPerThread; ++k) {
-        const int64_t d = d0 + k * kRowGroups;
-        ok[k] = d < p.dim;
-        dd[k] = ok[k] ? d : p.dim - 1;
-        x[k] = ldg1<T>(p.x, b * p.x_sb + dd[k]);
-        dt[k] = ldg1<T>(p.delta, b * p.dl_sb + dd[k]);
-        if constexpr (CONV) {
-            // the row's first lane steps the convolution state; u reaches the
-            // other three lanes of the row by shuffle
-            float u = 0.f;
-            if (q == 0) u = conv_step<T>(p, b, dd[k], x[k], ok[k]);
-            x[k] = __shfl_sync(0xffffffffu, u, (tid & 31) & ~3);
-        }
+    const bool ok = d < p.dim;
+    const int64_t dc = ok ? d : p.dim - 1;
+    float x = ldg1<T>(p.x, b * p.x_sb + dc);
+    const float dt = ldg1<T>(p.delta, b * p.dl_sb + dc);
+    if constexpr (CONV) {
+        float u = 0.f;
+        if (q == 0) u = conv_step<T>(p, b, dc, x, ok);
+        x = __shfl_sync(0xffffffffu, u, (tid & 31) & ~3);
     }
-    if constexpr (VEC) {
-        float4 h[kRowsPerThread], a[kRowsPerThread];
-#pragma unroll
-        for (int k = 0; k < kRowsPerThread; ++k) {
-            h[k] = reinterpret_cast<const float4 *>(p.state + b * p.s_sb + dd[k] * p.s_sd)[q];
-            a[k] = __ldg(reinterpret_cast<const float4 *>(p.A + dd[k] * 16) + q);
-        }
-        const float4 Bv = ldg4<T>(static_cast<const T *>(p.B) + b * p.B_sb + 4 * q);
-        const float4 Cv = ldg4<T>(static_cast<const T *>(p.C) + b * p.C_sb + 4 * q);
-#pragma unroll
-        for (int k = 0; k < kRowsPerThread; ++k) {
-            float v = dt[k];
-            if (p.delta_bias) v += __ldg(p.delta_bias + dd[k]);
-            if (p.softplus) v = softplus(v);
-            const float dtx = v * x[k];
-            float4 o;
-            o.x = fmaf(ex2_approx(v * (a[k].x * kLog2e)), h[k].x, dtx * Bv.x);
-            o.y = fmaf(ex2_approx(v * (a[k].y * kLog2e)), h[k].y, dtx * Bv.y);
-            o.z = fmaf(ex2_approx(v * (a[k].z * kLog2e)), h[k].z, dtx * Bv.z);
-            o.w = fmaf(ex2_approx(v * (a[k].w * kLog2e)), h[k].w, dtx * Bv.w);
-            float acc = fmaf(Cv.x, o.x, fmaf(Cv.y, o.y, fmaf(Cv.z, o.z, Cv.w * o.w)));
-            if (ok[k]) reinterpret_cast<float4 *>(p.state + b * p.s_sb + dd[k] * p.s_sd)[q] = o;
-            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-            if (ok[k] && q == 0) {
-                float yv = acc + (p.D ? __ldg(p.D + dd[k]) * x[k] : 0.f);
-                if (p.z) yv *= silu(ldg1<T>(p.z, b * p.z_sb + dd[k]));
-                static_cast<T *>(p.y)[b * p.y_sb + dd[k]] = from_f32<T>(yv);
-            }
-        }
-    } else {
-#pragma unroll
-        for (int k = 0; k < kRowsPerThread; ++k) {
-            float v = dt[k];
-            if (p.delta_bias) v += __ldg(p.delta_bias + dd[k]);
-            if (p.softplus) v = softplus(v);
-            const float dtx = v * x[k];
-            float *st = p.state + b * p.s_sb + dd[k] * p.s_sd;
-            float acc = 0.f;
-            for (int n = q; n < dstate; n += 4) {
-                const float an = ex2_approx(v * (__ldg(p.A + dd[k] * dstate + n) * kLog2e));
-                float hn = st[n];
-                hn = fmaf(an, hn, dtx * ldg1<T>(p.B, b * p.B_sb + n));
-                acc = fmaf(ldg1<T>(p.C, b * p.C_sb + n), hn, acc);
-                if (ok[k]) st[n] = hn;
-            }
-            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-            if (ok[k] && q == 0) {
-                float yv = acc + (p.D ? __ldg(p.D + dd[k]) * x[k] : 0.f);
-                if (p.z) yv *= silu(ldg1<T>(p.z, b * p.z_sb + dd[k]));
-                static_cast<T *>(p.y)[b * p.y_sb + dd[k]] = from_f32<T>(yv);
-            }
-        }
+    float v = dt;
+    if (p.delta_bias) v += __ldg(p.delta_bias + dc);
+    if (p.softplus) v = softplus(v);
+    const float dtx = v * x;
+    float *st = p.state + b * p.s_sb + dc * p.s_sd;
+    float acc = 0.f;
+    for (int n = q; n < dstate; n += 4) {
+        const float an = ex2_approx(v * (__ldg(p.A + dc * dstate + n) * kLog2e));
+        float hn = st[n];
+        hn = fmaf(an, hn, dtx * ldg1<T>(p.B, b * p.B_sb + n));
+        acc = fmaf(ldg1<T>(p.C, b * p.C_sb + n), hn, acc);
+        if (ok) st[n] = hn;
+    }
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+    if (ok && q == 0) {
+        float yv = acc + (p.D ? __ldg(p.D + dc) * x : 0.f);
+        if (p.z) yv *= silu(ldg1<T>(p.z, b * p.z_sb + dc));
+        static_cast<T *>(p.y)[b * p.y_sb + dc] = from_f32<T>(yv);
     }
 }
 
@@ -164,16 +175,16 @@ cudaError_t launch_t(const UpdateParams &p, cudaStream_t stream) {
     const bool vec = p.dstate == 16 && al(p.state, 16) && (p.s_sb % 4) == 0 && (p.s_sd % 4) == 0 &&
                      al(p.A, 16) && al(p.B, 4 * eb) && al(p.C, 4 * eb) && (p.B_sb % 4) == 0 &&
                      (p.C_sb % 4) == 0;
-    constexpr int kRows = 1;   // rows per thread (occupancy beats per-thread batching here)
-    const dim3 grid(static_cast<unsigned>((p.dim + kRowGroups * kRows - 1) / (kRowGroups * kRows)),
-                    static_cast<unsigned>(p.batch));
     const bool conv = p.conv_w != nullptr;
-    if (vec)
-        conv ? state_update_kernel<T, true, kRows, true><<<grid, kBlock, 0, stream>>>(p)
-             : state_update_kernel<T, true, kRows, false><<<grid, kBlock, 0, stream>>>(p);
-    else
-        conv ? state_update_kernel<T, false, kRows, true><<<grid, kBlock, 0, stream>>>(p)
-             : state_update_kernel<T, false, kRows, false><<<grid, kBlock, 0, stream>>>(p);
+    if (vec) {
+        const dim3 grid(static_cast<unsigned>((p.dim + kVecRows - 1) / kVecRows), static_cast<unsigned>(p.batch));
+        conv ? state_update_vec_kernel<T, true><<<grid, kBlock, 0, stream>>>(p)
+             : state_update_vec_kernel<T, false><<<grid, kBlock, 0, stream>>>(p);
+    } else {
+        const dim3 grid(static_cast<unsigned>((p.dim + kRowGroups - 1) / kRowGroups), static_cast<unsigned>(p.batch));
+        conv ? state_update_kernel<T, true><<<grid, kBlock, 0, stream>>>(p)
+             : state_update_kernel<T, false><<<grid, kBlock, 0, stream>>>(p);
+    }
     return cudaGetLastError();
 }
 

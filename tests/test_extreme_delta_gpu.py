@@ -39,7 +39,7 @@ def _ms():
     return ms
 
 
-def _scan_case(regime, dtype, *, batch=2, dim=70, N=16, L=300, seed=0, steep_A=False):
+def _scan_case(regime, dtype, *, batch=2, dim=70, N=16, L=296, seed=0, steep_A=False):
     inp = make_scan_inputs(LAYER, batch=batch, dim=dim, dstate=N, seqlen=L, dtype=dtype, seed=seed)
     if regime == "edge_bias":
         inp["delta_bias"] = make_delta_regime((dim,), "edge", "f32", seed + 1)
