@@ -21,6 +21,7 @@ and the max-over-ranks reduction of the elapsed device time use NCCL.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -60,6 +61,9 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="long_context_131k", choices=sorted(SCAN_WORKLOADS))
+    ap.add_argument("--seqlen", type=int, default=0,
+                    help="override the headline workload's sequence length (0: the workload's own); used for "
+                         "profiler captures of a shortened long-context layer")
     ap.add_argument("--leg-workloads", default="mamba130m_layer,mamba1p4b_layer",
                     help="other scan workloads timed as legs (comma separated; empty: none)")
     ap.add_argument("--leg-steps", type=int, default=50, help="timed steps of each scan-workload leg")
@@ -529,6 +533,8 @@ def run_ours(args, dist: Dist):
     torch.cuda.set_device(dev)
     dist.init("nccl")
     w = SCAN_WORKLOADS[args.workload]
+    if args.seqlen:
+        w = dataclasses.replace(w, seqlen=args.seqlen)
     peaks = load_peaks()
     mufu = measure_mufu(peaks)
     lib = ms.load_library()

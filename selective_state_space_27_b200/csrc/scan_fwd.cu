@@ -597,10 +597,25 @@ double config_cost(const Config &c) {
 constexpr int kRecLanes[] = {2, 4, 8, 16, 2, 4, 8};
 constexpr int kRecIow[] = {2, 2, 2, 2, 4, 4, 4};
 constexpr int kNumRec = sizeof(kRecLanes) / sizeof(kRecLanes[0]);
-constexpr double kRecCost[] = {1.6, 1.9, 2.5, 4.2, 1.6, 1.9, 2.5};
-// Relative cost of the persistent schedule's bookkeeping (cursors, carry
+// SM clocks per (row, step) of a sequential configuration when m of its CTAs
+// share an SM (m = 1 .. 4; larger m takes the last entry), measured on B200
+// with bf16 Mamba-130M-, Mamba-1.4B- and 131k-token layers (the MUFU floor is
+// 18/16 = 1.125: 16 exponentials of the states plus the softplus and the gate).
+// One CTA alone on an SM leaves each sub-partition a single recurrence warp
+// and runs markedly slower per row.
+constexpr double kRecCycles[][4] = {
+    {2.4, 1.85, 1.85, 1.85},   // 2 lanes per row, 2 I/O warps
+    {3.16, 2.06, 1.92, 1.92},  // 4 lanes, 2 I/O warps
+    {5.6, 3.2, 3.2, 2.9},      // 8 lanes, 2 I/O warps
+    {9.0, 8.0, 6.5, 6.5},      // 16 lanes, 2 I/O warps
+    {2.04, 1.65, 1.65, 1.65},  // 2 lanes, 4 I/O warps
+    {2.89, 2.1, 2.1, 2.1},     // 4 lanes, 4 I/O warps
+    {5.3, 3.5, 3.2, 3.2},      // 8 lanes, 4 I/O warps
+};
+double rec_cycles(int ri, int64_t m) { return kRecCycles[ri][m < 1 ? 0 : m > 4 ? 3 : m - 1]; }
+// Relative cost of the persistent schedule's bookkeeping (piece table, carry
 // hand-over) per unit of work.
-constexpr double kRecPersistentCost = 1.02;
+constexpr double kRecPersistentCost = 1.01;
 // SM clocks per unit of the chunked kernels' cost model (measured: a
 // Mamba-130M layer on cfg 7, 11 warps, took 485k clocks for 1.30M units).
 constexpr double kChunkedClocksPerUnit = 0.372;
@@ -684,11 +699,10 @@ ScanPlan plan_scan(const ScanParams &p, int in_dtype, int force_segments, int nu
         }
     }
     // Sequential kernels: no segments; an SM runs its CTAs in waves of as many
-    // as are resident, every resident CTA adds one recurrence warp per
-    // sub-partition, and a lone CTA runs 1.4x slower per row than a shared SM.
+    // as are resident, at the measured clocks per (row, step) for that many
+    // CTAs per SM; with the persistent schedule every SM gets the same share.
     int rec = -1, rec_ctas = 0;
     if (force_segments <= 1 && p.dstate <= kMaxN) {
-        const double mufu = (kMaxN + 3) / 16.0;   // MUFU clocks per (row, step): 16 states + softplus + gate
         best *= kChunkedClocksPerUnit;
         for (int ri = 0; ri < kNumRec; ++ri) {
             const int lpr = kRecLanes[ri], iow = kRecIow[ri];
@@ -698,8 +712,8 @@ ScanPlan plan_scan(const ScanParams &p, int in_dtype, int force_segments, int nu
             const int64_t R = rec_rows(lpr);
             const int64_t ctas = p.batch * ((p.dim + R - 1) / R);
             const int64_t heavy = (ctas + sms - 1) / sms;
-            auto wave = [&](double m) {
-                return (m <= 1.0 ? 1.4 : m) * R * static_cast<double>(p.seqlen) * mufu * kRecCost[ri];
+            auto wave = [&](int64_t m) {   // m CTAs side by side on one SM, each R rows x L steps
+                return static_cast<double>(m) * R * static_cast<double>(p.seqlen) * rec_cycles(ri, m);
             };
             const double t = (heavy / per_sm) * wave(per_sm) + (heavy % per_sm ? wave(heavy % per_sm) : 0.0);
             if (t < best * 0.999) {
@@ -710,8 +724,8 @@ ScanPlan plan_scan(const ScanParams &p, int in_dtype, int force_segments, int nu
             // persistent schedule: m CTAs on every SM share the units' work exactly
             if (variant == 0 && p.batch * p.dim <= (int64_t(1) << 30) && (p.seqlen + 15) / 16 < (int64_t(1) << 30)) {
                 for (int m = 1; m <= per_sm && static_cast<int64_t>(m) * sms <= ctas; ++m) {
-                    const double tp = static_cast<double>(ctas) / (static_cast<double>(m) * sms) * wave(m) *
-                                      kRecPersistentCost;
+                    const double tp = static_cast<double>(ctas) * R * static_cast<double>(p.seqlen) / sms *
+                                      rec_cycles(ri, m) * kRecPersistentCost;
                     if (tp < best * 0.999) {
                         best = tp;
                         rec = ri;

@@ -117,9 +117,13 @@ template <typename T, int LPR, int VAR = 0, int IOW = 2> struct Raw {
     static constexpr int EB = static_cast<int>(sizeof(T));
     static constexpr int PB = SH::IP * EB;                           // bytes of one u/delta/z piece
     static constexpr int PS = (PB + 15) / 16;                        // slots per piece
-    static constexpr int VE = 16 / EB;                               // elements per B/C piece
-    static constexpr int BC_TOTAL = 2 * kStates * (kSteps / VE);            // B/C pieces per chunk
-    static constexpr int BC_PER = (BC_TOTAL + IOT - 1) / IOT;                 // B/C pieces per thread (at most)
+    static constexpr int VE = 16 / EB;                               // elements in 16 bytes
+    // B/C pieces: the chunk's 2 x kStates x kSteps B and C values split evenly
+    // over the I/O threads, at most 16 bytes (VE elements) a piece
+    static constexpr int VB = (2 * kStates * kSteps / IOT) < VE ? (2 * kStates * kSteps / IOT) : VE;
+    static constexpr int BCB = VB * EB;                                      // bytes per B/C piece
+    static constexpr int BC_TOTAL = 2 * kStates * (kSteps / VB);             // B/C pieces per chunk
+    static constexpr int BC_PER = BC_TOTAL / IOT;                            // B/C pieces per thread
     static constexpr int HALO = 3 * PS + BC_PER;                     // slot of the look-back (variants 1, 2)
     static constexpr int LAM = HALO + 1;                             // first slot of lambda_raw (variant 2)
     static constexpr int SLOTS = 3 * PS + BC_PER + (VAR ? 1 : 0) + (TRAP ? PS : 0);
@@ -134,23 +138,29 @@ template <typename T, int LPR, int VAR = 0, int IOW = 2> struct Raw {
     static constexpr int SK_OFF = OFF + RS * STAGE;
     static constexpr int SK_STAGE = SH::R * SKR * 4;
     static constexpr int BYTES = SK_OFF + (CONV ? kTileStages * SK_STAGE : 0);   // total dynamic shared memory
-    static_assert(BC_TOTAL * VE == 2 * kStates * kSteps, "B/C pieces cover the tiles");
+    static_assert(BC_PER * IOT == BC_TOTAL && BC_TOTAL * VB == 2 * kStates * kSteps && (BCB == 8 || BCB == 16),
+                  "B/C pieces of 8 or 16 bytes, as many for every I/O thread");
     static_assert(PB == 4 || PB == 8 || PB % 16 == 0, "piece sizes cp.async can copy");
     static_assert(VAR == 0 || (PB % 16 == 0 && VE >= 4), "look-back: 16-byte aligned pieces, >= 3 earlier inputs");
     static_assert(RA >= 1, "at least one chunk staged ahead");
 };
 
 // Named barriers (0 is __syncthreads): the producer arrives, the consumer
-// waits; all NT threads of the CTA complete each phase. 4 kTileStages + 1 <= 16.
-//   XF(s): stage s's step and B/C tiles are ready       (I/O -> recurrence)
-//   XE(s): stage s's step and B/C tiles may be rewritten (recurrence -> I/O)
-//   YF(s): stage s's readout partials are ready          (recurrence -> I/O)
-//   YE(s): stage s's readout tile may be rewritten       (I/O -> recurrence)
+// waits; all NT threads of the CTA complete each phase.
+//   XF(s): the chunk in stage s is widened: its step and B/C tiles are ready
+//          (I/O -> recurrence)
+//   YF(s): the recurrence is done with the chunk in stage s: its readout
+//          partials are ready (recurrence -> I/O)
+// A stage needs no "free again" barriers: the I/O warps widen chunk c only
+// after finishing chunk c - kTileStages (their own program order, one sync on
+// YF before it), so by the time the recurrence sees XF for chunk c the readout
+// tile it is about to overwrite has been read; and the I/O warps' sync on YF
+// for chunk c - kTileStages, which precedes the widening of chunk c, already
+// says that the recurrence has stopped reading that stage's step tile. (The
+// protocol is model-checked on the CPU against random schedules.)
 __device__ __forceinline__ int bar_xf(int s) { return 1 + s; }
-__device__ __forceinline__ int bar_xe(int s) { return 1 + kTileStages + s; }
-__device__ __forceinline__ int bar_yf(int s) { return 1 + 2 * kTileStages + s; }
-__device__ __forceinline__ int bar_ye(int s) { return 1 + 3 * kTileStages + s; }
-static_assert(4 * kTileStages + 1 <= 16, "named barriers per CTA");
+__device__ __forceinline__ int bar_yf(int s) { return 1 + kTileStages + s; }
+static_assert(2 * kTileStages + 1 <= 13, "named barriers per CTA (13 and 14 serve the recurrence warps)");
 __device__ __forceinline__ int next_stage(int s, int n) { return s + 1 == n ? 0 : s + 1; }
 template <int NT> __device__ __forceinline__ void bar_wait(int id) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(NT) : "memory");
@@ -478,7 +488,6 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
         const float *Bl = reinterpret_cast<const float *>(st + S::B_OFF) + q * NPL;
         const float *Cl = reinterpret_cast<const float *>(st + S::C_OFF) + q * NPL;
         bar_wait<NT>(bar_xf(s));
-        if (it >= kTileStages) bar_wait<NT>(bar_ye(s));
 
         // Software pipelined over the chunk: step pairs are read one pair
         // ahead, B and C one step ahead, and the ex2 of step t + 1 is issued
@@ -584,7 +593,6 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
             }
         }
         }
-        if (it + kTileStages < sc.K) bar_signal<NT>(bar_xe(s));
         bar_signal<NT>(bar_yf(s));
         }
 
@@ -622,7 +630,7 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     using RW = Raw<T, LPR, VAR, IOW>;
     constexpr int NT = S::THREADS, IOT = S::IOT;
     constexpr int R = S::R, IP = S::IP, IPR = S::IPR, EB = RW::EB, PB = RW::PB, PS = RW::PS;
-    constexpr int VE = RW::VE, BC_PER = RW::BC_PER;
+    constexpr int VE = RW::VE, VB = RW::VB, BCB = RW::BCB, BC_PER = RW::BC_PER;
     static_assert(IP % 2 == 0, "pieces hold step pairs");
     const int r = i / IPR, k = i % IPR;
     const int dstate = static_cast<int>(p.dstate);
@@ -630,39 +638,47 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     const bool has_z = p.z != nullptr;
     const int tk = k * IP;   // the thread's first step within a chunk
     const Sched sc = make_sched(p, R);
+    const int nfull = static_cast<int>(L / kSteps);   // chunks with all kSteps steps inside the sequence
 
-    // The thread's B/C pieces: tensor (0 = B, 1 = C), state n, steps bt .. bt + VE - 1.
-    int bc_off[BC_PER], bc_t[BC_PER], bc_n[BC_PER], bc_tensor[BC_PER];
-    bool bc_mine[BC_PER];
+    // The thread's B/C pieces: tensor (0 = B, 1 = C), state n, steps bt .. bt + VB - 1.
+    int bc_off[BC_PER], bc_t[BC_PER], bc_n[BC_PER], bc_tensor[BC_PER], bc_bytes[BC_PER];
 #pragma unroll
     for (int j = 0; j < BC_PER; ++j) {
         const int pc = i + j * IOT;
-        bc_mine[j] = pc < RW::BC_TOTAL;
-        bc_tensor[j] = pc / (kStates * (kSteps / VE));
-        const int rem = pc % (kStates * (kSteps / VE));
+        bc_tensor[j] = pc / (kStates * (kSteps / VB));
+        const int rem = pc % (kStates * (kSteps / VB));
         bc_n[j] = rem % kStates;
-        bc_t[j] = (rem / kStates) * VE;
+        bc_t[j] = (rem / kStates) * VB;
         bc_off[j] = (bc_tensor[j] == 0 ? S::B_OFF : S::C_OFF) + (bc_t[j] * kStates + bc_n[j]) * 4;
+        bc_bytes[j] = bc_n[j] < dstate ? BCB : 0;   // states past dstate read as zero
     }
 
     // Per-piece data of the three steps, looked up when a step enters a new
-    // piece: the row's input pointers (at step tk of chunk 0) for staging; the
-    // bias (and convolution taps) for widening; the output pointer and D for
-    // finishing.
+    // piece and then advanced chunk by chunk: the input pointers of the
+    // thread's steps of the chunk to stage; the bias (and convolution taps)
+    // for widening; the output pointer and D for finishing.
     const T *srow[3], *lrow = nullptr, *bsrc[BC_PER];
-    auto stage_ctx = [&](int u) {
+    auto stage_ctx = [&](int u, int c) {
         const UnitRow x = unit_row(p, sc, u, R, r);
-        srow[0] = static_cast<const T *>(p.u) + x.b * p.u_sb + x.dc * p.u_sd + tk;
-        srow[1] = static_cast<const T *>(p.delta) + x.b * p.dl_sb + x.dc * p.dl_sd + tk;
-        srow[2] = has_z ? static_cast<const T *>(p.z) + x.b * p.z_sb + x.dc * p.z_sd + tk : srow[0];
-        if constexpr (TRAP) lrow = static_cast<const T *>(p.lambda_raw) + x.b * p.lm_sb + x.dc * p.lm_sd + tk;
+        const int64_t t = static_cast<int64_t>(c) * kSteps + tk;
+        srow[0] = static_cast<const T *>(p.u) + x.b * p.u_sb + x.dc * p.u_sd + t;
+        srow[1] = static_cast<const T *>(p.delta) + x.b * p.dl_sb + x.dc * p.dl_sd + t;
+        srow[2] = has_z ? static_cast<const T *>(p.z) + x.b * p.z_sb + x.dc * p.z_sd + t : srow[0];
+        if constexpr (TRAP) lrow = static_cast<const T *>(p.lambda_raw) + x.b * p.lm_sb + x.dc * p.lm_sd + t;
 #pragma unroll
         for (int j = 0; j < BC_PER; ++j) {
-            const bool live = bc_mine[j] && bc_n[j] < dstate;
             const T *base = bc_tensor[j] == 0 ? static_cast<const T *>(p.B) + x.b * p.B_sb
                                               : static_cast<const T *>(p.C) + x.b * p.C_sb;
-            bsrc[j] = (live ? base + bc_n[j] * (bc_tensor[j] == 0 ? p.B_sn : p.C_sn) : base) + bc_t[j];
+            bsrc[j] = (bc_bytes[j] ? base + bc_n[j] * (bc_tensor[j] == 0 ? p.B_sn : p.C_sn) : base) + bc_t[j] +
+                      static_cast<int64_t>(c) * kSteps;
         }
+    };
+    auto stage_advance = [&]() {
+#pragma unroll
+        for (int t = 0; t < 3; ++t) srow[t] += kSteps;
+        if constexpr (TRAP) lrow += kSteps;
+#pragma unroll
+        for (int j = 0; j < BC_PER; ++j) bsrc[j] += kSteps;
     };
     // Convolution taps right-aligned in a window of 4 (leading taps beyond
     // the width stay 0): cw[3] weighs the current input.
@@ -682,34 +698,41 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     T *yrow = nullptr;
     float Df = 0.f;
     bool fok = false;
-    auto finish_ctx = [&](int u) {
+    auto finish_ctx = [&](int u, int c) {
         const UnitRow x = unit_row(p, sc, u, R, r);
         fok = x.ok;
         Df = p.D ? __ldg(p.D + x.dc) : 0.f;
-        yrow = static_cast<T *>(p.y) + x.b * p.y_sb + x.dc * p.y_sd + tk;
+        yrow = static_cast<T *>(p.y) + x.b * p.y_sb + x.dc * p.y_sd + static_cast<int64_t>(c) * kSteps + tk;
     };
 
     unsigned char *ring = smem + RW::OFF;
     auto slot = [&](int rs, int sl) { return ring + rs * RW::STAGE + (sl * IOT + i) * 16; };
 
-    // Issue the copies of the raw inputs of chunk c (of the staging step's
-    // piece) into ring stage rs.
+    // Issue the copies of the raw inputs of chunk c (the staging step's
+    // pointers point at it) into ring stage rs. Chunks inside the sequence
+    // take fixed-size copies; the ragged last chunk copies what exists and
+    // zero-fills the rest.
     auto stage_chunk = [&](int c, int rs) {
-        const T *const *src_row = srow;
+        const bool full = c < nfull;
         const int64_t t0 = static_cast<int64_t>(c) * kSteps;
-        const bool full = t0 + kSteps <= L;
         const int valid = full ? IP : static_cast<int>(min64(IP, max64(0, L - (t0 + tk))));
+        constexpr int SB = PB < 16 ? PB : 16;   // bytes per slot
+        // an in-bounds, aligned address for copies of zero bytes (nothing is read)
+        const void *const tbase[3] = {p.u, p.delta, has_z ? p.z : p.u};
 #pragma unroll
         for (int tsr = 0; tsr < 3; ++tsr) {
             if (tsr == 2 && !has_z) break;
-            const T *src = src_row[tsr] + t0;
+            const T *src = srow[tsr];
             if constexpr (VEC) {
 #pragma unroll
                 for (int sl = 0; sl < PS; ++sl) {
-                    const int have = valid * EB - sl * 16;
-                    const int bytes = have < 0 ? 0 : (have > (PB < 16 ? PB : 16) ? (PB < 16 ? PB : 16) : have);
+                    int bytes = SB;
+                    if (!full) {
+                        const int have = valid * EB - sl * 16;
+                        bytes = have < 0 ? 0 : (have > SB ? SB : have);
+                    }
                     const void *g = bytes > 0 ? static_cast<const void *>(reinterpret_cast<const unsigned char *>(src) + sl * 16)
-                                              : static_cast<const void *>(src_row[tsr]);
+                                              : tbase[tsr];
                     if constexpr (PB >= 16) cp_async16(slot(rs, tsr * PS + sl), g, bytes);
                     else cp_async_small<PB>(slot(rs, tsr * PS + sl), g, bytes);
                 }
@@ -722,14 +745,15 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
             }
         }
         if constexpr (TRAP) {
-            const T *src = lrow + t0;
+            const T *src = lrow;
             if constexpr (VEC) {
 #pragma unroll
                 for (int sl = 0; sl < PS; ++sl) {
                     const int have = valid * EB - sl * 16;
                     const int bytes = have < 0 ? 0 : (have > 16 ? 16 : have);
-                    cp_async16(slot(rs, RW::LAM + sl), bytes > 0 ? static_cast<const void *>(
-                                   reinterpret_cast<const unsigned char *>(src) + sl * 16) : static_cast<const void *>(lrow),
+                    cp_async16(slot(rs, RW::LAM + sl),
+                               bytes > 0 ? static_cast<const void *>(reinterpret_cast<const unsigned char *>(src) + sl * 16)
+                                         : p.lambda_raw,
                                bytes);
                 }
             } else {
@@ -746,7 +770,7 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
             // they lie before t = 0 and read as 0
             const int64_t th = t0 + tk - VE;
             const int hv = th < 0 ? 0 : static_cast<int>(min64(VE, max64(0, L - th)));
-            const T *hsrc = hv > 0 ? src_row[0] + t0 - VE : src_row[0];
+            const T *hsrc = hv > 0 ? srow[0] - VE : static_cast<const T *>(p.u);
             if constexpr (VEC) {
                 cp_async16(slot(rs, RW::HALO), hsrc, hv * EB);
             } else {
@@ -757,16 +781,18 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
         }
 #pragma unroll
         for (int j = 0; j < BC_PER; ++j) {
-            if (!bc_mine[j]) continue;
-            const bool live = bc_n[j] < dstate;
-            const int vb = live ? (full ? VE : static_cast<int>(min64(VE, max64(0, L - (t0 + bc_t[j]))))) : 0;
+            int bytes = bc_bytes[j];
+            if (!full && bytes) bytes = static_cast<int>(min64(VB, max64(0, L - (t0 + bc_t[j])))) * EB;
             if constexpr (VEC) {
-                cp_async16(slot(rs, 3 * PS + j), vb > 0 ? static_cast<const void *>(bsrc[j] + t0)
-                                                       : static_cast<const void *>(bsrc[j]), vb * EB);
+                const void *g = bytes > 0 ? static_cast<const void *>(bsrc[j]) : p.B;
+                if constexpr (BCB == 16) cp_async16(slot(rs, 3 * PS + j), g, bytes);
+                else cp_async_small<BCB>(slot(rs, 3 * PS + j), g, bytes);
             } else {
-                Piece<T, VE> pc;
-                load_piece<T, VE, false>(pc, bsrc[j] + t0, vb);
-                *reinterpret_cast<uint4 *>(slot(rs, 3 * PS + j)) = make_uint4(pc.w[0], pc.w[1], pc.w[2], pc.w[3]);
+                Piece<T, VB> pc;
+                load_piece<T, VB, false>(pc, bsrc[j], bytes / EB);
+#pragma unroll
+                for (int w = 0; w < Piece<T, VB>::W; ++w)
+                    reinterpret_cast<uint32_t *>(slot(rs, 3 * PS + j))[w] = pc.w[w];
             }
         }
     };
@@ -793,7 +819,7 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     // sums + D u, gate, store.
     auto finish = [&](int c_, int s, int rs) {
         const int64_t c = c_;
-        const int64_t cnt = L - (c * kSteps + tk);
+        const int64_t cnt = c_ < nfull ? IP : L - (c * kSteps + tk);
         if (!fok || cnt <= 0) return;
         const float Dd = Df;
         const float *yp = reinterpret_cast<const float *>(smem + s * S::STAGE + S::Y_OFF) + r * S::YR + tk;
@@ -841,7 +867,7 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
                 outv[e + 1] = yv.y;
             }
         }
-        store_piece<T, IP, VEC>(yrow + c * kSteps, outv, cnt);
+        store_piece<T, IP, VEC>(yrow, outv, cnt);
     };
     // Chunk c's step tile (step pairs of delta, delta u) and B/C tiles from
     // ring stage rs into tile stage s.
@@ -877,7 +903,7 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
 #pragma unroll
             for (int e = 0; e < IP; e += 2) u2[e / 2] = f2(elem(xin, e), elem(xin, e + 1));
         }
-        const bool full = (c + 1) * kSteps <= L;
+        const bool full = c_ < nfull;
         const int64_t cnt = L - (c * kSteps + tk);
         float uprev = 0.f;   // trapezoidal rule: u_{t-1} of the piece's first step
         Piece<T, IP> lam;
@@ -914,13 +940,17 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
         }
 #pragma unroll
         for (int j = 0; j < BC_PER; ++j) {
-            if (!bc_mine[j]) continue;
-            const uint4 w = *reinterpret_cast<const uint4 *>(slot(rs, 3 * PS + j));
-            Piece<T, VE> pc;
-            pc.w[0] = w.x; pc.w[1] = w.y; pc.w[2] = w.z; pc.w[3] = w.w;
+            Piece<T, VB> pc;
+            if constexpr (BCB == 16) {
+                const uint4 w = *reinterpret_cast<const uint4 *>(slot(rs, 3 * PS + j));
+                pc.w[0] = w.x; pc.w[1] = w.y; pc.w[2] = w.z; pc.w[3] = w.w;
+            } else {
+                const uint2 w = *reinterpret_cast<const uint2 *>(slot(rs, 3 * PS + j));
+                pc.w[0] = w.x; pc.w[1] = w.y;
+            }
             float *dst = reinterpret_cast<float *>(st + bc_off[j]);
 #pragma unroll
-            for (int e = 0; e < VE; ++e) dst[e * kStates] = elem(pc, e);
+            for (int e = 0; e < VB; ++e) dst[e * kStates] = elem(pc, e);
         }
     };
 
@@ -936,14 +966,22 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     ka.begin(sc);
     kw = ka;
     kf = ka;
-    stage_ctx(ka.u);
+    stage_ctx(ka.u, ka.c);
     widen_ctx(kw.u);
-    finish_ctx(kf.u);
+    finish_ctx(kf.u, kf.c);
+    auto stage_next = [&]() {
+        if (ka.next(sc)) stage_ctx(ka.u, ka.c);
+        else stage_advance();
+    };
+    auto finish_next = [&]() {
+        if (kf.next(sc)) finish_ctx(kf.u, kf.c);
+        else yrow += kSteps;
+    };
 #pragma unroll
     for (int c0 = 0; c0 < RW::RA; ++c0) {
         if (c0 < K) {
             stage_chunk(ka.c, c0);
-            if (ka.next(sc)) stage_ctx(ka.u);
+            stage_next();
         }
         cp_async_commit();
     }
@@ -952,21 +990,19 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     int ra = RW::RA % RW::RS;             // ring stage of chunk it + RA
     for (int64_t it = 0; it < K; ++it) {
         cp_async_wait<RW::RA - 1>();      // chunk it's copies have landed
-        if (it >= kTileStages) bar_wait<NT>(bar_xe(s));
         widen(kw.c, s, rs);
         bar_signal<NT>(bar_xf(s));
         const int64_t j = it - (kTileStages - 1);
         if (j >= 0) {
             bar_wait<NT>(bar_yf(sf));
             finish(kf.c, sf, rf);
-            if (j + kTileStages < K) bar_signal<NT>(bar_ye(sf));
             sf = next_stage(sf, kTileStages);
             rf = next_stage(rf, RW::RS);
-            if (kf.next(sc)) finish_ctx(kf.u);
+            finish_next();
         }
         if (it + RW::RA < K) {
             stage_chunk(ka.c, ra);
-            if (ka.next(sc)) stage_ctx(ka.u);
+            stage_next();
         }
         cp_async_commit();
         s = next_stage(s, kTileStages);
@@ -979,7 +1015,7 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
         finish(kf.c, sf, rf);
         sf = next_stage(sf, kTileStages);
         rf = next_stage(rf, RW::RS);
-        if (kf.next(sc)) finish_ctx(kf.u);
+        finish_next();
     }
     cp_async_wait<0>();
 }

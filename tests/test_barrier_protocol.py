@@ -30,13 +30,25 @@ import pytest
 
 TILE_STAGES = 3   # kTileStages in csrc/scan_rec.cu
 
+# The kernel's protocol has two barriers per tile stage s:
+#   F(s): the I/O warps have widened the chunk now in stage s (its step and B/C
+#         tiles are ready); the recurrence warps sync on it before each chunk;
+#   D(s): the recurrence warps are done with the chunk in stage s (its readout
+#         partials are ready); the I/O warps sync on it before finishing it.
+# The "stage is free again" conditions need no barrier of their own, because
+# the I/O warps widen chunk c only after finishing chunk c - S + 1 ... c - S's
+# readout (program order), and the recurrence warps finish chunk c before it
+# is overwritten: the I/O warps' sync on D(s) for chunk c precedes their
+# widening of chunk c + S. PROTOCOL = "fd" checks that; PROTOCOL = "four" is
+# the earlier protocol with separate "empty" barriers XE(s) and YE(s).
 
-def rec_warp(n, mut, S):
+
+def rec_warp(n, mut, S, protocol="fd"):
     """One recurrence warp's operations for a sequence of n chunks."""
     for c in range(n):
         s = c % S
         yield ("sync", ("XF", s))
-        if c >= S and mut != "no_ye_wait":
+        if protocol == "four" and c >= S and mut != "no_ye_wait":
             yield ("sync", ("YE", s))
         yield ("begin_read", ("X", s), c)
         yield ("begin_write", ("Y", s), c)
@@ -44,18 +56,18 @@ def rec_warp(n, mut, S):
             yield ("arrive", ("YF", s))
         yield ("end_read", ("X", s), c)
         yield ("end_write", ("Y", s), c)
-        if c + S < n or mut == "xe_always":
+        if protocol == "four" and (c + S < n or mut == "xe_always"):
             yield ("arrive", ("XE", s))
         if mut != "yf_before_write":
             yield ("arrive", ("YF", s))
 
 
-def io_warp(n, mut, S):
+def io_warp(n, mut, S, protocol="fd"):
     """One I/O warp's operations: widen chunk c, then finish chunk c - (S - 1)."""
-    lag = S - 1
+    lag = S - 1 if mut != "finish_lag_s" else S
     for c in range(n):
         s = c % S
-        if c >= S and mut != "no_xe_wait":
+        if protocol == "four" and c >= S and mut != "no_xe_wait":
             yield ("sync", ("XE", s))
         if mut == "xf_before_write":
             yield ("arrive", ("XF", s))
@@ -69,7 +81,7 @@ def io_warp(n, mut, S):
             yield ("sync", ("YF", sf))
             yield ("begin_read", ("Y", sf), j)
             yield ("end_read", ("Y", sf), j)
-            if j + S < n or (mut == "ye_one_extra" and j + S == n):
+            if protocol == "four" and (j + S < n or (mut == "ye_one_extra" and j + S == n)):
                 yield ("arrive", ("YE", sf))
     for j in range(max(n - lag, 0), n):
         sf = j % S
@@ -82,12 +94,12 @@ class Violation(Exception):
     pass
 
 
-def simulate(n, rec_warps, io_warps, mut=None, stages=TILE_STAGES, seed=0, bias=0.0):
+def simulate(n, rec_warps, io_warps, mut=None, stages=TILE_STAGES, seed=0, bias=0.0, protocol="fd"):
     """Run one random interleaving; raise Violation on a protocol error."""
     rng = random.Random(seed)
     S = stages
-    procs = [("rec", i, rec_warp(n, mut, S)) for i in range(rec_warps)] + \
-            [("io", i, io_warp(n, mut, S)) for i in range(io_warps)]
+    procs = [("rec", i, rec_warp(n, mut, S, protocol)) for i in range(rec_warps)] + \
+            [("io", i, io_warp(n, mut, S, protocol)) for i in range(io_warps)]
     total = 32 * (rec_warps + io_warps)
     count = {}        # barrier -> threads arrived in the current phase
     waiting = {}      # barrier -> set of blocked process indices
@@ -163,24 +175,34 @@ def simulate(n, rec_warps, io_warps, mut=None, stages=TILE_STAGES, seed=0, bias=
         raise Violation(f"barriers left with pending arrivals: {left}")
 
 
-def check_protocol(mut=None, stages=TILE_STAGES, rec_warps=4, io_warps=2, schedules=60):
+def check_protocol(mut=None, stages=TILE_STAGES, rec_warps=4, io_warps=2, schedules=60, protocol="fd"):
     for n in range(1, 14):
         for k in range(schedules):
-            simulate(n, rec_warps, io_warps, mut=mut, stages=stages, seed=1000 * n + k, bias=(k % 4) * 0.3)
+            simulate(n, rec_warps, io_warps, mut=mut, stages=stages, seed=1000 * n + k, bias=(k % 4) * 0.3,
+                     protocol=protocol)
 
 
 @pytest.mark.parametrize("io_warps", [2, 4])
-def test_protocol_holds(io_warps):
-    """The kernel's protocol, for 1 to 13 chunks, random interleavings (some
-    biased so that one role runs far ahead of the other)."""
-    check_protocol(io_warps=io_warps)
+@pytest.mark.parametrize("protocol", ["fd", "four"])
+def test_protocol_holds(io_warps, protocol):
+    """The kernel's protocol (and the earlier four-barrier one), for 1 to 13
+    chunks, random interleavings (some biased so that one role runs far ahead
+    of the other)."""
+    check_protocol(io_warps=io_warps, protocol=protocol)
 
 
-@pytest.mark.parametrize("mut", ["no_ye_wait", "no_xe_wait", "xf_before_write", "yf_before_write", "xe_always",
-                                 "finish_wrong_stage", "ye_one_extra"])
+@pytest.mark.parametrize("mut", ["xf_before_write", "yf_before_write", "finish_wrong_stage", "finish_lag_s"])
 def test_planted_mistakes_are_caught(mut):
+    """Mistakes in the two-barrier protocol; finishing S chunks behind instead
+    of S - 1 lets the I/O warps overwrite a step tile still being read."""
     with pytest.raises(Violation):
         check_protocol(mut=mut)
+
+
+@pytest.mark.parametrize("mut", ["no_ye_wait", "no_xe_wait", "xe_always", "ye_one_extra"])
+def test_planted_mistakes_four_barrier_protocol(mut):
+    with pytest.raises(Violation):
+        check_protocol(mut=mut, protocol="four")
 
 
 def test_two_stages():
