@@ -75,14 +75,16 @@ template <int LPR, bool TRAP = false, int IOW = 2> struct Shape {
     static constexpr int IPR = IOT / R;                 // I/O threads per row
     static constexpr int IP = kSteps / IPR;             // steps per I/O thread
     static constexpr bool GROUP_MAJOR = LPR <= 4;
-    // LPR 4: the four groups of a row sit in lanes r, r + 8, r + 16, r + 24 of
-    // one warp and sum their partial readouts with shuffles; the readout tile
-    // then holds one float per (row, step), YR floats per row (36: the 32
-    // stores of a warp fall on distinct banks).
-    static constexpr bool WARP_SUM = LPR == 4;
+    // LPR 4 and 8: the groups of a row sit in one warp (lanes r + 8 q, or 8 r +
+    // q) and sum their partial readouts with shuffles, LPR steps at a time; the
+    // readout tile then holds one float per (row, step), YR floats per row (36
+    // and 40: the stores of a warp fall on distinct banks).
+    static constexpr bool WARP_SUM = LPR == 4 || LPR == 8;
+    static constexpr int EW = WARP_SUM ? LPR : 4;      // steps per readout store
+    static constexpr int QSTRIDE = GROUP_MAJOR ? 32 / LPR : 1;   // lane distance between a row's groups
     static constexpr int XR = TRAP ? kSteps + 1 : kSteps / 2 + 1;   // float4 per row of the step tile
     static constexpr int YQ = LPR <= 4 ? 16 : 20;
-    static constexpr int YR = LPR == 2 ? 36 : LPR == 4 ? 36 : LPR == 8 ? 168 : 328;
+    static constexpr int YR = LPR == 2 ? 36 : LPR == 4 ? 36 : LPR == 8 ? 40 : 328;
     static constexpr int X_OFF = 0;
     static constexpr int Y_OFF = X_OFF + R * XR * 16;
     static constexpr int B_OFF = Y_OFF + R * YR * 4;
@@ -470,17 +472,27 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
         unsigned char *st = smem + s * S::STAGE;
         const float4 *xrow = reinterpret_cast<const float4 *>(st + S::X_OFF) + r * S::XR;
         float *yl = reinterpret_cast<float *>(st + S::Y_OFF) + r * S::YR + (S::WARP_SUM ? 0 : q * S::YQ);
-        // The partial readouts of steps t0 .. t0 + 3: stored per lane, or (LPR
-        // 4) summed over the row's four groups in a transposed reduction whose
-        // lane q keeps step t0 + q.
-        auto emit4 = [&](int t0, const float (&o)[4]) {
+        // The partial readouts of steps t0 .. t0 + EW - 1: stored per lane, or
+        // (LPR 4 and 8) summed over the row's LPR groups in a transposed
+        // reduction: each round a lane keeps half of its values, adds the
+        // partner group's copy of that half, and passes on the other half, so
+        // that after log2(LPR) rounds lane q holds the total of step t0 + q.
+        auto emit = [&](int t0, const float (&o)[S::EW]) {
             if constexpr (S::WARP_SUM) {
-                const bool hi = q & 2, lo = q & 1;
-                float k0 = hi ? o[2] : o[0], k1 = hi ? o[3] : o[1];
-                k0 += __shfl_xor_sync(0xffffffffu, hi ? o[0] : o[2], 16);
-                k1 += __shfl_xor_sync(0xffffffffu, hi ? o[1] : o[3], 16);
-                const float tot = (lo ? k1 : k0) + __shfl_xor_sync(0xffffffffu, lo ? k0 : k1, 8);
-                yl[t0 + q] = tot;
+                float v[LPR];
+#pragma unroll
+                for (int e = 0; e < LPR; ++e) v[e] = o[e];
+#pragma unroll
+                for (int half = LPR / 2; half >= 1; half /= 2) {
+                    const bool hi = q & half;
+#pragma unroll
+                    for (int e = 0; e < half; ++e) {
+                        const float keep = hi ? v[e + half] : v[e];
+                        const float send = hi ? v[e] : v[e + half];
+                        v[e] = keep + __shfl_xor_sync(0xffffffffu, send, S::QSTRIDE * half);
+                    }
+                }
+                yl[t0 + q] = v[0];
             } else {
                 *reinterpret_cast<float4 *>(yl + t0) = make_float4(o[0], o[1], o[2], o[3]);
             }
@@ -533,7 +545,7 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
                     }
                     outs[t & 3] = acc.x + acc.y;
                 }
-                if ((t & 3) == 3) emit4(t - 3, outs);
+                if ((t & 3) == 3) emit(t - 3, outs);
 #pragma unroll
                 for (int j = 0; j < NP; ++j) bprev[j] = cur.b[j];
                 if (t + 1 < kSteps) {
@@ -563,7 +575,7 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
             bq[k] = load_bc_step<NPL>(Bl + k * kStates, Cl + k * kStates);
             decay(dlt(k, 0), aq[k]);
         }
-        float outs[4];
+        float outs[S::EW];
 #pragma unroll
         for (int t = 0; t < kSteps; ++t) {
             if (t + D < kSteps) {
@@ -573,9 +585,10 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
             const StepIn<NPL> &cur = bq[t % (D + 1)];
             const float2 (&acur)[NP] = aq[t % (D + 1)];
             const float du = (t & 1) ? xw[0].w : xw[0].y;
+            constexpr int E = S::EW;
             if constexpr (NPL == 1) {
                 hp[0].x = fmaf(acur[0].x, hp[0].x, du * cur.b[0].x);
-                outs[t & 3] = cur.c[0].x * hp[0].x;
+                outs[t % E] = cur.c[0].x * hp[0].x;
             } else {
                 float2 acc;
 #pragma unroll
@@ -583,9 +596,9 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
                     hp[j] = fma2(acur[j], hp[j], mul2(f2(du, du), cur.b[j]));
                     acc = j == 0 ? mul2(cur.c[j], hp[j]) : fma2(cur.c[j], hp[j], acc);
                 }
-                outs[t & 3] = acc.x + acc.y;
+                outs[t % E] = acc.x + acc.y;
             }
-            if ((t & 3) == 3) emit4(t - 3, outs);
+            if (t % E == E - 1) emit(t - E + 1, outs);
             if (t & 1) {   // the pair (t + 1, t + 2) becomes current
                 xw[0] = xw[1];
                 xw[1] = xw[2];
