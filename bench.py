@@ -47,11 +47,17 @@ ROTATE = 3  # input sets cycled through so that each step reads inputs not resid
 # transcendental results 16, FP32 lanes 128.
 SMS_B200 = 148
 MUFU_PER_CLK = 16
-# DRAM bytes (read + write) per launch from an ncu capture of the named kernel
-# on the named workload (profiles/ holds the summary); any other kernel or
-# workload reports traffic null.
-NCU_TRAFFIC = {("mamba130m_layer", "rec_kernel<bf16, 4>"): 152333056 + 31869696,
-               ("mamba2_layer_d2048", "ssd_kernel"): 563163904 + 244780288}
+# DRAM bytes (read + write) per launch from one ncu capture of the kernel and
+# plan (scan: workload, plan configuration, CTAs) on that workload; profiles/
+# holds the summaries. Any other kernel, plan or workload reports traffic null.
+# The long-context layer was captured at 16,384 of its 131,072 steps (same rows,
+# same plan): its traffic is proportional to the steps, so the capture is scaled
+# by 8.
+NCU_TRAFFIC = {("long_context_131k", 14, 148): (505816832 + 150104320) * 8,
+               ("mamba130m_layer", 10, 296): 152303104 + 34911744,
+               ("mamba1p4b_layer", 10, 444): 813753600 + 252538112,
+               ("mamba2_layer_d2048", "ssd_kernel"): 563170560 + 243913472,
+               ("decode_b256_d5120", "state_update_vec_kernel"): 92143104 + 32728832}
 FP32_PER_CLK = 128
 
 
@@ -362,6 +368,7 @@ class ScanSetup:
                        else "scan_kernel")
         self.kernel_desc = (
             f"{self.kernel} (sequential, warp-specialised, {self.plan.lanes} lanes per row, "
+            f"{self.plan.warps_per_cta - 4} I/O warps, config {self.plan.config}, "
             + (f"persistent schedule over {self.plan.ctas} CTAs)" if self.plan.ctas else "one CTA per block of rows)")
             if kind == 1 else
             f"scan_kernel (chunked, config {self.plan.config}, {self.plan.warps_per_cta} warps, "
@@ -409,7 +416,7 @@ def scan_roofline(setup, us, mufu, peaks):
     return {
         "bound": "alu", "unit": "Tmufu/s", "achieved": c["mufu"] / t / 1e12, "peak": mufu["measured_per_s"] / 1e12,
         "frac": c["mufu"] / t / mufu["measured_per_s"],
-        "traffic": NCU_TRAFFIC.get((setup.w.name, setup.kernel)),
+        "traffic": NCU_TRAFFIC.get((setup.w.name, setup.plan.config, setup.plan.ctas)),
         "kernel": setup.kernel_desc,
         "peak_note": (f"measured: ex2.approx throughput of this device ({mufu['measured_per_clk_per_sm']:.2f} per clk "
                       f"per SM, mamba_probe_unit_throughput); nominal {SMS_B200} SMs x {MUFU_PER_CLK}/clk x "
@@ -924,12 +931,15 @@ def run_decode(args, dist: Dist, dev):
         "value": dist.world * elems / (hot_us * 1e-6), "us_per_step": hot_us,
         "value_l2_flushed": dist.world * elems / (cold_us * 1e-6), "us_per_step_l2_flushed": cold_us,
         "tokens": "8 seeded token sets cycled",
+        "kernel": "state_update_vec_kernel (dstate 16, two threads per row, float4 state pieces)",
         "roofline": {"bound": "hbm", "unit": "GB/s", "algorithmic_bytes_per_step": bytes_step,
                      "achieved_l2_flushed": bytes_step / (cold_us * 1e-6) / 1e9,
                      "achieved_back_to_back": bytes_step / (hot_us * 1e-6) / 1e9,
                      "peak": peaks["hbm_gbs"], "frac": bytes_step / (cold_us * 1e-6) / 1e9 / peaks["hbm_gbs"],
                      "peak_source": peaks["source"],
-                     "note": "frac uses the L2-flushed timing; back-to-back steps keep the 84 MB state in L2"},
+                     "traffic": NCU_TRAFFIC.get((w.name, "state_update_vec_kernel")),
+                     "note": "frac uses the L2-flushed timing; back-to-back steps keep the 84 MB state in L2; "
+                             "traffic counts the state write-back that leaves L2 during the launch"},
         "gpu_launches": n + nf,
     }
 
