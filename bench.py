@@ -721,8 +721,8 @@ def run_trap(args, dist: Dist, dev, w, sets, params, y, hT, counts, mufu_peak):
 
 def run_bwd(args, dist: Dist, dev, w, sets, params, counts, mufu_peak):
     """Time the scan backward (gradients for a seeded dy, recomputing the
-    states from 16-step checkpoints) on the headline workload, through the C
-    ABI with preallocated outputs and workspace."""
+    states from 8-step checkpoints) on the side workload, through the C ABI
+    with preallocated outputs and workspace."""
     import ctypes
 
     import torch

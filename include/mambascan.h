@@ -364,8 +364,8 @@ typedef struct ms_scan_bwd_args {
     float *dinitial_state;                                                    /* or NULL */
 } ms_scan_bwd_args;
 
-/* Device workspace for mamba_scan_bwd (the chunk checkpoints of the states:
- * batch * dim * ceil(seqlen / 16) * 16 floats). */
+/* Device workspace for mamba_scan_bwd (the states at every 8-step checkpoint:
+ * batch * dim * ceil(seqlen / 8) * 16 floats). */
 ms_status mamba_scan_bwd_workspace_size(const ms_scan_args *args, size_t *bytes);
 
 /*

@@ -462,6 +462,7 @@ ms_status mamba_scan_bwd(const ms_scan_args *args, const ms_scan_bwd_args *g, vo
     ms_status st = check_scan(args);
     if (st != MS_OK) return st;
     if (!g) return invalid("bwd is NULL");
+    if (args->seqlen > (int64_t(1) << 30)) return invalid("seqlen above 2^30 is not supported by the backward");
     if (!g->dy || !g->du || !g->ddelta || !g->dA || !g->dB || !g->dC)
         return invalid("dy, du, ddelta, dA, dB and dC are required");
     if ((args->z && !g->dz) || (args->D && !g->dD) || (args->delta_bias && !g->ddelta_bias))

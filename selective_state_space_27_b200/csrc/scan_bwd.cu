@@ -9,23 +9,32 @@
 //   ds_t = dy_t silu(z_t),  dz_t = dy_t s_t silu'(z_t)
 //   g_tn = ds_t C_tn + a_{t+1,n} g_{t+1,n}      (g_{L-1} also receives dh_T)
 //   dC_tn += ds_t h_tn, dB_tn += g_tn delta_t u_t      (summed over d)
-//   du_t = sum_n g_tn delta_t B_tn + ds_t D
-//   ddelta_t = sum_n g_tn (B_tn u_t + h_{t-1,n} a_tn A_n)  (* sigmoid(raw) under softplus)
+//   du_t = delta_t sum_n g_tn B_tn + ds_t D
+//   ddelta_t = u_t sum_n g_tn B_tn + sum_n g_tn h_{t-1,n} a_tn A_n  (* sigmoid(raw) under softplus)
 //   dA_n += g_tn h_{t-1,n} a_tn delta_t, dD += ds_t u_t, dh_0 = a_0 g_0.
 //
-// Design. A CTA owns 16 rows of one batch entry and runs one thread per
-// (row, state) chain (256 threads). Phase F walks the sequence forward in
-// chunks of 16 steps and writes each chunk's end state to a workspace (one
-// float per chain and chunk: 1/16 of the expanded state). Phase B walks the
-// chunks backward: it recomputes the chunk's 16 states from the previous
-// checkpoint into registers and runs the adjoint recurrence through them.
-// Per-(row, t) sums over the 16 states go through [row][step][state] tiles
-// in shared memory (written by the chain threads, summed by one thread per
-// (row, step) with four vector loads; both access patterns are free of bank
-// conflicts); the B and C
-// gradients are summed over the CTA's rows the same way and added to global
-// memory with atomics, as are the A, D and delta_bias gradients (sums over
-// the batch). The caller's reduction outputs are zeroed first.
+// Design. The lanes hold the state as the forward's sequential kernel does:
+// LPR lanes per channel row (4 or 8), each with 16 / LPR of its 16 states,
+// 32 / LPR rows per warp, four warps per CTA. Phase F runs the
+// recurrence forward and leaves the state at the end of every chunk of 8
+// steps in a workspace (one float per chain and chunk). Phase B walks the
+// chunks backward: it recomputes the chunk's 8 states and decays from the
+// previous checkpoint into registers, then runs the adjoint recurrence
+// through them. Every sum is a register reduction inside the warp:
+//   - per (row, step) sums over the states (s_t, sum g B, sum g h a A) are
+//     summed over the row's LPR lanes in a transposed shuffle reduction, so
+//     that lane q ends with the totals of steps q, q + LPR, ..., the steps
+//     whose scalar work (gate, softplus derivative, stores) it does;
+//   - per (step, state) sums over the rows (the B and C gradients) are summed
+//     over the warp's rows the same way, leaving each lane one (tensor,
+//     state) total per step, which it adds to global memory in one float4
+//     atomic add per 4 steps.
+// The warps are independent: each stages its own rows' per-chunk inputs
+// (delta, delta u, u, ds per row and step) and its own copy of the chunk's B
+// and C ([step][state]) in shared memory, read as broadcasts, and only
+// synchronises with itself. The checkpoint a chunk starts from is loaded one
+// chunk ahead. The A, D and delta_bias gradients are register sums added once
+// per row. The caller's reduction outputs are zeroed first.
 #include <type_traits>
 
 #include "device_math.cuh"
@@ -34,251 +43,436 @@
 namespace ms {
 namespace {
 
-constexpr int kRows = 16;       // rows per CTA
-constexpr int kN = 16;          // states per row (smaller dstate is zero-padded)
-constexpr int kT = 16;          // steps per chunk
-constexpr int kBwdThreads = kRows * kN;
+constexpr int kN = 16;                 // states per row (smaller dstate is zero-padded)
+constexpr int kW = 4;                  // warps per CTA
+constexpr int kT = 8;                  // steps per chunk (checkpoint interval)
+constexpr int kBwdThreads = kW * 32;
+constexpr int kBCL = kT * kN / 32;     // B (and C) entries a lane stages per chunk
+static_assert(kT * kN % 32 == 0 && 32 % kT == 0, "whole B/C entries per lane");
 
-template <typename T>
-__device__ __forceinline__ float ldv(const void *p, int64_t i) {
-    return to_f32<T>(static_cast<const T *>(p)[i]);
-}
+// Shared memory of a warp, in floats. Per row: delta, delta u, u and ds of
+// the chunk's steps at offsets 0, 8, 16, 24, rows 36 floats apart so that the
+// rows fall on distinct bank groups; then the B and C tiles, [step][state]
+// with steps 20 floats apart (the staging stores, eight steps of one state
+// per quarter-warp, hit distinct banks; the reads are broadcasts).
+constexpr int kF_DT = 0, kF_DU = kT, kF_U = 2 * kT, kF_DS = 3 * kT;
+constexpr int kXR = 4 * kT + 4;
+constexpr int kBS = kN + 4;
+constexpr int kBC = kT * kBS;
 
-// Sum over the 16 lanes of a half-warp (the 16 states of a row).
-__device__ __forceinline__ float half_warp_sum(float v) {
+template <int LPR> struct BwdShape {
+    static constexpr int NPL = kN / LPR;        // states per lane
+    static constexpr int NP = NPL / 2;          // ... as float2 pairs
+    static constexpr int RW = 32 / LPR;         // rows per warp
+    static constexpr int ROWS = kW * RW;        // rows per CTA
+    static constexpr int IPL = kT / LPR;        // steps a lane finishes per chunk
+    static constexpr int WARP_FLOATS = RW * kXR + 2 * kBC;
+    static constexpr int SMEM_FLOATS = kW * WARP_FLOATS;
+    static constexpr int MINB = LPR == 4 ? 3 : 4;
+    static_assert(LPR == 4 || LPR == 8, "4 or 8 lanes per row");
+    static_assert(2 * NPL == RW, "the row reduction leaves one value per lane");
+};
+
+// Transposed sum over the row's K lanes (the low lane bits, K a power of 2)
+// of v[0..K-1], partial sums of K consecutive steps: lane q returns the total
+// of step q. Each round a lane keeps half of its values, adds the partner's
+// copy of that half and passes on the other half.
+// With STRIDE > 1 the same over the lanes q STRIDE (the rows of a warp).
+template <int K, int STRIDE>
+__device__ __forceinline__ float transposed_sum(float (&v)[K], int q) {
 #pragma unroll
-    for (int o = 1; o < 16; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
+    for (int half = K / 2; half >= 1; half /= 2) {
+        const bool hi = q & half;
+#pragma unroll
+        for (int e = 0; e < half; ++e) {
+            const float keep = hi ? v[e + half] : v[e];
+            const float send = hi ? v[e] : v[e + half];
+            v[e] = keep + __shfl_xor_sync(0xffffffffu, send, half * STRIDE);
+        }
+    }
+    return v[0];
 }
 
-// Dynamic shared memory of a CTA, in floats. The per-row step tiles have rows
-// of 20 floats (16-byte aligned) so that a chain thread reads four steps of its
-// row with one vector load.
-constexpr int kTS = kT + 4;
-constexpr int kRT = kRows * kTS;                 // a [row][step] tile
-constexpr int kTN = kT * (kN + 1);               // a [step][state] tile
-// [step][row][state] tiles summed over the rows by one thread per (step, state):
-// rows 16 floats apart, steps 272, so that the two rows a warp writes and the
-// two steps a warp sums fall on disjoint banks
-constexpr int kBR = kN, kBT = kRows * kN + 16;
-constexpr int kRNT = kT * kBT;
-// [row][step][state] tiles summed over the states by one thread per (row, step):
-// steps 20 floats apart, rows 336 (both write and read patterns conflict free)
-constexpr int kQS = kN + 4, kQR = kT * kQS + 16;
-constexpr int kRTN = kRows * kQR;
-constexpr int kBwdSmemFloats = 4 * kRT + 2 * kTN + 2 * kRNT + 2 * kRTN;
-static_assert(kRTN <= 2 * kRNT, "the readout tile aliases the B and C gradient tiles");
+__device__ __forceinline__ float sigmoid(float x) { return __fdividef(1.f, 1.f + ex2_approx(-x * kLog2e)); }
 
-template <typename T>
-__global__ void __launch_bounds__(kBwdThreads, 2) bwd_kernel(const ScanParams p, const BwdParams q) {
+// The lane's NPL entries of step t of a [step][state] tile, as pairs.
+template <int NP>
+__device__ __forceinline__ void ld_pairs(const float *src, float2 (&o)[NP]) {
+    if constexpr (NP == 2) {
+        const float4 w = *reinterpret_cast<const float4 *>(src);
+        o[0] = f2(w.x, w.y);
+        o[1] = f2(w.z, w.w);
+    } else {
+        o[0] = *reinterpret_cast<const float2 *>(src);
+    }
+}
+
+template <typename T, int LPR>
+__global__ void __launch_bounds__(kBwdThreads, BwdShape<LPR>::MINB) bwd_kernel(const ScanParams p, const BwdParams g) {
+    using S = BwdShape<LPR>;
+    constexpr int NPL = S::NPL, NP = S::NP, RW = S::RW, IPL = S::IPL;
     extern __shared__ __align__(16) float smf[];
-    auto dts = reinterpret_cast<float (*)[kTS]>(smf);
-    auto dus = reinterpret_cast<float (*)[kTS]>(smf + kRT);
-    auto uus = reinterpret_cast<float (*)[kTS]>(smf + 2 * kRT);
-    auto dss = reinterpret_cast<float (*)[kTS]>(smf + 3 * kRT);
-    auto Bs = reinterpret_cast<float (*)[kN + 1]>(smf + 4 * kRT);
-    auto Cs = reinterpret_cast<float (*)[kN + 1]>(smf + 4 * kRT + kTN);
-    float *tiles = smf + 4 * kRT + 2 * kTN;
-    float *pB = tiles;                                                          // [step][row][state]
-    float *pC = tiles + kRNT;
-    auto trs = [](int step, int row, int state) { return step * kBT + row * kBR + state; };
-    float *pS = tiles;                                                          // [row][step][state], before pB
-    float *pDU = tiles + 2 * kRNT;
-    float *pDD = tiles + 2 * kRNT + kRTN;
-    auto rts = [](int row, int step, int state) { return row * kQR + step * kQS + state; };
-    // sum over the 16 states of (row, step) in a [row][step][state] tile
-    auto state_sum = [&](const float *tile, int row, int step) {
-        const float4 *v = reinterpret_cast<const float4 *>(tile + rts(row, step, 0));
-        const float4 a = v[0], b4 = v[1], c4 = v[2], d4 = v[3];
-        return ((a.x + a.y) + (a.z + a.w)) + ((b4.x + b4.y) + (b4.z + b4.w)) + ((c4.x + c4.y) + (c4.z + c4.w)) +
-               ((d4.x + d4.y) + (d4.z + d4.w));
-    };
-
-    const int tid = threadIdx.x;
-    const int r = tid / kN, n = tid % kN;          // chain (row, state); also item (row, step n)
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int q = lane % LPR, rw = lane / LPR;
+    float *xt = smf + warp * S::WARP_FLOATS;
+    float *bt = xt + RW * kXR;
+    float *ct = bt + kBC;
     const int64_t b = blockIdx.y;
-    const int64_t d = static_cast<int64_t>(blockIdx.x) * kRows + r;
+    const int64_t row0 = static_cast<int64_t>(blockIdx.x) * S::ROWS + warp * RW;   // the warp's first row
+    const int64_t d = row0 + rw;
     const bool ok = d < p.dim;
+    const bool warp_live = row0 < p.dim;
     const int64_t dc = ok ? d : p.dim - 1;
     const int dstate = static_cast<int>(p.dstate);
-    const bool live = n < dstate;
-    const int64_t L = p.seqlen;
-    const int64_t nchunks = (L + kT - 1) / kT;
+    const int L = static_cast<int>(p.seqlen);   // at most 2^30 (checked by the caller)
+    const int nchunks = (L + kT - 1) / kT;
     const int64_t row = b * p.dim + dc;
-    const float Areal = live ? __ldg(p.A + dc * dstate + n) : 0.f;
-    const float A2 = Areal * kLog2e;
+    float *xr = xt + rw * kXR;
+    // the row's sequences, indexed by step
+    const T *u_row = static_cast<const T *>(p.u) + b * p.u_sb + dc * p.u_sd;
+    const T *dl_row = static_cast<const T *>(p.delta) + b * p.dl_sb + dc * p.dl_sd;
+    const T *dy_row = static_cast<const T *>(g.dy) + b * g.dy_sb + dc * g.dy_sd;
+    const T *z_row = p.z ? static_cast<const T *>(p.z) + b * p.z_sb + dc * p.z_sd : u_row;
+    T *du_row = static_cast<T *>(g.du) + b * g.du_sb + dc * g.du_sd;
+    T *dd_row = static_cast<T *>(g.ddelta) + b * g.dd_sb + dc * g.dd_sd;
+    T *dz_row = g.dz ? static_cast<T *>(g.dz) + b * g.dz_sb + dc * g.dz_sd : du_row;
+    // the lane's B / C tile entries j: state lane / 8 + 4 j, step lane % 8 of the chunk
+    const T *b_lane = static_cast<const T *>(p.B) + b * p.B_sb + (lane / kT) * p.B_sn + lane % kT;
+    const T *c_lane = static_cast<const T *>(p.C) + b * p.C_sb + (lane / kT) * p.C_sn + lane % kT;
+    const int64_t b_jstride = (32 / kT) * p.B_sn, c_jstride = (32 / kT) * p.C_sn;
+
+    // the lane's states n = NPL q .. NPL q + NPL - 1: A (and A log2 e), padded with 0
+    float Ar[NPL];
+    float2 ap[NP];
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+        const int n = NPL * q + i;
+        Ar[i] = n < dstate ? __ldg(p.A + dc * dstate + n) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < NP; ++j) ap[j] = f2(Ar[2 * j] * kLog2e, Ar[2 * j + 1] * kLog2e);
     const float bias = p.delta_bias ? __ldg(p.delta_bias + dc) : 0.f;
     const float Dd = p.D ? __ldg(p.D + dc) : 0.f;
-    float *ckpt = q.ckpt + row * nchunks * kN + n;
+    // checkpoint c (the state at the end of chunk c) of the lane's states
+    float *ck = g.ckpt + row * nchunks * kN + NPL * q;
+    auto ck_store = [&](int c, const float2 (&h)[NP]) {
+        if constexpr (NP == 2)
+            *reinterpret_cast<float4 *>(ck + c * kN) = make_float4(h[0].x, h[0].y, h[1].x, h[1].y);
+        else
+            *reinterpret_cast<float2 *>(ck + c * kN) = h[0];
+    };
 
-    // The raw values one thread contributes to chunk c's tiles: item (row r,
-    // step n) -- u, delta_raw, dy, z -- and (step, state) (tid / 16, tid % 16)
-    // of the B and C tiles. Loaded one chunk ahead of use, so the global
-    // latency hides behind the current chunk's work.
-    struct RawVals { float u, dl, dy, z, bv, cv; };
-    auto load_raw = [&](int64_t c, bool grads) {
-        RawVals v{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        const int64_t t = c * kT + n;
-        if (ok && t < L) {
-            v.u = ldv<T>(p.u, b * p.u_sb + dc * p.u_sd + t);
-            v.dl = ldv<T>(p.delta, b * p.dl_sb + dc * p.dl_sd + t);
-            if (grads) {
-                v.dy = ldv<T>(q.dy, b * q.dy_sb + dc * q.dy_sd + t);
-                if (p.z) v.z = ldv<T>(p.z, b * p.z_sb + dc * p.z_sd + t);
+    // The raw values one lane contributes to chunk c: its row's steps
+    // q + LPR k (u, delta_raw and, in phase B, dy and z) and entries
+    // lane + 32 j of its warp's B and C tiles (state e / 8, step e % 8: eight
+    // lanes read eight consecutive steps of one state). Loaded a chunk ahead.
+    struct Raw {
+        float u[IPL], dl[IPL], dy[IPL], z[IPL], bv[kBCL], cv[kBCL];
+    };
+    // (bounds are checked only in the ragged last chunk)
+    auto load_raw = [&](int c, bool grads) {
+        Raw v;
+        const int t0 = c * kT;
+        const bool full = t0 + kT <= L;
+#pragma unroll
+        for (int k = 0; k < IPL; ++k) {
+            v.u[k] = v.dl[k] = v.dy[k] = v.z[k] = 0.f;
+            const int t = t0 + q + LPR * k;
+            if (ok && (full || t < L)) {
+                v.u[k] = to_f32<T>(u_row[t]);
+                v.dl[k] = to_f32<T>(dl_row[t]);
+                if (grads) {
+                    v.dy[k] = to_f32<T>(dy_row[t]);
+                    if (p.z) v.z[k] = to_f32<T>(z_row[t]);
+                }
             }
         }
-        const int tt = tid / kN, nn = tid % kN;
-        const int64_t ts = c * kT + tt;
-        if (nn < dstate && ts < L) {
-            v.bv = ldv<T>(p.B, b * p.B_sb + nn * p.B_sn + ts);
-            if (grads) v.cv = ldv<T>(p.C, b * p.C_sb + nn * p.C_sn + ts);
+        const bool tin = full || t0 + lane % kT < L;
+#pragma unroll
+        for (int j = 0; j < kBCL; ++j) {
+            v.bv[j] = v.cv[j] = 0.f;
+            if (tin && lane / kT + (32 / kT) * j < dstate) {
+                v.bv[j] = to_f32<T>(b_lane[j * b_jstride + t0]);
+                if (grads) v.cv[j] = to_f32<T>(c_lane[j * c_jstride + t0]);
+            }
         }
         return v;
     };
-    // Stage chunk c's tiles from its raw values: per (row, step) delta, delta u
-    // and u (steps past the end: delta = 0, the identity); per (step, state) B, C.
-    auto stage = [&](int64_t c, const RawVals &v) {
-        const bool in = ok && c * kT + n < L;
-        const float dt = in ? (p.softplus ? softplus(v.dl + bias) : v.dl + bias) : 0.f;
-        dts[r][n] = dt;
-        dus[r][n] = dt * v.u;
-        uus[r][n] = v.u;
-        Bs[tid / kN][tid % kN] = v.bv;
-        Cs[tid / kN][tid % kN] = v.cv;
+    // Stage chunk c: delta, delta u and u of the lane's steps (steps past the
+    // end: delta = 0, the identity), its B and C entries.
+    auto stage = [&](int c, const Raw &v) {
+#pragma unroll
+        for (int k = 0; k < IPL; ++k) {
+            const int t = q + LPR * k;
+            const bool in = ok && c * kT + t < L;
+            const float x = v.dl[k] + bias;
+            const float dt = in ? (p.softplus ? softplus(x) : x) : 0.f;
+            xr[kF_DT + t] = dt;
+            xr[kF_DU + t] = dt * v.u[k];
+            xr[kF_U + t] = v.u[k];
+        }
+#pragma unroll
+        for (int j = 0; j < kBCL; ++j) {
+            const int e = lane + 32 * j, nn = e / kT, tt = e % kT;
+            bt[tt * kBS + nn] = v.bv[j];
+            ct[tt * kBS + nn] = v.cv[j];
+        }
+    };
+    // eight steps of a per-row field
+    auto row8 = [&](int f, float (&o)[kT]) {
+        const float4 a = *reinterpret_cast<const float4 *>(xr + f);
+        const float4 c4 = *reinterpret_cast<const float4 *>(xr + f + 4);
+        o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+        o[4] = c4.x; o[5] = c4.y; o[6] = c4.z; o[7] = c4.w;
     };
 
-    // ---- Phase F: checkpoints at the end of every chunk but the last ----
-    const float h_init = (live && p.h0) ? p.h0[row * dstate + n] : 0.f;
-    float h = h_init;
-    RawVals nxt = nchunks > 1 ? load_raw(0, false) : RawVals{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int64_t c = 0; c + 1 < nchunks; ++c) {
-        const RawVals cur = nxt;
-        stage(c, cur);
-        if (c + 2 < nchunks) nxt = load_raw(c + 1, false);
-        __syncthreads();
+    // ---- Phase F: the state at the end of every chunk but the last ----
+    float2 h_init[NP];
 #pragma unroll
-        for (int t4 = 0; t4 < kT; t4 += 4) {
-            const float4 dt4 = *reinterpret_cast<const float4 *>(&dts[r][t4]);
-            const float4 du4 = *reinterpret_cast<const float4 *>(&dus[r][t4]);
-            const float dtv[4] = {dt4.x, dt4.y, dt4.z, dt4.w}, duv[4] = {du4.x, du4.y, du4.z, du4.w};
+    for (int j = 0; j < NP; ++j) {
+        float h2[2] = {0.f, 0.f};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) h = fmaf(ex2_approx(dtv[e] * A2), h, duv[e] * Bs[t4 + e][n]);
+        for (int e = 0; e < 2; ++e) {
+            const int n = NPL * q + 2 * j + e;
+            if (p.h0 && ok && n < dstate) h2[e] = __ldg(p.h0 + row * dstate + n);
         }
-        if (ok) ckpt[c * kN] = h;   // rows past the end share a clamped index: no checkpoints
-        __syncthreads();
+        h_init[j] = f2(h2[0], h2[1]);
+    }
+    {
+        float2 hp[NP];
+#pragma unroll
+        for (int j = 0; j < NP; ++j) hp[j] = h_init[j];
+        Raw nxt;
+        if (nchunks > 1) nxt = load_raw(0, false);
+        for (int c = 0; c + 1 < nchunks; ++c) {
+            const Raw cur = nxt;
+            stage(c, cur);
+            if (c + 2 < nchunks) nxt = load_raw(c + 1, false);
+            __syncwarp();
+            float dtv[kT], duv[kT];
+            row8(kF_DT, dtv);
+            row8(kF_DU, duv);
+#pragma unroll
+            for (int t = 0; t < kT; ++t) {
+                float2 Bp[NP];
+                ld_pairs<NP>(bt + t * kBS + NPL * q, Bp);
+                const float2 dt2 = f2(dtv[t], dtv[t]), du2 = f2(duv[t], duv[t]);
+#pragma unroll
+                for (int j = 0; j < NP; ++j) hp[j] = fma2(ex2x2(mul2(dt2, ap[j])), hp[j], mul2(du2, Bp[j]));
+            }
+            if (ok) ck_store(c, hp);
+            __syncwarp();
+        }
     }
 
     // ---- Phase B ----
-    float G = (live && ok && q.dhT) ? q.dhT[row * dstate + n] : 0.f;   // a_{t+1} g_{t+1}, carried down
-    float dA_acc = 0.f, dD_acc = 0.f, dbias_acc = 0.f;
-    nxt = load_raw(nchunks - 1, true);
-    for (int64_t c = nchunks - 1; c >= 0; --c) {
-        const RawVals cur = nxt;
+    float2 G[NP];   // a_{t+1} g_{t+1}, carried down
+    float2 dA[NP];
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+        float g2[2] = {0.f, 0.f};
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int n = NPL * q + 2 * j + e;
+            if (ok && g.dhT && n < dstate) g2[e] = g.dhT[row * dstate + n];
+        }
+        G[j] = f2(g2[0], g2[1]);
+        dA[j] = f2(0.f, 0.f);
+    }
+    float dD_acc = 0.f, dbias_acc = 0.f;
+    const bool vec_atomic =
+        ((reinterpret_cast<uintptr_t>(g.dB) | reinterpret_cast<uintptr_t>(g.dC)) & 15u) == 0 && (L & 3) == 0;
+    // the state chunk c starts from: its predecessor's checkpoint (rows past
+    // the end have none and carry zeros), or the initial state
+    auto start_state = [&](int c, float2 (&h)[NP]) {
+        if (c > 0 && ok) {
+            ld_pairs<NP>(ck + (c - 1) * kN, h);
+        } else {
+#pragma unroll
+            for (int j = 0; j < NP; ++j) h[j] = h_init[j];
+        }
+    };
+    Raw nxt = load_raw(nchunks - 1, true);
+    float2 hnext[NP];
+    start_state(nchunks - 1, hnext);
+    for (int c = nchunks - 1; c >= 0; --c) {
+        const Raw cur = nxt;
+        float2 hs[NP];
+#pragma unroll
+        for (int j = 0; j < NP; ++j) hs[j] = hnext[j];
         stage(c, cur);
-        if (c > 0) nxt = load_raw(c - 1, true);
-        // dy and z of item (row r, step n)
-        const int64_t ti = c * kT + n;
-        const bool in = ok && ti < L;
-        const float dyv = cur.dy, zv = cur.z;
-        __syncthreads();
+        if (c > 0) {
+            nxt = load_raw(c - 1, true);
+            start_state(c - 1, hnext);
+        }
+        __syncwarp();
 
-        // recompute the chunk's states from the previous checkpoint
-        const float hs = (c > 0 && ok) ? ckpt[(c - 1) * kN] : h_init;
-        float H[kT], Av[kT];
+        float dtv[kT], duv[kT];
+        row8(kF_DT, dtv);
+        row8(kF_DU, duv);
+        // recompute the chunk's states and decays from the previous checkpoint
+        float2 H[kT][NP], Av[kT][NP];
+        float s_own[IPL];   // C h summed over the row's states, the lane's steps
         {
-            float hh = hs;
+            float2 hh[NP];
 #pragma unroll
-            for (int t4 = 0; t4 < kT; t4 += 4) {
-                const float4 dt4 = *reinterpret_cast<const float4 *>(&dts[r][t4]);
-                const float4 du4 = *reinterpret_cast<const float4 *>(&dus[r][t4]);
-                const float dtv[4] = {dt4.x, dt4.y, dt4.z, dt4.w}, duv[4] = {du4.x, du4.y, du4.z, du4.w};
+            for (int j = 0; j < NP; ++j) hh[j] = hs[j];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    Av[t4 + e] = ex2_approx(dtv[e] * A2);
-                    hh = fmaf(Av[t4 + e], hh, duv[e] * Bs[t4 + e][n]);
-                    H[t4 + e] = hh;
+            for (int t0 = 0; t0 < kT; t0 += LPR) {
+                float ps[LPR];
+#pragma unroll
+                for (int e = 0; e < LPR; ++e) {
+                    const int t = t0 + e;
+                    float2 Bp[NP], Cp[NP];
+                    ld_pairs<NP>(bt + t * kBS + NPL * q, Bp);
+                    ld_pairs<NP>(ct + t * kBS + NPL * q, Cp);
+                    const float2 dt2 = f2(dtv[t], dtv[t]), du2 = f2(duv[t], duv[t]);
+                    float2 sc = f2(0.f, 0.f);
+#pragma unroll
+                    for (int j = 0; j < NP; ++j) {
+                        Av[t][j] = ex2x2(mul2(dt2, ap[j]));
+                        hh[j] = fma2(Av[t][j], hh[j], mul2(du2, Bp[j]));
+                        H[t][j] = hh[j];
+                        sc = fma2(Cp[j], hh[j], sc);
+                    }
+                    ps[e] = sc.x + sc.y;
                 }
+                s_own[t0 / LPR] = transposed_sum<LPR, 1>(ps, q);
             }
         }
-        // ds, dz of item (row r, step n); s_t sums C h over the row's states
+        // the lane's steps: ds (to the tile), dz, the D gradient
 #pragma unroll
-        for (int t = 0; t < kT; ++t) pS[rts(r, t, n)] = Cs[t][n] * H[t];
-        __syncthreads();
-        const float s_mine = Dd * uus[r][n] + state_sum(pS, r, n);
-        float dsv = dyv;
-        if (p.z) {
-            const float sg = __fdividef(1.f, 1.f + ex2_approx(-zv * kLog2e));
-            if (in && q.dz)
-                static_cast<T *>(q.dz)[b * q.dz_sb + dc * q.dz_sd + ti] =
-                    from_f32<T>(dyv * s_mine * sg * (1.f + zv * (1.f - sg)));
-            dsv = dyv * zv * sg;
-        }
-        dss[r][n] = dsv;
-        dD_acc = fmaf(dsv, uus[r][n], dD_acc);
-        __syncthreads();
-
-        // adjoint recurrence through the chunk
-#pragma unroll
-        for (int t4 = kT - 4; t4 >= 0; t4 -= 4) {
-            const float4 ds4 = *reinterpret_cast<const float4 *>(&dss[r][t4]);
-            const float4 dt4 = *reinterpret_cast<const float4 *>(&dts[r][t4]);
-            const float4 du4 = *reinterpret_cast<const float4 *>(&dus[r][t4]);
-            const float4 uu4 = *reinterpret_cast<const float4 *>(&uus[r][t4]);
-            const float dsv4[4] = {ds4.x, ds4.y, ds4.z, ds4.w}, dtv4[4] = {dt4.x, dt4.y, dt4.z, dt4.w};
-            const float duv4[4] = {du4.x, du4.y, du4.z, du4.w}, uuv4[4] = {uu4.x, uu4.y, uu4.z, uu4.w};
-#pragma unroll
-            for (int e = 3; e >= 0; --e) {
-                const int t = t4 + e;
-                const float ds = dsv4[e], dt = dtv4[e], Bv = Bs[t][n];
-                const float hprev = t > 0 ? H[t - 1] : hs;
-                const float gn = fmaf(ds, Cs[t][n], G);
-                pC[trs(t, r, n)] = ds * H[t];
-                pB[trs(t, r, n)] = gn * duv4[e];
-                pDU[rts(r, t, n)] = gn * dt * Bv;
-                pDD[rts(r, t, n)] = gn * fmaf(Bv, uuv4[e], hprev * Av[t] * Areal);
-                dA_acc = fmaf(gn * hprev, Av[t] * dt, dA_acc);
-                G = Av[t] * gn;
-            }
-        }
-        __syncthreads();
-
-        // item (row r, step n): du, ddelta; B/C gradients of (step, state) = (tid / 16, tid % 16)
-        if (in) {
-            const float du = dss[r][n] * Dd + state_sum(pDU, r, n);
-            float dd = state_sum(pDD, r, n);
-            if (p.softplus) dd *= __fdividef(1.f, 1.f + ex2_approx(-(cur.dl + bias) * kLog2e));
-            static_cast<T *>(q.du)[b * q.du_sb + dc * q.du_sd + ti] = from_f32<T>(du);
-            static_cast<T *>(q.ddelta)[b * q.dd_sb + dc * q.dd_sd + ti] = from_f32<T>(dd);
-            dbias_acc += dd;
-        }
-        {
-            const int tt = tid / kN, nn = tid % kN;
-            const int64_t ts = c * kT + tt;
-            if (nn < dstate && ts < L) {
-                float sb = 0.f, sc = 0.f;
-#pragma unroll
-                for (int rr = 0; rr < kRows; ++rr) {
-                    sb += pB[trs(tt, rr, nn)];
-                    sc += pC[trs(tt, rr, nn)];
+        for (int k = 0; k < IPL; ++k) {
+            const int t = q + LPR * k;
+            const int ti = c * kT + t;
+            const bool in = ok && ti < L;
+            const float u = cur.u[k], dy = cur.dy[k];
+            float ds = dy;
+            if (p.z) {
+                const float zv = cur.z[k];
+                const float sg = sigmoid(zv);
+                if (in && g.dz) {
+                    const float s = s_own[k] + Dd * u;
+                    dz_row[ti] = from_f32<T>(dy * s * sg * (1.f + zv * (1.f - sg)));
                 }
-                atomicAdd(q.dB + (b * dstate + nn) * L + ts, sb);
-                atomicAdd(q.dC + (b * dstate + nn) * L + ts, sc);
+                ds = dy * zv * sg;
+            }
+            xr[kF_DS + t] = ds;   // 0 past the end (dy = 0 there)
+            dD_acc = fmaf(ds, u, dD_acc);
+        }
+        __syncwarp();
+        float dsv[kT];
+        row8(kF_DS, dsv);
+
+        // adjoint recurrence through the chunk, last step first
+        float red[kT];   // the warp's rows summed: value rw (tensor rw / NPL, state NPL q + rw % NPL) per step
+#pragma unroll
+        for (int t0 = kT - LPR; t0 >= 0; t0 -= LPR) {
+            float s1[LPR], s2[LPR];   // per step: sum of g B, sum of g h_{t-1} a A over the lane's states
+#pragma unroll
+            for (int e = LPR - 1; e >= 0; --e) {
+                const int t = t0 + e;
+                float2 Bp[NP], Cp[NP];
+                ld_pairs<NP>(bt + t * kBS + NPL * q, Bp);
+                ld_pairs<NP>(ct + t * kBS + NPL * q, Cp);
+                const float2 ds2 = f2(dsv[t], dsv[t]), du2 = f2(duv[t], duv[t]), dt2 = f2(dtv[t], dtv[t]);
+                float v[2 * NPL];   // B gradient partials of the lane's states, then C gradient partials
+                float2 a1 = f2(0.f, 0.f), a2 = f2(0.f, 0.f);
+#pragma unroll
+                for (int j = 0; j < NP; ++j) {
+                    const float2 gn = fma2(ds2, Cp[j], G[j]);
+                    const float2 gB = mul2(gn, du2);
+                    const float2 gC = mul2(ds2, H[t][j]);
+                    v[2 * j] = gB.x;
+                    v[2 * j + 1] = gB.y;
+                    v[NPL + 2 * j] = gC.x;
+                    v[NPL + 2 * j + 1] = gC.y;
+                    a1 = fma2(gn, Bp[j], a1);
+                    const float2 hprev = t > 0 ? H[t - 1][j] : hs[j];
+                    const float2 gx = mul2(gn, mul2(hprev, Av[t][j]));
+                    a2 = fma2(gx, f2(Ar[2 * j], Ar[2 * j + 1]), a2);
+                    dA[j] = fma2(gx, dt2, dA[j]);
+                    G[j] = mul2(Av[t][j], gn);
+                }
+                s1[e] = a1.x + a1.y;
+                s2[e] = a2.x + a2.y;
+                red[t] = transposed_sum<RW, LPR>(v, rw);
+            }
+            // the lane's step t0 + q: du, ddelta
+            const float S1 = transposed_sum<LPR, 1>(s1, q);
+            const float S2 = transposed_sum<LPR, 1>(s2, q);
+            const int k = t0 / LPR;
+            const int t = t0 + q;
+            const int ti = c * kT + t;
+            if (ok && ti < L) {
+                const float u = cur.u[k];
+                const float du = fmaf(xr[kF_DT + t], S1, xr[kF_DS + t] * Dd);
+                float dd = fmaf(u, S1, S2);
+                if (p.softplus) dd *= sigmoid(cur.dl[k] + bias);
+                du_row[ti] = from_f32<T>(du);
+                dd_row[ti] = from_f32<T>(dd);
+                dbias_acc += dd;
             }
         }
-        __syncthreads();
+        // the lane's (tensor, state) of the B and C gradients, steps c kT .. c kT + 7
+        const int n = NPL * q + rw % NPL;
+        if (warp_live && n < dstate) {
+            const int ts = c * kT;
+            float *dst = (rw < NPL ? g.dB : g.dC) + (b * dstate + n) * L + ts;
+            if (vec_atomic && ts + kT <= L) {
+#pragma unroll
+                for (int t4 = 0; t4 < kT; t4 += 4)
+                    atomicAdd(reinterpret_cast<float4 *>(dst + t4),
+                              make_float4(red[t4], red[t4 + 1], red[t4 + 2], red[t4 + 3]));
+            } else {
+#pragma unroll
+                for (int t = 0; t < kT; ++t)
+                    if (ts + t < L) atomicAdd(dst + t, red[t]);
+            }
+        }
+        __syncwarp();   // the tiles are read: the next chunk may stage
     }
 
-    if (ok && live) {
-        if (q.dh0) q.dh0[row * dstate + n] = G;
-        atomicAdd(q.dA + dc * dstate + n, dA_acc);
+    if (ok) {
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+            const int n = NPL * q + i;
+            if (n < dstate) {
+                const float gi = (i & 1) ? G[i / 2].y : G[i / 2].x;
+                if (g.dh0) g.dh0[row * dstate + n] = gi;
+                atomicAdd(g.dA + dc * dstate + n, (i & 1) ? dA[i / 2].y : dA[i / 2].x);
+            }
+        }
     }
-    // per-row sums over the 16 step-slots of the row's threads
-    const float dD_row = half_warp_sum(dD_acc);
-    const float db_row = half_warp_sum(dbias_acc);
-    if (ok && n == 0) {
-        if (q.dD) atomicAdd(q.dD + dc, dD_row);
-        if (q.dbias) atomicAdd(q.dbias + dc, db_row);
+    // per-row sums over the row's lanes
+#pragma unroll
+    for (int m = 1; m < LPR; m *= 2) {
+        dD_acc += __shfl_xor_sync(0xffffffffu, dD_acc, m);
+        dbias_acc += __shfl_xor_sync(0xffffffffu, dbias_acc, m);
     }
+    if (ok && q == 0) {
+        if (g.dD) atomicAdd(g.dD + dc, dD_acc);
+        if (g.dbias) atomicAdd(g.dbias + dc, dbias_acc);
+    }
+}
+
+#ifndef MS_BWD_LANES
+#define MS_BWD_LANES 4
+#endif
+
+template <int LPR>
+cudaError_t launch_lpr(const ScanParams &p, const BwdParams &q, int in_dtype, cudaStream_t stream) {
+    using S = BwdShape<LPR>;
+    const dim3 grid(static_cast<unsigned>((p.dim + S::ROWS - 1) / S::ROWS), static_cast<unsigned>(p.batch));
+    const int smem = S::SMEM_FLOATS * static_cast<int>(sizeof(float));
+    const void *k = in_dtype == 0 ? reinterpret_cast<const void *>(bwd_kernel<float, LPR>)
+                                  : reinterpret_cast<const void *>(bwd_kernel<__nv_bfloat16, LPR>);
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    void *args[] = {const_cast<ScanParams *>(&p), const_cast<BwdParams *>(&q)};
+    e = cudaLaunchKernel(k, grid, dim3(kBwdThreads), args, static_cast<size_t>(smem), stream);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -289,16 +483,7 @@ size_t bwd_workspace_bytes(const ScanParams &p) {
 }
 
 cudaError_t launch_bwd(const ScanParams &p, const BwdParams &q, int in_dtype, cudaStream_t stream) {
-    const dim3 grid(static_cast<unsigned>((p.dim + kRows - 1) / kRows), static_cast<unsigned>(p.batch));
-    const int smem = kBwdSmemFloats * static_cast<int>(sizeof(float));
-    const void *k = in_dtype == 0 ? reinterpret_cast<const void *>(bwd_kernel<float>)
-                                  : reinterpret_cast<const void *>(bwd_kernel<__nv_bfloat16>);
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    void *args[] = {const_cast<ScanParams *>(&p), const_cast<BwdParams *>(&q)};
-    e = cudaLaunchKernel(k, grid, dim3(kBwdThreads), args, static_cast<size_t>(smem), stream);
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
+    return launch_lpr<MS_BWD_LANES>(p, q, in_dtype, stream);
 }
 
 }  // namespace ms
