@@ -15,7 +15,7 @@
 //
 // Design. The lanes hold the state as the forward's sequential kernel does:
 // LPR lanes per channel row (4 or 8), each with 16 / LPR of its 16 states,
-// 32 / LPR rows per warp, four warps per CTA. Phase F runs the
+// 32 / LPR rows per warp, one warp per CTA. Phase F runs the
 // recurrence forward and leaves the state at the end of every chunk of 8
 // steps in a workspace (one float per chain and chunk). Phase B walks the
 // chunks backward: it recomputes the chunk's 8 states and decays from the
@@ -27,8 +27,8 @@
 //     whose scalar work (gate, softplus derivative, stores) it does;
 //   - per (step, state) sums over the rows (the B and C gradients) are summed
 //     over the warp's rows the same way, leaving each lane one (tensor,
-//     state) total per step, which it adds to global memory in one float4
-//     atomic add per 4 steps.
+//     state) total per step, which it adds to global memory in one vector
+//     reduction (red.global.add.v4.f32) per 4 steps.
 // The warps are independent: each stages its own rows' per-chunk inputs
 // (delta, delta u, u, ds per row and step) and its own copy of the chunk's B
 // and C ([step][state]) in shared memory, read as broadcasts, and only
@@ -44,7 +44,7 @@ namespace ms {
 namespace {
 
 constexpr int kN = 16;                 // states per row (smaller dstate is zero-padded)
-constexpr int kW = 4;                  // warps per CTA
+constexpr int kW = 1;                  // warps per CTA (independent; one-warp CTAs balance best)
 constexpr int kT = 8;                  // steps per chunk (checkpoint interval)
 constexpr int kBwdThreads = kW * 32;
 constexpr int kBCL = kT * kN / 32;     // B (and C) entries a lane stages per chunk
@@ -68,7 +68,7 @@ template <int LPR> struct BwdShape {
     static constexpr int IPL = kT / LPR;        // steps a lane finishes per chunk
     static constexpr int WARP_FLOATS = RW * kXR + 2 * kBC;
     static constexpr int SMEM_FLOATS = kW * WARP_FLOATS;
-    static constexpr int MINB = LPR == 4 ? 3 : 4;
+    static constexpr int MINB = LPR == 4 ? 10 : 16;   // resident CTAs: the register budget per thread
     static_assert(LPR == 4 || LPR == 8, "4 or 8 lanes per row");
     static_assert(2 * NPL == RW, "the row reduction leaves one value per lane");
 };
@@ -91,6 +91,13 @@ __device__ __forceinline__ float transposed_sum(float (&v)[K], int q) {
         }
     }
     return v[0];
+}
+
+// Fire-and-forget vector reduction into global memory (16-byte aligned dst):
+// no value comes back, so nothing waits on the round trip.
+__device__ __forceinline__ void red_add4(float *dst, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
 }
 
 __device__ __forceinline__ float sigmoid(float x) { return __fdividef(1.f, 1.f + ex2_approx(-x * kLog2e)); }
@@ -422,8 +429,7 @@ __global__ void __launch_bounds__(kBwdThreads, BwdShape<LPR>::MINB) bwd_kernel(c
             if (vec_atomic && ts + kT <= L) {
 #pragma unroll
                 for (int t4 = 0; t4 < kT; t4 += 4)
-                    atomicAdd(reinterpret_cast<float4 *>(dst + t4),
-                              make_float4(red[t4], red[t4 + 1], red[t4 + 2], red[t4 + 3]));
+                    red_add4(dst + t4, red[t4], red[t4 + 1], red[t4 + 2], red[t4 + 3]);
             } else {
 #pragma unroll
                 for (int t = 0; t < kT; ++t)
