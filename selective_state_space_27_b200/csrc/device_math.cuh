@@ -126,6 +126,16 @@ __device__ __forceinline__ void cp_async_small(void *smem, const void *gmem, int
                  "r"(src_bytes)
                  : "memory");
 }
+// Asynchronous copy of BYTES (4, 8 or 16) bytes, all read, to a shared-memory
+// address given as a 32-bit shared-window offset.
+template <int BYTES>
+__device__ __forceinline__ void cp_async_full(unsigned smem_addr, const void *gmem) {
+    static_assert(BYTES == 4 || BYTES == 8 || BYTES == 16, "cp.async copies 4, 8 or 16 bytes");
+    if constexpr (BYTES == 16)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_addr), "l"(gmem) : "memory");
+    else
+        asm volatile("cp.async.ca.shared.global [%0], [%1], %2;\n" ::"r"(smem_addr), "l"(gmem), "n"(BYTES) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 // Wait until at most N of this thread's committed groups are still in flight.
 template <int N>

@@ -725,8 +725,36 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     // pointers point at it) into ring stage rs. Chunks inside the sequence
     // take fixed-size copies; the ragged last chunk copies what exists and
     // zero-fills the rest.
+    // shared-window address of the thread's slot 0 in ring stage 0
+    const unsigned ring_s = static_cast<unsigned>(__cvta_generic_to_shared(ring)) + i * 16;
     auto stage_chunk = [&](int c, int rs) {
         const bool full = c < nfull;
+        if constexpr (VEC && !CONV && !TRAP) {
+            if (full) {
+                // chunks inside the sequence: fixed-size copies from the running pointers
+                const unsigned sb = ring_s + rs * RW::STAGE;
+                constexpr int SB = PB < 16 ? PB : 16;
+#pragma unroll
+                for (int tsr = 0; tsr < 3; ++tsr) {
+                    if (tsr == 2 && !has_z) break;
+#pragma unroll
+                    for (int sl = 0; sl < PS; ++sl)
+                        cp_async_full<SB>(sb + (tsr * PS + sl) * IOT * 16,
+                                          reinterpret_cast<const unsigned char *>(srow[tsr]) + sl * 16);
+                }
+#pragma unroll
+                for (int j = 0; j < BC_PER; ++j) {
+                    const unsigned dst = sb + (3 * PS + j) * IOT * 16;
+                    if (bc_bytes[j]) {
+                        cp_async_full<BCB>(dst, bsrc[j]);
+                    } else {   // a state past dstate: zeros
+                        if constexpr (BCB == 16) cp_async16(slot(rs, 3 * PS + j), p.B, 0);
+                        else cp_async_small<BCB>(slot(rs, 3 * PS + j), p.B, 0);
+                    }
+                }
+                return;
+            }
+        }
         const int64_t t0 = static_cast<int64_t>(c) * kSteps;
         const int valid = full ? IP : static_cast<int>(min64(IP, max64(0, L - (t0 + tk))));
         constexpr int SB = PB < 16 ? PB : 16;   // bytes per slot
