@@ -727,8 +727,8 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     // zero-fills the rest.
     // shared-window address of the thread's slot 0 in ring stage 0
     const unsigned ring_s = static_cast<unsigned>(__cvta_generic_to_shared(ring)) + i * 16;
-    auto stage_chunk = [&](int c, int rs) {
-        const bool full = c < nfull;
+    auto stage_chunk = [&](int c, int rs, bool known_full = false) {
+        const bool full = known_full || c < nfull;
         if constexpr (VEC && !CONV && !TRAP) {
             if (full) {
                 // chunks inside the sequence: fixed-size copies from the running pointers
@@ -858,9 +858,9 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     auto ring_piece = [&](int rs, int tsr) { return ring_slots(rs, tsr * PS); };
     // Readout of chunk c from tile stage s (u, z from ring stage rs): partial
     // sums + D u, gate, store.
-    auto finish = [&](int c_, int s, int rs) {
+    auto finish = [&](int c_, int s, int rs, bool known_full = false) {
         const int64_t c = c_;
-        const int64_t cnt = c_ < nfull ? IP : L - (c * kSteps + tk);
+        const int64_t cnt = (known_full || c_ < nfull) ? IP : L - (c * kSteps + tk);
         if (!fok || cnt <= 0) return;
         const float Dd = Df;
         const float *yp = reinterpret_cast<const float *>(smem + s * S::STAGE + S::Y_OFF) + r * S::YR + tk;
@@ -912,7 +912,7 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     };
     // Chunk c's step tile (step pairs of delta, delta u) and B/C tiles from
     // ring stage rs into tile stage s.
-    auto widen = [&](int c_, int s, int rs) {
+    auto widen = [&](int c_, int s, int rs, bool known_full = false) {
         const int64_t c = c_;
         const float Dd = Dw;
         unsigned char *st = smem + s * S::STAGE;
@@ -944,7 +944,7 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
 #pragma unroll
             for (int e = 0; e < IP; e += 2) u2[e / 2] = f2(elem(xin, e), elem(xin, e + 1));
         }
-        const bool full = c_ < nfull;
+        const bool full = known_full || c_ < nfull;
         const int64_t cnt = L - (c * kSteps + tk);
         float uprev = 0.f;   // trapezoidal rule: u_{t-1} of the piece's first step
         Piece<T, IP> lam;
@@ -1030,6 +1030,41 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     int sf = 0, rf = 0;                   // tile and ring stage of the next chunk to finish
     int ra = RW::RA % RW::RS;             // ring stage of chunk it + RA
     for (int64_t it = 0; it < K; ++it) {
+        // Steady state: while the three cursors stay inside their pieces, the
+        // chunks they touch are whole and both the finish and the staging of
+        // this iteration are due, a lean body runs with no cursor or bounds
+        // logic; it stops one chunk before any of them would cross, and the
+        // general body below takes that chunk.
+        if (VAR == 0 && it >= kTileStages - 1) {   // (the variants would spill with a second body)
+            auto room = [&](const PCur &k) {
+                const int left = k.c1 - k.c;   // chunks left in the piece, this one included
+                const int whole = nfull - k.c;
+                return left < whole ? left : whole;
+            };
+            int64_t n = K - RW::RA - it;      // iterations that still stage a chunk
+            n = min64(n, room(kw));
+            n = min64(n, room(kf));
+            n = min64(n, room(ka));
+            for (int64_t m = 1; m < n; ++m, ++it) {
+                cp_async_wait<RW::RA - 1>();
+                widen(kw.c, s, rs, true);
+                bar_signal<NT>(bar_xf(s));
+                bar_wait<NT>(bar_yf(sf));
+                finish(kf.c, sf, rf, true);
+                stage_chunk(ka.c, ra, true);
+                cp_async_commit();
+                ++kw.c;
+                ++kf.c;
+                ++ka.c;
+                stage_advance();
+                yrow += kSteps;
+                s = next_stage(s, kTileStages);
+                rs = next_stage(rs, RW::RS);
+                ra = next_stage(ra, RW::RS);
+                sf = next_stage(sf, kTileStages);
+                rf = next_stage(rf, RW::RS);
+            }
+        }
         cp_async_wait<RW::RA - 1>();      // chunk it's copies have landed
         widen(kw.c, s, rs);
         bar_signal<NT>(bar_xf(s));
