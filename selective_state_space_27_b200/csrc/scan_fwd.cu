@@ -605,12 +605,12 @@ constexpr int kNumRec = sizeof(kRecLanes) / sizeof(kRecLanes[0]);
 // and runs markedly slower per row.
 constexpr double kRecCycles[][4] = {
     {2.4, 1.85, 1.85, 1.85},   // 2 lanes per row, 2 I/O warps
-    {3.0, 1.99, 1.81, 1.81},   // 4 lanes, 2 I/O warps
-    {4.5, 2.77, 2.67, 2.59},   // 8 lanes, 2 I/O warps
+    {2.51, 1.89, 1.69, 1.69},  // 4 lanes, 2 I/O warps
+    {4.5, 2.57, 2.54, 2.54},   // 8 lanes, 2 I/O warps
     {9.0, 8.0, 6.5, 6.5},      // 16 lanes, 2 I/O warps
     {2.06, 1.68, 1.68, 1.68},  // 2 lanes, 4 I/O warps
-    {2.70, 2.2, 2.2, 2.2},     // 4 lanes, 4 I/O warps
-    {4.8, 3.3, 3.28, 3.28},    // 8 lanes, 4 I/O warps
+    {2.59, 2.22, 2.2, 2.2},    // 4 lanes, 4 I/O warps
+    {3.98, 3.25, 3.25, 3.25},  // 8 lanes, 4 I/O warps
 };
 double rec_cycles(int ri, int64_t m) { return kRecCycles[ri][m < 1 ? 0 : m > 4 ? 3 : m - 1]; }
 // Relative cost of the persistent schedule's bookkeeping (piece table, carry
