@@ -856,13 +856,32 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     };
     // The thread's piece of tensor tsr (0 u, 1 delta, 2 z) from ring stage rs.
     auto ring_piece = [&](int rs, int tsr) { return ring_slots(rs, tsr * PS); };
-    // Readout of chunk c from tile stage s (u, z from ring stage rs): partial
-    // sums + D u, gate, store.
-    auto finish = [&](int c_, int s, int rs, bool known_full = false) {
+    // Readout of chunk c in two parts. finish_pre (before the wait for the
+    // recurrence) takes what does not depend on it from ring stage rs: D u
+    // and the gate; finish then adds the partial sums from tile stage s and
+    // stores.
+    float2 fskip[IP / 2], fgate[IP / 2];   // D u and silu(z) of the chunk to finish
+    auto finish_pre = [&](int s, int rs) {
+        if constexpr (CONV) {
+            const float *sk = reinterpret_cast<const float *>(smem + RW::SK_OFF + s * RW::SK_STAGE) + r * RW::SKR + tk;
+#pragma unroll
+            for (int e = 0; e < IP; e += 2) fskip[e / 2] = *reinterpret_cast<const float2 *>(sk + e);
+        } else {
+            const float Dd = Df;
+            const Piece<T, IP> u = ring_piece(rs, 0);
+#pragma unroll
+            for (int e = 0; e < IP; e += 2) fskip[e / 2] = mul2(f2(Dd, Dd), f2(elem(u, e), elem(u, e + 1)));
+        }
+        if (has_z) {
+            const Piece<T, IP> z = ring_piece(rs, 2);
+#pragma unroll
+            for (int e = 0; e < IP; e += 2) fgate[e / 2] = silu2_out<T>(f2(elem(z, e), elem(z, e + 1)));
+        }
+    };
+    auto finish = [&](int c_, int s, bool known_full = false) {
         const int64_t c = c_;
         const int64_t cnt = (known_full || c_ < nfull) ? IP : L - (c * kSteps + tk);
         if (!fok || cnt <= 0) return;
-        const float Dd = Df;
         const float *yp = reinterpret_cast<const float *>(smem + s * S::STAGE + S::Y_OFF) + r * S::YR + tk;
         float2 sum[IP / 2];
 #pragma unroll
@@ -880,33 +899,13 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
                 }
             }
         }
-        float2 skip[IP / 2];   // D u
-        if constexpr (CONV) {
-            const float *sk = reinterpret_cast<const float *>(smem + RW::SK_OFF + s * RW::SK_STAGE) + r * RW::SKR + tk;
-#pragma unroll
-            for (int e = 0; e < IP; e += 2) skip[e / 2] = *reinterpret_cast<const float2 *>(sk + e);
-        } else {
-            const Piece<T, IP> u = ring_piece(rs, 0);
-#pragma unroll
-            for (int e = 0; e < IP; e += 2) skip[e / 2] = mul2(f2(Dd, Dd), f2(elem(u, e), elem(u, e + 1)));
-        }
         float outv[IP];
-        if (has_z) {
-            const Piece<T, IP> z = ring_piece(rs, 2);
 #pragma unroll
-            for (int e = 0; e < IP; e += 2) {
-                const float2 yv = add2(skip[e / 2], sum[e / 2]);
-                const float2 g = mul2(yv, silu2_out<T>(f2(elem(z, e), elem(z, e + 1))));
-                outv[e] = g.x;
-                outv[e + 1] = g.y;
-            }
-        } else {
-#pragma unroll
-            for (int e = 0; e < IP; e += 2) {
-                const float2 yv = add2(skip[e / 2], sum[e / 2]);
-                outv[e] = yv.x;
-                outv[e + 1] = yv.y;
-            }
+        for (int e = 0; e < IP; e += 2) {
+            float2 yv = add2(fskip[e / 2], sum[e / 2]);
+            if (has_z) yv = mul2(yv, fgate[e / 2]);
+            outv[e] = yv.x;
+            outv[e + 1] = yv.y;
         }
         store_piece<T, IP, VEC>(yrow, outv, cnt);
     };
@@ -1049,8 +1048,9 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
                 cp_async_wait<RW::RA - 1>();
                 widen(kw.c, s, rs, true);
                 bar_signal<NT>(bar_xf(s));
+                finish_pre(sf, rf);
                 bar_wait<NT>(bar_yf(sf));
-                finish(kf.c, sf, rf, true);
+                finish(kf.c, sf, true);
                 stage_chunk(ka.c, ra, true);
                 cp_async_commit();
                 ++kw.c;
@@ -1070,8 +1070,9 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
         bar_signal<NT>(bar_xf(s));
         const int64_t j = it - (kTileStages - 1);
         if (j >= 0) {
+            finish_pre(sf, rf);
             bar_wait<NT>(bar_yf(sf));
-            finish(kf.c, sf, rf);
+            finish(kf.c, sf);
             sf = next_stage(sf, kTileStages);
             rf = next_stage(rf, RW::RS);
             finish_next();
@@ -1087,8 +1088,9 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
         if (kw.next(sc)) widen_ctx(kw.u);
     }
     for (int64_t j = max64(K - (kTileStages - 1), 0); j < K; ++j) {
+        finish_pre(sf, rf);
         bar_wait<NT>(bar_yf(sf));
-        finish(kf.c, sf, rf);
+        finish(kf.c, sf);
         sf = next_stage(sf, kTileStages);
         rf = next_stage(rf, RW::RS);
         finish_next();
@@ -1096,8 +1098,10 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     cp_async_wait<0>();
 }
 
-template <typename T, int LPR, bool VEC, int VAR, int IOW>
-__global__ void __launch_bounds__(Shape<LPR, VAR == 2, IOW>::THREADS, Shape<LPR, VAR == 2, IOW>::MINB)
+// ONE: the instantiation for launches with at most one CTA per SM, whose
+// threads may take every register the SM has.
+template <typename T, int LPR, bool VEC, int VAR, int IOW, bool ONE = false>
+__global__ void __launch_bounds__(Shape<LPR, VAR == 2, IOW>::THREADS, ONE ? 1 : Shape<LPR, VAR == 2, IOW>::MINB)
     rec_kernel(const ScanParams p) {
     extern __shared__ __align__(16) unsigned char smem[];
     if (threadIdx.x < kScanThreads) {
@@ -1116,36 +1120,51 @@ bool variant_compiled(int lpr, int variant, int iow) {
 }
 
 template <typename T, int LPR, int VAR, int IOW>
-const void *rec_ptr_v(bool vec) {
+const void *rec_ptr_v(bool vec, bool one = false) {
+    if constexpr (VAR == 0 && LPR <= 8) {   // one CTA per SM: the aligned plain scan
+        if (vec && one) return reinterpret_cast<const void *>(rec_kernel<T, LPR, true, VAR, IOW, true>);
+    }
     return vec ? reinterpret_cast<const void *>(rec_kernel<T, LPR, true, VAR, IOW>)
                : reinterpret_cast<const void *>(rec_kernel<T, LPR, false, VAR, IOW>);
 }
 
 template <typename T, int LPR>
-const void *rec_ptr(bool vec, int variant, int iow) {
+const void *rec_ptr(bool vec, int variant, int iow, bool one) {
     if constexpr (LPR != 16) {
-        if (iow == 4) return rec_ptr_v<T, LPR, 0, 4>(vec);
+        if (iow == 4) return rec_ptr_v<T, LPR, 0, 4>(vec, one);
     }
     if constexpr (LPR == 2 || LPR == 4) {   // the variants need 16-byte pieces
         if (variant == 1) return rec_ptr_v<T, LPR, 1, 2>(vec);
         if (variant == 2) return rec_ptr_v<T, LPR, 2, 2>(vec);
     }
-    return rec_ptr_v<T, LPR, 0, 2>(vec);
+    return rec_ptr_v<T, LPR, 0, 2>(vec, one);
 }
 
 template <typename T>
-const void *rec_select(int lpr, bool vec, int variant, int iow) {
+const void *rec_select(int lpr, bool vec, int variant, int iow, bool one) {
     switch (lpr) {
-        case 2: return rec_ptr<T, 2>(vec, variant, iow);
-        case 4: return rec_ptr<T, 4>(vec, variant, iow);
-        case 8: return rec_ptr<T, 8>(vec, variant, iow);
-        default: return rec_ptr<T, 16>(vec, variant, iow);
+        case 2: return rec_ptr<T, 2>(vec, variant, iow, one);
+        case 4: return rec_ptr<T, 4>(vec, variant, iow, one);
+        case 8: return rec_ptr<T, 8>(vec, variant, iow, one);
+        default: return rec_ptr<T, 16>(vec, variant, iow, one);
     }
 }
 
-const void *rec_kernel_for(int in_dtype, int lpr, bool vec, int variant, int iow) {
-    return in_dtype == 0 ? rec_select<float>(lpr, vec, variant, iow)
-                         : rec_select<__nv_bfloat16>(lpr, vec, variant, iow);
+const void *rec_kernel_for(int in_dtype, int lpr, bool vec, int variant, int iow, bool one) {
+    return in_dtype == 0 ? rec_select<float>(lpr, vec, variant, iow, one)
+                         : rec_select<__nv_bfloat16>(lpr, vec, variant, iow, one);
+}
+
+// Streaming multiprocessors of the current device (cached per device).
+int device_sms() {
+    static int cached[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess) cached[dev] = n;
+    }
+    return cached[dev];
 }
 
 template <typename T, int LPR>
@@ -1191,7 +1210,7 @@ int rec_ctas_per_sm(int in_dtype, int lpr, bool vec, int variant, int iow) {
     static int vals[kSlots];
     static int used = 0;
     static std::mutex mu;
-    const void *k = rec_kernel_for(in_dtype, lpr, vec, variant, iow);
+    const void *k = rec_kernel_for(in_dtype, lpr, vec, variant, iow, false);
     std::lock_guard<std::mutex> lk(mu);
     for (int i = 0; i < used; ++i)
         if (keys[i] == k) return vals[i];
@@ -1248,7 +1267,10 @@ cudaError_t launch_rec(const ScanParams &p, int lpr, bool vec, int in_dtype, int
     const int variant = rec_variant(p);
     if (!rec_supports_variant(lpr, variant, iow) || (p.conv_w && p.lambda_raw)) return cudaErrorInvalidValue;
     if (p.sk_ctas > 0 && (variant == 2 || !p.sk_carry || !p.sk_flag || !p.sk_status)) return cudaErrorInvalidValue;
-    const void *k = rec_kernel_for(in_dtype, lpr, vec, variant, iow);
+    // a persistent launch with at most one CTA per SM takes the instantiation
+    // without the occupancy bound on registers
+    const bool one = p.sk_ctas > 0 && p.sk_ctas <= device_sms();
+    const void *k = rec_kernel_for(in_dtype, lpr, vec, variant, iow, one);
     const int smem = rec_smem_bytes(in_dtype, lpr, variant, iow);
     const int threads = rec_threads(iow);
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
