@@ -777,15 +777,67 @@ def run_bwd(args, dist: Dist, dev, w, sets, params, counts, mufu_peak):
     e1.record(stream)
     torch.cuda.synchronize()
     us = dist.max(e0.elapsed_time(e1) * 1e3 / n, dev)
+
+    # The training pair: the forward keeps the states of every 8th step
+    # (mamba_scan_fwd_checkpointed) and the backward recomputes from them
+    # (mamba_scan_bwd_checkpointed) instead of sweeping the sequence first.
+    y_buf = torch.empty_like(s0["u"])
+    hT_buf = torch.empty((w.batch, w.dim, w.dstate), **f32)
+    fargs = ms.build_scan_args(s0["u"], s0["delta"], params["A"], s0["B"], s0["C"], y_buf, D=params["D"],
+                               z=s0.get("z"), delta_bias=params["delta_bias"], final_state=hT_buf)
+    ck = torch.empty(max(n_ws.value // 4, 64), dtype=torch.float32, device=dev)
+    fws = torch.empty(max(ms.scan_workspace_size(fargs), 256), dtype=torch.uint8, device=dev)
+
+    def fwd_plain():
+        rc = lib.mamba_scan_fwd(ctypes.byref(fargs), fws.data_ptr(), fws.numel(), stream.cuda_stream)
+        if rc != 0:
+            raise ms.MambaScanError(rc, lib.mamba_last_error().decode())
+
+    def fwd_ck():
+        rc = lib.mamba_scan_fwd_checkpointed(ctypes.byref(fargs), ck.data_ptr(), ck.numel() * 4, fws.data_ptr(),
+                                             fws.numel(), stream.cuda_stream)
+        if rc != 0:
+            raise ms.MambaScanError(rc, lib.mamba_last_error().decode())
+
+    def bwd_ck():
+        rc = lib.mamba_scan_bwd_checkpointed(ctypes.byref(args0), ctypes.byref(gb), ck.data_ptr(), ck.numel() * 4,
+                                             stream.cuda_stream)
+        if rc != 0:
+            raise ms.MambaScanError(rc, lib.mamba_last_error().decode())
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return dist.max(e0.elapsed_time(e1) * 1e3 / n, dev)
+
+    fwd_ck()
+    fwd_plain_us, fwd_ck_us, bwd_ck_us = timed(fwd_plain), timed(fwd_ck), timed(bwd_ck)
     rows_t = w.batch * w.dim * w.seqlen
     mufu = 2 * counts["elements"] + 6 * rows_t   # forward sweep + recompute ex2 per element; softplus, gates per (b,d,t)
+    mufu_ck = counts["elements"] + 6 * rows_t     # the recompute only
     return {
         "workload": w.name, "steps": n, "metric": "scan backward B*D*L*N elems/s", "unit": UNIT,
         "value": dist.world * counts["elements"] / (us * 1e-6), "us_per_step": us,
         "roofline": {"bound": "alu", "unit": "Tmufu/s", "achieved": mufu / (us * 1e-6) / 1e12,
                      "peak": mufu_peak / 1e12, "frac": mufu / (us * 1e-6) / mufu_peak, "algorithmic_mufu": mufu,
                      "note": "two ex2 per element: the checkpoint sweep and the per-chunk recomputation"},
-        "gpu_launches": 6 * n,
+        "checkpointed": {
+            "note": "forward with 8-step checkpoints (mamba_scan_fwd_checkpointed), backward from them "
+                    "(mamba_scan_bwd_checkpointed)",
+            "fwd_plain_us": fwd_plain_us, "fwd_checkpointed_us": fwd_ck_us, "bwd_us": bwd_ck_us,
+            "pair_us": fwd_ck_us + bwd_ck_us, "pair_without_checkpoints_us": fwd_plain_us + us,
+            "bwd_roofline": {"bound": "alu", "unit": "Tmufu/s", "achieved": mufu_ck / (bwd_ck_us * 1e-6) / 1e12,
+                             "peak": mufu_peak / 1e12, "frac": mufu_ck / (bwd_ck_us * 1e-6) / mufu_peak,
+                             "algorithmic_mufu": mufu_ck,
+                             "note": "one ex2 per element (the recomputation) plus the per-(b,d,t) terms"},
+        },
+        "gpu_launches": 6 * n + 3 * (n + 3) + 1,
     }
 
 

@@ -379,6 +379,34 @@ ms_status mamba_scan_bwd_workspace_size(const ms_scan_args *args, size_t *bytes)
 ms_status mamba_scan_bwd(const ms_scan_args *args, const ms_scan_bwd_args *bwd, void *workspace,
                          size_t workspace_bytes, void *stream);
 
+/*
+ * Training pair with the checkpoints kept from the forward ("Notas sobre
+ * Mamba", section "A varredura paralela ciente do hardware": the backward
+ * recomputes the states; here it recomputes them from the forward's states at
+ * every 8th step instead of sweeping the sequence a second time).
+ *
+ * mamba_scan_fwd_checkpointed: mamba_scan_fwd, and in addition the state after
+ * every 8th step (t = 7, 15, ...) of every (batch, dim) row goes to
+ * `checkpoints`: (batch * dim, ceil(seqlen / 8), 16) float32 (states past
+ * dstate unspecified), caller-owned, 256-byte aligned, at least the size
+ * mamba_scan_bwd_workspace_size reports (checkpoint_bytes). Only the sequential
+ * kernels write them: MS_ERR_UNSUPPORTED when the plan for the arguments is a
+ * chunked kernel (force_segments > 1, or very few rows). `workspace` is the
+ * forward's own, as for mamba_scan_fwd. Other errors as mamba_scan_fwd, plus
+ * MS_ERR_INVALID_ARG for NULL checkpoints, MS_ERR_WORKSPACE for a short
+ * buffer, MS_ERR_ALIGNMENT for a misaligned one.
+ *
+ * mamba_scan_bwd_checkpointed: mamba_scan_bwd with the checkpoints of a
+ * mamba_scan_fwd_checkpointed call on the same arguments (same u, delta, A, B,
+ * C, D, z, delta_bias, initial_state and flags) in place of the workspace; it
+ * only reads them. Errors as mamba_scan_bwd (MS_ERR_WORKSPACE for a short
+ * buffer).
+ */
+ms_status mamba_scan_fwd_checkpointed(const ms_scan_args *args, float *checkpoints, size_t checkpoint_bytes,
+                                      void *workspace, size_t workspace_bytes, void *stream);
+ms_status mamba_scan_bwd_checkpointed(const ms_scan_args *args, const ms_scan_bwd_args *bwd,
+                                      const float *checkpoints, size_t checkpoint_bytes, void *stream);
+
 /* ---- Mamba-2 scalar-decay SSM (structured state space duality, SSD) --------
  * Per batch b and head h, sequentially in t, on a state H of 64 x 128 values
  * (headdim x dstate):

@@ -163,6 +163,12 @@ def load_library():
                                             ctypes.POINTER(ScanPlan), _vp]
         lib.mamba_scan_bwd_workspace_size.restype = ctypes.c_int
         lib.mamba_scan_bwd_workspace_size.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(ctypes.c_size_t)]
+        lib.mamba_scan_fwd_checkpointed.restype = ctypes.c_int
+        lib.mamba_scan_fwd_checkpointed.argtypes = [ctypes.POINTER(ScanArgs), _vp, ctypes.c_size_t, _vp,
+                                                    ctypes.c_size_t, _vp]
+        lib.mamba_scan_bwd_checkpointed.restype = ctypes.c_int
+        lib.mamba_scan_bwd_checkpointed.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(ScanBwdArgs), _vp,
+                                                    ctypes.c_size_t, _vp]
         lib.mamba_scan_bwd.restype = ctypes.c_int
         lib.mamba_scan_bwd.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(ScanBwdArgs), _vp, ctypes.c_size_t,
                                        _vp]
@@ -332,7 +338,7 @@ def scan_plan(args: ScanArgs) -> ScanPlan:
 
 def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
              initial_state=None, return_last_state=True, out=None, force_segments=0,
-             workspace=None, stream=None, plan=None):
+             workspace=None, stream=None, plan=None, checkpoints=None):
     """Selective scan forward on the current (or given) CUDA stream.
 
     u, delta, z: (batch, dim, L); B, C: (batch, dstate, L) -- all float32 or
@@ -340,7 +346,10 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=
     -exp(A_log)); D, delta_bias: (dim,) float32. Returns y (u's dtype), and
     the final float32 state (batch, dim, dstate) when ``return_last_state``.
     ``workspace``: optional uint8 CUDA tensor reused for the multi-block carry
-    (allocated here when needed and not given).
+    (allocated here when needed and not given). ``checkpoints``: optional
+    float32 CUDA tensor of at least :func:`checkpoint_numel` elements that
+    receives the state after every 8th step, for :func:`scan_bwd` (automatic
+    plan only).
     """
     torch = _torch()
     y = torch.empty_like(u) if out is None else out
@@ -362,7 +371,15 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=
                 workspace = torch.empty(need, dtype=torch.uint8, device=u.device)
                 own_ws = True
             ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
-        if plan is None:
+        if checkpoints is not None:
+            if plan is not None:
+                raise ValueError("checkpoints are written with the automatic plan only")
+            _need_cuda("checkpoints", checkpoints, torch.float32, None)
+            if not checkpoints.is_contiguous():
+                raise ValueError("checkpoints must be contiguous")
+            _check(lib.mamba_scan_fwd_checkpointed(ctypes.byref(args), checkpoints.data_ptr(),
+                                                   checkpoints.numel() * 4, ws_ptr, ws_bytes, _stream_ptr(stream)))
+        elif plan is None:
             _check(lib.mamba_scan_fwd(ctypes.byref(args), ws_ptr, ws_bytes, _stream_ptr(stream)))
         else:
             _check(lib.mamba_scan_fwd_with_plan(ctypes.byref(args), ctypes.byref(plan), ws_ptr, ws_bytes,
@@ -505,8 +522,15 @@ def trap_scan_fwd(u, delta, lambda_raw, A, B, C, D=None, z=None, delta_bias=None
     return (y, hT) if return_last_state else y
 
 
+def checkpoint_numel(u, B):
+    """float32 elements of the checkpoint buffer of :func:`scan_fwd` /
+    :func:`scan_bwd` for u (batch, dim, L) and B (batch, dstate, L)."""
+    batch, dim, L = u.shape
+    return batch * dim * ((L + 7) // 8) * 16
+
+
 def scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, delta_softplus=True, initial_state=None,
-             dfinal_state=None, workspace=None, stream=None):
+             dfinal_state=None, workspace=None, stream=None, checkpoints=None):
     """Gradients of :func:`scan_fwd` for the loss sum(y * dy) + sum(h_T * dfinal_state).
 
     Forward inputs as :func:`scan_fwd`; ``dy`` (batch, dim, L) in u's dtype;
@@ -514,6 +538,9 @@ def scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, delta_softp
     du, ddelta (w.r.t. the raw delta), dz (None without z) in u's dtype; dA
     (dim, dstate), dB, dC (batch, dstate, L), dD, ddelta_bias (dim,) (None
     when the input is None) and dinitial_state (batch, dim, dstate), float32.
+    ``checkpoints``: the tensor a :func:`scan_fwd` call on the same inputs
+    filled; the backward then recomputes from it instead of sweeping the
+    sequence forward first.
     """
     torch = _torch()
     batch, dim, L = u.shape
@@ -547,6 +574,13 @@ def scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, delta_softp
         setattr(g, k, _ptr(out[k]))
     lib = load_library()
     with torch.cuda.device(u.device):
+        if checkpoints is not None:
+            _need_cuda("checkpoints", checkpoints, torch.float32, None)
+            if not checkpoints.is_contiguous():
+                raise ValueError("checkpoints must be contiguous")
+            _check(lib.mamba_scan_bwd_checkpointed(ctypes.byref(args), ctypes.byref(g), checkpoints.data_ptr(),
+                                                   checkpoints.numel() * 4, _stream_ptr(stream)))
+            return out
         n = ctypes.c_size_t(0)
         _check(lib.mamba_scan_bwd_workspace_size(ctypes.byref(args), ctypes.byref(n)))
         own_ws = workspace is None or workspace.numel() < n.value

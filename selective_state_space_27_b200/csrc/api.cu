@@ -456,9 +456,8 @@ ms_status mamba_scan_bwd_workspace_size(const ms_scan_args *args, size_t *bytes)
     return MS_OK;
 }
 
-ms_status mamba_scan_bwd(const ms_scan_args *args, const ms_scan_bwd_args *g, void *workspace,
-                         size_t workspace_bytes, void *stream) {
-    const CallRange range("mamba_scan_bwd");
+static ms_status scan_bwd_impl(const ms_scan_args *args, const ms_scan_bwd_args *g, void *workspace,
+                               size_t workspace_bytes, void *stream, int ckpt_ready) {
     ms_status st = check_scan(args);
     if (st != MS_OK) return st;
     if (!g) return invalid("bwd is NULL");
@@ -484,7 +483,8 @@ ms_status mamba_scan_bwd(const ms_scan_args *args, const ms_scan_bwd_args *g, vo
     const ms::ScanParams p = to_params(args);
     const size_t need = ms::bwd_workspace_bytes(p);
     if (!workspace || workspace_bytes < need) {
-        set_error("workspace of %zu bytes needed, %zu given", need, workspace ? workspace_bytes : static_cast<size_t>(0));
+        set_error("%s of %zu bytes needed, %zu given", ckpt_ready ? "checkpoints" : "workspace", need,
+                  workspace ? workspace_bytes : static_cast<size_t>(0));
         return MS_ERR_WORKSPACE;
     }
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) {
@@ -500,6 +500,7 @@ ms_status mamba_scan_bwd(const ms_scan_args *args, const ms_scan_bwd_args *g, vo
     q.dA = g->dA; q.dB = g->dB; q.dC = g->dC; q.dD = g->dD; q.dbias = g->ddelta_bias;
     q.dh0 = g->dinitial_state;
     q.ckpt = static_cast<float *>(workspace);
+    q.ckpt_ready = ckpt_ready;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     const size_t bc = static_cast<size_t>(args->batch * args->dstate * args->seqlen) * sizeof(float);
     cudaError_t e = cudaMemsetAsync(g->dA, 0, static_cast<size_t>(args->dim * args->dstate) * sizeof(float), s);
@@ -512,6 +513,48 @@ ms_status mamba_scan_bwd(const ms_scan_args *args, const ms_scan_bwd_args *g, vo
     e = ms::launch_bwd(p, q, args->in_dtype, s);
     if (e != cudaSuccess) return cuda_fail(e, "backward kernel launch");
     return MS_OK;
+}
+
+ms_status mamba_scan_bwd(const ms_scan_args *args, const ms_scan_bwd_args *g, void *workspace,
+                         size_t workspace_bytes, void *stream) {
+    const CallRange range("mamba_scan_bwd");
+    return scan_bwd_impl(args, g, workspace, workspace_bytes, stream, 0);
+}
+
+ms_status mamba_scan_bwd_checkpointed(const ms_scan_args *args, const ms_scan_bwd_args *g,
+                                      const float *checkpoints, size_t checkpoint_bytes, void *stream) {
+    const CallRange range("mamba_scan_bwd_checkpointed");
+    if (!checkpoints) return invalid("checkpoints is NULL");
+    return scan_bwd_impl(args, g, const_cast<float *>(checkpoints), checkpoint_bytes, stream, 1);
+}
+
+ms_status mamba_scan_fwd_checkpointed(const ms_scan_args *args, float *checkpoints, size_t checkpoint_bytes,
+                                      void *workspace, size_t workspace_bytes, void *stream) {
+    const CallRange range("mamba_scan_fwd_checkpointed");
+    ms_status st = check_scan(args);
+    if (st != MS_OK) return st;
+    if (!checkpoints) return invalid("checkpoints is NULL");
+    const ms::ScanParams p0 = to_params(args);
+    const size_t need = ms::bwd_workspace_bytes(p0);
+    if (checkpoint_bytes < need) {
+        set_error("checkpoints of %zu bytes needed, %zu given", need, checkpoint_bytes);
+        return MS_ERR_WORKSPACE;
+    }
+    if ((reinterpret_cast<uintptr_t>(checkpoints) & 255u) != 0) {
+        set_error("checkpoints must be 256-byte aligned");
+        return MS_ERR_ALIGNMENT;
+    }
+    int sms = 0;
+    st = device_sms(&sms);
+    if (st != MS_OK) return st;
+    ms::ScanParams p = p0;
+    p.ckpt = checkpoints;   // (the planner then considers the sequential kernels only)
+    const ms::ScanPlan plan = ms::plan_scan(p, args->in_dtype, args->force_segments, sms);
+    if (plan.kind != 1) {
+        set_error("checkpoints are written by the sequential kernels only, which run no forced segments");
+        return MS_ERR_UNSUPPORTED;
+    }
+    return run_plan(p, plan, args->in_dtype, workspace, workspace_bytes, stream);
 }
 
 ms_status mamba_ssd_fwd(const ms_ssd_args *a, void *workspace, size_t workspace_bytes, void *stream) {

@@ -32,6 +32,10 @@ struct ScanParams {
     // current input, h_t = a_t h_{t-1} + (1-lambda_t) delta_t a_t B_{t-1} u_{t-1}
     // + lambda_t delta_t B_t u_t.
     const void *lambda_raw; int64_t lm_sb, lm_sd;
+    // Checkpoints for the backward pass (sequential kernels, plain scan only):
+    // when set, the state after every 8th step, (batch*dim, ceil(L/8), 16)
+    // float32, as the backward's workspace lays it out.
+    float *ckpt;
     // Persistent schedule of the sequential kernels (sk_ctas > 0): the chunks
     // of all units (one batch entry x one block of rows) form one list, cut
     // into sk_ctas equal ranges, one per CTA. A unit whose chunks fall into two
@@ -119,6 +123,7 @@ struct BwdParams {
     void *dz;          int64_t dz_sb, dz_sd;
     float *dA, *dB, *dC, *dD, *dbias, *dh0;
     float *ckpt;
+    int ckpt_ready;   // ckpt already holds the checkpoints (written by the forward): skip the forward sweep
 };
 size_t bwd_workspace_bytes(const ScanParams &p);
 cudaError_t launch_bwd(const ScanParams &p, const BwdParams &q, int in_dtype, cudaStream_t stream);

@@ -245,7 +245,7 @@ __global__ void __launch_bounds__(kBwdThreads, BwdShape<LPR>::MINB) bwd_kernel(c
         }
         h_init[j] = f2(h2[0], h2[1]);
     }
-    {
+    if (!g.ckpt_ready) {   // (skipped when the forward left the checkpoints)
         float2 hp[NP];
 #pragma unroll
         for (int j = 0; j < NP; ++j) hp[j] = h_init[j];

@@ -662,7 +662,8 @@ ScanPlan plan_scan(const ScanParams &p, int in_dtype, int force_segments, int nu
     // only sequential kernels fuse the convolution prologue or run the trapezoidal rule
     const int variant = rec_variant(p);
     double best = 1e300;
-    for (int ci = 0; ci < (variant ? 0 : kNumConfigs); ++ci) {
+    // (checkpoints for the backward are written by the sequential kernels only)
+    for (int ci = 0; ci < ((variant || p.ckpt) ? 0 : kNumConfigs); ++ci) {
         const Config cf = kConfigs[ci];
         if (cf.ni != 1 && !plan.vec) continue;
         if (cf.ni == 0 && p.dstate != kMaxN) continue;

@@ -417,6 +417,20 @@ __device__ __forceinline__ void store_piece(T *dst, const float (&v)[P], int64_t
     }
 }
 
+// Store the lane's NPL states (kept as pairs; NPL = 1 keeps one value in .x).
+template <int NPL, int NP>
+__device__ __forceinline__ void store_states(float *dst, const float2 (&hp)[NP]) {
+    if constexpr (NPL == 1) {
+        dst[0] = hp[0].x;
+    } else if constexpr (NPL == 2) {
+        *reinterpret_cast<float2 *>(dst) = hp[0];
+    } else {
+#pragma unroll
+        for (int j = 0; j < NP; j += 2)
+            reinterpret_cast<float4 *>(dst)[j / 2] = make_float4(hp[j].x, hp[j].y, hp[j + 1].x, hp[j + 1].y);
+    }
+}
+
 // The recurrence warps: lane (r, q) owns states q NPL .. q NPL + NPL - 1 of
 // row r of the unit being processed.
 template <typename T, int LPR, bool TRAP, int IOW>
@@ -431,6 +445,7 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
     const int q = S::GROUP_MAJOR ? lane / RW : tid % LPR;
     const int dstate = static_cast<int>(p.dstate);
     const Sched sc = make_sched(p, R);
+    const int n8 = static_cast<int>((p.seqlen + 7) / 8);   // 8-step checkpoints per row
 
     // A log2(e) and the state of the lane's states, kept as the register pairs
     // the packed instructions take (no moves in the loop); set at the start of
@@ -448,6 +463,8 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
         const int64_t row = ur.b * p.dim + ur.dc;
         const bool carried = pr.c0 > 0;
         if (carried) wait_carry(p, pr.u, tid);
+        // checkpoints of this row (the lane's states), if asked for
+        float *ckpt_row = (p.ckpt && ur.ok) ? p.ckpt + row * n8 * kStates + q * NPL : nullptr;
         {
             const int64_t dc = ur.dc;
             const float *hsrc = carried ? p.sk_carry + (static_cast<int64_t>(pr.u) * R + r) * kStates
@@ -599,6 +616,10 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
                 outs[t % E] = acc.x + acc.y;
             }
             if (t % E == E - 1) emit(t - E + 1, outs);
+            if ((t & 7) == 7 && ckpt_row) {   // the state after step 8 k + 7 of the sequence
+                const int k8 = 2 * c + t / 8;
+                if (k8 < n8) store_states<NPL>(ckpt_row + static_cast<int64_t>(k8) * kStates, hp);
+            }
             if (t & 1) {   // the pair (t + 1, t + 2) becomes current
                 xw[0] = xw[1];
                 xw[1] = xw[2];

@@ -229,13 +229,28 @@ def test_bwd_validation_rejects(lib, field, value, status):
                               None) == status
 
 
+def test_checkpoint_calls_validate_before_launching(lib):
+    """The checkpointed forward and backward refuse a missing, short or
+    misaligned checkpoint buffer with no device work (CPU: nothing launches)."""
+    a = _valid_scan_args()
+    n = ctypes.c_size_t(0)
+    assert lib.mamba_scan_bwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
+    base = (1 << 20) * 40
+    assert lib.mamba_scan_fwd_checkpointed(ctypes.byref(a), None, n.value, None, 0, None) == 1
+    assert lib.mamba_scan_fwd_checkpointed(ctypes.byref(a), base, n.value - 1, None, 0, None) == 6
+    assert lib.mamba_scan_fwd_checkpointed(ctypes.byref(a), base + 16, n.value, None, 0, None) == 3
+    assert lib.mamba_scan_bwd_checkpointed(ctypes.byref(a), ctypes.byref(_valid_bwd()), None, n.value, None) == 1
+    assert lib.mamba_scan_bwd_checkpointed(ctypes.byref(a), ctypes.byref(_valid_bwd()), base, n.value - 1,
+                                           None) == 6
+
+
 def test_bwd_needs_workspace_and_matching_gradients(lib):
     a = _valid_scan_args()
     assert lib.mamba_scan_bwd(ctypes.byref(a), None, None, 0, None) == 1
     assert lib.mamba_scan_bwd(ctypes.byref(a), ctypes.byref(_valid_bwd()), None, 0, None) == 6
     n = ctypes.c_size_t(0)
     assert lib.mamba_scan_bwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
-    assert n.value == 2 * 8 * 4 * 16 * 4
+    assert n.value == 2 * 8 * 8 * 16 * 4      # batch x dim x ceil(64 / 8) checkpoints x 16 states, float32
     a.D = (1 << 20) * 7                      # D given: dD required
     assert lib.mamba_scan_bwd(ctypes.byref(a), ctypes.byref(_valid_bwd()), (1 << 20) * 30, 1 << 30, None) == 1
 

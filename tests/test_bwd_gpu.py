@@ -24,7 +24,7 @@ def _tol(dtype, name):
     return 5e-3 if name in ROUNDED else 1e-3
 
 
-def _check(inp, *, seed, use_h0=True, use_dhT=True, softplus=True):
+def _check(inp, *, seed, use_h0=True, use_dhT=True, softplus=True, checkpointed=False):
     import torch
     import selective_state_space_27_b200 as ms
     dt = inp["dtype"]
@@ -35,10 +35,25 @@ def _check(inp, *, seed, use_h0=True, use_dhT=True, softplus=True):
     h0 = g.normal(size=(batch, dim, N)).astype(np.float32) if use_h0 else None
     dhT = g.normal(size=(batch, dim, N)).astype(np.float32) if use_dhT else None
     dev = device_inputs(inp)
+    h0_dev = None if h0 is None else torch.from_numpy(h0).cuda()
+    ckpt = None
+    if checkpointed:
+        # the forward keeps the states of every 8th step; its y and final state match the plain forward's
+        # (bit for bit when the automatic plan is the same sequential kernel; a shape the planner gives
+        # to a chunked kernel differs by rounding only)
+        ckpt = torch.full((ms.checkpoint_numel(dev["u"], dev["B"]),), float("nan"), device="cuda")
+        y_ck, hT_ck = ms.scan_fwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], D=dev["D"], z=dev["z"],
+                                  delta_bias=dev["delta_bias"], delta_softplus=softplus, initial_state=h0_dev,
+                                  checkpoints=ckpt)
+        y_pl, hT_pl = ms.scan_fwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], D=dev["D"], z=dev["z"],
+                                  delta_bias=dev["delta_bias"], delta_softplus=softplus, initial_state=h0_dev)
+        torch.cuda.synchronize()
+        fwd_tol = 1e-4 if dt == "f32" else 5e-3
+        assert rel_err(to_host64(y_ck), to_host64(y_pl)) <= fwd_tol
+        assert rel_err(to_host64(hT_ck), to_host64(hT_pl)) <= fwd_tol
     out = ms.scan_bwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], to_device(dy_store, dt), D=dev["D"],
-                      z=dev["z"], delta_bias=dev["delta_bias"], delta_softplus=softplus,
-                      initial_state=None if h0 is None else torch.from_numpy(h0).cuda(),
-                      dfinal_state=None if dhT is None else torch.from_numpy(dhT).cuda())
+                      z=dev["z"], delta_bias=dev["delta_bias"], delta_softplus=softplus, initial_state=h0_dev,
+                      dfinal_state=None if dhT is None else torch.from_numpy(dhT).cuda(), checkpoints=ckpt)
     torch.cuda.synchronize()
     ref = oracle.scan_bwd(u=inp["u"], delta=inp["delta"], A=inp["A"], B=inp["B"], C=inp["C"], dy=dy_store,
                           D=inp["D"], z=inp["z"], delta_bias=inp["delta_bias"], delta_softplus=softplus, h0=h0,
@@ -64,6 +79,38 @@ def test_scan_bwd_matches_oracle(dtype, batch, dim, N, L):
     (partial last chunk), dstate < 16, with z, D, delta_bias, h0 and dh_T."""
     inp = make_scan_inputs(LAYER, batch=batch, dim=dim, dstate=N, seqlen=L, dtype=dtype, seed=4100 + dim + L)
     _check(inp, seed=4200 + L)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("batch,dim,N,L", [(1, 3, 16, 1), (2, 37, 16, 33), (2, 20, 5, 100), (1, 16, 16, 256),
+                                           (2, 40, 16, 1030)])
+def test_scan_bwd_checkpointed_matches_oracle(dtype, batch, dim, N, L):
+    """The training pair: the forward keeps the 8-step checkpoints (its y and
+    final state unchanged), the backward recomputes from them. Ragged rows and
+    lengths (partial last 8- and 16-step chunks), dstate < 16."""
+    inp = make_scan_inputs(LAYER, batch=batch, dim=dim, dstate=N, seqlen=L, dtype=dtype, seed=4150 + dim + L)
+    _check(inp, seed=4250 + L, checkpointed=True)
+
+
+def test_scan_checkpoint_errors():
+    """A short checkpoint buffer is refused by both calls; a forced segmented
+    (chunked) plan cannot write checkpoints."""
+    import torch
+    import selective_state_space_27_b200 as ms
+    inp = make_scan_inputs(LAYER, batch=1, dim=8, seqlen=64, dtype="f32", seed=4400)
+    dev = device_inputs(inp)
+    short = torch.zeros(ms.checkpoint_numel(dev["u"], dev["B"]) - 1, device="cuda")
+    with pytest.raises(ms.MambaScanError, match="MS_ERR_WORKSPACE"):
+        ms.scan_fwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], D=dev["D"], z=dev["z"],
+                    delta_bias=dev["delta_bias"], checkpoints=short)
+    dy = torch.zeros_like(dev["u"])
+    with pytest.raises(ms.MambaScanError, match="MS_ERR_WORKSPACE"):
+        ms.scan_bwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], dy, D=dev["D"], z=dev["z"],
+                    delta_bias=dev["delta_bias"], checkpoints=short)
+    full = torch.zeros(ms.checkpoint_numel(dev["u"], dev["B"]), device="cuda")
+    with pytest.raises(ms.MambaScanError, match="MS_ERR_UNSUPPORTED"):
+        ms.scan_fwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], D=dev["D"], z=dev["z"],
+                    delta_bias=dev["delta_bias"], force_segments=2, checkpoints=full)
 
 
 @pytest.mark.parametrize("softplus", [True, False])
