@@ -750,8 +750,9 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
     const unsigned ring_s = static_cast<unsigned>(__cvta_generic_to_shared(ring)) + i * 16;
     auto stage_chunk = [&](int c, int rs, bool known_full = false) {
         const bool full = known_full || c < nfull;
-        if constexpr (VEC && !CONV && !TRAP) {
-            if (full) {
+        if constexpr (VEC) {
+            // (the variants' look-back lies before t = 0 in the sequence's first chunk: general path)
+            if (full && (!(CONV || TRAP) || c > 0 || tk >= VE)) {
                 // chunks inside the sequence: fixed-size copies from the running pointers
                 const unsigned sb = ring_s + rs * RW::STAGE;
                 constexpr int SB = PB < 16 ? PB : 16;
@@ -773,6 +774,13 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
                         else cp_async_small<BCB>(slot(rs, 3 * PS + j), p.B, 0);
                     }
                 }
+                if constexpr (TRAP) {
+#pragma unroll
+                    for (int sl = 0; sl < PS; ++sl)
+                        cp_async_full<16>(sb + (RW::LAM + sl) * IOT * 16,
+                                          reinterpret_cast<const unsigned char *>(lrow) + sl * 16);
+                }
+                if constexpr (CONV || TRAP) cp_async_full<16>(sb + RW::HALO * IOT * 16, srow[0] - VE);
                 return;
             }
         }
@@ -1055,7 +1063,7 @@ __device__ __forceinline__ void io_role(const ScanParams &p, unsigned char *smem
         // this iteration are due, a lean body runs with no cursor or bounds
         // logic; it stops one chunk before any of them would cross, and the
         // general body below takes that chunk.
-        if (VAR == 0 && it >= kTileStages - 1) {   // (the variants would spill with a second body)
+        if (it >= kTileStages - 1) {
             auto room = [&](const PCur &k) {
                 const int left = k.c1 - k.c;   // chunks left in the piece, this one included
                 const int whole = nfull - k.c;
