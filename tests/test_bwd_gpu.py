@@ -124,6 +124,9 @@ def test_scan_bwd_without_optional_terms(softplus):
 
 
 @pytest.mark.slow
-def test_scan_bwd_mamba130m_layer_full():
-    """The Mamba-130M-shaped layer (bf16, gate), every row and gradient."""
-    _check(make_scan_inputs(LAYER), seed=4400)
+@pytest.mark.parametrize("checkpointed", [False, True])
+def test_scan_bwd_mamba130m_layer_full(checkpointed):
+    """The Mamba-130M-shaped layer (bf16, gate), every row and gradient; with
+    checkpoints from the forward, whose persistent schedule here cuts units
+    between CTAs (the carry hand-over and the checkpoint stores meet)."""
+    _check(make_scan_inputs(LAYER), seed=4400, checkpointed=checkpointed)
