@@ -81,6 +81,8 @@ def parse_args(argv=None):
     ap.add_argument("--leg-workloads", default="mamba130m_layer,mamba1p4b_layer",
                     help="other scan workloads timed as legs (comma separated; empty: none)")
     ap.add_argument("--leg-steps", type=int, default=50, help="timed steps of each scan-workload leg")
+    ap.add_argument("--segments-leg", type=int, default=8,
+                    help="also time the headline workload with this many forced time segments per row (0: skip)")
     ap.add_argument("--side-workload", default="mamba130m_layer", choices=sorted(SCAN_WORKLOADS),
                     help="workload of the convolution-prologue, trapezoidal and backward legs")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -348,10 +350,11 @@ class ScanSetup:
     """Seeded inputs of one scan workload on the device, the C-ABI argument
     structs of its rotating input sets, the workspace and the launch plan."""
 
-    def __init__(self, w, dev, rank, pin=False):
+    def __init__(self, w, dev, rank, pin=False, force_segments=0):
         import torch
         import selective_state_space_27_b200 as ms
         self.w = w
+        self.force_segments = force_segments
         self.in_bytes = 4 if w.dtype == "f32" else 2
         self.tdt = torch.float32 if w.dtype == "f32" else torch.bfloat16
         self.inp = make_scan_inputs(w, seed=w.seed + 1000 * rank)
@@ -388,7 +391,8 @@ class ScanSetup:
     def scan_args(self, st, y, hT):
         import selective_state_space_27_b200 as ms
         return ms.build_scan_args(st["u"], st["delta"], self.params["A"], st["B"], st["C"], y, D=self.params["D"],
-                                  z=st.get("z"), delta_bias=self.params["delta_bias"], final_state=hT)
+                                  z=st.get("z"), delta_bias=self.params["delta_bias"], final_state=hT,
+                                  force_segments=self.force_segments)
 
     def step(self, lib, i, stream, args=None):
         import ctypes
@@ -459,16 +463,22 @@ def measure_mufu(peaks):
             "nominal_per_s": SMS_B200 * MUFU_PER_CLK * peaks["sm_max_mhz"] * 1e6}
 
 
-def run_scan_leg(args, dist, dev, w, mufu, peaks, lib, stream):
+def run_scan_leg(args, dist, dev, w, mufu, peaks, lib, stream, force_segments=0):
     """Time another scan workload through mamba_scan_fwd: its own plan,
-    rotating input sets when they fit in L2, and roofline."""
-    setup = ScanSetup(w, dev, dist.rank)
+    rotating input sets when they fit in L2, and roofline. With
+    force_segments > 1 the call forces that many time segments per row (the
+    chunked kernels' multi-block carry), timed against the same algorithmic
+    bound."""
+    setup = ScanSetup(w, dev, dist.rank, force_segments=force_segments)
     for i in range(max(3, args.warmup)):
         setup.step(lib, i, stream)
     n = args.leg_steps
     ms_ = dist.max(time_steps(lambda i: setup.step(lib, i, stream), n, stream), dev)
     us = ms_ * 1e3 / n
-    out = {"workload": w.name, "config": workload_config(w, {"l2": l2_note(w)}), "steps": n, "us_per_step": us,
+    cfg = {"l2": l2_note(w)}
+    if force_segments:
+        cfg["force_segments"] = force_segments
+    out = {"workload": w.name, "config": workload_config(w, cfg), "steps": n, "us_per_step": us,
            "value": dist.world * setup.counts["elements"] / (us * 1e-6), "unit": UNIT,
            "roofline": scan_roofline(setup, us, mufu, peaks), "gpu_launches": n * setup.launches_per_step}
     del setup
@@ -617,6 +627,11 @@ def run_ours(args, dist: Dist):
             legs[name] = run_scan_leg(args, dist, dev, SCAN_WORKLOADS[name], mufu, peaks, lib, stream)
             torch.cuda.empty_cache()
 
+    segmented = None
+    if args.segments_leg > 1:
+        segmented = run_scan_leg(args, dist, dev, w, mufu, peaks, lib, stream, force_segments=args.segments_leg)
+        torch.cuda.empty_cache()
+
     decode = run_decode(args, dist, dev) if args.decode_steps > 0 else None
     side = None
     if args.prologue_steps > 0 or args.trap_steps > 0 or args.bwd_steps > 0:
@@ -643,6 +658,7 @@ def run_ours(args, dist: Dist):
         "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded)", "config": workload_config(w, {"l2": l2_note(w)}),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "mufu_probe": mufu, "scan_legs": legs,
+        "segmented": segmented,
         "decode": decode, "conv_prologue": prologue, "trapezoidal": trap, "backward": bwd, "ssd": ssd,
         "gpu_launches": launches, "clocks": clocks,
     }
