@@ -53,9 +53,9 @@ MUFU_PER_CLK = 16
 # The long-context layer was captured at 16,384 of its 131,072 steps (same rows,
 # same plan): its traffic is proportional to the steps, so the capture is scaled
 # by 8.
-NCU_TRAFFIC = {("long_context_131k", 10, 148): (505165824 + 150080512) * 8,
-               ("mamba130m_layer", 10, 296): 152304896 + 32461312,
-               ("mamba1p4b_layer", 10, 444): 813843968 + 256621056,
+NCU_TRAFFIC = {("long_context_131k", 10, 148): (505176320 + 150065408) * 8,
+               ("mamba130m_layer", 10, 296): 152307456 + 32844800,
+               ("mamba1p4b_layer", 10, 444): 813864448 + 252678912,
                ("mamba2_layer_d2048", "ssd_kernel"): 563170560 + 243913472,
                ("decode_b256_d5120", "state_update_vec_kernel"): 92157440 + 29935104}
 FP32_PER_CLK = 128
