@@ -686,10 +686,16 @@ def run_prologue(args, dist: Dist, dev, w, sets, params, y, hT, counts, mufu_pea
                                delta_bias=params["delta_bias"], final_state=hT) for s in sets]
     lib = ms.load_library()
     stream = torch.cuda.current_stream()
+    nbytes = ctypes.c_size_t(0)
+    rc = lib.mamba_conv_scan_workspace_size(ctypes.byref(argl[0]), ctypes.byref(conv), None, ctypes.byref(nbytes))
+    if rc != 0:
+        raise ms.MambaScanError(rc, lib.mamba_last_error().decode())
+    workspace = torch.empty(max(1, nbytes.value), dtype=torch.uint8, device=dev)
 
     def step(i):
-        rc = lib.mamba_conv_scan_fwd(ctypes.byref(argl[i % len(argl)]), ctypes.byref(conv), None,
-                                     stream.cuda_stream)
+        rc = lib.mamba_conv_scan_fwd_ws(ctypes.byref(argl[i % len(argl)]), ctypes.byref(conv), None,
+                                        workspace.data_ptr() if nbytes.value else None, nbytes.value,
+                                        stream.cuda_stream)
         if rc != 0:
             raise ms.MambaScanError(rc, lib.mamba_last_error().decode())
 

@@ -300,6 +300,23 @@ ms_status mamba_conv_scan_fwd(const ms_scan_args *args, const ms_conv1d_args *co
                               const ms_scan_plan *plan, void *stream);
 
 /*
+ * The same with a caller-owned device workspace (256-byte aligned), which
+ * lets the automatic plan (plan NULL) or the caller's plan (ctas > 0) use the
+ * persistent schedule of the sequential kernels: the chunks of all rows cut
+ * evenly over the SMs, a row's state handed between CTAs through the
+ * workspace. mamba_conv_scan_workspace_size reports the bytes the plan the
+ * call would run needs (0: none; the workspace pointer may then be NULL).
+ * Errors as mamba_conv_scan_fwd, plus MS_ERR_WORKSPACE for a missing or short
+ * workspace and MS_ERR_ALIGNMENT for a misaligned one; a persistent launch
+ * whose carry wait runs out leaves MS_ERR_TIMEOUT in the workspace's status
+ * word (see mamba_scan_fwd_with_plan).
+ */
+ms_status mamba_conv_scan_workspace_size(const ms_scan_args *args, const ms_conv1d_args *conv,
+                                         const ms_scan_plan *plan, size_t *bytes);
+ms_status mamba_conv_scan_fwd_ws(const ms_scan_args *args, const ms_conv1d_args *conv, const ms_scan_plan *plan,
+                                 void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Decode step with the convolution prologue: args->x is the new convolution
  * input. conv_state (batch, dim, width) in the input dtype (element strides
  * conv_state_batch_stride and conv_state_dim_stride; the width axis is

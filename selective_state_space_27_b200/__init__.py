@@ -163,6 +163,12 @@ def load_library():
                                             ctypes.POINTER(ScanPlan), _vp]
         lib.mamba_scan_bwd_workspace_size.restype = ctypes.c_int
         lib.mamba_scan_bwd_workspace_size.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(ctypes.c_size_t)]
+        lib.mamba_conv_scan_workspace_size.restype = ctypes.c_int
+        lib.mamba_conv_scan_workspace_size.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(Conv1dArgs),
+                                                       ctypes.POINTER(ScanPlan), ctypes.POINTER(ctypes.c_size_t)]
+        lib.mamba_conv_scan_fwd_ws.restype = ctypes.c_int
+        lib.mamba_conv_scan_fwd_ws.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(Conv1dArgs),
+                                               ctypes.POINTER(ScanPlan), _vp, ctypes.c_size_t, _vp]
         lib.mamba_scan_fwd_checkpointed.restype = ctypes.c_int
         lib.mamba_scan_fwd_checkpointed.argtypes = [ctypes.POINTER(ScanArgs), _vp, ctypes.c_size_t, _vp,
                                                     ctypes.c_size_t, _vp]
@@ -462,7 +468,9 @@ def conv_scan_fwd(x, conv_weight, delta, A, B, C, D=None, z=None, delta_bias=Non
     """Causal depthwise convolution + SiLU prologue fused into the selective
     scan: ``x`` (batch, dim, L) is the convolution input, ``conv_weight``
     (dim, width) and ``conv_bias`` (dim,) float32; the scan input is
-    u = silu(conv(x)). Other arguments as :func:`scan_fwd` (no segments)."""
+    u = silu(conv(x)). Other arguments as :func:`scan_fwd` (no segments);
+    ``plan`` may ask for the persistent schedule (ctas > 0), whose workspace
+    is allocated here."""
     torch = _torch()
     y = torch.empty_like(x) if out is None else out
     hT = None
@@ -473,10 +481,17 @@ def conv_scan_fwd(x, conv_weight, delta, A, B, C, D=None, z=None, delta_bias=Non
     conv = build_conv_args(conv_weight, conv_bias, conv_silu)
     if conv_weight.shape[0] != x.shape[1]:
         raise ValueError("conv weight must have one row per channel")
+    lib = load_library()
+    plan_ref = None if plan is None else ctypes.byref(plan)
     with torch.cuda.device(x.device):
-        _check(load_library().mamba_conv_scan_fwd(ctypes.byref(args), ctypes.byref(conv),
-                                                  None if plan is None else ctypes.byref(plan),
-                                                  _stream_ptr(stream)))
+        n = ctypes.c_size_t(0)
+        _check(lib.mamba_conv_scan_workspace_size(ctypes.byref(args), ctypes.byref(conv), plan_ref, ctypes.byref(n)))
+        workspace = torch.empty(n.value, dtype=torch.uint8, device=x.device) if n.value else None
+        _check(lib.mamba_conv_scan_fwd_ws(ctypes.byref(args), ctypes.byref(conv), plan_ref,
+                                          None if workspace is None else workspace.data_ptr(), n.value,
+                                          _stream_ptr(stream)))
+        if workspace is not None:
+            _keep_until_done(workspace, stream)
     return (y, hT) if return_last_state else y
 
 

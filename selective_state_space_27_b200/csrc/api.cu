@@ -370,9 +370,9 @@ ms_status mamba_conv_state_update(const ms_update_args *a, const ms_conv1d_args 
     return MS_OK;
 }
 
-ms_status mamba_conv_scan_fwd(const ms_scan_args *args, const ms_conv1d_args *conv, const ms_scan_plan *plan,
-                              void *stream) {
-    const CallRange range("mamba_conv_scan_fwd");
+static ms_status conv_scan_impl(const ms_scan_args *args, const ms_conv1d_args *conv, const ms_scan_plan *plan,
+                                void *workspace, size_t workspace_bytes, void *stream, bool with_workspace,
+                                size_t *query) {
     ms_status st = check_scan(args);
     if (st != MS_OK) return st;
     st = check_conv(conv);
@@ -386,25 +386,49 @@ ms_status mamba_conv_scan_fwd(const ms_scan_args *args, const ms_conv1d_args *co
     p.conv_b = conv->bias;
     p.conv_width = conv->width;
     p.conv_silu = conv->silu;
+    int sms = 0;
+    st = device_sms(&sms);
+    if (st != MS_OK) return st;
     ms::ScanPlan pl{};
     if (plan) {
-        if (plan->ctas != 0 || plan->reserved != 0 ||
-            !ms::make_plan(p, args->in_dtype, plan->config, plan->warps_per_cta, plan->segments, 0, 0, &pl)) {
-            set_error("plan (config %d, %d warps, %d segments) cannot run the convolution prologue", plan->config,
-                      plan->warps_per_cta, plan->segments);
+        if ((!with_workspace && plan->ctas != 0) || plan->reserved != 0 ||
+            !ms::make_plan(p, args->in_dtype, plan->config, plan->warps_per_cta, plan->segments, plan->ctas, sms,
+                           &pl)) {
+            set_error("plan (config %d, %d warps, %d segments, %d CTAs) cannot run the convolution prologue",
+                      plan->config, plan->warps_per_cta, plan->segments, plan->ctas);
             return MS_ERR_UNSUPPORTED;
         }
     } else {
-        int sms = 0;
-        st = device_sms(&sms);
-        if (st != MS_OK) return st;
-        pl = ms::plan_scan(p, args->in_dtype, 0, sms);
+        pl = ms::plan_scan(p, args->in_dtype, 0, sms, with_workspace);
         if (pl.kind != 1) {
             set_error("no kernel configuration fuses the convolution prologue for these arguments");
             return MS_ERR_UNSUPPORTED;
         }
     }
-    return run_plan(p, pl, args->in_dtype, nullptr, 0, stream);
+    if (query) {
+        *query = pl.ws_bytes;
+        return MS_OK;
+    }
+    return run_plan(p, pl, args->in_dtype, workspace, workspace_bytes, stream);
+}
+
+ms_status mamba_conv_scan_fwd(const ms_scan_args *args, const ms_conv1d_args *conv, const ms_scan_plan *plan,
+                              void *stream) {
+    const CallRange range("mamba_conv_scan_fwd");
+    return conv_scan_impl(args, conv, plan, nullptr, 0, stream, false, nullptr);
+}
+
+ms_status mamba_conv_scan_workspace_size(const ms_scan_args *args, const ms_conv1d_args *conv,
+                                         const ms_scan_plan *plan, size_t *bytes) {
+    if (!bytes) return invalid("bytes is NULL");
+    *bytes = 0;
+    return conv_scan_impl(args, conv, plan, nullptr, 0, nullptr, true, bytes);
+}
+
+ms_status mamba_conv_scan_fwd_ws(const ms_scan_args *args, const ms_conv1d_args *conv, const ms_scan_plan *plan,
+                                 void *workspace, size_t workspace_bytes, void *stream) {
+    const CallRange range("mamba_conv_scan_fwd_ws");
+    return conv_scan_impl(args, conv, plan, workspace, workspace_bytes, stream, true, nullptr);
 }
 
 ms_status mamba_trap_scan_fwd(const ms_scan_args *args, const void *lambda_raw, int64_t lambda_batch_stride,

@@ -77,7 +77,8 @@ void rec_bind_workspace(ScanParams &p, void *ws, int64_t units, int ctas);
 // With p.conv_w or p.lambda_raw set only the sequential configurations that
 // fuse the convolution prologue or run the trapezoidal rule (lanes 2 and 4)
 // are considered.
-ScanPlan plan_scan(const ScanParams &p, int in_dtype, int force_segments, int num_sms);
+// persistent_ok: the caller can provide the persistent schedule's workspace.
+ScanPlan plan_scan(const ScanParams &p, int in_dtype, int force_segments, int num_sms, bool persistent_ok = true);
 // A plan with a fixed configuration, CTA size and segment count; returns false
 // (and leaves `out` unspecified) when the configuration cannot run `p`.
 // ctas: sequential configurations only, 0 = one CTA per unit, > 0 = persistent

@@ -648,7 +648,7 @@ int kernel_regs(const void *k) {
 // as many as fit (registers, shared memory, warps), an SM with fewer than 8
 // resident warps runs proportionally slower, and a segmented run costs 1.75x
 // the arithmetic (summary pass + main pass).
-ScanPlan plan_scan(const ScanParams &p, int in_dtype, int force_segments, int num_sms) {
+ScanPlan plan_scan(const ScanParams &p, int in_dtype, int force_segments, int num_sms, bool persistent_ok) {
     const int eb = in_dtype == 0 ? 4 : 2;
     ScanPlan plan{};
     auto strides_ok = [&](int64_t s1, int64_t s2) { return (s1 * eb) % 16 == 0 && (s2 * eb) % 16 == 0; };
@@ -722,8 +722,10 @@ ScanPlan plan_scan(const ScanParams &p, int in_dtype, int force_segments, int nu
                 rec = ri;
                 rec_ctas = 0;
             }
-            // persistent schedule: m CTAs on every SM share the units' work exactly
-            if (variant == 0 && p.batch * p.dim <= (int64_t(1) << 30) && (p.seqlen + 15) / 16 < (int64_t(1) << 30)) {
+            // persistent schedule: m CTAs on every SM share the units' work exactly (not the trapezoidal
+            // rule, whose carry would need the previous step's input)
+            if (persistent_ok && variant != 2 && p.batch * p.dim <= (int64_t(1) << 30) &&
+                (p.seqlen + 15) / 16 < (int64_t(1) << 30)) {
                 for (int m = 1; m <= per_sm && static_cast<int64_t>(m) * sms <= ctas; ++m) {
                     const double tp = static_cast<double>(ctas) * R * static_cast<double>(p.seqlen) / sms *
                                       rec_cycles(ri, m) * kRecPersistentCost;

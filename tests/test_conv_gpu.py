@@ -78,6 +78,33 @@ def test_conv_scan_matches_oracle(dtype, batch, dim, N, L, width, silu, offset):
         assert rel_err(hT, hr) <= TOL[dtype], tag
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_conv_scan_persistent_schedule(dtype):
+    """The prologue under the persistent schedule: every configuration that
+    fuses it at CTA counts from 1 to one per unit, including counts that cut
+    units between CTAs (the convolution's look-back then starts a piece in the
+    middle of a row)."""
+    import torch
+    ms = _ms()
+    batch, dim, N, L = 2, 100, 16, 300
+    inp = make_scan_inputs(LAYER, batch=batch, dim=dim, dstate=N, seqlen=L, dtype=dtype, seed=2950)
+    dev = device_inputs(inp)
+    conv = make_conv_params(dim, 4, seed=2951)
+    conv_t = {k: to_device(v, "f32") for k, v in conv.items()}
+    h0 = np.random.default_rng(2952).normal(size=(batch, dim, N)).astype(np.float32)
+    h0_t = torch.from_numpy(h0).cuda()
+    yr, hr = _oracle(inp, conv, h0=h0.reshape(-1, N))
+    for c, lanes, w in _conv_configs():
+        rows = 128 // lanes
+        units = batch * ((dim + rows - 1) // rows)
+        for ctas in sorted({1, 2, 3, max(1, units // 2), max(1, units - 1), units}):
+            plan = ms.ScanPlan(config=c, warps_per_cta=w, segments=1, ctas=ctas)
+            y, hT = _run(dev, conv_t, plan=plan, h0=h0_t)
+            tag = f"config {c}, {ctas} CTAs of {units} units"
+            assert rel_err(y, yr) <= TOL[dtype], tag
+            assert rel_err(hT, hr) <= TOL[dtype], tag
+
+
 def test_conv_scan_mamba130m_layer_full():
     """The Mamba-130M-shaped layer (bf16, gate) with a width-4 prologue, every row."""
     inp = make_scan_inputs(LAYER)
