@@ -740,10 +740,17 @@ def run_trap(args, dist: Dist, dev, w, sets, params, y, hT, counts, mufu_peak):
                                delta_bias=params["delta_bias"], final_state=hT) for s in sets]
     lib = ms.load_library()
     stream = torch.cuda.current_stream()
+    lam_args = (lam.data_ptr(), lam.stride(0), lam.stride(1))
+    nbytes = ctypes.c_size_t(0)
+    rc = lib.mamba_trap_scan_workspace_size(ctypes.byref(argl[0]), *lam_args, None, ctypes.byref(nbytes))
+    if rc != 0:
+        raise ms.MambaScanError(rc, lib.mamba_last_error().decode())
+    workspace = torch.empty(max(1, nbytes.value), dtype=torch.uint8, device=dev)
 
     def step(i):
-        rc = lib.mamba_trap_scan_fwd(ctypes.byref(argl[i % len(argl)]), lam.data_ptr(), lam.stride(0),
-                                     lam.stride(1), None, stream.cuda_stream)
+        rc = lib.mamba_trap_scan_fwd_ws(ctypes.byref(argl[i % len(argl)]), *lam_args, None,
+                                        workspace.data_ptr() if nbytes.value else None, nbytes.value,
+                                        stream.cuda_stream)
         if rc != 0:
             raise ms.MambaScanError(rc, lib.mamba_last_error().decode())
 

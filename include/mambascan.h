@@ -347,13 +347,34 @@ ms_status mamba_conv_state_update(const ms_update_args *args, const ms_conv1d_ar
  * exponential-Euler scan of mamba_scan_fwd. A nonzero initial state is the
  * state before t = 0; the previous-input term still starts at zero. Runs on the
  * sequential kernels with 2 or 4 lanes per row, in one segment, with no
- * workspace; `plan` is NULL (automatic) or one of those configurations.
+ * workspace; `plan` is NULL (automatic) or one of those configurations without
+ * CTAs (ctas 0).
  * Errors: as mamba_scan_fwd; MS_ERR_INVALID_ARG for a NULL lambda_raw or
  * negative strides; MS_ERR_UNSUPPORTED for force_segments > 1 or a plan that
  * cannot run the rule; MS_ERR_ALIGNMENT for a misaligned lambda_raw.
  */
 ms_status mamba_trap_scan_fwd(const ms_scan_args *args, const void *lambda_raw, int64_t lambda_batch_stride,
                               int64_t lambda_dim_stride, const ms_scan_plan *plan, void *stream);
+
+/*
+ * The same with a caller-owned device workspace (256-byte aligned), which
+ * lets the automatic plan (plan NULL) or the caller's plan (ctas > 0) use the
+ * persistent schedule of the sequential kernels (a row's state handed between
+ * CTAs through the workspace; the CTA that takes a row over reads B at the
+ * step before its first one from B itself).
+ * mamba_trap_scan_workspace_size reports the bytes the plan the call would run
+ * needs (0: none; the workspace pointer may then be NULL). Errors as
+ * mamba_trap_scan_fwd, plus MS_ERR_WORKSPACE for a missing or short workspace
+ * and MS_ERR_ALIGNMENT for a misaligned one; a persistent launch whose carry
+ * wait runs out leaves MS_ERR_TIMEOUT in the workspace's status word (see
+ * mamba_scan_fwd_with_plan).
+ */
+ms_status mamba_trap_scan_workspace_size(const ms_scan_args *args, const void *lambda_raw,
+                                         int64_t lambda_batch_stride, int64_t lambda_dim_stride,
+                                         const ms_scan_plan *plan, size_t *bytes);
+ms_status mamba_trap_scan_fwd_ws(const ms_scan_args *args, const void *lambda_raw, int64_t lambda_batch_stride,
+                                 int64_t lambda_dim_stride, const ms_scan_plan *plan, void *workspace,
+                                 size_t workspace_bytes, void *stream);
 
 /* ---- Backward pass ---------------------------------------------------------
  * Gradients of the selective scan for the loss sum(y dy) + sum(h_T dh_T)

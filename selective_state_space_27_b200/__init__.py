@@ -169,6 +169,12 @@ def load_library():
         lib.mamba_conv_scan_fwd_ws.restype = ctypes.c_int
         lib.mamba_conv_scan_fwd_ws.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(Conv1dArgs),
                                                ctypes.POINTER(ScanPlan), _vp, ctypes.c_size_t, _vp]
+        lib.mamba_trap_scan_workspace_size.restype = ctypes.c_int
+        lib.mamba_trap_scan_workspace_size.argtypes = [ctypes.POINTER(ScanArgs), _vp, ctypes.c_int64, ctypes.c_int64,
+                                                       ctypes.POINTER(ScanPlan), ctypes.POINTER(ctypes.c_size_t)]
+        lib.mamba_trap_scan_fwd_ws.restype = ctypes.c_int
+        lib.mamba_trap_scan_fwd_ws.argtypes = [ctypes.POINTER(ScanArgs), _vp, ctypes.c_int64, ctypes.c_int64,
+                                               ctypes.POINTER(ScanPlan), _vp, ctypes.c_size_t, _vp]
         lib.mamba_scan_fwd_checkpointed.restype = ctypes.c_int
         lib.mamba_scan_fwd_checkpointed.argtypes = [ctypes.POINTER(ScanArgs), _vp, ctypes.c_size_t, _vp,
                                                     ctypes.c_size_t, _vp]
@@ -519,7 +525,8 @@ def trap_scan_fwd(u, delta, lambda_raw, A, B, C, D=None, z=None, delta_bias=None
                   initial_state=None, return_last_state=True, out=None, stream=None, plan=None):
     """Exponential-trapezoidal selective scan (Mamba-3): as :func:`scan_fwd`
     plus ``lambda_raw`` (batch, dim, L) in u's dtype, lambda = sigmoid(lambda_raw)
-    mixing the previous and the current input (no segments)."""
+    mixing the previous and the current input (no segments); ``plan`` may ask
+    for the persistent schedule (ctas > 0), whose workspace is allocated here."""
     torch = _torch()
     _need_cuda("lambda_raw", lambda_raw, u.dtype, 3)
     if tuple(lambda_raw.shape) != tuple(u.shape):
@@ -530,10 +537,18 @@ def trap_scan_fwd(u, delta, lambda_raw, A, B, C, D=None, z=None, delta_bias=None
         hT = torch.empty((u.shape[0], u.shape[1], B.shape[1]), device=u.device, dtype=torch.float32)
     args = build_scan_args(u, delta, A, B, C, y, D=D, z=z, delta_bias=delta_bias, delta_softplus=delta_softplus,
                            initial_state=initial_state, final_state=hT)
+    lib = load_library()
+    plan_ref = None if plan is None else ctypes.byref(plan)
+    lam = (_ptr(lambda_raw), lambda_raw.stride(0), lambda_raw.stride(1))
     with torch.cuda.device(u.device):
-        _check(load_library().mamba_trap_scan_fwd(ctypes.byref(args), _ptr(lambda_raw), lambda_raw.stride(0),
-                                                  lambda_raw.stride(1), None if plan is None else ctypes.byref(plan),
-                                                  _stream_ptr(stream)))
+        n = ctypes.c_size_t(0)
+        _check(lib.mamba_trap_scan_workspace_size(ctypes.byref(args), *lam, plan_ref, ctypes.byref(n)))
+        workspace = torch.empty(n.value, dtype=torch.uint8, device=u.device) if n.value else None
+        _check(lib.mamba_trap_scan_fwd_ws(ctypes.byref(args), *lam, plan_ref,
+                                          None if workspace is None else workspace.data_ptr(), n.value,
+                                          _stream_ptr(stream)))
+        if workspace is not None:
+            _keep_until_done(workspace, stream)
     return (y, hT) if return_last_state else y
 
 

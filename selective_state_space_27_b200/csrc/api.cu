@@ -431,9 +431,9 @@ ms_status mamba_conv_scan_fwd_ws(const ms_scan_args *args, const ms_conv1d_args 
     return conv_scan_impl(args, conv, plan, workspace, workspace_bytes, stream, true, nullptr);
 }
 
-ms_status mamba_trap_scan_fwd(const ms_scan_args *args, const void *lambda_raw, int64_t lambda_batch_stride,
-                              int64_t lambda_dim_stride, const ms_scan_plan *plan, void *stream) {
-    const CallRange range("mamba_trap_scan_fwd");
+static ms_status trap_scan_impl(const ms_scan_args *args, const void *lambda_raw, int64_t lambda_batch_stride,
+                                int64_t lambda_dim_stride, const ms_scan_plan *plan, void *workspace,
+                                size_t workspace_bytes, void *stream, bool with_workspace, size_t *query) {
     ms_status st = check_scan(args);
     if (st != MS_OK) return st;
     if (!lambda_raw) return invalid("lambda_raw is required");
@@ -450,25 +450,54 @@ ms_status mamba_trap_scan_fwd(const ms_scan_args *args, const void *lambda_raw, 
     p.lambda_raw = lambda_raw;
     p.lm_sb = lambda_batch_stride;
     p.lm_sd = lambda_dim_stride;
+    int sms = 0;
+    st = device_sms(&sms);
+    if (st != MS_OK) return st;
     ms::ScanPlan pl{};
     if (plan) {
-        if (plan->ctas != 0 || plan->reserved != 0 ||
-            !ms::make_plan(p, args->in_dtype, plan->config, plan->warps_per_cta, plan->segments, 0, 0, &pl)) {
-            set_error("plan (config %d, %d warps, %d segments) cannot run the trapezoidal rule", plan->config,
-                      plan->warps_per_cta, plan->segments);
+        if ((!with_workspace && plan->ctas != 0) || plan->reserved != 0 ||
+            !ms::make_plan(p, args->in_dtype, plan->config, plan->warps_per_cta, plan->segments, plan->ctas, sms,
+                           &pl)) {
+            set_error("plan (config %d, %d warps, %d segments, %d CTAs) cannot run the trapezoidal rule",
+                      plan->config, plan->warps_per_cta, plan->segments, plan->ctas);
             return MS_ERR_UNSUPPORTED;
         }
     } else {
-        int sms = 0;
-        st = device_sms(&sms);
-        if (st != MS_OK) return st;
-        pl = ms::plan_scan(p, args->in_dtype, 0, sms);
+        pl = ms::plan_scan(p, args->in_dtype, 0, sms, with_workspace);
         if (pl.kind != 1) {
             set_error("no kernel configuration runs the trapezoidal rule for these arguments");
             return MS_ERR_UNSUPPORTED;
         }
     }
-    return run_plan(p, pl, args->in_dtype, nullptr, 0, stream);
+    if (query) {
+        *query = pl.ws_bytes;
+        return MS_OK;
+    }
+    return run_plan(p, pl, args->in_dtype, workspace, workspace_bytes, stream);
+}
+
+ms_status mamba_trap_scan_fwd(const ms_scan_args *args, const void *lambda_raw, int64_t lambda_batch_stride,
+                              int64_t lambda_dim_stride, const ms_scan_plan *plan, void *stream) {
+    const CallRange range("mamba_trap_scan_fwd");
+    return trap_scan_impl(args, lambda_raw, lambda_batch_stride, lambda_dim_stride, plan, nullptr, 0, stream, false,
+                          nullptr);
+}
+
+ms_status mamba_trap_scan_workspace_size(const ms_scan_args *args, const void *lambda_raw,
+                                         int64_t lambda_batch_stride, int64_t lambda_dim_stride,
+                                         const ms_scan_plan *plan, size_t *bytes) {
+    if (!bytes) return invalid("bytes is NULL");
+    *bytes = 0;
+    return trap_scan_impl(args, lambda_raw, lambda_batch_stride, lambda_dim_stride, plan, nullptr, 0, nullptr, true,
+                          bytes);
+}
+
+ms_status mamba_trap_scan_fwd_ws(const ms_scan_args *args, const void *lambda_raw, int64_t lambda_batch_stride,
+                                 int64_t lambda_dim_stride, const ms_scan_plan *plan, void *workspace,
+                                 size_t workspace_bytes, void *stream) {
+    const CallRange range("mamba_trap_scan_fwd_ws");
+    return trap_scan_impl(args, lambda_raw, lambda_batch_stride, lambda_dim_stride, plan, workspace,
+                          workspace_bytes, stream, true, nullptr);
 }
 
 ms_status mamba_scan_bwd_workspace_size(const ms_scan_args *args, size_t *bytes) {

@@ -722,9 +722,8 @@ ScanPlan plan_scan(const ScanParams &p, int in_dtype, int force_segments, int nu
                 rec = ri;
                 rec_ctas = 0;
             }
-            // persistent schedule: m CTAs on every SM share the units' work exactly (not the trapezoidal
-            // rule, whose carry would need the previous step's input)
-            if (persistent_ok && variant != 2 && p.batch * p.dim <= (int64_t(1) << 30) &&
+            // persistent schedule: m CTAs on every SM share the units' work exactly
+            if (persistent_ok && p.batch * p.dim <= (int64_t(1) << 30) &&
                 (p.seqlen + 15) / 16 < (int64_t(1) << 30)) {
                 for (int m = 1; m <= per_sm && static_cast<int64_t>(m) * sms <= ctas; ++m) {
                     const double tp = static_cast<double>(ctas) * R * static_cast<double>(p.seqlen) / sms *
@@ -775,10 +774,9 @@ bool make_plan(const ScanParams &p, int in_dtype, int config, int warps, int seg
         plan.ws_bytes = 0;
         plan.ctas = 0;
         if (ctas > 0) {
-            // persistent schedule: every CTA resident, at most one per unit,
-            // no trapezoidal rule (its carry would need the previous step's input)
+            // persistent schedule: every CTA resident, at most one per unit
             const int64_t units = p.batch * ((p.dim + plan.rows_per_cta - 1) / plan.rows_per_cta);
-            if (rec_variant(p) == 2 || units > (int64_t(1) << 30) || p.batch * p.dim > (int64_t(1) << 30) ||
+            if (units > (int64_t(1) << 30) || p.batch * p.dim > (int64_t(1) << 30) ||
                 (p.seqlen + rec_chunk() - 1) / rec_chunk() >= (int64_t(1) << 30))
                 return false;
             if (ctas > rec_max_ctas(p, in_dtype, plan.lg, plan.vec != 0, num_sms > 0 ? num_sms : 148, iow)) return false;

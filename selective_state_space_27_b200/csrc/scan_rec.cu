@@ -451,7 +451,8 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
     // the packed instructions take (no moves in the loop); set at the start of
     // every piece of work.
     float2 ap[NP], hp[NP];
-    float2 bprev[NP];   // trapezoidal rule: the lane's B_{t-1} entries (B_{-1} u_{-1} = 0 via its coefficient)
+    float2 bprev[NP];   // trapezoidal rule: the lane's B_{t-1} entries (B_{-1} u_{-1} = 0 via its coefficient;
+                        // a piece that starts inside a row reads B at its step before from memory)
     int s = 0;          // tile stage of chunk it
     int64_t it = 0;     // position in the CTA's list of chunks
     const int npieces = num_pieces(sc);
@@ -469,20 +470,28 @@ __device__ __forceinline__ void recurrence_role(const ScanParams &p, unsigned ch
             const int64_t dc = ur.dc;
             const float *hsrc = carried ? p.sk_carry + (static_cast<int64_t>(pr.u) * R + r) * kStates
                                         : (p.h0 ? p.h0 + row * dstate : nullptr);
+            const T *bsrc = nullptr;
+            if constexpr (TRAP) {
+                if (carried)
+                    bsrc = static_cast<const T *>(p.B) + ur.b * p.B_sb + static_cast<int64_t>(pr.c0) * kSteps - 1;
+            }
 #pragma unroll
             for (int j = 0; j < NP; ++j) {
-                float a2[2] = {0.f, 0.f}, h2[2] = {0.f, 0.f};
+                float a2[2] = {0.f, 0.f}, h2[2] = {0.f, 0.f}, b2[2] = {0.f, 0.f};
 #pragma unroll
                 for (int e = 0; e < 2 && 2 * j + e < NPL; ++e) {
                     const int n = q * NPL + 2 * j + e;
                     if (n < dstate) {
                         a2[e] = __ldg(p.A + dc * dstate + n) * kLog2e;
                         if (hsrc) h2[e] = carried ? __ldcg(hsrc + n) : __ldg(hsrc + n);
+                        if constexpr (TRAP) {
+                            if (bsrc) b2[e] = to_f32<T>(bsrc[n * p.B_sn]);
+                        }
                     }
                 }
                 ap[j] = f2(a2[0], a2[1]);
                 hp[j] = f2(h2[0], h2[1]);
-                bprev[j] = f2(0.f, 0.f);
+                bprev[j] = f2(b2[0], b2[1]);
             }
         }
         for (int c = pr.c0; c < pr.c1; ++c, ++it, s = next_stage(s, kTileStages)) {
@@ -1295,7 +1304,7 @@ int rec_max_ctas(const ScanParams &p, int in_dtype, int lpr, bool vec, int num_s
 cudaError_t launch_rec(const ScanParams &p, int lpr, bool vec, int in_dtype, int iow, cudaStream_t stream) {
     const int variant = rec_variant(p);
     if (!rec_supports_variant(lpr, variant, iow) || (p.conv_w && p.lambda_raw)) return cudaErrorInvalidValue;
-    if (p.sk_ctas > 0 && (variant == 2 || !p.sk_carry || !p.sk_flag || !p.sk_status)) return cudaErrorInvalidValue;
+    if (p.sk_ctas > 0 && (!p.sk_carry || !p.sk_flag || !p.sk_status)) return cudaErrorInvalidValue;
     // a persistent launch with at most one CTA per SM takes the instantiation
     // without the occupancy bound on registers
     const bool one = p.sk_ctas > 0 && p.sk_ctas <= device_sms();

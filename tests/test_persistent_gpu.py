@@ -78,7 +78,10 @@ def test_long_rows_split_many_times():
 
 
 def test_refused_plans():
-    """More CTAs than units, or the trapezoidal rule, are refused before any launch."""
+    """More CTAs than units, or CTAs on an entry point that takes no workspace,
+    are refused before any launch."""
+    import ctypes
+
     import torch
     ms = _ms()
     inp = make_scan_inputs(LAYER, batch=1, dim=64, seqlen=100, seed=8200)
@@ -90,8 +93,14 @@ def test_refused_plans():
     lam = torch.zeros_like(dev["u"])
     with pytest.raises(ms.MambaScanError) as ei:
         ms.trap_scan_fwd(dev["u"], dev["delta"], lam, dev["A"], dev["B"], dev["C"],
-                         plan=ms.ScanPlan(config=cfg, warps_per_cta=6, segments=1, ctas=1))
+                         plan=ms.ScanPlan(config=cfg, warps_per_cta=6, segments=1, ctas=3))
     assert ei.value.status == 2
+    lib = ms.load_library()
+    args = ms.build_scan_args(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], torch.empty_like(dev["u"]))
+    plan = ms.ScanPlan(config=cfg, warps_per_cta=6, segments=1, ctas=1)
+    assert lib.mamba_trap_scan_fwd(ctypes.byref(args), lam.data_ptr(), lam.stride(0), lam.stride(1),
+                                   ctypes.byref(plan), None) == 2
+    torch.cuda.synchronize()
 
 
 def test_automatic_plan_long_context_shape():

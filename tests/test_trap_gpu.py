@@ -71,6 +71,34 @@ def test_trap_scan_matches_oracle(dtype, batch, dim, N, L, offset):
         assert rel_err(hT, hr) <= TOL[dtype], tag
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("batch,dim,N,L", [(2, 100, 16, 300), (3, 40, 5, 257)])
+def test_trap_scan_persistent_schedule(dtype, batch, dim, N, L):
+    """The rule under the persistent schedule: every configuration that runs it
+    at CTA counts from 1 to one per unit, including counts that cut units
+    between CTAs (the CTA that takes a row over starts from the handed-over
+    state and reads B at the step before its first one), on ragged lengths and
+    a state size below 16."""
+    import torch
+    ms = _ms()
+    inp = make_scan_inputs(LAYER, batch=batch, dim=dim, dstate=N, seqlen=L, dtype=dtype, seed=3500 + L)
+    lam = make_lambda_raw(batch, dim, L, dtype, seed=3600 + L)
+    dev = device_inputs(inp)
+    lam_t = to_device(lam, dtype)
+    h0 = np.random.default_rng(3700 + L).normal(size=(batch, dim, N)).astype(np.float32)
+    h0_t = torch.from_numpy(h0).cuda()
+    yr, hr = _oracle(inp, lam, h0=h0.reshape(-1, N))
+    for c, lanes, w in _trap_configs():
+        rows = 128 // lanes
+        units = batch * ((dim + rows - 1) // rows)
+        for ctas in sorted({1, 2, 3, max(1, units // 2), max(1, units - 1), units}):
+            plan = ms.ScanPlan(config=c, warps_per_cta=w, segments=1, ctas=ctas)
+            y, hT = _run(dev, lam_t, plan=plan, h0=h0_t)
+            tag = f"config {c}, {ctas} CTAs of {units} units"
+            assert rel_err(y, yr) <= TOL[dtype], tag
+            assert rel_err(hT, hr) <= TOL[dtype], tag
+
+
 def test_trap_with_lambda_one_is_the_euler_scan():
     """lambda = sigmoid(20) = 1 in float32: the rule reduces to exponential-Euler,
     so the result matches the plain scan's oracle."""
