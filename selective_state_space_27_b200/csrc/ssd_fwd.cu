@@ -55,10 +55,9 @@ constexpr uint32_t kBCTile = 2 * kQ * 128;               // 128 tokens x 128 bf1
 constexpr uint32_t kStageBytes = kXTile + 2 * kBCTile;   // X, B, C
 constexpr uint32_t kOffM = kStages * kStageBytes;        // M' (128 x 128 bf16, two atoms along i)
 constexpr uint32_t kOffXt = kOffM + 2 * kQ * 128;        // Xt (128 tokens x 64 bf16)
-constexpr uint32_t kOffH = kOffXt + kXTile;              // H (64 rows p x 128 bf16, two atoms along n)
-constexpr uint32_t kHAtom = kP * 128;
+constexpr uint32_t kOffH = kOffXt + kXTile;              // H (128 rows n x 64 bf16 along p)
 // step data of two chunks: float delta[2][Q], float s2[2][Q], bf16 cf[2][Q]; then int abort
-constexpr uint32_t kOffStep = kOffH + 2 * kHAtom;
+constexpr uint32_t kOffStep = kOffH + kN * 128;
 constexpr uint32_t kOffAbort = kOffStep + 2 * kQ * 10;
 constexpr uint32_t kOffBar = kOffAbort + 16;
 // mbarriers and their phases (chunk c completes phase c of a single barrier, or
@@ -329,27 +328,21 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr)
     return v;
 }
 
-__device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v)
-{
-    asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
-}
-
 __device__ __forceinline__ float load_bf16(const void *p, int64_t i)
 {
     return __uint_as_float((uint32_t)reinterpret_cast<const uint16_t *>(p)[i] << 16);
 }
 
 // The running state H[p][n] of this thread (n = its row r, p = 16 hq + j) as
-// bf16 into the K-major operand tile of the Yo product (rows p, K = n).
+// bf16 into the MN-major operand tile of the Yo product (rows K = n, p
+// contiguous): the thread's 16 values are two 16-byte chunks of row r.
 __device__ __forceinline__ void store_state_tile(uint32_t tile, int r, int hq, const float (&H)[16])
 {
-    const uint32_t col = tile + (uint32_t)(r >> 6) * kHAtom + (uint32_t)(r & 7) * 2u;
-    const uint32_t q = (uint32_t)(r & 63) >> 3;
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-        const __nv_bfloat16 v = __float2bfloat16_rn(H[j]);
-        st_shared_u16(col + sw128((uint32_t)(16 * hq + j), q), *reinterpret_cast<const uint16_t *>(&v));
-    }
+    for (int q = 0; q < 2; ++q)
+        st_shared_v4(tile + sw128((uint32_t)r, (uint32_t)(2 * hq + q)), pack_bf16(H[8 * q], H[8 * q + 1]),
+                     pack_bf16(H[8 * q + 2], H[8 * q + 3]), pack_bf16(H[8 * q + 4], H[8 * q + 5]),
+                     pack_bf16(H[8 * q + 6], H[8 * q + 7]));
 }
 
 // M' for row r (row block K, this warp's quarter hq): column groups of 8 at
@@ -547,7 +540,7 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
         // ---- MMA issue (one thread) ----
         if (lane == 0) {
             constexpr uint32_t id_g = bf16_idesc(128, 128, false, false);   // G = C B^T
-            constexpr uint32_t id_yo = bf16_idesc(128, 64, false, false);   // Yo = C H^T
+            constexpr uint32_t id_yo = bf16_idesc(128, 64, false, true);    // Yo = C H^T
             constexpr uint32_t id_s = bf16_idesc(128, 64, true, true);      // S = B^T Xt
             constexpr uint32_t id_yd = bf16_idesc(128, 64, false, true);    // Yd = M' X
             for (int c = 0; c < nchunks; ++c) {
@@ -575,9 +568,8 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const uint32_t offc = (uint32_t)(k >> 2) * (kQ * 128) + (uint32_t)(k & 3) * 32u;
-                    const uint32_t offh = (uint32_t)(k >> 2) * kHAtom + (uint32_t)(k & 3) * 32u;
                     mma_bf16(tmem + kColYo, sw128_desc(sc + offc, 16, 1024),
-                             sw128_desc(base + kOffH + offh, 16, 1024), id_yo, k > 0);
+                             sw128_desc(base + kOffH + (uint32_t)k * 2048u, kXTile, 1024), id_yo, k > 0);
                 }
                 // S and Yd need M' and Xt of this chunk
                 if (!role_wait(bar(kPReady), c & 1, abort_flag, wlim)) {
@@ -662,16 +654,26 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
                 case 2: build_mask_rows<2>(tg, base + kOffM, r, hq, sr, dl, s2, cf); break;
                 default: build_mask_rows<3>(tg, base + kOffM, r, hq, sr, dl, s2, cf); break;
                 }
-                const float wr = ex2(se - sr) * dl[r];
+                // Xt: the 1024 16-byte pieces (token i, 8 p each) go mostly to the
+                // sub-partitions with the fewest mask groups: 4, 3, 1 and 0
+                // pieces per thread on sub-partitions 0..3.
                 const uint32_t sx = base + (uint32_t)stk * kStageBytes;
+                const int tsub = hq * 32 + lane;
+                const int npc = sub == 0 ? 4 : sub == 1 ? 3 : sub == 2 ? 1 : 0;
+                const int pc0 = sub == 0 ? 0 : sub == 1 ? 512 : 896;
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const uint32_t off = sw128((uint32_t)r, (uint32_t)(2 * hq + q));
-                    const uint4 v = ld_shared_v4(sx + off);
-                    st_shared_v4(base + kOffXt + off, pack_bf16(bf16_lo(v.x) * wr, bf16_hi(v.x) * wr),
-                                 pack_bf16(bf16_lo(v.y) * wr, bf16_hi(v.y) * wr),
-                                 pack_bf16(bf16_lo(v.z) * wr, bf16_hi(v.z) * wr),
-                                 pack_bf16(bf16_lo(v.w) * wr, bf16_hi(v.w) * wr));
+                for (int k = 0; k < 4; ++k) {
+                    if (k < npc) {
+                        const int pc = pc0 + 128 * k + tsub;
+                        const int i = pc >> 3;
+                        const float wr = ex2(se - s2[i]) * dl[i];
+                        const uint32_t off = sw128((uint32_t)i, (uint32_t)(pc & 7));
+                        const uint4 v = ld_shared_v4(sx + off);
+                        st_shared_v4(base + kOffXt + off, pack_bf16(bf16_lo(v.x) * wr, bf16_hi(v.x) * wr),
+                                     pack_bf16(bf16_lo(v.y) * wr, bf16_hi(v.y) * wr),
+                                     pack_bf16(bf16_lo(v.z) * wr, bf16_hi(v.z) * wr),
+                                     pack_bf16(bf16_lo(v.w) * wr, bf16_hi(v.w) * wr));
+                    }
                 }
             }
             async_proxy_fence();
