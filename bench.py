@@ -56,7 +56,6 @@ MUFU_PER_CLK = 16
 NCU_TRAFFIC = {("long_context_131k", 10, 148): (505176320 + 150065408) * 8,
                ("mamba130m_layer", 10, 296): 152307456 + 32844800,
                ("mamba1p4b_layer", 10, 444): 813864448 + 252678912,
-               ("mamba2_layer_d2048", "ssd_kernel"): 563170560 + 243913472,
                ("decode_b256_d5120", "state_update_vec_kernel"): 92157440 + 29935104}
 FP32_PER_CLK = 128
 # FP32 operations of one exponential on the FMA pipe (the combined MUFU + FMA bound)
@@ -931,11 +930,18 @@ def run_ssd(args, dist: Dist, dev, peaks):
     prm = {k: dev_t(inp[k], False) for k in ("A", "D", "dt_bias")}
     y = torch.empty_like(t["x"])
     hT = torch.empty((w.batch, w.nheads, w.headdim, w.dstate), dtype=torch.float32, device=dev)
-    status = torch.zeros(ms.SSD_WORKSPACE_BYTES, dtype=torch.uint8, device=dev)
     a = ms.build_ssd_args(t["x"], t["dt"], prm["A"], t["B"], t["C"], y, D=prm["D"], z=t["z"],
                           dt_bias=prm["dt_bias"], final_state=hT)
     lib = ms.load_library()
     stream = torch.cuda.current_stream()
+    nbytes = ctypes.c_size_t(0)
+    rc = lib.mamba_ssd_workspace_size(ctypes.byref(a), ctypes.byref(nbytes))
+    if rc != 0:
+        raise ms.MambaScanError(rc, lib.mamba_last_error().decode())
+    status = torch.zeros(nbytes.value, dtype=torch.uint8, device=dev)   # status word (+ hand-over slots)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    schedule = (f"persistent: {sms} CTAs over {w.batch * w.nheads} (batch, head) sequences"
+                if nbytes.value > ms.SSD_WORKSPACE_BYTES else "one CTA per (batch, head)")
 
     def step():
         rc = lib.mamba_ssd_fwd(ctypes.byref(a), status.data_ptr(), status.numel(), stream.cuda_stream)
@@ -962,7 +968,7 @@ def run_ssd(args, dist: Dist, dev, peaks):
         "value": dist.world * c["elements"] / (us * 1e-6), "us_per_step": us,
         "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "nheads": w.nheads,
                    "headdim": w.headdim, "dstate": w.dstate, "ngroups": w.ngroups, "chunk": 128, "dtype": "bf16",
-                   "l2": "inputs larger than L2"},
+                   "l2": "inputs larger than L2", "schedule": schedule},
         "roofline": {"bound": "hbm", "unit": "GB/s", "achieved": gbs, "peak": peaks["hbm_gbs"],
                      "frac": gbs / peaks["hbm_gbs"], "traffic": NCU_TRAFFIC.get((w.name, "ssd_kernel")),
                      "peak_source": peaks["source"], "algorithmic_per_launch": c,

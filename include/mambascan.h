@@ -503,19 +503,36 @@ typedef struct ms_ssd_args {
     int32_t withhold_block;
 } ms_ssd_args;
 
-/* Device workspace of mamba_ssd_fwd: a status word (int32 at offset 0). */
+/* Smallest device workspace of mamba_ssd_fwd: a status word (int32 at offset
+ * 0). Enough for one CTA per (batch, head); see mamba_ssd_workspace_size. */
 #define MS_SSD_WORKSPACE_BYTES 256
 
 /*
- * SSD forward: one kernel launch on `stream` (after clearing the status word),
- * one CTA per (batch, head) walking the sequence in blocks of 128 tokens. The
- * block products run on the tensor cores in bf16 with fp32 accumulation; the
- * state passed between blocks stays in fp32 on chip. The caller owns the
- * workspace (MS_SSD_WORKSPACE_BYTES, 16-byte aligned). After synchronizing,
- * its first int32 is 0 when the kernel finished normally, MS_ERR_TIMEOUT when
- * one of the kernel's internal pipeline waits gave up after about a second
- * (the outputs are then incomplete), or MS_ERR_ALIGNMENT when the kernel's
- * shared memory window was not 1024-byte aligned (nothing was computed).
+ * Workspace bytes with which mamba_ssd_fwd takes its best schedule for these
+ * arguments on the current device (at least MS_SSD_WORKSPACE_BYTES). When
+ * there are more (batch, head) pairs than SMs and they would leave the last
+ * wave partly empty, that is the persistent schedule: one resident CTA per SM,
+ * the chunks of all pairs cut evenly over them, and a pair's state handed
+ * from one CTA to the next through the workspace (status word, one flag per
+ * CTA, then 64 x 128 floats per CTA). Errors as mamba_ssd_fwd's argument checks;
+ * MS_ERR_INVALID_ARG for a NULL bytes.
+ */
+ms_status mamba_ssd_workspace_size(const ms_ssd_args *args, size_t *bytes);
+
+/*
+ * SSD forward: one kernel launch on `stream` (after clearing the status word
+ * and, for the persistent schedule, the flags). A CTA walks a sequence in
+ * blocks of 128 tokens: one CTA per (batch, head), or, with a workspace of at
+ * least mamba_ssd_workspace_size bytes that asks for it, the persistent
+ * schedule (a cooperative launch). The block products run on the tensor cores
+ * in bf16 with fp32 accumulation; the state passed between blocks stays in
+ * fp32 (on chip, or in the workspace between two CTAs). The caller owns the
+ * workspace (at least MS_SSD_WORKSPACE_BYTES, 16-byte aligned). After
+ * synchronizing, its first int32 is 0 when the kernel finished normally,
+ * MS_ERR_TIMEOUT when one of the kernel's internal waits (pipeline, or the
+ * hand-over between CTAs) gave up after about a second (the outputs are then
+ * incomplete), or MS_ERR_ALIGNMENT when the kernel's shared memory window was
+ * not 1024-byte aligned (nothing was computed).
  * The tensor maps the kernel reads through are encoded on the host by the
  * driver's encoder, looked up once per process. Errors: MS_ERR_INVALID_ARG
  * for NULL or negative sizes, strides or pointers, or nheads not a multiple

@@ -196,6 +196,8 @@ def load_library():
                                                  ctypes.c_size_t, _vp]
         lib.mamba_ssd_fwd.restype = ctypes.c_int
         lib.mamba_ssd_fwd.argtypes = [ctypes.POINTER(SsdArgs), _vp, ctypes.c_size_t, _vp]
+        lib.mamba_ssd_workspace_size.restype = ctypes.c_int
+        lib.mamba_ssd_workspace_size.argtypes = [ctypes.POINTER(SsdArgs), ctypes.POINTER(ctypes.c_size_t)]
         lib.mamba_probe_unit_throughput.restype = ctypes.c_int
         lib.mamba_probe_unit_throughput.argtypes = [ctypes.c_int, _vp, ctypes.POINTER(ctypes.c_double),
                                                     ctypes.POINTER(ctypes.c_double), _vp]
@@ -687,8 +689,9 @@ def ssd_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True, init
 
     Shapes as :func:`build_ssd_args`. Returns ``(y, final_state)``
     (final_state None when not asked for). ``workspace``: a uint8 CUDA tensor
-    of at least ``SSD_WORKSPACE_BYTES`` bytes holding the status word (one is
-    allocated when None). With ``check`` the call synchronizes the stream and
+    of at least ``SSD_WORKSPACE_BYTES`` bytes holding the status word; when
+    None, one of ``mamba_ssd_workspace_size`` bytes is allocated, which lets
+    the call take the persistent schedule. With ``check`` the call synchronizes the stream and
     raises if the kernel reported a failed wait; without it, call
     :func:`ssd_check` on the workspace later. ``wait_limit_us`` bounds each
     of the kernel's pipeline waits (0: about one second); ``withhold_block``
@@ -704,11 +707,13 @@ def ssd_fwd(x, dt, A, B, C, D=None, z=None, dt_bias=None, dt_softplus=True, init
     args.wait_limit_us = int(wait_limit_us)
     args.withhold_block = int(withhold_block)
     own_ws = workspace is None
-    if own_ws:
-        workspace = torch.empty(SSD_WORKSPACE_BYTES, dtype=torch.uint8, device=x.device)
+    lib = load_library()
     with torch.cuda.device(x.device):
-        _check(load_library().mamba_ssd_fwd(ctypes.byref(args), workspace.data_ptr(), workspace.numel(),
-                                             _stream_ptr(stream)))
+        if own_ws:
+            n = ctypes.c_size_t(0)
+            _check(lib.mamba_ssd_workspace_size(ctypes.byref(args), ctypes.byref(n)))
+            workspace = torch.empty(n.value, dtype=torch.uint8, device=x.device)
+        _check(lib.mamba_ssd_fwd(ctypes.byref(args), workspace.data_ptr(), workspace.numel(), _stream_ptr(stream)))
         if own_ws:
             _keep_until_done(workspace, stream)
     if check:

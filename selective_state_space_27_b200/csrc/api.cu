@@ -610,8 +610,7 @@ ms_status mamba_scan_fwd_checkpointed(const ms_scan_args *args, float *checkpoin
     return run_plan(p, plan, args->in_dtype, workspace, workspace_bytes, stream);
 }
 
-ms_status mamba_ssd_fwd(const ms_ssd_args *a, void *workspace, size_t workspace_bytes, void *stream) {
-    const CallRange range("mamba_ssd_fwd");
+static ms_status check_ssd(const ms_ssd_args *a) {
     if (!a) return invalid("args is NULL");
     if (a->batch <= 0 || a->seqlen <= 0 || a->nheads <= 0 || a->ngroups <= 0)
         return invalid("batch, seqlen, nheads and ngroups must be positive");
@@ -653,6 +652,35 @@ ms_status mamba_ssd_fwd(const ms_ssd_args *a, void *workspace, size_t workspace_
         set_error("x, y, B, C and z must be 16-byte aligned, the other pointers aligned to their elements");
         return MS_ERR_ALIGNMENT;
     }
+    if (a->withhold_block < 0) return invalid("withhold_block must be >= 0");
+    return MS_OK;
+}
+
+// CTAs of the persistent schedule the call would take (0: one CTA per (batch, head)).
+static ms_status ssd_plan_ctas(const ms_ssd_args *a, int *ctas) {
+    int sms = 0;
+    const ms_status st = device_sms(&sms);
+    if (st != MS_OK) return st;
+    *ctas = ms::ssd_persistent_ctas(a->batch, a->nheads, a->seqlen, sms);
+    return MS_OK;
+}
+
+ms_status mamba_ssd_workspace_size(const ms_ssd_args *a, size_t *bytes) {
+    if (!bytes) return invalid("bytes is NULL");
+    *bytes = 0;
+    ms_status st = check_ssd(a);
+    if (st != MS_OK) return st;
+    int ctas = 0;
+    st = ssd_plan_ctas(a, &ctas);
+    if (st != MS_OK) return st;
+    *bytes = ctas ? ms::ssd_persistent_ws_bytes(ctas) : static_cast<size_t>(MS_SSD_WORKSPACE_BYTES);
+    return MS_OK;
+}
+
+ms_status mamba_ssd_fwd(const ms_ssd_args *a, void *workspace, size_t workspace_bytes, void *stream) {
+    const CallRange range("mamba_ssd_fwd");
+    ms_status st = check_ssd(a);
+    if (st != MS_OK) return st;
     if (!workspace || workspace_bytes < MS_SSD_WORKSPACE_BYTES) {
         set_error("workspace of %d bytes needed, %zu given", MS_SSD_WORKSPACE_BYTES,
                   workspace ? workspace_bytes : static_cast<size_t>(0));
@@ -673,13 +701,18 @@ ms_status mamba_ssd_fwd(const ms_ssd_args *a, void *workspace, size_t workspace_
     p.batch = a->batch; p.seqlen = a->seqlen; p.nheads = a->nheads; p.ngroups = a->ngroups;
     p.softplus = a->dt_softplus ? 1 : 0;
     p.status = static_cast<int *>(workspace);
-    if (a->withhold_block < 0) return invalid("withhold_block must be >= 0");
     p.wait_limit_ns = a->wait_limit_us ? 1000ull * a->wait_limit_us : 1000000000ull;
     p.withhold_block = a->withhold_block;
+    int ctas = 0;
+    st = ssd_plan_ctas(a, &ctas);
+    if (st != MS_OK) return st;
+    if (ctas > 0 && workspace_bytes >= ms::ssd_persistent_ws_bytes(ctas)) {
+        p.sk_ctas = ctas;
+        p.sk_flag = reinterpret_cast<int *>(static_cast<char *>(workspace) + ms::ssd_flag_offset());
+        p.sk_carry = reinterpret_cast<float *>(static_cast<char *>(workspace) + ms::ssd_carry_offset(ctas));
+    }
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int), s);
-    if (e != cudaSuccess) return cuda_fail(e, "clearing the SSD status word");
-    e = ms::launch_ssd(p, s);
+    const cudaError_t e = ms::launch_ssd(p, s);
     if (e == cudaErrorNotSupported) {
         set_error("the driver offers no tensor-map encoder");
         return MS_ERR_UNSUPPORTED;

@@ -171,13 +171,30 @@ struct SsdParams {
     int *status;
     uint64_t wait_limit_ns;   // limit of each pipeline wait
     int withhold_block;       // tests: k > 0 withholds block k - 1's loads (the wait for them runs out)
+    // Persistent schedule (sk_ctas > 0): the chunks of all (batch, head) pairs
+    // form one list cut evenly over sk_ctas resident CTAs; CTA g hands the
+    // state at the end of its first piece to CTA g + 1 through sk_carry[g]
+    // (64 x 128 floats) and raises sk_flag[g]. 0: one CTA per (batch, head).
+    int sk_ctas;
+    int *sk_flag;
+    float *sk_carry;
 };
 constexpr int kSsdHeadDim = 64;
 constexpr int kSsdState = 128;
 constexpr int kSsdChunk = 128;
-// Encodes the kernel's tensor maps and launches it. Returns cudaErrorNotSupported
-// when the driver offers no tensor-map encoder.
+// Encodes the kernel's tensor maps and launches it (cooperatively for the
+// persistent schedule, after clearing the status word and the carry flags).
+// Returns cudaErrorNotSupported when the driver offers no tensor-map encoder.
 cudaError_t launch_ssd(const SsdParams &p, cudaStream_t stream);
+// CTAs of the persistent schedule for these sizes on num_sms SMs (one CTA per
+// SM), or 0 when one CTA per (batch, head) does as well.
+int ssd_persistent_ctas(int64_t batch, int64_t nheads, int64_t seqlen, int num_sms);
+// Workspace bytes of the persistent schedule over ctas CTAs (status word,
+// flags and carries).
+size_t ssd_persistent_ws_bytes(int ctas);
+// Offsets of the flags and the carries in that workspace.
+size_t ssd_flag_offset();
+size_t ssd_carry_offset(int ctas);
 
 // Record the message that mamba_last_error() returns on this thread.
 void record_error(const char *fmt, ...);

@@ -79,7 +79,8 @@ constexpr uint32_t kOffBar = kOffAbort + 16;
 enum Bar { kFull0, kFull1, kEmpty0, kEmpty1, kGFull0, kGFull1, kPReady, kSFull, kYFull, kHReady, kYFree, kDrain,
            kStep0, kStep1, kNumBars };
 constexpr uint32_t kOffTmemSlot = kOffBar + kNumBars * 8;
-constexpr uint32_t kSmemBytes = kOffTmemSlot + 8;
+constexpr uint32_t kOffSched = kOffTmemSlot + 8;          // the CTA's SsdSched (seven ints)
+constexpr uint32_t kSmemBytes = kOffSched + 32;
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 static_assert(kOffM % 1024 == 0 && kOffXt % 1024 == 0 && kOffH % 1024 == 0 && kStageBytes % 1024 == 0,
               "swizzle atoms need 1024-byte alignment");
@@ -405,17 +406,88 @@ __device__ __forceinline__ void build_mask_rows(uint32_t tg, uint32_t m_tile, in
     }
 }
 
+// ---- schedule ----------------------------------------------------------------
+// One CTA per (batch, head) walks that sequence's chunks; or, persistent, CTA g
+// of G takes chunks [g T / G, (g + 1) T / G) of the list of all T chunks
+// (sequence u = b * nheads + h, chunk c at u * nc + c). Such a range is the
+// tail of sequence us from chunk cs, whole sequences, and the head of sequence
+// ue up to chunk ce. The CTA runs the head first (its end state goes to the
+// next CTA), then the whole sequences, then the tail (which starts from the
+// state the previous CTA handed over): by then that state is ready whenever the
+// range holds at least one sequence's worth of chunks.
+struct SsdSched {
+    int us, cs, ue, ce, nc, np;   // np pieces
+    int K;                        // chunks of this CTA
+};
+struct SsdPiece {
+    int u, c0, c1;   // chunks [c0, c1) of sequence u
+};
+
+__device__ __forceinline__ SsdSched ssd_sched(const ms::SsdParams &p, int nc)
+{
+    SsdSched s;
+    s.nc = nc;
+    if (p.sk_ctas == 0) {
+        s.us = s.ue = (int)blockIdx.x;
+        s.cs = 0;
+        s.ce = nc;
+        s.K = nc;
+        s.np = nc > 0 ? 1 : 0;
+        return s;
+    }
+    const int64_t T = p.batch * p.nheads * (int64_t)nc, G = p.sk_ctas, g = blockIdx.x;
+    const int64_t q = T / G, rm = T % G;
+    const int64_t a = g * q + (g * rm) / G, e = (g + 1) * q + ((g + 1) * rm) / G;
+    s.K = (int)(e - a);
+    if (s.K <= 0) {
+        s.us = s.ue = s.cs = s.ce = 0;
+        s.np = 0;
+        s.K = 0;
+        return s;
+    }
+    s.us = (int)(a / nc);
+    s.cs = (int)(a % nc);
+    s.ue = (int)((e - 1) / nc);
+    s.ce = (int)((e - 1) % nc) + 1;
+    s.np = s.ue - s.us + 1;
+    return s;
+}
+
+__device__ __forceinline__ SsdPiece ssd_piece(const SsdSched &s, int i)
+{
+    if (s.us == s.ue)
+        return {s.us, s.cs, s.ce};
+    if (i == 0)
+        return {s.ue, 0, s.ce};
+    if (i < s.np - 1)
+        return {s.us + i, 0, s.nc};
+    return {s.us, s.cs, s.nc};
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int *f)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(int *f, int v)
+{
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(f), "r"(v) : "memory");
+}
+
+// Barrier of the 512 epilogue threads (named barrier 1).
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory"); }
+
 __global__ void __launch_bounds__(kThreads, 1)
 ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap b_map,
            const __grid_constant__ CUtensorMap c_map, const ms::SsdParams p)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t bh = blockIdx.x;
-    const int64_t b = bh / p.nheads, h = bh % p.nheads;
-    const int64_t g = h / (p.nheads / p.ngroups);
     const int L = (int)p.seqlen;
-    const int nchunks = (L + kQ - 1) / kQ;
+    const int hpg = (int)(p.nheads / p.ngroups);
+    SsdSched *sched = reinterpret_cast<SsdSched *>(smem + kOffSched);
     const uint32_t base = smem_addr(smem);
     if (base & 1023u) {   // the swizzled tiles need a 1024-byte aligned window
         if (threadIdx.x == 0)
@@ -442,6 +514,7 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
         mbar_init(bar(kStep0), 32);
         mbar_init(bar(kStep1), 32);
         *abort_flag = 0;
+        *sched = ssd_sched(p, (L + kQ - 1) / kQ);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == kMmaWarp)
@@ -450,90 +523,103 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
     __syncthreads();
     tc_after_sync();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + kOffTmemSlot);
+    const int K = sched->K;
 
     if (warp == kTmaWarp) {
-        // ---- producer: X, B and C of chunk c into stage c % 2 (lane 0), and the chunk's step
-        // data (all lanes, four tokens each) into step buffer c % 2 ----
+        // ---- producer: X, B and C of chunk i into stage i % 2 (lane 0), and the chunk's step
+        // data (all lanes, four tokens each) into step buffer i % 2 ----
         float *dl_all = reinterpret_cast<float *>(smem + kOffStep);
         float *s2_all = dl_all + 2 * kQ;
         uint16_t *cf_all = reinterpret_cast<uint16_t *>(s2_all + 2 * kQ);
-        const float Ah2 = p.A[h] * kLog2e;
-        const float bias = p.dt_bias ? p.dt_bias[h] : 0.f;
-        const uint16_t *dtp = reinterpret_cast<const uint16_t *>(p.dt) + b * p.dt_sb + h;
-        auto load_dt = [&](int c, float (&v)[4]) {
+        int issued = 0;            // chunks whose loads went out (or were withheld)
+        unsigned withheld = 0u;    // bit i % 2: chunk i's loads withheld
+        bool stop = false;
+        int i = 0;
+        const int np = sched->np;
+        for (int pi = 0; pi < np && !stop; ++pi) {
+            const SsdPiece pc = ssd_piece(*sched, pi);
+            const int b = pc.u / (int)p.nheads, h = pc.u - b * (int)p.nheads, g = h / hpg;
+            const float Ah2 = p.A[h] * kLog2e;
+            const float bias = p.dt_bias ? p.dt_bias[h] : 0.f;
+            const uint16_t *dtp = reinterpret_cast<const uint16_t *>(p.dt) + b * p.dt_sb + h;
+            auto load_dt = [&](int c, float (&v)[4]) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int t = c * kQ + 4 * lane + k;
-                v[k] = t < L ? load_bf16(dtp, (int64_t)t * p.dt_st) : 0.f;
-            }
-        };
-        float dtv[4];
-        load_dt(0, dtv);
-        int issued = 0;
-        for (int c = 0; c < nchunks; ++c) {
-            const int st = c & 1;
-            if (c >= 2 && !__all_sync(0xffffffffu, role_wait(bar(kEmpty0 + st), ((c >> 1) + 1) & 1, abort_flag, wlim))) {
-                if (lane == 0)
-                    give_up(p.status, abort_flag);
-                break;
-            }
-            // (a test can withhold one block's loads: its full barrier then never completes)
-            if (lane == 0 && c + 1 != p.withhold_block) {
-                const uint32_t sx = base + (uint32_t)st * kStageBytes, sb = sx + kXTile, sc = sb + kBCTile;
-                const uint32_t full = bar(kFull0 + st);
-                mbar_arrive_tx(full, kStageTx);
-                tma_load_3d(sx, &x_map, full, (int)(h * kP), c * kQ, (int)b);
-                tma_load_3d(sb, &b_map, full, (int)(g * kN), c * kQ, (int)b);
-                tma_load_3d(sb + kQ * 128, &b_map, full, (int)(g * kN + 64), c * kQ, (int)b);
-                tma_load_3d(sc, &c_map, full, (int)(g * kN), c * kQ, (int)b);
-                tma_load_3d(sc + kQ * 128, &c_map, full, (int)(g * kN + 64), c * kQ, (int)b);
-            }
-            issued = c + 1;
-            // step sizes of tokens 4 lane .. 4 lane + 3 and the running sum of delta A (log2 units)
-            float d[4], v[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int t = c * kQ + 4 * lane + k;
-                d[k] = 0.f;
-                if (t < L) {
-                    d[k] = dtv[k] + bias;
-                    if (p.softplus)
-                        d[k] = ms::softplus(d[k]);
+                for (int k = 0; k < 4; ++k) {
+                    const int t = c * kQ + 4 * lane + k;
+                    v[k] = t < L ? load_bf16(dtp, (int64_t)t * p.dt_st) : 0.f;
                 }
+            };
+            float dtv[4];
+            load_dt(pc.c0, dtv);
+            for (int c = pc.c0; c < pc.c1; ++c, ++i) {
+                const int st = i & 1;
+                if (i >= 2 &&
+                    !__all_sync(0xffffffffu, role_wait(bar(kEmpty0 + st), ((i >> 1) + 1) & 1, abort_flag, wlim))) {
+                    if (lane == 0)
+                        give_up(p.status, abort_flag);
+                    stop = true;
+                    break;
+                }
+                // (a test can withhold one block's loads: its full barrier then never completes)
+                const bool hold = c + 1 == p.withhold_block;
+                withheld = hold ? (withheld | (1u << st)) : (withheld & ~(1u << st));
+                if (lane == 0 && !hold) {
+                    const uint32_t sx = base + (uint32_t)st * kStageBytes, sb = sx + kXTile, sc2 = sb + kBCTile;
+                    const uint32_t full = bar(kFull0 + st);
+                    mbar_arrive_tx(full, kStageTx);
+                    tma_load_3d(sx, &x_map, full, (int)(h * kP), c * kQ, (int)b);
+                    tma_load_3d(sb, &b_map, full, (int)(g * kN), c * kQ, (int)b);
+                    tma_load_3d(sb + kQ * 128, &b_map, full, (int)(g * kN + 64), c * kQ, (int)b);
+                    tma_load_3d(sc2, &c_map, full, (int)(g * kN), c * kQ, (int)b);
+                    tma_load_3d(sc2 + kQ * 128, &c_map, full, (int)(g * kN + 64), c * kQ, (int)b);
+                }
+                issued = i + 1;
+                // step sizes of tokens 4 lane .. 4 lane + 3 and the running sum of delta A (log2 units)
+                float d[4], v[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int t = c * kQ + 4 * lane + k;
+                    d[k] = 0.f;
+                    if (t < L) {
+                        d[k] = dtv[k] + bias;
+                        if (p.softplus)
+                            d[k] = ms::softplus(d[k]);
+                    }
+                }
+                if (c + 1 < pc.c1)
+                    load_dt(c + 1, dtv);
+                v[0] = d[0] * Ah2;
+#pragma unroll
+                for (int k = 1; k < 4; ++k)
+                    v[k] = fmaf(d[k], Ah2, v[k - 1]);
+                float incl = v[3];
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float u = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o)
+                        incl += u;
+                }
+                const float excl = incl - v[3];
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    v[k] += excl;
+                // s at the last token of this 32-token block (lanes 8 j .. 8 j + 7 hold block j)
+                const float vend = __shfl_sync(0xffffffffu, v[3], (lane & ~7) | 7);
+                float cfv[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    cfv[k] = ex2(vend - v[k]) * d[k];
+                *reinterpret_cast<float4 *>(dl_all + st * kQ + 4 * lane) = make_float4(d[0], d[1], d[2], d[3]);
+                *reinterpret_cast<float4 *>(s2_all + st * kQ + 4 * lane) = make_float4(v[0], v[1], v[2], v[3]);
+                *reinterpret_cast<uint2 *>(cf_all + st * kQ + 4 * lane) =
+                    make_uint2(pack_bf16(cfv[0], cfv[1]), pack_bf16(cfv[2], cfv[3]));
+                mbar_arrive(bar(kStep0 + st));
             }
-            if (c + 1 < nchunks)
-                load_dt(c + 1, dtv);
-            v[0] = d[0] * Ah2;
-#pragma unroll
-            for (int k = 1; k < 4; ++k)
-                v[k] = fmaf(d[k], Ah2, v[k - 1]);
-            float incl = v[3];
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float u = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o)
-                    incl += u;
-            }
-            const float excl = incl - v[3];
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                v[k] += excl;
-            // s at the last token of this 32-token block (lanes 8 j .. 8 j + 7 hold block j)
-            const float vend = __shfl_sync(0xffffffffu, v[3], (lane & ~7) | 7);
-            float cfv[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                cfv[k] = ex2(vend - v[k]) * d[k];
-            *reinterpret_cast<float4 *>(dl_all + st * kQ + 4 * lane) = make_float4(d[0], d[1], d[2], d[3]);
-            *reinterpret_cast<float4 *>(s2_all + st * kQ + 4 * lane) = make_float4(v[0], v[1], v[2], v[3]);
-            *reinterpret_cast<uint2 *>(cf_all + st * kQ + 4 * lane) =
-                make_uint2(pack_bf16(cfv[0], cfv[1]), pack_bf16(cfv[2], cfv[3]));
-            mbar_arrive(bar(kStep0 + st));
         }
         // the loads in flight must land before the CTA leaves
         if (lane == 0)
             for (int c = issued > 2 ? issued - 2 : 0; c < issued; ++c)
-                if (c + 1 != p.withhold_block)
+                if (!(withheld & (1u << (c & 1))))
                     mbar_wait(bar(kFull0 + (c & 1)), (c >> 1) & 1);
         __syncwarp();
     } else if (warp == kMmaWarp) {
@@ -543,7 +629,7 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
             constexpr uint32_t id_yo = bf16_idesc(128, 64, false, true);    // Yo = C H^T
             constexpr uint32_t id_s = bf16_idesc(128, 64, true, true);      // S = B^T Xt
             constexpr uint32_t id_yd = bf16_idesc(128, 64, false, true);    // Yd = M' X
-            for (int c = 0; c < nchunks; ++c) {
+            for (int c = 0; c < K; ++c) {   // c: position in the CTA's list of chunks
                 const int st = c & 1;
                 const uint32_t sx = base + (uint32_t)st * kStageBytes, sb = sx + kXTile, sc = sb + kBCTile;
                 if (!role_wait(bar(kFull0 + st), (c >> 1) & 1, abort_flag, wlim)) {
@@ -605,13 +691,85 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
         const float *dl_all = reinterpret_cast<const float *>(smem + kOffStep);
         const float *s2_all = dl_all + 2 * kQ;
         const uint16_t *cf_all = reinterpret_cast<const uint16_t *>(s2_all + 2 * kQ);
-        const float Dh = p.D ? p.D[h] : 0.f;
+        bool ok = true;
+        auto epi_wait = [&](uint32_t barrier, uint32_t parity) {
+            if (ok)
+                ok = __all_sync(0xffffffffu, role_wait(barrier, parity, abort_flag, wlim));
+            if (!ok && lane == 0)
+                give_up(p.status, abort_flag);
+            return ok;
+        };
+
         // this thread keeps H[p][n] for n = r and p = 16 hq + j
-        const int64_t hoff = (bh * kP + 16 * hq) * kN + r;
         float H[16];
+        // The state a piece starts from: the initial state (or zero) at the start of a
+        // sequence, else the one the previous CTA handed over (bounded wait for its flag).
+        auto load_state = [&](const SsdPiece &pc) {
+            if (pc.c0 > 0) {
+                const int src = (int)blockIdx.x - 1;
+                bool got = true;
+                if (lane == 0 && ok) {
+                    got = ld_acquire_gpu(p.sk_flag + src) != 0;
+                    if (!got) {
+                        const uint64_t t0 = global_ns();
+                        while (!(got = ld_acquire_gpu(p.sk_flag + src) != 0)) {
+                            if (*abort_flag || global_ns() - t0 > wlim)
+                                break;
+                            __nanosleep(256);
+                        }
+                    }
+                }
+                if (!__all_sync(0xffffffffu, got) && ok) {
+                    ok = false;
+                    if (lane == 0)
+                        give_up(p.status, abort_flag);
+                }
+                const float *src_h = p.sk_carry + ((int64_t)src * kP + 16 * hq) * kN + r;
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-            H[j] = p.h0 ? p.h0[hoff + (int64_t)j * kN] : 0.f;
+                for (int j = 0; j < 16; ++j)
+                    H[j] = ok ? __ldcg(src_h + (int64_t)j * kN) : 0.f;
+            } else {
+                const int64_t hoff = ((int64_t)pc.u * kP + 16 * hq) * kN + r;
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    H[j] = p.h0 ? p.h0[hoff + (int64_t)j * kN] : 0.f;
+            }
+        };
+        // The state a piece ends with: the final state at the end of a sequence, else
+        // the hand-over to the next CTA (stored, fenced, then the flag raised once all
+        // 512 threads have stored; raised even after a timeout so no CTA waits on it).
+        auto save_state = [&](const SsdPiece &pc, int nc) {
+            if (pc.c1 == nc) {
+                if (ok && p.hT) {
+                    const int64_t hoff = ((int64_t)pc.u * kP + 16 * hq) * kN + r;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        p.hT[hoff + (int64_t)j * kN] = H[j];
+                }
+            } else {
+                float *dst = p.sk_carry + ((int64_t)blockIdx.x * kP + 16 * hq) * kN + r;
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    __stcg(dst + (int64_t)j * kN, H[j]);
+                __threadfence();
+                epi_bar();
+                if (threadIdx.x == 0)
+                    st_release_gpu(p.sk_flag + blockIdx.x, 1);
+            }
+        };
+
+        // position: piece pi, chunk c of its sequence, `left` chunks to the piece's end
+        int pi = 0, c = 0, left = 0;
+        if (sched->np > 0) {
+            const SsdPiece f = ssd_piece(*sched, 0);
+            c = f.c0;
+            left = f.c1 - f.c0;
+            load_state(f);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                H[j] = 0.f;
+        }
         // rows of block sub: M' columns in blocks above the diagonal are zero (causal mask)
         // and are written once, this warp taking the groups 32 j + 8 hq
         for (int j = sub + 1; j < 4; ++j) {
@@ -625,15 +783,6 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
         __syncwarp();
         if (lane == 0)
             mbar_arrive(bar(kHReady));
-
-        bool ok = true;
-        auto epi_wait = [&](uint32_t barrier, uint32_t parity) {
-            if (ok)
-                ok = __all_sync(0xffffffffu, role_wait(barrier, parity, abort_flag, wlim));
-            if (!ok && lane == 0)
-                give_up(p.status, abort_flag);
-            return ok;
-        };
 
         // Build the operands M' and Xt of chunk k from its step data; returns s_r and s_end.
         auto prepare = [&](int k, float &sr, float &se) {
@@ -683,24 +832,39 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
                 mbar_arrive(bar(kPReady));
         };
 
+        // per piece: this thread's columns of y and z at token 0 of the sequence, and D
+        const uint16_t *zcol = nullptr;
+        uint16_t *ycol = nullptr;
+        float Dh = 0.f;
+        auto enter = [&](int u) {
+            const int b = u / (int)p.nheads, h = u - b * (int)p.nheads;
+            Dh = p.D ? p.D[h] : 0.f;
+            ycol = reinterpret_cast<uint16_t *>(p.y) + (int64_t)b * p.y_sb + (int64_t)h * kP + 16 * hq;
+            if (p.z)
+                zcol = reinterpret_cast<const uint16_t *>(p.z) + (int64_t)b * p.z_sb + (int64_t)h * kP + 16 * hq;
+        };
         float sr_c = 0.f, se_c = 0.f;   // s_r and s_end of the chunk being finished
-        if (nchunks > 0)
+        if (K > 0) {
+            enter(ssd_piece(*sched, 0).u);
             prepare(0, sr_c, se_c);
-        for (int c = 0; c < nchunks; ++c) {
-            const int st = c & 1, t0 = c * kQ;
+        }
+        for (int i = 0; i < K; ++i) {
+            const int st = i & 1, t0 = c * kQ;
             const bool live = t0 + r < L;
             const uint32_t sx = base + (uint32_t)st * kStageBytes;
             // the gate of this thread's 16 outputs
             uint4 zq[2] = {};
             if (p.z && live) {
-                const uint4 *zp = reinterpret_cast<const uint4 *>(reinterpret_cast<const uint16_t *>(p.z) + b * p.z_sb +
-                                                                  (int64_t)(t0 + r) * p.z_st + h * kP + 16 * hq);
+                const uint4 *zp = reinterpret_cast<const uint4 *>(zcol + (int64_t)(t0 + r) * p.z_st);
                 zq[0] = __ldg(zp);
                 zq[1] = __ldg(zp + 1);
             }
+            const float Dc = Dh;
+            const uint16_t *ycol_c = ycol;   // the piece's, before a change of piece below
 
-            // (2) state passing: H = exp(s_end) H + S^T
-            epi_wait(bar(kSFull), c & 1);
+            // (2) state passing: H = exp(s_end) H + S^T; at the end of a piece the state
+            // leaves (final state or hand-over) and the next piece's initial state enters
+            epi_wait(bar(kSFull), i & 1);
             if (ok) {
                 tc_after_sync();
                 float sv[16];
@@ -709,7 +873,23 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
 #pragma unroll
                 for (int j = 0; j < 16; ++j)
                     H[j] = fmaf(ac, H[j], sv[j]);
-                store_state_tile(base + kOffH, r, hq, H);
+                // (stored at once inside a piece: the Yo product of the next chunk waits for it)
+                if (left > 1)
+                    store_state_tile(base + kOffH, r, hq, H);
+            }
+            ++c;
+            if (--left == 0) {
+                const SsdSched s2 = *sched;
+                save_state(ssd_piece(s2, pi), s2.nc);
+                if (pi + 1 < s2.np) {
+                    const SsdPiece nx = ssd_piece(s2, ++pi);
+                    load_state(nx);
+                    enter(nx.u);
+                    c = nx.c0;
+                    left = nx.c1 - nx.c0;
+                }
+                if (ok)
+                    store_state_tile(base + kOffH, r, hq, H);
             }
             async_proxy_fence();
             tc_before_sync();
@@ -719,7 +899,7 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
 
             // (3a) y = Yd + exp(s_r) Yo + D x into registers; the Y columns and the stage are then free
             float yv[16];
-            epi_wait(bar(kYFull), c & 1);
+            epi_wait(bar(kYFull), i & 1);
             if (ok) {
                 tc_after_sync();
                 float yd[16];
@@ -737,8 +917,8 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int j = 8 * q + 2 * e;
-                        yv[j] = fmaf(er, yv[j], fmaf(Dh, bf16_lo(xw[e]), yd[j]));
-                        yv[j + 1] = fmaf(er, yv[j + 1], fmaf(Dh, bf16_hi(xw[e]), yd[j + 1]));
+                        yv[j] = fmaf(er, yv[j], fmaf(Dc, bf16_lo(xw[e]), yd[j]));
+                        yv[j + 1] = fmaf(er, yv[j + 1], fmaf(Dc, bf16_hi(xw[e]), yd[j + 1]));
                     }
                 }
             }
@@ -748,10 +928,10 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
 
             // (1) operands of the next chunk, so that its products overlap the rest of this one
             float sr_n = 0.f, se_n = 0.f;
-            if (c + 1 < nchunks)
-                prepare(c + 1, sr_n, se_n);
+            if (i + 1 < K)
+                prepare(i + 1, sr_n, se_n);
 
-            // (3b) gate and store y of chunk c
+            // (3b) gate and store y of this chunk
             if (ok && live) {
                 uint4 out[2];
 #pragma unroll
@@ -770,18 +950,12 @@ ssd_kernel(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CU
                     }
                     out[q] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
                 }
-                uint4 *yp = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.y) + b * p.y_sb +
-                                                      (int64_t)(t0 + r) * p.y_st + h * kP + 16 * hq);
+                uint4 *yp = reinterpret_cast<uint4 *>(const_cast<uint16_t *>(ycol_c) + (int64_t)(t0 + r) * p.y_st);
                 yp[0] = out[0];
                 yp[1] = out[1];
             }
             sr_c = sr_n;
             se_c = se_n;
-        }
-        if (ok && p.hT) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-                p.hT[hoff + (int64_t)j * kN] = H[j];
         }
     }
     tc_before_sync();
@@ -837,6 +1011,26 @@ bool encode_map(CUtensorMap *m, const void *ptr, int64_t inner, int64_t tokens, 
 
 }  // namespace
 
+// The persistent schedule pays when the (batch, head) pairs leave the last wave
+// of one-CTA-per-pair partly empty: it then takes ceil(T / SMs) chunk times plus
+// about one for the hand-over, against waves x chunks. Each CTA must hold at
+// least one sequence's worth of chunks so that no hand-over waits.
+int ssd_persistent_ctas(int64_t batch, int64_t nheads, int64_t seqlen, int num_sms)
+{
+    const int64_t units = batch * nheads, nc = (seqlen + kQ - 1) / kQ;
+    if (num_sms <= 0 || nc < 2 || units <= num_sms || units % num_sms == 0)
+        return 0;
+    const int64_t waves = (units + num_sms - 1) / num_sms;
+    const int64_t per_cta = (units * nc + num_sms - 1) / num_sms;
+    return per_cta + 2 < waves * nc ? num_sms : 0;
+}
+
+size_t ssd_flag_offset() { return 256; }
+
+size_t ssd_carry_offset(int ctas) { return 256 + (((size_t)ctas * sizeof(int) + 255) / 256) * 256; }
+
+size_t ssd_persistent_ws_bytes(int ctas) { return ssd_carry_offset(ctas) + (size_t)ctas * kP * kN * sizeof(float); }
+
 cudaError_t launch_ssd(const SsdParams &p, cudaStream_t stream)
 {
     CUtensorMap xm, bm, cm;
@@ -847,7 +1041,34 @@ cudaError_t launch_ssd(const SsdParams &p, cudaStream_t stream)
     cudaError_t e = cudaFuncSetAttribute(ssd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess)
         return e;
-    ssd_kernel<<<(unsigned)(p.batch * p.nheads), kThreads, kSmemBytes, stream>>>(xm, bm, cm, p);
+    if (p.sk_ctas == 0) {
+        e = cudaMemsetAsync(p.status, 0, sizeof(int), stream);
+        if (e != cudaSuccess)
+            return e;
+        ssd_kernel<<<(unsigned)(p.batch * p.nheads), kThreads, kSmemBytes, stream>>>(xm, bm, cm, p);
+        return cudaGetLastError();
+    }
+    // status word and flags, then a cooperative launch: every CTA is resident, so a
+    // CTA waiting for its predecessor's hand-over never waits for one that has not started
+    if (!p.sk_flag || !p.sk_carry)
+        return cudaErrorInvalidValue;
+    e = cudaMemsetAsync(p.status, 0, ssd_carry_offset(p.sk_ctas), stream);
+    if (e != cudaSuccess)
+        return e;
+    void *args[] = {&xm, &bm, &cm, const_cast<SsdParams *>(&p)};
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)p.sk_ctas);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr{};
+    attr.id = cudaLaunchAttributeCooperative;
+    attr.val.cooperative = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelExC(&cfg, reinterpret_cast<const void *>(ssd_kernel), args);
+    if (e != cudaSuccess)
+        return e;
     return cudaGetLastError();
 }
 

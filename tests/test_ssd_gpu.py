@@ -236,6 +236,68 @@ def test_ssd_timeout_path(block):
     assert rel_err(to_host64(hT), hr) <= TOL["bf16"]
 
 
+def _ssd_ws_bytes(dev):
+    import ctypes
+    ms = _ms()
+    args = ms.build_ssd_args(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["x"])
+    n = ctypes.c_size_t(0)
+    assert ms.load_library().mamba_ssd_workspace_size(ctypes.byref(args), ctypes.byref(n)) == 0
+    return n.value
+
+
+@pytest.mark.parametrize("batch,L,nheads,ngroups", [(2, 1000, 80, 2), (1, 1300, 150, 1)])
+def test_ssd_persistent_schedule(batch, L, nheads, ngroups):
+    """More (batch, head) pairs than SMs, leaving the last wave partly empty:
+    the call takes the persistent schedule (a larger workspace), which cuts
+    the chunks of all pairs evenly over the SMs and hands a pair's state from
+    one CTA to the next. Every pair against the oracle, from an initial state."""
+    import torch
+    inp = make_ssd_inputs(SMALL, batch=batch, seqlen=L, nheads=nheads, ngroups=ngroups, seed=3800 + nheads)
+    dev = _dev(inp)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    if batch * nheads <= sms or (batch * nheads) % sms == 0:
+        pytest.skip("the shape fills whole waves of this device")
+    assert _ssd_ws_bytes(dev) > _ms().SSD_WORKSPACE_BYTES
+    h0 = make_ssd_state(batch, nheads, seed=3801)
+    y, hT = _run(dev, h0=torch.from_numpy(h0).cuda())
+    yr, hr = _oracle(inp, h0=h0.reshape(-1, 64, 128))
+    assert rel_err(y, yr) <= TOL["bf16"]
+    assert rel_err(hT, hr.reshape(hT.shape)) <= TOL["bf16"]
+    # the same call with the smallest workspace runs one CTA per pair: same result
+    ws = torch.zeros(_ms().SSD_WORKSPACE_BYTES, dtype=torch.uint8, device="cuda")
+    y2, hT2 = _ms().ssd_fwd(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], D=dev["D"], z=dev["z"],
+                            dt_bias=dev["dt_bias"], initial_state=torch.from_numpy(h0).cuda(), workspace=ws)
+    assert rel_err(to_host64(y2), yr) <= TOL["bf16"]
+    assert rel_err(to_host64(hT2), hr.reshape(hT.shape)) <= TOL["bf16"]
+
+
+def test_ssd_persistent_timeout_path():
+    """The persistent schedule's bounded waits: with block 2's loads withheld
+    and a 2 ms limit, every CTA gives up, still raises its hand-over flag (so
+    no CTA waits on it for longer than the limit), drains and exits; the status
+    word reads MS_ERR_TIMEOUT and a normal call straight after matches the
+    oracle."""
+    import torch
+    ms = _ms()
+    inp = make_ssd_inputs(SMALL, batch=2, seqlen=600, nheads=80, seed=3900)
+    dev = _dev(inp)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    if 160 <= sms or 160 % sms == 0:
+        pytest.skip("the shape fills whole waves of this device")
+    nbytes = _ssd_ws_bytes(dev)
+    assert nbytes > ms.SSD_WORKSPACE_BYTES
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    ms.ssd_fwd(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], D=dev["D"], z=dev["z"], dt_bias=dev["dt_bias"],
+               workspace=ws, check=False, wait_limit_us=2000, withhold_block=3)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32)[0].item()) == 5   # MS_ERR_TIMEOUT
+    y, hT = ms.ssd_fwd(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], D=dev["D"], z=dev["z"],
+                       dt_bias=dev["dt_bias"], workspace=ws)
+    yr, hr = _oracle(inp)
+    assert rel_err(to_host64(y), yr) <= TOL["bf16"]
+    assert rel_err(to_host64(hT), hr) <= TOL["bf16"]
+
+
 def test_ssd_withheld_block_past_the_end_is_harmless():
     """A withheld block index beyond the sequence changes nothing."""
     inp = make_ssd_inputs(SMALL, batch=1, seqlen=200, nheads=2, seed=3400)
