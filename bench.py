@@ -56,6 +56,7 @@ MUFU_PER_CLK = 16
 NCU_TRAFFIC = {("long_context_131k", 10, 148): (505176320 + 150065408) * 8,
                ("mamba130m_layer", 10, 296): 152307456 + 32844800,
                ("mamba1p4b_layer", 10, 444): 813864448 + 252678912,
+               ("mamba2_layer_d2048", "ssd_kernel"): 565090000 + 247200000,
                ("decode_b256_d5120", "state_update_vec_kernel"): 92157440 + 29935104}
 FP32_PER_CLK = 128
 # FP32 operations of one exponential on the FMA pipe (the combined MUFU + FMA bound)

@@ -992,8 +992,12 @@ EncodeTiled encoder()
 
 // A bf16 map over (inner, tokens, batch) delivering 64 x 128 x 1 boxes into
 // 128-byte-swizzled shared memory; rows past the last token read as zero.
+// L2 fills: 256 bytes for B and C (a chunk reads both 128-byte halves of each
+// row), 128 bytes for x (one head's 128 bytes of a token; the other half of a
+// 256-byte fill is another head's, which the persistent schedule reaches at
+// another time).
 bool encode_map(CUtensorMap *m, const void *ptr, int64_t inner, int64_t tokens, int64_t batch, int64_t token_stride,
-                int64_t batch_stride)
+                int64_t batch_stride, CUtensorMapL2promotion promo)
 {
     const EncodeTiled fn = encoder();
     if (!fn)
@@ -1005,7 +1009,7 @@ bool encode_map(CUtensorMap *m, const void *ptr, int64_t inner, int64_t tokens, 
     const cuuint32_t box[3] = {64u, (cuuint32_t)kQ, 1u};
     const cuuint32_t elem[3] = {1u, 1u, 1u};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, elem,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, promo,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -1034,9 +1038,9 @@ size_t ssd_persistent_ws_bytes(int ctas) { return ssd_carry_offset(ctas) + (size
 cudaError_t launch_ssd(const SsdParams &p, cudaStream_t stream)
 {
     CUtensorMap xm, bm, cm;
-    if (!encode_map(&xm, p.x, p.nheads * kP, p.seqlen, p.batch, p.x_st, p.x_sb) ||
-        !encode_map(&bm, p.B, p.ngroups * kN, p.seqlen, p.batch, p.B_st, p.B_sb) ||
-        !encode_map(&cm, p.C, p.ngroups * kN, p.seqlen, p.batch, p.C_st, p.C_sb))
+    if (!encode_map(&xm, p.x, p.nheads * kP, p.seqlen, p.batch, p.x_st, p.x_sb, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) ||
+        !encode_map(&bm, p.B, p.ngroups * kN, p.seqlen, p.batch, p.B_st, p.B_sb, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
+        !encode_map(&cm, p.C, p.ngroups * kN, p.seqlen, p.batch, p.C_st, p.C_sb, CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
         return cudaErrorNotSupported;
     cudaError_t e = cudaFuncSetAttribute(ssd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess)
