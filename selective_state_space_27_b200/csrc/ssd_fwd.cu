@@ -19,8 +19,11 @@
 //   H     = exp(s_end) H_prev + S^T                 (state passing)
 // The four products are tcgen05 MMAs (bf16 operands from shared memory,
 // fp32 accumulators in tensor memory); the decay, the state passing, the
-// skip and the gate run in the epilogue warps. One CTA owns one (b, h) and
-// walks its chunks in order, so the state never leaves the SM.
+// skip and the gate run in the epilogue warps. A CTA walks the chunks of a
+// (b, h) in order, so the state stays on the SM: one CTA per (b, h), or, when
+// the pairs would leave the last wave partly empty, one resident CTA per SM
+// taking an even share of all pairs' chunks, where a pair cut between two CTAs
+// hands its state over through global memory (see the schedule below).
 //
 // Roles (576 threads): warps 0-15 epilogue (warp w reads TMEM lanes
 // 32 (w % 4) .. +31, i.e. rows of the chunk, and handles column quarter
