@@ -217,7 +217,8 @@ int mamba_scan_num_configs(void);
  *    segments).
  *  - Sequential kernels (kind 1): lanes per row, states per lane (16 / lanes)
  *    and the fixed CTA size in warps (4); plans take exactly that many warps
- *    and one segment, and need no workspace.
+ *    and one segment, and need no workspace unless they ask for the
+ *    persistent schedule (ctas > 0).
  * Returns MS_ERR_INVALID_ARG for an unknown index.
  */
 ms_status mamba_scan_config_info(int config, int *lanes, int *states_per_pass, int *max_warps);
@@ -288,8 +289,9 @@ typedef struct ms_conv1d_args {
  * convolution input ((batch, dim, seqlen), the layout and dtype of u); every
  * other argument means what it means for mamba_scan_fwd. u itself is never
  * written to memory. Runs on the sequential kernels with 2 or 4 lanes per row,
- * in one segment, with no workspace. `plan` is NULL (automatic) or one of those
- * configurations (warps_per_cta = max_warps, segments = 1). The caller owns
+ * in one segment, with no workspace (mamba_conv_scan_fwd_ws below takes one,
+ * for the persistent schedule). `plan` is NULL (automatic) or one of those
+ * configurations (warps_per_cta = max_warps, segments = 1, ctas 0). The caller owns
  * every buffer; the call enqueues one kernel on `stream`.
  * Errors: as mamba_scan_fwd; MS_ERR_INVALID_ARG for a NULL conv or weight or a
  * silu flag other than 0/1, or width < 1; MS_ERR_UNSUPPORTED for width >
