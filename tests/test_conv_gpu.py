@@ -11,7 +11,7 @@ import pytest
 import oracle
 from selective_state_space_27_b200.inputs import (SCAN_WORKLOADS, f32_from_bf16_bits, make_conv_params,
                                                   make_conv_state, make_scan_inputs)
-from tests.gpu_util import TOL, device_inputs, rel_err, sample_rows, to_device, to_host64
+from tests.gpu_util import TOL, device_inputs, rel_err, to_device, to_host64
 
 pytestmark = pytest.mark.gpu
 
