@@ -130,10 +130,11 @@ template <typename T, int LPR, int VAR = 0, int IOW = 2> struct Raw {
     static constexpr int LAM = HALO + 1;                             // first slot of lambda_raw (variant 2)
     static constexpr int SLOTS = 3 * PS + BC_PER + (VAR ? 1 : 0) + (TRAP ? PS : 0);
     static constexpr int STAGE = SLOTS * IOT * 16;
-    // ring depth: shorter for the variants, whose larger slots, skip tiles
-    // (prologue) or wider step tiles (trapezoidal) must still leave room for
-    // 3 (LPR 4) CTAs per SM
-    static constexpr int RS = TRAP ? kRawStages - 2 : CONV ? kRawStages - 1 : kRawStages;
+    // ring depth: one stage shorter for the convolution prologue, whose larger
+    // slots and skip tiles must still leave room for 3 (LPR 4) CTAs per SM. The
+    // trapezoidal rule keeps the full ring: its plans run 2 CTAs per SM, and
+    // prefetching three chunks ahead beat a third CTA.
+    static constexpr int RS = CONV ? kRawStages - 1 : kRawStages;
     static constexpr int RA = RS - kTileStages + 1;                   // chunks staged ahead
     static constexpr int OFF = SH::BYTES;
     static constexpr int SKR = kSteps + 4;                            // floats per row of the skip tile
