@@ -1027,6 +1027,8 @@ int ssd_persistent_ctas(int64_t batch, int64_t nheads, int64_t seqlen, int num_s
     const int64_t units = batch * nheads, nc = (seqlen + kQ - 1) / kQ;
     if (num_sms <= 0 || nc < 2 || units <= num_sms || units % num_sms == 0)
         return 0;
+    if (units * nc / num_sms >= (int64_t(1) << 30))   // a CTA's count of chunks is kept in an int
+        return 0;
     const int64_t waves = (units + num_sms - 1) / num_sms;
     const int64_t per_cta = (units * nc + num_sms - 1) / num_sms;
     return per_cta + 2 < waves * nc ? num_sms : 0;
