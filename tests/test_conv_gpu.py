@@ -105,6 +105,34 @@ def test_conv_scan_persistent_schedule(dtype):
             assert rel_err(hT, hr) <= TOL[dtype], tag
 
 
+def test_conv_scan_persistent_on_side_stream():
+    """The persistent schedule on a stream other than the current one, with
+    the hand-over workspace allocated by the binding: work queued meanwhile on
+    the current stream must not receive the workspace's memory while the scan
+    still uses it."""
+    import torch
+    ms = _ms()
+    batch, dim, N, L = 2, 100, 16, 3000
+    inp = make_scan_inputs(LAYER, batch=batch, dim=dim, dstate=N, seqlen=L, seed=2960)
+    dev = device_inputs(inp)
+    conv = make_conv_params(dim, 4, seed=2961)
+    conv_t = {k: to_device(v, "f32") for k, v in conv.items()}
+    c, lanes, w = _conv_configs()[0]
+    units = batch * ((dim + 128 // lanes - 1) // (128 // lanes))
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    y, hT = ms.conv_scan_fwd(dev["u"], conv_t["conv_w"], dev["delta"], dev["A"], dev["B"], dev["C"], D=dev["D"],
+                             z=dev["z"], delta_bias=dev["delta_bias"], conv_bias=conv_t["conv_b"], stream=side,
+                             plan=ms.ScanPlan(config=c, warps_per_cta=w, segments=1, ctas=max(1, units - 1)))
+    junk = [torch.full((1 << 16,), 7, dtype=torch.uint8, device="cuda") for _ in range(64)]
+    del junk
+    side.synchronize()
+    torch.cuda.synchronize()
+    yr, hr = _oracle(inp, conv)
+    assert rel_err(to_host64(y), yr) <= TOL["bf16"]
+    assert rel_err(to_host64(hT), hr) <= TOL["bf16"]
+
+
 def test_conv_scan_mamba130m_layer_full():
     """The Mamba-130M-shaped layer (bf16, gate) with a width-4 prologue, every row."""
     inp = make_scan_inputs(LAYER)

@@ -271,6 +271,30 @@ def test_ssd_persistent_schedule(batch, L, nheads, ngroups):
     assert rel_err(to_host64(hT2), hr.reshape(hT.shape)) <= TOL["bf16"]
 
 
+def test_ssd_persistent_on_side_stream():
+    """The persistent schedule on a stream other than the current one, with
+    its hand-over workspace allocated by the binding, while the current stream
+    churns the allocator."""
+    import torch
+    ms = _ms()
+    inp = make_ssd_inputs(SMALL, batch=2, seqlen=700, nheads=80, seed=3950)
+    dev = _dev(inp)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    if 160 <= sms or 160 % sms == 0:
+        pytest.skip("the shape fills whole waves of this device")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    y, hT = ms.ssd_fwd(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], D=dev["D"], z=dev["z"],
+                       dt_bias=dev["dt_bias"], stream=side, check=False)
+    junk = [torch.full((1 << 16,), 7, dtype=torch.uint8, device="cuda") for _ in range(64)]
+    del junk
+    side.synchronize()
+    torch.cuda.synchronize()
+    yr, hr = _oracle(inp)
+    assert rel_err(to_host64(y), yr) <= TOL["bf16"]
+    assert rel_err(to_host64(hT), hr) <= TOL["bf16"]
+
+
 def test_ssd_persistent_timeout_path():
     """The persistent schedule's bounded waits: with block 2's loads withheld
     and a 2 ms limit, every CTA gives up, still raises its hand-over flag (so
