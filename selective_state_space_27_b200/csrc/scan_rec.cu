@@ -83,8 +83,8 @@ template <int LPR, bool TRAP = false, int IOW = 2> struct Shape {
     static constexpr int EW = WARP_SUM ? LPR : 4;      // steps per readout store
     static constexpr int QSTRIDE = GROUP_MAJOR ? 32 / LPR : 1;   // lane distance between a row's groups
     static constexpr int XR = TRAP ? kSteps + 1 : kSteps / 2 + 1;   // float4 per row of the step tile
-    static constexpr int YQ = LPR <= 4 ? 16 : 20;
-    static constexpr int YR = LPR == 2 ? 36 : LPR == 4 ? 36 : LPR == 8 ? 40 : 328;
+    static constexpr int YQ = LPR <= 4 ? kSteps : kSteps + 4;
+    static constexpr int YR = LPR == 2 ? 2 * kSteps + 4 : LPR == 4 ? kSteps + 20 : LPR == 8 ? kSteps + 24 : LPR * YQ + 8;
     static constexpr int X_OFF = 0;
     static constexpr int Y_OFF = X_OFF + R * XR * 16;
     static constexpr int B_OFF = Y_OFF + R * YR * 4;
