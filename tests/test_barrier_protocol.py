@@ -209,3 +209,10 @@ def test_two_stages():
     """The same protocol with two stages (the I/O warps then finish one chunk
     behind instead of two) is also consistent."""
     check_protocol(stages=2)
+
+
+@pytest.mark.parametrize("io_warps", [2, 4])
+def test_four_stages(io_warps):
+    """Four stages (the I/O warps finishing three chunks behind), as the
+    kernel's static bound on named barriers allows, with 2 or 4 I/O warps."""
+    check_protocol(stages=4, io_warps=io_warps)
