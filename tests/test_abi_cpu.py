@@ -303,3 +303,53 @@ def test_ssd_needs_args_and_workspace(lib):
     assert lib.mamba_ssd_fwd(ctypes.byref(a), None, 0, None) == 6
     assert lib.mamba_ssd_fwd(ctypes.byref(a), (1 << 20) * 9, 128, None) == 6
     assert lib.mamba_ssd_fwd(ctypes.byref(a), (1 << 20) * 9 + 4, 256, None) == 3
+
+
+# The workspace entry points (and their size queries) validate exactly as the
+# plain ones, before any device query or launch.
+
+@pytest.mark.parametrize("field,value,status", [
+    ("weight", None, 1), ("width", 0, 1), ("width", 5, 2), ("silu", 2, 1), ("weight", (1 << 20) * 9 + 2, 3),
+])
+def test_conv_scan_ws_entries_validate(lib, field, value, status):
+    c = _valid_conv()
+    setattr(c, field, value)
+    n = ctypes.c_size_t(7)
+    a = _valid_scan_args()
+    assert lib.mamba_conv_scan_workspace_size(ctypes.byref(a), ctypes.byref(c), None, ctypes.byref(n)) == status
+    assert n.value == 0
+    assert lib.mamba_conv_scan_fwd_ws(ctypes.byref(a), ctypes.byref(c), None, None, 0, None) == status
+
+
+@pytest.mark.parametrize("lam,sb,sd,segments,status", [
+    (None, 512, 64, 0, 1), ((1 << 20) * 12, -1, 64, 0, 1), ((1 << 20) * 12 + 1, 512, 64, 0, 3),
+    ((1 << 20) * 12, 512, 64, 2, 2),
+])
+def test_trap_scan_ws_entries_validate(lib, lam, sb, sd, segments, status):
+    a = _valid_scan_args()
+    a.force_segments = segments
+    n = ctypes.c_size_t(7)
+    assert lib.mamba_trap_scan_workspace_size(ctypes.byref(a), lam, sb, sd, None, ctypes.byref(n)) == status
+    assert n.value == 0
+    assert lib.mamba_trap_scan_fwd_ws(ctypes.byref(a), lam, sb, sd, None, None, 0, None) == status
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("batch", 0, 1), ("ngroups", 3, 1), ("in_dtype", 0, 2), ("x_token_stride", 260, 3),
+])
+def test_ssd_workspace_size_validates(lib, field, value, status):
+    a = _valid_ssd_args()
+    setattr(a, field, value)
+    n = ctypes.c_size_t(7)
+    assert lib.mamba_ssd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == status
+    assert n.value == 0
+
+
+def test_workspace_queries_need_their_arguments(lib):
+    a, c = _valid_scan_args(), _valid_conv()
+    n = ctypes.c_size_t(0)
+    assert lib.mamba_conv_scan_workspace_size(ctypes.byref(a), ctypes.byref(c), None, None) == 1
+    assert lib.mamba_conv_scan_workspace_size(ctypes.byref(a), None, None, ctypes.byref(n)) == 1
+    assert lib.mamba_trap_scan_workspace_size(ctypes.byref(a), (1 << 20) * 12, 512, 64, None, None) == 1
+    assert lib.mamba_ssd_workspace_size(ctypes.byref(_valid_ssd_args()), None) == 1
+    assert lib.mamba_ssd_workspace_size(None, ctypes.byref(n)) == 1
